@@ -1,0 +1,432 @@
+"""Pins of the fp64 oracle to facts other than itself: hand-derived fixtures,
+closed forms, textbook / library routines and brute force on tiny inputs.
+
+Each group names the passage of the SeKV pages it pins.
+"""
+import json
+import math
+import os
+import statistics
+
+import numpy as np
+import pytest
+from scipy.special import expit, logsumexp, softmax
+
+import oracle as O
+from tests.textbook import dense_attention
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------
+# Segmentation  (SeKV blog 2.1: H_t > mu + alpha*sigma; boundary tokens -> anchors)
+# ---------------------------------------------------------------------------
+def _two_level():
+    g = _gold("two_level_stream.json")
+    H = np.full(g["n"], g["c"])
+    H[g["spikes"]] = g["h"]
+    return g, H
+
+
+def test_segment_two_level_closed_form():
+    g, H = _two_level()
+    seg = O.segment(H, g["alpha"], g["window"])
+    assert seg.mu == pytest.approx(g["mu"], abs=1e-14)
+    assert seg.sigma == pytest.approx(math.sqrt(g["sigma_sq"]), abs=1e-14)
+    assert seg.anchor_pos.tolist() == g["anchors"]
+    assert seg.spans.tolist() == g["spans"]
+
+
+def test_segment_threshold_above_spikes_gives_one_span():
+    g, H = _two_level()
+    # (h - mu) / sigma = 3.75 / 0.968 = 3.87 < alpha_none = 4, so nothing crosses.
+    seg = O.segment(H, g["alpha_none"], 0)
+    assert seg.anchor_pos.tolist() == []
+    assert seg.spans.tolist() == g["spans_none"]
+
+
+def test_segment_local_window():
+    g, H = _two_level()
+    seg = O.segment(H, g["alpha"], g["window_w"])
+    assert seg.anchor_pos.tolist() == g["anchors_w"]
+    assert seg.spans.tolist() == g["spans_w"]
+
+
+def _brute_segment(H, alpha, window):
+    mu = statistics.fmean(H)
+    sigma = statistics.pstdev(H)
+    thr = mu + alpha * sigma
+    n = len(H)
+    anchor = [H[t] > thr or t >= n - window for t in range(n)]
+    spans, cur = [], None
+    for t in range(n):
+        if not anchor[t] and cur is None:
+            cur = t
+        if anchor[t] and cur is not None:
+            spans.append([cur, t])
+            cur = None
+    if cur is not None:
+        spans.append([cur, n])
+    return [t for t in range(n) if anchor[t]], spans, thr
+
+
+def test_segment_bruteforce_tiny():
+    rng = np.random.default_rng(7)
+    checked = 0
+    for trial in range(400):
+        n = int(rng.integers(1, 13))
+        H = rng.gamma(2.0, 1.0, size=n)
+        alpha = float(rng.choice([0.0, 0.5, 1.0, 1.5]))
+        window = int(rng.integers(0, 3))
+        anchors, spans, thr = _brute_segment(H.tolist(), alpha, window)
+        if np.min(np.abs(H - thr)) < 1e-9:
+            continue
+        seg = O.segment(H, alpha, window)
+        assert seg.anchor_pos.tolist() == anchors
+        assert seg.spans.tolist() == spans
+        checked += 1
+    assert checked > 300
+
+
+def test_segment_partition_and_maximality():
+    rng = np.random.default_rng(3)
+    H = rng.gamma(2.0, 1.0, size=3000)
+    H[rng.random(3000) < 1 / 64] += 6
+    seg = O.segment(H, 1.0, 37)
+    cover = np.zeros(3000, int)
+    cover[seg.anchor_pos] += 1
+    for b, e in seg.spans:
+        assert e > b
+        cover[b:e] += 1
+        assert b == 0 or seg.anchor[b - 1]
+        assert e == 3000 or seg.anchor[e]
+    assert (cover == 1).all()
+    assert seg.anchor[-37:].all()
+
+
+# ---------------------------------------------------------------------------
+# Weights and weighted means (SeKV blog 2.2 Eq. (2); SeKV summary workflow)
+# ---------------------------------------------------------------------------
+def test_eq2_hand_example():
+    g = _gold("eq2_weighted_mean.json")
+    w = O.span_weights(g["H"], "surprisal")
+    np.testing.assert_allclose(w, g["weights"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(O.weighted_mean(g["K"], w), g["kbar"], rtol=0, atol=1e-14)
+
+
+def test_uniform_weights_are_arithmetic_mean():
+    rng = np.random.default_rng(1)
+    X = rng.normal(size=(17, 5))
+    np.testing.assert_allclose(O.weighted_mean(X, O.span_weights(np.ones(17), "uniform")),
+                               np.mean(X, axis=0), rtol=1e-14, atol=1e-14)
+
+
+def test_softmax_weights_match_scipy():
+    Hs = np.array([0.3, 2.5, 1.1, 7.0])
+    np.testing.assert_allclose(O.span_weights(Hs, "softmax"), softmax(Hs), rtol=1e-14)
+
+
+def test_eq2_zero_sum_falls_back_to_uniform():
+    np.testing.assert_array_equal(O.span_weights(np.zeros(3), "surprisal"), np.ones(3))
+
+
+@pytest.mark.parametrize("wmode", ["uniform", "surprisal", "softmax"])
+def test_constant_span_summary_is_the_row(wmode):
+    row = np.array([0.5, -1.25, 3.0])
+    X = np.tile(row, (6, 1))
+    w = O.span_weights(np.array([1.0, 2.0, 0.5, 3.0, 4.0, 0.1]), wmode)
+    np.testing.assert_allclose(O.weighted_mean(X, w), row, rtol=1e-15)
+
+
+def test_summary_norm_and_logS_closed_form():
+    H = np.array([9.0, 1.0, 1.0, 1.0, 1.0, 9.0])
+    seg = O.segment(H, 1.0, 0)                 # anchors 0 and 5, one span [1, 5)
+    K = np.zeros((6, 2)); K[1:5] = [3.0, 4.0]
+    V = np.ones((6, 2))
+    kbar, vbar, inv_norm, logS = O.span_summaries(K, V, H, seg, "uniform", "f32")
+    assert seg.spans.tolist() == [[1, 5]]
+    assert inv_norm[0] == pytest.approx(0.2, rel=1e-7)
+    assert logS[0] == pytest.approx(math.log(4), rel=1e-7)
+    K[1:5] = 0.0
+    _, _, inv_norm0, _ = O.span_summaries(K, V, H, seg, "uniform", "f32")
+    assert inv_norm0[0] == 0.0
+
+
+def test_bf16_rounding_matches_library_conversion():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.normal(size=2000) * 10 ** rng.uniform(-3, 3, 2000),
+                        [1 + 2 ** -8, 1 + 3 * 2 ** -8, -1 - 2 ** -8, 0.0]])
+    ref = torch.tensor(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.to_storage(x, "bf16"), ref)
+    assert O.to_storage([1 + 2 ** -8], "bf16")[0] == 1.0          # tie to even
+    assert O.to_storage([1 + 3 * 2 ** -8], "bf16")[0] == 1 + 2 ** -6
+
+
+# ---------------------------------------------------------------------------
+# Truncated bases (SeKV blog 2.2 Eq. (6)-(8), gate m_i = 1)
+# ---------------------------------------------------------------------------
+def _orth(rng, rows, cols):
+    q, _ = np.linalg.qr(rng.normal(size=(rows, cols)))
+    return q
+
+
+@pytest.mark.parametrize("ns,d", [(12, 20), (20, 12), (16, 16)])
+@pytest.mark.parametrize("r", [1, 3, 5])
+def test_basis_known_singular_structure(ns, d, r):
+    rng = np.random.default_rng(ns * 100 + d + r)
+    k = min(ns, d)
+    U, W = _orth(rng, ns, k), _orth(rng, d, k)
+    s = np.linspace(10.0, 1.0, k) ** 1.5            # distinct, descending
+    X = (U * s) @ W.T
+    A, B = O.truncated_basis(X, r, "f64")
+    expect = (U[:, :r] * s[:r]) @ W[:, :r].T
+    np.testing.assert_allclose(A @ B, expect, rtol=0, atol=1e-10 * s[0])
+    if ns <= d:
+        np.testing.assert_allclose(A.T @ A, np.eye(r), atol=1e-12)
+    else:
+        np.testing.assert_allclose(B @ B.T, np.eye(r), atol=1e-12)
+
+
+@pytest.mark.parametrize("ns,d,g", [(30, 16, 4), (9, 16, 4), (5, 8, 5)])
+def test_basis_exact_for_low_rank_and_full_rank(ns, d, g):
+    rng = np.random.default_rng(ns + d)
+    X = rng.normal(size=(ns, g)) @ rng.normal(size=(g, d))
+    for r in (g, g + 2, min(ns, d), 100):
+        A, B = O.truncated_basis(X, r, "f64")
+        np.testing.assert_allclose(A @ B, X, atol=1e-10 * np.abs(X).max())
+
+
+@pytest.mark.parametrize("ns,d", [(40, 16), (10, 32)])
+def test_basis_eckart_young(ns, d):
+    rng = np.random.default_rng(11)
+    X = rng.normal(size=(ns, d))
+    lam = np.sort(np.linalg.eigvalsh(X.T @ X))[::-1]      # sigma_i^2, another routine
+    for r in (1, 4, 7):
+        A, B = O.truncated_basis(X, r, "f64")
+        resid = np.sum((X - A @ B) ** 2)
+        assert resid == pytest.approx(np.sum(lam[r:]), rel=1e-9, abs=1e-9)
+
+
+# ---------------------------------------------------------------------------
+# Routing (SeKV blog 2.3 Eq. (5), Eq. (9))
+# ---------------------------------------------------------------------------
+def test_tau_to_theta_closed_form():
+    th = O.tau_to_theta(np.array([0.5, math.e / (1 + math.e), 0.0, 1.0, -0.2, 1.5]))
+    assert th[0] == 0.0
+    assert th[1] == pytest.approx(1.0, abs=1e-15)
+    assert th[2] == -np.inf and th[4] == -np.inf
+    assert th[3] == np.inf and th[5] == np.inf
+
+
+def test_routing_hand_example():
+    g = _gold("routing_example.json")
+    kbar = np.array([g["kbar"]])
+    inv = np.array([1.0 / np.linalg.norm(kbar)])
+    ell = O.routing_logits(g["q"], kbar, inv, np.array([math.log(g["len"])]), 1 / math.sqrt(2))
+    assert ell[0] == pytest.approx(g["ell"], abs=1e-14)
+    assert O.zoom_decisions(ell, O.tau_to_theta(g["tau_zoom"]))[0]
+    assert not O.zoom_decisions(ell, O.tau_to_theta(g["tau_nozoom"]))[0]
+
+
+def test_logit_space_decision_equals_sigmoid_decision():
+    rng = np.random.default_rng(2)
+    ell = rng.normal(scale=3.0, size=5000)
+    for tau in (0.05, 0.3, 0.5, 0.77, 0.99):
+        th = O.tau_to_theta(tau)
+        gap = np.abs(ell - th) > 1e-9
+        np.testing.assert_array_equal(O.zoom_decisions(ell, th)[gap], (expit(ell) > tau)[gap])
+
+
+def test_singleton_routing_has_no_size_prior():
+    rng = np.random.default_rng(4)
+    kb, q = rng.normal(size=(1, 8)), rng.normal(size=8)
+    inv = np.array([1 / np.linalg.norm(kb)])
+    ell = O.routing_logits(q, kb, inv, np.array([math.log(1)]), 0.5)
+    cos = kb[0] @ q / np.linalg.norm(kb) / np.linalg.norm(q)
+    assert ell[0] == pytest.approx(cos * np.linalg.norm(q) * 0.5, rel=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Stage-2 decode (SeKV summary workflow: one softmax over anchors,
+# reconstructed zoomed tokens and log|S|-corrected summaries; Fig. 2 merge)
+# ---------------------------------------------------------------------------
+def _random_unit(rng, n, d, anchor_frac=0.2, identical=()):
+    K = rng.normal(size=(n, d))
+    V = rng.normal(size=(n, d))
+    H = rng.gamma(2.0, 1.0, size=n)
+    anchor = rng.random(n) < anchor_frac
+    anchor[0] = True
+    spans, cur = [], None
+    for t in range(n):
+        if not anchor[t] and cur is None:
+            cur = t
+        if anchor[t] and cur is not None:
+            spans.append((cur, t)); cur = None
+    if cur is not None:
+        spans.append((cur, n))
+    seg = O.Segmentation(0.0, 0.0, 0.0, anchor, np.flatnonzero(anchor),
+                         np.array(spans, dtype=np.int64).reshape(-1, 2))
+    for S in identical:
+        b, e = seg.spans[S]
+        K[b:e] = K[b]
+        V[b:e] = V[b]
+    return K, V, H, seg
+
+
+def _decode(K, V, H, seg, wmode, rank, zoom, q, scale):
+    c = O.build_unit(K, V, H, seg, wmode, rank, "f64")
+    return O.decode_unit(q, c.Ka, c.Va, c.kbar, c.vbar, c.logS, zoom, c.bases, scale)
+
+
+def test_singleton_spans_equal_dense_attention():
+    rng = np.random.default_rng(21)
+    n, d, G = 60, 8, 3
+    K, V = rng.normal(size=(n, d)), rng.normal(size=(n, d))
+    anchor = rng.random(n) < 0.3
+    spans = np.array([[t, t + 1] for t in range(n) if not anchor[t]])
+    seg = O.Segmentation(0, 0, 0, anchor, np.flatnonzero(anchor), spans)
+    q = rng.normal(size=(G, d))
+    for wmode in ("uniform", "surprisal", "softmax"):
+        Oo, lse = _decode(K, V, rng.gamma(2, 1, n), seg, wmode, 4, np.zeros((G, len(spans)), bool), q, 0.35)
+        for h in range(G):
+            o_ref, l_ref = dense_attention(q[h], K, V, 0.35)
+            np.testing.assert_allclose(Oo[h], o_ref, atol=1e-12)
+            assert lse[h] == pytest.approx(l_ref, abs=1e-12)
+
+
+def test_all_zoom_full_rank_equals_dense_attention():
+    rng = np.random.default_rng(22)
+    n, d, G = 80, 6, 2
+    K, V, H, seg = _random_unit(rng, n, d)
+    q = rng.normal(size=(G, d))
+    zoom = np.ones((G, len(seg.spans)), bool)
+    Oo, lse = _decode(K, V, H, seg, "softmax", d, zoom, q, 0.4)
+    for h in range(G):
+        o_ref, l_ref = dense_attention(q[h], K, V, 0.4)
+        np.testing.assert_allclose(Oo[h], o_ref, atol=1e-11)
+        assert lse[h] == pytest.approx(l_ref, abs=1e-11)
+
+
+def test_identical_span_is_represented_exactly():
+    rng = np.random.default_rng(23)
+    n, d, G = 70, 5, 2
+    K, V, H, seg = _random_unit(rng, n, d)
+    long_spans = [i for i, (b, e) in enumerate(seg.spans) if e - b >= 2]
+    K, V, H, seg = _random_unit(np.random.default_rng(23), n, d, identical=())
+    # make EVERY span constant, so every coarse entry must be exact
+    for b, e in seg.spans:
+        K[b:e] = K[b]
+        V[b:e] = V[b]
+    q = rng.normal(size=(G, d))
+    zoom = np.zeros((G, len(seg.spans)), bool)
+    Oo, lse = _decode(K, V, H, seg, "surprisal", 2, zoom, q, 0.5)
+    assert long_spans
+    for h in range(G):
+        o_ref, l_ref = dense_attention(q[h], K, V, 0.5)
+        np.testing.assert_allclose(Oo[h], o_ref, atol=1e-12)
+        assert lse[h] == pytest.approx(l_ref, abs=1e-12)
+
+
+def test_coarse_entry_equals_replicated_summary():
+    """Brute force: each non-zoomed summary replicated |S| times in a plain
+    softmax (no correction) equals the oracle's +log|S| entry; zoomed spans
+    with full-rank bases contribute their exact tokens."""
+    rng = np.random.default_rng(24)
+    n, d, G = 90, 7, 4
+    K, V, H, seg = _random_unit(rng, n, d)
+    m = len(seg.spans)
+    q = rng.normal(size=(G, d))
+    zoom = rng.random((G, m)) < 0.4
+    c = O.build_unit(K, V, H, seg, "softmax", d, "f64")
+    Oo, lse = O.decode_unit(q, c.Ka, c.Va, c.kbar, c.vbar, c.logS, zoom, c.bases, 0.3)
+    for h in range(G):
+        rowsK, rowsV = [K[t] for t in seg.anchor_pos], [V[t] for t in seg.anchor_pos]
+        for S, (b, e) in enumerate(seg.spans):
+            if zoom[h, S]:
+                rowsK += list(K[b:e]); rowsV += list(V[b:e])
+            else:
+                rowsK += [c.kbar[S]] * (e - b); rowsV += [c.vbar[S]] * (e - b)
+        o_ref, l_ref = dense_attention(q[h], np.array(rowsK), np.array(rowsV), 0.3)
+        np.testing.assert_allclose(Oo[h], o_ref, atol=1e-11)
+        assert lse[h] == pytest.approx(l_ref, abs=1e-11)
+
+
+def test_zoomed_low_rank_span_uses_reconstruction():
+    """A zoomed span contributes the tokens of A@B / C@D, not the originals."""
+    rng = np.random.default_rng(25)
+    n, d = 40, 6
+    K, V, H, seg = _random_unit(rng, n, d, anchor_frac=0.1)
+    q = rng.normal(size=(1, d))
+    zoom = np.ones((1, len(seg.spans)), bool)
+    c = O.build_unit(K, V, H, seg, "uniform", 2, "f64")
+    Oo, lse = O.decode_unit(q, c.Ka, c.Va, c.kbar, c.vbar, c.logS, zoom, c.bases, 0.4)
+    rowsK, rowsV = [K[seg.anchor_pos]], [V[seg.anchor_pos]]
+    for S, (b, e) in enumerate(seg.spans):
+        A, B, C, D = c.bases[S]
+        rowsK.append(A @ B); rowsV.append(C @ D)
+    o_ref, l_ref = dense_attention(q[0], np.concatenate(rowsK), np.concatenate(rowsV), 0.4)
+    np.testing.assert_allclose(Oo[0], o_ref, atol=1e-12)
+    o_orig, _ = dense_attention(q[0], K, V, 0.4)
+    assert np.abs(Oo[0] - o_orig).max() > 1e-3      # rank 2 is lossy here
+
+
+def test_empty_unit():
+    Oo, lse = O.decode_unit(np.ones((2, 4)), np.zeros((0, 4)), np.zeros((0, 4)), np.zeros((0, 4)),
+                            np.zeros((0, 4)), np.zeros(0), np.zeros((2, 0), bool), [], 0.5)
+    assert (Oo == 0).all() and np.isneginf(lse).all()
+
+
+def test_lse_is_log_partition():
+    rng = np.random.default_rng(26)
+    K, V, H, seg = _random_unit(rng, 50, 4)
+    q = rng.normal(size=(1, 4))
+    zoom = np.zeros((1, len(seg.spans)), bool)
+    c = O.build_unit(K, V, H, seg, "uniform", 2, "f64")
+    _, lse = O.decode_unit(q, c.Ka, c.Va, c.kbar, c.vbar, c.logS, zoom, c.bases, 0.7)
+    x = np.concatenate([c.Ka @ q[0] * 0.7, c.kbar @ q[0] * 0.7 + c.logS])
+    assert lse[0] == pytest.approx(logsumexp(x), abs=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Planted mistakes: each pin above must catch a plausible oracle bug.
+# ---------------------------------------------------------------------------
+def test_planted_dropped_log_correction_is_caught():
+    rng = np.random.default_rng(24)
+    K, V, H, seg = _random_unit(rng, 60, 5)
+    for b, e in seg.spans:
+        K[b:e] = K[b]; V[b:e] = V[b]
+    q = rng.normal(size=(1, 5))
+    c = O.build_unit(K, V, H, seg, "uniform", 2, "f64")
+    zoom = np.zeros((1, len(seg.spans)), bool)
+    bad, _ = O.decode_unit(q, c.Ka, c.Va, c.kbar, c.vbar, 0 * c.logS, zoom, c.bases, 0.5)
+    o_ref, _ = dense_attention(q[0], K, V, 0.5)
+    assert np.abs(bad[0] - o_ref).max() > 1e-3
+
+
+def test_planted_sample_std_is_caught(monkeypatch):
+    g, H = _two_level()
+    real_sqrt = np.sqrt
+
+    def ddof1_sqrt(x):                     # turns the population variance into the sample one
+        return real_sqrt(x * g["n"] / (g["n"] - 1))
+    monkeypatch.setattr(O.sekv_oracle.np, "sqrt", ddof1_sqrt)
+    seg = O.segment(H, g["alpha"], 0)
+    monkeypatch.undo()
+    assert seg.sigma != pytest.approx(math.sqrt(g["sigma_sq"]), abs=1e-6)
+
+
+def test_planted_swapped_basis_factors_are_caught():
+    rng = np.random.default_rng(9)
+    U, W = _orth(rng, 12, 8), _orth(rng, 20, 8)
+    X = (U * np.arange(8, 0, -1.0)) @ W.T
+    A, B = O.truncated_basis(X, 3, "f64")
+    expect = (U[:, :3] * np.arange(8, 5, -1.0)) @ W[:, :3].T
+    assert np.abs(A @ B - expect).max() < 1e-10
+    A2, B2 = O.truncated_basis(X.T, 3, "f64")       # a transposed operand
+    assert (A2 @ B2).shape != expect.shape or np.abs(A2 @ B2 - expect).max() > 1e-3
