@@ -1,0 +1,285 @@
+// C ABI of the SeKV span-cache library: argument checks, workspace carving,
+// launches, and the host side of the cold-basis fetch.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "sekv_common.cuh"
+#include "sekv_internal.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+sekv_status fail(sekv_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+sekv_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(SEKV_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int esize(int dtype) { return dtype == SEKV_F32 ? 4 : 2; }
+
+#define SEKV_REQUIRE(cond, ...)                                   \
+    do {                                                          \
+        if (!(cond)) return fail(SEKV_ERR_INVALID_ARG, __VA_ARGS__); \
+    } while (0)
+
+sekv_status check_build(const sekv_build_desc* d) {
+    SEKV_REQUIRE(d, "build: null descriptor");
+    SEKV_REQUIRE(d->B >= 1 && d->L >= 1 && d->Hkv >= 1 && d->n >= 1, "build: B, L, Hkv, n must be >= 1");
+    SEKV_REQUIRE(d->dtype == SEKV_F32 || d->dtype == SEKV_BF16, "build: dtype %d", d->dtype);
+    SEKV_REQUIRE(d->steps >= 1 && d->steps <= SEKV_BUILD_ALL, "build: steps mask %d", d->steps);
+    SEKV_REQUIRE(d->a_cap >= 1 && d->m_cap >= 32 && d->m_cap % 32 == 0,
+                 "build: a_cap >= 1 and m_cap a positive multiple of 32 required");
+    SEKV_REQUIRE(d->window >= 0, "build: window < 0");
+    SEKV_REQUIRE(d->dev_status, "build: dev_status is required");
+    if (d->steps & SEKV_BUILD_SCAN)
+        SEKV_REQUIRE(d->H && d->a_count && d->m_count && d->anchor_pos && d->span_beg && d->span_end,
+                     "build/scan: H, a_count, m_count, anchor_pos, span_beg, span_end required");
+    if (d->steps & SEKV_BUILD_LAYOUT) {
+        SEKV_REQUIRE(d->m_count && d->span_beg && d->span_end && d->logS && d->blk_off,
+                     "build/layout: m_count, span_beg, span_end, logS, blk_off required");
+        SEKV_REQUIRE(d->rank >= 1, "build/layout: rank >= 1 required");
+    }
+    if (d->steps & (SEKV_BUILD_SUMMARY | SEKV_BUILD_BASES)) {
+        SEKV_REQUIRE(d->l0 >= 0 && d->l0 < d->l1 && d->l1 <= d->L, "build: layer range [%d, %d) of %d",
+                     d->l0, d->l1, d->L);
+        if (d->d != 64 && d->d != 128) return fail(SEKV_ERR_UNSUPPORTED, "build: d = %d (64 or 128)", d->d);
+        SEKV_REQUIRE(d->K && d->V && aligned(d->K, 16) && aligned(d->V, 16),
+                     "build: K and V must be non-null and 16-byte aligned");
+    }
+    if (d->steps & SEKV_BUILD_SUMMARY) {
+        SEKV_REQUIRE(d->H && d->Ka && d->Va && d->kbar && d->vbar && d->inv_norm && d->anchor_pos &&
+                         d->a_count && d->m_count && d->span_beg && d->span_end,
+                     "build/summary: missing pointer");
+        SEKV_REQUIRE(aligned(d->Ka, 16) && aligned(d->Va, 16) && aligned(d->kbar, 16) && aligned(d->vbar, 16),
+                     "build/summary: Ka, Va, kbar, vbar must be 16-byte aligned");
+        SEKV_REQUIRE(d->wmode >= SEKV_W_UNIFORM && d->wmode <= SEKV_W_SOFTMAX, "build: wmode %d", d->wmode);
+    }
+    if (d->steps & SEKV_BUILD_BASES) {
+        SEKV_REQUIRE(d->basis_home && d->blk_off && d->m_count && d->span_beg && d->span_end,
+                     "build/bases: basis_home, blk_off and the span arrays are required");
+        SEKV_REQUIRE(d->rank >= 1 && d->max_sweeps >= 1, "build/bases: rank and max_sweeps >= 1");
+        SEKV_REQUIRE(d->region_elems > 0 && d->region_elems % 64 == 0 && aligned(d->basis_home, 256),
+                     "build/bases: region_elems a positive multiple of 64, basis_home 256-byte aligned");
+        SEKV_REQUIRE(d->workspace && aligned(d->workspace, 256) &&
+                         (size_t)d->workspace_bytes >= sekv::basis_workspace_bytes(*d),
+                     "build/bases: workspace of %zu bytes (256-byte aligned) required",
+                     sekv::basis_workspace_bytes(*d));
+    }
+    return SEKV_OK;
+}
+
+sekv_status check_decode(const sekv_decode_desc* d) {
+    SEKV_REQUIRE(d, "decode: null descriptor");
+    SEKV_REQUIRE(d->B >= 1 && d->L >= 1 && d->Hq >= 1 && d->Hkv >= 1 && d->Hq % d->Hkv == 0,
+                 "decode: B, L, Hq, Hkv >= 1 and Hq a multiple of Hkv");
+    SEKV_REQUIRE(d->l0 >= 0 && d->l0 < d->l1 && d->l1 <= d->L, "decode: layer range [%d, %d) of %d", d->l0,
+                 d->l1, d->L);
+    SEKV_REQUIRE(d->phase >= SEKV_FUSED && d->phase <= SEKV_ATTEND, "decode: phase %d", d->phase);
+    SEKV_REQUIRE(d->a_cap >= 1 && d->m_cap >= 32 && d->m_cap % 32 == 0, "decode: a_cap >= 1, m_cap % 32 == 0");
+    SEKV_REQUIRE(d->m_cap < (1 << 24), "decode: m_cap must be < 2^24");
+    if (!sekv::decode_supported(*d))
+        return fail(SEKV_ERR_UNSUPPORTED, "decode: d=%d, Hq/Hkv=%d, rank=%d, dtype=%d not compiled", d->d,
+                    d->Hq / d->Hkv, d->rank, d->dtype);
+    SEKV_REQUIRE(d->dev_status && d->q && d->a_count && d->m_count && d->span_beg && d->span_end && d->logS &&
+                     d->kbar && d->inv_norm && d->theta,
+                 "decode: missing input pointer");
+    SEKV_REQUIRE(aligned(d->q, 16) && aligned(d->kbar, 16) && aligned(d->inv_norm, 16) && aligned(d->logS, 16),
+                 "decode: q, kbar, inv_norm, logS must be 16-byte aligned");
+    if (d->phase == SEKV_ROUTE) {
+        SEKV_REQUIRE(d->zmask || d->route_logits, "decode/route: zmask or route_logits required");
+    } else {
+        SEKV_REQUIRE(d->Ka && d->Va && d->vbar && d->arena && d->O && d->lse,
+                     "decode: Ka, Va, vbar, arena, O, lse required");
+        SEKV_REQUIRE(aligned(d->Ka, 16) && aligned(d->Va, 16) && aligned(d->vbar, 16) && aligned(d->arena, 256),
+                     "decode: Ka, Va, vbar 16-byte and arena 256-byte aligned");
+        if (d->phase == SEKV_ATTEND) SEKV_REQUIRE(d->slot, "decode/attend: slot table required");
+        if (!d->slot)
+            SEKV_REQUIRE(d->blk_off && d->region_elems > 0 && d->region_elems % 64 == 0,
+                         "decode: blk_off and region_elems (multiple of 64) required without a slot table");
+        const size_t need = sekv::decode_workspace_bytes(*d);
+        SEKV_REQUIRE(d->workspace && aligned(d->workspace, 256) && (size_t)d->workspace_bytes >= need,
+                     "decode: workspace of %zu bytes (256-byte aligned) required", need);
+    }
+    return SEKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sekv_status_str(int32_t s) {
+    switch (s) {
+        case SEKV_OK: return "ok";
+        case SEKV_ERR_INVALID_ARG: return "invalid argument";
+        case SEKV_ERR_CAPACITY: return "capacity exceeded";
+        case SEKV_ERR_CUDA: return "CUDA error";
+        case SEKV_ERR_COLD_SPAN: return "zoomed span has no resident bases";
+        case SEKV_ERR_TIMEOUT: return "bounded device wait ran out";
+        case SEKV_ERR_UNSUPPORTED: return "unsupported shape";
+        case SEKV_WARN_NOT_CONVERGED: return "Jacobi solve hit max_sweeps";
+        default: return "unknown status";
+    }
+}
+
+const char* sekv_last_error(void) { return g_err.c_str(); }
+
+int32_t sekv_version(void) { return SEKV_VERSION; }
+
+size_t sekv_desc_size(int32_t which) {
+    switch (which) {
+        case 0: return sizeof(sekv_build_desc);
+        case 1: return sizeof(sekv_decode_desc);
+        case 2: return sizeof(sekv_fetch_desc);
+        default: return 0;
+    }
+}
+
+int64_t sekv_block_elems(int32_t len, int32_t d, int32_t rank) {
+    if (len < 1 || d < 1 || rank < 1) return 0;
+    return sekv::block_elems(len, d, rank);
+}
+
+int64_t sekv_basis_region_bound(int32_t n, int32_t m_cap, int32_t Hkv, int32_t d, int32_t rank) {
+    const int64_t per = 2LL * n * rank + (int64_t)m_cap * (2LL * rank * d + 80);
+    return sekv::round_up((int64_t)Hkv * per, 64);
+}
+
+size_t sekv_build_workspace_bytes(const sekv_build_desc* d) {
+    if (!d) return 0;
+    return (d->steps & SEKV_BUILD_BASES) ? sekv::basis_workspace_bytes(*d) : 0;
+}
+
+sekv_status sekv_build_spans(const sekv_build_desc* d, sekv_stream_t stream) {
+    sekv_status s = check_build(d);
+    if (s != SEKV_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (d->steps & SEKV_BUILD_SCAN)
+        if ((e = sekv::launch_scan(*d, st)) != cudaSuccess) return cuda_fail(e, "scan");
+    if (d->steps & SEKV_BUILD_LAYOUT)
+        if ((e = sekv::launch_layout(*d, (d->steps & SEKV_BUILD_BASES) != 0, st)) != cudaSuccess)
+            return cuda_fail(e, "layout");
+    if (d->steps & SEKV_BUILD_SUMMARY)
+        if ((e = sekv::launch_summary(*d, st)) != cudaSuccess) return cuda_fail(e, "summary");
+    if (d->steps & SEKV_BUILD_BASES)
+        if ((e = sekv::launch_basis(*d, st)) != cudaSuccess) return cuda_fail(e, "bases");
+    return SEKV_OK;
+}
+
+size_t sekv_decode_workspace_bytes(const sekv_decode_desc* d) {
+    if (!d || d->Hkv < 1 || d->Hq < 1 || d->l1 <= d->l0) return 0;
+    return sekv::decode_workspace_bytes(*d);
+}
+
+sekv_status sekv_decode_attn(const sekv_decode_desc* d, sekv_stream_t stream) {
+    sekv_status s = check_decode(d);
+    if (s != SEKV_OK) return s;
+    const sekv::DecodePlan p = sekv::plan_decode(*d);
+    cudaError_t e = sekv::launch_decode(*d, p, d->workspace, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode");
+    return SEKV_OK;
+}
+
+sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, sekv_stream_t copy,
+                             sekv_event_t done) {
+    SEKV_REQUIRE(d, "fetch: null descriptor");
+    SEKV_REQUIRE(d->zmask_dev && d->zmask_host && d->m_count_host && d->blk_off_host && d->home && d->arena &&
+                     d->slot_dev && d->slot_host && done,
+                 "fetch: missing pointer or event");
+    SEKV_REQUIRE(d->B >= 1 && d->L >= 1 && d->Hq >= 1 && d->Hkv >= 1 && d->l0 >= 0 && d->l0 < d->l1 &&
+                     d->l1 <= d->L && d->m_cap >= 32 && d->m_cap % 32 == 0 && d->region_elems > 0 &&
+                     d->arena_elems >= 0 && (d->dtype == SEKV_F32 || d->dtype == SEKV_BF16),
+                 "fetch: bad shape");
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(compute);
+    cudaStream_t xs = reinterpret_cast<cudaStream_t>(copy);
+    cudaEvent_t ev = reinterpret_cast<cudaEvent_t>(done);
+    const int mw = d->m_cap / 32, Lr = d->l1 - d->l0;
+    const int64_t es = esize(d->dtype);
+    cudaError_t e;
+    // the previous call's slot upload must be finished before the mirror is rewritten
+    if ((e = cudaEventSynchronize(ev)) != cudaSuccess) return cuda_fail(e, "fetch: previous done event");
+    for (int b = 0; b < d->B; ++b) {
+        const int64_t w0 = ((int64_t)b * d->L + d->l0) * d->Hq * mw;
+        if ((e = cudaMemcpyAsync(d->zmask_host + w0, d->zmask_dev + w0, sizeof(uint32_t) * Lr * d->Hq * mw,
+                                 cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+            return cuda_fail(e, "fetch: zmask readback");
+    }
+    // the host needs the routing result; this also orders the copies after the
+    // previous step's ATTEND (which ran earlier on `compute`)
+    if ((e = cudaStreamSynchronize(cs)) != cudaSuccess) return cuda_fail(e, "fetch: compute stream");
+
+    struct Run { int64_t src, dst, elems; };
+    std::vector<Run> runs;
+    std::vector<uint32_t> uni(mw);
+    int64_t bump = 0, spans = 0;
+    for (int b = 0; b < d->B; ++b) {
+        const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
+        const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
+        for (int l = d->l0; l < d->l1; ++l) {
+            int64_t* sl = d->slot_host + ((int64_t)b * d->L + l) * d->m_cap;
+            for (int S = 0; S < d->m_cap; ++S) sl[S] = -1;
+            std::fill(uni.begin(), uni.end(), 0u);
+            const uint32_t* zm = d->zmask_host + ((int64_t)b * d->L + l) * d->Hq * mw;
+            for (int h = 0; h < d->Hq; ++h)
+                for (int w = 0; w < mw; ++w) uni[w] |= zm[h * mw + w];
+            const int64_t region0 = ((int64_t)b * d->L + l) * d->region_elems;
+            int S = 0;
+            while (S < m) {
+                if (!((uni[S >> 5] >> (S & 31)) & 1u)) { ++S; continue; }
+                const int Sa = S;
+                while (S < m && ((uni[S >> 5] >> (S & 31)) & 1u)) {
+                    sl[S] = bump + (bo[S] - bo[Sa]);
+                    ++S;
+                    ++spans;
+                }
+                const int64_t elems = bo[S] - bo[Sa];
+                runs.push_back({region0 + bo[Sa], bump, elems});
+                bump += elems;
+            }
+        }
+    }
+    if (d->stats) {
+        d->stats[0] = bump * es;
+        d->stats[1] = spans;
+        d->stats[2] = (int64_t)runs.size();
+        d->stats[3] = 0;
+    }
+    if (bump > d->arena_elems) {
+        // leave the device slot table untouched; nothing was copied
+        if ((e = cudaEventRecord(ev, xs)) != cudaSuccess) return cuda_fail(e, "fetch: record");
+        return fail(SEKV_ERR_CAPACITY, "fetch: zoomed bases need %lld elements, arena holds %lld",
+                    (long long)bump, (long long)d->arena_elems);
+    }
+    const char* home = reinterpret_cast<const char*>(d->home);
+    char* arena = reinterpret_cast<char*>(d->arena);
+    for (const Run& r : runs) {
+        if ((e = cudaMemcpyAsync(arena + r.dst * es, home + r.src * es, r.elems * es, cudaMemcpyHostToDevice,
+                                 xs)) != cudaSuccess)
+            return cuda_fail(e, "fetch: basis copy");
+    }
+    for (int b = 0; b < d->B; ++b) {
+        const int64_t o = ((int64_t)b * d->L + d->l0) * d->m_cap;
+        if ((e = cudaMemcpyAsync(d->slot_dev + o, d->slot_host + o, sizeof(int64_t) * Lr * d->m_cap,
+                                 cudaMemcpyHostToDevice, xs)) != cudaSuccess)
+            return cuda_fail(e, "fetch: slot upload");
+    }
+    if ((e = cudaEventRecord(ev, xs)) != cudaSuccess) return cuda_fail(e, "fetch: record");
+    return SEKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,203 @@
+// Device-side helpers shared by the SeKV kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sekv.h"
+
+#define SEKV_DEV __device__ __forceinline__
+
+namespace sekv {
+
+constexpr int kWarp = 32;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ---------------------------------------------------------------------------
+// element types: DT 0 = float, 1 = bfloat16
+// ---------------------------------------------------------------------------
+template <int DT> struct Elt;
+template <> struct Elt<SEKV_F32> {
+    using T = float;
+    static constexpr int bytes = 4;
+};
+template <> struct Elt<SEKV_BF16> {
+    using T = __nv_bfloat16;
+    static constexpr int bytes = 2;
+};
+
+SEKV_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+SEKV_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// load N (2 or 4) consecutive elements starting at p (aligned to N elements) as floats
+template <int DT, int N> struct Vec;
+template <> struct Vec<SEKV_F32, 4> {
+    SEKV_DEV static void load(const void* p, float* v) {
+        float4 x = *reinterpret_cast<const float4*>(p);
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    }
+};
+template <> struct Vec<SEKV_F32, 2> {
+    SEKV_DEV static void load(const void* p, float* v) {
+        float2 x = *reinterpret_cast<const float2*>(p);
+        v[0] = x.x; v[1] = x.y;
+    }
+};
+template <> struct Vec<SEKV_BF16, 4> {
+    SEKV_DEV static void load(const void* p, float* v) {
+        uint2 x = *reinterpret_cast<const uint2*>(p);
+        v[0] = bf16_lo(x.x); v[1] = bf16_hi(x.x); v[2] = bf16_lo(x.y); v[3] = bf16_hi(x.y);
+    }
+};
+template <> struct Vec<SEKV_BF16, 2> {
+    SEKV_DEV static void load(const void* p, float* v) {
+        uint32_t x = *reinterpret_cast<const uint32_t*>(p);
+        v[0] = bf16_lo(x); v[1] = bf16_hi(x);
+    }
+};
+
+template <int DT> SEKV_DEV float load1(const void* p, int64_t i);
+template <> SEKV_DEV float load1<SEKV_F32>(const void* p, int64_t i) {
+    return reinterpret_cast<const float*>(p)[i];
+}
+template <> SEKV_DEV float load1<SEKV_BF16>(const void* p, int64_t i) {
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+template <int DT> SEKV_DEV void store1(void* p, int64_t i, float v);
+template <> SEKV_DEV void store1<SEKV_F32>(void* p, int64_t i, float v) {
+    reinterpret_cast<float*>(p)[i] = v;
+}
+template <> SEKV_DEV void store1<SEKV_BF16>(void* p, int64_t i, float v) {
+    reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+}
+// value after a round trip through the storage type
+template <int DT> SEKV_DEV float round_storage(float v);
+template <> SEKV_DEV float round_storage<SEKV_F32>(float v) { return v; }
+template <> SEKV_DEV float round_storage<SEKV_BF16>(float v) {
+    return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+// ---------------------------------------------------------------------------
+// status: first error wins
+// ---------------------------------------------------------------------------
+SEKV_DEV void set_status(int32_t* st, int code) {
+    if (st) atomicCAS(st, 0, code);
+}
+
+// ---------------------------------------------------------------------------
+// basis block layout (must match sekv_block_elems on the host)
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+__host__ __device__ __forceinline__ int block_rank(int len, int d, int rank) {
+    int r = rank < len ? rank : len;
+    return r < d ? r : d;
+}
+__host__ __device__ __forceinline__ int64_t block_ac_elems(int len, int rS) { return round_up((int64_t)len * rS, 8); }
+__host__ __device__ __forceinline__ int64_t block_elems(int len, int d, int rank) {
+    int rS = block_rank(len, d, rank);
+    return round_up(2 * block_ac_elems(len, rS) + 2 * (int64_t)rS * d, 64);
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier + bulk copy (1-D, global -> shared, no multicast)
+// ---------------------------------------------------------------------------
+SEKV_DEV uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+SEKV_DEV void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+SEKV_DEV void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+SEKV_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .b64 st;\n\t"
+                 "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
+                 ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+SEKV_DEV void mbar_arrive(uint64_t* bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\t"
+                 "mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+SEKV_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Bounded wait: gives up after ~2^22 polls with back-off (far above any
+// legitimate wait, well under a second of wall time).
+constexpr uint32_t kWaitPolls = 1u << 22;
+SEKV_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (i > 64) __nanosleep(64);
+    }
+    return false;
+}
+SEKV_DEV void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst_smem)), "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// warp helpers
+// ---------------------------------------------------------------------------
+SEKV_DEV float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+SEKV_DEV float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Transpose-reduce: every lane holds 32 partial sums v[0..31]; afterwards lane L
+// holds the warp-wide sum of index L. 31 shuffles for 32 reductions.
+SEKV_DEV float transpose_reduce32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const bool up = lane & 16;
+        float send = up ? v[i] : v[i + 16];
+        float keep = up ? v[i + 16] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const bool up = lane & 8;
+        float send = up ? v[i] : v[i + 8];
+        float keep = up ? v[i + 8] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool up = lane & 4;
+        float send = up ? v[i] : v[i + 4];
+        float keep = up ? v[i + 4] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool up = lane & 2;
+        float send = up ? v[i] : v[i + 2];
+        float keep = up ? v[i + 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+    {
+        const bool up = lane & 1;
+        float send = up ? v[0] : v[1];
+        float keep = up ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+    return v[0];
+}
+
+}  // namespace sekv

@@ -1,0 +1,613 @@
+// K-d: split-K mixed-resolution flash-decoding over the span-structured cache.
+//
+// SeKV blog walkthrough, section 2.3: Eq. (5) routing gate
+//   alpha_S = sigmoid(q . Kbar_S / sqrt(d') + log|S|), Kbar_S = kbar_S / ||kbar_S|| (W = I, d' = d)
+// and Eq. (9) zoom decision z_S = 1[alpha_S > tau^(l,h)], compared here in logit
+// space against theta = ln(tau / (1 - tau)). SeKV summary page, workflow paragraph
+// (Stage 2): anchors and zoomed spans enter with token-level keys/values (zoomed
+// ones reconstructed from their bases), non-zoomed spans with (kbar_S, vbar_S) and
+// a +log|S| logit correction, all in ONE softmax (Fig. 2's "merge").
+//
+// Work decomposition: one CTA per (split, kv head, sequence x layer). A producer
+// warp streams 32-row tiles (anchor K/V rows, then span kbar/vbar rows with
+// inv_norm and log|S|) into a ring of shared-memory stages with 1-D bulk copies
+// (cp.async.bulk, mbarrier completion, no multicast). Four consumer warps each
+// take R = 32/G rows of a tile for all G query heads of the kv head (GQA: one K/V
+// read serves G heads); each lane owns D/32 dimensions. 32 partial dot products
+// per lane are finished with one transpose-reduce (31 shuffles), after which
+// lane L holds the logit of (row L/G, head L%G). The routing logit reuses that
+// same q.kbar value. Zoomed spans go to a per-warp queue and are attended after
+// the stream, without materialising K_S: u = B_S q, scores A_S u, y = C_S^T p,
+// contribution y^T D_S. Softmax state is kept in the log2 domain; splits are
+// merged by log-sum-exp in a second small kernel.
+#include "sekv_common.cuh"
+#include "sekv_internal.h"
+
+namespace sekv {
+
+constexpr int kNW = 4;          // consumer warps per CTA
+constexpr int kRMax = 64;       // largest basis rank the decode accepts
+
+template <int DT, int D, int G>
+struct DecCfg {
+    static constexpr int DPL = D / 32;                      // dims per lane
+    static constexpr int R = 32 / G;                        // rows per warp per tile
+    static constexpr int TR = kNW * R;                      // rows per tile
+    static constexpr int ESZ = Elt<DT>::bytes;
+    static constexpr int ROWB = D * ESZ;                    // bytes of one K/V row
+    static constexpr int TILE = TR * ROWB;                  // bytes of one K (or V) tile
+    static constexpr int STAGE = 2 * TILE + 2 * TR * 4;     // + inv_norm + logS
+    static constexpr int NS0 = (64 * 1024) / STAGE;             // ~64 KB of stages
+    static constexpr int NS = NS0 < 2 ? 2 : (NS0 > 6 ? 6 : NS0);   // ring depth
+    static constexpr int YPL = kRMax * G / 32;              // y entries per lane
+    static constexpr int WSCR = (32 * G) + 2 * kRMax * G;   // per-warp scratch floats
+};
+
+struct DecArgs {
+    const char* q;
+    const int32_t* a_count;
+    const int32_t* m_count;
+    const int32_t* span_beg;
+    const int32_t* span_end;
+    const float* logS;
+    const int64_t* blk_off;
+    const char* Ka;
+    const char* Va;
+    const char* kbar;
+    const char* vbar;
+    const float* inv_norm;
+    const float* theta;
+    const char* arena;
+    const int64_t* slot;
+    uint32_t* zmask;
+    float* route_logits;
+    int32_t* status;
+    float* part_o;    // [B*Lr*Hkv][G][nsplit][D]
+    float* part_ml;   // [B*Lr*Hkv][G][nsplit][2]  (max, sum) in the log2 domain
+    int64_t region;
+    float scale;
+    int L, l0, Lr, Hq, Hkv, a_cap, m_cap, rank, phase, nsplit, sch_max, qcap, mw;
+};
+
+template <int DT, int D, int G>
+static size_t decode_smem_bytes(int sch_max, int qcap) {
+    using C = DecCfg<DT, D, G>;
+    size_t s = 128;                                            // barriers + flags
+    s += (size_t)C::NS * C::STAGE;
+    s += (size_t)kNW * qcap * 4;                               // zoom queues
+    s += (size_t)G * (sch_max / 32) * 4;                       // zoom-mask words
+    s += (size_t)kNW * C::WSCR * 4;                            // per-warp scratch
+    return round_up(s, 128);
+}
+
+template <int DT, int D, int G>
+__global__ void __launch_bounds__((kNW + 1) * 32)
+decode_kernel(const DecArgs a) {
+    using C = DecCfg<DT, D, G>;
+    constexpr int DPL = C::DPL, R = C::R, TR = C::TR, NS = C::NS;
+    extern __shared__ __align__(128) unsigned char sm[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm);
+    uint64_t* empty = full + NS;
+    unsigned char* stages = sm + 128;
+    int* zq = reinterpret_cast<int*>(stages + (size_t)NS * C::STAGE);
+    uint32_t* zw = reinterpret_cast<uint32_t*>(zq + kNW * a.qcap);
+    const int zwords = a.sch_max / 32;
+    float* wscr = reinterpret_cast<float*>(zw + G * zwords);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int kvh = blockIdx.y;
+    const int b = blockIdx.z / a.Lr, li = blockIdx.z % a.Lr, l = a.l0 + li;
+    const int split = blockIdx.x;
+    const int64_t unit = ((int64_t)b * a.L + l) * a.Hkv + kvh;            // global (b, l, kvh)
+    const int64_t lunit = ((int64_t)b * a.Lr + li) * a.Hkv + kvh;         // within this launch
+    const bool route_only = a.phase == SEKV_ROUTE;
+
+    const int ab = min(a.a_count[b], a.a_cap);
+    const int mb = min(a.m_count[b], a.m_cap);
+    int a0 = 0, a1 = 0;
+    if (!route_only) {
+        const int ach = (ab + a.nsplit - 1) / a.nsplit;
+        a0 = min(ab, split * ach);
+        a1 = min(ab, a0 + ach);
+    }
+    const int sch = (((mb + a.nsplit - 1) / a.nsplit) + 31) & ~31;
+    const int s0 = split * sch;
+    const int s1 = min(mb, s0 + sch);
+    const int nta = (a1 - a0 + TR - 1) / TR;
+    const int nts = s1 > s0 ? (s1 - s0 + TR - 1) / TR : 0;
+    const int ntiles = nta + nts;
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kNW);
+        }
+        fence_barrier_init();
+    }
+    for (int i = tid; i < G * zwords; i += blockDim.x) zw[i] = 0u;
+    __syncthreads();
+
+    const float sl2 = a.scale * kLog2e;
+    // per-warp softmax state (warp-uniform) and per-lane output slice
+    float m_run[G], l_run[G], o[G][DPL];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        m_run[h] = -INFINITY;
+        l_run[h] = 0.f;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) o[h][i] = 0.f;
+    }
+
+    if (warp == kNW) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < ntiles; ++i) {
+                const int s = i % NS;
+                if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) {
+                    set_status(a.status, SEKV_ERR_TIMEOUT);
+                    break;
+                }
+                unsigned char* st = stages + (size_t)s * C::STAGE;
+                if (i < nta) {
+                    const int r0 = a0 + i * TR;
+                    const uint32_t bytes = (uint32_t)min(TR, a1 - r0) * C::ROWB;
+                    mbar_arrive_expect_tx(&full[s], 2 * bytes);
+                    const int64_t off = (unit * a.a_cap + r0) * C::ROWB;
+                    bulk_g2s(st, a.Ka + off, bytes, &full[s]);
+                    bulk_g2s(st + C::TILE, a.Va + off, bytes, &full[s]);
+                } else {
+                    const int S0 = s0 + (i - nta) * TR;
+                    const int rows = min(TR, s1 - S0);
+                    const uint32_t bytes = (uint32_t)rows * C::ROWB;
+                    const uint32_t mbytes = (uint32_t)((rows + 3) & ~3) * 4;
+                    mbar_arrive_expect_tx(&full[s], (route_only ? bytes : 2 * bytes) + 2 * mbytes);
+                    const int64_t off = (unit * a.m_cap + S0) * C::ROWB;
+                    bulk_g2s(st, a.kbar + off, bytes, &full[s]);
+                    if (!route_only) bulk_g2s(st + C::TILE, a.vbar + off, bytes, &full[s]);
+                    bulk_g2s(st + 2 * C::TILE, a.inv_norm + unit * a.m_cap + S0, mbytes, &full[s]);
+                    bulk_g2s(st + 2 * C::TILE + TR * 4, a.logS + (int64_t)b * a.m_cap + S0, mbytes, &full[s]);
+                }
+                issued = i + 1;
+            }
+            // drain: every issued copy has landed before the CTA may exit
+            for (int i = max(0, issued - NS); i < issued; ++i)
+                if (!mbar_wait(&full[i % NS], (i / NS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
+        }
+    } else {
+        // ------------------------------------------------------------ consumers
+        const int rL = lane / G, hL = lane % G;
+        float q[G][DPL];
+        {
+            const char* qp = a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB +
+                             lane * DPL * C::ESZ;
+#pragma unroll
+            for (int h = 0; h < G; ++h) Vec<DT, DPL>::load(qp + h * C::ROWB, q[h]);
+        }
+        const float th = a.theta[(int64_t)l * a.Hq + kvh * G + hL];
+        float m_lane = -INFINITY;                       // == m_run[hL]
+        int qn = 0;                                     // zoom-queue length (warp-uniform)
+        int* myq = zq + warp * a.qcap;
+        float* pb = wscr + warp * C::WSCR;              // 32*G floats (tile p / token p)
+        float* ub = pb + 32 * G;                        // kRMax*G floats
+        float* yb = ub + kRMax * G;                     // kRMax*G floats
+        const int rbase = warp * R;
+        bool ok = true;
+
+        for (int i = 0; i < ntiles && ok; ++i) {
+            const int s = i % NS;
+            if (!mbar_wait(&full[s], (i / NS) & 1)) {
+                set_status(a.status, SEKV_ERR_TIMEOUT);
+                ok = false;
+                break;
+            }
+            const unsigned char* st = stages + (size_t)s * C::STAGE;
+            const bool anchor_tile = i < nta;
+            const int S0 = s0 + (i - nta) * TR;
+            const int trows = anchor_tile ? min(TR, a1 - (a0 + i * TR)) : min(TR, s1 - S0);
+            float part[32];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                float kk[DPL];
+                if (rbase + r < trows) {
+                    Vec<DT, DPL>::load(st + (rbase + r) * C::ROWB + lane * DPL * C::ESZ, kk);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < DPL; ++k) kk[k] = 0.f;
+                }
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int k = 0; k < DPL; ++k) acc = fmaf(kk[k], q[h][k], acc);
+                    part[r * G + h] = acc;
+                }
+            }
+            const float x = transpose_reduce32(part, lane);
+            const int rowL = rbase + rL;
+            const bool validL = rowL < trows;
+            float lg2 = -INFINITY;
+            if (anchor_tile) {
+                if (validL) lg2 = x * sl2;
+            } else {
+                const float invn = reinterpret_cast<const float*>(st + 2 * C::TILE)[rowL];
+                const float ls = reinterpret_cast<const float*>(st + 2 * C::TILE + TR * 4)[rowL];
+                const int SL = S0 + rowL;
+                const float ell = fmaf(x * invn, a.scale, ls);      // Eq. (5) pre-sigmoid logit
+                const bool z = validL && (ell > th);                // Eq. (9)
+                if (validL && a.route_logits)
+                    a.route_logits[(((int64_t)b * a.L + l) * a.Hq + kvh * G + hL) * a.m_cap + SL] = ell;
+                if (z) atomicOr(&zw[hL * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
+                if (!route_only) {
+                    const uint32_t zb = __ballot_sync(0xffffffffu, z);
+                    const uint32_t hm = (zb >> (rL * G)) & ((1u << G) - 1u);
+                    const bool head_lane = (hL == 0) && validL && hm != 0u;
+                    const uint32_t rows_with = __ballot_sync(0xffffffffu, head_lane);
+                    if (head_lane) {
+                        const int pos = qn + __popc(rows_with & ((1u << lane) - 1u));
+                        if (pos < a.qcap) myq[pos] = SL | (int)(hm << 24);
+                    }
+                    qn += __popc(rows_with);
+                    if (validL && !z) lg2 = fmaf(x, a.scale, ls) * kLog2e;
+                }
+            }
+            if (!route_only) {
+                // online softmax over this tile's rows, per head
+                float mx = lg2;
+#pragma unroll
+                for (int off = G; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                const float m_lane_new = fmaxf(m_lane, mx);
+                const float p = (lg2 == -INFINITY) ? 0.f : exp2f(lg2 - m_lane_new);
+                float ps = p;
+#pragma unroll
+                for (int off = G; off < 32; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+                float alpha[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float mnew = fmaxf(m_run[h], __shfl_sync(0xffffffffu, mx, h));
+                    alpha[h] = (mnew == -INFINITY) ? 1.f : exp2f(m_run[h] - mnew);
+                    l_run[h] = fmaf(l_run[h], alpha[h], __shfl_sync(0xffffffffu, ps, h));
+                    m_run[h] = mnew;
+                }
+                m_lane = m_lane_new;
+                pb[lane] = p;
+                __syncwarp();
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+#pragma unroll
+                    for (int k = 0; k < DPL; ++k) o[h][k] *= alpha[h];
+                const unsigned char* vt = st + C::TILE;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    if (rbase + r < trows) {
+                        float vv[DPL];
+                        Vec<DT, DPL>::load(vt + (rbase + r) * C::ROWB + lane * DPL * C::ESZ, vv);
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float pr = pb[r * G + h];
+#pragma unroll
+                            for (int k = 0; k < DPL; ++k) o[h][k] = fmaf(pr, vv[k], o[h][k]);
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+
+        // ---------------------------------------------------- zoomed spans
+        if (!route_only && ok) {
+            const int nq = min(qn, a.qcap);
+            for (int e = 0; e < nq; ++e) {
+                const int ent = myq[e];
+                const int S = ent & 0xffffff;
+                const uint32_t hm = (uint32_t)ent >> 24;
+                const int beg = a.span_beg[(int64_t)b * a.m_cap + S];
+                const int len = a.span_end[(int64_t)b * a.m_cap + S] - beg;
+                if (len < 1) {
+                    set_status(a.status, SEKV_ERR_INVALID_ARG);
+                    continue;
+                }
+                const int rS = block_rank(len, D, a.rank);
+                const int64_t pa = block_ac_elems(len, rS);
+                const int64_t be = block_elems(len, D, a.rank);
+                int64_t off;
+                if (a.slot) {
+                    off = a.slot[((int64_t)b * a.L + l) * a.m_cap + S];
+                    if (off < 0) {
+                        set_status(a.status, SEKV_ERR_COLD_SPAN);
+                        continue;
+                    }
+                } else {
+                    off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S];
+                }
+                const char* blk = a.arena + (off + (int64_t)kvh * be) * C::ESZ;
+                const char* Ap = blk;
+                const char* Cp = blk + pa * C::ESZ;
+                const char* Bp = blk + 2 * pa * C::ESZ;
+                const char* Dp = Bp + (int64_t)rS * D * C::ESZ;
+
+                // (1) u[i][h] = B_i . q_h
+                for (int i0 = 0; i0 < rS; i0 += R) {
+                    float part[32];
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        float kk[DPL];
+                        if (i0 + r < rS) {
+                            Vec<DT, DPL>::load(Bp + (int64_t)(i0 + r) * C::ROWB + lane * DPL * C::ESZ, kk);
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < DPL; ++k) kk[k] = 0.f;
+                        }
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            float acc = 0.f;
+#pragma unroll
+                            for (int k = 0; k < DPL; ++k) acc = fmaf(kk[k], q[h][k], acc);
+                            part[r * G + h] = acc;
+                        }
+                    }
+                    const float u = transpose_reduce32(part, lane);
+                    if (i0 + rL < rS) ub[(i0 + rL) * G + hL] = u;
+                }
+                __syncwarp();
+
+                // (2) token scores s_t = A_t . u (scaled), span-local online softmax, y = C^T p
+                float msp[G], lsp[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) { msp[h] = -INFINITY; lsp[h] = 0.f; }
+                float y[C::YPL];
+#pragma unroll
+                for (int j = 0; j < C::YPL; ++j) y[j] = 0.f;
+                for (int t0 = 0; t0 < len; t0 += 32) {
+                    const int t = t0 + lane;
+                    float xs[G];
+#pragma unroll
+                    for (int h = 0; h < G; ++h) xs[h] = 0.f;
+                    if (t < len) {
+                        for (int i = 0; i < rS; ++i) {
+                            const float av = load1<DT>(Ap, (int64_t)t * rS + i);
+#pragma unroll
+                            for (int h = 0; h < G; ++h) xs[h] = fmaf(av, ub[i * G + h], xs[h]);
+                        }
+                    }
+                    float alL = 1.f;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float lg = (t < len && ((hm >> h) & 1u)) ? xs[h] * sl2 : -INFINITY;
+                        const float cm = warp_max(lg);
+                        const float mnew = fmaxf(msp[h], cm);
+                        const float al = (mnew == -INFINITY) ? 1.f : exp2f(msp[h] - mnew);
+                        const float p = (lg == -INFINITY) ? 0.f : exp2f(lg - mnew);
+                        lsp[h] = fmaf(lsp[h], al, warp_sum(p));
+                        msp[h] = mnew;
+                        pb[lane * G + h] = p;
+                        if (h == hL) alL = al;
+                    }
+                    __syncwarp();
+                    const int tn = min(32, len - t0);
+#pragma unroll
+                    for (int j = 0; j < C::YPL; ++j) {
+                        const int i = (lane + 32 * j) / G;
+                        if (i < rS) {
+                            float acc = y[j] * alL;
+                            for (int tt = 0; tt < tn; ++tt)
+                                acc = fmaf(pb[tt * G + hL], load1<DT>(Cp, (int64_t)(t0 + tt) * rS + i), acc);
+                            y[j] = acc;
+                        }
+                    }
+                    __syncwarp();
+                }
+
+                // (3) merge the span into the running state: o += beta * y^T D
+                float betaL = 0.f;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    float al = 1.f, be2 = 0.f;
+                    if ((hm >> h) & 1u) {
+                        const float mnew = fmaxf(m_run[h], msp[h]);
+                        al = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mnew);
+                        be2 = exp2f(msp[h] - mnew);
+                        l_run[h] = l_run[h] * al + lsp[h] * be2;
+                        m_run[h] = mnew;
+                    }
+#pragma unroll
+                    for (int k = 0; k < DPL; ++k) o[h][k] *= al;
+                    if (h == hL) { betaL = be2; m_lane = m_run[h]; }
+                }
+#pragma unroll
+                for (int j = 0; j < C::YPL; ++j) {
+                    const int i = (lane + 32 * j) / G;
+                    if (i < rS) yb[i * G + hL] = y[j] * betaL;
+                }
+                __syncwarp();
+                for (int i = 0; i < rS; ++i) {
+                    float dv[DPL];
+                    Vec<DT, DPL>::load(Dp + (int64_t)i * C::ROWB + lane * DPL * C::ESZ, dv);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float yv = yb[i * G + h];
+#pragma unroll
+                        for (int k = 0; k < DPL; ++k) o[h][k] = fmaf(yv, dv[k], o[h][k]);
+                    }
+                }
+                __syncwarp();
+            }
+        }
+    }
+    __syncthreads();
+
+    // ------------------------------------------------ zoom-mask words of this CTA
+    if (a.zmask) {
+        const int w0 = s0 >> 5;
+        const int wend = (split == a.nsplit - 1) ? a.mw : min(a.mw, w0 + (sch >> 5));
+        for (int i = tid; i < G * max(0, wend - w0); i += blockDim.x) {
+            const int h = i / (wend - w0), j = i % (wend - w0);
+            a.zmask[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.mw + w0 + j] =
+                (j < zwords) ? zw[h * zwords + j] : 0u;
+        }
+    }
+    if (route_only) return;
+
+    // ------------------------------------------------ merge the warps of this CTA
+    float* wm = reinterpret_cast<float*>(stages);          // [kNW][G]
+    float* wl = wm + kNW * G;                               // [kNW][G]
+    float* wo = wl + kNW * G;                               // [kNW][G][D]
+    if (warp < kNW) {
+        if (lane == 0) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                wm[warp * G + h] = m_run[h];
+                wl[warp * G + h] = l_run[h];
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int k = 0; k < DPL; ++k) wo[(warp * G + h) * D + lane * DPL + k] = o[h][k];
+    }
+    __syncthreads();
+    for (int i = tid; i < G * D; i += blockDim.x) {
+        const int h = i / D, k = i % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) M = fmaxf(M, wm[w * G + h]);
+        float Ls = 0.f, Os = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kNW; ++w) {
+                const float f = exp2f(wm[w * G + h] - M);
+                Ls = fmaf(wl[w * G + h], f, Ls);
+                Os = fmaf(wo[(w * G + h) * D + k], f, Os);
+            }
+        }
+        const int64_t pidx = (lunit * G + h) * a.nsplit + split;
+        a.part_o[pidx * D + k] = Os;
+        if (k == 0) {
+            a.part_ml[pidx * 2 + 0] = M;
+            a.part_ml[pidx * 2 + 1] = Ls;
+        }
+    }
+}
+
+// one CTA of D threads per (b, l, query head)
+template <int D>
+__global__ void merge_kernel(const float* part_o, const float* part_ml, float* O, float* lse, int nsplit,
+                             int G, int Hkv, int L, int l0, int Lr, int Hq) {
+    const int idx = blockIdx.x;
+    const int hq = idx % Hq;
+    const int li = (idx / Hq) % Lr;
+    const int b = idx / (Hq * Lr);
+    const int kvh = hq / G, h = hq % G;
+    const int64_t lunit = ((int64_t)b * Lr + li) * Hkv + kvh;
+    const int64_t base = (lunit * G + h) * nsplit;
+    const int k = threadIdx.x;
+    float M = -INFINITY;
+    for (int j = 0; j < nsplit; ++j) M = fmaxf(M, part_ml[(base + j) * 2]);
+    float Ls = 0.f, Os = 0.f;
+    if (M != -INFINITY) {
+        for (int j = 0; j < nsplit; ++j) {
+            const float f = exp2f(part_ml[(base + j) * 2] - M);
+            Ls = fmaf(part_ml[(base + j) * 2 + 1], f, Ls);
+            Os = fmaf(part_o[(base + j) * D + k], f, Os);
+        }
+    }
+    const int64_t out = ((int64_t)b * L + l0 + li) * Hq + hq;
+    O[out * D + k] = Ls > 0.f ? Os / Ls : 0.f;
+    if (k == 0) lse[out] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static int num_sms() {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 148;
+}
+
+bool decode_supported(const sekv_decode_desc& d) {
+    const int G = d.Hkv > 0 ? d.Hq / d.Hkv : 0;
+    return (d.d == 64 || d.d == 128) && (G == 1 || G == 2 || G == 4 || G == 8) && d.rank >= 1 &&
+           d.rank <= kRMax && (d.dtype == SEKV_F32 || d.dtype == SEKV_BF16);
+}
+
+DecodePlan plan_decode(const sekv_decode_desc& d) {
+    DecodePlan p{};
+    const int Lr = d.l1 - d.l0;
+    const int64_t units = (int64_t)d.B * Lr * d.Hkv;
+    int ns = d.nsplit;
+    if (ns <= 0) {
+        // about two waves of ~3 resident CTAs per SM
+        const int64_t target = 2LL * 3 * num_sms();
+        ns = (int)((target + units - 1) / units);
+        const int by_rows = (int)((d.a_cap + d.m_cap) / 256);     // keep >= ~256 rows per split
+        ns = ns < by_rows ? ns : by_rows;
+    }
+    const int max_ns = d.m_cap / 32 > 0 ? d.m_cap / 32 : 1;
+    if (ns > max_ns) ns = max_ns;
+    if (ns < 1) ns = 1;
+    p.nsplit = ns;
+    p.span_chunk = (int)round_up((d.m_cap + ns - 1) / ns, 32);
+    p.anchor_chunk = (d.a_cap + ns - 1) / ns;
+    const int G = d.Hq / d.Hkv;
+    p.partial_bytes = (size_t)round_up((int64_t)units * G * ns * (d.d + 2) * 4, 256);
+    return p;
+}
+
+size_t decode_workspace_bytes(const sekv_decode_desc& d) { return plan_decode(d).partial_bytes; }
+
+template <int DT, int D, int G>
+static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st) {
+    using C = DecCfg<DT, D, G>;
+    const int Lr = d.l1 - d.l0;
+    const int64_t units = (int64_t)d.B * Lr * d.Hkv;
+    DecArgs a;
+    a.q = (const char*)d.q;
+    a.a_count = d.a_count; a.m_count = d.m_count; a.span_beg = d.span_beg; a.span_end = d.span_end;
+    a.logS = d.logS; a.blk_off = d.blk_off;
+    a.Ka = (const char*)d.Ka; a.Va = (const char*)d.Va; a.kbar = (const char*)d.kbar; a.vbar = (const char*)d.vbar;
+    a.inv_norm = d.inv_norm; a.theta = d.theta; a.arena = (const char*)d.arena; a.slot = d.slot;
+    a.zmask = d.zmask; a.route_logits = d.route_logits; a.status = d.dev_status;
+    a.part_o = reinterpret_cast<float*>(partials);
+    a.part_ml = a.part_o + units * G * p.nsplit * D;
+    a.region = d.region_elems; a.scale = d.scale;
+    a.L = d.L; a.l0 = d.l0; a.Lr = Lr; a.Hq = d.Hq; a.Hkv = d.Hkv; a.a_cap = d.a_cap; a.m_cap = d.m_cap;
+    a.rank = d.rank; a.phase = d.phase; a.nsplit = p.nsplit; a.sch_max = p.span_chunk;
+    a.qcap = ((p.span_chunk + C::TR - 1) / C::TR) * C::R;
+    a.mw = d.m_cap / 32;
+    const size_t smem = decode_smem_bytes<DT, D, G>(a.sch_max, a.qcap);
+    if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.nsplit, d.Hkv, d.B * Lr);
+    decode_kernel<DT, D, G><<<grid, (kNW + 1) * 32, smem, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (d.phase != SEKV_ROUTE) {
+        merge_kernel<D><<<d.B * Lr * d.Hq, D, 0, st>>>(a.part_o, a.part_ml, d.O, d.lse, p.nsplit, G, d.Hkv,
+                                                        d.L, d.l0, Lr, d.Hq);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+template <int DT, int D>
+static cudaError_t launch_g(const sekv_decode_desc& d, const DecodePlan& p, void* w, cudaStream_t st) {
+    switch (d.Hq / d.Hkv) {
+        case 1: return launch_t<DT, D, 1>(d, p, w, st);
+        case 2: return launch_t<DT, D, 2>(d, p, w, st);
+        case 4: return launch_t<DT, D, 4>(d, p, w, st);
+        default: return launch_t<DT, D, 8>(d, p, w, st);
+    }
+}
+
+cudaError_t launch_decode(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st) {
+    if (d.dtype == SEKV_F32)
+        return d.d == 64 ? launch_g<SEKV_F32, 64>(d, p, partials, st) : launch_g<SEKV_F32, 128>(d, p, partials, st);
+    return d.d == 64 ? launch_g<SEKV_BF16, 64>(d, p, partials, st) : launch_g<SEKV_BF16, 128>(d, p, partials, st);
+}
+
+}  // namespace sekv

@@ -1,0 +1,30 @@
+// Host-side launchers shared between the kernel files and the C ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "../../include/sekv.h"
+
+namespace sekv {
+
+cudaError_t launch_scan(const sekv_build_desc& d, cudaStream_t st);
+cudaError_t launch_layout(const sekv_build_desc& d, bool check_region, cudaStream_t st);
+cudaError_t launch_summary(const sekv_build_desc& d, cudaStream_t st);
+
+// basis build: workspace layout and launch
+size_t basis_workspace_bytes(const sekv_build_desc& d);
+cudaError_t launch_basis(const sekv_build_desc& d, cudaStream_t st);
+
+// decode
+struct DecodePlan {
+    int nsplit;        // CTAs per (b, l, kv head)
+    int span_chunk;    // spans per split (multiple of 32)
+    int anchor_chunk;  // anchors per split
+    size_t partial_bytes;
+};
+DecodePlan plan_decode(const sekv_decode_desc& d);
+size_t decode_workspace_bytes(const sekv_decode_desc& d);
+bool decode_supported(const sekv_decode_desc& d);
+cudaError_t launch_decode(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st);
+
+}  // namespace sekv

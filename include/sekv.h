@@ -1,0 +1,242 @@
+/*
+ * sekv.h - C ABI of the SeKV span-structured KV cache library (CUDA, sm_100a).
+ *
+ * The library implements the data-parallel hot path of SeKV (resolution-adaptive
+ * KV cache with hierarchical semantic memory):
+ *
+ *   prefill  sekv_build_spans   surprisal boundary scan -> anchors and spans,
+ *                               anchor gather, per-span weighted-mean key/value,
+ *                               per-span rank-r bases (Gram + Jacobi);
+ *   decode   sekv_decode_attn   per-head routing over span summaries, zoom mask,
+ *                               one softmax over anchors, summaries (+log|S|) and
+ *                               low-rank reconstructed tokens of zoomed spans;
+ *   fetch    sekv_fetch_bases   copy the bases of zoomed spans from pinned host
+ *                               memory into a device arena (cold spans).
+ *
+ * Sources, by page title and section:
+ *   "SeKV: Resolution-Adaptive KV Cache with Hierarchical Semantic Memory" -
+ *   the SeKV blog walkthrough (liuzhao09.github.io), section 2.1 Eq. (1) and the
+ *   rule H_t > mu + alpha*sigma; section 2.2 Eq. (2), (3), Fig. 2, Eq. (6)-(8);
+ *   section 2.3 Eq. (5), (9); and the SeKV summary page (paper.rainbus.top),
+ *   workflow paragraph (Stage-2 shared softmax with the log|S| correction).
+ *
+ * Conventions for every entry point
+ *   - All buffers are caller-owned. The library never allocates device or pinned
+ *     memory and never frees anything. "device" pointers must be device memory
+ *     of the current device; "host" pointers are ordinary or pinned host memory
+ *     as stated; the basis home may be pinned host memory (it is read and written
+ *     through unified addressing).
+ *   - Element types: SEKV_F32 = float, SEKV_BF16 = bfloat16 (2 bytes). K, V, q
+ *     and every stored K/V-shaped output use the descriptor's dtype; logS,
+ *     inv_norm, theta, O and lse are float; counts and positions are int32;
+ *     block offsets and slots are int64 element offsets.
+ *   - Arrays are dense row-major in the bracket order given.
+ *   - Host-side argument checks happen before any launch; on failure the call
+ *     returns SEKV_ERR_INVALID_ARG / SEKV_ERR_UNSUPPORTED and launches nothing.
+ *     A CUDA launch error returns SEKV_ERR_CUDA (text: sekv_last_error()).
+ *     Errors found on the device (capacity overflow, a cold span in ATTEND, a
+ *     bounded wait that ran out, a Jacobi solve that did not converge) are
+ *     written to *dev_status (device int32; first error wins; 0 = ok); kernels
+ *     then skip the offending work and return, they never trap.
+ *   - Work is enqueued on the given stream; calls do not synchronise unless
+ *     stated (sekv_fetch_bases waits on the host for the routing result).
+ *   - Calls are stateless: concurrent calls on different streams with disjoint
+ *     output buffers are safe.
+ */
+#ifndef SEKV_H_
+#define SEKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SEKV_VERSION 1
+
+typedef enum {
+    SEKV_OK = 0,
+    SEKV_ERR_INVALID_ARG = 1,   /* a pointer, size or enum is out of range      */
+    SEKV_ERR_CAPACITY = 2,      /* a_cap, m_cap, region or arena too small        */
+    SEKV_ERR_CUDA = 3,          /* a CUDA call failed (see sekv_last_error)       */
+    SEKV_ERR_COLD_SPAN = 4,     /* ATTEND met a zoomed span whose bases are cold */
+    SEKV_ERR_TIMEOUT = 5,       /* a bounded device wait ran out                  */
+    SEKV_ERR_UNSUPPORTED = 6,   /* shape outside the compiled variants            */
+    SEKV_WARN_NOT_CONVERGED = 7 /* a Jacobi solve hit max_sweeps (result kept)    */
+} sekv_status;
+
+enum { SEKV_F32 = 0, SEKV_BF16 = 1 };
+
+/* Per-token span weights for the weighted means (SeKV blog 2.2):
+ * UNIFORM w_t = 1; SURPRISAL w_t = H_t / sum_S H (Eq. 2, uniform if the sum is 0);
+ * SOFTMAX w_t = exp(H_t) / sum_S exp(H). */
+enum { SEKV_W_UNIFORM = 0, SEKV_W_SURPRISAL = 1, SEKV_W_SOFTMAX = 2 };
+
+/* Build steps (bit mask). SCAN and LAYOUT work per sequence, SUMMARY and BASES
+ * per layer range [l0, l1). Without SCAN, LAYOUT/SUMMARY/BASES use the anchor and
+ * span arrays already in the descriptor (caller-supplied segmentation). */
+enum {
+    SEKV_BUILD_SCAN = 1,     /* boundary rule -> a_count, anchor_pos, m_count, span_beg/end */
+    SEKV_BUILD_LAYOUT = 2,   /* logS and blk_off from the spans                             */
+    SEKV_BUILD_SUMMARY = 4,  /* Ka/Va gather, kbar/vbar, inv_norm                           */
+    SEKV_BUILD_BASES = 8,    /* per-span A,B (keys) and C,D (values) into basis_home        */
+    SEKV_BUILD_ALL = 15
+};
+
+/* Decode phases. FUSED: routing + attention in one pass over a hot cache.
+ * ROUTE: routing only (writes zmask / route_logits). ATTEND: routing again
+ * (bit-identical) + attention, reading bases through the slot table. */
+enum { SEKV_FUSED = 0, SEKV_ROUTE = 1, SEKV_ATTEND = 2 };
+
+typedef void* sekv_stream_t;   /* a cudaStream_t (NULL = legacy default stream) */
+typedef void* sekv_event_t;    /* a cudaEvent_t */
+
+/*
+ * Basis storage. For each (b, l) there is a region of region_elems elements
+ * (storage dtype). Span S of sequence b owns the Hkv consecutive blocks starting
+ * at element blk_off[b][S] of the region, one block per kv head:
+ *     block = [ A (|S| x rS) | pad | C (|S| x rS) | pad | B (rS x d) | D (rS x d) | pad ]
+ * with rS = min(rank, |S|, d); A and C each take roundup(|S|*rS, 8) elements and
+ * the block is padded to a multiple of 64 elements (sekv_block_elems). K_S ~ A B,
+ * V_S ~ C D (SeKV blog 2.2, Eq. (6)-(8) with the rank gate fixed to 1).
+ */
+int64_t sekv_block_elems(int32_t len, int32_t d, int32_t rank);
+/* An upper bound of the region size for any segmentation with <= m_cap spans of a
+ * sequence of n tokens: Hkv * (2*n*rank + m_cap*(2*rank*d + 80)). */
+int64_t sekv_basis_region_bound(int32_t n, int32_t m_cap, int32_t Hkv, int32_t d, int32_t rank);
+
+/* ------------------------------------------------------------------------- */
+/* Prefill build (SeKV blog 2.1 Eq. (1) + boundary rule; 2.2 Eq. (2), (6)-(8)) */
+/* ------------------------------------------------------------------------- */
+typedef struct sekv_build_desc {
+    /* inputs (device) */
+    const float* H;          /* [B][n] surprisal H_t = -log p(x_t | x_<t)                 */
+    const void* K;           /* [B][L][Hkv][n][d] keys (all L layers; rows of [l0,l1) read) */
+    const void* V;           /* [B][L][Hkv][n][d] values                                   */
+    /* segmentation (device; outputs of SCAN/LAYOUT, inputs otherwise) */
+    int32_t* a_count;        /* [B] anchors per sequence (boundaries + local window)       */
+    int32_t* m_count;        /* [B] spans per sequence                                     */
+    int32_t* anchor_pos;     /* [B][a_cap] ascending token positions of the anchors        */
+    int32_t* span_beg;       /* [B][m_cap] first token of span S                           */
+    int32_t* span_end;       /* [B][m_cap] one past the last token of span S               */
+    float* logS;             /* [B][m_cap] log|S| (float)                                  */
+    int64_t* blk_off;        /* [B][m_cap+1] element offset of span S's blocks in a region */
+    double* stats;           /* optional [B][3]: mu, sigma, threshold (fp64)               */
+    /* anchor and summary store (device; outputs of SUMMARY) */
+    void* Ka;                /* [B][L][Hkv][a_cap][d] anchor keys                          */
+    void* Va;                /* [B][L][Hkv][a_cap][d] anchor values                        */
+    void* kbar;              /* [B][L][Hkv][m_cap][d] weighted-mean key per span           */
+    void* vbar;              /* [B][L][Hkv][m_cap][d] weighted-mean value per span         */
+    float* inv_norm;         /* [B][L][Hkv][m_cap] 1/||stored kbar|| (0 for a zero vector) */
+    /* bases (output of BASES): device memory (hot) or pinned host memory (cold) */
+    void* basis_home;        /* [B][L][region_elems]                                       */
+    int32_t* dev_status;     /* device int32, required                                     */
+    void* workspace;         /* device, sekv_build_workspace_bytes() bytes, 256-B aligned  */
+    int64_t region_elems;    /* elements per (b, l) region of basis_home                   */
+    int64_t workspace_bytes;
+    double alpha;            /* boundary sensitivity: boundary iff H_t > mu + alpha*sigma   */
+    int32_t B, L, Hkv, n, d, dtype;
+    int32_t l0, l1;          /* layer range of SUMMARY/BASES, 0 <= l0 < l1 <= L            */
+    int32_t a_cap, m_cap;    /* capacities; m_cap must be a multiple of 32                 */
+    int32_t window;          /* the last `window` positions are anchors                    */
+    int32_t wmode;           /* SEKV_W_*                                                    */
+    int32_t rank;            /* basis rank r >= 1                                           */
+    int32_t max_sweeps;      /* Jacobi sweep limit (e.g. 15)                               */
+    int32_t steps;           /* SEKV_BUILD_* mask                                           */
+    int32_t reserved;
+} sekv_build_desc;
+
+size_t sekv_build_workspace_bytes(const sekv_build_desc* desc);
+/* Enqueue the requested build steps on `stream`. d must be 64 or 128. */
+sekv_status sekv_build_spans(const sekv_build_desc* desc, sekv_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Decode attention (SeKV blog 2.3 Eq. (5), (9); SeKV summary, Stage 2)      */
+/* ------------------------------------------------------------------------- */
+typedef struct sekv_decode_desc {
+    const void* q;           /* [B][L][Hq][d] queries (storage dtype)                      */
+    const int32_t* a_count;  /* [B]                                                        */
+    const int32_t* m_count;  /* [B]                                                        */
+    const int32_t* span_beg; /* [B][m_cap]                                                 */
+    const int32_t* span_end; /* [B][m_cap]                                                 */
+    const float* logS;       /* [B][m_cap]                                                 */
+    const int64_t* blk_off;  /* [B][m_cap+1]                                               */
+    const void* Ka;          /* [B][L][Hkv][a_cap][d]                                      */
+    const void* Va;
+    const void* kbar;        /* [B][L][Hkv][m_cap][d]                                      */
+    const void* vbar;
+    const float* inv_norm;   /* [B][L][Hkv][m_cap]                                         */
+    const float* theta;      /* [L][Hq] zoom threshold in logit space, ln(tau/(1-tau))      */
+    const void* arena;       /* bases: the device home [B][L][region_elems] when slot is   */
+                             /* NULL, else a device arena addressed through slot           */
+    const int64_t* slot;     /* NULL or [B][L][m_cap]: element offset in arena of span S's  */
+                             /* Hkv blocks, -1 = cold                                      */
+    float* O;                /* [B][L][Hq][d] attention output (FUSED/ATTEND)              */
+    float* lse;              /* [B][L][Hq] natural-log partition (FUSED/ATTEND)            */
+    uint32_t* zmask;         /* optional [B][L][Hq][m_cap/32] zoom bits (bit S%32 of word   */
+                             /* S/32); required for ROUTE. Bits of spans >= m_count are 0  */
+    float* route_logits;     /* optional [B][L][Hq][m_cap] routing logits l_S              */
+    int32_t* dev_status;     /* device int32, required                                     */
+    void* workspace;         /* device, sekv_decode_workspace_bytes() bytes, 256-B aligned */
+    int64_t region_elems;
+    int64_t workspace_bytes;
+    float scale;             /* logit scale, normally 1/sqrt(d) (routing uses it too, d'=d) */
+    int32_t B, L, Hq, Hkv, d, dtype;
+    int32_t l0, l1;          /* layers decoded by this call                                */
+    int32_t a_cap, m_cap;
+    int32_t rank;
+    int32_t phase;           /* SEKV_FUSED / SEKV_ROUTE / SEKV_ATTEND                       */
+    int32_t nsplit;          /* CTAs per (b, l, kv head); 0 = automatic                    */
+} sekv_decode_desc;
+
+size_t sekv_decode_workspace_bytes(const sekv_decode_desc* desc);
+/* Enqueue one decode step for layers [l0, l1) on `stream`. Hq/Hkv must be 1, 2, 4
+ * or 8 and d 64 or 128. Routing logit per query head h and span S:
+ *   l_S = (q_h . kbar_S) * inv_norm_S * scale + logS_S, zoom iff l_S > theta[l][h];
+ * attention over anchors (q.Ka*scale), non-zoomed spans (q.kbar*scale + logS,
+ * value vbar) and the tokens of zoomed spans ((A_S (B_S q))*scale, value C_S^T-
+ * weighted D_S rows), all in one softmax. */
+sekv_status sekv_decode_attn(const sekv_decode_desc* desc, sekv_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Cold-basis fetch (SeKV summary: zoomed spans' bases fetched from the CPU;  */
+/* SeKV blog Fig. 2)                                                          */
+/* ------------------------------------------------------------------------- */
+typedef struct sekv_fetch_desc {
+    const uint32_t* zmask_dev;    /* [B][L][Hq][m_cap/32] device, written by ROUTE           */
+    uint32_t* zmask_host;         /* pinned host staging of the same shape                   */
+    const int32_t* m_count_host;  /* [B] host copy of m_count                                */
+    const int64_t* blk_off_host;  /* [B][m_cap+1] host copy of blk_off                       */
+    const void* home;             /* pinned host basis home [B][L][region_elems]             */
+    void* arena;                  /* device arena, arena_elems elements                      */
+    int64_t* slot_dev;            /* [B][L][m_cap] device slot table (written on `copy`)     */
+    int64_t* slot_host;           /* pinned host mirror of the slot table                    */
+    int64_t* stats;               /* optional host [4]: bytes copied, spans, copies, -       */
+    int64_t region_elems;
+    int64_t arena_elems;
+    int32_t B, L, Hq, Hkv, d, dtype;
+    int32_t l0, l1, m_cap, rank;
+} sekv_fetch_desc;
+
+/* Copy the bases of every span that any query head of (b, l) zooms, for layers
+ * [l0, l1), into the arena, and point the slot table at them (-1 elsewhere).
+ * Order: zmask is read back on `compute` (the host waits for it); the copies
+ * (one cudaMemcpyAsync per run of consecutive zoomed spans of a layer) and the
+ * slot-table upload go on `copy`; `done` is recorded on `copy`. The caller makes
+ * `compute` wait on `done` before ATTEND. Arena contents from earlier calls are
+ * overwritten. Returns SEKV_ERR_CAPACITY (nothing copied) if the zoomed bases
+ * exceed arena_elems. */
+sekv_status sekv_fetch_bases(const sekv_fetch_desc* desc, sekv_stream_t compute,
+                             sekv_stream_t copy, sekv_event_t done);
+
+/* ------------------------------------------------------------------------- */
+const char* sekv_status_str(int32_t status);
+const char* sekv_last_error(void);           /* thread-local detail of the last error */
+size_t sekv_desc_size(int32_t which);        /* sizeof: 0 build, 1 decode, 2 fetch     */
+int32_t sekv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SEKV_H_ */

@@ -1,0 +1,100 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, the ctypes descriptors match the C structs, and argument
+validation rejects bad calls before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "sekv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sekv_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    from hierarchical_kv_cache_span_b200 import sekv as S
+    names = _header_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(S.LIB, n), n
+        assert hasattr(S, n), f"binding lacks {n}"
+
+
+def test_descriptor_layouts_match():
+    from hierarchical_kv_cache_span_b200 import sekv as S
+    for i, cls in enumerate([S.sekv_build_desc, S.sekv_decode_desc, S.sekv_fetch_desc]):
+        assert ctypes.sizeof(cls) == S.sekv_desc_size(i)
+
+
+def test_version_and_status_strings():
+    from hierarchical_kv_cache_span_b200 import sekv as S
+    assert S.sekv_version() == 1
+    assert S.sekv_status_str(S.SEKV_ERR_COLD_SPAN).startswith("zoomed span")
+    assert S.sekv_status_str(99) == "unknown status"
+
+
+def test_block_layout_formula():
+    from hierarchical_kv_cache_span_b200 import sekv as S
+    # rS = min(r, |S|, d); A, C padded to 8 elements; block padded to 64
+    for ln, d, r in [(1, 128, 16), (5, 128, 16), (64, 128, 16), (300, 128, 32), (7, 64, 4)]:
+        rs = min(r, ln, d)
+        pa = -(-(ln * rs) // 8) * 8
+        want = -(-(2 * pa + 2 * rs * d) // 64) * 64
+        assert S.sekv_block_elems(ln, d, r) == want
+    assert S.sekv_block_elems(0, 128, 16) == 0
+
+
+def test_region_bound_covers_worst_case():
+    from hierarchical_kv_cache_span_b200 import sekv as S
+    n, m_cap, Hkv, d, r = 1000, 512, 2, 64, 8
+    bound = S.sekv_basis_region_bound(n, m_cap, Hkv, d, r)
+    # any segmentation: spans of total length <= n, count <= m_cap
+    for lens in ([1] * 500, [2] * 500, [n], [3] * 333):
+        assert Hkv * sum(S.sekv_block_elems(x, d, r) for x in lens) <= bound
+
+
+def test_invalid_build_arguments_are_rejected_before_launch():
+    from hierarchical_kv_cache_span_b200 import sekv as S
+    d = S.sekv_build_desc()
+    assert S.sekv_build_spans(d, 0) == S.SEKV_ERR_INVALID_ARG
+    d.B, d.L, d.Hkv, d.n, d.d, d.dtype, d.steps = 1, 1, 1, 16, 128, S.SEKV_BF16, S.SEKV_BUILD_SCAN
+    d.a_cap, d.m_cap = 16, 30                        # m_cap not a multiple of 32
+    assert S.sekv_build_spans(d, 0) == S.SEKV_ERR_INVALID_ARG
+    assert "multiple of 32" in S.sekv_last_error()
+    d.m_cap = 32
+    assert S.sekv_build_spans(d, 0) == S.SEKV_ERR_INVALID_ARG   # no dev_status / buffers
+
+
+def test_invalid_decode_arguments_are_rejected_before_launch():
+    from hierarchical_kv_cache_span_b200 import sekv as S
+    d = S.sekv_decode_desc()
+    d.B, d.L, d.Hq, d.Hkv, d.d, d.dtype, d.l0, d.l1 = 1, 1, 12, 4, 128, S.SEKV_BF16, 0, 1
+    d.a_cap, d.m_cap, d.rank = 32, 32, 16
+    assert S.sekv_decode_attn(d, 0) == S.SEKV_ERR_UNSUPPORTED        # G = 3 not compiled
+    d.Hq = 8
+    d.rank = 65
+    assert S.sekv_decode_attn(d, 0) == S.SEKV_ERR_UNSUPPORTED        # rank above 64
+    d.rank = 16
+    assert S.sekv_decode_attn(d, 0) == S.SEKV_ERR_INVALID_ARG        # pointers missing
+    d.phase = 7
+    assert S.sekv_decode_attn(d, 0) == S.SEKV_ERR_INVALID_ARG
+
+
+def test_invalid_fetch_arguments_are_rejected():
+    from hierarchical_kv_cache_span_b200 import sekv as S
+    d = S.sekv_fetch_desc()
+    assert S.sekv_fetch_bases(d, 0, 0, 0) == S.SEKV_ERR_INVALID_ARG
+
+
+def test_product_path_has_no_oracle_or_cpu_fallback():
+    pkg = os.path.join(ROOT, "hierarchical_kv_cache_span_b200")
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            src = open(os.path.join(pkg, fn)).read()
+            assert "oracle" not in src.replace("no oracle", ""), fn
+            assert "import numpy" not in src, fn

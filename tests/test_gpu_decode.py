@@ -1,0 +1,262 @@
+"""GPU parity of the decode attention against the fp64 oracle.
+
+Kernel level: the oracle's own stored-dtype cache is uploaded, so both sides see
+identical inputs; zoom masks must be bit-exact (routing logits kept DELTA_L away
+from theta) and O / lse within 1e-4 (fp32) or 2e-2 (bf16 inputs, fp32
+accumulation) max-abs. End to end: the library builds the cache itself.
+Invariants: singleton spans and all-zoom full-rank reduce to dense attention; the
+split count does not change the result; ROUTE + fetch + ATTEND equals FUSED.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from sekv_synth import WORKLOADS, gen
+from tests import helpers as T
+from tests.textbook import dense_attention
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    import hierarchical_kv_cache_span_b200 as P
+    return P
+
+
+def _tol(wl):
+    return 1e-4 if wl.dtype == "f32" else 2e-2
+
+
+def _cache(wl, home="device", a_cap=None, m_cap=None):
+    P = _lib()
+    ac, mc = T.caps(wl)
+    return P.SpanCache(wl.B, wl.L, wl.Hq, wl.Hkv, wl.n, wl.d, wl.dtype, a_cap or ac, m_cap or mc,
+                       wl.rank, home=home)
+
+
+def _setup(wl, quantile=None, with_bases=True):
+    """inputs + oracle cache + thresholds with margin"""
+    H, K, V = T.make_inputs(wl)
+    segs = T.oracle_segments(H, wl)
+    units = T.oracle_units(K, V, H, segs, wl, with_bases=with_bases)
+    q = gen.queries(wl)
+    scale = 1.0 / math.sqrt(wl.d)
+    taus = gen.taus(wl)
+    if quantile is None and taus is None:
+        quantile = wl.tau_a
+    theta, q = T.thetas_with_margin(q, units, segs, wl, scale, wl.G, taus=taus, quantile=quantile)
+    return H, K, V, segs, units, q, theta, scale
+
+
+def _compare(wl, c, q, theta, scale, segs, units, O_gpu, lse_gpu, zmask):
+    Oo, lseo, zooms = T.oracle_decode(q, units, segs, theta, scale, wl.G)
+    for (b, l, h), z in zooms.items():
+        np.testing.assert_array_equal(T.zmask_bits(zmask, b, l, h, len(z)), z, err_msg=str((b, l, h)))
+    err = np.abs(T.f64(O_gpu) - Oo).max()
+    lerr = np.abs(T.f64(lse_gpu) - lseo).max()
+    assert err <= _tol(wl), err
+    assert lerr <= _tol(wl), lerr
+    return err, lerr, sum(int(z.sum()) for z in zooms.values())
+
+
+KERNEL_CASES = [
+    ("c1", dict()),                                         # fp32 tiny config, tau = 0.5
+    ("c1", dict(n=777, window=40)),                         # ragged tail, window
+    ("c2", dict(n=4096, L=2)),                              # Llama shape, bf16, ~2% zoom
+    ("c4", dict(n=2048, L=2, B=3)),                         # batch, tau ~ U(0.3, 0.9)
+    ("c5", dict(n=4096, L=1, Hq=8, Hkv=2)),                 # rank 32, 25% zoom
+    ("c2", dict(n=2048, L=1, d=64, Hq=16, Hkv=2, rank=8)),  # G = 8, d = 64
+    ("c2", dict(n=2048, L=1, Hq=16, Hkv=8)),                # G = 2
+]
+
+
+@pytest.mark.parametrize("name,over", KERNEL_CASES)
+def test_decode_kernel_level(name, over):
+    P = _lib()
+    wl = WORKLOADS[name].scaled(**over)
+    H, K, V, segs, units, q, theta, scale = _setup(wl)
+    c = _cache(wl)
+    T.upload_oracle_cache(c, segs, units)
+    zmask = c.new_zmask()
+    th = torch.tensor(theta, dtype=torch.float32, device="cuda")
+    O_gpu, lse_gpu = c.decode(q.cuda(), th, zmask=zmask)
+    torch.cuda.synchronize()
+    assert c.read_status() == 0
+    err, lerr, nz = _compare(wl, c, q, theta, scale, segs, units, O_gpu, lse_gpu, zmask)
+    print(f"{name} {over}: max|dO|={err:.2e} max|dlse|={lerr:.2e} zoomed={nz}")
+
+
+@pytest.mark.parametrize("name,over", [("c1", dict()), ("c2", dict(n=4096, L=2)), ("c5", dict(n=2048, L=1))])
+def test_decode_end_to_end(name, over):
+    """library build (scan, summaries, Jacobi bases) + decode vs oracle build + decode"""
+    wl = WORKLOADS[name].scaled(**over)
+    H, K, V, segs, units, q, theta, scale = _setup(wl)
+    c = _cache(wl)
+    c.build(H.cuda(), K.cuda(), V.cuda(), wl.alpha, wl.window, wl.wmode)
+    zmask = c.new_zmask()
+    th = torch.tensor(theta, dtype=torch.float32, device="cuda")
+    O_gpu, lse_gpu = c.decode(q.cuda(), th, zmask=zmask)
+    torch.cuda.synchronize()
+    assert c.read_status() == 0
+    err, lerr, nz = _compare(wl, c, q, theta, scale, segs, units, O_gpu, lse_gpu, zmask)
+    print(f"e2e {name}: max|dO|={err:.2e} max|dlse|={lerr:.2e} zoomed={nz}")
+
+
+def test_split_count_does_not_change_result():
+    wl = WORKLOADS["c2"].scaled(n=4096, L=1)
+    H, K, V, segs, units, q, theta, scale = _setup(wl)
+    c = _cache(wl)
+    T.upload_oracle_cache(c, segs, units)
+    th = torch.tensor(theta, dtype=torch.float32, device="cuda")
+    ref = None
+    for ns in (1, 2, 3, 7, 0):
+        O_gpu, lse_gpu = c.decode(q.cuda(), th, nsplit=ns)
+        torch.cuda.synchronize()
+        if ref is None:
+            ref = (O_gpu.clone(), lse_gpu.clone())
+        else:
+            assert (O_gpu - ref[0]).abs().max().item() < 2e-5
+            assert (lse_gpu - ref[1]).abs().max().item() < 2e-5
+
+
+def test_route_fetch_attend_equals_fused():
+    """cold bases in pinned host memory: ROUTE, fetch zoomed bases, ATTEND"""
+    P = _lib()
+    wl = WORKLOADS["c3"].scaled(n=8192, L=2)
+    H, K, V, segs, units, q, theta, scale = _setup(wl, quantile=0.9)
+    hot = _cache(wl)
+    T.upload_oracle_cache(hot, segs, units)
+    cold = _cache(wl, home="host")
+    T.upload_oracle_cache(cold, segs, units)
+    th = torch.tensor(theta, dtype=torch.float32, device="cuda")
+    qd = q.cuda()
+    zm_f = hot.new_zmask()
+    O_f, lse_f = hot.decode(qd, th, zmask=zm_f)
+    fetch = P.ColdFetcher(cold, arena_elems=cold.region * wl.L)
+    for step in range(2):                                   # the arena is reused across steps
+        zm = cold.new_zmask()
+        cold.decode(qd, th, phase=P.SEKV_ROUTE, zmask=zm)
+        info = fetch.fetch(zm)
+        torch.cuda.current_stream().wait_event(fetch.done)
+        O_a, lse_a = cold.decode(qd, th, phase=P.SEKV_ATTEND, slot=fetch.slot_dev, arena=fetch.arena)
+        torch.cuda.synchronize()
+        assert cold.read_status() == 0
+        assert torch.equal(zm, zm_f)
+        assert info["spans"] > 0 and info["bytes"] > 0
+        assert (O_a - O_f).abs().max().item() <= 1e-6
+        assert (lse_a - lse_f).abs().max().item() <= 1e-6
+    _compare(wl, hot, q, theta, scale, segs, units, O_f, lse_f, zm_f)
+
+
+def test_attend_without_fetch_reports_cold_span():
+    P = _lib()
+    wl = WORKLOADS["c2"].scaled(n=4096, L=1)
+    H, K, V, segs, units, q, theta, scale = _setup(wl, quantile=0.5)
+    c = _cache(wl, home="host")
+    T.upload_oracle_cache(c, segs, units)
+    slot = torch.full((wl.B, wl.L, c.m_cap), -1, dtype=torch.int64, device="cuda")
+    arena = torch.zeros(1024, dtype=c.dt, device="cuda")
+    th = torch.tensor(theta, dtype=torch.float32, device="cuda")
+    c.decode(q.cuda(), th, phase=P.SEKV_ATTEND, slot=slot, arena=arena)
+    torch.cuda.synchronize()
+    assert c.read_status() == P.sekv.SEKV_ERR_COLD_SPAN
+
+
+def test_fetch_capacity_error_copies_nothing():
+    P = _lib()
+    wl = WORKLOADS["c2"].scaled(n=4096, L=1)
+    H, K, V, segs, units, q, theta, scale = _setup(wl, quantile=0.5)
+    c = _cache(wl, home="host")
+    T.upload_oracle_cache(c, segs, units)
+    th = torch.tensor(theta, dtype=torch.float32, device="cuda")
+    zm = c.new_zmask()
+    c.decode(q.cuda(), th, phase=P.SEKV_ROUTE, zmask=zm)
+    fetch = P.ColdFetcher(c, arena_elems=64)
+    with pytest.raises(P.SekvError) as ei:
+        fetch.fetch(zm)
+    assert ei.value.status == P.sekv.SEKV_ERR_CAPACITY
+    assert (fetch.slot_dev == -1).all()
+
+
+def _dense_unit_check(wl, c, q, K, V, scale, tol):
+    O_gpu, lse_gpu = c.last
+    for b in range(wl.B):
+        for l in range(wl.L):
+            for h in range(wl.Hq):
+                o, ls = dense_attention(T.f64(q[b, l, h]), T.f64(K[b, l, h // wl.G]), T.f64(V[b, l, h // wl.G]), scale)
+                assert np.abs(T.f64(O_gpu[b, l, h]) - o).max() <= tol
+                assert abs(float(lse_gpu[b, l, h]) - ls) <= tol
+
+
+def test_singleton_spans_give_dense_attention():
+    """caller-supplied segmentation: every non-anchor token its own span"""
+    P = _lib()
+    wl = WORKLOADS["c1"].scaled(n=300)
+    H, K, V = T.make_inputs(wl)
+    c = _cache(wl)
+    rng = np.random.default_rng(0)
+    anchor = rng.random(wl.n) < 0.3
+    ap = np.flatnonzero(anchor)
+    sp = np.flatnonzero(~anchor)
+    c.a_count[0] = len(ap)
+    c.m_count[0] = len(sp)
+    c.anchor_pos[0, :len(ap)] = torch.tensor(ap, dtype=torch.int32)
+    c.span_beg[0, :len(sp)] = torch.tensor(sp, dtype=torch.int32)
+    c.span_end[0, :len(sp)] = torch.tensor(sp + 1, dtype=torch.int32)
+    c.build(H.cuda(), K.cuda(), V.cuda(), wl.alpha, wl.window, wl.wmode,
+            steps=P.SEKV_BUILD_LAYOUT | P.SEKV_BUILD_SUMMARY | P.SEKV_BUILD_BASES)
+    q = gen.queries(wl)
+    scale = 1.0 / math.sqrt(wl.d)
+    for theta in (math.inf, -math.inf):         # nothing zoomed / everything zoomed
+        th = torch.full((wl.L, wl.Hq), theta, dtype=torch.float32, device="cuda")
+        c.last = c.decode(q.cuda(), th)
+        torch.cuda.synchronize()
+        assert c.read_status() == 0
+        _dense_unit_check(wl, c, q, K, V, scale, 1e-4)
+
+
+def test_all_zoom_full_rank_gives_dense_attention():
+    wl = WORKLOADS["c1"].scaled(n=700, rank=64)                 # r = d: exact bases
+    H, K, V = T.make_inputs(wl)
+    c = _cache(wl)
+    c.build(H.cuda(), K.cuda(), V.cuda(), wl.alpha, wl.window, wl.wmode, max_sweeps=40)
+    q = gen.queries(wl)
+    th = torch.full((wl.L, wl.Hq), -math.inf, dtype=torch.float32, device="cuda")
+    c.last = c.decode(q.cuda(), th)
+    torch.cuda.synchronize()
+    assert c.read_status() == 0
+    _dense_unit_check(wl, c, q, K, V, 1.0 / math.sqrt(wl.d), 1e-4)
+
+
+def test_empty_cache_rows():
+    """a sequence with no spans and one with no anchors"""
+    P = _lib()
+    wl = WORKLOADS["c1"].scaled(n=64, B=2, window=0)
+    H = torch.ones(2, 64)
+    H[1, 5] = 50.0
+    K = torch.randn(2, 1, wl.Hkv, 64, wl.d)
+    V = torch.randn_like(K)
+    c = _cache(wl)
+    c.build(H.cuda(), K.cuda(), V.cuda(), 1.0, 64, "uniform")   # window covers all: no spans
+    q = gen.queries(wl)
+    th = torch.zeros(wl.L, wl.Hq, device="cuda")
+    O1, l1 = c.decode(q.cuda(), th)
+    torch.cuda.synchronize()
+    assert int(c.m_count[0]) == 0 and int(c.a_count[0]) == 64
+    c.last = (O1, l1)
+    _dense_unit_check(wl, c, q, K, V, 1.0 / math.sqrt(wl.d), 1e-4)
+    c2 = _cache(wl)
+    c2.build(H.cuda(), K.cuda(), V.cuda(), 100.0, 0, "uniform")  # no boundary: one span, no anchors
+    th = torch.full((wl.L, wl.Hq), math.inf, device="cuda")
+    O2, l2 = c2.decode(q.cuda(), th)
+    torch.cuda.synchronize()
+    assert int(c2.a_count[0]) == 0 and int(c2.m_count[0]) == 1
+    kb = T.f64(K[0, 0]).mean(0)
+    vb = T.f64(V[0, 0]).mean(0)
+    for h in range(wl.Hq):
+        np.testing.assert_allclose(T.f64(O2[0, 0, h]), vb, atol=1e-5)   # one entry: softmax weight 1
+        lo = float(T.f64(q[0, 0, h]) @ kb / math.sqrt(wl.d) + math.log(64))
+        assert float(l2[0, 0, h]) == pytest.approx(lo, abs=1e-4)
