@@ -66,15 +66,34 @@ class SpanCache:
         self.kbar = torch.zeros(B, L, Hkv, m_cap, d, dtype=self.dt, device=dev)
         self.vbar = torch.zeros_like(self.kbar)
         self.inv_norm = torch.zeros(B, L, Hkv, m_cap, dtype=torch.float32, device=dev)
-        self.region = S.sekv_basis_region_bound(n, m_cap, Hkv, d, rank)
-        self.home_kind = home
-        if home == "device":
-            self.home = torch.zeros(B, L, self.region, dtype=self.dt, device=dev)
-        else:
-            self.home = torch.zeros(B, L, self.region, dtype=self.dt, pin_memory=True)
         self.status = torch.zeros(1, **i32)
+        self.home_kind = home
+        self.home = None
+        self.region = S.sekv_basis_region_bound(n, m_cap, Hkv, d, rank)
+        if home is not None:
+            self.alloc_home(home)
         self._bws = None
         self._dws = {}
+
+    def alloc_home(self, kind: str, region: Optional[int] = None):
+        """Allocate the basis home: ``kind`` 'device' (hot) or 'host' (pinned, cold).
+        ``region`` (elements per (b, l)) defaults to the worst-case bound; after a
+        SCAN+LAYOUT pass ``exact_region()`` gives the realised size."""
+        if region is not None:
+            self.region = int(region)
+        self.home_kind = kind
+        self.home = None
+        if kind == "device":
+            self.home = torch.zeros(self.B, self.L, self.region, dtype=self.dt, device=self.device)
+        else:
+            self.home = torch.empty(self.B, self.L, self.region, dtype=self.dt, pin_memory=True)
+        return self.home
+
+    def exact_region(self) -> int:
+        """Elements per (b, l) region the realised segmentation needs (after LAYOUT)."""
+        m = self.m_count.to("cpu").long()
+        tot = self.blk_off.to("cpu").gather(1, m.view(-1, 1)).max().item()
+        return max(64, int((tot + 63) // 64 * 64))
 
     # ------------------------------------------------------------------ build
     def build_desc(self, H, K, V, alpha, window, wmode, max_sweeps=15, steps=S.SEKV_BUILD_ALL,

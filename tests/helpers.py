@@ -24,9 +24,10 @@ def f64(t: torch.Tensor) -> np.ndarray:
 
 
 def caps(wl, n=None):
+    """capacities with headroom for every generator recipe (C1 has ~15% boundaries)"""
     n = wl.n if n is None else n
-    a_cap = max(64, int(n / 16) + wl.window + 64)
-    m_cap = max(64, ((int(n / 8) + 64 + 31) // 32) * 32)
+    a_cap = max(64, min(n, n // 4 + wl.window + 64))
+    m_cap = max(64, ((min(n, n // 4 + 64) + 31) // 32) * 32)
     return a_cap, m_cap
 
 

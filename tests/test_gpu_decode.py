@@ -196,7 +196,7 @@ def test_singleton_spans_give_dense_attention():
     P = _lib()
     wl = WORKLOADS["c1"].scaled(n=300)
     H, K, V = T.make_inputs(wl)
-    c = _cache(wl)
+    c = _cache(wl, a_cap=320, m_cap=320)
     rng = np.random.default_rng(0)
     anchor = rng.random(wl.n) < 0.3
     ap = np.flatnonzero(anchor)
@@ -254,9 +254,9 @@ def test_empty_cache_rows():
     O2, l2 = c2.decode(q.cuda(), th)
     torch.cuda.synchronize()
     assert int(c2.a_count[0]) == 0 and int(c2.m_count[0]) == 1
-    kb = T.f64(K[0, 0]).mean(0)
-    vb = T.f64(V[0, 0]).mean(0)
     for h in range(wl.Hq):
+        kb = T.f64(K[0, 0, h // wl.G]).mean(0)
+        vb = T.f64(V[0, 0, h // wl.G]).mean(0)
         np.testing.assert_allclose(T.f64(O2[0, 0, h]), vb, atol=1e-5)   # one entry: softmax weight 1
         lo = float(T.f64(q[0, 0, h]) @ kb / math.sqrt(wl.d) + math.log(64))
         assert float(l2[0, 0, h]) == pytest.approx(lo, abs=1e-4)
