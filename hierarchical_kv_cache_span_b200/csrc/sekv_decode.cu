@@ -23,6 +23,8 @@
 #include "sekv_common.cuh"
 #include "sekv_internal.h"
 
+#include <cmath>
+
 namespace sekv {
 
 constexpr int kNW = 4;          // consumer warps per CTA
@@ -37,10 +39,17 @@ struct DecCfg {
     static constexpr int ROWB = D * ESZ;                    // bytes of one K/V row
     static constexpr int TILE = TR * ROWB;                  // bytes of one K (or V) tile
     static constexpr int STAGE = 2 * TILE + 2 * TR * 4;     // + inv_norm + logS
-    static constexpr int NS0 = (64 * 1024) / STAGE;             // ~64 KB of stages
+    static constexpr int NS0 = (64 * 1024) / STAGE;         // ~64 KB of stages
     static constexpr int NS = NS0 < 2 ? 2 : (NS0 > 6 ? 6 : NS0);   // ring depth
     static constexpr int YPL = kRMax * G / 32;              // y entries per lane
     static constexpr int WSCR = (32 * G) + 2 * kRMax * G;   // per-warp scratch floats
+    // zoom phase: per-warp ring of ZNS slots of ZSLOT bytes, carved from the stage ring
+    static constexpr int ZNS = 3;
+    static constexpr int ZSLOT = 4096;
+    static constexpr int RB = ZSLOT / ROWB;                 // B / D rows per slot
+    static constexpr int RING0 = NS * STAGE;
+    static constexpr int RING = RING0 > kNW * ZNS * ZSLOT ? RING0 : kNW * ZNS * ZSLOT;
+    static constexpr int HDR = 256;                         // mbarriers + counters
 };
 
 struct DecArgs {
@@ -72,24 +81,37 @@ struct DecArgs {
 template <int DT, int D, int G>
 static size_t decode_smem_bytes(int sch_max, int qcap) {
     using C = DecCfg<DT, D, G>;
-    size_t s = 128;                                            // barriers + flags
-    s += (size_t)C::NS * C::STAGE;
+    size_t s = C::HDR;
+    s += (size_t)C::RING;
     s += (size_t)kNW * qcap * 4;                               // zoom queues
     s += (size_t)G * (sch_max / 32) * 4;                       // zoom-mask words
     s += (size_t)kNW * C::WSCR * 4;                            // per-warp scratch
     return round_up(s, 128);
 }
 
+// A zoomed span as the zoom pipeline sees it (warp-uniform values).
+struct ZSpan {
+    const char* blk;     // the span's block for this kv head
+    int S;
+    uint32_t hm;         // query heads of the group that zoom it
+    int len, rS, nB, nAC, TC;
+    int64_t pa;          // elements of the A (and of the C) section
+    bool valid;
+};
+
 template <int DT, int D, int G>
-__global__ void __launch_bounds__((kNW + 1) * 32)
+__global__ void __launch_bounds__((kNW + 1) * 32, 3)
 decode_kernel(const DecArgs a) {
     using C = DecCfg<DT, D, G>;
     constexpr int DPL = C::DPL, R = C::R, TR = C::TR, NS = C::NS;
     extern __shared__ __align__(128) unsigned char sm[];
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm);
-    uint64_t* empty = full + NS;
-    unsigned char* stages = sm + 128;
-    int* zq = reinterpret_cast<int*>(stages + (size_t)NS * C::STAGE);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm);          // [NS]
+    uint64_t* empty = full + 6;                                 // [NS]
+    uint64_t* zbar = full + 12;                                 // [kNW][ZNS]
+    int* qcnt = reinterpret_cast<int*>(sm + 192);               // [kNW]
+    int* zq_next = qcnt + kNW;
+    unsigned char* stages = sm + C::HDR;
+    int* zq = reinterpret_cast<int*>(stages + C::RING);
     uint32_t* zw = reinterpret_cast<uint32_t*>(zq + kNW * a.qcap);
     const int zwords = a.sch_max / 32;
     float* wscr = reinterpret_cast<float*>(zw + G * zwords);
@@ -122,14 +144,17 @@ decode_kernel(const DecArgs a) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kNW);
         }
+        for (int s = 0; s < kNW * C::ZNS; ++s) mbar_init(&zbar[s], 1);
+        *zq_next = 0;
         fence_barrier_init();
     }
     for (int i = tid; i < G * zwords; i += blockDim.x) zw[i] = 0u;
     __syncthreads();
 
     const float sl2 = a.scale * kLog2e;
+    const int rL = lane / G, hL = lane % G;
     // per-warp softmax state (warp-uniform) and per-lane output slice
-    float m_run[G], l_run[G], o[G][DPL];
+    float m_run[G], l_run[G], o[G][DPL], q[G][DPL];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         m_run[h] = -INFINITY;
@@ -137,6 +162,17 @@ decode_kernel(const DecArgs a) {
 #pragma unroll
         for (int i = 0; i < DPL; ++i) o[h][i] = 0.f;
     }
+    {
+        const char* qp = a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB +
+                         lane * DPL * C::ESZ;
+#pragma unroll
+        for (int h = 0; h < G; ++h) Vec<DT, DPL>::load(qp + h * C::ROWB, q[h]);
+    }
+    float m_lane = -INFINITY;                       // == m_run[hL]
+    bool ok = true;
+    float* pb = wscr + (warp < kNW ? warp : 0) * C::WSCR;   // 32*G floats (tile p / token p)
+    float* ub = pb + 32 * G;                                // kRMax*G floats
+    float* yb = ub + kRMax * G;                             // kRMax*G floats
 
     if (warp == kNW) {
         // ------------------------------------------------------------ producer
@@ -170,29 +206,16 @@ decode_kernel(const DecArgs a) {
                 }
                 issued = i + 1;
             }
-            // drain: every issued copy has landed before the CTA may exit
+            // drain: every issued copy has landed before the ring is reused
             for (int i = max(0, issued - NS); i < issued; ++i)
                 if (!mbar_wait(&full[i % NS], (i / NS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
         }
     } else {
         // ------------------------------------------------------------ consumers
-        const int rL = lane / G, hL = lane % G;
-        float q[G][DPL];
-        {
-            const char* qp = a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB +
-                             lane * DPL * C::ESZ;
-#pragma unroll
-            for (int h = 0; h < G; ++h) Vec<DT, DPL>::load(qp + h * C::ROWB, q[h]);
-        }
         const float th = a.theta[(int64_t)l * a.Hq + kvh * G + hL];
-        float m_lane = -INFINITY;                       // == m_run[hL]
         int qn = 0;                                     // zoom-queue length (warp-uniform)
         int* myq = zq + warp * a.qcap;
-        float* pb = wscr + warp * C::WSCR;              // 32*G floats (tile p / token p)
-        float* ub = pb + 32 * G;                        // kRMax*G floats
-        float* yb = ub + kRMax * G;                     // kRMax*G floats
         const int rbase = warp * R;
-        bool ok = true;
 
         for (int i = 0; i < ntiles && ok; ++i) {
             const int s = i % NS;
@@ -295,145 +318,263 @@ decode_kernel(const DecArgs a) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
+        if (lane == 0) qcnt[warp] = ok ? min(qn, a.qcap) : 0;
+    }
+    __syncthreads();    // the stream is done: the stage ring is free, the zoom queues are complete
 
-        // ---------------------------------------------------- zoomed spans
-        if (!route_only && ok) {
-            const int nq = min(qn, a.qcap);
-            for (int e = 0; e < nq; ++e) {
-                const int ent = myq[e];
-                const int S = ent & 0xffffff;
-                const uint32_t hm = (uint32_t)ent >> 24;
-                const int beg = a.span_beg[(int64_t)b * a.m_cap + S];
-                const int len = a.span_end[(int64_t)b * a.m_cap + S] - beg;
-                if (len < 1) {
-                    set_status(a.status, SEKV_ERR_INVALID_ARG);
-                    continue;
-                }
-                const int rS = block_rank(len, D, a.rank);
-                const int64_t pa = block_ac_elems(len, rS);
-                const int64_t be = block_elems(len, D, a.rank);
-                int64_t off;
+    // ---------------------------------------------------- zoomed spans
+    // Each consumer warp pulls spans from the CTA's queue and streams the span's
+    // block through its own ring of ZNS shared-memory slots (bulk copies, one
+    // mbarrier per slot): B rows -> u = B q; A/C token chunks -> scores A u, online
+    // softmax, y = C^T p; D rows -> o += beta * y^T D.
+    if (warp < kNW && !route_only && ok) {
+        const int nq_total = qcnt[0] + qcnt[1] + qcnt[2] + qcnt[3];
+        unsigned char* zring = stages + (size_t)warp * C::ZNS * C::ZSLOT;
+        uint64_t* zb = zbar + warp * C::ZNS;
+
+        auto grab = [&]() -> ZSpan {
+            ZSpan sp;
+            sp.valid = false;
+            sp.blk = nullptr;
+            sp.S = 0; sp.hm = 0u; sp.len = 0; sp.rS = 1; sp.nB = 0; sp.nAC = 0; sp.TC = 8; sp.pa = 0;
+            int e = 0;
+            if (lane == 0) e = atomicAdd(zq_next, 1);
+            e = __shfl_sync(0xffffffffu, e, 0);
+            if (e >= nq_total) return sp;
+            int w = 0;
+            while (w < kNW - 1 && e >= qcnt[w]) { e -= qcnt[w]; ++w; }
+            const int ent = zq[w * a.qcap + e];
+            sp.S = ent & 0xffffff;
+            sp.hm = (uint32_t)ent >> 24;
+            const int beg = a.span_beg[(int64_t)b * a.m_cap + sp.S];
+            sp.len = a.span_end[(int64_t)b * a.m_cap + sp.S] - beg;
+            if (sp.len < 1) {
+                set_status(a.status, SEKV_ERR_INVALID_ARG);
+                sp.len = 0;
+            }
+            sp.rS = sp.len > 0 ? block_rank(sp.len, D, a.rank) : 1;
+            sp.pa = block_ac_elems(sp.len, sp.rS);
+            const int64_t be = block_elems(sp.len > 0 ? sp.len : 1, D, a.rank);
+            int64_t off = -1;
+            if (sp.len > 0) {
                 if (a.slot) {
-                    off = a.slot[((int64_t)b * a.L + l) * a.m_cap + S];
-                    if (off < 0) {
-                        set_status(a.status, SEKV_ERR_COLD_SPAN);
-                        continue;
-                    }
+                    off = a.slot[((int64_t)b * a.L + l) * a.m_cap + sp.S];
+                    if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
                 } else {
-                    off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S];
+                    off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + sp.S];
                 }
-                const char* blk = a.arena + (off + (int64_t)kvh * be) * C::ESZ;
-                const char* Ap = blk;
-                const char* Cp = blk + pa * C::ESZ;
-                const char* Bp = blk + 2 * pa * C::ESZ;
-                const char* Dp = Bp + (int64_t)rS * D * C::ESZ;
+            }
+            sp.blk = off >= 0 ? a.arena + (off + (int64_t)kvh * be) * C::ESZ : nullptr;
+            int tc = (C::ZSLOT / 2) / (sp.rS * C::ESZ);
+            tc = tc > 64 ? 64 : tc;
+            sp.TC = (tc & ~7) < 8 ? 8 : (tc & ~7);
+            sp.nB = (sp.rS + C::RB - 1) / C::RB;
+            sp.nAC = (sp.len + sp.TC - 1) / sp.TC;
+            sp.valid = true;
+            return sp;
+        };
+        auto nslots = [](const ZSpan& sp) { return sp.blk ? 2 * sp.nB + sp.nAC : 0; };
 
-                // (1) u[i][h] = B_i . q_h
-                for (int i0 = 0; i0 < rS; i0 += R) {
-                    float part[32];
+        ZSpan cur = grab(), nxt;
+        nxt.valid = false;
+        nxt.blk = nullptr;
+        bool i_next = false;       // the issue cursor is in nxt
+        int i_k = 0;               // slots issued of the span under the issue cursor
+        uint32_t nis = 0, ncons = 0;
+        bool zok = true;
+
+        auto issue = [&]() {
+            // order this warp's earlier shared-memory reads of a slot before the
+            // bulk copy that refills it
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            while (nis - ncons < (uint32_t)C::ZNS) {
+                if (!i_next && i_k >= nslots(cur)) {
+                    if (!cur.valid) break;
+                    nxt = grab();
+                    i_next = true;
+                    i_k = 0;
+                }
+                // fields of the span under the issue cursor, selected by value
+                const bool sv = i_next ? nxt.valid : cur.valid;
+                const char* sblk = i_next ? nxt.blk : cur.blk;
+                const int snB = i_next ? nxt.nB : cur.nB, snAC = i_next ? nxt.nAC : cur.nAC;
+                const int srS = i_next ? nxt.rS : cur.rS, slen = i_next ? nxt.len : cur.len;
+                const int sTC = i_next ? nxt.TC : cur.TC;
+                const int64_t spa = i_next ? nxt.pa : cur.pa;
+                if (!sv || !sblk || i_k >= 2 * snB + snAC) break;
+                const int slot = nis % C::ZNS;
+                unsigned char* dst = zring + slot * C::ZSLOT;
+                if (lane == 0) {
+                    const int k = i_k;
+                    if (k < snB || k >= snB + snAC) {
+                        const bool isD = k >= snB;
+                        const int j = isD ? k - snB - snAC : k;
+                        const int r0 = j * C::RB;
+                        const uint32_t bytes = (uint32_t)min(C::RB, srS - r0) * C::ROWB;
+                        const char* src = sblk + (2 * spa + (isD ? (int64_t)srS * D : 0) + (int64_t)r0 * D) * C::ESZ;
+                        mbar_arrive_expect_tx(&zb[slot], bytes);
+                        bulk_g2s(dst, src, bytes, &zb[slot]);
+                    } else {
+                        const int t0 = (k - snB) * sTC;
+                        const int nt = min(sTC, slen - t0);
+                        const uint32_t bytes = (uint32_t)round_up((int64_t)nt * srS * C::ESZ, 16);
+                        const int64_t off = (int64_t)t0 * srS * C::ESZ;
+                        mbar_arrive_expect_tx(&zb[slot], 2 * bytes);
+                        bulk_g2s(dst, sblk + off, bytes, &zb[slot]);
+                        bulk_g2s(dst + C::ZSLOT / 2, sblk + spa * C::ESZ + off, bytes, &zb[slot]);
+                    }
+                }
+                ++i_k;
+                ++nis;
+            }
+        };
+
+        while (cur.valid && zok) {
+            const int total = nslots(cur);
+            float msp[G], lsp[G];
 #pragma unroll
-                    for (int r = 0; r < R; ++r) {
-                        float kk[DPL];
-                        if (i0 + r < rS) {
-                            Vec<DT, DPL>::load(Bp + (int64_t)(i0 + r) * C::ROWB + lane * DPL * C::ESZ, kk);
-                        } else {
+            for (int h = 0; h < G; ++h) { msp[h] = -INFINITY; lsp[h] = 0.f; }
+            float y[C::YPL];
 #pragma unroll
-                            for (int k = 0; k < DPL; ++k) kk[k] = 0.f;
+            for (int j = 0; j < C::YPL; ++j) y[j] = 0.f;
+            float betaL = 0.f;
+            for (int k = 0; k < total; ++k) {
+                issue();
+                const int slot = ncons % C::ZNS;
+                if (!mbar_wait(&zb[slot], (ncons / C::ZNS) & 1)) {
+                    set_status(a.status, SEKV_ERR_TIMEOUT);
+                    zok = false;
+                    break;
+                }
+                const unsigned char* zs = zring + slot * C::ZSLOT;
+                if (k < cur.nB) {
+                    // (1) u[i][h] = B_i . q_h for the slot's rows
+                    const int r0 = k * C::RB;
+                    const int rows = min(C::RB, cur.rS - r0);
+                    for (int i0 = 0; i0 < rows; i0 += R) {
+                        float part[32];
+#pragma unroll
+                        for (int r = 0; r < R; ++r) {
+                            float kk[DPL];
+                            if (i0 + r < rows) {
+                                Vec<DT, DPL>::load(zs + (i0 + r) * C::ROWB + lane * DPL * C::ESZ, kk);
+                            } else {
+#pragma unroll
+                                for (int t = 0; t < DPL; ++t) kk[t] = 0.f;
+                            }
+#pragma unroll
+                            for (int h = 0; h < G; ++h) {
+                                float acc = 0.f;
+#pragma unroll
+                                for (int t = 0; t < DPL; ++t) acc = fmaf(kk[t], q[h][t], acc);
+                                part[r * G + h] = acc;
+                            }
                         }
+                        const float u = transpose_reduce32(part, lane);
+                        if (i0 + rL < rows) ub[(r0 + i0 + rL) * G + hL] = u;
+                    }
+                } else if (k < cur.nB + cur.nAC) {
+                    // (2) token scores, span-local online softmax, y = C^T p
+                    __syncwarp();
+                    const int t0 = (k - cur.nB) * cur.TC;
+                    const int nt = min(cur.TC, cur.len - t0);
+                    const unsigned char* As = zs;
+                    const unsigned char* Cs = zs + C::ZSLOT / 2;
+                    for (int c0 = 0; c0 < nt; c0 += 32) {
+                        const int t = c0 + lane;
+                        float xs[G];
+#pragma unroll
+                        for (int h = 0; h < G; ++h) xs[h] = 0.f;
+                        if (t < nt) {
+                            for (int i = 0; i < cur.rS; ++i) {
+                                const float av = load1<DT>(As, (int64_t)t * cur.rS + i);
+#pragma unroll
+                                for (int h = 0; h < G; ++h) xs[h] = fmaf(av, ub[i * G + h], xs[h]);
+                            }
+                        }
+                        float alL = 1.f;
 #pragma unroll
                         for (int h = 0; h < G; ++h) {
-                            float acc = 0.f;
-#pragma unroll
-                            for (int k = 0; k < DPL; ++k) acc = fmaf(kk[k], q[h][k], acc);
-                            part[r * G + h] = acc;
+                            const float lg = (t < nt && ((cur.hm >> h) & 1u)) ? xs[h] * sl2 : -INFINITY;
+                            const float cm = warp_max(lg);
+                            const float mnew = fmaxf(msp[h], cm);
+                            const float al = (mnew == -INFINITY) ? 1.f : exp2f(msp[h] - mnew);
+                            const float p = (lg == -INFINITY) ? 0.f : exp2f(lg - mnew);
+                            lsp[h] = fmaf(lsp[h], al, warp_sum(p));
+                            msp[h] = mnew;
+                            pb[lane * G + h] = p;
+                            if (h == hL) alL = al;
                         }
-                    }
-                    const float u = transpose_reduce32(part, lane);
-                    if (i0 + rL < rS) ub[(i0 + rL) * G + hL] = u;
-                }
-                __syncwarp();
-
-                // (2) token scores s_t = A_t . u (scaled), span-local online softmax, y = C^T p
-                float msp[G], lsp[G];
+                        __syncwarp();
+                        const int tn = min(32, nt - c0);
 #pragma unroll
-                for (int h = 0; h < G; ++h) { msp[h] = -INFINITY; lsp[h] = 0.f; }
-                float y[C::YPL];
-#pragma unroll
-                for (int j = 0; j < C::YPL; ++j) y[j] = 0.f;
-                for (int t0 = 0; t0 < len; t0 += 32) {
-                    const int t = t0 + lane;
-                    float xs[G];
-#pragma unroll
-                    for (int h = 0; h < G; ++h) xs[h] = 0.f;
-                    if (t < len) {
-                        for (int i = 0; i < rS; ++i) {
-                            const float av = load1<DT>(Ap, (int64_t)t * rS + i);
-#pragma unroll
-                            for (int h = 0; h < G; ++h) xs[h] = fmaf(av, ub[i * G + h], xs[h]);
+                        for (int j = 0; j < C::YPL; ++j) {
+                            const int i = (lane + 32 * j) / G;
+                            if (i < cur.rS) {
+                                float acc = y[j] * alL;
+                                for (int tt = 0; tt < tn; ++tt)
+                                    acc = fmaf(pb[tt * G + hL], load1<DT>(Cs, (int64_t)(c0 + tt) * cur.rS + i), acc);
+                                y[j] = acc;
+                            }
                         }
+                        __syncwarp();
                     }
-                    float alL = 1.f;
+                } else {
+                    if (k == cur.nB + cur.nAC) {
+                        // (3) merge the span's softmax state into the warp's running state
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float lg = (t < len && ((hm >> h) & 1u)) ? xs[h] * sl2 : -INFINITY;
-                        const float cm = warp_max(lg);
-                        const float mnew = fmaxf(msp[h], cm);
-                        const float al = (mnew == -INFINITY) ? 1.f : exp2f(msp[h] - mnew);
-                        const float p = (lg == -INFINITY) ? 0.f : exp2f(lg - mnew);
-                        lsp[h] = fmaf(lsp[h], al, warp_sum(p));
-                        msp[h] = mnew;
-                        pb[lane * G + h] = p;
-                        if (h == hL) alL = al;
-                    }
-                    __syncwarp();
-                    const int tn = min(32, len - t0);
+                        for (int h = 0; h < G; ++h) {
+                            float al = 1.f, be2 = 0.f;
+                            if ((cur.hm >> h) & 1u) {
+                                const float mnew = fmaxf(m_run[h], msp[h]);
+                                al = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mnew);
+                                be2 = exp2f(msp[h] - mnew);
+                                l_run[h] = l_run[h] * al + lsp[h] * be2;
+                                m_run[h] = mnew;
+                            }
 #pragma unroll
-                    for (int j = 0; j < C::YPL; ++j) {
-                        const int i = (lane + 32 * j) / G;
-                        if (i < rS) {
-                            float acc = y[j] * alL;
-                            for (int tt = 0; tt < tn; ++tt)
-                                acc = fmaf(pb[tt * G + hL], load1<DT>(Cp, (int64_t)(t0 + tt) * rS + i), acc);
-                            y[j] = acc;
+                            for (int t = 0; t < DPL; ++t) o[h][t] *= al;
+                            if (h == hL) { betaL = be2; m_lane = m_run[h]; }
                         }
+#pragma unroll
+                        for (int j = 0; j < C::YPL; ++j) {
+                            const int i = (lane + 32 * j) / G;
+                            if (i < cur.rS) yb[i * G + hL] = y[j] * betaL;
+                        }
+                        __syncwarp();
                     }
-                    __syncwarp();
-                }
-
-                // (3) merge the span into the running state: o += beta * y^T D
-                float betaL = 0.f;
+                    // o += sum_i (beta y_i) D_i over the slot's rows
+                    const int r0 = (k - cur.nB - cur.nAC) * C::RB;
+                    const int rows = min(C::RB, cur.rS - r0);
+                    for (int r = 0; r < rows; ++r) {
+                        float dv[DPL];
+                        Vec<DT, DPL>::load(zs + r * C::ROWB + lane * DPL * C::ESZ, dv);
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    float al = 1.f, be2 = 0.f;
-                    if ((hm >> h) & 1u) {
-                        const float mnew = fmaxf(m_run[h], msp[h]);
-                        al = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mnew);
-                        be2 = exp2f(msp[h] - mnew);
-                        l_run[h] = l_run[h] * al + lsp[h] * be2;
-                        m_run[h] = mnew;
-                    }
+                        for (int h = 0; h < G; ++h) {
+                            const float yv = yb[(r0 + r) * G + h];
 #pragma unroll
-                    for (int k = 0; k < DPL; ++k) o[h][k] *= al;
-                    if (h == hL) { betaL = be2; m_lane = m_run[h]; }
-                }
-#pragma unroll
-                for (int j = 0; j < C::YPL; ++j) {
-                    const int i = (lane + 32 * j) / G;
-                    if (i < rS) yb[i * G + hL] = y[j] * betaL;
-                }
-                __syncwarp();
-                for (int i = 0; i < rS; ++i) {
-                    float dv[DPL];
-                    Vec<DT, DPL>::load(Dp + (int64_t)i * C::ROWB + lane * DPL * C::ESZ, dv);
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float yv = yb[i * G + h];
-#pragma unroll
-                        for (int k = 0; k < DPL; ++k) o[h][k] = fmaf(yv, dv[k], o[h][k]);
+                            for (int t = 0; t < DPL; ++t) o[h][t] = fmaf(yv, dv[t], o[h][t]);
+                        }
                     }
                 }
                 __syncwarp();
+                ++ncons;
             }
+            if (!zok) break;
+            // advance to the next span (the issue cursor may already be in it)
+            if (i_next) {
+                cur = nxt;
+                i_next = false;
+                nxt.valid = false;
+            } else {
+                cur = grab();
+                i_k = 0;
+            }
+        }
+        // drain anything still in flight (only after an error)
+        while (ncons < nis) {
+            if (!mbar_wait(&zb[ncons % C::ZNS], (ncons / C::ZNS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
+            ++ncons;
         }
     }
     __syncthreads();
@@ -539,14 +680,26 @@ DecodePlan plan_decode(const sekv_decode_desc& d) {
     const int Lr = d.l1 - d.l0;
     const int64_t units = (int64_t)d.B * Lr * d.Hkv;
     int ns = d.nsplit;
-    if (ns <= 0) {
-        // about two waves of ~3 resident CTAs per SM
-        const int64_t target = 2LL * 3 * num_sms();
-        ns = (int)((target + units - 1) / units);
-        const int by_rows = (int)((d.a_cap + d.m_cap) / 256);     // keep >= ~256 rows per split
-        ns = ns < by_rows ? ns : by_rows;
-    }
     const int max_ns = d.m_cap / 32 > 0 ? d.m_cap / 32 : 1;
+    if (ns <= 0) {
+        // Fill whole waves of resident CTAs (3 per SM for the bf16 / d=128 / G=4
+        // variant): the smallest split count with >= 1.5 waves and >= 85% of the
+        // last wave busy; otherwise the best such ratio. Splits keep >= ~128 rows.
+        const double slots = 3.0 * num_sms();
+        int lim = (int)((d.a_cap + d.m_cap) / 128);
+        lim = lim < 1 ? 1 : (lim > max_ns ? max_ns : lim);
+        if (lim > 64) lim = 64;
+        int best = 1;
+        double best_score = -1.0;
+        for (int c = 1; c <= lim; ++c) {
+            const double waves = (double)units * c / slots;
+            const double eff = waves / std::ceil(waves);
+            if (waves >= 1.5 && eff >= 0.85) { best = c; break; }
+            const double score = eff * (waves < 2.0 ? waves / 2.0 : 1.0);
+            if (score > best_score + 1e-9) { best_score = score; best = c; }
+        }
+        ns = best;
+    }
     if (ns > max_ns) ns = max_ns;
     if (ns < 1) ns = 1;
     p.nsplit = ns;
