@@ -8,22 +8,30 @@
 // ones reconstructed from their bases), non-zoomed spans with (kbar_S, vbar_S) and
 // a +log|S| logit correction, all in ONE softmax (Fig. 2's "merge").
 //
-// Work decomposition: one CTA per (split, kv head, sequence x layer). A producer
-// warp streams 32-row tiles (anchor K/V rows, then span kbar/vbar rows with
-// inv_norm and log|S|) into a ring of shared-memory stages with 1-D bulk copies
-// (cp.async.bulk, mbarrier completion, no multicast). Four consumer warps each
-// take R = 32/G rows of a tile for all G query heads of the kv head (GQA: one K/V
-// read serves G heads); each lane owns D/32 dimensions. 32 partial dot products
-// per lane are finished with one transpose-reduce (31 shuffles), after which
-// lane L holds the logit of (row L/G, head L%G). The routing logit reuses that
-// same q.kbar value. Zoomed spans go to a per-warp queue and are attended after
-// the stream, without materialising K_S: u = B_S q, scores A_S u, y = C_S^T p,
-// contribution y^T D_S. Softmax state is kept in the log2 domain; splits are
-// merged by log-sum-exp in a second small kernel.
-#include "sekv_common.cuh"
-#include "sekv_internal.h"
+// Work decomposition: one CTA per (split, kv head, sequence x layer); a producer
+// warp and four consumer warps. Phase 1 streams the split's anchor rows (K, V)
+// and then its span rows (kbar, vbar, 1/||kbar||, log|S|) through a ring of
+// shared-memory stages:
+//   bf16: 2-D TMA tensor copies with 128-byte swizzle; each consumer warp takes
+//         16 rows of a 64-row tile and runs q.K^T and p.V on the tensor cores
+//         (mma.sync m16n8k16, the G query heads of the kv head padded to M = 16:
+//         GQA, one K/V read serves all G heads). The q.kbar accumulator of a span
+//         row is both its routing logit and its coarse attention logit.
+//   fp32: 1-D bulk copies and CUDA-core dot products (each lane owns d/32 dims,
+//         a 32-way transpose-reduce finishes the dots).
+// Spans zoomed by any head of the group are queued. Phase 2 attends them without
+// materialising K_S: each consumer warp pulls spans from the queue and streams
+// B_S rows, A_S/C_S token chunks and D_S rows through its own 3-slot ring:
+// u = B_S q, scores A_S u, y = C_S^T p, contribution y^T D_S. Softmax state is
+// kept in the log2 domain; the CTA merges its warps' states, a second small
+// kernel merges the splits by log-sum-exp.
+#include <cuda.h>
 
 #include <cmath>
+#include <cstring>
+
+#include "sekv_common.cuh"
+#include "sekv_internal.h"
 
 namespace sekv {
 
@@ -32,24 +40,35 @@ constexpr int kRMax = 64;       // largest basis rank the decode accepts
 
 template <int DT, int D, int G>
 struct DecCfg {
-    static constexpr int DPL = D / 32;                      // dims per lane
-    static constexpr int R = 32 / G;                        // rows per warp per tile
-    static constexpr int TR = kNW * R;                      // rows per tile
+    static constexpr bool MMA = DT == SEKV_BF16;
+    static constexpr int DPL = D / 32;                      // dims per lane (CUDA-core layout)
     static constexpr int ESZ = Elt<DT>::bytes;
     static constexpr int ROWB = D * ESZ;                    // bytes of one K/V row
+    // rows per warp per tile: 16 on the tensor-core path, 32/G on the CUDA-core path
+    static constexpr int R = MMA ? 16 : 32 / G;
+    static constexpr int TR = kNW * R;                      // rows per tile
+    static constexpr int NBOX = D / 64;                     // 128-byte-wide TMA boxes per row
     static constexpr int TILE = TR * ROWB;                  // bytes of one K (or V) tile
-    static constexpr int STAGE = 2 * TILE + 2 * TR * 4;     // + inv_norm + logS
-    static constexpr int NS0 = (64 * 1024) / STAGE;         // ~64 KB of stages
+    static constexpr int META = 2 * TR * 4;                 // inv_norm + logS of a span tile
+    static constexpr int STAGE0 = 2 * TILE + META;
+    static constexpr int STAGE = MMA ? (STAGE0 + 1023) / 1024 * 1024 : STAGE0;
+    static constexpr int NS0 = (MMA ? 68 * 1024 : 64 * 1024) / STAGE;     // 2 CTAs / SM on the bf16 path
     static constexpr int NS = NS0 < 2 ? 2 : (NS0 > 6 ? 6 : NS0);   // ring depth
-    static constexpr int YPL = kRMax * G / 32;              // y entries per lane
+    static constexpr int YPL = kRMax * G / 32;              // y entries per lane (zoom)
     static constexpr int WSCR = (32 * G) + 2 * kRMax * G;   // per-warp scratch floats
     // zoom phase: per-warp ring of ZNS slots of ZSLOT bytes, carved from the stage ring
     static constexpr int ZNS = 3;
     static constexpr int ZSLOT = 4096;
     static constexpr int RB = ZSLOT / ROWB;                 // B / D rows per slot
+    static constexpr int ZBYTES = kNW * ZNS * ZSLOT;
+    // partial softmax states merged at the end: per warp one for the stream and,
+    // on the tensor-core path, one for its zoomed spans
+    static constexpr int NSTATE = MMA ? 2 * kNW : kNW;
+    static constexpr int SBYTES = NSTATE * (G * D + 2 * G) * 4;
     static constexpr int RING0 = NS * STAGE;
-    static constexpr int RING = RING0 > kNW * ZNS * ZSLOT ? RING0 : kNW * ZNS * ZSLOT;
-    static constexpr int HDR = 256;                         // mbarriers + counters
+    static constexpr int RING1 = ZBYTES + SBYTES;
+    static constexpr int RING = RING0 > RING1 ? RING0 : RING1;
+    static constexpr int HDR = 1024;                        // mbarriers + counters (keeps stages 1 KB aligned)
 };
 
 struct DecArgs {
@@ -78,6 +97,12 @@ struct DecArgs {
     int L, l0, Lr, Hq, Hkv, a_cap, m_cap, rank, phase, nsplit, sch_max, qcap, mw;
 };
 
+// TMA descriptors of the anchor and summary stores (bf16 path), viewed as 2-D
+// [rows][d] tensors with 64 x 64 boxes and 128-byte swizzle.
+struct DecMaps {
+    CUtensorMap Ka, Va, kbar, vbar;
+};
+
 template <int DT, int D, int G>
 static size_t decode_smem_bytes(int sch_max, int qcap) {
     using C = DecCfg<DT, D, G>;
@@ -86,7 +111,7 @@ static size_t decode_smem_bytes(int sch_max, int qcap) {
     s += (size_t)kNW * qcap * 4;                               // zoom queues
     s += (size_t)G * (sch_max / 32) * 4;                       // zoom-mask words
     s += (size_t)kNW * C::WSCR * 4;                            // per-warp scratch
-    return round_up(s, 128);
+    return round_up(s, 128) + 1024;                            // + alignment slack
 }
 
 // A zoomed span as the zoom pipeline sees it (warp-uniform values).
@@ -99,22 +124,339 @@ struct ZSpan {
     bool valid;
 };
 
+// shared-memory carve-up common to both paths
+struct DecSmem {
+    uint64_t* full;      // [NS]
+    uint64_t* empty;     // [NS]
+    uint64_t* zbar;      // [kNW][ZNS]
+    int* qcnt;           // [kNW]
+    int* zq_next;
+    unsigned char* stages;
+    int* zq;             // [kNW][qcap]
+    uint32_t* zw;        // [G][zwords]
+    float* wscr;         // [kNW][WSCR]
+    float* st_m;         // [NSTATE][G]   (in the ring, after the zoom slots)
+    float* st_l;         // [NSTATE][G]
+    float* st_o;         // [NSTATE][G][D]
+};
+
+template <class C, int G, int D>
+SEKV_DEV DecSmem carve_smem(unsigned char* base, int qcap, int zwords) {
+    DecSmem s;
+    s.full = reinterpret_cast<uint64_t*>(base);
+    s.empty = s.full + 8;
+    s.zbar = s.full + 16;
+    s.qcnt = reinterpret_cast<int*>(base + 256);
+    s.zq_next = s.qcnt + kNW;
+    s.stages = base + C::HDR;
+    s.zq = reinterpret_cast<int*>(s.stages + C::RING);
+    s.zw = reinterpret_cast<uint32_t*>(s.zq + kNW * qcap);
+    s.wscr = reinterpret_cast<float*>(s.zw + G * zwords);
+    s.st_m = reinterpret_cast<float*>(s.stages + C::ZBYTES);
+    s.st_l = s.st_m + C::NSTATE * G;
+    s.st_o = s.st_l + C::NSTATE * G;
+    return s;
+}
+
+// ---------------------------------------------------------------------------
+// Phase 2: attend the queued zoomed spans (one warp per span at a time).
+// (m_run, l_run, o, m_lane) is the softmax state the spans are merged into.
+// ---------------------------------------------------------------------------
 template <int DT, int D, int G>
-__global__ void __launch_bounds__((kNW + 1) * 32, 3)
-decode_kernel(const DecArgs a) {
+SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane, int b, int l, int kvh,
+                         float (&m_run)[G], float (&l_run)[G], float (&o)[G][D / 32], float& m_lane) {
+    using C = DecCfg<DT, D, G>;
+    constexpr int DPL = C::DPL;
+    constexpr int R = 32 / G;                      // rows per transpose-reduce batch
+    const int rL = lane / G, hL = lane % G;
+    const float sl2 = a.scale * kLog2e;
+    float q[G][DPL];
+    {
+        const char* qp = a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB + lane * DPL * C::ESZ;
+#pragma unroll
+        for (int h = 0; h < G; ++h) Vec<DT, DPL>::load(qp + h * C::ROWB, q[h]);
+    }
+    const int nq_total = sm.qcnt[0] + sm.qcnt[1] + sm.qcnt[2] + sm.qcnt[3];
+    unsigned char* zring = sm.stages + (size_t)warp * C::ZNS * C::ZSLOT;
+    uint64_t* zb = sm.zbar + warp * C::ZNS;
+    float* pb = sm.wscr + warp * C::WSCR;          // 32*G floats (token p)
+    float* ub = pb + 32 * G;                       // kRMax*G floats
+    float* yb = ub + kRMax * G;                    // kRMax*G floats
+
+    auto grab = [&]() -> ZSpan {
+        ZSpan sp;
+        sp.valid = false;
+        sp.blk = nullptr;
+        sp.S = 0; sp.hm = 0u; sp.len = 0; sp.rS = 1; sp.nB = 0; sp.nAC = 0; sp.TC = 8; sp.pa = 0;
+        int e = 0;
+        if (lane == 0) e = atomicAdd(sm.zq_next, 1);
+        e = __shfl_sync(0xffffffffu, e, 0);
+        if (e >= nq_total) return sp;
+        int w = 0;
+        while (w < kNW - 1 && e >= sm.qcnt[w]) { e -= sm.qcnt[w]; ++w; }
+        const int ent = sm.zq[w * a.qcap + e];
+        sp.S = ent & 0xffffff;
+        sp.hm = (uint32_t)ent >> 24;
+        const int beg = a.span_beg[(int64_t)b * a.m_cap + sp.S];
+        sp.len = a.span_end[(int64_t)b * a.m_cap + sp.S] - beg;
+        if (sp.len < 1) {
+            set_status(a.status, SEKV_ERR_INVALID_ARG);
+            sp.len = 0;
+        }
+        sp.rS = sp.len > 0 ? block_rank(sp.len, D, a.rank) : 1;
+        sp.pa = block_ac_elems(sp.len, sp.rS);
+        const int64_t be = block_elems(sp.len > 0 ? sp.len : 1, D, a.rank);
+        int64_t off = -1;
+        if (sp.len > 0) {
+            if (a.slot) {
+                off = a.slot[((int64_t)b * a.L + l) * a.m_cap + sp.S];
+                if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
+            } else {
+                off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + sp.S];
+            }
+        }
+        sp.blk = off >= 0 ? a.arena + (off + (int64_t)kvh * be) * C::ESZ : nullptr;
+        int tc = (C::ZSLOT / 2) / (sp.rS * C::ESZ);
+        tc = tc > 64 ? 64 : tc;
+        sp.TC = (tc & ~7) < 8 ? 8 : (tc & ~7);
+        sp.nB = (sp.rS + C::RB - 1) / C::RB;
+        sp.nAC = (sp.len + sp.TC - 1) / sp.TC;
+        sp.valid = true;
+        return sp;
+    };
+    auto nslots = [](const ZSpan& sp) { return sp.blk ? 2 * sp.nB + sp.nAC : 0; };
+
+    ZSpan cur = grab(), nxt;
+    nxt.valid = false;
+    nxt.blk = nullptr;
+    nxt.nB = nxt.nAC = 0;
+    bool i_next = false;       // the issue cursor is in nxt
+    int i_k = 0;               // slots issued of the span under the issue cursor
+    uint32_t nis = 0, ncons = 0;
+    bool zok = true;
+
+    auto issue = [&]() {
+        // order this warp's earlier shared-memory reads of a slot before the bulk
+        // copy that refills it
+        fence_proxy_async();
+        while (nis - ncons < (uint32_t)C::ZNS) {
+            if (!i_next && i_k >= nslots(cur)) {
+                if (!cur.valid) break;
+                nxt = grab();
+                i_next = true;
+                i_k = 0;
+            }
+            // fields of the span under the issue cursor, selected by value
+            const bool sv = i_next ? nxt.valid : cur.valid;
+            const char* sblk = i_next ? nxt.blk : cur.blk;
+            const int snB = i_next ? nxt.nB : cur.nB, snAC = i_next ? nxt.nAC : cur.nAC;
+            const int srS = i_next ? nxt.rS : cur.rS, slen = i_next ? nxt.len : cur.len;
+            const int sTC = i_next ? nxt.TC : cur.TC;
+            const int64_t spa = i_next ? nxt.pa : cur.pa;
+            if (!sv || !sblk || i_k >= 2 * snB + snAC) break;
+            const int slot = nis % C::ZNS;
+            unsigned char* dst = zring + slot * C::ZSLOT;
+            if (lane == 0) {
+                const int k = i_k;
+                if (k < snB || k >= snB + snAC) {
+                    const bool isD = k >= snB;
+                    const int j = isD ? k - snB - snAC : k;
+                    const int r0 = j * C::RB;
+                    const uint32_t bytes = (uint32_t)min(C::RB, srS - r0) * C::ROWB;
+                    const char* src = sblk + (2 * spa + (isD ? (int64_t)srS * D : 0) + (int64_t)r0 * D) * C::ESZ;
+                    mbar_arrive_expect_tx(&zb[slot], bytes);
+                    bulk_g2s(dst, src, bytes, &zb[slot]);
+                } else {
+                    const int t0 = (k - snB) * sTC;
+                    const int nt = min(sTC, slen - t0);
+                    const uint32_t bytes = (uint32_t)round_up((int64_t)nt * srS * C::ESZ, 16);
+                    const int64_t off = (int64_t)t0 * srS * C::ESZ;
+                    mbar_arrive_expect_tx(&zb[slot], 2 * bytes);
+                    bulk_g2s(dst, sblk + off, bytes, &zb[slot]);
+                    bulk_g2s(dst + C::ZSLOT / 2, sblk + spa * C::ESZ + off, bytes, &zb[slot]);
+                }
+            }
+            ++i_k;
+            ++nis;
+        }
+    };
+
+    while (cur.valid && zok) {
+        const int total = nslots(cur);
+        float msp[G], lsp[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) { msp[h] = -INFINITY; lsp[h] = 0.f; }
+        float y[C::YPL];
+#pragma unroll
+        for (int j = 0; j < C::YPL; ++j) y[j] = 0.f;
+        float betaL = 0.f;
+        for (int k = 0; k < total; ++k) {
+            issue();
+            const int slot = ncons % C::ZNS;
+            if (!mbar_wait(&zb[slot], (ncons / C::ZNS) & 1)) {
+                set_status(a.status, SEKV_ERR_TIMEOUT);
+                zok = false;
+                break;
+            }
+            const unsigned char* zs = zring + slot * C::ZSLOT;
+            if (k < cur.nB) {
+                // (1) u[i][h] = B_i . q_h for the slot's rows
+                const int r0 = k * C::RB;
+                const int rows = min(C::RB, cur.rS - r0);
+                for (int i0 = 0; i0 < rows; i0 += R) {
+                    float part[32];
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        float kk[DPL];
+                        if (i0 + r < rows) {
+                            Vec<DT, DPL>::load(zs + (i0 + r) * C::ROWB + lane * DPL * C::ESZ, kk);
+                        } else {
+#pragma unroll
+                            for (int t = 0; t < DPL; ++t) kk[t] = 0.f;
+                        }
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            float acc = 0.f;
+#pragma unroll
+                            for (int t = 0; t < DPL; ++t) acc = fmaf(kk[t], q[h][t], acc);
+                            part[r * G + h] = acc;
+                        }
+                    }
+                    const float u = transpose_reduce32(part, lane);
+                    if (i0 + rL < rows) ub[(r0 + i0 + rL) * G + hL] = u;
+                }
+            } else if (k < cur.nB + cur.nAC) {
+                // (2) token scores A u, span-local online softmax, y = C^T p
+                __syncwarp();
+                const int t0 = (k - cur.nB) * cur.TC;
+                const int nt = min(cur.TC, cur.len - t0);
+                const unsigned char* As = zs;
+                const unsigned char* Cs = zs + C::ZSLOT / 2;
+                for (int c0 = 0; c0 < nt; c0 += 32) {
+                    const int t = c0 + lane;
+                    float xs[G];
+#pragma unroll
+                    for (int h = 0; h < G; ++h) xs[h] = 0.f;
+                    if (t < nt) {
+                        for (int i = 0; i < cur.rS; ++i) {
+                            const float av = load1<DT>(As, (int64_t)t * cur.rS + i);
+#pragma unroll
+                            for (int h = 0; h < G; ++h) xs[h] = fmaf(av, ub[i * G + h], xs[h]);
+                        }
+                    }
+                    float alL = 1.f;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float lg = (t < nt && ((cur.hm >> h) & 1u)) ? xs[h] * sl2 : -INFINITY;
+                        const float cm = warp_max(lg);
+                        const float mnew = fmaxf(msp[h], cm);
+                        const float al = (mnew == -INFINITY) ? 1.f : exp2f(msp[h] - mnew);
+                        const float p = (lg == -INFINITY) ? 0.f : exp2f(lg - mnew);
+                        lsp[h] = fmaf(lsp[h], al, warp_sum(p));
+                        msp[h] = mnew;
+                        pb[lane * G + h] = p;
+                        if (h == hL) alL = al;
+                    }
+                    __syncwarp();
+                    const int tn = min(32, nt - c0);
+#pragma unroll
+                    for (int j = 0; j < C::YPL; ++j) {
+                        const int i = (lane + 32 * j) / G;
+                        if (i < cur.rS) {
+                            float acc = y[j] * alL;
+                            for (int tt = 0; tt < tn; ++tt)
+                                acc = fmaf(pb[tt * G + hL], load1<DT>(Cs, (int64_t)(c0 + tt) * cur.rS + i), acc);
+                            y[j] = acc;
+                        }
+                    }
+                    __syncwarp();
+                }
+            } else {
+                if (k == cur.nB + cur.nAC) {
+                    // (3) merge the span's softmax state into the running state
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        float al = 1.f, be2 = 0.f;
+                        if ((cur.hm >> h) & 1u) {
+                            const float mnew = fmaxf(m_run[h], msp[h]);
+                            al = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mnew);
+                            be2 = exp2f(msp[h] - mnew);
+                            l_run[h] = l_run[h] * al + lsp[h] * be2;
+                            m_run[h] = mnew;
+                        }
+#pragma unroll
+                        for (int t = 0; t < DPL; ++t) o[h][t] *= al;
+                        if (h == hL) { betaL = be2; m_lane = m_run[h]; }
+                    }
+#pragma unroll
+                    for (int j = 0; j < C::YPL; ++j) {
+                        const int i = (lane + 32 * j) / G;
+                        if (i < cur.rS) yb[i * G + hL] = y[j] * betaL;
+                    }
+                    __syncwarp();
+                }
+                // o += sum_i (beta y_i) D_i over the slot's rows
+                const int r0 = (k - cur.nB - cur.nAC) * C::RB;
+                const int rows = min(C::RB, cur.rS - r0);
+                for (int r = 0; r < rows; ++r) {
+                    float dv[DPL];
+                    Vec<DT, DPL>::load(zs + r * C::ROWB + lane * DPL * C::ESZ, dv);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float yv = yb[(r0 + r) * G + h];
+#pragma unroll
+                        for (int t = 0; t < DPL; ++t) o[h][t] = fmaf(yv, dv[t], o[h][t]);
+                    }
+                }
+            }
+            __syncwarp();
+            ++ncons;
+        }
+        if (!zok) break;
+        // advance to the next span (the issue cursor may already be in it)
+        if (i_next) {
+            cur = nxt;
+            i_next = false;
+            nxt.valid = false;
+        } else {
+            cur = grab();
+            i_k = 0;
+        }
+    }
+    // drain anything still in flight (only after an error)
+    while (ncons < nis) {
+        if (!mbar_wait(&zb[ncons % C::ZNS], (ncons / C::ZNS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
+        ++ncons;
+    }
+}
+
+// write one partial softmax state in the dims-per-lane layout
+template <int D, int G>
+SEKV_DEV void store_state_lanes(const DecSmem& sm, int idx, int lane, const float (&m)[G], const float (&l)[G],
+                                const float (&o)[G][D / 32]) {
+    constexpr int DPL = D / 32;
+    if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            sm.st_m[idx * G + h] = m[h];
+            sm.st_l[idx * G + h] = l[h];
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) sm.st_o[(idx * G + h) * D + lane * DPL + k] = o[h][k];
+}
+
+template <int DT, int D, int G>
+__global__ void __launch_bounds__((kNW + 1) * 32, DT == SEKV_BF16 ? 2 : 3)
+decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     using C = DecCfg<DT, D, G>;
     constexpr int DPL = C::DPL, R = C::R, TR = C::TR, NS = C::NS;
-    extern __shared__ __align__(128) unsigned char sm[];
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm);          // [NS]
-    uint64_t* empty = full + 6;                                 // [NS]
-    uint64_t* zbar = full + 12;                                 // [kNW][ZNS]
-    int* qcnt = reinterpret_cast<int*>(sm + 192);               // [kNW]
-    int* zq_next = qcnt + kNW;
-    unsigned char* stages = sm + C::HDR;
-    int* zq = reinterpret_cast<int*>(stages + C::RING);
-    uint32_t* zw = reinterpret_cast<uint32_t*>(zq + kNW * a.qcap);
+    extern __shared__ __align__(1024) unsigned char sm_raw[];
+    unsigned char* base = sm_raw + ((1024 - (smem_u32(sm_raw) & 1023)) & 1023);
     const int zwords = a.sch_max / 32;
-    float* wscr = reinterpret_cast<float*>(zw + G * zwords);
+    const DecSmem sm = carve_smem<C, G, D>(base, a.qcap, zwords);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kvh = blockIdx.y;
@@ -141,20 +483,24 @@ decode_kernel(const DecArgs a) {
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kNW);
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], kNW);
         }
-        for (int s = 0; s < kNW * C::ZNS; ++s) mbar_init(&zbar[s], 1);
-        *zq_next = 0;
+        for (int s = 0; s < kNW * C::ZNS; ++s) mbar_init(&sm.zbar[s], 1);
+        *sm.zq_next = 0;
         fence_barrier_init();
     }
-    for (int i = tid; i < G * zwords; i += blockDim.x) zw[i] = 0u;
+    for (int i = tid; i < G * zwords; i += blockDim.x) sm.zw[i] = 0u;
     __syncthreads();
 
     const float sl2 = a.scale * kLog2e;
-    const int rL = lane / G, hL = lane % G;
-    // per-warp softmax state (warp-uniform) and per-lane output slice
-    float m_run[G], l_run[G], o[G][DPL], q[G][DPL];
+    bool ok = true;
+
+    // stream state of a consumer warp
+    //   tensor-core path: lane (g = lane/4, c = lane%4) holds head g's (m, l) and the
+    //   accumulator fragments oc[n][0..1] = O[g][8n + 2c .. 8n + 2c + 1]
+    //   CUDA-core path:   every lane holds (m, l) of all heads and o[h][dims of lane]
+    float m_run[G], l_run[G], o[G][DPL];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         m_run[h] = -INFINITY;
@@ -162,17 +508,11 @@ decode_kernel(const DecArgs a) {
 #pragma unroll
         for (int i = 0; i < DPL; ++i) o[h][i] = 0.f;
     }
-    {
-        const char* qp = a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB +
-                         lane * DPL * C::ESZ;
+    float m_lane = -INFINITY;
+    float oc[C::MMA ? D / 8 : 1][4];
+    float mm = -INFINITY, lm = 0.f;           // tensor-core path: this lane's head
 #pragma unroll
-        for (int h = 0; h < G; ++h) Vec<DT, DPL>::load(qp + h * C::ROWB, q[h]);
-    }
-    float m_lane = -INFINITY;                       // == m_run[hL]
-    bool ok = true;
-    float* pb = wscr + (warp < kNW ? warp : 0) * C::WSCR;   // 32*G floats (tile p / token p)
-    float* ub = pb + 32 * G;                                // kRMax*G floats
-    float* yb = ub + kRMax * G;                             // kRMax*G floats
+    for (int n = 0; n < (C::MMA ? D / 8 : 1); ++n) oc[n][0] = oc[n][1] = oc[n][2] = oc[n][3] = 0.f;
 
     if (warp == kNW) {
         // ------------------------------------------------------------ producer
@@ -180,51 +520,222 @@ decode_kernel(const DecArgs a) {
             int issued = 0;
             for (int i = 0; i < ntiles; ++i) {
                 const int s = i % NS;
-                if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) {
+                if (i >= NS && !mbar_wait(&sm.empty[s], ((i / NS) - 1) & 1)) {
                     set_status(a.status, SEKV_ERR_TIMEOUT);
                     break;
                 }
-                unsigned char* st = stages + (size_t)s * C::STAGE;
+                unsigned char* st = sm.stages + (size_t)s * C::STAGE;
                 if (i < nta) {
                     const int r0 = a0 + i * TR;
-                    const uint32_t bytes = (uint32_t)min(TR, a1 - r0) * C::ROWB;
-                    mbar_arrive_expect_tx(&full[s], 2 * bytes);
-                    const int64_t off = (unit * a.a_cap + r0) * C::ROWB;
-                    bulk_g2s(st, a.Ka + off, bytes, &full[s]);
-                    bulk_g2s(st + C::TILE, a.Va + off, bytes, &full[s]);
+                    if constexpr (C::MMA) {
+                        const int y = (int)(unit * a.a_cap + r0);
+                        mbar_arrive_expect_tx(&sm.full[s], 2 * C::NBOX * 8192);
+#pragma unroll
+                        for (int h = 0; h < C::NBOX; ++h) {
+                            tma_load_2d(st + h * 8192, &maps.Ka, 64 * h, y, &sm.full[s]);
+                            tma_load_2d(st + C::TILE + h * 8192, &maps.Va, 64 * h, y, &sm.full[s]);
+                        }
+                    } else {
+                        const uint32_t bytes = (uint32_t)min(TR, a1 - r0) * C::ROWB;
+                        mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
+                        const int64_t off = (unit * a.a_cap + r0) * C::ROWB;
+                        bulk_g2s(st, a.Ka + off, bytes, &sm.full[s]);
+                        bulk_g2s(st + C::TILE, a.Va + off, bytes, &sm.full[s]);
+                    }
                 } else {
                     const int S0 = s0 + (i - nta) * TR;
                     const int rows = min(TR, s1 - S0);
-                    const uint32_t bytes = (uint32_t)rows * C::ROWB;
                     const uint32_t mbytes = (uint32_t)((rows + 3) & ~3) * 4;
-                    mbar_arrive_expect_tx(&full[s], (route_only ? bytes : 2 * bytes) + 2 * mbytes);
-                    const int64_t off = (unit * a.m_cap + S0) * C::ROWB;
-                    bulk_g2s(st, a.kbar + off, bytes, &full[s]);
-                    if (!route_only) bulk_g2s(st + C::TILE, a.vbar + off, bytes, &full[s]);
-                    bulk_g2s(st + 2 * C::TILE, a.inv_norm + unit * a.m_cap + S0, mbytes, &full[s]);
-                    bulk_g2s(st + 2 * C::TILE + TR * 4, a.logS + (int64_t)b * a.m_cap + S0, mbytes, &full[s]);
+                    if constexpr (C::MMA) {
+                        const int y = (int)(unit * a.m_cap + S0);
+                        mbar_arrive_expect_tx(&sm.full[s], (route_only ? 1 : 2) * C::NBOX * 8192 + 2 * mbytes);
+#pragma unroll
+                        for (int h = 0; h < C::NBOX; ++h) {
+                            tma_load_2d(st + h * 8192, &maps.kbar, 64 * h, y, &sm.full[s]);
+                            if (!route_only) tma_load_2d(st + C::TILE + h * 8192, &maps.vbar, 64 * h, y, &sm.full[s]);
+                        }
+                    } else {
+                        const uint32_t bytes = (uint32_t)rows * C::ROWB;
+                        mbar_arrive_expect_tx(&sm.full[s], (route_only ? bytes : 2 * bytes) + 2 * mbytes);
+                        const int64_t off = (unit * a.m_cap + S0) * C::ROWB;
+                        bulk_g2s(st, a.kbar + off, bytes, &sm.full[s]);
+                        if (!route_only) bulk_g2s(st + C::TILE, a.vbar + off, bytes, &sm.full[s]);
+                    }
+                    bulk_g2s(st + 2 * C::TILE, a.inv_norm + unit * a.m_cap + S0, mbytes, &sm.full[s]);
+                    bulk_g2s(st + 2 * C::TILE + TR * 4, a.logS + (int64_t)b * a.m_cap + S0, mbytes, &sm.full[s]);
                 }
                 issued = i + 1;
             }
             // drain: every issued copy has landed before the ring is reused
             for (int i = max(0, issued - NS); i < issued; ++i)
-                if (!mbar_wait(&full[i % NS], (i / NS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
+                if (!mbar_wait(&sm.full[i % NS], (i / NS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
         }
-    } else {
-        // ------------------------------------------------------------ consumers
-        const float th = a.theta[(int64_t)l * a.Hq + kvh * G + hL];
-        int qn = 0;                                     // zoom-queue length (warp-uniform)
-        int* myq = zq + warp * a.qcap;
-        const int rbase = warp * R;
-
+    } else if constexpr (C::MMA) {
+        // ------------------------------------------------ consumers, tensor cores
+        const int g = lane >> 2, c = lane & 3;
+        const bool gv = g < G;
+        const float th = gv ? a.theta[(int64_t)l * a.Hq + kvh * G + g] : INFINITY;
+        // q as m16n8k16 A fragments (rows = heads, zero-padded to 16): a0, a2 per k-step
+        uint32_t qa[D / 16][2];
+        {
+            const uint32_t* qp = reinterpret_cast<const uint32_t*>(
+                a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G + (gv ? g : 0)) * C::ROWB);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                qa[kk][0] = gv ? qp[(16 * kk + 2 * c) / 2] : 0u;
+                qa[kk][1] = gv ? qp[(16 * kk + 8 + 2 * c) / 2] : 0u;
+            }
+        }
+        int qn = 0;
+        int* myq = sm.zq + warp * a.qcap;
+        const int rbase = warp * R;                       // 16 rows of each tile
         for (int i = 0; i < ntiles && ok; ++i) {
             const int s = i % NS;
-            if (!mbar_wait(&full[s], (i / NS) & 1)) {
+            if (!mbar_wait(&sm.full[s], (i / NS) & 1)) {
                 set_status(a.status, SEKV_ERR_TIMEOUT);
                 ok = false;
                 break;
             }
-            const unsigned char* st = stages + (size_t)s * C::STAGE;
+            const unsigned char* st = sm.stages + (size_t)s * C::STAGE;
+            const bool anchor_tile = i < nta;
+            const int S0 = s0 + (i - nta) * TR;
+            const int trows = anchor_tile ? min(TR, a1 - (a0 + i * TR)) : min(TR, s1 - S0);
+            if (rbase < trows) {
+                // ---- logits: q . K^T for the warp's 16 rows (two n-tiles of 8)
+                float acc[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+                    const int row = rbase + 8 * nt + (lane & 7);
+#pragma unroll
+                    for (int p = 0; p < D / 32; ++p) {
+                        const int chunk = (p & 1) * 4 + (lane >> 3);
+                        uint32_t kb[4];
+                        ldsm_x4(kb, st + (p >> 1) * 8192 + row * 128 + ((chunk ^ (row & 7)) << 4));
+                        const uint32_t a0f[4] = {qa[2 * p][0], 0u, qa[2 * p][1], 0u};
+                        const uint32_t a1f[4] = {qa[2 * p + 1][0], 0u, qa[2 * p + 1][1], 0u};
+                        const uint32_t b0[2] = {kb[0], kb[1]};
+                        const uint32_t b1[2] = {kb[2], kb[3]};
+                        mma_bf16_16816(acc[nt], a0f, b0);
+                        mma_bf16_16816(acc[nt], a1f, b1);
+                    }
+                }
+                // ---- routing, zoom decisions, logits in the log2 domain
+                float lg[2][2];
+                if (anchor_tile) {
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int tk = rbase + 8 * nt + 2 * c + e;
+                            lg[nt][e] = (gv && tk < trows) ? acc[nt][e] * sl2 : -INFINITY;
+                        }
+                } else {
+                    const float* invn = reinterpret_cast<const float*>(st + 2 * C::TILE);
+                    const float* lsv = invn + TR;
+                    uint32_t zbal[2][2];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int tk = rbase + 8 * nt + 2 * c + e;
+                            const bool valid = gv && tk < trows;
+                            const float x = acc[nt][e];
+                            const float ls = lsv[tk];
+                            const float ell = fmaf(x * invn[tk], a.scale, ls);     // Eq. (5) pre-sigmoid
+                            const bool z = valid && (ell > th);                    // Eq. (9)
+                            const int SL = S0 + tk;
+                            if (valid && a.route_logits)
+                                a.route_logits[(((int64_t)b * a.L + l) * a.Hq + kvh * G + g) * a.m_cap + SL] = ell;
+                            if (z) atomicOr(&sm.zw[g * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
+                            zbal[nt][e] = __ballot_sync(0xffffffffu, z);
+                            lg[nt][e] = (valid && !z) ? fmaf(x, a.scale, ls) * kLog2e : -INFINITY;
+                        }
+                    if (!route_only) {
+                        // queue every span of the warp's 16 rows that some head zooms
+                        const int t = lane & 15;
+                        const int tnt = t >> 3, tc = (t & 7) >> 1, te = t & 1;
+                        const uint32_t zb = tnt ? (te ? zbal[1][1] : zbal[1][0]) : (te ? zbal[0][1] : zbal[0][0]);
+                        uint32_t hm = 0u;
+#pragma unroll
+                        for (int h = 0; h < G; ++h) hm |= ((zb >> (4 * h + tc)) & 1u) << h;
+                        const bool has = lane < 16 && rbase + t < trows && hm != 0u;
+                        const uint32_t rows_with = __ballot_sync(0xffffffffu, has);
+                        if (has) {
+                            const int pos = qn + __popc(rows_with & ((1u << lane) - 1u));
+                            if (pos < a.qcap) myq[pos] = (S0 + rbase + t) | (int)(hm << 24);
+                        }
+                        qn += __popc(rows_with);
+                    }
+                }
+                if (!route_only) {
+                    // ---- online softmax for head g over the warp's 16 rows
+                    float mx = fmaxf(fmaxf(lg[0][0], lg[0][1]), fmaxf(lg[1][0], lg[1][1]));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    const float mnew = fmaxf(mm, mx);
+                    const float alpha = (mnew == -INFINITY) ? 1.f : exp2f(mm - mnew);
+                    float p[2][2];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) p[nt][e] = (lg[nt][e] == -INFINITY) ? 0.f : exp2f(lg[nt][e] - mnew);
+                    float ps = p[0][0] + p[0][1] + p[1][0] + p[1][1];
+                    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+                    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+                    lm = fmaf(lm, alpha, ps);
+                    mm = mnew;
+                    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                        for (int n = 0; n < D / 8; ++n) {
+                            oc[n][0] *= alpha;
+                            oc[n][1] *= alpha;
+                        }
+                    }
+                    // ---- O += P V (P as the A fragment: k = the 16 rows)
+                    const uint32_t pa[4] = {pack_bf16(p[0][0], p[0][1]), 0u, pack_bf16(p[1][0], p[1][1]), 0u};
+                    const unsigned char* vt = st + C::TILE;
+                    const int mi = lane >> 3;
+                    const int vrow = rbase + (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+                    for (int qd = 0; qd < D / 16; ++qd) {
+                        const int chunk = (qd & 3) * 2 + (mi >> 1);
+                        uint32_t vb[4];
+                        ldsm_x4_t(vb, vt + (qd >> 2) * 8192 + vrow * 128 + ((chunk ^ (vrow & 7)) << 4));
+                        const uint32_t b0[2] = {vb[0], vb[1]};
+                        const uint32_t b1[2] = {vb[2], vb[3]};
+                        mma_bf16_16816(oc[2 * qd], pa, b0);
+                        mma_bf16_16816(oc[2 * qd + 1], pa, b1);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[s]);
+        }
+        if (lane == 0) sm.qcnt[warp] = ok ? min(qn, a.qcap) : 0;
+    } else {
+        // ------------------------------------------------ consumers, CUDA cores
+        const int rL = lane / G, hL = lane % G;
+        float q[G][DPL];
+        {
+            const char* qp = a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB +
+                             lane * DPL * C::ESZ;
+#pragma unroll
+            for (int h = 0; h < G; ++h) Vec<DT, DPL>::load(qp + h * C::ROWB, q[h]);
+        }
+        const float th = a.theta[(int64_t)l * a.Hq + kvh * G + hL];
+        float* pb = reinterpret_cast<float*>(base + 512) + warp * 32;     // per-warp tile p
+        int qn = 0;
+        int* myq = sm.zq + warp * a.qcap;
+        const int rbase = warp * R;
+        for (int i = 0; i < ntiles && ok; ++i) {
+            const int s = i % NS;
+            if (!mbar_wait(&sm.full[s], (i / NS) & 1)) {
+                set_status(a.status, SEKV_ERR_TIMEOUT);
+                ok = false;
+                break;
+            }
+            const unsigned char* st = sm.stages + (size_t)s * C::STAGE;
             const bool anchor_tile = i < nta;
             const int S0 = s0 + (i - nta) * TR;
             const int trows = anchor_tile ? min(TR, a1 - (a0 + i * TR)) : min(TR, s1 - S0);
@@ -260,7 +771,7 @@ decode_kernel(const DecArgs a) {
                 const bool z = validL && (ell > th);                // Eq. (9)
                 if (validL && a.route_logits)
                     a.route_logits[(((int64_t)b * a.L + l) * a.Hq + kvh * G + hL) * a.m_cap + SL] = ell;
-                if (z) atomicOr(&zw[hL * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
+                if (z) atomicOr(&sm.zw[hL * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
                 if (!route_only) {
                     const uint32_t zb = __ballot_sync(0xffffffffu, z);
                     const uint32_t hm = (zb >> (rL * G)) & ((1u << G) - 1u);
@@ -275,7 +786,6 @@ decode_kernel(const DecArgs a) {
                 }
             }
             if (!route_only) {
-                // online softmax over this tile's rows, per head
                 float mx = lg2;
 #pragma unroll
                 for (int off = G; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -316,265 +826,36 @@ decode_kernel(const DecArgs a) {
                 __syncwarp();
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            if (lane == 0) mbar_arrive(&sm.empty[s]);
         }
-        if (lane == 0) qcnt[warp] = ok ? min(qn, a.qcap) : 0;
+        if (lane == 0) sm.qcnt[warp] = ok ? min(qn, a.qcap) : 0;
     }
     __syncthreads();    // the stream is done: the stage ring is free, the zoom queues are complete
 
-    // ---------------------------------------------------- zoomed spans
-    // Each consumer warp pulls spans from the CTA's queue and streams the span's
-    // block through its own ring of ZNS shared-memory slots (bulk copies, one
-    // mbarrier per slot): B rows -> u = B q; A/C token chunks -> scores A u, online
-    // softmax, y = C^T p; D rows -> o += beta * y^T D.
-    if (warp < kNW && !route_only && ok) {
-        const int nq_total = qcnt[0] + qcnt[1] + qcnt[2] + qcnt[3];
-        unsigned char* zring = stages + (size_t)warp * C::ZNS * C::ZSLOT;
-        uint64_t* zb = zbar + warp * C::ZNS;
-
-        auto grab = [&]() -> ZSpan {
-            ZSpan sp;
-            sp.valid = false;
-            sp.blk = nullptr;
-            sp.S = 0; sp.hm = 0u; sp.len = 0; sp.rS = 1; sp.nB = 0; sp.nAC = 0; sp.TC = 8; sp.pa = 0;
-            int e = 0;
-            if (lane == 0) e = atomicAdd(zq_next, 1);
-            e = __shfl_sync(0xffffffffu, e, 0);
-            if (e >= nq_total) return sp;
-            int w = 0;
-            while (w < kNW - 1 && e >= qcnt[w]) { e -= qcnt[w]; ++w; }
-            const int ent = zq[w * a.qcap + e];
-            sp.S = ent & 0xffffff;
-            sp.hm = (uint32_t)ent >> 24;
-            const int beg = a.span_beg[(int64_t)b * a.m_cap + sp.S];
-            sp.len = a.span_end[(int64_t)b * a.m_cap + sp.S] - beg;
-            if (sp.len < 1) {
-                set_status(a.status, SEKV_ERR_INVALID_ARG);
-                sp.len = 0;
-            }
-            sp.rS = sp.len > 0 ? block_rank(sp.len, D, a.rank) : 1;
-            sp.pa = block_ac_elems(sp.len, sp.rS);
-            const int64_t be = block_elems(sp.len > 0 ? sp.len : 1, D, a.rank);
-            int64_t off = -1;
-            if (sp.len > 0) {
-                if (a.slot) {
-                    off = a.slot[((int64_t)b * a.L + l) * a.m_cap + sp.S];
-                    if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
-                } else {
-                    off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + sp.S];
-                }
-            }
-            sp.blk = off >= 0 ? a.arena + (off + (int64_t)kvh * be) * C::ESZ : nullptr;
-            int tc = (C::ZSLOT / 2) / (sp.rS * C::ESZ);
-            tc = tc > 64 ? 64 : tc;
-            sp.TC = (tc & ~7) < 8 ? 8 : (tc & ~7);
-            sp.nB = (sp.rS + C::RB - 1) / C::RB;
-            sp.nAC = (sp.len + sp.TC - 1) / sp.TC;
-            sp.valid = true;
-            return sp;
-        };
-        auto nslots = [](const ZSpan& sp) { return sp.blk ? 2 * sp.nB + sp.nAC : 0; };
-
-        ZSpan cur = grab(), nxt;
-        nxt.valid = false;
-        nxt.blk = nullptr;
-        bool i_next = false;       // the issue cursor is in nxt
-        int i_k = 0;               // slots issued of the span under the issue cursor
-        uint32_t nis = 0, ncons = 0;
-        bool zok = true;
-
-        auto issue = [&]() {
-            // order this warp's earlier shared-memory reads of a slot before the
-            // bulk copy that refills it
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            while (nis - ncons < (uint32_t)C::ZNS) {
-                if (!i_next && i_k >= nslots(cur)) {
-                    if (!cur.valid) break;
-                    nxt = grab();
-                    i_next = true;
-                    i_k = 0;
-                }
-                // fields of the span under the issue cursor, selected by value
-                const bool sv = i_next ? nxt.valid : cur.valid;
-                const char* sblk = i_next ? nxt.blk : cur.blk;
-                const int snB = i_next ? nxt.nB : cur.nB, snAC = i_next ? nxt.nAC : cur.nAC;
-                const int srS = i_next ? nxt.rS : cur.rS, slen = i_next ? nxt.len : cur.len;
-                const int sTC = i_next ? nxt.TC : cur.TC;
-                const int64_t spa = i_next ? nxt.pa : cur.pa;
-                if (!sv || !sblk || i_k >= 2 * snB + snAC) break;
-                const int slot = nis % C::ZNS;
-                unsigned char* dst = zring + slot * C::ZSLOT;
-                if (lane == 0) {
-                    const int k = i_k;
-                    if (k < snB || k >= snB + snAC) {
-                        const bool isD = k >= snB;
-                        const int j = isD ? k - snB - snAC : k;
-                        const int r0 = j * C::RB;
-                        const uint32_t bytes = (uint32_t)min(C::RB, srS - r0) * C::ROWB;
-                        const char* src = sblk + (2 * spa + (isD ? (int64_t)srS * D : 0) + (int64_t)r0 * D) * C::ESZ;
-                        mbar_arrive_expect_tx(&zb[slot], bytes);
-                        bulk_g2s(dst, src, bytes, &zb[slot]);
-                    } else {
-                        const int t0 = (k - snB) * sTC;
-                        const int nt = min(sTC, slen - t0);
-                        const uint32_t bytes = (uint32_t)round_up((int64_t)nt * srS * C::ESZ, 16);
-                        const int64_t off = (int64_t)t0 * srS * C::ESZ;
-                        mbar_arrive_expect_tx(&zb[slot], 2 * bytes);
-                        bulk_g2s(dst, sblk + off, bytes, &zb[slot]);
-                        bulk_g2s(dst + C::ZSLOT / 2, sblk + spa * C::ESZ + off, bytes, &zb[slot]);
+    if (!route_only) {
+        if constexpr (C::MMA) {
+            // stream state of warp w -> state w; zoomed spans -> state kNW + w
+            if (warp < kNW) {
+                const int g = lane >> 2, c = lane & 3;
+                if (g < G) {
+                    if (c == 0) {
+                        sm.st_m[warp * G + g] = mm;
+                        sm.st_l[warp * G + g] = lm;
+                    }
+#pragma unroll
+                    for (int n = 0; n < D / 8; ++n) {
+                        sm.st_o[(warp * G + g) * D + 8 * n + 2 * c] = oc[n][0];
+                        sm.st_o[(warp * G + g) * D + 8 * n + 2 * c + 1] = oc[n][1];
                     }
                 }
-                ++i_k;
-                ++nis;
+                if (ok) zoom_phase<DT, D, G>(a, sm, warp, lane, b, l, kvh, m_run, l_run, o, m_lane);
+                store_state_lanes<D, G>(sm, kNW + warp, lane, m_run, l_run, o);
             }
-        };
-
-        while (cur.valid && zok) {
-            const int total = nslots(cur);
-            float msp[G], lsp[G];
-#pragma unroll
-            for (int h = 0; h < G; ++h) { msp[h] = -INFINITY; lsp[h] = 0.f; }
-            float y[C::YPL];
-#pragma unroll
-            for (int j = 0; j < C::YPL; ++j) y[j] = 0.f;
-            float betaL = 0.f;
-            for (int k = 0; k < total; ++k) {
-                issue();
-                const int slot = ncons % C::ZNS;
-                if (!mbar_wait(&zb[slot], (ncons / C::ZNS) & 1)) {
-                    set_status(a.status, SEKV_ERR_TIMEOUT);
-                    zok = false;
-                    break;
-                }
-                const unsigned char* zs = zring + slot * C::ZSLOT;
-                if (k < cur.nB) {
-                    // (1) u[i][h] = B_i . q_h for the slot's rows
-                    const int r0 = k * C::RB;
-                    const int rows = min(C::RB, cur.rS - r0);
-                    for (int i0 = 0; i0 < rows; i0 += R) {
-                        float part[32];
-#pragma unroll
-                        for (int r = 0; r < R; ++r) {
-                            float kk[DPL];
-                            if (i0 + r < rows) {
-                                Vec<DT, DPL>::load(zs + (i0 + r) * C::ROWB + lane * DPL * C::ESZ, kk);
-                            } else {
-#pragma unroll
-                                for (int t = 0; t < DPL; ++t) kk[t] = 0.f;
-                            }
-#pragma unroll
-                            for (int h = 0; h < G; ++h) {
-                                float acc = 0.f;
-#pragma unroll
-                                for (int t = 0; t < DPL; ++t) acc = fmaf(kk[t], q[h][t], acc);
-                                part[r * G + h] = acc;
-                            }
-                        }
-                        const float u = transpose_reduce32(part, lane);
-                        if (i0 + rL < rows) ub[(r0 + i0 + rL) * G + hL] = u;
-                    }
-                } else if (k < cur.nB + cur.nAC) {
-                    // (2) token scores, span-local online softmax, y = C^T p
-                    __syncwarp();
-                    const int t0 = (k - cur.nB) * cur.TC;
-                    const int nt = min(cur.TC, cur.len - t0);
-                    const unsigned char* As = zs;
-                    const unsigned char* Cs = zs + C::ZSLOT / 2;
-                    for (int c0 = 0; c0 < nt; c0 += 32) {
-                        const int t = c0 + lane;
-                        float xs[G];
-#pragma unroll
-                        for (int h = 0; h < G; ++h) xs[h] = 0.f;
-                        if (t < nt) {
-                            for (int i = 0; i < cur.rS; ++i) {
-                                const float av = load1<DT>(As, (int64_t)t * cur.rS + i);
-#pragma unroll
-                                for (int h = 0; h < G; ++h) xs[h] = fmaf(av, ub[i * G + h], xs[h]);
-                            }
-                        }
-                        float alL = 1.f;
-#pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            const float lg = (t < nt && ((cur.hm >> h) & 1u)) ? xs[h] * sl2 : -INFINITY;
-                            const float cm = warp_max(lg);
-                            const float mnew = fmaxf(msp[h], cm);
-                            const float al = (mnew == -INFINITY) ? 1.f : exp2f(msp[h] - mnew);
-                            const float p = (lg == -INFINITY) ? 0.f : exp2f(lg - mnew);
-                            lsp[h] = fmaf(lsp[h], al, warp_sum(p));
-                            msp[h] = mnew;
-                            pb[lane * G + h] = p;
-                            if (h == hL) alL = al;
-                        }
-                        __syncwarp();
-                        const int tn = min(32, nt - c0);
-#pragma unroll
-                        for (int j = 0; j < C::YPL; ++j) {
-                            const int i = (lane + 32 * j) / G;
-                            if (i < cur.rS) {
-                                float acc = y[j] * alL;
-                                for (int tt = 0; tt < tn; ++tt)
-                                    acc = fmaf(pb[tt * G + hL], load1<DT>(Cs, (int64_t)(c0 + tt) * cur.rS + i), acc);
-                                y[j] = acc;
-                            }
-                        }
-                        __syncwarp();
-                    }
-                } else {
-                    if (k == cur.nB + cur.nAC) {
-                        // (3) merge the span's softmax state into the warp's running state
-#pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            float al = 1.f, be2 = 0.f;
-                            if ((cur.hm >> h) & 1u) {
-                                const float mnew = fmaxf(m_run[h], msp[h]);
-                                al = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mnew);
-                                be2 = exp2f(msp[h] - mnew);
-                                l_run[h] = l_run[h] * al + lsp[h] * be2;
-                                m_run[h] = mnew;
-                            }
-#pragma unroll
-                            for (int t = 0; t < DPL; ++t) o[h][t] *= al;
-                            if (h == hL) { betaL = be2; m_lane = m_run[h]; }
-                        }
-#pragma unroll
-                        for (int j = 0; j < C::YPL; ++j) {
-                            const int i = (lane + 32 * j) / G;
-                            if (i < cur.rS) yb[i * G + hL] = y[j] * betaL;
-                        }
-                        __syncwarp();
-                    }
-                    // o += sum_i (beta y_i) D_i over the slot's rows
-                    const int r0 = (k - cur.nB - cur.nAC) * C::RB;
-                    const int rows = min(C::RB, cur.rS - r0);
-                    for (int r = 0; r < rows; ++r) {
-                        float dv[DPL];
-                        Vec<DT, DPL>::load(zs + r * C::ROWB + lane * DPL * C::ESZ, dv);
-#pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            const float yv = yb[(r0 + r) * G + h];
-#pragma unroll
-                            for (int t = 0; t < DPL; ++t) o[h][t] = fmaf(yv, dv[t], o[h][t]);
-                        }
-                    }
-                }
-                __syncwarp();
-                ++ncons;
+        } else {
+            if (warp < kNW) {
+                if (ok) zoom_phase<DT, D, G>(a, sm, warp, lane, b, l, kvh, m_run, l_run, o, m_lane);
+                store_state_lanes<D, G>(sm, warp, lane, m_run, l_run, o);
             }
-            if (!zok) break;
-            // advance to the next span (the issue cursor may already be in it)
-            if (i_next) {
-                cur = nxt;
-                i_next = false;
-                nxt.valid = false;
-            } else {
-                cur = grab();
-                i_k = 0;
-            }
-        }
-        // drain anything still in flight (only after an error)
-        while (ncons < nis) {
-            if (!mbar_wait(&zb[ncons % C::ZNS], (ncons / C::ZNS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
-            ++ncons;
         }
     }
     __syncthreads();
@@ -586,41 +867,24 @@ decode_kernel(const DecArgs a) {
         for (int i = tid; i < G * max(0, wend - w0); i += blockDim.x) {
             const int h = i / (wend - w0), j = i % (wend - w0);
             a.zmask[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.mw + w0 + j] =
-                (j < zwords) ? zw[h * zwords + j] : 0u;
+                (j < zwords) ? sm.zw[h * zwords + j] : 0u;
         }
     }
     if (route_only) return;
 
-    // ------------------------------------------------ merge the warps of this CTA
-    float* wm = reinterpret_cast<float*>(stages);          // [kNW][G]
-    float* wl = wm + kNW * G;                               // [kNW][G]
-    float* wo = wl + kNW * G;                               // [kNW][G][D]
-    if (warp < kNW) {
-        if (lane == 0) {
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                wm[warp * G + h] = m_run[h];
-                wl[warp * G + h] = l_run[h];
-            }
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int k = 0; k < DPL; ++k) wo[(warp * G + h) * D + lane * DPL + k] = o[h][k];
-    }
-    __syncthreads();
+    // ------------------------------------------------ merge the partial states of this CTA
     for (int i = tid; i < G * D; i += blockDim.x) {
         const int h = i / D, k = i % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kNW; ++w) M = fmaxf(M, wm[w * G + h]);
+        for (int w = 0; w < C::NSTATE; ++w) M = fmaxf(M, sm.st_m[w * G + h]);
         float Ls = 0.f, Os = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < kNW; ++w) {
-                const float f = exp2f(wm[w * G + h] - M);
-                Ls = fmaf(wl[w * G + h], f, Ls);
-                Os = fmaf(wo[(w * G + h) * D + k], f, Os);
+            for (int w = 0; w < C::NSTATE; ++w) {
+                const float f = exp2f(sm.st_m[w * G + h] - M);
+                Ls = fmaf(sm.st_l[w * G + h], f, Ls);
+                Os = fmaf(sm.st_o[(w * G + h) * D + k], f, Os);
             }
         }
         const int64_t pidx = (lunit * G + h) * a.nsplit + split;
@@ -712,6 +976,36 @@ DecodePlan plan_decode(const sekv_decode_desc& d) {
 
 size_t decode_workspace_bytes(const sekv_decode_desc& d) { return plan_decode(d).partial_bytes; }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// [rows][d] bf16 viewed with 64 x 64 boxes (128-byte rows of the box) and 128-byte swizzle
+static bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int d) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || !base) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int DT, int D, int G>
 static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st) {
     using C = DecCfg<DT, D, G>;
@@ -736,8 +1030,20 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
+    DecMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (C::MMA) {
+        const int64_t units_all = (int64_t)d.B * d.L * d.Hkv;
+        bool ok = encode_rows(&maps.kbar, d.kbar, units_all * d.m_cap, D);
+        if (d.phase != SEKV_ROUTE) {
+            ok = ok && encode_rows(&maps.vbar, d.vbar, units_all * d.m_cap, D) &&
+                 encode_rows(&maps.Ka, d.Ka, units_all * d.a_cap, D) &&
+                 encode_rows(&maps.Va, d.Va, units_all * d.a_cap, D);
+        }
+        if (!ok) return cudaErrorInvalidValue;
+    }
     dim3 grid(p.nsplit, d.Hkv, d.B * Lr);
-    decode_kernel<DT, D, G><<<grid, (kNW + 1) * 32, smem, st>>>(a);
+    decode_kernel<DT, D, G><<<grid, (kNW + 1) * 32, smem, st>>>(a, maps);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (d.phase != SEKV_ROUTE) {
         merge_kernel<D><<<d.B * Lr * d.Hq, D, 0, st>>>(a.part_o, a.part_ml, d.O, d.lse, p.nsplit, G, d.Hkv,
