@@ -106,6 +106,8 @@ def test_decode_end_to_end(name, over):
 
 
 def test_split_count_does_not_change_result():
+    """split-K + log-sum-exp merge equals a single pass, up to the rounding of the
+    bf16 probabilities fed to the tensor-core p.V product (2^-9 relative)"""
     wl = WORKLOADS["c2"].scaled(n=4096, L=1)
     H, K, V, segs, units, q, theta, scale = _setup(wl)
     c = _cache(wl)
@@ -118,7 +120,7 @@ def test_split_count_does_not_change_result():
         if ref is None:
             ref = (O_gpu.clone(), lse_gpu.clone())
         else:
-            assert (O_gpu - ref[0]).abs().max().item() < 2e-5
+            assert (O_gpu - ref[0]).abs().max().item() < 1e-3
             assert (lse_gpu - ref[1]).abs().max().item() < 2e-5
 
 
