@@ -55,7 +55,7 @@ struct DecCfg {
     static constexpr int NS0 = (MMA ? 68 * 1024 : 64 * 1024) / STAGE;     // 2 CTAs / SM on the bf16 path
     static constexpr int NS = NS0 < 2 ? 2 : (NS0 > 6 ? 6 : NS0);   // ring depth
     static constexpr int YPL = kRMax * G / 32;              // y entries per lane (zoom)
-    static constexpr int WSCR = (32 * G) + 2 * kRMax * G;   // per-warp scratch floats
+    static constexpr int WSCR = (64 * G) + 2 * kRMax * G;   // per-warp scratch floats
     // zoom phase: per-warp ring of ZNS slots of ZSLOT bytes, carved from the stage ring
     static constexpr int ZNS = 3;
     static constexpr int ZSLOT = 4096;
@@ -179,8 +179,8 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
     const int nq_total = sm.qcnt[0] + sm.qcnt[1] + sm.qcnt[2] + sm.qcnt[3];
     unsigned char* zring = sm.stages + (size_t)warp * C::ZNS * C::ZSLOT;
     uint64_t* zb = sm.zbar + warp * C::ZNS;
-    float* pb = sm.wscr + warp * C::WSCR;          // 32*G floats (token p)
-    float* ub = pb + 32 * G;                       // kRMax*G floats
+    float* pb = sm.wscr + warp * C::WSCR;          // 64*G floats (token p of a chunk)
+    float* ub = pb + 64 * G;                       // kRMax*G floats
     float* yb = ub + kRMax * G;                    // kRMax*G floats
 
     auto grab = [&]() -> ZSpan {
@@ -326,51 +326,120 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
                     if (i0 + rL < rows) ub[(r0 + i0 + rL) * G + hL] = u;
                 }
             } else if (k < cur.nB + cur.nAC) {
-                // (2) token scores A u, span-local online softmax, y = C^T p
+                // (2) token scores A u (lane owns tokens lane and lane+32 of the chunk),
+                //     span-local online softmax, y = C^T p
                 __syncwarp();
                 const int t0 = (k - cur.nB) * cur.TC;
                 const int nt = min(cur.TC, cur.len - t0);
                 const unsigned char* As = zs;
                 const unsigned char* Cs = zs + C::ZSLOT / 2;
-                for (int c0 = 0; c0 < nt; c0 += 32) {
-                    const int t = c0 + lane;
-                    float xs[G];
+                const int rS = cur.rS;
+                float xs[2][G];
 #pragma unroll
-                    for (int h = 0; h < G; ++h) xs[h] = 0.f;
-                    if (t < nt) {
-                        for (int i = 0; i < cur.rS; ++i) {
-                            const float av = load1<DT>(As, (int64_t)t * cur.rS + i);
+                for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
-                            for (int h = 0; h < G; ++h) xs[h] = fmaf(av, ub[i * G + h], xs[h]);
+                    for (int h = 0; h < G; ++h) xs[tt][h] = 0.f;
+                if (DT == SEKV_BF16 && (rS & 7) == 0) {
+                    for (int i0 = 0; i0 < rS; i0 += 8) {
+                        float av[2][8];
+#pragma unroll
+                        for (int tt = 0; tt < 2; ++tt) {
+                            const int t = lane + 32 * tt;
+                            if (t < nt) {
+                                const uint4 w = *reinterpret_cast<const uint4*>(As + ((int64_t)t * rS + i0) * 2);
+                                av[tt][0] = bf16_lo(w.x); av[tt][1] = bf16_hi(w.x);
+                                av[tt][2] = bf16_lo(w.y); av[tt][3] = bf16_hi(w.y);
+                                av[tt][4] = bf16_lo(w.z); av[tt][5] = bf16_hi(w.z);
+                                av[tt][6] = bf16_lo(w.w); av[tt][7] = bf16_hi(w.w);
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) av[tt][e] = 0.f;
+                            }
+                        }
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            float uv[G];
+                            if constexpr (G == 4) {
+                                const float4 u4 = *reinterpret_cast<const float4*>(ub + (i0 + e) * 4);
+                                uv[0] = u4.x; uv[1] = u4.y; uv[2] = u4.z; uv[3] = u4.w;
+                            } else {
+#pragma unroll
+                                for (int h = 0; h < G; ++h) uv[h] = ub[(i0 + e) * G + h];
+                            }
+#pragma unroll
+                            for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                                for (int h = 0; h < G; ++h) xs[tt][h] = fmaf(av[tt][e], uv[h], xs[tt][h]);
                         }
                     }
-                    float alL = 1.f;
+                } else {
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float lg = (t < nt && ((cur.hm >> h) & 1u)) ? xs[h] * sl2 : -INFINITY;
-                        const float cm = warp_max(lg);
-                        const float mnew = fmaxf(msp[h], cm);
-                        const float al = (mnew == -INFINITY) ? 1.f : exp2f(msp[h] - mnew);
-                        const float p = (lg == -INFINITY) ? 0.f : exp2f(lg - mnew);
-                        lsp[h] = fmaf(lsp[h], al, warp_sum(p));
-                        msp[h] = mnew;
-                        pb[lane * G + h] = p;
-                        if (h == hL) alL = al;
-                    }
-                    __syncwarp();
-                    const int tn = min(32, nt - c0);
+                    for (int tt = 0; tt < 2; ++tt) {
+                        const int t = lane + 32 * tt;
+                        if (t < nt) {
+                            for (int i = 0; i < rS; ++i) {
+                                const float av = load1<DT>(As, (int64_t)t * rS + i);
 #pragma unroll
-                    for (int j = 0; j < C::YPL; ++j) {
-                        const int i = (lane + 32 * j) / G;
-                        if (i < cur.rS) {
-                            float acc = y[j] * alL;
-                            for (int tt = 0; tt < tn; ++tt)
-                                acc = fmaf(pb[tt * G + hL], load1<DT>(Cs, (int64_t)(c0 + tt) * cur.rS + i), acc);
-                            y[j] = acc;
+                                for (int h = 0; h < G; ++h) xs[tt][h] = fmaf(av, ub[i * G + h], xs[tt][h]);
+                            }
                         }
                     }
-                    __syncwarp();
                 }
+                // logits of the heads that zoom this span; the others get no entries here
+                float mx[G], ps[G], al[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const bool zh = (cur.hm >> h) & 1u;
+#pragma unroll
+                    for (int tt = 0; tt < 2; ++tt)
+                        xs[tt][h] = (zh && lane + 32 * tt < nt) ? xs[tt][h] * sl2 : -INFINITY;
+                    mx[h] = fmaxf(xs[0][h], xs[1][h]);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                    for (int h = 0; h < G; ++h) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], off));
+                float alL = 1.f;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float mnew = fmaxf(msp[h], mx[h]);
+                    al[h] = (mnew == -INFINITY) ? 1.f : exp2f(msp[h] - mnew);
+                    ps[h] = 0.f;
+#pragma unroll
+                    for (int tt = 0; tt < 2; ++tt) {
+                        const float pv = (xs[tt][h] == -INFINITY) ? 0.f : exp2f(xs[tt][h] - mnew);
+                        ps[h] += pv;
+                        pb[(lane + 32 * tt) * G + h] = pv;
+                    }
+                    msp[h] = mnew;
+                    if (h == hL) alL = al[h];
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                    for (int h = 0; h < G; ++h) ps[h] += __shfl_xor_sync(0xffffffffu, ps[h], off);
+#pragma unroll
+                for (int h = 0; h < G; ++h) lsp[h] = fmaf(lsp[h], al[h], ps[h]);
+                __syncwarp();
+                // y[i][h] += sum_t p[t][h] C[t][i]; lanes own (i, h) pairs
+#pragma unroll
+                for (int j = 0; j < C::YPL; ++j) {
+                    const int i = (lane + 32 * j) / G;
+                    if (i < rS) {
+                        float acc0 = y[j] * alL, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+                        int tt = 0;
+                        for (; tt + 4 <= nt; tt += 4) {
+                            acc0 = fmaf(pb[(tt + 0) * G + hL], load1<DT>(Cs, (int64_t)(tt + 0) * rS + i), acc0);
+                            acc1 = fmaf(pb[(tt + 1) * G + hL], load1<DT>(Cs, (int64_t)(tt + 1) * rS + i), acc1);
+                            acc2 = fmaf(pb[(tt + 2) * G + hL], load1<DT>(Cs, (int64_t)(tt + 2) * rS + i), acc2);
+                            acc3 = fmaf(pb[(tt + 3) * G + hL], load1<DT>(Cs, (int64_t)(tt + 3) * rS + i), acc3);
+                        }
+                        for (; tt < nt; ++tt)
+                            acc0 = fmaf(pb[tt * G + hL], load1<DT>(Cs, (int64_t)tt * rS + i), acc0);
+                        y[j] = (acc0 + acc1) + (acc2 + acc3);
+                    }
+                }
+                __syncwarp();
             } else {
                 if (k == cur.nB + cur.nAC) {
                     // (3) merge the span's softmax state into the running state
