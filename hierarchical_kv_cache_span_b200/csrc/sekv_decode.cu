@@ -55,7 +55,7 @@ struct DecCfg {
     static constexpr int NS0 = (MMA ? 68 * 1024 : 64 * 1024) / STAGE;     // 2 CTAs / SM on the bf16 path
     static constexpr int NS = NS0 < 2 ? 2 : (NS0 > 6 ? 6 : NS0);   // ring depth
     static constexpr int YPL = kRMax * G / 32;              // y entries per lane (zoom)
-    static constexpr int WSCR = (64 * G) + 2 * kRMax * G;   // per-warp scratch floats
+    static constexpr int WSCR = MMA ? 0 : (64 * G) + 2 * kRMax * G;   // per-warp scratch floats (fp32 zoom)
     // zoom phase: per-warp ring of ZNS slots of ZSLOT bytes, carved from the stage ring
     static constexpr int ZNS = 3;
     static constexpr int ZSLOT = 4096;
@@ -63,10 +63,12 @@ struct DecCfg {
     static constexpr int ZBYTES = kNW * ZNS * ZSLOT;
     // partial softmax states merged at the end: per warp one for the stream and,
     // on the tensor-core path, one for its zoomed spans
-    static constexpr int NSTATE = MMA ? 2 * kNW : kNW;
+    static constexpr int NSTATE = kNW;
     static constexpr int SBYTES = NSTATE * (G * D + 2 * G) * 4;
+    // tensor-core zoom scratch per warp: u^T and (beta y)^T as hi/lo bf16 [2][8][72], p^T [8][24]
+    static constexpr int ZSCR = 5120;
     static constexpr int RING0 = NS * STAGE;
-    static constexpr int RING1 = ZBYTES + SBYTES;
+    static constexpr int RING1 = ZBYTES + (MMA ? kNW * ZSCR : 0) > SBYTES ? ZBYTES + (MMA ? kNW * ZSCR : 0) : SBYTES;
     static constexpr int RING = RING0 > RING1 ? RING0 : RING1;
     static constexpr int HDR = 1024;                        // mbarriers + counters (keeps stages 1 KB aligned)
 };
@@ -135,7 +137,7 @@ struct DecSmem {
     int* zq;             // [kNW][qcap]
     uint32_t* zw;        // [G][zwords]
     float* wscr;         // [kNW][WSCR]
-    float* st_m;         // [NSTATE][G]   (in the ring, after the zoom slots)
+    float* st_m;         // [NSTATE][G]   (in the ring, once the zoom phase is over)
     float* st_l;         // [NSTATE][G]
     float* st_o;         // [NSTATE][G][D]
 };
@@ -152,7 +154,7 @@ SEKV_DEV DecSmem carve_smem(unsigned char* base, int qcap, int zwords) {
     s.zq = reinterpret_cast<int*>(s.stages + C::RING);
     s.zw = reinterpret_cast<uint32_t*>(s.zq + kNW * qcap);
     s.wscr = reinterpret_cast<float*>(s.zw + G * zwords);
-    s.st_m = reinterpret_cast<float*>(s.stages + C::ZBYTES);
+    s.st_m = reinterpret_cast<float*>(s.stages);             // written after the zoom phase
     s.st_l = s.st_m + C::NSTATE * G;
     s.st_o = s.st_l + C::NSTATE * G;
     return s;
@@ -499,6 +501,343 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
     }
 }
 
+// ---------------------------------------------------------------------------
+// Phase 2 on the tensor cores (bf16). Per zoomed span and the heads h that zoom
+// it, with r = rank of the span:
+//   u = B_S q          (mma: M = r basis rows, K = d, N = heads)
+//   s = A_S u          (mma: M = 16 tokens, K = r)             -> online softmax p
+//   y = C_S^T p        (mma: M = r, K = 16 tokens)
+//   O += (beta y)^T D_S (mma: M = heads, K = r, N = d)  into the stream accumulators
+// u and beta*y are rounded to bf16 as a hi + lo pair (about 16 significant bits);
+// p is rounded to bf16 as on the streaming path. The span's (max, sum) merge into
+// the warp's stream state (mm, lm, oc) for head gid = lane/4.
+// ---------------------------------------------------------------------------
+template <int D, int G>
+SEKV_DEV void zoom_phase_mma(const DecArgs& a, const DecSmem& sm, int warp, int lane, int b, int l, int kvh,
+                             const uint32_t (&qa)[D / 16][2], float& mm, float& lm, float (&oc)[D / 8][4]) {
+    using C = DecCfg<SEKV_BF16, D, G>;
+    constexpr int ROWB = C::ROWB;
+    constexpr int RB = C::RB;
+    const int gid = lane >> 2, cq = lane & 3;
+    const float sl2 = a.scale * kLog2e;
+    const int nq_total = sm.qcnt[0] + sm.qcnt[1] + sm.qcnt[2] + sm.qcnt[3];
+    unsigned char* zring = sm.stages + (size_t)warp * C::ZNS * C::ZSLOT;
+    uint64_t* zb = sm.zbar + warp * C::ZNS;
+    __nv_bfloat16* ut = reinterpret_cast<__nv_bfloat16*>(sm.stages + C::ZBYTES + warp * C::ZSCR);  // [2][8][72]
+    __nv_bfloat16* yt = ut + 2 * 8 * 72;                                                        // [2][8][72]
+    __nv_bfloat16* pt = yt + 2 * 8 * 72;                                                        // [8][24]
+
+    auto grab = [&]() -> ZSpan {
+        ZSpan sp;
+        sp.valid = false;
+        sp.blk = nullptr;
+        sp.S = 0; sp.hm = 0u; sp.len = 0; sp.rS = 1; sp.nB = 0; sp.nAC = 0; sp.TC = 8; sp.pa = 0;
+        int e = 0;
+        if (lane == 0) e = atomicAdd(sm.zq_next, 1);
+        e = __shfl_sync(0xffffffffu, e, 0);
+        if (e >= nq_total) return sp;
+        int w = 0;
+        while (w < kNW - 1 && e >= sm.qcnt[w]) { e -= sm.qcnt[w]; ++w; }
+        const int ent = sm.zq[w * a.qcap + e];
+        sp.S = ent & 0xffffff;
+        sp.hm = (uint32_t)ent >> 24;
+        const int beg = a.span_beg[(int64_t)b * a.m_cap + sp.S];
+        sp.len = a.span_end[(int64_t)b * a.m_cap + sp.S] - beg;
+        if (sp.len < 1) {
+            set_status(a.status, SEKV_ERR_INVALID_ARG);
+            sp.len = 0;
+        }
+        sp.rS = sp.len > 0 ? block_rank(sp.len, D, a.rank) : 1;
+        sp.pa = block_ac_elems(sp.len, sp.rS);
+        const int64_t be = block_elems(sp.len > 0 ? sp.len : 1, D, a.rank);
+        int64_t off = -1;
+        if (sp.len > 0) {
+            if (a.slot) {
+                off = a.slot[((int64_t)b * a.L + l) * a.m_cap + sp.S];
+                if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
+            } else {
+                off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + sp.S];
+            }
+        }
+        sp.blk = off >= 0 ? a.arena + (off + (int64_t)kvh * be) * 2 : nullptr;
+        int tc = (C::ZSLOT / 2) / (sp.rS * 2);
+        tc = tc > 64 ? 64 : tc;
+        sp.TC = (tc & ~7) < 8 ? 8 : (tc & ~7);
+        sp.nB = (sp.rS + RB - 1) / RB;
+        sp.nAC = (sp.len + sp.TC - 1) / sp.TC;
+        sp.valid = true;
+        return sp;
+    };
+    auto nslots = [](const ZSpan& sp) { return sp.blk ? 2 * sp.nB + sp.nAC : 0; };
+
+    ZSpan cur = grab(), nxt;
+    nxt.valid = false;
+    nxt.blk = nullptr;
+    nxt.nB = nxt.nAC = 0;
+    bool i_next = false;
+    int i_k = 0;
+    uint32_t nis = 0, ncons = 0;
+    bool zok = true;
+
+    auto issue = [&]() {
+        fence_proxy_async();
+        while (nis - ncons < (uint32_t)C::ZNS) {
+            if (!i_next && i_k >= nslots(cur)) {
+                if (!cur.valid) break;
+                nxt = grab();
+                i_next = true;
+                i_k = 0;
+            }
+            const bool sv = i_next ? nxt.valid : cur.valid;
+            const char* sblk = i_next ? nxt.blk : cur.blk;
+            const int snB = i_next ? nxt.nB : cur.nB, snAC = i_next ? nxt.nAC : cur.nAC;
+            const int srS = i_next ? nxt.rS : cur.rS, slen = i_next ? nxt.len : cur.len;
+            const int sTC = i_next ? nxt.TC : cur.TC;
+            const int64_t spa = i_next ? nxt.pa : cur.pa;
+            if (!sv || !sblk || i_k >= 2 * snB + snAC) break;
+            const int slot = nis % C::ZNS;
+            unsigned char* dst = zring + slot * C::ZSLOT;
+            if (lane == 0) {
+                const int k = i_k;
+                if (k < snB || k >= snB + snAC) {
+                    const bool isD = k >= snB;
+                    const int j = isD ? k - snB - snAC : k;
+                    const int r0 = j * RB;
+                    const uint32_t bytes = (uint32_t)min(RB, srS - r0) * ROWB;
+                    const char* src = sblk + (2 * spa + (isD ? (int64_t)srS * D : 0) + (int64_t)r0 * D) * 2;
+                    mbar_arrive_expect_tx(&zb[slot], bytes);
+                    bulk_g2s(dst, src, bytes, &zb[slot]);
+                } else {
+                    const int t0 = (k - snB) * sTC;
+                    const int nt = min(sTC, slen - t0);
+                    const uint32_t bytes = (uint32_t)round_up((int64_t)nt * srS * 2, 16);
+                    const int64_t off = (int64_t)t0 * srS * 2;
+                    mbar_arrive_expect_tx(&zb[slot], 2 * bytes);
+                    bulk_g2s(dst, sblk + off, bytes, &zb[slot]);
+                    bulk_g2s(dst + C::ZSLOT / 2, sblk + spa * 2 + off, bytes, &zb[slot]);
+                }
+            }
+            ++i_k;
+            ++nis;
+        }
+    };
+
+    while (cur.valid && zok) {
+        const int total = nslots(cur);
+        const int rS = cur.rS;
+        const int nig = (rS + 15) >> 4;                 // groups of 16 basis rows
+        float msp[2] = {-INFINITY, -INFINITY}, lsp[2] = {0.f, 0.f};   // heads 2cq, 2cq+1
+        float yacc[4][4];
+#pragma unroll
+        for (int ig = 0; ig < 4; ++ig) yacc[ig][0] = yacc[ig][1] = yacc[ig][2] = yacc[ig][3] = 0.f;
+        for (int k = 0; k < total; ++k) {
+            issue();
+            const int slot = ncons % C::ZNS;
+            if (!mbar_wait(&zb[slot], (ncons / C::ZNS) & 1)) {
+                set_status(a.status, SEKV_ERR_TIMEOUT);
+                zok = false;
+                break;
+            }
+            const unsigned char* zs = zring + slot * C::ZSLOT;
+            if (k < cur.nB) {
+                // (1) u = B q for the slot's basis rows, stored transposed as hi/lo bf16
+                const int r0 = k * RB;
+                const int rows = min(RB, rS - r0);
+                for (int g16 = 0; g16 < rows; g16 += 16) {
+                    float uacc[4] = {0.f, 0.f, 0.f, 0.f};
+                    const int arow = g16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        uint32_t af[4];
+                        ldsm_x4(af, zs + arow * ROWB + (16 * kk + ((lane >> 4) << 3)) * 2);
+                        const uint32_t bq[2] = {qa[kk][0], qa[kk][1]};
+                        mma_bf16_16816(uacc, af, bq);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int il = g16 + gid + ((e >> 1) << 3);          // row within the slot
+                        const int i = r0 + il;
+                        const int h = 2 * cq + (e & 1);
+                        const float u = (il < rows) ? uacc[e] : 0.f;       // stale rows beyond r
+                        const __nv_bfloat16 hi = __float2bfloat16_rn(u);
+                        ut[h * 72 + i] = hi;
+                        ut[(8 + h) * 72 + i] = __float2bfloat16_rn(u - __bfloat162float(hi));
+                    }
+                }
+            } else if (k < cur.nB + cur.nAC) {
+                // (2) scores s = A u, span-local online softmax, y += C^T p, 16 tokens at a time
+                __syncwarp();
+                const int t0 = (k - cur.nB) * cur.TC;
+                const int nt = min(cur.TC, cur.len - t0);
+                const uint16_t* A16 = reinterpret_cast<const uint16_t*>(zs);
+                const uint16_t* C16 = reinterpret_cast<const uint16_t*>(zs + C::ZSLOT / 2);
+                for (int ts = 0; ts < nt; ts += 16) {
+                    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int ks = 0; ks < nig; ++ks) {
+                        uint32_t af[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int t = ts + gid + ((e & 1) << 3);
+                            const int i = 16 * ks + 2 * cq + ((e >> 1) << 3);
+                            const uint32_t x0 = (t < nt && i < rS) ? A16[t * rS + i] : 0u;
+                            const uint32_t x1 = (t < nt && i + 1 < rS) ? A16[t * rS + i + 1] : 0u;
+                            af[e] = x0 | (x1 << 16);
+                        }
+                        const uint32_t* uh = reinterpret_cast<const uint32_t*>(ut + gid * 72 + 16 * ks + 2 * cq);
+                        const uint32_t* ul = reinterpret_cast<const uint32_t*>(ut + (8 + gid) * 72 + 16 * ks + 2 * cq);
+                        const uint32_t bh[2] = {uh[0], uh[4]};
+                        const uint32_t bl[2] = {ul[0], ul[4]};
+                        mma_bf16_16816(sacc, af, bh);
+                        mma_bf16_16816(sacc, af, bl);
+                    }
+                    // sacc[e]: token ts + gid + 8*(e>>1), head 2cq + (e&1)
+                    float lg[4], p[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int t = ts + gid + ((e >> 1) << 3);
+                        const int h = 2 * cq + (e & 1);
+                        lg[e] = (t < nt && h < G && ((cur.hm >> h) & 1u)) ? sacc[e] * sl2 : -INFINITY;
+                    }
+                    float mx0 = fmaxf(lg[0], lg[2]), mx1 = fmaxf(lg[1], lg[3]);
+#pragma unroll
+                    for (int off = 4; off < 32; off <<= 1) {
+                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                    }
+                    const float mn0 = fmaxf(msp[0], mx0), mn1 = fmaxf(msp[1], mx1);
+                    const float al0 = (mn0 == -INFINITY) ? 1.f : exp2f(msp[0] - mn0);
+                    const float al1 = (mn1 == -INFINITY) ? 1.f : exp2f(msp[1] - mn1);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        p[e] = (lg[e] == -INFINITY) ? 0.f : exp2f(lg[e] - ((e & 1) ? mn1 : mn0));
+                    float ps0 = p[0] + p[2], ps1 = p[1] + p[3];
+#pragma unroll
+                    for (int off = 4; off < 32; off <<= 1) {
+                        ps0 += __shfl_xor_sync(0xffffffffu, ps0, off);
+                        ps1 += __shfl_xor_sync(0xffffffffu, ps1, off);
+                    }
+                    lsp[0] = fmaf(lsp[0], al0, ps0);
+                    lsp[1] = fmaf(lsp[1], al1, ps1);
+                    msp[0] = mn0;
+                    msp[1] = mn1;
+                    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+                        for (int ig = 0; ig < 4; ++ig) {
+                            yacc[ig][0] *= al0; yacc[ig][1] *= al1;
+                            yacc[ig][2] *= al0; yacc[ig][3] *= al1;
+                        }
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        pt[(2 * cq + (e & 1)) * 24 + gid + ((e >> 1) << 3)] = __float2bfloat16_rn(p[e]);
+                    __syncwarp();
+                    const uint32_t* pp = reinterpret_cast<const uint32_t*>(pt + gid * 24 + 2 * cq);
+                    const uint32_t bp[2] = {pp[0], pp[4]};
+#pragma unroll
+                    for (int ig = 0; ig < 4; ++ig) {
+                        if (ig < nig) {
+                            uint32_t af[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int i = 16 * ig + gid + ((e & 1) << 3);
+                                const int t = ts + 2 * cq + ((e >> 1) << 3);
+                                const uint32_t x0 = (i < rS && t < nt) ? C16[t * rS + i] : 0u;
+                                const uint32_t x1 = (i < rS && t + 1 < nt) ? C16[(t + 1) * rS + i] : 0u;
+                                af[e] = x0 | (x1 << 16);
+                            }
+                            mma_bf16_16816(yacc[ig], af, bp);
+                        }
+                    }
+                }
+            } else {
+                if (k == cur.nB + cur.nAC) {
+                    // (3) merge: beta per zooming head, (beta y)^T to shared memory, stream state update
+                    const float mh0 = __shfl_sync(0xffffffffu, mm, 4 * (2 * cq));
+                    const float mh1 = __shfl_sync(0xffffffffu, mm, 4 * (2 * cq + 1));
+                    const bool z0 = 2 * cq < G && ((cur.hm >> (2 * cq)) & 1u);
+                    const bool z1 = 2 * cq + 1 < G && ((cur.hm >> (2 * cq + 1)) & 1u);
+                    const float be0 = z0 ? exp2f(msp[0] - fmaxf(mh0, msp[0])) : 0.f;
+                    const float be1 = z1 ? exp2f(msp[1] - fmaxf(mh1, msp[1])) : 0.f;
+#pragma unroll
+                    for (int ig = 0; ig < 4; ++ig) {
+                        if (ig < nig) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int i = 16 * ig + gid + ((e >> 1) << 3);
+                                const int h = 2 * cq + (e & 1);
+                                const float v = yacc[ig][e] * ((e & 1) ? be1 : be0);
+                                const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+                                yt[h * 72 + i] = hi;
+                                yt[(8 + h) * 72 + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
+                            }
+                        }
+                    }
+                    const int src = gid >> 1;
+                    const float ms0 = __shfl_sync(0xffffffffu, msp[0], src), ms1 = __shfl_sync(0xffffffffu, msp[1], src);
+                    const float ls0 = __shfl_sync(0xffffffffu, lsp[0], src), ls1 = __shfl_sync(0xffffffffu, lsp[1], src);
+                    const float msg = (gid & 1) ? ms1 : ms0, lsg = (gid & 1) ? ls1 : ls0;
+                    if (gid < G && ((cur.hm >> gid) & 1u)) {
+                        const float mnew = fmaxf(mm, msg);
+                        const float alpha = (mm == -INFINITY) ? 0.f : exp2f(mm - mnew);
+                        const float beta = exp2f(msg - mnew);
+                        lm = lm * alpha + lsg * beta;
+                        mm = mnew;
+#pragma unroll
+                        for (int n = 0; n < D / 8; ++n) {
+                            oc[n][0] *= alpha;
+                            oc[n][1] *= alpha;
+                        }
+                    }
+                    __syncwarp();
+                }
+                // (4) O += (beta y)^T D over the slot's basis rows
+                const int r0 = (k - cur.nB - cur.nAC) * RB;
+                const int rows = min(RB, rS - r0);
+                for (int g16 = 0; g16 < rows; g16 += 16) {
+                    const int ks = (r0 + g16) >> 4;
+                    const uint32_t* yh = reinterpret_cast<const uint32_t*>(yt + gid * 72 + 16 * ks + 2 * cq);
+                    const uint32_t* yl = reinterpret_cast<const uint32_t*>(yt + (8 + gid) * 72 + 16 * ks + 2 * cq);
+                    const uint32_t ah[4] = {yh[0], 0u, yh[4], 0u};
+                    const uint32_t al[4] = {yl[0], 0u, yl[4], 0u};
+                    const int mi = lane >> 3;
+                    const int drow = g16 + (lane & 7) + ((mi & 1) << 3);
+                    // this lane's B rows (k): g16 + 2cq, +1 (b0) and +8 (b1); zero the stale ones
+                    const int k0 = g16 + 2 * cq;
+                    const uint32_t m0 = (k0 < rows ? 0x0000ffffu : 0u) | (k0 + 1 < rows ? 0xffff0000u : 0u);
+                    const uint32_t m1 = (k0 + 8 < rows ? 0x0000ffffu : 0u) | (k0 + 9 < rows ? 0xffff0000u : 0u);
+#pragma unroll
+                    for (int qd = 0; qd < D / 16; ++qd) {
+                        uint32_t vb[4];
+                        ldsm_x4_t(vb, zs + drow * ROWB + (16 * qd + ((mi >> 1) << 3)) * 2);
+                        const uint32_t b0[2] = {vb[0] & m0, vb[1] & m1};
+                        const uint32_t b1[2] = {vb[2] & m0, vb[3] & m1};
+                        mma_bf16_16816(oc[2 * qd], ah, b0);
+                        mma_bf16_16816(oc[2 * qd], al, b0);
+                        mma_bf16_16816(oc[2 * qd + 1], ah, b1);
+                        mma_bf16_16816(oc[2 * qd + 1], al, b1);
+                    }
+                }
+            }
+            __syncwarp();
+            ++ncons;
+        }
+        if (!zok) break;
+        if (i_next) {
+            cur = nxt;
+            i_next = false;
+            nxt.valid = false;
+        } else {
+            cur = grab();
+            i_k = 0;
+        }
+    }
+    while (ncons < nis) {
+        if (!mbar_wait(&zb[ncons % C::ZNS], (ncons / C::ZNS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
+        ++ncons;
+    }
+}
+
 // write one partial softmax state in the dims-per-lane layout
 template <int D, int G>
 SEKV_DEV void store_state_lanes(const DecSmem& sm, int idx, int lane, const float (&m)[G], const float (&l)[G],
@@ -578,6 +917,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         for (int i = 0; i < DPL; ++i) o[h][i] = 0.f;
     }
     float m_lane = -INFINITY;
+    uint32_t qa[C::MMA ? D / 16 : 1][2];      // tensor-core path: q fragments (stream and zoom)
     float oc[C::MMA ? D / 8 : 1][4];
     float mm = -INFINITY, lm = 0.f;           // tensor-core path: this lane's head
 #pragma unroll
@@ -645,7 +985,6 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         const bool gv = g < G;
         const float th = gv ? a.theta[(int64_t)l * a.Hq + kvh * G + g] : INFINITY;
         // q as m16n8k16 A fragments (rows = heads, zero-padded to 16): a0, a2 per k-step
-        uint32_t qa[D / 16][2];
         {
             const uint32_t* qp = reinterpret_cast<const uint32_t*>(
                 a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G + (gv ? g : 0)) * C::ROWB);
@@ -901,30 +1240,27 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     }
     __syncthreads();    // the stream is done: the stage ring is free, the zoom queues are complete
 
-    if (!route_only) {
+    if (!route_only && warp < kNW && ok) {
+        if constexpr (C::MMA) zoom_phase_mma<D, G>(a, sm, warp, lane, b, l, kvh, qa, mm, lm, oc);
+        else zoom_phase<DT, D, G>(a, sm, warp, lane, b, l, kvh, m_run, l_run, o, m_lane);
+    }
+    __syncthreads();    // zoom slots and scratch are dead: the ring takes the partial states
+    if (!route_only && warp < kNW) {
         if constexpr (C::MMA) {
-            // stream state of warp w -> state w; zoomed spans -> state kNW + w
-            if (warp < kNW) {
-                const int g = lane >> 2, c = lane & 3;
-                if (g < G) {
-                    if (c == 0) {
-                        sm.st_m[warp * G + g] = mm;
-                        sm.st_l[warp * G + g] = lm;
-                    }
-#pragma unroll
-                    for (int n = 0; n < D / 8; ++n) {
-                        sm.st_o[(warp * G + g) * D + 8 * n + 2 * c] = oc[n][0];
-                        sm.st_o[(warp * G + g) * D + 8 * n + 2 * c + 1] = oc[n][1];
-                    }
+            const int g = lane >> 2, c = lane & 3;
+            if (g < G) {
+                if (c == 0) {
+                    sm.st_m[warp * G + g] = mm;
+                    sm.st_l[warp * G + g] = lm;
                 }
-                if (ok) zoom_phase<DT, D, G>(a, sm, warp, lane, b, l, kvh, m_run, l_run, o, m_lane);
-                store_state_lanes<D, G>(sm, kNW + warp, lane, m_run, l_run, o);
+#pragma unroll
+                for (int n = 0; n < D / 8; ++n) {
+                    sm.st_o[(warp * G + g) * D + 8 * n + 2 * c] = oc[n][0];
+                    sm.st_o[(warp * G + g) * D + 8 * n + 2 * c + 1] = oc[n][1];
+                }
             }
         } else {
-            if (warp < kNW) {
-                if (ok) zoom_phase<DT, D, G>(a, sm, warp, lane, b, l, kvh, m_run, l_run, o, m_lane);
-                store_state_lanes<D, G>(sm, warp, lane, m_run, l_run, o);
-            }
+            store_state_lanes<D, G>(sm, warp, lane, m_run, l_run, o);
         }
     }
     __syncthreads();
