@@ -65,8 +65,8 @@ struct DecCfg {
     // on the tensor-core path, one for its zoomed spans
     static constexpr int NSTATE = kNW;
     static constexpr int SBYTES = NSTATE * (G * D + 2 * G) * 4;
-    // tensor-core zoom scratch per warp: u^T and (beta y)^T as hi/lo bf16 [2][8][72], p^T [8][24]
-    static constexpr int ZSCR = 5120;
+    // tensor-core zoom scratch per warp: u^T and (beta y)^T as hi/lo bf16 [2][8][72], p^T [8][72]
+    static constexpr int ZSCR = 5888;
     static constexpr int RING0 = NS * STAGE;
     static constexpr int RING1 = ZBYTES + (MMA ? kNW * ZSCR : 0) > SBYTES ? ZBYTES + (MMA ? kNW * ZSCR : 0) : SBYTES;
     static constexpr int RING = RING0 > RING1 ? RING0 : RING1;
@@ -525,7 +525,7 @@ SEKV_DEV void zoom_phase_mma(const DecArgs& a, const DecSmem& sm, int warp, int 
     uint64_t* zb = sm.zbar + warp * C::ZNS;
     __nv_bfloat16* ut = reinterpret_cast<__nv_bfloat16*>(sm.stages + C::ZBYTES + warp * C::ZSCR);  // [2][8][72]
     __nv_bfloat16* yt = ut + 2 * 8 * 72;                                                        // [2][8][72]
-    __nv_bfloat16* pt = yt + 2 * 8 * 72;                                                        // [8][24]
+    __nv_bfloat16* pt = yt + 2 * 8 * 72;                                                        // [8][72]
 
     auto grab = [&]() -> ZSpan {
         ZSpan sp;
@@ -579,8 +579,14 @@ SEKV_DEV void zoom_phase_mma(const DecArgs& a, const DecSmem& sm, int warp, int 
     uint32_t nis = 0, ncons = 0;
     bool zok = true;
 
+    // slots start zeroed, so bytes past a copy are always finite
+    for (int i = lane; i < C::ZNS * C::ZSLOT / 16; i += 32)
+        reinterpret_cast<uint4*>(zring)[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncwarp();
+    fence_proxy_async();
+
     auto issue = [&]() {
-        fence_proxy_async();
+        if (nis - ncons < (uint32_t)C::ZNS) fence_proxy_async();
         while (nis - ncons < (uint32_t)C::ZNS) {
             if (!i_next && i_k >= nslots(cur)) {
                 if (!cur.valid) break;
@@ -665,88 +671,126 @@ SEKV_DEV void zoom_phase_mma(const DecArgs& a, const DecSmem& sm, int warp, int 
                     }
                 }
             } else if (k < cur.nB + cur.nAC) {
-                // (2) scores s = A u, span-local online softmax, y += C^T p, 16 tokens at a time
+                // (2) scores s = A u for up to 64 tokens (four 16-token sub-chunks),
+                //     span-local online softmax, y += C^T p
                 __syncwarp();
                 const int t0 = (k - cur.nB) * cur.TC;
                 const int nt = min(cur.TC, cur.len - t0);
-                const uint16_t* A16 = reinterpret_cast<const uint16_t*>(zs);
-                const uint16_t* C16 = reinterpret_cast<const uint16_t*>(zs + C::ZSLOT / 2);
-                for (int ts = 0; ts < nt; ts += 16) {
-                    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-                    for (int ks = 0; ks < nig; ++ks) {
-                        uint32_t af[4];
+                const int nsc = (nt + 15) >> 4;
+                const unsigned char* As = zs;
+                const unsigned char* Cs = zs + C::ZSLOT / 2;
+                const uint16_t* A16 = reinterpret_cast<const uint16_t*>(As);
+                const uint16_t* C16 = reinterpret_cast<const uint16_t*>(Cs);
+                const bool vec = (rS & 7) == 0;            // 16-byte rows: ldmatrix
+                float sacc[4][4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int t = ts + gid + ((e & 1) << 3);
-                            const int i = 16 * ks + 2 * cq + ((e >> 1) << 3);
-                            const uint32_t x0 = (t < nt && i < rS) ? A16[t * rS + i] : 0u;
-                            const uint32_t x1 = (t < nt && i + 1 < rS) ? A16[t * rS + i + 1] : 0u;
-                            af[e] = x0 | (x1 << 16);
+                for (int sc = 0; sc < 4; ++sc) {
+                    sacc[sc][0] = sacc[sc][1] = sacc[sc][2] = sacc[sc][3] = 0.f;
+                    if (sc < nsc) {
+                        const int ts = 16 * sc;
+                        for (int ks = 0; ks < nig; ++ks) {
+                            uint32_t af[4];
+                            if (vec) {
+                                const int arow = ts + (lane & 7) + (((lane >> 3) & 1) << 3);
+                                ldsm_x4(af, As + ((int64_t)arow * rS + 16 * ks + ((lane >> 4) << 3)) * 2);
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int t = ts + gid + ((e & 1) << 3);
+                                    const int i = 16 * ks + 2 * cq + ((e >> 1) << 3);
+                                    const uint32_t x0 = (t < nt && i < rS) ? A16[t * rS + i] : 0u;
+                                    const uint32_t x1 = (t < nt && i + 1 < rS) ? A16[t * rS + i + 1] : 0u;
+                                    af[e] = x0 | (x1 << 16);
+                                }
+                            }
+                            const uint32_t* uh = reinterpret_cast<const uint32_t*>(ut + gid * 72 + 16 * ks + 2 * cq);
+                            const uint32_t* ul = reinterpret_cast<const uint32_t*>(ut + (8 + gid) * 72 + 16 * ks + 2 * cq);
+                            const uint32_t bh[2] = {uh[0], uh[4]};
+                            const uint32_t bl[2] = {ul[0], ul[4]};
+                            mma_bf16_16816(sacc[sc], af, bh);
+                            mma_bf16_16816(sacc[sc], af, bl);
                         }
-                        const uint32_t* uh = reinterpret_cast<const uint32_t*>(ut + gid * 72 + 16 * ks + 2 * cq);
-                        const uint32_t* ul = reinterpret_cast<const uint32_t*>(ut + (8 + gid) * 72 + 16 * ks + 2 * cq);
-                        const uint32_t bh[2] = {uh[0], uh[4]};
-                        const uint32_t bl[2] = {ul[0], ul[4]};
-                        mma_bf16_16816(sacc, af, bh);
-                        mma_bf16_16816(sacc, af, bl);
                     }
-                    // sacc[e]: token ts + gid + 8*(e>>1), head 2cq + (e&1)
-                    float lg[4], p[4];
+                }
+                // sacc[sc][e]: token 16 sc + gid + 8 (e >> 1), head 2 cq + (e & 1)
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int sc = 0; sc < 4; ++sc)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int t = ts + gid + ((e >> 1) << 3);
+                        const int t = 16 * sc + gid + ((e >> 1) << 3);
                         const int h = 2 * cq + (e & 1);
-                        lg[e] = (t < nt && h < G && ((cur.hm >> h) & 1u)) ? sacc[e] * sl2 : -INFINITY;
+                        const float v = (t < nt && h < G && ((cur.hm >> h) & 1u)) ? sacc[sc][e] * sl2 : -INFINITY;
+                        sacc[sc][e] = v;
+                        if (e & 1) mx1 = fmaxf(mx1, v); else mx0 = fmaxf(mx0, v);
                     }
-                    float mx0 = fmaxf(lg[0], lg[2]), mx1 = fmaxf(lg[1], lg[3]);
 #pragma unroll
-                    for (int off = 4; off < 32; off <<= 1) {
-                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                for (int off = 4; off < 32; off <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                }
+                const float mn0 = fmaxf(msp[0], mx0), mn1 = fmaxf(msp[1], mx1);
+                const float al0 = (mn0 == -INFINITY) ? 1.f : exp2f(msp[0] - mn0);
+                const float al1 = (mn1 == -INFINITY) ? 1.f : exp2f(msp[1] - mn1);
+                float ps0 = 0.f, ps1 = 0.f;
+                __syncwarp();                                   // previous reads of pt are done
+#pragma unroll
+                for (int sc = 0; sc < 4; ++sc)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float v = sacc[sc][e];
+                        const float pv = (v == -INFINITY) ? 0.f : exp2f(v - ((e & 1) ? mn1 : mn0));
+                        if (e & 1) ps1 += pv; else ps0 += pv;
+                        pt[(2 * cq + (e & 1)) * 72 + 16 * sc + gid + ((e >> 1) << 3)] = __float2bfloat16_rn(pv);
                     }
-                    const float mn0 = fmaxf(msp[0], mx0), mn1 = fmaxf(msp[1], mx1);
-                    const float al0 = (mn0 == -INFINITY) ? 1.f : exp2f(msp[0] - mn0);
-                    const float al1 = (mn1 == -INFINITY) ? 1.f : exp2f(msp[1] - mn1);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        p[e] = (lg[e] == -INFINITY) ? 0.f : exp2f(lg[e] - ((e & 1) ? mn1 : mn0));
-                    float ps0 = p[0] + p[2], ps1 = p[1] + p[3];
-#pragma unroll
-                    for (int off = 4; off < 32; off <<= 1) {
-                        ps0 += __shfl_xor_sync(0xffffffffu, ps0, off);
-                        ps1 += __shfl_xor_sync(0xffffffffu, ps1, off);
-                    }
-                    lsp[0] = fmaf(lsp[0], al0, ps0);
-                    lsp[1] = fmaf(lsp[1], al1, ps1);
-                    msp[0] = mn0;
-                    msp[1] = mn1;
-                    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
-                        for (int ig = 0; ig < 4; ++ig) {
-                            yacc[ig][0] *= al0; yacc[ig][1] *= al1;
-                            yacc[ig][2] *= al0; yacc[ig][3] *= al1;
-                        }
-                    }
-                    __syncwarp();
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        pt[(2 * cq + (e & 1)) * 24 + gid + ((e >> 1) << 3)] = __float2bfloat16_rn(p[e]);
-                    __syncwarp();
-                    const uint32_t* pp = reinterpret_cast<const uint32_t*>(pt + gid * 24 + 2 * cq);
-                    const uint32_t bp[2] = {pp[0], pp[4]};
+                for (int off = 4; off < 32; off <<= 1) {
+                    ps0 += __shfl_xor_sync(0xffffffffu, ps0, off);
+                    ps1 += __shfl_xor_sync(0xffffffffu, ps1, off);
+                }
+                lsp[0] = fmaf(lsp[0], al0, ps0);
+                lsp[1] = fmaf(lsp[1], al1, ps1);
+                msp[0] = mn0;
+                msp[1] = mn1;
+                if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
                     for (int ig = 0; ig < 4; ++ig) {
-                        if (ig < nig) {
-                            uint32_t af[4];
+                        yacc[ig][0] *= al0; yacc[ig][1] *= al1;
+                        yacc[ig][2] *= al0; yacc[ig][3] *= al1;
+                    }
+                }
+                __syncwarp();
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int i = 16 * ig + gid + ((e & 1) << 3);
-                                const int t = ts + 2 * cq + ((e >> 1) << 3);
-                                const uint32_t x0 = (i < rS && t < nt) ? C16[t * rS + i] : 0u;
-                                const uint32_t x1 = (i < rS && t + 1 < nt) ? C16[(t + 1) * rS + i] : 0u;
-                                af[e] = x0 | (x1 << 16);
+                for (int sc = 0; sc < 4; ++sc) {
+                    if (sc < nsc) {
+                        const int ts = 16 * sc;
+                        const uint32_t* pp = reinterpret_cast<const uint32_t*>(pt + gid * 72 + ts + 2 * cq);
+                        const uint32_t bp[2] = {pp[0], pp[4]};
+                        // this lane's tokens in the C^T fragment: ts + 2cq, +1 (k 0..7) and +8
+                        const int tk = ts + 2 * cq;
+                        const uint32_t m0 = (tk < nt ? 0x0000ffffu : 0u) | (tk + 1 < nt ? 0xffff0000u : 0u);
+                        const uint32_t m1 = (tk + 8 < nt ? 0x0000ffffu : 0u) | (tk + 9 < nt ? 0xffff0000u : 0u);
+#pragma unroll
+                        for (int ig = 0; ig < 4; ++ig) {
+                            if (ig < nig) {
+                                uint32_t af[4];
+                                if (vec) {
+                                    const int mi = lane >> 3;
+                                    const int trow = ts + (lane & 7) + ((mi >> 1) << 3);
+                                    ldsm_x4_t(af, Cs + ((int64_t)trow * rS + 16 * ig + ((mi & 1) << 3)) * 2);
+                                    af[0] &= m0; af[1] &= m0; af[2] &= m1; af[3] &= m1;
+                                } else {
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        const int i = 16 * ig + gid + ((e & 1) << 3);
+                                        const int t = ts + 2 * cq + ((e >> 1) << 3);
+                                        const uint32_t x0 = (i < rS && t < nt) ? C16[t * rS + i] : 0u;
+                                        const uint32_t x1 = (i < rS && t + 1 < nt) ? C16[(t + 1) * rS + i] : 0u;
+                                        af[e] = x0 | (x1 << 16);
+                                    }
+                                }
+                                mma_bf16_16816(yacc[ig], af, bp);
                             }
-                            mma_bf16_16816(yacc[ig], af, bp);
                         }
                     }
                 }
@@ -766,7 +810,7 @@ SEKV_DEV void zoom_phase_mma(const DecArgs& a, const DecSmem& sm, int warp, int 
                             for (int e = 0; e < 4; ++e) {
                                 const int i = 16 * ig + gid + ((e >> 1) << 3);
                                 const int h = 2 * cq + (e & 1);
-                                const float v = yacc[ig][e] * ((e & 1) ? be1 : be0);
+                                const float v = i < rS ? yacc[ig][e] * ((e & 1) ? be1 : be0) : 0.f;
                                 const __nv_bfloat16 hi = __float2bfloat16_rn(v);
                                 yt[h * 72 + i] = hi;
                                 yt[(8 + h) * 72 + i] = __float2bfloat16_rn(v - __bfloat162float(hi));

@@ -11,7 +11,8 @@ import ctypes as C
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsekv.so")
+# the in-tree build; SEKV_LIBRARY may point at another build of the same ABI
+LIB_PATH = os.environ.get("SEKV_LIBRARY") or os.path.join(_HERE, "libsekv.so")
 
 SEKV_OK = 0
 SEKV_ERR_INVALID_ARG = 1
