@@ -110,6 +110,27 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest value over all ranks (timing is reported as the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Each rank runs an independent replica of the workload (its own sequences)."""
+    return base_seed + 1000 * rank
+
+
+def throughput(world: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job steps/s: every rank completes `steps` steps in the slowest rank's time."""
+    return world * steps / (elapsed_ms * 1e-3)
+
+
 def calibrate_theta(cache, q, quantile, P, torch):
     """Per (layer, query head): theta at the target quantile of the routing logits
     of a calibration query (the learned per-head thresholds are not available)."""
@@ -257,7 +278,7 @@ def run_sekv(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     wl = build_workload(args)
-    wl = wl.scaled(seed=wl.seed + 1000 * rank)          # independent replica per rank
+    wl = wl.scaled(seed=replica_seed(wl.seed, rank))     # independent replica per rank
     G = wl.Hq // wl.Hkv
     cold = wl.basis_home == "host"
     a_cap, m_cap = caps_for(wl)
@@ -398,10 +419,7 @@ def run_sekv(args, rank, world, local_rank):
     elapsed_ms = t0.elapsed_time(t1)
     if not cold:
         zhost.append(zm.cpu().numpy())
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
     if cache.read_status() != 0:
         raise RuntimeError(f"decode status {P.sekv.sekv_status_str(cache.read_status())}")
     route_ms = [r[0].elapsed_time(r[1]) for r in recs]
@@ -414,7 +432,7 @@ def run_sekv(args, rank, world, local_rank):
     achieved = alg_bytes / (attn_avg * 1e-3) / 1e9
     zr = statistics.mean(zoom_rate(cache, zh) for zh in zhost)
     ms_per_step = elapsed_ms / steps
-    value = world * steps / (elapsed_ms * 1e-3)
+    value = throughput(world, steps, elapsed_ms)
 
     # ---- e2e through the public API with host buffers
     e2e = None
@@ -438,13 +456,9 @@ def run_sekv(args, rank, world, local_rank):
             l_h.copy_(lse, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
         qb = qpool[0].numel() * qpool[0].element_size()
-        e2e = {"value": world * steps / (e_ms * 1e-3), "unit": "steps/s",
+        e2e = {"value": throughput(world, steps, e_ms), "unit": "steps/s",
                "h2d_bytes_per_step": int(qb + h2d_extra / steps),
                "d2h_bytes_per_step": int(O.numel() * 4 + lse.numel() * 4),
                "note": "per step: q H2D from pinned host, ROUTE, fetch (zmask D2H, bases + slot table H2D), "
