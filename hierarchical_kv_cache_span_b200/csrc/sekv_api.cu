@@ -83,7 +83,7 @@ sekv_status check_build(const sekv_build_desc* d) {
     return SEKV_OK;
 }
 
-sekv_status check_decode(const sekv_decode_desc* d) {
+sekv_status check_decode(const sekv_decode_desc* d, bool with_workspace = true) {
     SEKV_REQUIRE(d, "decode: null descriptor");
     SEKV_REQUIRE(d->B >= 1 && d->L >= 1 && d->Hq >= 1 && d->Hkv >= 1 && d->Hq % d->Hkv == 0,
                  "decode: B, L, Hq, Hkv >= 1 and Hq a multiple of Hkv");
@@ -111,9 +111,11 @@ sekv_status check_decode(const sekv_decode_desc* d) {
         if (!d->slot)
             SEKV_REQUIRE(d->blk_off && d->region_elems > 0 && d->region_elems % 64 == 0,
                          "decode: blk_off and region_elems (multiple of 64) required without a slot table");
-        const size_t need = sekv::decode_workspace_bytes(*d);
-        SEKV_REQUIRE(d->workspace && aligned(d->workspace, 256) && (size_t)d->workspace_bytes >= need,
-                     "decode: workspace of %zu bytes (256-byte aligned) required", need);
+        if (with_workspace) {
+            const size_t need = sekv::decode_workspace_bytes(*d);
+            SEKV_REQUIRE(d->workspace && aligned(d->workspace, 256) && (size_t)d->workspace_bytes >= need,
+                         "decode: workspace of %zu bytes (256-byte aligned) required", need);
+        }
     }
     return SEKV_OK;
 }
@@ -192,6 +194,24 @@ sekv_status sekv_decode_attn(const sekv_decode_desc* d, sekv_stream_t stream) {
     const sekv::DecodePlan p = sekv::plan_decode(*d);
     cudaError_t e = sekv::launch_decode(*d, p, d->workspace, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "decode");
+    return SEKV_OK;
+}
+
+sekv_status sekv_decode_attn_static(const sekv_decode_desc* d, sekv_stream_t stream) {
+    sekv_status s = check_decode(d, false);
+    if (s != SEKV_OK) return s;
+    const sekv::DecodePlan p = sekv::plan_decode(*d);
+    const size_t cap = sekv::decode_static_scratch_bytes();
+    if (p.partial_bytes > cap)
+        return fail(SEKV_ERR_CAPACITY,
+                    "decode_static: this call needs %zu bytes of split-K scratch, the static array holds %zu "
+                    "(fewer layers per call, a smaller batch or nsplit, or sekv_decode_attn with a workspace)",
+                    p.partial_bytes, cap);
+    cudaError_t e;
+    void* scratch = sekv::decode_static_scratch(&e);
+    if (!scratch) return cuda_fail(e, "decode_static: address of the static scratch");
+    e = sekv::launch_decode(*d, p, scratch, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode_static");
     return SEKV_OK;
 }
 

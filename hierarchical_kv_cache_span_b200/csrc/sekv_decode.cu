@@ -29,6 +29,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "sekv_common.cuh"
 #include "sekv_internal.h"
@@ -1510,6 +1511,40 @@ static cudaError_t launch_g(const sekv_decode_desc& d, const DecodePlan& p, void
         case 4: return launch_t<DT, D, 4>(d, p, w, st);
         default: return launch_t<DT, D, 8>(d, p, w, st);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Split-K partials for callers that pass no workspace: one static device array,
+// present on every device that loads this library until the process exits.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_decode_scratch[SEKV_STATIC_SCRATCH_BYTES];
+
+size_t decode_static_scratch_bytes() { return SEKV_STATIC_SCRATCH_BYTES; }
+
+// Device address of g_decode_scratch on the current device. In host code the
+// array's name only stands in for it, so the address is looked up once per
+// device (with that device current) and cached.
+void* decode_static_scratch(cudaError_t* err) {
+    static std::mutex mu;
+    static void* addr[256] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 256) {
+        *err = e != cudaSuccess ? e : cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+        if (e != cudaSuccess || !ptr) {
+            *err = e != cudaSuccess ? e : cudaErrorInvalidSymbol;
+            return nullptr;
+        }
+        addr[dev] = ptr;
+    }
+    *err = cudaSuccess;
+    return addr[dev];
 }
 
 cudaError_t launch_decode(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st) {

@@ -80,6 +80,7 @@ _SIGS = {
     "sekv_build_spans": (_i32, [C.POINTER(sekv_build_desc), _p]),
     "sekv_decode_workspace_bytes": (C.c_size_t, [C.POINTER(sekv_decode_desc)]),
     "sekv_decode_attn": (_i32, [C.POINTER(sekv_decode_desc), _p]),
+    "sekv_decode_attn_static": (_i32, [C.POINTER(sekv_decode_desc), _p]),
     "sekv_fetch_bases": (_i32, [C.POINTER(sekv_fetch_desc), _p, _p, _p]),
     "sekv_status_str": (C.c_char_p, [_i32]),
     "sekv_last_error": (C.c_char_p, []),
@@ -141,6 +142,13 @@ def sekv_decode_workspace_bytes(desc: sekv_decode_desc) -> int:
 
 def sekv_decode_attn(desc: sekv_decode_desc, stream: int = 0) -> int:
     return int(_lib.sekv_decode_attn(C.byref(desc), C.c_void_p(stream or None)))
+
+
+def sekv_decode_attn_static(desc: sekv_decode_desc, stream: int = 0) -> int:
+    return int(_lib.sekv_decode_attn_static(C.byref(desc), C.c_void_p(stream or None)))
+
+
+SEKV_STATIC_SCRATCH_BYTES = 8 << 20
 
 
 def sekv_fetch_bases(desc: sekv_fetch_desc, compute: int, copy: int, done: int) -> int:

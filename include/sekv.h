@@ -199,6 +199,30 @@ size_t sekv_decode_workspace_bytes(const sekv_decode_desc* desc);
  * weighted D_S rows), all in one softmax. */
 sekv_status sekv_decode_attn(const sekv_decode_desc* desc, sekv_stream_t stream);
 
+/*
+ * Decode without a workspace. The SeKV pages have no counterpart: this entry
+ * point exists for callers that cannot allocate device memory on the decode
+ * path - for example a serving loop that runs inside a memory pool it does not
+ * own, a plugin whose host framework forbids allocations after start-up, or code
+ * that must not call cudaMalloc because cudaMalloc can synchronize the device.
+ * Same contract as sekv_decode_attn, except that desc->workspace and
+ * desc->workspace_bytes are ignored: the split-K partials go to one static
+ * device array of SEKV_STATIC_SCRATCH_BYTES that every device which loads the
+ * library holds until the process exits.
+ *   - A call whose partials (sekv_decode_workspace_bytes) exceed the array is
+ *     rejected with SEKV_ERR_CAPACITY and launches nothing.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called. The first
+ *     call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current) and caches it: make that first call before any
+ *     stream capture.
+ *   - Every call uses the same array, which keeps the last call's contents; each
+ *     call writes all the scratch it reads, so nothing has to start at zero.
+ *     Calls whose kernels can overlap on the GPU (different streams without an
+ *     ordering between them) race on the array.
+ */
+#define SEKV_STATIC_SCRATCH_BYTES (8u << 20)
+sekv_status sekv_decode_attn_static(const sekv_decode_desc* desc, sekv_stream_t stream);
+
 /* ------------------------------------------------------------------------- */
 /* Cold-basis fetch (SeKV summary: zoomed spans' bases fetched from the CPU;  */
 /* SeKV blog Fig. 2)                                                          */
