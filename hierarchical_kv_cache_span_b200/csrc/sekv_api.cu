@@ -157,7 +157,9 @@ int64_t sekv_block_elems(int32_t len, int32_t d, int32_t rank) {
 }
 
 int64_t sekv_basis_region_bound(int32_t n, int32_t m_cap, int32_t Hkv, int32_t d, int32_t rank) {
-    const int64_t per = 2LL * n * rank + (int64_t)m_cap * (2LL * rank * d + 80);
+    // per span: 2 len8 r8 + 2 r8 d with len8 <= |S| + 7 and r8 <= min(roundup(rank, 8), d)
+    const int64_t r8 = std::min<int64_t>(sekv::round_up(rank, 8), d);
+    const int64_t per = 2 * r8 * n + (int64_t)m_cap * (14 * r8 + 2 * r8 * d);
     return sekv::round_up((int64_t)Hkv * per, 64);
 }
 

@@ -280,6 +280,7 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
         const int N = min(len, d);
         const int Ne = N + (N & 1);
         const int rS = block_rank(len, d, a.rank);
+        const int r8 = round8(rS);
         const int64_t pa = block_ac_elems(len, rS);
         const bool rows_form = len <= d;            // G = X X^T
         const char* src = reinterpret_cast<const char*>(which ? a.V : a.K) +
@@ -287,8 +288,8 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
         char* blk = reinterpret_cast<char*>(a.home) +
                     (((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S] +
                      (int64_t)kvh * block_elems(len, d, a.rank)) * E::bytes;
-        char* fac_row = blk + (which ? pa : 0) * E::bytes;              // A or C: len x rS
-        char* fac_col = blk + (2 * pa + (which ? (int64_t)rS * d : 0)) * E::bytes;  // B or D: rS x d
+        char* fac_row = blk + (which ? pa : 0) * E::bytes;              // A or C: len8 x r8, 8x8-blocked
+        char* fac_col = blk + (2 * pa + (which ? (int64_t)r8 * d : 0)) * E::bytes;  // B or D: r8 x d, 8x8-blocked
 
         // ---- Gram ---------------------------------------------------------------
         const int Mp = (N + 15) & ~15;              // padded for the MMA tiles
@@ -361,20 +362,20 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
             // A[t][j] = U[t][sel j];  B[j][k] = sum_t U[t][sel j] X[t][k]
             for (int i = tid; i < len * rS; i += T) {
                 const int t = i / rS, j = i % rS;
-                store1<DT>(fac_row, i, Vm[t * ld + sel[j]]);
+                store1<DT>(fac_row, tile8_index(t, j, r8), Vm[t * ld + sel[j]]);
             }
             for (int i = tid; i < rS * d; i += T) {
                 const int j = i / d, k = i % d;
                 const int cj = sel[j];
                 float acc = 0.f;
                 for (int t = 0; t < len; ++t) acc = fmaf(Vm[t * ld + cj], xs(t, k), acc);
-                store1<DT>(fac_col, i, acc);
+                store1<DT>(fac_col, tile8_index(j, k, d), acc);
             }
         } else {
             // B[j][k] = V[k][sel j];  A[t][j] = sum_k X[t][k] V[k][sel j]
             for (int i = tid; i < rS * d; i += T) {
                 const int j = i / d, k = i % d;
-                store1<DT>(fac_col, i, Vm[k * ld + sel[j]]);
+                store1<DT>(fac_col, tile8_index(j, k, d), Vm[k * ld + sel[j]]);
             }
             for (int t0 = 0; t0 < len; t0 += kChunkRows) {
                 const int rows = min(kChunkRows, len - t0);
@@ -389,12 +390,18 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
                     const int cj = sel[j];
                     float acc = 0.f;
                     for (int k = 0; k < d; ++k) acc = fmaf(xs(r, k), Vm[k * ld + cj], acc);
-                    store1<DT>(fac_row, (int64_t)(t0 + r) * rS + j, acc);
+                    store1<DT>(fac_row, tile8_index(t0 + r, j, r8), acc);
                 }
             }
         }
-        // zero the A/C padding so the block is fully defined
-        for (int i = len * rS + tid; i < pa; i += T) store1<DT>(fac_row, i, 0.f);
+        // zero the padding (token rows >= |S|, columns >= rS of A / C; rows >= rS of
+        // B / D) so the block is fully defined
+        const int len8 = round8(len);
+        for (int i = tid; i < len8 * r8; i += T) {
+            const int t = i / r8, j = i % r8;
+            if (t >= len || j >= rS) store1<DT>(fac_row, tile8_index(t, j, r8), 0.f);
+        }
+        for (int i = rS * d + tid; i < r8 * d; i += T) store1<DT>(fac_col, tile8_index(i / d, i % d, d), 0.f);
         __syncthreads();
     }
 }

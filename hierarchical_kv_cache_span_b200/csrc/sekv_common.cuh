@@ -89,16 +89,28 @@ SEKV_DEV void set_status(int32_t* st, int code) {
 
 // ---------------------------------------------------------------------------
 // basis block layout (must match sekv_block_elems on the host)
+//   block = [ A | C | B | D ], every factor stored 8x8-blocked: an R x W matrix
+//   (R, W padded with zeros to multiples of 8) is a row-major grid of 8 x 8 tiles,
+//   each tile 64 contiguous elements, row-major inside. A and C are len8 x r8,
+//   B and D are r8 x d, with len8 = roundup(|S|, 8), r8 = roundup(rS, 8).
 // ---------------------------------------------------------------------------
 __host__ __device__ __forceinline__ int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 __host__ __device__ __forceinline__ int block_rank(int len, int d, int rank) {
     int r = rank < len ? rank : len;
     return r < d ? r : d;
 }
-__host__ __device__ __forceinline__ int64_t block_ac_elems(int len, int rS) { return round_up((int64_t)len * rS, 8); }
+__host__ __device__ __forceinline__ int round8(int x) { return (x + 7) & ~7; }
+// elements of the A (and of the C) section
+__host__ __device__ __forceinline__ int64_t block_ac_elems(int len, int rS) {
+    return (int64_t)round8(len) * round8(rS);
+}
 __host__ __device__ __forceinline__ int64_t block_elems(int len, int d, int rank) {
-    int rS = block_rank(len, d, rank);
-    return round_up(2 * block_ac_elems(len, rS) + 2 * (int64_t)rS * d, 64);
+    const int rS = block_rank(len, d, rank);
+    return 2 * block_ac_elems(len, rS) + 2 * (int64_t)round8(rS) * d;
+}
+// position of element (r, c) of an 8x8-blocked matrix whose padded width is w8
+__host__ __device__ __forceinline__ int64_t tile8_index(int64_t r, int c, int w8) {
+    return ((r >> 3) * (w8 >> 3) + (c >> 3)) * 64 + ((r & 7) << 3) + (c & 7);
 }
 
 // ---------------------------------------------------------------------------
@@ -149,6 +161,19 @@ SEKV_DEV void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uin
 // ---------------------------------------------------------------------------
 // warp-level tensor-core helpers (ldmatrix + mma.sync m16n8k16 bf16 -> fp32)
 // ---------------------------------------------------------------------------
+// explicit shared-memory loads (a generic load of shared memory is slower)
+SEKV_DEV uint32_t lds_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
+    return v;
+}
+SEKV_DEV uint4 lds_u128(const void* p) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
+    return v;
+}
+SEKV_DEV float lds_f32(const void* p) { return __uint_as_float(lds_u32(p)); }
+
 SEKV_DEV void ldsm_x4(uint32_t (&r)[4], const void* p) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_u32(p)));

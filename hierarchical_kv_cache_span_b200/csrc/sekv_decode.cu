@@ -20,11 +20,14 @@
 //   fp32: 1-D bulk copies and CUDA-core dot products (each lane owns d/32 dims,
 //         a 32-way transpose-reduce finishes the dots).
 // Spans zoomed by any head of the group are queued. Phase 2 attends them without
-// materialising K_S: each consumer warp pulls spans from the queue and streams
-// B_S rows, A_S/C_S token chunks and D_S rows through its own 3-slot ring:
-// u = B_S q, scores A_S u, y = C_S^T p, contribution y^T D_S. Softmax state is
-// kept in the log2 domain; the CTA merges its warps' states, a second small
-// kernel merges the splits by log-sum-exp.
+// materialising K_S (u = B_S q, scores A_S u, y = C_S^T p, contribution y^T D_S):
+//   bf16: the producer warp streams each queued span's factor pieces through one
+//         CTA-wide ring; the four consumer warps share every span, 16 tokens at a
+//         time, on the tensor cores with u, p and y held in registers.
+//   fp32: each consumer warp pulls whole spans and streams them through its own
+//         3-slot ring, on the CUDA cores.
+// Softmax state is kept in the log2 domain; the CTA merges its warps' states, a
+// second small kernel merges the splits by log-sum-exp.
 #include <cuda.h>
 
 #include <cmath>
@@ -55,21 +58,25 @@ struct DecCfg {
     static constexpr int STAGE = MMA ? (STAGE0 + 1023) / 1024 * 1024 : STAGE0;
     static constexpr int NS0 = (MMA ? 68 * 1024 : 64 * 1024) / STAGE;     // 2 CTAs / SM on the bf16 path
     static constexpr int NS = NS0 < 2 ? 2 : (NS0 > 6 ? 6 : NS0);   // ring depth
-    static constexpr int YPL = kRMax * G / 32;              // y entries per lane (zoom)
+    static constexpr int YPL = kRMax * G / 32;              // y entries per lane (fp32 zoom)
     static constexpr int WSCR = MMA ? 0 : (64 * G) + 2 * kRMax * G;   // per-warp scratch floats (fp32 zoom)
-    // zoom phase: per-warp ring of ZNS slots of ZSLOT bytes, carved from the stage ring
+    // fp32 zoom phase: per-warp ring of ZNS slots of ZSLOT bytes, carved from the stage ring
     static constexpr int ZNS = 3;
     static constexpr int ZSLOT = 4096;
-    static constexpr int RB = ZSLOT / ROWB;                 // B / D rows per slot
+    static constexpr int RB = ZSLOT / ROWB;                 // B / D rows per slot (a multiple of 8)
     static constexpr int ZBYTES = kNW * ZNS * ZSLOT;
-    // partial softmax states merged at the end: per warp one for the stream and,
-    // on the tensor-core path, one for its zoomed spans
+    // tensor-core zoom phase: one CTA-wide ring of ZNSC slots of ZSLOTC bytes, filled
+    // by the producer warp and read by all consumer warps
+    static constexpr int ZSLOTC = 16384;
+    static constexpr int RBC = ZSLOTC / ROWB;               // B / D rows per piece (a multiple of 16)
+    static constexpr int ZNSC0 = (NS * STAGE) / ZSLOTC;
+    static constexpr int ZNSC = ZNSC0 > 16 ? 16 : ZNSC0;
+    // partial softmax states merged at the end, one per consumer warp
     static constexpr int NSTATE = kNW;
     static constexpr int SBYTES = NSTATE * (G * D + 2 * G) * 4;
-    // tensor-core zoom scratch per warp: u^T and (beta y)^T as hi/lo bf16 [2][8][72], p^T [8][72]
-    static constexpr int ZSCR = 5888;
     static constexpr int RING0 = NS * STAGE;
-    static constexpr int RING1 = ZBYTES + (MMA ? kNW * ZSCR : 0) > SBYTES ? ZBYTES + (MMA ? kNW * ZSCR : 0) : SBYTES;
+    static constexpr int ZRING = MMA ? ZNSC * ZSLOTC : ZBYTES;
+    static constexpr int RING1 = ZRING > SBYTES ? ZRING : SBYTES;
     static constexpr int RING = RING0 > RING1 ? RING0 : RING1;
     static constexpr int HDR = 1024;                        // mbarriers + counters (keeps stages 1 KB aligned)
 };
@@ -97,7 +104,7 @@ struct DecArgs {
     float* part_ml;   // [B*Lr*Hkv][G][nsplit][2]  (max, sum) in the log2 domain
     int64_t region;
     float scale;
-    int L, l0, Lr, Hq, Hkv, a_cap, m_cap, rank, phase, nsplit, sch_max, qcap, mw;
+    int B, L, l0, Lr, Hq, Hkv, a_cap, m_cap, rank, phase, nsplit, sch_max, qcap, mw;
 };
 
 // TMA descriptors of the anchor and summary stores (bf16 path), viewed as 2-D
@@ -114,10 +121,11 @@ static size_t decode_smem_bytes(int sch_max, int qcap) {
     s += (size_t)kNW * qcap * 4;                               // zoom queues
     s += (size_t)G * (sch_max / 32) * 4;                       // zoom-mask words
     s += (size_t)kNW * C::WSCR * 4;                            // per-warp scratch
+    s = round_up(s, 16) + (size_t)G * C::ROWB;                 // the group's query rows
     return round_up(s, 128) + 1024;                            // + alignment slack
 }
 
-// A zoomed span as the zoom pipeline sees it (warp-uniform values).
+// A zoomed span as the fp32 zoom pipeline sees it (warp-uniform values).
 struct ZSpan {
     const char* blk;     // the span's block for this kv head
     int S;
@@ -127,34 +135,62 @@ struct ZSpan {
     bool valid;
 };
 
+// One piece of the tensor-core zoom stream: what a ring slot holds. Written by
+// the producer before it arms the slot's full barrier (a release), read by the
+// consumers after their wait on it (an acquire).
+enum : int { ZP_B = 0, ZP_AC = 1, ZP_D = 2, ZP_END = 3 };
+struct __align__(16) ZPiece {
+    int kind;
+    int first;           // first B (or D) piece of its span
+    int r0;              // B / D: first basis row; AC: first token (span-local, a multiple of 32)
+    int cnt;             // B / D: basis rows (a multiple of 8); AC: tokens
+    int len, rS;
+    uint32_t hm;         // query heads of the group that zoom the span
+    int rot;             // the span's 32-token unit j belongs to consumer warp (j + rot) % 4
+};
+
 // shared-memory carve-up common to both paths
 struct DecSmem {
     uint64_t* full;      // [NS]
     uint64_t* empty;     // [NS]
-    uint64_t* zbar;      // [kNW][ZNS]
+    uint64_t* zbar;      // fp32 zoom: [kNW][ZNS]
+    uint64_t* zfull;     // tensor-core zoom: [ZNSC]
+    uint64_t* zempty;    // tensor-core zoom: [ZNSC]
     int* qcnt;           // [kNW]
     int* zq_next;
+    int* sfail;          // set when any warp gave up during the stream phase
+    ZPiece* zmeta;       // tensor-core zoom: [ZNSC]
     unsigned char* stages;
     int* zq;             // [kNW][qcap]
     uint32_t* zw;        // [G][zwords]
     float* wscr;         // [kNW][WSCR]
+    unsigned char* qs;   // [G][D] query rows of the kv head's group (storage dtype)
     float* st_m;         // [NSTATE][G]   (in the ring, once the zoom phase is over)
     float* st_l;         // [NSTATE][G]
     float* st_o;         // [NSTATE][G][D]
 };
 
+// header (HDR = 1024 bytes): full @0, empty @64, zbar / zfull @128, zempty @256,
+// counters @384, zmeta @512 (tensor-core path; the fp32 path keeps its per-warp
+// p tiles there)
 template <class C, int G, int D>
 SEKV_DEV DecSmem carve_smem(unsigned char* base, int qcap, int zwords) {
     DecSmem s;
     s.full = reinterpret_cast<uint64_t*>(base);
     s.empty = s.full + 8;
     s.zbar = s.full + 16;
-    s.qcnt = reinterpret_cast<int*>(base + 256);
+    s.zfull = s.full + 16;
+    s.zempty = s.full + 32;
+    s.qcnt = reinterpret_cast<int*>(base + 384);
     s.zq_next = s.qcnt + kNW;
+    s.sfail = s.zq_next + 1;
+    s.zmeta = reinterpret_cast<ZPiece*>(base + 512);
     s.stages = base + C::HDR;
     s.zq = reinterpret_cast<int*>(s.stages + C::RING);
     s.zw = reinterpret_cast<uint32_t*>(s.zq + kNW * qcap);
     s.wscr = reinterpret_cast<float*>(s.zw + G * zwords);
+    s.qs = reinterpret_cast<unsigned char*>(
+        round_up(reinterpret_cast<uintptr_t>(s.wscr + kNW * C::WSCR), 16));
     s.st_m = reinterpret_cast<float*>(s.stages);             // written after the zoom phase
     s.st_l = s.st_m + C::NSTATE * G;
     s.st_o = s.st_l + C::NSTATE * G;
@@ -219,10 +255,10 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
             }
         }
         sp.blk = off >= 0 ? a.arena + (off + (int64_t)kvh * be) * C::ESZ : nullptr;
-        int tc = (C::ZSLOT / 2) / (sp.rS * C::ESZ);
+        int tc = (C::ZSLOT / 2) / (round8(sp.rS) * C::ESZ);
         tc = tc > 64 ? 64 : tc;
         sp.TC = (tc & ~7) < 8 ? 8 : (tc & ~7);
-        sp.nB = (sp.rS + C::RB - 1) / C::RB;
+        sp.nB = (round8(sp.rS) + C::RB - 1) / C::RB;
         sp.nAC = (sp.len + sp.TC - 1) / sp.TC;
         sp.valid = true;
         return sp;
@@ -265,15 +301,16 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
                     const bool isD = k >= snB;
                     const int j = isD ? k - snB - snAC : k;
                     const int r0 = j * C::RB;
-                    const uint32_t bytes = (uint32_t)min(C::RB, srS - r0) * C::ROWB;
-                    const char* src = sblk + (2 * spa + (isD ? (int64_t)srS * D : 0) + (int64_t)r0 * D) * C::ESZ;
+                    const int sr8 = round8(srS);
+                    const uint32_t bytes = (uint32_t)min(C::RB, sr8 - r0) * C::ROWB;
+                    const char* src = sblk + (2 * spa + (isD ? (int64_t)sr8 * D : 0) + (int64_t)r0 * D) * C::ESZ;
                     mbar_arrive_expect_tx(&zb[slot], bytes);
                     bulk_g2s(dst, src, bytes, &zb[slot]);
                 } else {
                     const int t0 = (k - snB) * sTC;
                     const int nt = min(sTC, slen - t0);
-                    const uint32_t bytes = (uint32_t)round_up((int64_t)nt * srS * C::ESZ, 16);
-                    const int64_t off = (int64_t)t0 * srS * C::ESZ;
+                    const uint32_t bytes = (uint32_t)((int64_t)round8(nt) * round8(srS) * C::ESZ);
+                    const int64_t off = (int64_t)t0 * round8(srS) * C::ESZ;
                     mbar_arrive_expect_tx(&zb[slot], 2 * bytes);
                     bulk_g2s(dst, sblk + off, bytes, &zb[slot]);
                     bulk_g2s(dst + C::ZSLOT / 2, sblk + spa * C::ESZ + off, bytes, &zb[slot]);
@@ -312,7 +349,7 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
                     for (int r = 0; r < R; ++r) {
                         float kk[DPL];
                         if (i0 + r < rows) {
-                            Vec<DT, DPL>::load(zs + (i0 + r) * C::ROWB + lane * DPL * C::ESZ, kk);
+                            Vec<DT, DPL>::load(zs + tile8_index(i0 + r, lane * DPL, D) * C::ESZ, kk);
                         } else {
 #pragma unroll
                             for (int t = 0; t < DPL; ++t) kk[t] = 0.f;
@@ -336,7 +373,7 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
                 const int nt = min(cur.TC, cur.len - t0);
                 const unsigned char* As = zs;
                 const unsigned char* Cs = zs + C::ZSLOT / 2;
-                const int rS = cur.rS;
+                const int rS = cur.rS, r8 = round8(cur.rS);
                 float xs[2][G];
 #pragma unroll
                 for (int tt = 0; tt < 2; ++tt)
@@ -349,7 +386,7 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
                         for (int tt = 0; tt < 2; ++tt) {
                             const int t = lane + 32 * tt;
                             if (t < nt) {
-                                const uint4 w = *reinterpret_cast<const uint4*>(As + ((int64_t)t * rS + i0) * 2);
+                                const uint4 w = *reinterpret_cast<const uint4*>(As + tile8_index(t, i0, r8) * 2);
                                 av[tt][0] = bf16_lo(w.x); av[tt][1] = bf16_hi(w.x);
                                 av[tt][2] = bf16_lo(w.y); av[tt][3] = bf16_hi(w.y);
                                 av[tt][4] = bf16_lo(w.z); av[tt][5] = bf16_hi(w.z);
@@ -381,7 +418,7 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
                         const int t = lane + 32 * tt;
                         if (t < nt) {
                             for (int i = 0; i < rS; ++i) {
-                                const float av = load1<DT>(As, (int64_t)t * rS + i);
+                                const float av = load1<DT>(As, tile8_index(t, i, r8));
 #pragma unroll
                                 for (int h = 0; h < G; ++h) xs[tt][h] = fmaf(av, ub[i * G + h], xs[tt][h]);
                             }
@@ -432,13 +469,13 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
                         float acc0 = y[j] * alL, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
                         int tt = 0;
                         for (; tt + 4 <= nt; tt += 4) {
-                            acc0 = fmaf(pb[(tt + 0) * G + hL], load1<DT>(Cs, (int64_t)(tt + 0) * rS + i), acc0);
-                            acc1 = fmaf(pb[(tt + 1) * G + hL], load1<DT>(Cs, (int64_t)(tt + 1) * rS + i), acc1);
-                            acc2 = fmaf(pb[(tt + 2) * G + hL], load1<DT>(Cs, (int64_t)(tt + 2) * rS + i), acc2);
-                            acc3 = fmaf(pb[(tt + 3) * G + hL], load1<DT>(Cs, (int64_t)(tt + 3) * rS + i), acc3);
+                            acc0 = fmaf(pb[(tt + 0) * G + hL], load1<DT>(Cs, tile8_index(tt + 0, i, r8)), acc0);
+                            acc1 = fmaf(pb[(tt + 1) * G + hL], load1<DT>(Cs, tile8_index(tt + 1, i, r8)), acc1);
+                            acc2 = fmaf(pb[(tt + 2) * G + hL], load1<DT>(Cs, tile8_index(tt + 2, i, r8)), acc2);
+                            acc3 = fmaf(pb[(tt + 3) * G + hL], load1<DT>(Cs, tile8_index(tt + 3, i, r8)), acc3);
                         }
                         for (; tt < nt; ++tt)
-                            acc0 = fmaf(pb[tt * G + hL], load1<DT>(Cs, (int64_t)tt * rS + i), acc0);
+                            acc0 = fmaf(pb[tt * G + hL], load1<DT>(Cs, tile8_index(tt, i, r8)), acc0);
                         y[j] = (acc0 + acc1) + (acc2 + acc3);
                     }
                 }
@@ -472,7 +509,7 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
                 const int rows = min(C::RB, cur.rS - r0);
                 for (int r = 0; r < rows; ++r) {
                     float dv[DPL];
-                    Vec<DT, DPL>::load(zs + r * C::ROWB + lane * DPL * C::ESZ, dv);
+                    Vec<DT, DPL>::load(zs + tile8_index(r, lane * DPL, D) * C::ESZ, dv);
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
                         const float yv = yb[(r0 + r) * G + h];
@@ -503,330 +540,324 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
 }
 
 // ---------------------------------------------------------------------------
-// Phase 2 on the tensor cores (bf16). Per zoomed span and the heads h that zoom
-// it, with r = rank of the span:
-//   u = B_S q          (mma: M = r basis rows, K = d, N = heads)
-//   s = A_S u          (mma: M = 16 tokens, K = r)             -> online softmax p
-//   y = C_S^T p        (mma: M = r, K = 16 tokens)
-//   O += (beta y)^T D_S (mma: M = heads, K = r, N = d)  into the stream accumulators
-// u and beta*y are rounded to bf16 as a hi + lo pair (about 16 significant bits);
-// p is rounded to bf16 as on the streaming path. The span's (max, sum) merge into
-// the warp's stream state (mm, lm, oc) for head gid = lane/4.
+// Phase 2 on the tensor cores (bf16). The producer warp walks the CTA's zoom queue
+// and streams, per zoomed span, its B rows, its A/C token groups and its D rows
+// through one CTA-wide ring of 8 KB slots; every consumer warp reads every slot.
+// Per span, with r8 = roundup(r_S, 8) and the heads h that zoom it:
+//   u^T  = q^T B_S^T    (M = heads, N = basis rows, K = d)
+//   s^T  = u^T A_S^T    (M = heads, N = 16 tokens, K = r8)   -> online softmax p
+//   y^T += p^T C_S      (M = heads, N = basis rows, K = 16 tokens)
+//   O   += (beta y)^T D_S  into the warp's stream accumulators
+// Each accumulator is the next product's A fragment, so u, p and y never leave
+// registers. The span's 16-token sub-chunks are dealt round-robin to the four
+// consumer warps (continuing across spans); a warp with no sub-chunk in a span
+// skips it. u (pre-scaled by scale * log2 e) enters as a hi + lo bf16 pair (about
+// 16 significant bits); p and beta*y are rounded to bf16 as p on the stream path.
 // ---------------------------------------------------------------------------
-template <int D, int G>
-SEKV_DEV void zoom_phase_mma(const DecArgs& a, const DecSmem& sm, int warp, int lane, int b, int l, int kvh,
-                             const uint32_t (&qa)[D / 16][2], float& mm, float& lm, float (&oc)[D / 8][4]) {
-    using C = DecCfg<SEKV_BF16, D, G>;
-    constexpr int ROWB = C::ROWB;
-    constexpr int RB = C::RB;
-    const int gid = lane >> 2, cq = lane & 3;
-    const float sl2 = a.scale * kLog2e;
-    const int nq_total = sm.qcnt[0] + sm.qcnt[1] + sm.qcnt[2] + sm.qcnt[3];
-    unsigned char* zring = sm.stages + (size_t)warp * C::ZNS * C::ZSLOT;
-    uint64_t* zb = sm.zbar + warp * C::ZNS;
-    __nv_bfloat16* ut = reinterpret_cast<__nv_bfloat16*>(sm.stages + C::ZBYTES + warp * C::ZSCR);  // [2][8][72]
-    __nv_bfloat16* yt = ut + 2 * 8 * 72;                                                        // [2][8][72]
-    __nv_bfloat16* pt = yt + 2 * 8 * 72;                                                        // [8][72]
+// tokens of an A/C piece: both halves fit ZSLOTC / 2, a multiple of 32, at most 256
+SEKV_DEV int zoom_piece_tokens(int r8, int zslot) {
+    int t = ((zslot / 2) / (r8 * 2)) & ~31;
+    return t > 256 ? 256 : t;
+}
 
-    auto grab = [&]() -> ZSpan {
-        ZSpan sp;
-        sp.valid = false;
-        sp.blk = nullptr;
-        sp.S = 0; sp.hm = 0u; sp.len = 0; sp.rS = 1; sp.nB = 0; sp.nAC = 0; sp.TC = 8; sp.pa = 0;
-        int e = 0;
-        if (lane == 0) e = atomicAdd(sm.zq_next, 1);
-        e = __shfl_sync(0xffffffffu, e, 0);
-        if (e >= nq_total) return sp;
-        int w = 0;
-        while (w < kNW - 1 && e >= sm.qcnt[w]) { e -= sm.qcnt[w]; ++w; }
-        const int ent = sm.zq[w * a.qcap + e];
-        sp.S = ent & 0xffffff;
-        sp.hm = (uint32_t)ent >> 24;
-        const int beg = a.span_beg[(int64_t)b * a.m_cap + sp.S];
-        sp.len = a.span_end[(int64_t)b * a.m_cap + sp.S] - beg;
-        if (sp.len < 1) {
-            set_status(a.status, SEKV_ERR_INVALID_ARG);
-            sp.len = 0;
+template <int D, int G>
+SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b, int l, int kvh, int nq) {
+    using C = DecCfg<SEKV_BF16, D, G>;
+    constexpr int ZNS = C::ZNSC, ZSL = C::ZSLOTC, RBC = C::RBC;
+    uint32_t np = 0;          // pieces armed
+    bool good = true;
+    int rot = 0;
+    // the slots were last read through the generic proxy (stream phase)
+    fence_proxy_async();
+    // arm the next slot with piece pc and up to two bulk copies (lane 0 issues)
+    auto emit = [&](const ZPiece& pc, const char* src0, uint32_t n0, const char* src1, uint32_t n1) {
+        int okk = 1;
+        if (lane == 0) {
+            const int slot = (int)(np % ZNS);
+            if (np >= (uint32_t)ZNS && !mbar_wait(&sm.zempty[slot], ((np / ZNS) - 1) & 1)) okk = 0;
+            if (okk) {
+                sm.zmeta[slot] = pc;
+                unsigned char* dst = sm.stages + (size_t)slot * ZSL;
+                if (n0 + n1 == 0) {
+                    mbar_arrive(&sm.zfull[slot]);
+                } else {
+                    mbar_arrive_expect_tx(&sm.zfull[slot], n0 + n1);
+                    if (n0) bulk_g2s(dst, src0, n0, &sm.zfull[slot]);
+                    if (n1) bulk_g2s(dst + ZSL / 2, src1, n1, &sm.zfull[slot]);
+                }
+            } else {
+                set_status(a.status, SEKV_ERR_TIMEOUT);
+            }
         }
-        sp.rS = sp.len > 0 ? block_rank(sp.len, D, a.rank) : 1;
-        sp.pa = block_ac_elems(sp.len, sp.rS);
-        const int64_t be = block_elems(sp.len > 0 ? sp.len : 1, D, a.rank);
-        int64_t off = -1;
-        if (sp.len > 0) {
-            if (a.slot) {
-                off = a.slot[((int64_t)b * a.L + l) * a.m_cap + sp.S];
+        okk = __shfl_sync(0xffffffffu, okk, 0);
+        if (okk) ++np;
+        good = good && okk;
+    };
+    for (int e0 = 0; e0 < nq && good; e0 += 32) {
+        // lane j resolves queue entry e0 + j: span, zooming heads, block offset
+        int len = 0;
+        uint32_t hm = 0u;
+        long long off = -1;
+        const int e = e0 + lane;
+        if (e < nq) {
+            int w = 0, x = e;
+            while (w < kNW - 1 && x >= sm.qcnt[w]) { x -= sm.qcnt[w]; ++w; }
+            const int ent = sm.zq[w * a.qcap + x];
+            const int S = ent & 0xffffff;
+            hm = (uint32_t)ent >> 24;
+            const int beg = a.span_beg[(int64_t)b * a.m_cap + S];
+            len = a.span_end[(int64_t)b * a.m_cap + S] - beg;
+            if (len < 1) {
+                set_status(a.status, SEKV_ERR_INVALID_ARG);
+                len = 0;
+            } else if (a.slot) {
+                off = a.slot[((int64_t)b * a.L + l) * a.m_cap + S];
                 if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
             } else {
-                off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + sp.S];
+                off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S];
             }
         }
-        sp.blk = off >= 0 ? a.arena + (off + (int64_t)kvh * be) * 2 : nullptr;
-        int tc = (C::ZSLOT / 2) / (sp.rS * 2);
-        tc = tc > 64 ? 64 : tc;
-        sp.TC = (tc & ~7) < 8 ? 8 : (tc & ~7);
-        sp.nB = (sp.rS + RB - 1) / RB;
-        sp.nAC = (sp.len + sp.TC - 1) / sp.TC;
-        sp.valid = true;
-        return sp;
-    };
-    auto nslots = [](const ZSpan& sp) { return sp.blk ? 2 * sp.nB + sp.nAC : 0; };
-
-    ZSpan cur = grab(), nxt;
-    nxt.valid = false;
-    nxt.blk = nullptr;
-    nxt.nB = nxt.nAC = 0;
-    bool i_next = false;
-    int i_k = 0;
-    uint32_t nis = 0, ncons = 0;
-    bool zok = true;
-
-    // slots start zeroed, so bytes past a copy are always finite
-    for (int i = lane; i < C::ZNS * C::ZSLOT / 16; i += 32)
-        reinterpret_cast<uint4*>(zring)[i] = make_uint4(0u, 0u, 0u, 0u);
-    __syncwarp();
-    fence_proxy_async();
-
-    auto issue = [&]() {
-        if (nis - ncons < (uint32_t)C::ZNS) fence_proxy_async();
-        while (nis - ncons < (uint32_t)C::ZNS) {
-            if (!i_next && i_k >= nslots(cur)) {
-                if (!cur.valid) break;
-                nxt = grab();
-                i_next = true;
-                i_k = 0;
+        const int cnt = min(32, nq - e0);
+        for (int j = 0; j < cnt && good; ++j) {
+            const int jl = __shfl_sync(0xffffffffu, len, j);
+            const uint32_t jhm = __shfl_sync(0xffffffffu, hm, j);
+            const long long jo = __shfl_sync(0xffffffffu, off, j);
+            if (jl < 1 || jo < 0) continue;
+            const int rS = block_rank(jl, D, a.rank), r8 = round8(rS);
+            const int64_t pa = block_ac_elems(jl, rS);
+            const int64_t be = 2 * pa + 2 * (int64_t)r8 * D;
+            const char* blk = a.arena + ((int64_t)jo + (int64_t)kvh * be) * 2;
+            const int tcz = zoom_piece_tokens(r8, ZSL);
+            ZPiece pc;
+            pc.len = jl;
+            pc.rS = rS;
+            pc.hm = jhm;
+            pc.rot = rot;
+            for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
+                pc.kind = ZP_B; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
+                emit(pc, blk + (2 * pa + (int64_t)r0 * D) * 2, (uint32_t)pc.cnt * C::ROWB, nullptr, 0u);
             }
-            const bool sv = i_next ? nxt.valid : cur.valid;
-            const char* sblk = i_next ? nxt.blk : cur.blk;
-            const int snB = i_next ? nxt.nB : cur.nB, snAC = i_next ? nxt.nAC : cur.nAC;
-            const int srS = i_next ? nxt.rS : cur.rS, slen = i_next ? nxt.len : cur.len;
-            const int sTC = i_next ? nxt.TC : cur.TC;
-            const int64_t spa = i_next ? nxt.pa : cur.pa;
-            if (!sv || !sblk || i_k >= 2 * snB + snAC) break;
-            const int slot = nis % C::ZNS;
-            unsigned char* dst = zring + slot * C::ZSLOT;
-            if (lane == 0) {
-                const int k = i_k;
-                if (k < snB || k >= snB + snAC) {
-                    const bool isD = k >= snB;
-                    const int j = isD ? k - snB - snAC : k;
-                    const int r0 = j * RB;
-                    const uint32_t bytes = (uint32_t)min(RB, srS - r0) * ROWB;
-                    const char* src = sblk + (2 * spa + (isD ? (int64_t)srS * D : 0) + (int64_t)r0 * D) * 2;
-                    mbar_arrive_expect_tx(&zb[slot], bytes);
-                    bulk_g2s(dst, src, bytes, &zb[slot]);
-                } else {
-                    const int t0 = (k - snB) * sTC;
-                    const int nt = min(sTC, slen - t0);
-                    const uint32_t bytes = (uint32_t)round_up((int64_t)nt * srS * 2, 16);
-                    const int64_t off = (int64_t)t0 * srS * 2;
-                    mbar_arrive_expect_tx(&zb[slot], 2 * bytes);
-                    bulk_g2s(dst, sblk + off, bytes, &zb[slot]);
-                    bulk_g2s(dst + C::ZSLOT / 2, sblk + spa * 2 + off, bytes, &zb[slot]);
-                }
+            for (int t0 = 0; t0 < jl && good; t0 += tcz) {
+                pc.kind = ZP_AC; pc.first = t0 == 0; pc.r0 = t0; pc.cnt = min(tcz, jl - t0);
+                const uint32_t nb = (uint32_t)round8(pc.cnt) * r8 * 2;
+                const int64_t to = (int64_t)t0 * r8 * 2;
+                emit(pc, blk + to, nb, blk + pa * 2 + to, nb);
             }
-            ++i_k;
-            ++nis;
+            for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
+                pc.kind = ZP_D; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
+                emit(pc, blk + (2 * pa + (int64_t)r8 * D + (int64_t)r0 * D) * 2, (uint32_t)pc.cnt * C::ROWB,
+                     nullptr, 0u);
+            }
+            rot = (rot + ((jl + 31) >> 5)) & 3;
         }
-    };
+    }
+    if (good) {
+        ZPiece pc;
+        pc.kind = ZP_END; pc.first = 0; pc.r0 = 0; pc.cnt = 0; pc.len = 0; pc.rS = 0; pc.hm = 0u; pc.rot = 0;
+        emit(pc, nullptr, 0u, nullptr, 0u);
+    }
+    // every copy this warp started has landed before the CTA moves on (the full
+    // barrier of a slot is re-armed only by this warp, so its last phase is stable)
+    if (lane == 0) {
+        const uint32_t lo = np > (uint32_t)ZNS ? np - ZNS : 0u;
+        for (uint32_t i = lo; i < np; ++i)
+            if (!mbar_wait(&sm.zfull[i % ZNS], (i / ZNS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
+    }
+}
 
-    while (cur.valid && zok) {
-        const int total = nslots(cur);
-        const int rS = cur.rS;
-        const int nig = (rS + 15) >> 4;                 // groups of 16 basis rows
-        float msp[2] = {-INFINITY, -INFINITY}, lsp[2] = {0.f, 0.f};   // heads 2cq, 2cq+1
-        float yacc[4][4];
+// split v0, v1 into a hi + lo bf16x2 pair
+SEKV_DEV void split_bf16x2(float v0, float v1, uint32_t& hi, uint32_t& lo) {
+    hi = pack_bf16(v0, v1);
+    lo = pack_bf16(v0 - bf16_lo(hi), v1 - bf16_hi(hi));
+}
+
+// hardware 2^x (ex2.approx.ftz: relative error ~2^-22; 2^-inf = 0)
+SEKV_DEV float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// RM: the largest basis rank this instantiation handles (16, 32 or 64), which
+// sizes the y accumulators and the unrolled basis-row loops
+template <int D, int G, int RM>
+SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int lane, const uint32_t* qrow,
+                           float& mm, float& lm, float (&oc)[D / 8][4]) {
+    using C = DecCfg<SEKV_BF16, D, G>;
+    constexpr int ZNS = C::ZNSC, ZSL = C::ZSLOTC;
+    constexpr int NIB = RM / 8;          // basis-row blocks of 8
+    constexpr int NKS = RM / 16;         // k-steps of 16 basis rows
+    constexpr int DB = D / 8;            // column blocks of 8 in B / D rows
+    const int g = lane >> 2, cq = lane & 3, mi = lane >> 3, lr = lane & 7;
+    const float sl2 = a.scale * kLog2e;
+    uint32_t uf[NKS][4];                 // u^T A fragments per k-step: hi a0, hi a2, lo a0, lo a2 (then (beta y)^T)
+    float yacc[NIB][4];                  // y^T accumulators per block of 8 basis rows
+    float msp = -INFINITY, lsp = 0.f;    // the span's (max, partial sum) for head g
+    bool mine = false, zh = false;
+    int nib = 1, rS = 1, rot = 0;
 #pragma unroll
-        for (int ig = 0; ig < 4; ++ig) yacc[ig][0] = yacc[ig][1] = yacc[ig][2] = yacc[ig][3] = 0.f;
-        for (int k = 0; k < total; ++k) {
-            issue();
-            const int slot = ncons % C::ZNS;
-            if (!mbar_wait(&zb[slot], (ncons / C::ZNS) & 1)) {
-                set_status(a.status, SEKV_ERR_TIMEOUT);
-                zok = false;
-                break;
+    for (int ks = 0; ks < NKS; ++ks) uf[ks][0] = uf[ks][1] = uf[ks][2] = uf[ks][3] = 0u;
+#pragma unroll
+    for (int j = 0; j < NIB; ++j) yacc[j][0] = yacc[j][1] = yacc[j][2] = yacc[j][3] = 0.f;
+
+    for (uint32_t k = 0;; ++k) {
+        const int slot = (int)(k % ZNS);
+        if (!mbar_wait(&sm.zfull[slot], (k / ZNS) & 1)) {
+            set_status(a.status, SEKV_ERR_TIMEOUT);
+            break;
+        }
+        ZPiece pc;
+        {
+            const uint4 w0 = lds_u128(&sm.zmeta[slot]), w1 = lds_u128(reinterpret_cast<const char*>(&sm.zmeta[slot]) + 16);
+            pc.kind = (int)w0.x; pc.first = (int)w0.y; pc.r0 = (int)w0.z; pc.cnt = (int)w0.w;
+            pc.len = (int)w1.x; pc.rS = (int)w1.y; pc.hm = w1.z; pc.rot = (int)w1.w;
+        }
+        if (pc.kind == ZP_END) break;
+        const unsigned char* zs = sm.stages + (size_t)slot * ZSL;
+        if (pc.kind == ZP_B) {
+            if (pc.first) {
+                rS = pc.rS;
+                nib = (rS + 7) >> 3;
+                rot = pc.rot;
+                mine = ((pc.len + 31) >> 5) > ((warp - rot) & 3);
+                zh = g < G && ((pc.hm >> g) & 1u);
+                msp = -INFINITY;
+                lsp = 0.f;
+#pragma unroll
+                for (int j = 0; j < NIB; ++j) yacc[j][0] = yacc[j][1] = yacc[j][2] = yacc[j][3] = 0.f;
             }
-            const unsigned char* zs = zring + slot * C::ZSLOT;
-            if (k < cur.nB) {
-                // (1) u = B q for the slot's basis rows, stored transposed as hi/lo bf16
-                const int r0 = k * RB;
-                const int rows = min(RB, rS - r0);
-                for (int g16 = 0; g16 < rows; g16 += 16) {
-                    float uacc[4] = {0.f, 0.f, 0.f, 0.f};
-                    const int arow = g16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+            if (mine) {
+                // u^T for the basis-row blocks of this piece, two blocks (one k-step) at a time
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        uint32_t af[4];
-                        ldsm_x4(af, zs + arow * ROWB + (16 * kk + ((lane >> 4) << 3)) * 2);
-                        const uint32_t bq[2] = {qa[kk][0], qa[kk][1]};
-                        mma_bf16_16816(uacc, af, bq);
+                for (int ks = 0; ks < NKS; ++ks) {
+                    if (16 * ks < pc.r0 || 16 * ks >= pc.r0 + pc.cnt) continue;
+                    const int jl = (16 * ks - pc.r0) >> 3;          // piece-local block
+                    // two partial sums per n-tile (even / odd k-steps) keep the mma chains short
+                    float u0[4] = {0.f, 0.f, 0.f, 0.f}, u1[4] = {0.f, 0.f, 0.f, 0.f};
+                    float v0[4] = {0.f, 0.f, 0.f, 0.f}, v1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int p = 0; p < D / 32; ++p) {
+                        uint32_t b0[4], b1[4];
+                        ldsm_x4(b0, zs + ((jl * DB + 4 * p + mi) * 64 + lr * 8) * 2);
+                        ldsm_x4(b1, zs + (((jl + 1) * DB + 4 * p + mi) * 64 + lr * 8) * 2);
+                        // q of head g as A fragments (rows >= G are zero): k-steps 2p, 2p + 1
+                        const uint32_t qf0[4] = {qrow ? lds_u32(qrow + 16 * p + cq) : 0u, 0u,
+                                                 qrow ? lds_u32(qrow + 16 * p + 4 + cq) : 0u, 0u};
+                        const uint32_t qf1[4] = {qrow ? lds_u32(qrow + 16 * p + 8 + cq) : 0u, 0u,
+                                                 qrow ? lds_u32(qrow + 16 * p + 12 + cq) : 0u, 0u};
+                        const uint32_t c00[2] = {b0[0], b0[1]}, c01[2] = {b0[2], b0[3]};
+                        const uint32_t c10[2] = {b1[0], b1[1]}, c11[2] = {b1[2], b1[3]};
+                        mma_bf16_16816(u0, qf0, c00);
+                        mma_bf16_16816(u1, qf0, c10);
+                        mma_bf16_16816(v0, qf1, c01);
+                        mma_bf16_16816(v1, qf1, c11);
                     }
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int il = g16 + gid + ((e >> 1) << 3);          // row within the slot
-                        const int i = r0 + il;
-                        const int h = 2 * cq + (e & 1);
-                        const float u = (il < rows) ? uacc[e] : 0.f;       // stale rows beyond r
-                        const __nv_bfloat16 hi = __float2bfloat16_rn(u);
-                        ut[h * 72 + i] = hi;
-                        ut[(8 + h) * 72 + i] = __float2bfloat16_rn(u - __bfloat162float(hi));
+                        u0[e] += v0[e];
+                        u1[e] += v1[e];
                     }
+                    // basis rows i >= r_S do not exist: exact zeros (select, not multiply)
+                    const int i0 = 16 * ks + 2 * cq;
+                    split_bf16x2(i0 < rS ? u0[0] * sl2 : 0.f, i0 + 1 < rS ? u0[1] * sl2 : 0.f, uf[ks][0], uf[ks][2]);
+                    split_bf16x2(i0 + 8 < rS ? u1[0] * sl2 : 0.f, i0 + 9 < rS ? u1[1] * sl2 : 0.f, uf[ks][1],
+                                 uf[ks][3]);
                 }
-            } else if (k < cur.nB + cur.nAC) {
-                // (2) scores s = A u for up to 64 tokens (four 16-token sub-chunks),
-                //     span-local online softmax, y += C^T p
-                __syncwarp();
-                const int t0 = (k - cur.nB) * cur.TC;
-                const int nt = min(cur.TC, cur.len - t0);
-                const int nsc = (nt + 15) >> 4;
+            }
+        } else if (pc.kind == ZP_AC) {
+            if (mine) {
                 const unsigned char* As = zs;
-                const unsigned char* Cs = zs + C::ZSLOT / 2;
-                const uint16_t* A16 = reinterpret_cast<const uint16_t*>(As);
-                const uint16_t* C16 = reinterpret_cast<const uint16_t*>(Cs);
-                const bool vec = (rS & 7) == 0;            // 16-byte rows: ldmatrix
-                float sacc[4][4];
+                const unsigned char* Cs = zs + ZSL / 2;
+                const int nv = (pc.cnt + 31) >> 5;
+                for (int v = (warp - rot - (pc.r0 >> 5)) & 3; v < nv; v += 4) {
+                    // token groups 4v .. 4v+3 of the piece; those at or past ngp were not copied
+                    const int ngp = ((pc.cnt + 7) >> 3) - 4 * v;
+                    // s^T = u^T A^T for the unit's 32 tokens (four n-tiles of 8)
+                    float sc[4][4];
 #pragma unroll
-                for (int sc = 0; sc < 4; ++sc) {
-                    sacc[sc][0] = sacc[sc][1] = sacc[sc][2] = sacc[sc][3] = 0.f;
-                    if (sc < nsc) {
-                        const int ts = 16 * sc;
-                        for (int ks = 0; ks < nig; ++ks) {
-                            uint32_t af[4];
-                            if (vec) {
-                                const int arow = ts + (lane & 7) + (((lane >> 3) & 1) << 3);
-                                ldsm_x4(af, As + ((int64_t)arow * rS + 16 * ks + ((lane >> 4) << 3)) * 2);
-                            } else {
+                    for (int n = 0; n < 4; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
 #pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int t = ts + gid + ((e & 1) << 3);
-                                    const int i = 16 * ks + 2 * cq + ((e >> 1) << 3);
-                                    const uint32_t x0 = (t < nt && i < rS) ? A16[t * rS + i] : 0u;
-                                    const uint32_t x1 = (t < nt && i + 1 < rS) ? A16[t * rS + i + 1] : 0u;
-                                    af[e] = x0 | (x1 << 16);
-                                }
-                            }
-                            const uint32_t* uh = reinterpret_cast<const uint32_t*>(ut + gid * 72 + 16 * ks + 2 * cq);
-                            const uint32_t* ul = reinterpret_cast<const uint32_t*>(ut + (8 + gid) * 72 + 16 * ks + 2 * cq);
-                            const uint32_t bh[2] = {uh[0], uh[4]};
-                            const uint32_t bl[2] = {ul[0], ul[4]};
-                            mma_bf16_16816(sacc[sc], af, bh);
-                            mma_bf16_16816(sacc[sc], af, bl);
+                    for (int ks = 0; ks < NKS; ++ks) {
+                        if (2 * ks >= nib) continue;
+                        const bool two = 2 * ks + 1 < nib;
+                        uint32_t a0[4], a1[4];
+                        ldsm_x4(a0, As + (((4 * v + (mi >> 1)) * nib + 2 * ks + (mi & 1)) * 64 + lr * 8) * 2);
+                        ldsm_x4(a1, As + (((4 * v + 2 + (mi >> 1)) * nib + 2 * ks + (mi & 1)) * 64 + lr * 8) * 2);
+                        const uint32_t b0[2] = {a0[0], two ? a0[1] : 0u}, b1[2] = {a0[2], two ? a0[3] : 0u};
+                        const uint32_t b2[2] = {a1[0], two ? a1[1] : 0u}, b3[2] = {a1[2], two ? a1[3] : 0u};
+                        const uint32_t uh[4] = {uf[ks][0], 0u, uf[ks][1], 0u};
+                        const uint32_t ul[4] = {uf[ks][2], 0u, uf[ks][3], 0u};
+                        mma_bf16_16816(sc[0], uh, b0);
+                        mma_bf16_16816(sc[1], uh, b1);
+                        mma_bf16_16816(sc[2], uh, b2);
+                        mma_bf16_16816(sc[3], uh, b3);
+                        mma_bf16_16816(sc[0], ul, b0);
+                        mma_bf16_16816(sc[1], ul, b1);
+                        mma_bf16_16816(sc[2], ul, b2);
+                        mma_bf16_16816(sc[3], ul, b3);
+                    }
+                    // the span's online softmax for head g (log2 domain; u carries the scale)
+                    const int tk = 32 * v + 2 * cq;
+                    float x[8];
+#pragma unroll
+                    for (int n = 0; n < 4; ++n) {
+                        x[2 * n] = (zh && tk + 8 * n < pc.cnt) ? sc[n][0] : -INFINITY;
+                        x[2 * n + 1] = (zh && tk + 8 * n + 1 < pc.cnt) ? sc[n][1] : -INFINITY;
+                    }
+                    float mx = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    const float mnew = fmaxf(msp, mx);
+                    const float al = (mnew == -INFINITY) ? 1.f : ex2(msp - mnew);
+                    const float mref = (mnew == -INFINITY) ? 0.f : mnew;
+                    float pv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) pv[e] = ex2(x[e] - mref);
+                    lsp = fmaf(lsp, al, ((pv[0] + pv[1]) + (pv[2] + pv[3])) + ((pv[4] + pv[5]) + (pv[6] + pv[7])));
+                    msp = mnew;
+                    if (__any_sync(0xffffffffu, al != 1.f)) {
+#pragma unroll
+                        for (int j = 0; j < NIB; ++j) {
+                            yacc[j][0] *= al;
+                            yacc[j][1] *= al;
+                        }
+                    }
+                    // y^T += p^T C (p as A fragments: k = tokens 0..15 and 16..31 of the unit)
+                    const uint32_t p0[4] = {pack_bf16(pv[0], pv[1]), 0u, pack_bf16(pv[2], pv[3]), 0u};
+                    const uint32_t p1[4] = {pack_bf16(pv[4], pv[5]), 0u, pack_bf16(pv[6], pv[7]), 0u};
+#pragma unroll
+                    for (int jp = 0; jp < NKS; ++jp) {
+                        if (2 * jp >= nib) continue;
+                        uint32_t c0[4], c1[4];
+                        ldsm_x4_t(c0, Cs + (((4 * v + (mi & 1)) * nib + 2 * jp + (mi >> 1)) * 64 + lr * 8) * 2);
+                        ldsm_x4_t(c1, Cs + (((4 * v + 2 + (mi & 1)) * nib + 2 * jp + (mi >> 1)) * 64 + lr * 8) * 2);
+                        // C rows of groups that were not copied hold stale bytes: zero them
+                        const uint32_t g1 = ngp > 1 ? 0xffffffffu : 0u, g2 = ngp > 2 ? 0xffffffffu : 0u,
+                                       g3 = ngp > 3 ? 0xffffffffu : 0u;
+                        const uint32_t e00[2] = {c0[0], c0[1] & g1}, e10[2] = {c1[0] & g2, c1[1] & g3};
+                        mma_bf16_16816(yacc[2 * jp], p0, e00);
+                        mma_bf16_16816(yacc[2 * jp], p1, e10);
+                        if (2 * jp + 1 < nib) {
+                            const uint32_t e01[2] = {c0[2], c0[3] & g1}, e11[2] = {c1[2] & g2, c1[3] & g3};
+                            mma_bf16_16816(yacc[2 * jp + 1], p0, e01);
+                            mma_bf16_16816(yacc[2 * jp + 1], p1, e11);
                         }
                     }
                 }
-                // sacc[sc][e]: token 16 sc + gid + 8 (e >> 1), head 2 cq + (e & 1)
-                float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-                for (int sc = 0; sc < 4; ++sc)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int t = 16 * sc + gid + ((e >> 1) << 3);
-                        const int h = 2 * cq + (e & 1);
-                        const float v = (t < nt && h < G && ((cur.hm >> h) & 1u)) ? sacc[sc][e] * sl2 : -INFINITY;
-                        sacc[sc][e] = v;
-                        if (e & 1) mx1 = fmaxf(mx1, v); else mx0 = fmaxf(mx0, v);
-                    }
-#pragma unroll
-                for (int off = 4; off < 32; off <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-                }
-                const float mn0 = fmaxf(msp[0], mx0), mn1 = fmaxf(msp[1], mx1);
-                const float al0 = (mn0 == -INFINITY) ? 1.f : exp2f(msp[0] - mn0);
-                const float al1 = (mn1 == -INFINITY) ? 1.f : exp2f(msp[1] - mn1);
-                float ps0 = 0.f, ps1 = 0.f;
-                __syncwarp();                                   // previous reads of pt are done
-#pragma unroll
-                for (int sc = 0; sc < 4; ++sc)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float v = sacc[sc][e];
-                        const float pv = (v == -INFINITY) ? 0.f : exp2f(v - ((e & 1) ? mn1 : mn0));
-                        if (e & 1) ps1 += pv; else ps0 += pv;
-                        pt[(2 * cq + (e & 1)) * 72 + 16 * sc + gid + ((e >> 1) << 3)] = __float2bfloat16_rn(pv);
-                    }
-#pragma unroll
-                for (int off = 4; off < 32; off <<= 1) {
-                    ps0 += __shfl_xor_sync(0xffffffffu, ps0, off);
-                    ps1 += __shfl_xor_sync(0xffffffffu, ps1, off);
-                }
-                lsp[0] = fmaf(lsp[0], al0, ps0);
-                lsp[1] = fmaf(lsp[1], al1, ps1);
-                msp[0] = mn0;
-                msp[1] = mn1;
-                if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
-                    for (int ig = 0; ig < 4; ++ig) {
-                        yacc[ig][0] *= al0; yacc[ig][1] *= al1;
-                        yacc[ig][2] *= al0; yacc[ig][3] *= al1;
-                    }
-                }
-                __syncwarp();
-#pragma unroll
-                for (int sc = 0; sc < 4; ++sc) {
-                    if (sc < nsc) {
-                        const int ts = 16 * sc;
-                        const uint32_t* pp = reinterpret_cast<const uint32_t*>(pt + gid * 72 + ts + 2 * cq);
-                        const uint32_t bp[2] = {pp[0], pp[4]};
-                        // this lane's tokens in the C^T fragment: ts + 2cq, +1 (k 0..7) and +8
-                        const int tk = ts + 2 * cq;
-                        const uint32_t m0 = (tk < nt ? 0x0000ffffu : 0u) | (tk + 1 < nt ? 0xffff0000u : 0u);
-                        const uint32_t m1 = (tk + 8 < nt ? 0x0000ffffu : 0u) | (tk + 9 < nt ? 0xffff0000u : 0u);
-#pragma unroll
-                        for (int ig = 0; ig < 4; ++ig) {
-                            if (ig < nig) {
-                                uint32_t af[4];
-                                if (vec) {
-                                    const int mi = lane >> 3;
-                                    const int trow = ts + (lane & 7) + ((mi >> 1) << 3);
-                                    ldsm_x4_t(af, Cs + ((int64_t)trow * rS + 16 * ig + ((mi & 1) << 3)) * 2);
-                                    af[0] &= m0; af[1] &= m0; af[2] &= m1; af[3] &= m1;
-                                } else {
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        const int i = 16 * ig + gid + ((e & 1) << 3);
-                                        const int t = ts + 2 * cq + ((e >> 1) << 3);
-                                        const uint32_t x0 = (i < rS && t < nt) ? C16[t * rS + i] : 0u;
-                                        const uint32_t x1 = (i < rS && t + 1 < nt) ? C16[(t + 1) * rS + i] : 0u;
-                                        af[e] = x0 | (x1 << 16);
-                                    }
-                                }
-                                mma_bf16_16816(yacc[ig], af, bp);
-                            }
-                        }
-                    }
-                }
-            } else {
-                if (k == cur.nB + cur.nAC) {
-                    // (3) merge: beta per zooming head, (beta y)^T to shared memory, stream state update
-                    const float mh0 = __shfl_sync(0xffffffffu, mm, 4 * (2 * cq));
-                    const float mh1 = __shfl_sync(0xffffffffu, mm, 4 * (2 * cq + 1));
-                    const bool z0 = 2 * cq < G && ((cur.hm >> (2 * cq)) & 1u);
-                    const bool z1 = 2 * cq + 1 < G && ((cur.hm >> (2 * cq + 1)) & 1u);
-                    const float be0 = z0 ? exp2f(msp[0] - fmaxf(mh0, msp[0])) : 0.f;
-                    const float be1 = z1 ? exp2f(msp[1] - fmaxf(mh1, msp[1])) : 0.f;
-#pragma unroll
-                    for (int ig = 0; ig < 4; ++ig) {
-                        if (ig < nig) {
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int i = 16 * ig + gid + ((e >> 1) << 3);
-                                const int h = 2 * cq + (e & 1);
-                                const float v = i < rS ? yacc[ig][e] * ((e & 1) ? be1 : be0) : 0.f;
-                                const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-                                yt[h * 72 + i] = hi;
-                                yt[(8 + h) * 72 + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
-                            }
-                        }
-                    }
-                    const int src = gid >> 1;
-                    const float ms0 = __shfl_sync(0xffffffffu, msp[0], src), ms1 = __shfl_sync(0xffffffffu, msp[1], src);
-                    const float ls0 = __shfl_sync(0xffffffffu, lsp[0], src), ls1 = __shfl_sync(0xffffffffu, lsp[1], src);
-                    const float msg = (gid & 1) ? ms1 : ms0, lsg = (gid & 1) ? ls1 : ls0;
-                    if (gid < G && ((cur.hm >> gid) & 1u)) {
-                        const float mnew = fmaxf(mm, msg);
-                        const float alpha = (mm == -INFINITY) ? 0.f : exp2f(mm - mnew);
-                        const float beta = exp2f(msg - mnew);
-                        lm = lm * alpha + lsg * beta;
+            }
+        } else {  // ZP_D
+            if (mine) {
+                if (pc.first) {
+                    // merge the span's (max, sum) into the stream state of head g; keep
+                    // (beta y)^T as hi/lo A fragments in uf (u is dead by now)
+                    lsp += __shfl_xor_sync(0xffffffffu, lsp, 1);
+                    lsp += __shfl_xor_sync(0xffffffffu, lsp, 2);
+                    float be = 0.f;
+                    if (zh && msp != -INFINITY) {
+                        const float mnew = fmaxf(mm, msp);
+                        const float alpha = (mm == -INFINITY) ? 0.f : ex2(mm - mnew);
+                        be = ex2(msp - mnew);
+                        lm = lm * alpha + lsp * be;
                         mm = mnew;
 #pragma unroll
                         for (int n = 0; n < D / 8; ++n) {
@@ -834,52 +865,36 @@ SEKV_DEV void zoom_phase_mma(const DecArgs& a, const DecSmem& sm, int warp, int 
                             oc[n][1] *= alpha;
                         }
                     }
-                    __syncwarp();
+                    // beta y in bf16 (relative 2^-9, as p on the stream path)
+#pragma unroll
+                    for (int ks = 0; ks < NKS; ++ks) {
+                        const int i0 = 16 * ks + 2 * cq;
+                        uf[ks][0] = pack_bf16(i0 < rS ? yacc[2 * ks][0] * be : 0.f, i0 + 1 < rS ? yacc[2 * ks][1] * be : 0.f);
+                        uf[ks][1] = pack_bf16(i0 + 8 < rS ? yacc[2 * ks + 1][0] * be : 0.f,
+                                              i0 + 9 < rS ? yacc[2 * ks + 1][1] * be : 0.f);
+                    }
                 }
-                // (4) O += (beta y)^T D over the slot's basis rows
-                const int r0 = (k - cur.nB - cur.nAC) * RB;
-                const int rows = min(RB, rS - r0);
-                for (int g16 = 0; g16 < rows; g16 += 16) {
-                    const int ks = (r0 + g16) >> 4;
-                    const uint32_t* yh = reinterpret_cast<const uint32_t*>(yt + gid * 72 + 16 * ks + 2 * cq);
-                    const uint32_t* yl = reinterpret_cast<const uint32_t*>(yt + (8 + gid) * 72 + 16 * ks + 2 * cq);
-                    const uint32_t ah[4] = {yh[0], 0u, yh[4], 0u};
-                    const uint32_t al[4] = {yl[0], 0u, yl[4], 0u};
-                    const int mi = lane >> 3;
-                    const int drow = g16 + (lane & 7) + ((mi & 1) << 3);
-                    // this lane's B rows (k): g16 + 2cq, +1 (b0) and +8 (b1); zero the stale ones
-                    const int k0 = g16 + 2 * cq;
-                    const uint32_t m0 = (k0 < rows ? 0x0000ffffu : 0u) | (k0 + 1 < rows ? 0xffff0000u : 0u);
-                    const uint32_t m1 = (k0 + 8 < rows ? 0x0000ffffu : 0u) | (k0 + 9 < rows ? 0xffff0000u : 0u);
+                // O += (beta y)^T D over this piece's basis-row blocks
+#pragma unroll
+                for (int ks = 0; ks < NKS; ++ks) {
+                    if (16 * ks < pc.r0 || 16 * ks >= pc.r0 + pc.cnt) continue;
+                    const int jl = (16 * ks - pc.r0) >> 3;
+                    const bool two = 16 * ks + 8 < pc.r0 + pc.cnt;
+                    const uint32_t yh[4] = {uf[ks][0], 0u, uf[ks][1], 0u};
 #pragma unroll
                     for (int qd = 0; qd < D / 16; ++qd) {
                         uint32_t vb[4];
-                        ldsm_x4_t(vb, zs + drow * ROWB + (16 * qd + ((mi >> 1) << 3)) * 2);
-                        const uint32_t b0[2] = {vb[0] & m0, vb[1] & m1};
-                        const uint32_t b1[2] = {vb[2] & m0, vb[3] & m1};
-                        mma_bf16_16816(oc[2 * qd], ah, b0);
-                        mma_bf16_16816(oc[2 * qd], al, b0);
-                        mma_bf16_16816(oc[2 * qd + 1], ah, b1);
-                        mma_bf16_16816(oc[2 * qd + 1], al, b1);
+                        ldsm_x4_t(vb, zs + (((jl + (mi & 1)) * DB + 2 * qd + (mi >> 1)) * 64 + lr * 8) * 2);
+                        const uint32_t b0[2] = {vb[0], two ? vb[1] : 0u};
+                        const uint32_t b1[2] = {vb[2], two ? vb[3] : 0u};
+                        mma_bf16_16816(oc[2 * qd], yh, b0);
+                        mma_bf16_16816(oc[2 * qd + 1], yh, b1);
                     }
                 }
             }
-            __syncwarp();
-            ++ncons;
         }
-        if (!zok) break;
-        if (i_next) {
-            cur = nxt;
-            i_next = false;
-            nxt.valid = false;
-        } else {
-            cur = grab();
-            i_k = 0;
-        }
-    }
-    while (ncons < nis) {
-        if (!mbar_wait(&zb[ncons % C::ZNS], (ncons / C::ZNS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
-        ++ncons;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.zempty[slot]);
     }
 }
 
@@ -901,7 +916,7 @@ SEKV_DEV void store_state_lanes(const DecSmem& sm, int idx, int lane, const floa
         for (int k = 0; k < DPL; ++k) sm.st_o[(idx * G + h) * D + lane * DPL + k] = o[h][k];
 }
 
-template <int DT, int D, int G>
+template <int DT, int D, int G, int RM>
 __global__ void __launch_bounds__((kNW + 1) * 32, DT == SEKV_BF16 ? 2 : 3)
 decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     using C = DecCfg<DT, D, G>;
@@ -912,9 +927,15 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     const DecSmem sm = carve_smem<C, G, D>(base, a.qcap, zwords);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int kvh = blockIdx.y;
-    const int b = blockIdx.z / a.Lr, li = blockIdx.z % a.Lr, l = a.l0 + li;
-    const int split = blockIdx.x;
+    // one CTA per (split, kv head, sequence x layer); the split index varies
+    // slowest so that whole splits are dispatched in order (the zoom work of a
+    // unit tends to cluster in some splits; the lighter CTAs then fill the tail)
+    const int nu = a.Hkv * a.B * a.Lr;
+    const int split = blockIdx.x / nu;
+    const int ur = blockIdx.x % nu;
+    const int kvh = ur % a.Hkv;
+    const int bl = ur / a.Hkv;
+    const int b = bl / a.Lr, li = bl % a.Lr, l = a.l0 + li;
     const int64_t unit = ((int64_t)b * a.L + l) * a.Hkv + kvh;            // global (b, l, kvh)
     const int64_t lunit = ((int64_t)b * a.Lr + li) * a.Hkv + kvh;         // within this launch
     const bool route_only = a.phase == SEKV_ROUTE;
@@ -939,11 +960,23 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kNW);
         }
-        for (int s = 0; s < kNW * C::ZNS; ++s) mbar_init(&sm.zbar[s], 1);
+        if constexpr (C::MMA) {
+            for (int s = 0; s < C::ZNSC; ++s) {
+                mbar_init(&sm.zfull[s], 1);
+                mbar_init(&sm.zempty[s], kNW);
+            }
+        } else {
+            for (int s = 0; s < kNW * C::ZNS; ++s) mbar_init(&sm.zbar[s], 1);
+        }
         *sm.zq_next = 0;
+        *sm.sfail = 0;
         fence_barrier_init();
     }
     for (int i = tid; i < G * zwords; i += blockDim.x) sm.zw[i] = 0u;
+    {
+        const uint4* qg = reinterpret_cast<const uint4*>(a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB);
+        for (int i = tid; i < G * C::ROWB / 16; i += blockDim.x) reinterpret_cast<uint4*>(sm.qs)[i] = qg[i];
+    }
     __syncthreads();
 
     const float sl2 = a.scale * kLog2e;
@@ -976,6 +1009,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                 const int s = i % NS;
                 if (i >= NS && !mbar_wait(&sm.empty[s], ((i / NS) - 1) & 1)) {
                     set_status(a.status, SEKV_ERR_TIMEOUT);
+                    *sm.sfail = 1;
                     break;
                 }
                 unsigned char* st = sm.stages + (size_t)s * C::STAGE;
@@ -1022,7 +1056,10 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
             }
             // drain: every issued copy has landed before the ring is reused
             for (int i = max(0, issued - NS); i < issued; ++i)
-                if (!mbar_wait(&sm.full[i % NS], (i / NS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
+                if (!mbar_wait(&sm.full[i % NS], (i / NS) & 1)) {
+                    set_status(a.status, SEKV_ERR_TIMEOUT);
+                    *sm.sfail = 1;
+                }
         }
     } else if constexpr (C::MMA) {
         // ------------------------------------------------ consumers, tensor cores
@@ -1165,7 +1202,10 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[s]);
         }
-        if (lane == 0) sm.qcnt[warp] = ok ? min(qn, a.qcap) : 0;
+        if (lane == 0) {
+            sm.qcnt[warp] = ok ? min(qn, a.qcap) : 0;
+            if (!ok) *sm.sfail = 1;
+        }
     } else {
         // ------------------------------------------------ consumers, CUDA cores
         const int rL = lane / G, hL = lane % G;
@@ -1285,11 +1325,20 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     }
     __syncthreads();    // the stream is done: the stage ring is free, the zoom queues are complete
 
-    if (!route_only && warp < kNW && ok) {
-        if constexpr (C::MMA) zoom_phase_mma<D, G>(a, sm, warp, lane, b, l, kvh, qa, mm, lm, oc);
-        else zoom_phase<DT, D, G>(a, sm, warp, lane, b, l, kvh, m_run, l_run, o, m_lane);
+    if constexpr (C::MMA) {
+        const int nq = sm.qcnt[0] + sm.qcnt[1] + sm.qcnt[2] + sm.qcnt[3];
+        if (!route_only && nq > 0 && *sm.sfail == 0) {     // uniform over the CTA
+            if (warp == kNW) zoom_produce<D, G>(a, sm, lane, b, l, kvh, nq);
+            else {
+                const int g = lane >> 2;
+                const uint32_t* qrow = g < G ? reinterpret_cast<const uint32_t*>(sm.qs + g * C::ROWB) : nullptr;
+                zoom_consume<D, G, RM>(a, sm, warp, lane, qrow, mm, lm, oc);
+            }
+        }
+    } else {
+        if (!route_only && warp < kNW && ok) zoom_phase<DT, D, G>(a, sm, warp, lane, b, l, kvh, m_run, l_run, o, m_lane);
     }
-    __syncthreads();    // zoom slots and scratch are dead: the ring takes the partial states
+    __syncthreads();    // zoom slots are dead: the ring takes the partial states
     if (!route_only && warp < kNW) {
         if constexpr (C::MMA) {
             const int g = lane >> 2, c = lane & 3;
@@ -1456,7 +1505,7 @@ static bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int d) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DT, int D, int G>
+template <int DT, int D, int G, int RM>
 static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st) {
     using C = DecCfg<DT, D, G>;
     const int Lr = d.l1 - d.l0;
@@ -1471,13 +1520,13 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     a.part_o = reinterpret_cast<float*>(partials);
     a.part_ml = a.part_o + units * G * p.nsplit * D;
     a.region = d.region_elems; a.scale = d.scale;
-    a.L = d.L; a.l0 = d.l0; a.Lr = Lr; a.Hq = d.Hq; a.Hkv = d.Hkv; a.a_cap = d.a_cap; a.m_cap = d.m_cap;
+    a.B = d.B; a.L = d.L; a.l0 = d.l0; a.Lr = Lr; a.Hq = d.Hq; a.Hkv = d.Hkv; a.a_cap = d.a_cap; a.m_cap = d.m_cap;
     a.rank = d.rank; a.phase = d.phase; a.nsplit = p.nsplit; a.sch_max = p.span_chunk;
     a.qcap = ((p.span_chunk + C::TR - 1) / C::TR) * C::R;
     a.mw = d.m_cap / 32;
     const size_t smem = decode_smem_bytes<DT, D, G>(a.sch_max, a.qcap);
     if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT, D, G, RM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     DecMaps maps;
@@ -1492,8 +1541,10 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
         }
         if (!ok) return cudaErrorInvalidValue;
     }
-    dim3 grid(p.nsplit, d.Hkv, d.B * Lr);
-    decode_kernel<DT, D, G><<<grid, (kNW + 1) * 32, smem, st>>>(a, maps);
+    const int64_t nblk = (int64_t)p.nsplit * d.Hkv * d.B * Lr;
+    if (nblk > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    dim3 grid((unsigned)nblk);
+    decode_kernel<DT, D, G, RM><<<grid, (kNW + 1) * 32, smem, st>>>(a, maps);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (d.phase != SEKV_ROUTE) {
         merge_kernel<D><<<d.B * Lr * d.Hq, D, 0, st>>>(a.part_o, a.part_ml, d.O, d.lse, p.nsplit, G, d.Hkv,
@@ -1503,13 +1554,22 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     return e;
 }
 
+// the tensor-core zoom is compiled for basis ranks up to 16, 32 and 64; the
+// CUDA-core path handles any rank up to 64 in one variant
+template <int DT, int D, int G>
+static cudaError_t launch_r(const sekv_decode_desc& d, const DecodePlan& p, void* w, cudaStream_t st) {
+    if (DT == SEKV_BF16 && d.rank <= 16) return launch_t<DT, D, G, 16>(d, p, w, st);
+    if (DT == SEKV_BF16 && d.rank <= 32) return launch_t<DT, D, G, 32>(d, p, w, st);
+    return launch_t<DT, D, G, 64>(d, p, w, st);
+}
+
 template <int DT, int D>
 static cudaError_t launch_g(const sekv_decode_desc& d, const DecodePlan& p, void* w, cudaStream_t st) {
     switch (d.Hq / d.Hkv) {
-        case 1: return launch_t<DT, D, 1>(d, p, w, st);
-        case 2: return launch_t<DT, D, 2>(d, p, w, st);
-        case 4: return launch_t<DT, D, 4>(d, p, w, st);
-        default: return launch_t<DT, D, 8>(d, p, w, st);
+        case 1: return launch_r<DT, D, 1>(d, p, w, st);
+        case 2: return launch_r<DT, D, 2>(d, p, w, st);
+        case 4: return launch_r<DT, D, 4>(d, p, w, st);
+        default: return launch_r<DT, D, 8>(d, p, w, st);
     }
 }
 

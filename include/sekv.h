@@ -96,14 +96,22 @@ typedef void* sekv_event_t;    /* a cudaEvent_t */
  * Basis storage. For each (b, l) there is a region of region_elems elements
  * (storage dtype). Span S of sequence b owns the Hkv consecutive blocks starting
  * at element blk_off[b][S] of the region, one block per kv head:
- *     block = [ A (|S| x rS) | pad | C (|S| x rS) | pad | B (rS x d) | D (rS x d) | pad ]
- * with rS = min(rank, |S|, d); A and C each take roundup(|S|*rS, 8) elements and
- * the block is padded to a multiple of 64 elements (sekv_block_elems). K_S ~ A B,
- * V_S ~ C D (SeKV blog 2.2, Eq. (6)-(8) with the rank gate fixed to 1).
+ *     block = [ A (len8 x r8) | C (len8 x r8) | B (r8 x d) | D (r8 x d) ]
+ * with rS = min(rank, |S|, d), len8 = roundup(|S|, 8), r8 = roundup(rS, 8).
+ * Each factor is stored 8x8-blocked: the zero-padded matrix is a row-major grid
+ * of 8 x 8 tiles, every tile 64 contiguous elements (row-major inside), so that
+ * element (r, c) of a matrix of padded width w8 sits at
+ *     ((r / 8) * (w8 / 8) + c / 8) * 64 + (r % 8) * 8 + c % 8.
+ * A tile is one 128-byte line of a bf16 factor, which the decode reads with
+ * conflict-free shared-memory matrix loads; a run of token (or basis-row) groups
+ * is one contiguous byte range. Padding is zero. The block size,
+ * 2 len8 r8 + 2 r8 d, is a multiple of 64 elements (sekv_block_elems).
+ * K_S ~ A B, V_S ~ C D (SeKV blog 2.2, Eq. (6)-(8) with the rank gate fixed to 1).
  */
 int64_t sekv_block_elems(int32_t len, int32_t d, int32_t rank);
 /* An upper bound of the region size for any segmentation with <= m_cap spans of a
- * sequence of n tokens: Hkv * (2*n*rank + m_cap*(2*rank*d + 80)). */
+ * sequence of n tokens: Hkv * (2*r8*n + m_cap*(14*r8 + 2*r8*d)) rounded up to 64,
+ * r8 = min(roundup(rank, 8), d). */
 int64_t sekv_basis_region_bound(int32_t n, int32_t m_cap, int32_t Hkv, int32_t d, int32_t rank);
 
 /* ------------------------------------------------------------------------- */

@@ -80,6 +80,32 @@ def margin(ell, theta):
     return float(np.min(np.abs(np.asarray(ell) - theta))) if np.size(ell) else math.inf
 
 
+def r8(x):
+    return -(-int(x) // 8) * 8
+
+
+def to_tiles8(M):
+    """Flatten matrix M into the library's 8x8-blocked storage order (zero-padded
+    to multiples of 8): a row-major grid of 8 x 8 tiles, each row-major inside."""
+    R, W = M.shape
+    P = np.zeros((r8(R), r8(W)), dtype=np.float64)
+    P[:R, :W] = M
+    return P.reshape(r8(R) // 8, 8, r8(W) // 8, 8).transpose(0, 2, 1, 3).reshape(-1)
+
+
+def from_tiles8(flat, R, W):
+    """Inverse of to_tiles8: the R x W matrix stored at ``flat``."""
+    P = np.asarray(flat).reshape(r8(R) // 8, r8(W) // 8, 8, 8).transpose(0, 2, 1, 3).reshape(r8(R), r8(W))
+    return P[:R, :W]
+
+
+def block_sections(ln, rS, d):
+    """(offset, elements) of A, C, B, D inside a span's block."""
+    pa = r8(ln) * r8(rS)
+    pb = r8(rS) * d
+    return {"A": (0, pa), "C": (pa, pa), "B": (2 * pa, pb), "D": (2 * pa + pb, pb)}
+
+
 def pack_bases(cache, segs, units):
     """Write oracle factors into the library's basis layout (device or pinned home)."""
     c = cache
@@ -92,14 +118,12 @@ def pack_bases(cache, segs, units):
             ln = int(end - beg)
             A, Bm, Cm, Dm = u.bases[S]
             rS = A.shape[1]
-            pa = ((ln * rS + 7) // 8) * 8
             be = _lib().sekv.sekv_block_elems(ln, c.d, c.rank)
             o = int(blk_off[b, S]) + kvh * be
             seg = flat[b, l]
-            seg[o:o + ln * rS] = torch.tensor(A.reshape(-1), dtype=c.dt)
-            seg[o + pa:o + pa + ln * rS] = torch.tensor(Cm.reshape(-1), dtype=c.dt)
-            seg[o + 2 * pa:o + 2 * pa + rS * c.d] = torch.tensor(Bm.reshape(-1), dtype=c.dt)
-            seg[o + 2 * pa + rS * c.d:o + 2 * pa + 2 * rS * c.d] = torch.tensor(Dm.reshape(-1), dtype=c.dt)
+            for name, M in (("A", A), ("C", Cm), ("B", Bm), ("D", Dm)):
+                off, n = block_sections(ln, rS, c.d)[name]
+                seg[o + off:o + off + n] = torch.tensor(to_tiles8(M), dtype=c.dt)
     if c.home.device.type != "cpu":
         c.home.copy_(home)
 

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -40,22 +41,45 @@ def test_version_and_status_strings():
 
 def test_block_layout_formula():
     from hierarchical_kv_cache_span_b200 import sekv as S
-    # rS = min(r, |S|, d); A, C padded to 8 elements; block padded to 64
-    for ln, d, r in [(1, 128, 16), (5, 128, 16), (64, 128, 16), (300, 128, 32), (7, 64, 4)]:
+    # rS = min(r, |S|, d); A, C are len8 x r8; B, D are r8 x d (8x8-blocked, zero-padded)
+    for ln, d, r in [(1, 128, 16), (5, 128, 16), (64, 128, 16), (300, 128, 32), (7, 64, 4), (13, 64, 12)]:
         rs = min(r, ln, d)
-        pa = -(-(ln * rs) // 8) * 8
-        want = -(-(2 * pa + 2 * rs * d) // 64) * 64
+        r8 = -(-rs // 8) * 8
+        l8 = -(-ln // 8) * 8
+        want = 2 * l8 * r8 + 2 * r8 * d
+        assert want % 64 == 0
         assert S.sekv_block_elems(ln, d, r) == want
     assert S.sekv_block_elems(0, 128, 16) == 0
 
 
+def test_tiles8_order_is_the_documented_one():
+    """Element (r, c) of a matrix of padded width w8 sits at
+    ((r/8) * (w8/8) + c/8) * 64 + (r%8) * 8 + c%8 (the layout the header states)."""
+    from tests.helpers import to_tiles8, from_tiles8
+    rng = np.random.default_rng(3)
+    M = rng.standard_normal((13, 20))
+    flat = to_tiles8(M)
+    assert flat.size == 16 * 24
+    for r in range(13):
+        for c in range(20):
+            assert flat[((r // 8) * 3 + c // 8) * 64 + (r % 8) * 8 + c % 8] == M[r, c]
+    assert np.array_equal(from_tiles8(flat, 13, 20), M)
+    pad = np.ones(flat.size, dtype=bool)
+    for r in range(13):
+        for c in range(20):
+            pad[((r // 8) * 3 + c // 8) * 64 + (r % 8) * 8 + c % 8] = False
+    assert not flat[pad].any()
+
+
 def test_region_bound_covers_worst_case():
     from hierarchical_kv_cache_span_b200 import sekv as S
-    n, m_cap, Hkv, d, r = 1000, 512, 2, 64, 8
-    bound = S.sekv_basis_region_bound(n, m_cap, Hkv, d, r)
-    # any segmentation: spans of total length <= n, count <= m_cap
-    for lens in ([1] * 500, [2] * 500, [n], [3] * 333):
-        assert Hkv * sum(S.sekv_block_elems(x, d, r) for x in lens) <= bound
+    for n, m_cap, Hkv, d, r in [(1000, 512, 2, 64, 8), (1000, 1000, 1, 128, 16), (4096, 700, 8, 128, 12)]:
+        bound = S.sekv_basis_region_bound(n, m_cap, Hkv, d, r)
+        # any segmentation: spans of total length <= n, count <= m_cap
+        cases = ([1] * min(m_cap, n), [2] * min(m_cap, n // 2), [n], [3] * min(m_cap, n // 3),
+                 [9] * min(m_cap, n // 9), [r + 1] * min(m_cap, n // (r + 1)))
+        for lens in cases:
+            assert Hkv * sum(S.sekv_block_elems(x, d, r) for x in lens) <= bound
 
 
 def test_invalid_build_arguments_are_rejected_before_launch():

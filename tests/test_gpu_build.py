@@ -153,15 +153,21 @@ def _read_block(c, b, l, kvh, S, beg, end):
     P = _lib()
     ln = end - beg
     rS = min(c.rank, ln, c.d)
-    pa = -(-(ln * rS) // 8) * 8
     be = P.sekv.sekv_block_elems(ln, c.d, c.rank)
     o = int(c.blk_off[b, S]) + kvh * be
     blk = c.home[b, l, o:o + be].to("cpu", torch.float64).numpy()
-    A = blk[:ln * rS].reshape(ln, rS)
-    Cm = blk[pa:pa + ln * rS].reshape(ln, rS)
-    Bm = blk[2 * pa:2 * pa + rS * c.d].reshape(rS, c.d)
-    Dm = blk[2 * pa + rS * c.d:2 * pa + 2 * rS * c.d].reshape(rS, c.d)
-    return A, Bm, Cm, Dm
+    sec = T.block_sections(ln, rS, c.d)
+    out = {}
+    for name, (R, W) in (("A", (ln, rS)), ("C", (ln, rS)), ("B", (rS, c.d)), ("D", (rS, c.d))):
+        off, n = sec[name]
+        part = blk[off:off + n]
+        out[name] = T.from_tiles8(part, R, W)
+        # the padding of every section is exactly zero
+        full = T.from_tiles8(part, T.r8(R), T.r8(W))
+        mask = np.ones_like(full, dtype=bool)
+        mask[:R, :W] = False
+        assert not full[mask].any(), f"nonzero padding in {name}"
+    return out["A"], out["B"], out["C"], out["D"]
 
 
 BASIS_CASES = [

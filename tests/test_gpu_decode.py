@@ -70,6 +70,9 @@ KERNEL_CASES = [
     ("c5", dict(n=4096, L=1, Hq=8, Hkv=2)),                 # rank 32, 25% zoom
     ("c2", dict(n=2048, L=1, d=64, Hq=16, Hkv=2, rank=8)),  # G = 8, d = 64
     ("c2", dict(n=2048, L=1, Hq=16, Hkv=8)),                # G = 2
+    ("c5", dict(n=2048, L=1, Hq=8, Hkv=2, rank=48)),        # d = 128, r = 48: two B / D pieces per span
+    ("c5", dict(n=2048, L=1, Hq=8, Hkv=2, rank=20)),        # r8 = 24: odd count of 8-row basis blocks
+    ("c5", dict(n=2048, L=1, d=64, Hq=4, Hkv=1, rank=64)),  # d = 64, r = 64
 ]
 
 
@@ -87,6 +90,29 @@ def test_decode_kernel_level(name, over):
     assert c.read_status() == 0
     err, lerr, nz = _compare(wl, c, q, theta, scale, segs, units, O_gpu, lse_gpu, zmask)
     print(f"{name} {over}: max|dO|={err:.2e} max|dlse|={lerr:.2e} zoomed={nz}")
+
+
+@pytest.mark.parametrize("name,over", [
+    ("c2", dict(n=2048, L=1, Hq=8, Hkv=2)),                 # r = 16
+    ("c5", dict(n=1536, L=1, Hq=8, Hkv=2, rank=40)),        # r8 = 40: two B / D pieces, odd blocks
+    ("c2", dict(n=1024, L=1, d=64, Hq=8, Hkv=1, rank=12)),  # d = 64, G = 8, r8 = 16 with rS = 12
+])
+def test_decode_all_zoom_matches_oracle(name, over):
+    """theta = -inf: every span of every length is attended token by token through
+    its bases (short spans with r_S = |S| < r included)."""
+    wl = WORKLOADS[name].scaled(**over)
+    H, K, V, segs, units, q, _, scale = _setup(wl)
+    theta = np.full((wl.L, wl.Hq), -np.inf)
+    c = _cache(wl)
+    T.upload_oracle_cache(c, segs, units)
+    zmask = c.new_zmask()
+    th = torch.full((wl.L, wl.Hq), -math.inf, dtype=torch.float32, device="cuda")
+    O_gpu, lse_gpu = c.decode(q.cuda(), th, zmask=zmask)
+    torch.cuda.synchronize()
+    assert c.read_status() == 0
+    err, lerr, nz = _compare(wl, c, q, theta, scale, segs, units, O_gpu, lse_gpu, zmask)
+    assert nz == wl.L * wl.Hq * sum(len(s.spans) for s in segs)
+    print(f"all-zoom {name} {over}: max|dO|={err:.2e} max|dlse|={lerr:.2e} zoomed={nz}")
 
 
 @pytest.mark.parametrize("name,over", [("c1", dict()), ("c2", dict(n=4096, L=2)), ("c5", dict(n=2048, L=1))])
@@ -231,6 +257,22 @@ def test_all_zoom_full_rank_gives_dense_attention():
     torch.cuda.synchronize()
     assert c.read_status() == 0
     _dense_unit_check(wl, c, q, K, V, 1.0 / math.sqrt(wl.d), 1e-4)
+
+
+def test_all_zoom_full_rank_bf16_gives_dense_attention():
+    """bf16, r = d = 64, every span zoomed: K_S = A B and V_S = C D hold up to the
+    bf16 rounding of the stored factors (relative 2^-9 per factor), which moves
+    logits by ~1e-3 here, inside the bf16 tolerance."""
+    wl = WORKLOADS["c2"].scaled(n=1200, L=1, d=64, Hq=4, Hkv=2, rank=64)
+    H, K, V = T.make_inputs(wl)
+    c = _cache(wl)
+    c.build(H.cuda(), K.cuda(), V.cuda(), wl.alpha, wl.window, wl.wmode, max_sweeps=40)
+    q = gen.queries(wl)
+    th = torch.full((wl.L, wl.Hq), -math.inf, dtype=torch.float32, device="cuda")
+    c.last = c.decode(q.cuda(), th)
+    torch.cuda.synchronize()
+    assert c.read_status() == 0
+    _dense_unit_check(wl, c, q, K, V, 1.0 / math.sqrt(wl.d), 2e-2)
 
 
 def test_empty_cache_rows():
