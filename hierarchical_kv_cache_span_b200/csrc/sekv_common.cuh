@@ -161,6 +161,14 @@ SEKV_DEV void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uin
 // ---------------------------------------------------------------------------
 // warp-level tensor-core helpers (ldmatrix + mma.sync m16n8k16 bf16 -> fp32)
 // ---------------------------------------------------------------------------
+// transpose an 8 x 8 bf16 matrix held as one mma fragment register per lane
+// (lane l holds row l/4, columns 2(l%4), 2(l%4)+1; the result holds the transpose)
+SEKV_DEV uint32_t movm_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
 // explicit shared-memory loads (a generic load of shared memory is slower)
 SEKV_DEV uint32_t lds_u32(const void* p) {
     uint32_t v;

@@ -56,7 +56,7 @@ struct DecCfg {
     static constexpr int META = 2 * TR * 4;                 // inv_norm + logS of a span tile
     static constexpr int STAGE0 = 2 * TILE + META;
     static constexpr int STAGE = MMA ? (STAGE0 + 1023) / 1024 * 1024 : STAGE0;
-    static constexpr int NS0 = (MMA ? 68 * 1024 : 64 * 1024) / STAGE;     // 2 CTAs / SM on the bf16 path
+    static constexpr int NS0 = (MMA ? 102 * 1024 : 64 * 1024) / STAGE;    // 2 CTAs / SM on the bf16 path
     static constexpr int NS = NS0 < 2 ? 2 : (NS0 > 6 ? 6 : NS0);   // ring depth
     static constexpr int YPL = kRMax * G / 32;              // y entries per lane (fp32 zoom)
     static constexpr int WSCR = MMA ? 0 : (64 * G) + 2 * kRMax * G;   // per-warp scratch floats (fp32 zoom)
@@ -540,19 +540,21 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
 }
 
 // ---------------------------------------------------------------------------
-// Phase 2 on the tensor cores (bf16). The producer warp walks the CTA's zoom queue
-// and streams, per zoomed span, its B rows, its A/C token groups and its D rows
-// through one CTA-wide ring of 8 KB slots; every consumer warp reads every slot.
-// Per span, with r8 = roundup(r_S, 8) and the heads h that zoom it:
-//   u^T  = q^T B_S^T    (M = heads, N = basis rows, K = d)
-//   s^T  = u^T A_S^T    (M = heads, N = 16 tokens, K = r8)   -> online softmax p
-//   y^T += p^T C_S      (M = heads, N = basis rows, K = 16 tokens)
-//   O   += (beta y)^T D_S  into the warp's stream accumulators
-// Each accumulator is the next product's A fragment, so u, p and y never leave
-// registers. The span's 16-token sub-chunks are dealt round-robin to the four
-// consumer warps (continuing across spans); a warp with no sub-chunk in a span
-// skips it. u (pre-scaled by scale * log2 e) enters as a hi + lo bf16 pair (about
-// 16 significant bits); p and beta*y are rounded to bf16 as p on the stream path.
+// Phase 2 on the tensor cores (bf16). The producer warp reads the CTA's zoom
+// bitmask (span order) and streams, per zoomed span, its B rows, its A/C token
+// groups and its D rows through one CTA-wide ring of 16 KB slots; every consumer
+// warp reads every slot. Per span, with r8 = roundup(r_S, 8) and the heads h that
+// zoom it (heads on the mma N side, as on the stream path):
+//   u    = B_S q        (M = basis rows, N = heads, K = d)
+//   s    = A_S u        (M = tokens,     N = heads, K = r8)  -> online softmax p
+//   y   += C_S^T p      (M = basis rows, N = heads, K = tokens)
+//   O^T += D_S^T (beta y)  into the warp's stream accumulators
+// An accumulator becomes the next product's B fragment through an 8 x 8 register
+// transpose, so u, p and y never leave registers. The span's 32-token units are
+// dealt round-robin to the four consumer warps (continuing across spans); a warp
+// with no unit in a span skips it. u (pre-scaled by scale * log2 e) enters as a
+// hi + lo bf16 pair (about 16 significant bits); p and beta*y are rounded to
+// bf16 as p on the stream path.
 // ---------------------------------------------------------------------------
 // tokens of an A/C piece: both halves fit ZSLOTC / 2, a multiple of 32, at most 256
 SEKV_DEV int zoom_piece_tokens(int r8, int zslot) {
@@ -560,10 +562,27 @@ SEKV_DEV int zoom_piece_tokens(int r8, int zslot) {
     return t > 256 ? 256 : t;
 }
 
+// split v0, v1 into a hi + lo bf16x2 pair
+SEKV_DEV void split_bf16x2(float v0, float v1, uint32_t& hi, uint32_t& lo) {
+    hi = pack_bf16(v0, v1);
+    lo = pack_bf16(v0 - bf16_lo(hi), v1 - bf16_hi(hi));
+}
+
+// hardware 2^x (ex2.approx.ftz: relative error ~2^-22; 2^-inf = 0)
+SEKV_DEV float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// zoomed spans of the CTA: word w of zw[h] holds heads h's bits for spans
+// s0 + 32 w .. s0 + 32 w + 31; nwords words are in use
 template <int D, int G>
-SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b, int l, int kvh, int nq) {
+SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b, int l, int kvh, int s0, int nwords,
+                           int zwords) {
     using C = DecCfg<SEKV_BF16, D, G>;
     constexpr int ZNS = C::ZNSC, ZSL = C::ZSLOTC, RBC = C::RBC;
+    constexpr uint32_t FULL = 0xffffffffu;
     uint32_t np = 0;          // pieces armed
     bool good = true;
     int rot = 0;
@@ -589,66 +608,87 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
                 set_status(a.status, SEKV_ERR_TIMEOUT);
             }
         }
-        okk = __shfl_sync(0xffffffffu, okk, 0);
+        okk = __shfl_sync(FULL, okk, 0);
         if (okk) ++np;
         good = good && okk;
     };
-    for (int e0 = 0; e0 < nq && good; e0 += 32) {
-        // lane j resolves queue entry e0 + j: span, zooming heads, block offset
-        int len = 0;
-        uint32_t hm = 0u;
-        long long off = -1;
-        const int e = e0 + lane;
-        if (e < nq) {
-            int w = 0, x = e;
-            while (w < kNW - 1 && x >= sm.qcnt[w]) { x -= sm.qcnt[w]; ++w; }
-            const int ent = sm.zq[w * a.qcap + x];
-            const int S = ent & 0xffffff;
-            hm = (uint32_t)ent >> 24;
-            const int beg = a.span_beg[(int64_t)b * a.m_cap + S];
-            len = a.span_end[(int64_t)b * a.m_cap + S] - beg;
-            if (len < 1) {
-                set_status(a.status, SEKV_ERR_INVALID_ARG);
-                len = 0;
-            } else if (a.slot) {
-                off = a.slot[((int64_t)b * a.L + l) * a.m_cap + S];
-                if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
-            } else {
-                off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S];
-            }
+    for (int w0 = 0; w0 < nwords && good; w0 += 32) {
+        // lane j takes word w0 + j: spans zoomed by any head, counted and scanned
+        const int wi = w0 + lane;
+        uint32_t m = 0u;
+        if (wi < nwords) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) m |= sm.zw[h * zwords + wi];
         }
-        const int cnt = min(32, nq - e0);
-        for (int j = 0; j < cnt && good; ++j) {
-            const int jl = __shfl_sync(0xffffffffu, len, j);
-            const uint32_t jhm = __shfl_sync(0xffffffffu, hm, j);
-            const long long jo = __shfl_sync(0xffffffffu, off, j);
-            if (jl < 1 || jo < 0) continue;
-            const int rS = block_rank(jl, D, a.rank), r8 = round8(rS);
-            const int64_t pa = block_ac_elems(jl, rS);
-            const int64_t be = 2 * pa + 2 * (int64_t)r8 * D;
-            const char* blk = a.arena + ((int64_t)jo + (int64_t)kvh * be) * 2;
-            const int tcz = zoom_piece_tokens(r8, ZSL);
-            ZPiece pc;
-            pc.len = jl;
-            pc.rS = rS;
-            pc.hm = jhm;
-            pc.rot = rot;
-            for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
-                pc.kind = ZP_B; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
-                emit(pc, blk + (2 * pa + (int64_t)r0 * D) * 2, (uint32_t)pc.cnt * C::ROWB, nullptr, 0u);
+        const int cnt = __popc(m);
+        int inc = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(FULL, inc, o);
+            if (lane >= o) inc += t;
+        }
+        const int total = __shfl_sync(FULL, inc, 31);
+        for (int e0 = 0; e0 < total && good; e0 += 32) {
+            // lane j resolves entry e0 + j: its word, bit, heads and block offset
+            const int e = e0 + lane;
+            int k = 0;
+            for (int j = 0; j < 32; ++j) k += (__shfl_sync(FULL, inc, j) <= e) ? 1 : 0;
+            const int kw = k < 32 ? k : 31;
+            const int inck = __shfl_sync(FULL, inc, kw), cntk = __shfl_sync(FULL, cnt, kw);
+            const uint32_t mk = __shfl_sync(FULL, m, kw);
+            int len = 0;
+            uint32_t hm = 0u;
+            long long off = -1;
+            if (e < total) {
+                const int bit = (int)__fns(mk, 0u, e - (inck - cntk) + 1);
+                const int S = s0 + (w0 + kw) * 32 + bit;
+#pragma unroll
+                for (int h = 0; h < G; ++h) hm |= ((sm.zw[h * zwords + w0 + kw] >> bit) & 1u) << h;
+                const int beg = a.span_beg[(int64_t)b * a.m_cap + S];
+                len = a.span_end[(int64_t)b * a.m_cap + S] - beg;
+                if (len < 1) {
+                    set_status(a.status, SEKV_ERR_INVALID_ARG);
+                    len = 0;
+                } else if (a.slot) {
+                    off = a.slot[((int64_t)b * a.L + l) * a.m_cap + S];
+                    if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
+                } else {
+                    off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S];
+                }
             }
-            for (int t0 = 0; t0 < jl && good; t0 += tcz) {
-                pc.kind = ZP_AC; pc.first = t0 == 0; pc.r0 = t0; pc.cnt = min(tcz, jl - t0);
-                const uint32_t nb = (uint32_t)round8(pc.cnt) * r8 * 2;
-                const int64_t to = (int64_t)t0 * r8 * 2;
-                emit(pc, blk + to, nb, blk + pa * 2 + to, nb);
+            const int cntb = min(32, total - e0);
+            for (int j = 0; j < cntb && good; ++j) {
+                const int jl = __shfl_sync(FULL, len, j);
+                const uint32_t jhm = __shfl_sync(FULL, hm, j);
+                const long long jo = __shfl_sync(FULL, off, j);
+                if (jl < 1 || jo < 0) continue;
+                const int rS = block_rank(jl, D, a.rank), r8 = round8(rS);
+                const int64_t pa = block_ac_elems(jl, rS);
+                const int64_t be = 2 * pa + 2 * (int64_t)r8 * D;
+                const char* blk = a.arena + ((int64_t)jo + (int64_t)kvh * be) * 2;
+                const int tcz = zoom_piece_tokens(r8, ZSL);
+                ZPiece pc;
+                pc.len = jl;
+                pc.rS = rS;
+                pc.hm = jhm;
+                pc.rot = rot;
+                for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
+                    pc.kind = ZP_B; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
+                    emit(pc, blk + (2 * pa + (int64_t)r0 * D) * 2, (uint32_t)pc.cnt * C::ROWB, nullptr, 0u);
+                }
+                for (int t0 = 0; t0 < jl && good; t0 += tcz) {
+                    pc.kind = ZP_AC; pc.first = t0 == 0; pc.r0 = t0; pc.cnt = min(tcz, jl - t0);
+                    const uint32_t nb = (uint32_t)round8(pc.cnt) * r8 * 2;
+                    const int64_t to = (int64_t)t0 * r8 * 2;
+                    emit(pc, blk + to, nb, blk + pa * 2 + to, nb);
+                }
+                for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
+                    pc.kind = ZP_D; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
+                    emit(pc, blk + (2 * pa + (int64_t)r8 * D + (int64_t)r0 * D) * 2, (uint32_t)pc.cnt * C::ROWB,
+                         nullptr, 0u);
+                }
+                rot = (rot + ((jl + 31) >> 5)) & 3;
             }
-            for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
-                pc.kind = ZP_D; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
-                emit(pc, blk + (2 * pa + (int64_t)r8 * D + (int64_t)r0 * D) * 2, (uint32_t)pc.cnt * C::ROWB,
-                     nullptr, 0u);
-            }
-            rot = (rot + ((jl + 31) >> 5)) & 3;
         }
     }
     if (good) {
@@ -665,40 +705,29 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
     }
 }
 
-// split v0, v1 into a hi + lo bf16x2 pair
-SEKV_DEV void split_bf16x2(float v0, float v1, uint32_t& hi, uint32_t& lo) {
-    hi = pack_bf16(v0, v1);
-    lo = pack_bf16(v0 - bf16_lo(hi), v1 - bf16_hi(hi));
-}
-
-// hardware 2^x (ex2.approx.ftz: relative error ~2^-22; 2^-inf = 0)
-SEKV_DEV float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
 // RM: the largest basis rank this instantiation handles (16, 32 or 64), which
-// sizes the y accumulators and the unrolled basis-row loops
+// sizes the u / y fragments and the unrolled basis-row loops. Lane (g, c) holds
+// heads 2c, 2c+1 (the stream layout): mh, lh (partial) and the O^T columns.
 template <int D, int G, int RM>
-SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int lane, const uint32_t* qrow,
-                           float& mm, float& lm, float (&oc)[D / 8][4]) {
+SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int lane, const uint32_t (&qb)[D / 16][2],
+                           float (&mh)[2], float (&lh)[2], float (&oc)[D / 16][4]) {
     using C = DecCfg<SEKV_BF16, D, G>;
     constexpr int ZNS = C::ZNSC, ZSL = C::ZSLOTC;
-    constexpr int NIB = RM / 8;          // basis-row blocks of 8
-    constexpr int NKS = RM / 16;         // k-steps of 16 basis rows
+    constexpr int NKS = RM / 16;         // groups of 16 basis rows (m-tiles of u, y; k-steps of s, O)
     constexpr int DB = D / 8;            // column blocks of 8 in B / D rows
-    const int g = lane >> 2, cq = lane & 3, mi = lane >> 3, lr = lane & 7;
+    constexpr uint32_t FULL = 0xffffffffu;
+    const int g = lane >> 2, c = lane & 3, lj = lane >> 3, lr = lane & 7;
     const float sl2 = a.scale * kLog2e;
-    uint32_t uf[NKS][4];                 // u^T A fragments per k-step: hi a0, hi a2, lo a0, lo a2 (then (beta y)^T)
-    float yacc[NIB][4];                  // y^T accumulators per block of 8 basis rows
-    float msp = -INFINITY, lsp = 0.f;    // the span's (max, partial sum) for head g
-    bool mine = false, zh = false;
-    int nib = 1, rS = 1, rot = 0;
+    uint32_t ub[NKS][4];                 // u as B fragments per k-step: hi b0, hi b1, lo b0, lo b1 (then beta y)
+    float yacc[NKS][4];                  // y accumulators per 16 basis rows: (row g / g+8, heads 2c, 2c+1)
+    float msp[2] = {-INFINITY, -INFINITY}, lsp[2] = {0.f, 0.f};
+    bool mine = false, zh0 = false, zh1 = false;
+    int nib = 1, rS = 1;
 #pragma unroll
-    for (int ks = 0; ks < NKS; ++ks) uf[ks][0] = uf[ks][1] = uf[ks][2] = uf[ks][3] = 0u;
-#pragma unroll
-    for (int j = 0; j < NIB; ++j) yacc[j][0] = yacc[j][1] = yacc[j][2] = yacc[j][3] = 0.f;
+    for (int ks = 0; ks < NKS; ++ks) {
+        ub[ks][0] = ub[ks][1] = ub[ks][2] = ub[ks][3] = 0u;
+        yacc[ks][0] = yacc[ks][1] = yacc[ks][2] = yacc[ks][3] = 0.f;
+    }
 
     for (uint32_t k = 0;; ++k) {
         const int slot = (int)(k % ZNS);
@@ -718,50 +747,41 @@ SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int la
             if (pc.first) {
                 rS = pc.rS;
                 nib = (rS + 7) >> 3;
-                rot = pc.rot;
-                mine = ((pc.len + 31) >> 5) > ((warp - rot) & 3);
-                zh = g < G && ((pc.hm >> g) & 1u);
-                msp = -INFINITY;
-                lsp = 0.f;
+                mine = ((pc.len + 31) >> 5) > ((warp - pc.rot) & 3);
+                zh0 = 2 * c < G && ((pc.hm >> (2 * c)) & 1u);
+                zh1 = 2 * c + 1 < G && ((pc.hm >> (2 * c + 1)) & 1u);
+                msp[0] = msp[1] = -INFINITY;
+                lsp[0] = lsp[1] = 0.f;
 #pragma unroll
-                for (int j = 0; j < NIB; ++j) yacc[j][0] = yacc[j][1] = yacc[j][2] = yacc[j][3] = 0.f;
+                for (int ks = 0; ks < NKS; ++ks) yacc[ks][0] = yacc[ks][1] = yacc[ks][2] = yacc[ks][3] = 0.f;
             }
             if (mine) {
-                // u^T for the basis-row blocks of this piece, two blocks (one k-step) at a time
+                // u for the basis rows of this piece, 16 at a time (two partial sums
+                // over even / odd k-steps keep the mma chains short)
 #pragma unroll
                 for (int ks = 0; ks < NKS; ++ks) {
                     if (16 * ks < pc.r0 || 16 * ks >= pc.r0 + pc.cnt) continue;
-                    const int jl = (16 * ks - pc.r0) >> 3;          // piece-local block
-                    // two partial sums per n-tile (even / odd k-steps) keep the mma chains short
-                    float u0[4] = {0.f, 0.f, 0.f, 0.f}, u1[4] = {0.f, 0.f, 0.f, 0.f};
-                    float v0[4] = {0.f, 0.f, 0.f, 0.f}, v1[4] = {0.f, 0.f, 0.f, 0.f};
+                    const int ib = (16 * ks - pc.r0) >> 3;             // piece-local 8-row block
+                    const bool two = 16 * ks + 8 < pc.r0 + pc.cnt;
+                    float ua[4] = {0.f, 0.f, 0.f, 0.f}, uv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int p = 0; p < D / 32; ++p) {
-                        uint32_t b0[4], b1[4];
-                        ldsm_x4(b0, zs + ((jl * DB + 4 * p + mi) * 64 + lr * 8) * 2);
-                        ldsm_x4(b1, zs + (((jl + 1) * DB + 4 * p + mi) * 64 + lr * 8) * 2);
-                        // q of head g as A fragments (rows >= G are zero): k-steps 2p, 2p + 1
-                        const uint32_t qf0[4] = {qrow ? lds_u32(qrow + 16 * p + cq) : 0u, 0u,
-                                                 qrow ? lds_u32(qrow + 16 * p + 4 + cq) : 0u, 0u};
-                        const uint32_t qf1[4] = {qrow ? lds_u32(qrow + 16 * p + 8 + cq) : 0u, 0u,
-                                                 qrow ? lds_u32(qrow + 16 * p + 12 + cq) : 0u, 0u};
-                        const uint32_t c00[2] = {b0[0], b0[1]}, c01[2] = {b0[2], b0[3]};
-                        const uint32_t c10[2] = {b1[0], b1[1]}, c11[2] = {b1[2], b1[3]};
-                        mma_bf16_16816(u0, qf0, c00);
-                        mma_bf16_16816(u1, qf0, c10);
-                        mma_bf16_16816(v0, qf1, c01);
-                        mma_bf16_16816(v1, qf1, c11);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        uint32_t ba[4];
+                        ldsm_x4(ba, zs + (((ib + (lj & 1)) * DB + 2 * kk + (lj >> 1)) * 64 + lr * 8) * 2);
+                        if (!two) ba[1] = ba[3] = 0u;
+                        const uint32_t qf[2] = {qb[kk][0], qb[kk][1]};
+                        mma_bf16_16816((kk & 1) ? uv : ua, ba, qf);
                     }
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        u0[e] += v0[e];
-                        u1[e] += v1[e];
-                    }
-                    // basis rows i >= r_S do not exist: exact zeros (select, not multiply)
-                    const int i0 = 16 * ks + 2 * cq;
-                    split_bf16x2(i0 < rS ? u0[0] * sl2 : 0.f, i0 + 1 < rS ? u0[1] * sl2 : 0.f, uf[ks][0], uf[ks][2]);
-                    split_bf16x2(i0 + 8 < rS ? u1[0] * sl2 : 0.f, i0 + 9 < rS ? u1[1] * sl2 : 0.f, uf[ks][1],
-                                 uf[ks][3]);
+                    // rows i >= r_S do not exist: exact zeros (select, not multiply)
+                    const int i0 = 16 * ks + g;
+                    uint32_t h01, l01, h23, l23;
+                    split_bf16x2(i0 < rS ? (ua[0] + uv[0]) * sl2 : 0.f, i0 < rS ? (ua[1] + uv[1]) * sl2 : 0.f, h01, l01);
+                    split_bf16x2(i0 + 8 < rS ? (ua[2] + uv[2]) * sl2 : 0.f, i0 + 8 < rS ? (ua[3] + uv[3]) * sl2 : 0.f,
+                                 h23, l23);
+                    ub[ks][0] = movm_t(h01);
+                    ub[ks][1] = movm_t(h23);
+                    ub[ks][2] = movm_t(l01);
+                    ub[ks][3] = movm_t(l23);
                 }
             }
         } else if (pc.kind == ZP_AC) {
@@ -769,78 +789,78 @@ SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int la
                 const unsigned char* As = zs;
                 const unsigned char* Cs = zs + ZSL / 2;
                 const int nv = (pc.cnt + 31) >> 5;
-                for (int v = (warp - rot - (pc.r0 >> 5)) & 3; v < nv; v += 4) {
+                for (int v = (warp - pc.rot - (pc.r0 >> 5)) & 3; v < nv; v += 4) {
                     // token groups 4v .. 4v+3 of the piece; those at or past ngp were not copied
                     const int ngp = ((pc.cnt + 7) >> 3) - 4 * v;
-                    // s^T = u^T A^T for the unit's 32 tokens (four n-tiles of 8)
-                    float sc[4][4];
+                    // s = A u for the unit's 32 tokens (two m-tiles of 16)
+                    float sc[2][4];
 #pragma unroll
-                    for (int n = 0; n < 4; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+                    for (int mt = 0; mt < 2; ++mt) {
+                        sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
+                        if (ngp <= 2 * mt) continue;
 #pragma unroll
-                    for (int ks = 0; ks < NKS; ++ks) {
-                        if (2 * ks >= nib) continue;
-                        const bool two = 2 * ks + 1 < nib;
-                        uint32_t a0[4], a1[4];
-                        ldsm_x4(a0, As + (((4 * v + (mi >> 1)) * nib + 2 * ks + (mi & 1)) * 64 + lr * 8) * 2);
-                        ldsm_x4(a1, As + (((4 * v + 2 + (mi >> 1)) * nib + 2 * ks + (mi & 1)) * 64 + lr * 8) * 2);
-                        const uint32_t b0[2] = {a0[0], two ? a0[1] : 0u}, b1[2] = {a0[2], two ? a0[3] : 0u};
-                        const uint32_t b2[2] = {a1[0], two ? a1[1] : 0u}, b3[2] = {a1[2], two ? a1[3] : 0u};
-                        const uint32_t uh[4] = {uf[ks][0], 0u, uf[ks][1], 0u};
-                        const uint32_t ul[4] = {uf[ks][2], 0u, uf[ks][3], 0u};
-                        mma_bf16_16816(sc[0], uh, b0);
-                        mma_bf16_16816(sc[1], uh, b1);
-                        mma_bf16_16816(sc[2], uh, b2);
-                        mma_bf16_16816(sc[3], uh, b3);
-                        mma_bf16_16816(sc[0], ul, b0);
-                        mma_bf16_16816(sc[1], ul, b1);
-                        mma_bf16_16816(sc[2], ul, b2);
-                        mma_bf16_16816(sc[3], ul, b3);
-                    }
-                    // the span's online softmax for head g (log2 domain; u carries the scale)
-                    const int tk = 32 * v + 2 * cq;
-                    float x[8];
-#pragma unroll
-                    for (int n = 0; n < 4; ++n) {
-                        x[2 * n] = (zh && tk + 8 * n < pc.cnt) ? sc[n][0] : -INFINITY;
-                        x[2 * n + 1] = (zh && tk + 8 * n + 1 < pc.cnt) ? sc[n][1] : -INFINITY;
-                    }
-                    float mx = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])), fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                    const float mnew = fmaxf(msp, mx);
-                    const float al = (mnew == -INFINITY) ? 1.f : ex2(msp - mnew);
-                    const float mref = (mnew == -INFINITY) ? 0.f : mnew;
-                    float pv[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) pv[e] = ex2(x[e] - mref);
-                    lsp = fmaf(lsp, al, ((pv[0] + pv[1]) + (pv[2] + pv[3])) + ((pv[4] + pv[5]) + (pv[6] + pv[7])));
-                    msp = mnew;
-                    if (__any_sync(0xffffffffu, al != 1.f)) {
-#pragma unroll
-                        for (int j = 0; j < NIB; ++j) {
-                            yacc[j][0] *= al;
-                            yacc[j][1] *= al;
+                        for (int ks = 0; ks < NKS; ++ks) {
+                            if (2 * ks >= nib) continue;
+                            uint32_t aa[4];
+                            ldsm_x4(aa, As + (((4 * v + 2 * mt + (lj & 1)) * nib + 2 * ks + (lj >> 1)) * 64 + lr * 8) * 2);
+                            if (2 * ks + 1 >= nib) aa[2] = aa[3] = 0u;
+                            const uint32_t uh[2] = {ub[ks][0], ub[ks][1]}, ul[2] = {ub[ks][2], ub[ks][3]};
+                            mma_bf16_16816(sc[mt], aa, uh);
+                            mma_bf16_16816(sc[mt], aa, ul);
                         }
                     }
-                    // y^T += p^T C (p as A fragments: k = tokens 0..15 and 16..31 of the unit)
-                    const uint32_t p0[4] = {pack_bf16(pv[0], pv[1]), 0u, pack_bf16(pv[2], pv[3]), 0u};
-                    const uint32_t p1[4] = {pack_bf16(pv[4], pv[5]), 0u, pack_bf16(pv[6], pv[7]), 0u};
+                    // the span's online softmax for heads 2c, 2c+1 (log2 domain; u carries the scale)
+                    float x[2][4];
 #pragma unroll
-                    for (int jp = 0; jp < NKS; ++jp) {
-                        if (2 * jp >= nib) continue;
-                        uint32_t c0[4], c1[4];
-                        ldsm_x4_t(c0, Cs + (((4 * v + (mi & 1)) * nib + 2 * jp + (mi >> 1)) * 64 + lr * 8) * 2);
-                        ldsm_x4_t(c1, Cs + (((4 * v + 2 + (mi & 1)) * nib + 2 * jp + (mi >> 1)) * 64 + lr * 8) * 2);
-                        // C rows of groups that were not copied hold stale bytes: zero them
-                        const uint32_t g1 = ngp > 1 ? 0xffffffffu : 0u, g2 = ngp > 2 ? 0xffffffffu : 0u,
-                                       g3 = ngp > 3 ? 0xffffffffu : 0u;
-                        const uint32_t e00[2] = {c0[0], c0[1] & g1}, e10[2] = {c1[0] & g2, c1[1] & g3};
-                        mma_bf16_16816(yacc[2 * jp], p0, e00);
-                        mma_bf16_16816(yacc[2 * jp], p1, e10);
-                        if (2 * jp + 1 < nib) {
-                            const uint32_t e01[2] = {c0[2], c0[3] & g1}, e11[2] = {c1[2] & g2, c1[3] & g3};
-                            mma_bf16_16816(yacc[2 * jp + 1], p0, e01);
-                            mma_bf16_16816(yacc[2 * jp + 1], p1, e11);
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int tk = 32 * v + 16 * mt + g + ((e >> 1) << 3);
+                            const bool zz = (e & 1) ? zh1 : zh0;
+                            x[mt][e] = (zz && tk < pc.cnt) ? sc[mt][e] : -INFINITY;
+                        }
+                    float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
+                    float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
+#pragma unroll
+                    for (int o = 4; o < 32; o <<= 1) {
+                        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, o));
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, o));
+                    }
+                    const float mn0 = fmaxf(msp[0], mx0), mn1 = fmaxf(msp[1], mx1);
+                    const float al0 = (mn0 == -INFINITY) ? 1.f : ex2(msp[0] - mn0);
+                    const float al1 = (mn1 == -INFINITY) ? 1.f : ex2(msp[1] - mn1);
+                    const float r0 = (mn0 == -INFINITY) ? 0.f : mn0, r1 = (mn1 == -INFINITY) ? 0.f : mn1;
+                    float pv[2][4];
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) pv[mt][e] = ex2(x[mt][e] - ((e & 1) ? r1 : r0));
+                    lsp[0] = fmaf(lsp[0], al0, (pv[0][0] + pv[0][2]) + (pv[1][0] + pv[1][2]));
+                    lsp[1] = fmaf(lsp[1], al1, (pv[0][1] + pv[0][3]) + (pv[1][1] + pv[1][3]));
+                    msp[0] = mn0;
+                    msp[1] = mn1;
+                    if (__any_sync(FULL, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+                        for (int ks = 0; ks < NKS; ++ks) {
+                            yacc[ks][0] *= al0; yacc[ks][1] *= al1;
+                            yacc[ks][2] *= al0; yacc[ks][3] *= al1;
+                        }
+                    }
+                    // y += C^T p: p (k = tokens, n = heads) as B fragments by transposing
+                    // the 8 x 8 (token, head) blocks of the score accumulators
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        if (ngp <= 2 * mt) continue;
+                        const bool g2 = ngp > 2 * mt + 1;          // the m-tile's second token group was copied
+                        const uint32_t pb[2] = {movm_t(pack_bf16(pv[mt][0], pv[mt][1])),
+                                                movm_t(pack_bf16(pv[mt][2], pv[mt][3]))};
+#pragma unroll
+                        for (int js = 0; js < NKS; ++js) {
+                            if (2 * js >= nib) continue;
+                            uint32_t ca[4];
+                            ldsm_x4_t(ca, Cs + (((4 * v + 2 * mt + (lj >> 1)) * nib + 2 * js + (lj & 1)) * 64 + lr * 8) * 2);
+                            if (!g2) ca[2] = ca[3] = 0u;
+                            mma_bf16_16816(yacc[js], ca, pb);
                         }
                     }
                 }
@@ -848,47 +868,46 @@ SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int la
         } else {  // ZP_D
             if (mine) {
                 if (pc.first) {
-                    // merge the span's (max, sum) into the stream state of head g; keep
-                    // (beta y)^T as hi/lo A fragments in uf (u is dead by now)
-                    lsp += __shfl_xor_sync(0xffffffffu, lsp, 1);
-                    lsp += __shfl_xor_sync(0xffffffffu, lsp, 2);
-                    float be = 0.f;
-                    if (zh && msp != -INFINITY) {
-                        const float mnew = fmaxf(mm, msp);
-                        const float alpha = (mm == -INFINITY) ? 0.f : ex2(mm - mnew);
-                        be = ex2(msp - mnew);
-                        lm = lm * alpha + lsp * be;
-                        mm = mnew;
+                    // merge the span's (max, partial sum) into the stream state of heads
+                    // 2c, 2c+1; keep (beta y) as B fragments in ub (u is dead by now)
+                    float be[2] = {0.f, 0.f};
 #pragma unroll
-                        for (int n = 0; n < D / 8; ++n) {
-                            oc[n][0] *= alpha;
-                            oc[n][1] *= alpha;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const bool zz = hh ? zh1 : zh0;
+                        if (zz && msp[hh] != -INFINITY) {
+                            const float mnew = fmaxf(mh[hh], msp[hh]);
+                            const float alpha = (mh[hh] == -INFINITY) ? 0.f : ex2(mh[hh] - mnew);
+                            be[hh] = ex2(msp[hh] - mnew);
+                            lh[hh] = lh[hh] * alpha + lsp[hh] * be[hh];
+                            mh[hh] = mnew;
+#pragma unroll
+                            for (int mt = 0; mt < D / 16; ++mt) {
+                                oc[mt][hh] *= alpha;
+                                oc[mt][2 + hh] *= alpha;
+                            }
                         }
                     }
-                    // beta y in bf16 (relative 2^-9, as p on the stream path)
 #pragma unroll
                     for (int ks = 0; ks < NKS; ++ks) {
-                        const int i0 = 16 * ks + 2 * cq;
-                        uf[ks][0] = pack_bf16(i0 < rS ? yacc[2 * ks][0] * be : 0.f, i0 + 1 < rS ? yacc[2 * ks][1] * be : 0.f);
-                        uf[ks][1] = pack_bf16(i0 + 8 < rS ? yacc[2 * ks + 1][0] * be : 0.f,
-                                              i0 + 9 < rS ? yacc[2 * ks + 1][1] * be : 0.f);
+                        const int i0 = 16 * ks + g;
+                        ub[ks][0] = movm_t(pack_bf16(i0 < rS ? yacc[ks][0] * be[0] : 0.f, i0 < rS ? yacc[ks][1] * be[1] : 0.f));
+                        ub[ks][1] = movm_t(pack_bf16(i0 + 8 < rS ? yacc[ks][2] * be[0] : 0.f,
+                                                     i0 + 8 < rS ? yacc[ks][3] * be[1] : 0.f));
                     }
                 }
-                // O += (beta y)^T D over this piece's basis-row blocks
+                // O^T += D^T (beta y) over this piece's basis-row blocks
 #pragma unroll
                 for (int ks = 0; ks < NKS; ++ks) {
                     if (16 * ks < pc.r0 || 16 * ks >= pc.r0 + pc.cnt) continue;
-                    const int jl = (16 * ks - pc.r0) >> 3;
+                    const int ib = (16 * ks - pc.r0) >> 3;
                     const bool two = 16 * ks + 8 < pc.r0 + pc.cnt;
-                    const uint32_t yh[4] = {uf[ks][0], 0u, uf[ks][1], 0u};
+                    const uint32_t yb[2] = {ub[ks][0], ub[ks][1]};
 #pragma unroll
-                    for (int qd = 0; qd < D / 16; ++qd) {
-                        uint32_t vb[4];
-                        ldsm_x4_t(vb, zs + (((jl + (mi & 1)) * DB + 2 * qd + (mi >> 1)) * 64 + lr * 8) * 2);
-                        const uint32_t b0[2] = {vb[0], two ? vb[1] : 0u};
-                        const uint32_t b1[2] = {vb[2], two ? vb[3] : 0u};
-                        mma_bf16_16816(oc[2 * qd], yh, b0);
-                        mma_bf16_16816(oc[2 * qd + 1], yh, b1);
+                    for (int mt = 0; mt < D / 16; ++mt) {
+                        uint32_t da[4];
+                        ldsm_x4_t(da, zs + (((ib + (lj >> 1)) * DB + 2 * mt + (lj & 1)) * 64 + lr * 8) * 2);
+                        if (!two) da[2] = da[3] = 0u;
+                        mma_bf16_16816(oc[mt], da, yb);
                     }
                 }
             }
@@ -983,8 +1002,9 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     bool ok = true;
 
     // stream state of a consumer warp
-    //   tensor-core path: lane (g = lane/4, c = lane%4) holds head g's (m, l) and the
-    //   accumulator fragments oc[n][0..1] = O[g][8n + 2c .. 8n + 2c + 1]
+    //   tensor-core path: lane (g = lane/4, c = lane%4) holds heads 2c, 2c+1: their
+    //   running max mh, partial sums lh (over the lane's own rows) and the O^T
+    //   accumulator fragments oc[t] = O[2c + (e & 1)][16t + g + 8 (e >> 1)]
     //   CUDA-core path:   every lane holds (m, l) of all heads and o[h][dims of lane]
     float m_run[G], l_run[G], o[G][DPL];
 #pragma unroll
@@ -995,11 +1015,11 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         for (int i = 0; i < DPL; ++i) o[h][i] = 0.f;
     }
     float m_lane = -INFINITY;
-    uint32_t qa[C::MMA ? D / 16 : 1][2];      // tensor-core path: q fragments (stream and zoom)
-    float oc[C::MMA ? D / 8 : 1][4];
-    float mm = -INFINITY, lm = 0.f;           // tensor-core path: this lane's head
+    uint32_t qb[C::MMA ? D / 16 : 1][2];      // tensor-core path: q as B fragments (stream and zoom)
+    float oc[C::MMA ? D / 16 : 1][4];
+    float mh[2] = {-INFINITY, -INFINITY}, lh[2] = {0.f, 0.f};
 #pragma unroll
-    for (int n = 0; n < (C::MMA ? D / 8 : 1); ++n) oc[n][0] = oc[n][1] = oc[n][2] = oc[n][3] = 0.f;
+    for (int n = 0; n < (C::MMA ? D / 16 : 1); ++n) oc[n][0] = oc[n][1] = oc[n][2] = oc[n][3] = 0.f;
 
     if (warp == kNW) {
         // ------------------------------------------------------------ producer
@@ -1063,22 +1083,27 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         }
     } else if constexpr (C::MMA) {
         // ------------------------------------------------ consumers, tensor cores
-        const int g = lane >> 2, c = lane & 3;
-        const bool gv = g < G;
-        const float th = gv ? a.theta[(int64_t)l * a.Hq + kvh * G + g] : INFINITY;
-        // q as m16n8k16 A fragments (rows = heads, zero-padded to 16): a0, a2 per k-step
+        // Each warp owns 16 rows of every 64-row tile. S = K q^T (M = the 16 rows,
+        // N = 8 query heads, K = d); online softmax per head over the rows;
+        // O^T += V^T P^T (M = 16 dims, N = heads, K = the 16 rows), P^T reaching the
+        // B-fragment layout through 8 x 8 register transposes. Heads >= G are zero
+        // columns. The q.kbar accumulator of a span row is both its routing logit
+        // and its coarse attention logit.
+        constexpr uint32_t FULL = 0xffffffffu;
+        const int g = lane >> 2, c = lane & 3, lj = lane >> 3, lr = lane & 7;
+        const float th0 = 2 * c < G ? a.theta[(int64_t)l * a.Hq + kvh * G + 2 * c] : INFINITY;
+        const float th1 = 2 * c + 1 < G ? a.theta[(int64_t)l * a.Hq + kvh * G + 2 * c + 1] : INFINITY;
         {
-            const uint32_t* qp = reinterpret_cast<const uint32_t*>(
-                a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G + (gv ? g : 0)) * C::ROWB);
+            const uint32_t* qp = reinterpret_cast<const uint32_t*>(sm.qs + (g < G ? g : 0) * C::ROWB);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                qa[kk][0] = gv ? qp[(16 * kk + 2 * c) / 2] : 0u;
-                qa[kk][1] = gv ? qp[(16 * kk + 8 + 2 * c) / 2] : 0u;
+                qb[kk][0] = g < G ? lds_u32(qp + 8 * kk + c) : 0u;
+                qb[kk][1] = g < G ? lds_u32(qp + 8 * kk + 4 + c) : 0u;
             }
         }
-        int qn = 0;
-        int* myq = sm.zq + warp * a.qcap;
         const int rbase = warp * R;                       // 16 rows of each tile
+        const int krow = rbase + lr + ((lj & 1) << 3);    // this lane's ldmatrix row for K
+        const int vrow = rbase + lr + ((lj >> 1) << 3);   // ... and for V
         for (int i = 0; i < ntiles && ok; ++i) {
             const int s = i % NS;
             if (!mbar_wait(&sm.full[s], (i / NS) & 1)) {
@@ -1091,121 +1116,88 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
             const int S0 = s0 + (i - nta) * TR;
             const int trows = anchor_tile ? min(TR, a1 - (a0 + i * TR)) : min(TR, s1 - S0);
             if (rbase < trows) {
-                // ---- logits: q . K^T for the warp's 16 rows (two n-tiles of 8)
-                float acc[2][4];
+                // ---- S for the warp's 16 rows; two partial sums over even / odd k-steps
+                float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-                    const int row = rbase + 8 * nt + (lane & 7);
-#pragma unroll
-                    for (int p = 0; p < D / 32; ++p) {
-                        const int chunk = (p & 1) * 4 + (lane >> 3);
-                        uint32_t kb[4];
-                        ldsm_x4(kb, st + (p >> 1) * 8192 + row * 128 + ((chunk ^ (row & 7)) << 4));
-                        const uint32_t a0f[4] = {qa[2 * p][0], 0u, qa[2 * p][1], 0u};
-                        const uint32_t a1f[4] = {qa[2 * p + 1][0], 0u, qa[2 * p + 1][1], 0u};
-                        const uint32_t b0[2] = {kb[0], kb[1]};
-                        const uint32_t b1[2] = {kb[2], kb[3]};
-                        mma_bf16_16816(acc[nt], a0f, b0);
-                        mma_bf16_16816(acc[nt], a1f, b1);
-                    }
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int chunk = 2 * (kk & 3) + (lj >> 1);
+                    uint32_t ka[4];
+                    ldsm_x4(ka, st + (kk >> 2) * 8192 + krow * 128 + ((chunk ^ (krow & 7)) << 4));
+                    const uint32_t qf[2] = {qb[kk][0], qb[kk][1]};
+                    mma_bf16_16816((kk & 1) ? sb : sa, ka, qf);
                 }
-                // ---- routing, zoom decisions, logits in the log2 domain
-                float lg[2][2];
+                // sc[e]: row rbase + g + 8 (e >> 1), head 2c + (e & 1)
+                float lg[4];
                 if (anchor_tile) {
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int tk = rbase + 8 * nt + 2 * c + e;
-                            lg[nt][e] = (gv && tk < trows) ? acc[nt][e] * sl2 : -INFINITY;
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        const int tk = rbase + g + ((e >> 1) << 3);
+                        lg[e] = (2 * c + (e & 1) < G && tk < trows) ? (sa[e] + sb[e]) * sl2 : -INFINITY;
+                    }
                 } else {
                     const float* invn = reinterpret_cast<const float*>(st + 2 * C::TILE);
                     const float* lsv = invn + TR;
-                    uint32_t zbal[2][2];
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const int tk = rbase + g + 8 * rr;
+                        const bool rv = tk < trows;
+                        const float inv = rv ? lds_f32(invn + tk) : 0.f;
+                        const float ls = rv ? lds_f32(lsv + tk) : 0.f;
+                        const int SL = S0 + tk;
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int tk = rbase + 8 * nt + 2 * c + e;
-                            const bool valid = gv && tk < trows;
-                            const float x = acc[nt][e];
-                            const float ls = lsv[tk];
-                            const float ell = fmaf(x * invn[tk], a.scale, ls);     // Eq. (5) pre-sigmoid
-                            const bool z = valid && (ell > th);                    // Eq. (9)
-                            const int SL = S0 + tk;
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int e = 2 * rr + hh, h = 2 * c + hh;
+                            const bool valid = rv && h < G;
+                            const float x = sa[e] + sb[e];
+                            const float ell = fmaf(x * inv, a.scale, ls);          // Eq. (5) pre-sigmoid
+                            const bool z = valid && (ell > (hh ? th1 : th0));      // Eq. (9)
                             if (valid && a.route_logits)
-                                a.route_logits[(((int64_t)b * a.L + l) * a.Hq + kvh * G + g) * a.m_cap + SL] = ell;
-                            if (z) atomicOr(&sm.zw[g * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
-                            zbal[nt][e] = __ballot_sync(0xffffffffu, z);
-                            lg[nt][e] = (valid && !z) ? fmaf(x, a.scale, ls) * kLog2e : -INFINITY;
+                                a.route_logits[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.m_cap + SL] = ell;
+                            if (z) atomicOr(&sm.zw[h * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
+                            lg[e] = (valid && !z) ? fmaf(x, a.scale, ls) * kLog2e : -INFINITY;
                         }
-                    if (!route_only) {
-                        // queue every span of the warp's 16 rows that some head zooms
-                        const int t = lane & 15;
-                        const int tnt = t >> 3, tc = (t & 7) >> 1, te = t & 1;
-                        const uint32_t zb = tnt ? (te ? zbal[1][1] : zbal[1][0]) : (te ? zbal[0][1] : zbal[0][0]);
-                        uint32_t hm = 0u;
-#pragma unroll
-                        for (int h = 0; h < G; ++h) hm |= ((zb >> (4 * h + tc)) & 1u) << h;
-                        const bool has = lane < 16 && rbase + t < trows && hm != 0u;
-                        const uint32_t rows_with = __ballot_sync(0xffffffffu, has);
-                        if (has) {
-                            const int pos = qn + __popc(rows_with & ((1u << lane) - 1u));
-                            if (pos < a.qcap) myq[pos] = (S0 + rbase + t) | (int)(hm << 24);
-                        }
-                        qn += __popc(rows_with);
                     }
                 }
                 if (!route_only) {
-                    // ---- online softmax for head g over the warp's 16 rows
-                    float mx = fmaxf(fmaxf(lg[0][0], lg[0][1]), fmaxf(lg[1][0], lg[1][1]));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                    const float mnew = fmaxf(mm, mx);
-                    const float alpha = (mnew == -INFINITY) ? 1.f : exp2f(mm - mnew);
-                    float p[2][2];
+                    // ---- online softmax of heads 2c, 2c+1 over the warp's 16 rows
+                    float mx0 = fmaxf(lg[0], lg[2]), mx1 = fmaxf(lg[1], lg[3]);
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int o = 4; o < 32; o <<= 1) {
+                        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, o));
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, o));
+                    }
+                    const float mn0 = fmaxf(mh[0], mx0), mn1 = fmaxf(mh[1], mx1);
+                    const float al0 = (mn0 == -INFINITY) ? 1.f : ex2(mh[0] - mn0);
+                    const float al1 = (mn1 == -INFINITY) ? 1.f : ex2(mh[1] - mn1);
+                    const float r0 = (mn0 == -INFINITY) ? 0.f : mn0, r1 = (mn1 == -INFINITY) ? 0.f : mn1;
+                    const float p0 = ex2(lg[0] - r0), p1 = ex2(lg[1] - r1), p2 = ex2(lg[2] - r0), p3 = ex2(lg[3] - r1);
+                    lh[0] = fmaf(lh[0], al0, p0 + p2);
+                    lh[1] = fmaf(lh[1], al1, p1 + p3);
+                    mh[0] = mn0;
+                    mh[1] = mn1;
+                    if (__any_sync(FULL, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) p[nt][e] = (lg[nt][e] == -INFINITY) ? 0.f : exp2f(lg[nt][e] - mnew);
-                    float ps = p[0][0] + p[0][1] + p[1][0] + p[1][1];
-                    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-                    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-                    lm = fmaf(lm, alpha, ps);
-                    mm = mnew;
-                    if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-                        for (int n = 0; n < D / 8; ++n) {
-                            oc[n][0] *= alpha;
-                            oc[n][1] *= alpha;
+                        for (int t = 0; t < D / 16; ++t) {
+                            oc[t][0] *= al0; oc[t][1] *= al1;
+                            oc[t][2] *= al0; oc[t][3] *= al1;
                         }
                     }
-                    // ---- O += P V (P as the A fragment: k = the 16 rows)
-                    const uint32_t pa[4] = {pack_bf16(p[0][0], p[0][1]), 0u, pack_bf16(p[1][0], p[1][1]), 0u};
+                    // ---- O^T += V^T P^T, 16 dims at a time
+                    const uint32_t pb[2] = {movm_t(pack_bf16(p0, p1)), movm_t(pack_bf16(p2, p3))};
                     const unsigned char* vt = st + C::TILE;
-                    const int mi = lane >> 3;
-                    const int vrow = rbase + (lane & 7) + ((mi & 1) << 3);
 #pragma unroll
-                    for (int qd = 0; qd < D / 16; ++qd) {
-                        const int chunk = (qd & 3) * 2 + (mi >> 1);
-                        uint32_t vb[4];
-                        ldsm_x4_t(vb, vt + (qd >> 2) * 8192 + vrow * 128 + ((chunk ^ (vrow & 7)) << 4));
-                        const uint32_t b0[2] = {vb[0], vb[1]};
-                        const uint32_t b1[2] = {vb[2], vb[3]};
-                        mma_bf16_16816(oc[2 * qd], pa, b0);
-                        mma_bf16_16816(oc[2 * qd + 1], pa, b1);
+                    for (int t = 0; t < D / 16; ++t) {
+                        const int chunk = 2 * (t & 3) + (lj & 1);
+                        uint32_t va[4];
+                        ldsm_x4_t(va, vt + (t >> 2) * 8192 + vrow * 128 + ((chunk ^ (vrow & 7)) << 4));
+                        mma_bf16_16816(oc[t], va, pb);
                     }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[s]);
         }
-        if (lane == 0) {
-            sm.qcnt[warp] = ok ? min(qn, a.qcap) : 0;
-            if (!ok) *sm.sfail = 1;
-        }
+        if (lane == 0 && !ok) *sm.sfail = 1;
     } else {
         // ------------------------------------------------ consumers, CUDA cores
         const int rL = lane / G, hL = lane % G;
@@ -1326,14 +1318,14 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     __syncthreads();    // the stream is done: the stage ring is free, the zoom queues are complete
 
     if constexpr (C::MMA) {
-        const int nq = sm.qcnt[0] + sm.qcnt[1] + sm.qcnt[2] + sm.qcnt[3];
-        if (!route_only && nq > 0 && *sm.sfail == 0) {     // uniform over the CTA
-            if (warp == kNW) zoom_produce<D, G>(a, sm, lane, b, l, kvh, nq);
-            else {
-                const int g = lane >> 2;
-                const uint32_t* qrow = g < G ? reinterpret_cast<const uint32_t*>(sm.qs + g * C::ROWB) : nullptr;
-                zoom_consume<D, G, RM>(a, sm, warp, lane, qrow, mm, lm, oc);
-            }
+        // any zoomed span in this CTA's range (the same answer in every warp)
+        const int nwords = s1 > s0 ? (s1 - s0 + 31) >> 5 : 0;
+        bool zany = false;
+        for (int i = lane; i < G * zwords; i += 32) zany = zany || sm.zw[i] != 0u;
+        zany = __any_sync(0xffffffffu, zany);
+        if (!route_only && zany && *sm.sfail == 0) {     // uniform over the CTA
+            if (warp == kNW) zoom_produce<D, G>(a, sm, lane, b, l, kvh, s0, nwords, zwords);
+            else zoom_consume<D, G, RM>(a, sm, warp, lane, qb, mh, lh, oc);
         }
     } else {
         if (!route_only && warp < kNW && ok) zoom_phase<DT, D, G>(a, sm, warp, lane, b, l, kvh, m_run, l_run, o, m_lane);
@@ -1341,16 +1333,27 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     __syncthreads();    // zoom slots are dead: the ring takes the partial states
     if (!route_only && warp < kNW) {
         if constexpr (C::MMA) {
-            const int g = lane >> 2, c = lane & 3;
-            if (g < G) {
-                if (c == 0) {
-                    sm.st_m[warp * G + g] = mm;
-                    sm.st_l[warp * G + g] = lm;
-                }
+            // the partial sums of each head column over its 8 lanes
+            float l0 = lh[0], l1 = lh[1];
 #pragma unroll
-                for (int n = 0; n < D / 8; ++n) {
-                    sm.st_o[(warp * G + g) * D + 8 * n + 2 * c] = oc[n][0];
-                    sm.st_o[(warp * G + g) * D + 8 * n + 2 * c + 1] = oc[n][1];
+            for (int o = 4; o < 32; o <<= 1) {
+                l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+            }
+            const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int h = 2 * c + hh;
+                if (h < G) {
+                    if (g == 0) {
+                        sm.st_m[warp * G + h] = mh[hh];
+                        sm.st_l[warp * G + h] = hh ? l1 : l0;
+                    }
+#pragma unroll
+                    for (int t = 0; t < D / 16; ++t) {
+                        sm.st_o[(warp * G + h) * D + 16 * t + g] = oc[t][hh];
+                        sm.st_o[(warp * G + h) * D + 16 * t + g + 8] = oc[t][2 + hh];
+                    }
                 }
             }
         } else {
@@ -1522,7 +1525,7 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     a.region = d.region_elems; a.scale = d.scale;
     a.B = d.B; a.L = d.L; a.l0 = d.l0; a.Lr = Lr; a.Hq = d.Hq; a.Hkv = d.Hkv; a.a_cap = d.a_cap; a.m_cap = d.m_cap;
     a.rank = d.rank; a.phase = d.phase; a.nsplit = p.nsplit; a.sch_max = p.span_chunk;
-    a.qcap = ((p.span_chunk + C::TR - 1) / C::TR) * C::R;
+    a.qcap = C::MMA ? 0 : ((p.span_chunk + C::TR - 1) / C::TR) * C::R;   // the tensor-core path reads the bitmask
     a.mw = d.m_cap / 32;
     const size_t smem = decode_smem_bytes<DT, D, G>(a.sch_max, a.qcap);
     if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
