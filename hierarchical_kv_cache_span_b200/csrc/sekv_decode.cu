@@ -56,7 +56,7 @@ struct DecCfg {
     static constexpr int META = 2 * TR * 4;                 // inv_norm + logS of a span tile
     static constexpr int STAGE0 = 2 * TILE + META;
     static constexpr int STAGE = MMA ? (STAGE0 + 1023) / 1024 * 1024 : STAGE0;
-    static constexpr int NS0 = (MMA ? 102 * 1024 : 64 * 1024) / STAGE;    // 2 CTAs / SM on the bf16 path
+    static constexpr int NS0 = (MMA ? 68 * 1024 : 64 * 1024) / STAGE;     // 3 CTAs / SM on the bf16 path
     static constexpr int NS = NS0 < 2 ? 2 : (NS0 > 6 ? 6 : NS0);   // ring depth
     static constexpr int YPL = kRMax * G / 32;              // y entries per lane (fp32 zoom)
     static constexpr int WSCR = MMA ? 0 : (64 * G) + 2 * kRMax * G;   // per-warp scratch floats (fp32 zoom)
@@ -936,7 +936,7 @@ SEKV_DEV void store_state_lanes(const DecSmem& sm, int idx, int lane, const floa
 }
 
 template <int DT, int D, int G, int RM>
-__global__ void __launch_bounds__((kNW + 1) * 32, DT == SEKV_BF16 ? 2 : 3)
+__global__ void __launch_bounds__((kNW + 1) * 32, 3)
 decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     using C = DecCfg<DT, D, G>;
     constexpr int DPL = C::DPL, R = C::R, TR = C::TR, NS = C::NS;
