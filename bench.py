@@ -53,6 +53,30 @@ def parse_args(argv=None):
 
 
 # ---------------------------------------------------------------------------
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_attend_c3_4layers.txt")
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes (read + write) per ATTEND launch from the committed ncu summary, or
+    None when the summary covers another workload or the decode source has changed
+    since the counters were taken."""
+    import hashlib
+    try:
+        with open(PROFILE_SUMMARY) as f:
+            text = f.read()
+        with open(os.path.join(ROOT, "hierarchical_kv_cache_span_b200", "csrc", "sekv_decode.cu"), "rb") as f:
+            h16 = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if f"decode source sha256[:16] = {h16}" not in text:
+        return None
+    key = f"traffic_per_launch_bytes {workload} = "
+    for line in text.splitlines():
+        if line.startswith(key):
+            return int(line[len(key):].strip())
+    return None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -480,6 +504,8 @@ def run_sekv(args, rank, world, local_rank):
                "oracle_build_s_per_unit": statistics.mean(t_build)}
 
     launches_per_step = 3 if cold else 2
+    from sekv_synth import WORKLOADS as _WL
+    full_size = (wl.L, wl.n) == (_WL[wl.name].L, _WL[wl.name].n)
     kv_total = kv_bytes
     out = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": steps, "warmup": warm,
@@ -497,7 +523,9 @@ def run_sekv(args, rank, world, local_rank):
         "route_us": statistics.mean(route_ms) * 1e3,
         "zoom_rate": zr,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak,
+                     "traffic": profiled_traffic(wl.name) if full_size else None,
+                     "traffic_unit": "DRAM bytes read + written per ATTEND launch (ncu, profiles/)",
                      "kernel": "sekv_decode_attn ATTEND call (decode_kernel + merge_kernel)",
                      "peak_source": peak_src, "frac_of_8TBps_nominal": achieved / 8000.0},
         "prefill_build": build,
