@@ -245,40 +245,77 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
     // previous step's ATTEND (which ran earlier on `compute`)
     if ((e = cudaStreamSynchronize(cs)) != cudaSuccess) return cuda_fail(e, "fetch: compute stream");
 
-    struct Run { int64_t src, dst, elems; };
-    std::vector<Run> runs;
-    std::vector<uint32_t> uni(mw);
+    // A span's blocks sit at the same offset blk_off[b][S] of every layer's region,
+    // so a run of consecutive spans zoomed in a run of consecutive layers is one
+    // pitched rectangle of the home: width = the spans' blocks, height = the
+    // layers, source pitch = the region. The copy engine pays a fixed cost per
+    // copy (a few microseconds), so one rectangle per (span run, layer run)
+    // instead of one copy per (span run, layer) is what keeps the fetch near the
+    // PCIe rate.
+    struct Rect { int64_t src, dst, width, height; };
+    std::vector<Rect> rects;
+    std::vector<uint32_t> uni;
+    std::vector<uint64_t> lmask;
     int64_t bump = 0, spans = 0;
+    int dev = 0, max_pitch = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&max_pitch, cudaDevAttrMaxPitch, dev) != cudaSuccess)
+        max_pitch = 0;
+    const bool pitched = (int64_t)max_pitch >= d->region_elems * es;
     for (int b = 0; b < d->B; ++b) {
         const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
         const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
         for (int l = d->l0; l < d->l1; ++l) {
             int64_t* sl = d->slot_host + ((int64_t)b * d->L + l) * d->m_cap;
             for (int S = 0; S < d->m_cap; ++S) sl[S] = -1;
-            std::fill(uni.begin(), uni.end(), 0u);
-            const uint32_t* zm = d->zmask_host + ((int64_t)b * d->L + l) * d->Hq * mw;
-            for (int h = 0; h < d->Hq; ++h)
-                for (int w = 0; w < mw; ++w) uni[w] |= zm[h * mw + w];
-            const int64_t region0 = ((int64_t)b * d->L + l) * d->region_elems;
+        }
+        // layers in chunks of 64: lmask[S] bit j = span S zoomed (by any head) in layer lc + j
+        for (int lc = d->l0; lc < d->l1; lc += 64) {
+            const int nl = d->l1 - lc < 64 ? d->l1 - lc : 64;
+            lmask.assign(m, 0ull);
+            uni.assign(mw, 0u);
+            for (int j = 0; j < nl; ++j) {
+                std::fill(uni.begin(), uni.end(), 0u);
+                const uint32_t* zm = d->zmask_host + ((int64_t)b * d->L + lc + j) * d->Hq * mw;
+                for (int h = 0; h < d->Hq; ++h)
+                    for (int w = 0; w < mw; ++w) uni[w] |= zm[h * mw + w];
+                for (int S = 0; S < m; ++S)
+                    if ((uni[S >> 5] >> (S & 31)) & 1u) lmask[S] |= 1ull << j;
+            }
             int S = 0;
             while (S < m) {
-                if (!((uni[S >> 5] >> (S & 31)) & 1u)) { ++S; continue; }
+                if (!lmask[S]) { ++S; continue; }
                 const int Sa = S;
-                while (S < m && ((uni[S >> 5] >> (S & 31)) & 1u)) {
-                    sl[S] = bump + (bo[S] - bo[Sa]);
-                    ++S;
-                    ++spans;
+                const uint64_t mk = lmask[S];
+                while (S < m && lmask[S] == mk) ++S;          // spans [Sa, S) share the layer set
+                const int64_t width = bo[S] - bo[Sa];
+                spans += (int64_t)(S - Sa) * __builtin_popcountll(mk);
+                int j = 0;
+                while (j < nl) {
+                    if (!((mk >> j) & 1ull)) { ++j; continue; }
+                    const int ja = j;
+                    while (j < nl && ((mk >> j) & 1ull)) ++j;  // layers [lc + ja, lc + j)
+                    const int hgt = j - ja;
+                    for (int q = 0; q < hgt; ++q) {
+                        int64_t* sl = d->slot_host + ((int64_t)b * d->L + lc + ja + q) * d->m_cap;
+                        for (int t = Sa; t < S; ++t) sl[t] = bump + (int64_t)q * width + (bo[t] - bo[Sa]);
+                    }
+                    const int64_t src = ((int64_t)b * d->L + lc + ja) * d->region_elems + bo[Sa];
+                    if (pitched) {
+                        rects.push_back({src, bump, width, hgt});
+                    } else {
+                        for (int q = 0; q < hgt; ++q)
+                            rects.push_back({src + (int64_t)q * d->region_elems, bump + (int64_t)q * width, width, 1});
+                    }
+                    bump += (int64_t)hgt * width;
                 }
-                const int64_t elems = bo[S] - bo[Sa];
-                runs.push_back({region0 + bo[Sa], bump, elems});
-                bump += elems;
             }
         }
     }
     if (d->stats) {
         d->stats[0] = bump * es;
         d->stats[1] = spans;
-        d->stats[2] = (int64_t)runs.size();
+        d->stats[2] = (int64_t)rects.size();
         d->stats[3] = 0;
     }
     if (bump > d->arena_elems) {
@@ -289,10 +326,13 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
     }
     const char* home = reinterpret_cast<const char*>(d->home);
     char* arena = reinterpret_cast<char*>(d->arena);
-    for (const Run& r : runs) {
-        if ((e = cudaMemcpyAsync(arena + r.dst * es, home + r.src * es, r.elems * es, cudaMemcpyHostToDevice,
-                                 xs)) != cudaSuccess)
-            return cuda_fail(e, "fetch: basis copy");
+    for (const Rect& r : rects) {
+        if (r.height == 1)
+            e = cudaMemcpyAsync(arena + r.dst * es, home + r.src * es, r.width * es, cudaMemcpyHostToDevice, xs);
+        else
+            e = cudaMemcpy2DAsync(arena + r.dst * es, r.width * es, home + r.src * es, d->region_elems * es,
+                                  r.width * es, r.height, cudaMemcpyHostToDevice, xs);
+        if (e != cudaSuccess) return cuda_fail(e, "fetch: basis copy");
     }
     for (int b = 0; b < d->B; ++b) {
         const int64_t o = ((int64_t)b * d->L + d->l0) * d->m_cap;

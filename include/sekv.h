@@ -254,11 +254,14 @@ typedef struct sekv_fetch_desc {
 /* Copy the bases of every span that any query head of (b, l) zooms, for layers
  * [l0, l1), into the arena, and point the slot table at them (-1 elsewhere).
  * Order: zmask is read back on `compute` (the host waits for it); the copies
- * (one cudaMemcpyAsync per run of consecutive zoomed spans of a layer) and the
- * slot-table upload go on `copy`; `done` is recorded on `copy`. The caller makes
- * `compute` wait on `done` before ATTEND. Arena contents from earlier calls are
- * overwritten. Returns SEKV_ERR_CAPACITY (nothing copied) if the zoomed bases
- * exceed arena_elems. */
+ * and the slot-table upload go on `copy`; `done` is recorded on `copy`. The
+ * caller makes `compute` wait on `done` before ATTEND. A run of consecutive
+ * spans zoomed in the same layers is one rectangle of the home (its blocks sit
+ * at the same offset of every layer's region); each rectangle is one
+ * cudaMemcpy2DAsync (cudaMemcpyAsync for a single layer, or per layer when the
+ * region pitch exceeds the device's maximum copy pitch). stats[2] counts the
+ * copies. Arena contents from earlier calls are overwritten. Returns
+ * SEKV_ERR_CAPACITY (nothing copied) if the zoomed bases exceed arena_elems. */
 sekv_status sekv_fetch_bases(const sekv_fetch_desc* desc, sekv_stream_t compute,
                              sekv_stream_t copy, sekv_event_t done);
 
