@@ -123,12 +123,22 @@ class SpanCache:
               l1=None, stream=None):
         d = self.build_desc(H, K, V, alpha, window, wmode, max_sweeps, steps, l0, l1)
         S.check(S.sekv_build_spans(d, _stream(stream)), "sekv_build_spans")
+        if steps & S.SEKV_BUILD_SCAN:
+            self._rows_hint = None          # re-read from the new counts at the next decode_desc
         return self
+
+    @property
+    def rows_hint(self) -> int:
+        """Largest anchors + spans over the batch (one device read per build)."""
+        if getattr(self, "_rows_hint", None) is None:
+            self._rows_hint = int((self.a_count.clamp(max=self.a_cap) +
+                                   self.m_count.clamp(max=self.m_cap)).max().item())
+        return self._rows_hint
 
     # ------------------------------------------------------------------ decode
     def decode_desc(self, q, theta, phase=S.SEKV_FUSED, scale=None, O=None, lse=None, zmask=None,
                     route_logits=None, nsplit=0, slot=None, arena=None, l0=0, l1=None,
-                    workspace=None) -> S.sekv_decode_desc:
+                    workspace=None, rows_hint=None) -> S.sekv_decode_desc:
         d = S.sekv_decode_desc()
         d.q = _ptr(q)
         d.a_count, d.m_count, d.span_beg, d.span_end = (_ptr(self.a_count), _ptr(self.m_count),
@@ -146,9 +156,10 @@ class SpanCache:
         d.B, d.L, d.Hq, d.Hkv, d.d, d.dtype = self.B, self.L, self.Hq, self.Hkv, self.d, self.code
         d.l0, d.l1 = l0, self.L if l1 is None else l1
         d.a_cap, d.m_cap, d.rank, d.phase, d.nsplit = self.a_cap, self.m_cap, self.rank, phase, nsplit
+        d.rows_hint = self.rows_hint if rows_hint is None else int(rows_hint)
         need = S.sekv_decode_workspace_bytes(d)
         if workspace is None:
-            key = (d.l0, d.l1, nsplit)
+            key = (d.l0, d.l1, nsplit, d.rows_hint)
             ws = self._dws.get(key)
             if ws is None or ws.numel() < need:
                 ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)

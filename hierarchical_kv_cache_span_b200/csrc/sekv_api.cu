@@ -92,6 +92,7 @@ sekv_status check_decode(const sekv_decode_desc* d, bool with_workspace = true) 
     SEKV_REQUIRE(d->phase >= SEKV_FUSED && d->phase <= SEKV_ATTEND, "decode: phase %d", d->phase);
     SEKV_REQUIRE(d->a_cap >= 1 && d->m_cap >= 32 && d->m_cap % 32 == 0, "decode: a_cap >= 1, m_cap % 32 == 0");
     SEKV_REQUIRE(d->m_cap < (1 << 24), "decode: m_cap must be < 2^24");
+    SEKV_REQUIRE(d->nsplit >= 0 && d->rows_hint >= 0, "decode: nsplit and rows_hint must be >= 0");
     if (!sekv::decode_supported(*d))
         return fail(SEKV_ERR_UNSUPPORTED, "decode: d=%d, Hq/Hkv=%d, rank=%d, dtype=%d not compiled", d->d,
                     d->Hq / d->Hkv, d->rank, d->dtype);

@@ -1448,23 +1448,39 @@ DecodePlan plan_decode(const sekv_decode_desc& d) {
     int ns = d.nsplit;
     const int max_ns = d.m_cap / 32 > 0 ? d.m_cap / 32 : 1;
     if (ns <= 0) {
-        // Fill whole waves of resident CTAs (3 per SM for the bf16 / d=128 / G=4
-        // variant): the smallest split count with >= 1.5 waves and >= 85% of the
-        // last wave busy; otherwise the best such ratio. Splits keep >= ~128 rows.
-        const double slots = 3.0 * num_sms();
+        const double slots = 3.0 * num_sms();     // resident CTAs (3 per SM on the bf16 / d=128 variant)
         int lim = (int)((d.a_cap + d.m_cap) / 128);
         lim = lim < 1 ? 1 : (lim > max_ns ? max_ns : lim);
         if (lim > 64) lim = 64;
-        int best = 1;
-        double best_score = -1.0;
-        for (int c = 1; c <= lim; ++c) {
-            const double waves = (double)units * c / slots;
-            const double eff = waves / std::ceil(waves);
-            if (waves >= 1.5 && eff >= 0.85) { best = c; break; }
-            const double score = eff * (waves < 2.0 ? waves / 2.0 : 1.0);
-            if (score > best_score + 1e-9) { best_score = score; best = c; }
+        if (d.rows_hint > 0) {
+            // Makespan model over ns: the grid is units * ns CTAs of rows / ns rows
+            // each plus a fixed cost (setup, partial write, merge; ~64 rows' worth),
+            // scheduled dynamically onto the resident slots, plus half a CTA of tail.
+            const double rows = (double)d.rows_hint;
+            const double o = 64.0;
+            int best = 1;
+            double best_t = 1e300;
+            for (int c = 1; c <= lim; ++c) {
+                const double cta = rows / c + o;
+                const double t = (double)units * c / slots * cta + 0.5 * cta;
+                if (t < best_t * (1.0 - 1e-9)) { best_t = t; best = c; }
+            }
+            ns = best;
+        } else {
+            // Capacities only: fill whole waves of resident CTAs: the smallest split
+            // count with >= 1.5 waves and >= 85% of the last wave busy; otherwise the
+            // best such ratio. Splits keep >= ~128 rows of the capacities.
+            int best = 1;
+            double best_score = -1.0;
+            for (int c = 1; c <= lim; ++c) {
+                const double waves = (double)units * c / slots;
+                const double eff = waves / std::ceil(waves);
+                if (waves >= 1.5 && eff >= 0.85) { best = c; break; }
+                const double score = eff * (waves < 2.0 ? waves / 2.0 : 1.0);
+                if (score > best_score + 1e-9) { best_score = score; best = c; }
+            }
+            ns = best;
         }
-        ns = best;
     }
     if (ns > max_ns) ns = max_ns;
     if (ns < 1) ns = 1;

@@ -196,6 +196,9 @@ typedef struct sekv_decode_desc {
     int32_t rank;
     int32_t phase;           /* SEKV_FUSED / SEKV_ROUTE / SEKV_ATTEND                       */
     int32_t nsplit;          /* CTAs per (b, l, kv head); 0 = automatic                    */
+    int32_t rows_hint;       /* expected anchors + spans of a sequence (e.g. the last
+                                build's counts), used by the automatic split choice;
+                                0 = unknown (the choice then assumes the capacities)   */
 } sekv_decode_desc;
 
 size_t sekv_decode_workspace_bytes(const sekv_decode_desc* desc);
