@@ -221,9 +221,23 @@ def routing_logits(qh, kbar, inv_norm, logS, scale: float) -> np.ndarray:
     return s * np.asarray(inv_norm, dtype=np.float64) * scale + np.asarray(logS, dtype=np.float64)
 
 
-def zoom_decisions(ell, theta: float) -> np.ndarray:
-    """Eq. (9): z_S = 1[sigma(l_S) > tau], i.e. l_S > theta = ln(tau/(1-tau))."""
-    return np.asarray(ell) > theta
+def zoom_decisions(ell, theta: float, budget=None) -> np.ndarray:
+    """Eq. (9): z_S = 1[sigma(l_S) > tau], i.e. l_S > theta = ln(tau/(1-tau)).
+
+    With a budget (SeKV blog 2.3, the paragraph under Eq. (9)): when more spans
+    pass the threshold than the budget allows, the spans are kept in descending
+    alpha~ order; alpha~ = sigma(l_S) is monotone in l_S, so the `budget` largest
+    logits stay. Equal logits keep the lower span index first (a reading: the
+    pages give no tie rule)."""
+    ell = np.asarray(ell, dtype=np.float64)
+    z = ell > theta
+    if budget is None or int(z.sum()) <= int(budget):
+        return z
+    passing = [int(s) for s in np.flatnonzero(z)]
+    passing.sort(key=lambda s: (-ell[s], s))       # descending logit, then lower span index
+    keep = np.zeros(z.shape, dtype=bool)
+    keep[passing[:int(budget)]] = True
+    return keep
 
 
 def decode_unit(q, Ka, Va, kbar, vbar, logS, zoom, bases, scale: float):

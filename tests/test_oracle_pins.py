@@ -430,3 +430,59 @@ def test_planted_swapped_basis_factors_are_caught():
     assert np.abs(A @ B - expect).max() < 1e-10
     A2, B2 = O.truncated_basis(X.T, 3, "f64")       # a transposed operand
     assert (A2 @ B2).shape != expect.shape or np.abs(A2 @ B2 - expect).max() > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# Zoom budget cap (SeKV blog 2.3, paragraph under Eq. (9)): keep the passing
+# spans in descending alpha~ order up to the budget.
+def test_budget_cap_worked_example():
+    # logits [0.5, 2.0, 1.0, 2.0, -1.0], theta 0: spans 0..3 pass. Descending alpha~
+    # (equivalently descending l): span 1 and span 3 (equal, lower index first), then
+    # span 2, then span 0.
+    ell = [0.5, 2.0, 1.0, 2.0, -1.0]
+    assert np.flatnonzero(O.zoom_decisions(ell, 0.0, budget=1)).tolist() == [1]
+    assert np.flatnonzero(O.zoom_decisions(ell, 0.0, budget=2)).tolist() == [1, 3]
+    assert np.flatnonzero(O.zoom_decisions(ell, 0.0, budget=3)).tolist() == [1, 2, 3]
+    assert np.flatnonzero(O.zoom_decisions(ell, 0.0, budget=4)).tolist() == [0, 1, 2, 3]
+    assert np.flatnonzero(O.zoom_decisions(ell, 0.0, budget=9)).tolist() == [0, 1, 2, 3]
+    assert not O.zoom_decisions(ell, 0.0, budget=0).any()
+    # the cap never adds a span the threshold rejected
+    assert np.flatnonzero(O.zoom_decisions(ell, 1.5, budget=3)).tolist() == [1, 3]
+
+
+def test_budget_cap_is_top_k_of_the_passing_set_brute_force():
+    """Against the definition: the kept set is the unique size-min(k, #pass) subset of
+    the passing spans such that no dropped passing span ranks before a kept one in
+    (descending logit, ascending index) order; checked by enumerating subsets."""
+    import itertools
+    rng = np.random.default_rng(11)
+    for trial in range(200):
+        m = int(rng.integers(1, 8))
+        # few distinct values so that ties are common
+        ell = rng.integers(-3, 4, size=m).astype(np.float64) / 2.0
+        theta = float(rng.choice([-10.0, -0.5, 0.0, 0.75]))
+        k = int(rng.integers(0, m + 2))
+        got = O.zoom_decisions(ell, theta, budget=k)
+        passing = [s for s in range(m) if ell[s] > theta]
+        want = None
+        for sub in itertools.combinations(passing, min(k, len(passing))):
+            dropped = [t for t in passing if t not in sub]
+            ok = all((ell[s] > ell[t]) or (ell[s] == ell[t] and s < t) for s in sub for t in dropped)
+            if ok:
+                assert want is None, "the kept set must be unique"
+                want = set(sub)
+        assert want is not None
+        assert set(np.flatnonzero(got).tolist()) == want
+
+
+def test_budget_cap_none_is_the_threshold_rule():
+    rng = np.random.default_rng(5)
+    ell = rng.standard_normal(300)
+    for theta in (-1.0, 0.0, 0.7):
+        z = O.zoom_decisions(ell, theta)
+        np.testing.assert_array_equal(O.zoom_decisions(ell, theta, budget=None), z)
+        np.testing.assert_array_equal(O.zoom_decisions(ell, theta, budget=int(z.sum())), z)
+        capped = O.zoom_decisions(ell, theta, budget=7)
+        assert capped.sum() == min(7, z.sum()) and not (capped & ~z).any()
+        # the kept logits are the 7 largest passing ones
+        np.testing.assert_allclose(np.sort(ell[capped]), np.sort(ell[z])[-7:])
