@@ -49,6 +49,9 @@ def parse_args(argv=None):
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--budget", type=int, default=0,
+                    help="zoom budget per (layer, query head), keeping the largest routing logits; 0 = none "
+                         "(the configs run without one)")
     return ap.parse_args(argv)
 
 
@@ -218,7 +221,7 @@ def zoom_rate(cache, zmask_host):
 def _oracle_unit_task(args):
     import numpy as np
     import oracle as O
-    kv_path, H, alpha, window, wmode, rank, dtype, q, theta, quantile, scale, reps = args
+    kv_path, H, alpha, window, wmode, rank, dtype, q, theta, quantile, scale, reps, budget = args
     with np.load(kv_path) as f:
         K, V = f["K"].astype(np.float64), f["V"].astype(np.float64)
     seg = O.segment(H, alpha, window)
@@ -234,14 +237,15 @@ def _oracle_unit_task(args):
     times = []
     for _ in range(reps):
         t0 = time.perf_counter()
-        z = np.stack([O.zoom_decisions(O.routing_logits(q[g], u.kbar, u.inv_norm, u.logS, scale), theta[g])
+        z = np.stack([O.zoom_decisions(O.routing_logits(q[g], u.kbar, u.inv_norm, u.logS, scale), theta[g],
+                                       budget=budget or None)
                       for g in range(q.shape[0])])
         O.decode_unit(q, u.Ka, u.Va, u.kbar, u.vbar, u.logS, z, u.bases, scale)
         times.append(time.perf_counter() - t0)
     return t_build, times
 
 
-def oracle_sample(wl, H, KV_units, q, theta, reps, workers, quantile=None):
+def oracle_sample(wl, H, KV_units, q, theta, reps, workers, quantile=None, budget=0):
     """Time the oracle on the sampled (layer, kv head) units (one per process of a
     spawn pool). K/V of each unit go through a temporary .npz file (float32 holds
     the bf16 values exactly). Returns per-unit build seconds and decode seconds."""
@@ -256,7 +260,7 @@ def oracle_sample(wl, H, KV_units, q, theta, reps, workers, quantile=None):
             np.savez(path, K=K, V=V)
             th = None if theta is None else theta[l, h * G:(h + 1) * G]
             tasks.append((path, H, wl.alpha, wl.window, wl.wmode, wl.rank, wl.dtype,
-                          q[l, h * G:(h + 1) * G], th, quantile, scale, reps))
+                          q[l, h * G:(h + 1) * G], th, quantile, scale, reps, budget))
         ctx = mp.get_context("spawn")
         saved = {k: os.environ.get(k) for k in _BLAS_ENV}
         os.environ.update({k: "1" for k in _BLAS_ENV})      # one BLAS thread per worker process
@@ -373,7 +377,7 @@ def run_sekv(args, rank, world, local_rank):
     fetcher = None
     if cold:
         # size the arena from a calibration step: 3x its zoomed bytes
-        cache.decode(qpool[0], theta, phase=P.SEKV_ROUTE, zmask=zm)
+        cache.decode(qpool[0], theta, phase=P.SEKV_ROUTE, zmask=zm, budget=args.budget)
         probe = P.ColdFetcher(cache, arena_elems=64)
         try:
             probe.fetch(zm)
@@ -387,12 +391,13 @@ def run_sekv(args, rank, world, local_rank):
     # descriptors are built once; each step copies its query into q_buf and calls the C ABI
     q_buf = torch.empty_like(qpool[0])
     sid = comp.cuda_stream
+    bud = args.budget
     if cold:
-        d_route = cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm)
+        d_route = cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud)
         d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_ATTEND, O=O, lse=lse, slot=fetcher.slot_dev,
-                                   arena=fetcher.arena)
+                                   arena=fetcher.arena, zmask=zm if bud else None, budget=bud)
     else:
-        d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_FUSED, O=O, lse=lse, zmask=zm)
+        d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_FUSED, O=O, lse=lse, zmask=zm, budget=bud)
 
     def one_step(q, rec=None):
         if q is not None:
@@ -493,7 +498,7 @@ def run_sekv(args, rank, world, local_rank):
     if want_cpu:
         qs = qpool[warm].double().cpu().numpy()[0]
         th = theta.double().cpu().numpy()
-        t_build, t_dec = oracle_sample(wl, H0, cpu_units, qs, th, reps=2, workers=workers)
+        t_build, t_dec = oracle_sample(wl, H0, cpu_units, qs, th, reps=2, workers=workers, budget=args.budget)
         per_unit = statistics.mean(min(t) for t in t_dec)
         units_total = wl.B * wl.L * wl.Hkv
         oracle_step_s = per_unit * units_total / workers
@@ -503,7 +508,9 @@ def run_sekv(args, rank, world, local_rank):
                          f"{workers} cores. Oracle build of those units: mean {statistics.mean(t_build):.2f} s/unit",
                "oracle_build_s_per_unit": statistics.mean(t_build)}
 
-    launches_per_step = 3 if cold else 2
+    # ROUTE + ATTEND + merge (cold) or FUSED + merge (hot); a budget adds the cap
+    # kernel, and on the hot path the routing pass before the capped FUSED pass
+    launches_per_step = (3 + (1 if args.budget else 0)) if cold else (2 + (2 if args.budget else 0))
     from sekv_synth import WORKLOADS as _WL
     full_size = (wl.L, wl.n) == (_WL[wl.name].L, _WL[wl.name].n)
     kv_total = kv_bytes
@@ -517,7 +524,8 @@ def run_sekv(args, rank, world, local_rank):
                    "B": wl.B, "n": wl.n, "L": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "rank": wl.rank,
                    "anchors": int(cache.a_count.sum()), "spans": int(cache.m_count.sum()),
                    "l2": f"inputs larger than L2 ({alg_bytes / 1e6:.0f} MB read per ATTEND)",
-                   "parallelism": f"replicas x{world} (no collective)"},
+                   "parallelism": f"replicas x{world} (no collective)",
+                   **({"budget": args.budget} if args.budget else {})},
         "decode_attn": {"us_per_step": attn_avg * 1e3, "steps_per_s": 1e3 / attn_avg,
                         "alg_bytes_per_step": int(alg_bytes), "GBps": achieved},
         "route_us": statistics.mean(route_ms) * 1e3,
@@ -568,7 +576,7 @@ def run_reference(args):
     theta = O.tau_to_theta(taus.numpy()) if taus is not None else None
     reps = min(5, max(1, args.steps))
     t_build, t_dec = oracle_sample(wl, H0, units, q, theta, reps=reps, workers=workers,
-                                   quantile=wl.tau_a)
+                                   quantile=wl.tau_a, budget=args.budget)
     per_unit = [min(t) for t in t_dec]
     units_total = wl.B * wl.L * wl.Hkv
     step_s = statistics.mean(per_unit) * units_total / workers

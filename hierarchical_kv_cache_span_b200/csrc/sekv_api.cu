@@ -92,7 +92,10 @@ sekv_status check_decode(const sekv_decode_desc* d, bool with_workspace = true) 
     SEKV_REQUIRE(d->phase >= SEKV_FUSED && d->phase <= SEKV_ATTEND, "decode: phase %d", d->phase);
     SEKV_REQUIRE(d->a_cap >= 1 && d->m_cap >= 32 && d->m_cap % 32 == 0, "decode: a_cap >= 1, m_cap % 32 == 0");
     SEKV_REQUIRE(d->m_cap < (1 << 24), "decode: m_cap must be < 2^24");
-    SEKV_REQUIRE(d->nsplit >= 0 && d->rows_hint >= 0, "decode: nsplit and rows_hint must be >= 0");
+    SEKV_REQUIRE(d->nsplit >= 0 && d->rows_hint >= 0 && d->budget >= 0,
+                 "decode: nsplit, rows_hint and budget must be >= 0");
+    SEKV_REQUIRE(d->budget == 0 || d->zmask, "decode: a budget needs the zmask buffer (output of ROUTE / FUSED, "
+                                             "input of ATTEND)");
     if (!sekv::decode_supported(*d))
         return fail(SEKV_ERR_UNSUPPORTED, "decode: d=%d, Hq/Hkv=%d, rank=%d, dtype=%d not compiled", d->d,
                     d->Hq / d->Hkv, d->rank, d->dtype);
@@ -103,6 +106,12 @@ sekv_status check_decode(const sekv_decode_desc* d, bool with_workspace = true) 
                  "decode: q, kbar, inv_norm, logS must be 16-byte aligned");
     if (d->phase == SEKV_ROUTE) {
         SEKV_REQUIRE(d->zmask || d->route_logits, "decode/route: zmask or route_logits required");
+        if (d->budget > 0 && !d->route_logits && with_workspace) {
+            // the capped routing pass keeps its logits in the workspace
+            const size_t need = sekv::decode_workspace_bytes(*d);
+            SEKV_REQUIRE(d->workspace && aligned(d->workspace, 256) && (size_t)d->workspace_bytes >= need,
+                         "decode/route: budget without route_logits needs a workspace of %zu bytes", need);
+        }
     } else {
         SEKV_REQUIRE(d->Ka && d->Va && d->vbar && d->arena && d->O && d->lse,
                      "decode: Ka, Va, vbar, arena, O, lse required");
@@ -205,11 +214,11 @@ sekv_status sekv_decode_attn_static(const sekv_decode_desc* d, sekv_stream_t str
     if (s != SEKV_OK) return s;
     const sekv::DecodePlan p = sekv::plan_decode(*d);
     const size_t cap = sekv::decode_static_scratch_bytes();
-    if (p.partial_bytes > cap)
+    if (p.partial_bytes + p.logit_bytes > cap)
         return fail(SEKV_ERR_CAPACITY,
                     "decode_static: this call needs %zu bytes of split-K scratch, the static array holds %zu "
                     "(fewer layers per call, a smaller batch or nsplit, or sekv_decode_attn with a workspace)",
-                    p.partial_bytes, cap);
+                    p.partial_bytes + p.logit_bytes, cap);
     cudaError_t e;
     void* scratch = sekv::decode_static_scratch(&e);
     if (!scratch) return cuda_fail(e, "decode_static: address of the static scratch");

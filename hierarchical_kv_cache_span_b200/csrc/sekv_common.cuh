@@ -222,6 +222,11 @@ SEKV_DEV void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;
 // ---------------------------------------------------------------------------
 // warp helpers
 // ---------------------------------------------------------------------------
+SEKV_DEV unsigned warp_sum_u(unsigned v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
 SEKV_DEV float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

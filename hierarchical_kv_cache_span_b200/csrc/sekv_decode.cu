@@ -105,7 +105,14 @@ struct DecArgs {
     int64_t region;
     float scale;
     int B, L, l0, Lr, Hq, Hkv, a_cap, m_cap, rank, phase, nsplit, sch_max, qcap, mw;
+    int zin;          // zoom decisions come from zmask (a capped mask) instead of l > theta
 };
+
+// zoom bit of span S for query head hq of (b, l) in a caller-supplied (capped) mask
+SEKV_DEV bool zmask_bit(const DecArgs& a, int b, int l, int hq, int S) {
+    const uint32_t w = a.zmask[(((int64_t)b * a.L + l) * a.Hq + hq) * a.mw + (S >> 5)];
+    return (w >> (S & 31)) & 1u;
+}
 
 // TMA descriptors of the anchor and summary stores (bf16 path), viewed as 2-D
 // [rows][d] tensors with 64 x 64 boxes and 128-byte swizzle.
@@ -1150,7 +1157,8 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                             const bool valid = rv && h < G;
                             const float x = sa[e] + sb[e];
                             const float ell = fmaf(x * inv, a.scale, ls);          // Eq. (5) pre-sigmoid
-                            const bool z = valid && (ell > (hh ? th1 : th0));      // Eq. (9)
+                            const bool z = valid && (a.zin ? zmask_bit(a, b, l, kvh * G + h, SL)
+                                                           : (ell > (hh ? th1 : th0)));   // Eq. (9)
                             if (valid && a.route_logits)
                                 a.route_logits[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.m_cap + SL] = ell;
                             if (z) atomicOr(&sm.zw[h * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
@@ -1253,7 +1261,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                 const float ls = reinterpret_cast<const float*>(st + 2 * C::TILE + TR * 4)[rowL];
                 const int SL = S0 + rowL;
                 const float ell = fmaf(x * invn, a.scale, ls);      // Eq. (5) pre-sigmoid logit
-                const bool z = validL && (ell > th);                // Eq. (9)
+                const bool z = validL && (a.zin ? zmask_bit(a, b, l, kvh * G + hL, SL) : (ell > th));   // Eq. (9)
                 if (validL && a.route_logits)
                     a.route_logits[(((int64_t)b * a.L + l) * a.Hq + kvh * G + hL) * a.m_cap + SL] = ell;
                 if (z) atomicOr(&sm.zw[hL * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
@@ -1363,7 +1371,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     __syncthreads();
 
     // ------------------------------------------------ zoom-mask words of this CTA
-    if (a.zmask) {
+    if (a.zmask && !a.zin) {
         const int w0 = s0 >> 5;
         const int wend = (split == a.nsplit - 1) ? a.mw : min(a.mw, w0 + (sch >> 5));
         for (int i = tid; i < G * max(0, wend - w0); i += blockDim.x) {
@@ -1423,6 +1431,138 @@ __global__ void merge_kernel(const float* part_o, const float* part_ml, float* O
     const int64_t out = ((int64_t)b * L + l0 + li) * Hq + hq;
     O[out * D + k] = Ls > 0.f ? Os / Ls : 0.f;
     if (k == 0) lse[out] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
+}
+
+// ---------------------------------------------------------------------------
+// Zoom budget cap (SeKV blog 2.3, the paragraph under Eq. (9)): when more spans
+// pass the threshold than the budget allows, keep them in descending alpha~ order
+// (monotone in the routing logit); equal logits keep the lower span index. One CTA
+// per (b, l, query head): an exact radix select (8 bits at a time, most
+// significant first) finds the budget-th largest logit among the zoomed spans,
+// then the mask keeps every larger one and the lowest-index ties up to the budget.
+// ---------------------------------------------------------------------------
+SEKV_DEV uint32_t order_key(float f) {       // larger float <=> larger key
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr unsigned kCapDirect = 512;   // zoomed spans ranked directly (O(n^2) per CTA)
+
+__global__ void __launch_bounds__(256) cap_kernel(const float* logits, uint32_t* zmask, const int32_t* m_count,
+                                                  int L, int l0, int Lr, int Hq, int m_cap, int budget) {
+    const int idx = blockIdx.x;
+    const int h = idx % Hq, li = (idx / Hq) % Lr, b = idx / (Hq * Lr);
+    const int l = l0 + li;
+    const int mw = m_cap / 32;
+    const int m = min(m_count[b], m_cap);
+    const int nw = (m + 31) >> 5;
+    uint32_t* zw = zmask + (((int64_t)b * L + l) * Hq + h) * mw;
+    const float* lg = logits + (((int64_t)b * L + l) * Hq + h) * m_cap;
+    __shared__ unsigned hist[256];
+    __shared__ unsigned red[8];
+    __shared__ uint32_t s_prefix;
+    __shared__ unsigned s_k;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // zoomed count
+    unsigned c = 0;
+    for (int w = tid; w < nw; w += blockDim.x) c += __popc(zw[w]);
+    c = warp_sum_u(c);
+    if (lane == 0) red[warp] = c;
+    __syncthreads();
+    unsigned total = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) total += red[i];
+    if (total <= (unsigned)budget) return;          // uniform over the CTA
+    if (total <= kCapDirect) {
+        // few zoomed spans: gather them, rank each by (logit descending, index
+        // ascending) against all the others, keep ranks below the budget
+        __shared__ uint32_t ck[kCapDirect];
+        __shared__ int cs[kCapDirect];
+        __shared__ unsigned cn;
+        if (tid == 0) cn = 0u;
+        __syncthreads();
+        for (int w = tid; w < nw; w += blockDim.x) {
+            uint32_t zb = zw[w];
+            while (zb) {
+                const int j = __ffs(zb) - 1;
+                zb &= zb - 1u;
+                const unsigned pos = atomicAdd(&cn, 1u);
+                ck[pos] = order_key(lg[32 * w + j]);
+                cs[pos] = 32 * w + j;
+            }
+        }
+        __syncthreads();
+        const unsigned n = cn;
+        for (int w = tid; w < nw; w += blockDim.x) zw[w] = 0u;
+        __syncthreads();
+        for (unsigned i = tid; i < n; i += blockDim.x) {
+            const uint32_t ki = ck[i];
+            const int si = cs[i];
+            unsigned rank = 0;
+            for (unsigned j = 0; j < n; ++j) rank += (ck[j] > ki) || (ck[j] == ki && cs[j] < si);
+            if (rank < (unsigned)budget) atomicOr(&zw[si >> 5], 1u << (si & 31));
+        }
+        return;
+    }
+    // radix select of the budget-th largest key among the zoomed spans
+    uint32_t prefix = 0u;
+    unsigned k = (unsigned)budget;                   // rank (1-based) within the current prefix class
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0u;
+        __syncthreads();
+        for (int S = tid; S < m; S += blockDim.x) {
+            if (!((zw[S >> 5] >> (S & 31)) & 1u)) continue;
+            const uint32_t key = order_key(lg[S]);
+            if (shift < 24 && (key >> (shift + 8)) != (prefix >> (shift + 8))) continue;
+            atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        }
+        // (the zoomed keys of a head often share their top bytes: the atomics above
+        // then serialise, which is why small sets take the direct path)
+        __syncthreads();
+        if (tid == 0) {
+            unsigned cum = 0;
+            int dg = 255;
+            for (; dg > 0; --dg) {
+                if (cum + hist[dg] >= k) break;
+                cum += hist[dg];
+            }
+            s_prefix = prefix | ((uint32_t)dg << shift);
+            s_k = k - cum;
+        }
+        __syncthreads();
+        prefix = s_prefix;
+        k = s_k;
+    }
+    // prefix is the budget-th largest key; keep the k lowest-index spans holding it
+    if (warp != 0) return;
+    unsigned carry = 0;                              // ties kept so far (span order)
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t gt = 0u, eq = 0u;
+        if (w < nw) {
+            const uint32_t zb = zw[w];
+            for (int j = 0; j < 32; ++j) {
+                if (!((zb >> j) & 1u)) continue;
+                const uint32_t key = order_key(lg[32 * w + j]);
+                if (key > prefix) gt |= 1u << j;
+                else if (key == prefix) eq |= 1u << j;
+            }
+        }
+        const unsigned ne = __popc(eq);
+        unsigned inc = ne;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned t = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += t;
+        }
+        const unsigned before = carry + inc - ne;     // ties in earlier words
+        uint32_t keep_eq = 0u;
+        if (before < k) {
+            const unsigned take = min(ne, k - before);
+            keep_eq = take >= 32 ? eq : (take == 0 ? 0u : (eq & ((2u << (__fns(eq, 0u, (int)take))) - 1u)));
+        }
+        if (w < nw) zw[w] = gt | keep_eq;
+        carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1489,10 +1629,17 @@ DecodePlan plan_decode(const sekv_decode_desc& d) {
     p.anchor_chunk = (d.a_cap + ns - 1) / ns;
     const int G = d.Hq / d.Hkv;
     p.partial_bytes = (size_t)round_up((int64_t)units * G * ns * (d.d + 2) * 4, 256);
+    // routing logits for the budget cap when the caller passes no buffer
+    p.logit_bytes = (d.budget > 0 && d.phase != SEKV_ATTEND && !d.route_logits)
+                        ? (size_t)round_up((int64_t)d.B * d.L * d.Hq * d.m_cap * 4, 256)
+                        : 0;
     return p;
 }
 
-size_t decode_workspace_bytes(const sekv_decode_desc& d) { return plan_decode(d).partial_bytes; }
+size_t decode_workspace_bytes(const sekv_decode_desc& d) {
+    const DecodePlan p = plan_decode(d);
+    return p.partial_bytes + p.logit_bytes;
+}
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -1525,7 +1672,8 @@ static bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int d) {
 }
 
 template <int DT, int D, int G, int RM>
-static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st) {
+static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st,
+                            int zin) {
     using C = DecCfg<DT, D, G>;
     const int Lr = d.l1 - d.l0;
     const int64_t units = (int64_t)d.B * Lr * d.Hkv;
@@ -1543,6 +1691,7 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     a.rank = d.rank; a.phase = d.phase; a.nsplit = p.nsplit; a.sch_max = p.span_chunk;
     a.qcap = C::MMA ? 0 : ((p.span_chunk + C::TR - 1) / C::TR) * C::R;   // the tensor-core path reads the bitmask
     a.mw = d.m_cap / 32;
+    a.zin = zin;
     const size_t smem = decode_smem_bytes<DT, D, G>(a.sch_max, a.qcap);
     if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT, D, G, RM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1576,20 +1725,29 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
 // the tensor-core zoom is compiled for basis ranks up to 16, 32 and 64; the
 // CUDA-core path handles any rank up to 64 in one variant
 template <int DT, int D, int G>
-static cudaError_t launch_r(const sekv_decode_desc& d, const DecodePlan& p, void* w, cudaStream_t st) {
-    if (DT == SEKV_BF16 && d.rank <= 16) return launch_t<DT, D, G, 16>(d, p, w, st);
-    if (DT == SEKV_BF16 && d.rank <= 32) return launch_t<DT, D, G, 32>(d, p, w, st);
-    return launch_t<DT, D, G, 64>(d, p, w, st);
+static cudaError_t launch_r(const sekv_decode_desc& d, const DecodePlan& p, void* w, cudaStream_t st, int zin) {
+    if (DT == SEKV_BF16 && d.rank <= 16) return launch_t<DT, D, G, 16>(d, p, w, st, zin);
+    if (DT == SEKV_BF16 && d.rank <= 32) return launch_t<DT, D, G, 32>(d, p, w, st, zin);
+    return launch_t<DT, D, G, 64>(d, p, w, st, zin);
 }
 
 template <int DT, int D>
-static cudaError_t launch_g(const sekv_decode_desc& d, const DecodePlan& p, void* w, cudaStream_t st) {
+static cudaError_t launch_g(const sekv_decode_desc& d, const DecodePlan& p, void* w, cudaStream_t st, int zin) {
     switch (d.Hq / d.Hkv) {
-        case 1: return launch_r<DT, D, 1>(d, p, w, st);
-        case 2: return launch_r<DT, D, 2>(d, p, w, st);
-        case 4: return launch_r<DT, D, 4>(d, p, w, st);
-        default: return launch_r<DT, D, 8>(d, p, w, st);
+        case 1: return launch_r<DT, D, 1>(d, p, w, st, zin);
+        case 2: return launch_r<DT, D, 2>(d, p, w, st, zin);
+        case 4: return launch_r<DT, D, 4>(d, p, w, st, zin);
+        default: return launch_r<DT, D, 8>(d, p, w, st, zin);
     }
+}
+
+static cudaError_t launch_pass(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st,
+                               int zin) {
+    if (d.dtype == SEKV_F32)
+        return d.d == 64 ? launch_g<SEKV_F32, 64>(d, p, partials, st, zin)
+                         : launch_g<SEKV_F32, 128>(d, p, partials, st, zin);
+    return d.d == 64 ? launch_g<SEKV_BF16, 64>(d, p, partials, st, zin)
+                     : launch_g<SEKV_BF16, 128>(d, p, partials, st, zin);
 }
 
 // ---------------------------------------------------------------------------
@@ -1626,10 +1784,24 @@ void* decode_static_scratch(cudaError_t* err) {
     return addr[dev];
 }
 
+// Without a budget: one pass (FUSED / ROUTE / ATTEND). With a budget: ROUTE and
+// FUSED run the routing pass (threshold mask + routing logits), then the cap;
+// FUSED then attends with the capped mask as input. ATTEND takes the caller's
+// (capped) mask as input.
 cudaError_t launch_decode(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st) {
-    if (d.dtype == SEKV_F32)
-        return d.d == 64 ? launch_g<SEKV_F32, 64>(d, p, partials, st) : launch_g<SEKV_F32, 128>(d, p, partials, st);
-    return d.d == 64 ? launch_g<SEKV_BF16, 64>(d, p, partials, st) : launch_g<SEKV_BF16, 128>(d, p, partials, st);
+    if (d.budget <= 0) return launch_pass(d, p, partials, st, 0);
+    if (d.phase == SEKV_ATTEND) return launch_pass(d, p, partials, st, 1);
+    sekv_decode_desc r = d;
+    r.phase = SEKV_ROUTE;
+    if (!r.route_logits) r.route_logits = reinterpret_cast<float*>(reinterpret_cast<char*>(partials) + p.partial_bytes);
+    cudaError_t e = launch_pass(r, p, partials, st, 0);
+    if (e != cudaSuccess) return e;
+    const int Lr = d.l1 - d.l0;
+    cap_kernel<<<d.B * Lr * d.Hq, 256, 0, st>>>(r.route_logits, d.zmask, d.m_count, d.L, d.l0, Lr, d.Hq, d.m_cap,
+                                                 d.budget);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (d.phase == SEKV_ROUTE) return cudaSuccess;
+    return launch_pass(d, p, partials, st, 1);
 }
 
 }  // namespace sekv

@@ -21,6 +21,7 @@ struct DecodePlan {
     int span_chunk;    // spans per split (multiple of 32)
     int anchor_chunk;  // anchors per split
     size_t partial_bytes;
+    size_t logit_bytes;  // routing logits kept for the budget cap (after the partials)
 };
 DecodePlan plan_decode(const sekv_decode_desc& d);
 size_t decode_workspace_bytes(const sekv_decode_desc& d);

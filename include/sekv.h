@@ -199,6 +199,13 @@ typedef struct sekv_decode_desc {
     int32_t rows_hint;       /* expected anchors + spans of a sequence (e.g. the last
                                 build's counts), used by the automatic split choice;
                                 0 = unknown (the choice then assumes the capacities)   */
+    int32_t budget;          /* zoom budget per (b, l, query head); 0 = none. SeKV blog
+                                2.3 (under Eq. (9)): when more spans pass the threshold,
+                                keep them in descending alpha~ (= logit) order, equal
+                                logits lower span index first. Needs zmask: ROUTE writes
+                                the capped mask; ATTEND reads it as input (no re-routing);
+                                FUSED routes, caps, then attends with the capped mask.
+                                Without route_logits the workspace holds the logits.     */
 } sekv_decode_desc;
 
 size_t sekv_decode_workspace_bytes(const sekv_decode_desc* desc);

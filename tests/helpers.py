@@ -158,7 +158,26 @@ def upload_oracle_cache(cache, segs, units, with_bases=True):
     torch.cuda.synchronize()
 
 
-def oracle_decode(q, units, segs, theta, scale, G):
+def budget_with_margin(q, units, segs, theta, scale, G, candidates=range(1, 41), delta=DELTA_L):
+    """A zoom budget k such that, for every (b, l, query head) with more than k spans
+    past theta, the k-th and (k+1)-th largest passing routing logits (oracle, fp64)
+    are at least delta apart (so the fp32 kernel and the fp64 oracle keep the same
+    spans), and at least one head is actually capped. None if no candidate works."""
+    qn = f64(q)
+    rows = []
+    for (b, l, kvh), u in units.items():
+        for g in range(G):
+            h = kvh * G + g
+            ell = O.routing_logits(qn[b, l, h], u.kbar, u.inv_norm, u.logS, scale)
+            rows.append(np.sort(ell[ell > theta[l, h]])[::-1])
+    for k in candidates:
+        capped = [r for r in rows if len(r) > k]
+        if capped and all(r[k - 1] - r[k] >= delta for r in capped):
+            return k
+    return None
+
+
+def oracle_decode(q, units, segs, theta, scale, G, budget=None):
     """O [B][L][Hq][d], lse [B][L][Hq], zoom masks {(b,l,h): bool[m]} from the oracle."""
     B, L, Hq, d = q.shape
     Oo = np.zeros((B, L, Hq, d))
@@ -170,7 +189,7 @@ def oracle_decode(q, units, segs, theta, scale, G):
         z = np.zeros((G, len(segs[b].spans)), bool)
         for g in range(G):
             ell = O.routing_logits(qg[g], u.kbar, u.inv_norm, u.logS, scale)
-            z[g] = O.zoom_decisions(ell, theta[l, kvh * G + g])
+            z[g] = O.zoom_decisions(ell, theta[l, kvh * G + g], budget=budget)
             zooms[(b, l, kvh * G + g)] = z[g]
         o, ls = O.decode_unit(qg, u.Ka, u.Va, u.kbar, u.vbar, u.logS, z, u.bases, scale)
         Oo[b, l, kvh * G:(kvh + 1) * G] = o
