@@ -49,6 +49,9 @@ def parse_args(argv=None):
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cache", action="store_true",
+                    help="cold workloads: keep fetched bases resident in a device cache across steps "
+                         "(the configs fetch every step)")
     ap.add_argument("--budget", type=int, default=0,
                     help="zoom budget per (layer, query head), keeping the largest routing logits; 0 = none "
                          "(the configs run without one)")
@@ -386,7 +389,7 @@ def run_sekv(args, rank, world, local_rank):
             need = int(probe.stats[0].item())
         es = 2 if wl.dtype == "bf16" else 4
         del probe
-        fetcher = P.ColdFetcher(cache, arena_elems=max(1 << 20, 3 * need // es))
+        fetcher = P.ColdFetcher(cache, arena_elems=max(1 << 20, 3 * need // es), keep=args.cache)
 
     # descriptors are built once; each step copies its query into q_buf and calls the C ABI
     q_buf = torch.empty_like(qpool[0])
@@ -546,6 +549,11 @@ def run_sekv(args, rank, world, local_rank):
                         "GBps": fb / (statistics.mean(fetch_ms) * 1e-3) / 1e9,
                         "copies_per_step": statistics.mean(f["copies"] for f in fetched),
                         "note": "includes the zmask read-back and the host wait for the routing result"}
+        if args.cache:
+            out["fetch"]["cache"] = "device cache across steps (resident spans not copied again)"
+            out["fetch"]["resident_spans_per_step"] = statistics.mean(f["resident"] for f in fetched)
+            out["fetch"]["copied_spans_per_step"] = statistics.mean(f["spans"] for f in fetched)
+            out["config"]["fetch"] = "cached across steps"
     if e2e:
         out["e2e"] = e2e
     if cpu:

@@ -193,10 +193,16 @@ class SpanCache:
 
 
 class ColdFetcher:
-    """Pinned mirrors, device arena and slot table for fetching cold bases."""
+    """Pinned mirrors, device arena and slot table for fetching cold bases.
 
-    def __init__(self, cache: SpanCache, arena_elems: int):
+    keep=False: every fetch refills the arena with the step's zoomed spans.
+    keep=True: the arena is a device cache across fetches (resident spans are not
+    copied again; a full arena is flushed and refilled)."""
+
+    def __init__(self, cache: SpanCache, arena_elems: int, keep: bool = False):
         self.c = cache
+        self.keep = bool(keep)
+        self.arena_used = torch.zeros(1, dtype=torch.int64)
         B, L, Hq, m_cap = cache.B, cache.L, cache.Hq, cache.m_cap
         dev = cache.device
         self.arena = torch.zeros(max(arena_elems, 64), dtype=cache.dt, device=dev)
@@ -224,7 +230,9 @@ class ColdFetcher:
         d.region_elems, d.arena_elems = c.region, self.arena.numel()
         d.B, d.L, d.Hq, d.Hkv, d.d, d.dtype = c.B, c.L, c.Hq, c.Hkv, c.d, c.code
         d.l0, d.l1, d.m_cap, d.rank = l0, c.L if l1 is None else l1, c.m_cap, c.rank
+        d.keep, d.arena_used = int(self.keep), _ptr(self.arena_used)
         cs = _stream(compute)
         st = S.sekv_fetch_bases(d, cs, self.copy_stream.cuda_stream, self.done.cuda_event)
         S.check(st, "sekv_fetch_bases")
-        return dict(bytes=int(self.stats[0]), spans=int(self.stats[1]), copies=int(self.stats[2]))
+        return dict(bytes=int(self.stats[0]), spans=int(self.stats[1]), copies=int(self.stats[2]),
+                    resident=int(self.stats[3]))

@@ -237,6 +237,9 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
                      d->l1 <= d->L && d->m_cap >= 32 && d->m_cap % 32 == 0 && d->region_elems > 0 &&
                      d->arena_elems >= 0 && (d->dtype == SEKV_F32 || d->dtype == SEKV_BF16),
                  "fetch: bad shape");
+    SEKV_REQUIRE(d->keep == 0 || (d->keep == 1 && d->arena_used && *d->arena_used >= 0 &&
+                                  *d->arena_used <= d->arena_elems),
+                 "fetch: keep must be 0 or 1, and keep mode needs arena_used in [0, arena_elems]");
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(compute);
     cudaStream_t xs = reinterpret_cast<cudaStream_t>(copy);
     cudaEvent_t ev = reinterpret_cast<cudaEvent_t>(done);
@@ -266,74 +269,110 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
     std::vector<Rect> rects;
     std::vector<uint32_t> uni;
     std::vector<uint64_t> lmask;
-    int64_t bump = 0, spans = 0;
     int dev = 0, max_pitch = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&max_pitch, cudaDevAttrMaxPitch, dev) != cudaSuccess)
         max_pitch = 0;
     const bool pitched = (int64_t)max_pitch >= d->region_elems * es;
-    for (int b = 0; b < d->B; ++b) {
-        const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
-        const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
-        for (int l = d->l0; l < d->l1; ++l) {
-            int64_t* sl = d->slot_host + ((int64_t)b * d->L + l) * d->m_cap;
-            for (int S = 0; S < d->m_cap; ++S) sl[S] = -1;
-        }
-        // layers in chunks of 64: lmask[S] bit j = span S zoomed (by any head) in layer lc + j
-        for (int lc = d->l0; lc < d->l1; lc += 64) {
-            const int nl = d->l1 - lc < 64 ? d->l1 - lc : 64;
-            lmask.assign(m, 0ull);
-            uni.assign(mw, 0u);
-            for (int j = 0; j < nl; ++j) {
-                std::fill(uni.begin(), uni.end(), 0u);
-                const uint32_t* zm = d->zmask_host + ((int64_t)b * d->L + lc + j) * d->Hq * mw;
-                for (int h = 0; h < d->Hq; ++h)
-                    for (int w = 0; w < mw; ++w) uni[w] |= zm[h * mw + w];
-                for (int S = 0; S < m; ++S)
-                    if ((uni[S >> 5] >> (S & 31)) & 1u) lmask[S] |= 1ull << j;
+    const bool keep = d->keep == 1;
+    int64_t bump = 0, spans = 0, hits = 0;
+    // Plan the copies of every zoomed (b, l, S) that is not resident, appending at
+    // `start`; fill the host slot mirror. Returns the arena end.
+    auto plan = [&](int64_t start) -> int64_t {
+        rects.clear();
+        spans = hits = 0;
+        int64_t end = start;
+        for (int b = 0; b < d->B; ++b) {
+            const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
+            const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
+            if (!keep) {
+                for (int l = d->l0; l < d->l1; ++l) {
+                    int64_t* sl = d->slot_host + ((int64_t)b * d->L + l) * d->m_cap;
+                    for (int S = 0; S < d->m_cap; ++S) sl[S] = -1;
+                }
             }
-            int S = 0;
-            while (S < m) {
-                if (!lmask[S]) { ++S; continue; }
-                const int Sa = S;
-                const uint64_t mk = lmask[S];
-                while (S < m && lmask[S] == mk) ++S;          // spans [Sa, S) share the layer set
-                const int64_t width = bo[S] - bo[Sa];
-                spans += (int64_t)(S - Sa) * __builtin_popcountll(mk);
-                int j = 0;
-                while (j < nl) {
-                    if (!((mk >> j) & 1ull)) { ++j; continue; }
-                    const int ja = j;
-                    while (j < nl && ((mk >> j) & 1ull)) ++j;  // layers [lc + ja, lc + j)
-                    const int hgt = j - ja;
-                    for (int q = 0; q < hgt; ++q) {
-                        int64_t* sl = d->slot_host + ((int64_t)b * d->L + lc + ja + q) * d->m_cap;
-                        for (int t = Sa; t < S; ++t) sl[t] = bump + (int64_t)q * width + (bo[t] - bo[Sa]);
+            // layers in chunks of 64: lmask[S] bit j = span S zoomed (by any head) in
+            // layer lc + j and not resident
+            for (int lc = d->l0; lc < d->l1; lc += 64) {
+                const int nl = d->l1 - lc < 64 ? d->l1 - lc : 64;
+                lmask.assign(m, 0ull);
+                uni.assign(mw, 0u);
+                for (int j = 0; j < nl; ++j) {
+                    std::fill(uni.begin(), uni.end(), 0u);
+                    const uint32_t* zm = d->zmask_host + ((int64_t)b * d->L + lc + j) * d->Hq * mw;
+                    for (int h = 0; h < d->Hq; ++h)
+                        for (int w = 0; w < mw; ++w) uni[w] |= zm[h * mw + w];
+                    const int64_t* sl = d->slot_host + ((int64_t)b * d->L + lc + j) * d->m_cap;
+                    for (int S = 0; S < m; ++S)
+                        if ((uni[S >> 5] >> (S & 31)) & 1u) {
+                            if (keep && sl[S] >= 0) ++hits;
+                            else lmask[S] |= 1ull << j;
+                        }
+                }
+                int S = 0;
+                while (S < m) {
+                    if (!lmask[S]) { ++S; continue; }
+                    const int Sa = S;
+                    const uint64_t mk = lmask[S];
+                    while (S < m && lmask[S] == mk) ++S;      // spans [Sa, S) share the layer set
+                    const int64_t width = bo[S] - bo[Sa];
+                    spans += (int64_t)(S - Sa) * __builtin_popcountll(mk);
+                    int j = 0;
+                    while (j < nl) {
+                        if (!((mk >> j) & 1ull)) { ++j; continue; }
+                        const int ja = j;
+                        while (j < nl && ((mk >> j) & 1ull)) ++j;   // layers [lc + ja, lc + j)
+                        const int hgt = j - ja;
+                        for (int q = 0; q < hgt; ++q) {
+                            int64_t* sl = d->slot_host + ((int64_t)b * d->L + lc + ja + q) * d->m_cap;
+                            for (int t = Sa; t < S; ++t) sl[t] = end + (int64_t)q * width + (bo[t] - bo[Sa]);
+                        }
+                        const int64_t src = ((int64_t)b * d->L + lc + ja) * d->region_elems + bo[Sa];
+                        if (pitched) {
+                            rects.push_back({src, end, width, hgt});
+                        } else {
+                            for (int q = 0; q < hgt; ++q)
+                                rects.push_back({src + (int64_t)q * d->region_elems, end + (int64_t)q * width, width, 1});
+                        }
+                        end += (int64_t)hgt * width;
                     }
-                    const int64_t src = ((int64_t)b * d->L + lc + ja) * d->region_elems + bo[Sa];
-                    if (pitched) {
-                        rects.push_back({src, bump, width, hgt});
-                    } else {
-                        for (int q = 0; q < hgt; ++q)
-                            rects.push_back({src + (int64_t)q * d->region_elems, bump + (int64_t)q * width, width, 1});
-                    }
-                    bump += (int64_t)hgt * width;
                 }
             }
         }
+        return end;
+    };
+    auto reset_slots = [&]() {
+        for (int b = 0; b < d->B; ++b)
+            for (int l = d->l0; l < d->l1; ++l) {
+                int64_t* sl = d->slot_host + ((int64_t)b * d->L + l) * d->m_cap;
+                for (int S = 0; S < d->m_cap; ++S) sl[S] = -1;
+            }
+    };
+    bump = plan(keep ? *d->arena_used : 0);
+    if (keep && bump > d->arena_elems) {
+        // the misses do not fit behind the resident spans: flush and refill
+        reset_slots();
+        bump = plan(0);
     }
     if (d->stats) {
-        d->stats[0] = bump * es;
+        d->stats[0] = 0;
+        for (const Rect& r : rects) d->stats[0] += r.width * r.height * es;
         d->stats[1] = spans;
         d->stats[2] = (int64_t)rects.size();
-        d->stats[3] = 0;
+        d->stats[3] = hits;
     }
     if (bump > d->arena_elems) {
-        // leave the device slot table untouched; nothing was copied
+        // nothing is copied and the device slot table stays as it was; a keep-mode
+        // cache is emptied on the host side
+        if (keep) {
+            reset_slots();
+            *d->arena_used = 0;
+        }
         if ((e = cudaEventRecord(ev, xs)) != cudaSuccess) return cuda_fail(e, "fetch: record");
         return fail(SEKV_ERR_CAPACITY, "fetch: zoomed bases need %lld elements, arena holds %lld",
                     (long long)bump, (long long)d->arena_elems);
     }
+    if (keep) *d->arena_used = bump;
     const char* home = reinterpret_cast<const char*>(d->home);
     char* arena = reinterpret_cast<char*>(d->arena);
     for (const Rect& r : rects) {

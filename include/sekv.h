@@ -254,15 +254,26 @@ typedef struct sekv_fetch_desc {
     void* arena;                  /* device arena, arena_elems elements                      */
     int64_t* slot_dev;            /* [B][L][m_cap] device slot table (written on `copy`)     */
     int64_t* slot_host;           /* pinned host mirror of the slot table                    */
-    int64_t* stats;               /* optional host [4]: bytes copied, spans, copies, -       */
+    int64_t* stats;               /* optional host [4]: bytes copied, spans copied, copies,
+                                     spans already resident (keep mode)                      */
+    int64_t* arena_used;          /* host, keep mode only: elements of the arena in use; the
+                                     caller sets it to 0 (and slot_host to -1) once            */
     int64_t region_elems;
     int64_t arena_elems;
     int32_t B, L, Hq, Hkv, d, dtype;
     int32_t l0, l1, m_cap, rank;
+    int32_t keep;                 /* 0: every call refills the arena (the zoomed spans of the
+                                     step only). 1: a device cache across calls: spans whose
+                                     slot (host mirror) is set stay resident and are not
+                                     copied again; misses are appended; when they do not fit,
+                                     the arena is flushed (every slot of [l0, l1) reset) and
+                                     refilled with this step's spans                         */
+    int32_t reserved;
 } sekv_fetch_desc;
 
 /* Copy the bases of every span that any query head of (b, l) zooms, for layers
- * [l0, l1), into the arena, and point the slot table at them (-1 elsewhere).
+ * [l0, l1), into the arena, and point the slot table at them (-1 elsewhere; in
+ * keep mode resident spans keep their slots).
  * Order: zmask is read back on `compute` (the host waits for it); the copies
  * and the slot-table upload go on `copy`; `done` is recorded on `copy`. The
  * caller makes `compute` wait on `done` before ATTEND. A run of consecutive
