@@ -376,6 +376,15 @@ def run_sekv(args, rank, world, local_rank):
     O, lse = cache.new_outputs()
     zm = cache.new_zmask()
     comp = torch.cuda.current_stream()
+    # zoom_hint: zoomed spans per (b, l, kv head), the union over the group's query
+    # heads, from one routing pass with a query outside the timed pool (a previous
+    # step's count, as a serving loop would pass it)
+    cache.decode(gen.queries(wl, step=10 ** 6 + 1, device=dev), theta, phase=P.SEKV_ROUTE, zmask=zm,
+                 budget=args.budget)
+    zw_ = zm.view(torch.int32).cpu().numpy().view(np.uint32).reshape(wl.B, wl.L, wl.Hkv, wl.Hq // wl.Hkv, -1)
+    union = np.bitwise_or.reduce(zw_, axis=3)
+    zoom_hint = int(np.unpackbits(union.view(np.uint8), axis=-1).sum() // max(1, wl.B * wl.L * wl.Hkv))
+    zm.zero_()
 
     fetcher = None
     if cold:
@@ -398,9 +407,10 @@ def run_sekv(args, rank, world, local_rank):
     if cold:
         d_route = cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud)
         d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_ATTEND, O=O, lse=lse, slot=fetcher.slot_dev,
-                                   arena=fetcher.arena, zmask=zm if bud else None, budget=bud)
+                                   arena=fetcher.arena, zmask=zm if bud else None, budget=bud, zoom_hint=zoom_hint)
     else:
-        d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_FUSED, O=O, lse=lse, zmask=zm, budget=bud)
+        d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_FUSED, O=O, lse=lse, zmask=zm, budget=bud,
+                                   zoom_hint=zoom_hint)
 
     def one_step(q, rec=None):
         if q is not None:
@@ -533,6 +543,7 @@ def run_sekv(args, rank, world, local_rank):
                         "alg_bytes_per_step": int(alg_bytes), "GBps": achieved},
         "route_us": statistics.mean(route_ms) * 1e3,
         "zoom_rate": zr,
+        "zoom_hint": zoom_hint,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
                      "traffic": profiled_traffic(wl.name) if full_size else None,

@@ -138,7 +138,7 @@ class SpanCache:
     # ------------------------------------------------------------------ decode
     def decode_desc(self, q, theta, phase=S.SEKV_FUSED, scale=None, O=None, lse=None, zmask=None,
                     route_logits=None, nsplit=0, slot=None, arena=None, l0=0, l1=None,
-                    workspace=None, rows_hint=None, budget=0) -> S.sekv_decode_desc:
+                    workspace=None, rows_hint=None, budget=0, zoom_hint=0) -> S.sekv_decode_desc:
         d = S.sekv_decode_desc()
         d.q = _ptr(q)
         d.a_count, d.m_count, d.span_beg, d.span_end = (_ptr(self.a_count), _ptr(self.m_count),
@@ -158,6 +158,7 @@ class SpanCache:
         d.a_cap, d.m_cap, d.rank, d.phase, d.nsplit = self.a_cap, self.m_cap, self.rank, phase, nsplit
         d.rows_hint = self.rows_hint if rows_hint is None else int(rows_hint)
         d.budget = int(budget)
+        d.zoom_hint = int(zoom_hint)
         need = S.sekv_decode_workspace_bytes(d)
         if workspace is None:
             key = (d.l0, d.l1, nsplit, d.rows_hint, d.budget > 0 and phase != S.SEKV_ATTEND)

@@ -92,8 +92,8 @@ sekv_status check_decode(const sekv_decode_desc* d, bool with_workspace = true) 
     SEKV_REQUIRE(d->phase >= SEKV_FUSED && d->phase <= SEKV_ATTEND, "decode: phase %d", d->phase);
     SEKV_REQUIRE(d->a_cap >= 1 && d->m_cap >= 32 && d->m_cap % 32 == 0, "decode: a_cap >= 1, m_cap % 32 == 0");
     SEKV_REQUIRE(d->m_cap < (1 << 24), "decode: m_cap must be < 2^24");
-    SEKV_REQUIRE(d->nsplit >= 0 && d->rows_hint >= 0 && d->budget >= 0,
-                 "decode: nsplit, rows_hint and budget must be >= 0");
+    SEKV_REQUIRE(d->nsplit >= 0 && d->rows_hint >= 0 && d->budget >= 0 && d->zoom_hint >= 0,
+                 "decode: nsplit, rows_hint, budget and zoom_hint must be >= 0");
     SEKV_REQUIRE(d->budget == 0 || d->zmask, "decode: a budget needs the zmask buffer (output of ROUTE / FUSED, "
                                              "input of ATTEND)");
     if (!sekv::decode_supported(*d))

@@ -40,6 +40,7 @@
 namespace sekv {
 
 constexpr int kNW = 4;          // consumer warps per CTA
+constexpr unsigned kSpanModeSpans = 64;   // zoomed spans in a CTA for whole-span pieces
 constexpr int kRMax = 64;       // largest basis rank the decode accepts
 
 template <int DT, int D, int G>
@@ -145,7 +146,8 @@ struct ZSpan {
 // One piece of the tensor-core zoom stream: what a ring slot holds. Written by
 // the producer before it arms the slot's full barrier (a release), read by the
 // consumers after their wait on it (an acquire).
-enum : int { ZP_B = 0, ZP_AC = 1, ZP_D = 2, ZP_END = 3 };
+// ZP_SPAN: a whole span's block [A | C | B | D] in one slot, handled by one warp.
+enum : int { ZP_B = 0, ZP_AC = 1, ZP_D = 2, ZP_END = 3, ZP_SPAN = 4 };
 struct __align__(16) ZPiece {
     int kind;
     int first;           // first B (or D) piece of its span
@@ -153,7 +155,8 @@ struct __align__(16) ZPiece {
     int cnt;             // B / D: basis rows (a multiple of 8); AC: tokens
     int len, rS;
     uint32_t hm;         // query heads of the group that zoom the span
-    int rot;             // the span's 32-token unit j belongs to consumer warp (j + rot) % 4
+    int rot;             // B / AC / D: the span's 32-token unit j belongs to consumer warp
+                         // (j + rot) % 4; SPAN: the warp that handles the whole span
 };
 
 // shared-memory carve-up common to both paths
@@ -584,7 +587,7 @@ SEKV_DEV float ex2(float x) {
 
 // zoomed spans of the CTA: word w of zw[h] holds heads h's bits for spans
 // s0 + 32 w .. s0 + 32 w + 31; nwords words are in use
-template <int D, int G>
+template <int D, int G, bool SP>
 SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b, int l, int kvh, int s0, int nwords,
                            int zwords) {
     using C = DecCfg<SEKV_BF16, D, G>;
@@ -593,6 +596,21 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
     uint32_t np = 0;          // pieces armed
     bool good = true;
     int rot = 0;
+    // Whole-span pieces (one warp per small span, no repeated u / D work) pay off
+    // when the CTA has enough zoomed spans to keep the four consumer warps busy
+    // with different spans; with few, sharing each span's units across the warps
+    // keeps the critical path shorter.
+    bool span_mode = false;
+    if (SP) {
+        unsigned nz = 0;
+        for (int w = lane; w < nwords; w += 32) {
+            uint32_t m = 0u;
+#pragma unroll
+            for (int h = 0; h < G; ++h) m |= sm.zw[h * zwords + w];
+            nz += __popc(m);
+        }
+        span_mode = warp_sum_u(nz) >= kSpanModeSpans;
+    }
     // the slots were last read through the generic proxy (stream phase)
     fence_proxy_async();
     // arm the next slot with piece pc and up to two bulk copies (lane 0 issues)
@@ -679,6 +697,14 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
                 pc.rS = rS;
                 pc.hm = jhm;
                 pc.rot = rot;
+                if (span_mode && be * 2 + D * 16 <= ZSL) {
+                    // the whole block fits one slot (with room for the D projection's
+                    // read of one 8-row block past D): one piece, one owner warp
+                    pc.kind = ZP_SPAN; pc.first = 1; pc.r0 = 0; pc.cnt = jl;
+                    emit(pc, blk, (uint32_t)(be * 2), nullptr, 0u);
+                    rot = (rot + 1) & 3;
+                    continue;
+                }
                 for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
                     pc.kind = ZP_B; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
                     emit(pc, blk + (2 * pa + (int64_t)r0 * D) * 2, (uint32_t)pc.cnt * C::ROWB, nullptr, 0u);
@@ -715,7 +741,7 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
 // RM: the largest basis rank this instantiation handles (16, 32 or 64), which
 // sizes the u / y fragments and the unrolled basis-row loops. Lane (g, c) holds
 // heads 2c, 2c+1 (the stream layout): mh, lh (partial) and the O^T columns.
-template <int D, int G, int RM>
+template <int D, int G, int RM, bool SP>
 SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int lane, const uint32_t (&qb)[D / 16][2],
                            float (&mh)[2], float (&lh)[2], float (&oc)[D / 16][4]) {
     using C = DecCfg<SEKV_BF16, D, G>;
@@ -736,6 +762,173 @@ SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int la
         yacc[ks][0] = yacc[ks][1] = yacc[ks][2] = yacc[ks][3] = 0.f;
     }
 
+    // a span starts: its rank, the heads of this lane that zoom it, a fresh state
+    auto span_begin = [&](const ZPiece& pc) {
+        rS = pc.rS;
+        nib = (rS + 7) >> 3;
+        zh0 = 2 * c < G && ((pc.hm >> (2 * c)) & 1u);
+        zh1 = 2 * c + 1 < G && ((pc.hm >> (2 * c + 1)) & 1u);
+        msp[0] = msp[1] = -INFINITY;
+        lsp[0] = lsp[1] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < NKS; ++ks) yacc[ks][0] = yacc[ks][1] = yacc[ks][2] = yacc[ks][3] = 0.f;
+    };
+    // u for the basis rows [r0, r0 + cnt) of the B rows at Bp (8x8 tiles; r0 a
+    // multiple of 16), 16 rows at a time; two partial sums over even / odd k-steps
+    // keep the mma chains short
+    auto do_u = [&](const unsigned char* Bp, int r0, int cnt) {
+#pragma unroll
+        for (int ks = 0; ks < NKS; ++ks) {
+            if (16 * ks < r0 || 16 * ks >= r0 + cnt) continue;
+            const int ib = (16 * ks - r0) >> 3;                 // local 8-row block
+            const bool two = 16 * ks + 8 < r0 + cnt;
+            float ua[4] = {0.f, 0.f, 0.f, 0.f}, uv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                uint32_t ba[4];
+                ldsm_x4(ba, Bp + (((ib + (lj & 1)) * DB + 2 * kk + (lj >> 1)) * 64 + lr * 8) * 2);
+                if (!two) ba[1] = ba[3] = 0u;
+                const uint32_t qf[2] = {qb[kk][0], qb[kk][1]};
+                mma_bf16_16816((kk & 1) ? uv : ua, ba, qf);
+            }
+            // rows i >= r_S do not exist: exact zeros (select, not multiply)
+            const int i0 = 16 * ks + g;
+            uint32_t h01, l01, h23, l23;
+            split_bf16x2(i0 < rS ? (ua[0] + uv[0]) * sl2 : 0.f, i0 < rS ? (ua[1] + uv[1]) * sl2 : 0.f, h01, l01);
+            split_bf16x2(i0 + 8 < rS ? (ua[2] + uv[2]) * sl2 : 0.f, i0 + 8 < rS ? (ua[3] + uv[3]) * sl2 : 0.f,
+                         h23, l23);
+            ub[ks][0] = movm_t(h01);
+            ub[ks][1] = movm_t(h23);
+            ub[ks][2] = movm_t(l01);
+            ub[ks][3] = movm_t(l23);
+        }
+    };
+    // the 32-token units v = v0, v0 + vstep, ... of cnt tokens whose A rows are at
+    // As and C rows at Cs (8x8 tiles, r8 wide); groups at or past ceil(cnt / 8)
+    // hold other bytes and are masked
+    auto do_units = [&](const unsigned char* As, const unsigned char* Cs, int cnt, int v0, int vstep) {
+        const int nv = (cnt + 31) >> 5;
+        for (int v = v0; v < nv; v += vstep) {
+            const int ngp = ((cnt + 7) >> 3) - 4 * v;           // token groups of the unit that exist
+            // s = A u for the unit's 32 tokens (two m-tiles of 16)
+            float sc[2][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
+                if (ngp <= 2 * mt) continue;
+#pragma unroll
+                for (int ks = 0; ks < NKS; ++ks) {
+                    if (2 * ks >= nib) continue;
+                    uint32_t aa[4];
+                    ldsm_x4(aa, As + (((4 * v + 2 * mt + (lj & 1)) * nib + 2 * ks + (lj >> 1)) * 64 + lr * 8) * 2);
+                    if (2 * ks + 1 >= nib) aa[2] = aa[3] = 0u;
+                    const uint32_t uh[2] = {ub[ks][0], ub[ks][1]}, ul[2] = {ub[ks][2], ub[ks][3]};
+                    mma_bf16_16816(sc[mt], aa, uh);
+                    mma_bf16_16816(sc[mt], aa, ul);
+                }
+            }
+            // the span's online softmax for heads 2c, 2c+1 (log2 domain; u carries the scale)
+            float x[2][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int tk = 32 * v + 16 * mt + g + ((e >> 1) << 3);
+                    const bool zz = (e & 1) ? zh1 : zh0;
+                    x[mt][e] = (zz && tk < cnt) ? sc[mt][e] : -INFINITY;
+                }
+            float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
+            float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, o));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, o));
+            }
+            const float mn0 = fmaxf(msp[0], mx0), mn1 = fmaxf(msp[1], mx1);
+            const float al0 = (mn0 == -INFINITY) ? 1.f : ex2(msp[0] - mn0);
+            const float al1 = (mn1 == -INFINITY) ? 1.f : ex2(msp[1] - mn1);
+            const float r0 = (mn0 == -INFINITY) ? 0.f : mn0, r1 = (mn1 == -INFINITY) ? 0.f : mn1;
+            float pv[2][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) pv[mt][e] = ex2(x[mt][e] - ((e & 1) ? r1 : r0));
+            lsp[0] = fmaf(lsp[0], al0, (pv[0][0] + pv[0][2]) + (pv[1][0] + pv[1][2]));
+            lsp[1] = fmaf(lsp[1], al1, (pv[0][1] + pv[0][3]) + (pv[1][1] + pv[1][3]));
+            msp[0] = mn0;
+            msp[1] = mn1;
+            if (__any_sync(FULL, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+                for (int ks = 0; ks < NKS; ++ks) {
+                    yacc[ks][0] *= al0; yacc[ks][1] *= al1;
+                    yacc[ks][2] *= al0; yacc[ks][3] *= al1;
+                }
+            }
+            // y += C^T p: p (k = tokens, n = heads) as B fragments by transposing the
+            // 8 x 8 (token, head) blocks of the score accumulators
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                if (ngp <= 2 * mt) continue;
+                const bool g2 = ngp > 2 * mt + 1;                 // the m-tile's second token group exists
+                const uint32_t pb[2] = {movm_t(pack_bf16(pv[mt][0], pv[mt][1])),
+                                        movm_t(pack_bf16(pv[mt][2], pv[mt][3]))};
+#pragma unroll
+                for (int js = 0; js < NKS; ++js) {
+                    if (2 * js >= nib) continue;
+                    uint32_t ca[4];
+                    ldsm_x4_t(ca, Cs + (((4 * v + 2 * mt + (lj >> 1)) * nib + 2 * js + (lj & 1)) * 64 + lr * 8) * 2);
+                    if (!g2) ca[2] = ca[3] = 0u;
+                    mma_bf16_16816(yacc[js], ca, pb);
+                }
+            }
+        }
+    };
+    // merge the span's (max, partial sum) into the stream state of heads 2c, 2c+1;
+    // keep (beta y) as B fragments in ub (u is dead by now)
+    auto do_merge = [&]() {
+        float be[2] = {0.f, 0.f};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const bool zz = hh ? zh1 : zh0;
+            if (zz && msp[hh] != -INFINITY) {
+                const float mnew = fmaxf(mh[hh], msp[hh]);
+                const float alpha = (mh[hh] == -INFINITY) ? 0.f : ex2(mh[hh] - mnew);
+                be[hh] = ex2(msp[hh] - mnew);
+                lh[hh] = lh[hh] * alpha + lsp[hh] * be[hh];
+                mh[hh] = mnew;
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    oc[mt][hh] *= alpha;
+                    oc[mt][2 + hh] *= alpha;
+                }
+            }
+        }
+#pragma unroll
+        for (int ks = 0; ks < NKS; ++ks) {
+            const int i0 = 16 * ks + g;
+            ub[ks][0] = movm_t(pack_bf16(i0 < rS ? yacc[ks][0] * be[0] : 0.f, i0 < rS ? yacc[ks][1] * be[1] : 0.f));
+            ub[ks][1] = movm_t(pack_bf16(i0 + 8 < rS ? yacc[ks][2] * be[0] : 0.f,
+                                         i0 + 8 < rS ? yacc[ks][3] * be[1] : 0.f));
+        }
+    };
+    // O^T += D^T (beta y) over the basis rows [r0, r0 + cnt) of the D rows at Dp
+    auto do_D = [&](const unsigned char* Dp, int r0, int cnt) {
+#pragma unroll
+        for (int ks = 0; ks < NKS; ++ks) {
+            if (16 * ks < r0 || 16 * ks >= r0 + cnt) continue;
+            const int ib = (16 * ks - r0) >> 3;
+            const bool two = 16 * ks + 8 < r0 + cnt;
+            const uint32_t yb[2] = {ub[ks][0], ub[ks][1]};
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+                uint32_t da[4];
+                ldsm_x4_t(da, Dp + (((ib + (lj >> 1)) * DB + 2 * mt + (lj & 1)) * 64 + lr * 8) * 2);
+                if (!two) da[2] = da[3] = 0u;
+                mma_bf16_16816(oc[mt], da, yb);
+            }
+        }
+    };
+
     for (uint32_t k = 0;; ++k) {
         const int slot = (int)(k % ZNS);
         if (!mbar_wait(&sm.zfull[slot], (k / ZNS) & 1)) {
@@ -750,173 +943,29 @@ SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int la
         }
         if (pc.kind == ZP_END) break;
         const unsigned char* zs = sm.stages + (size_t)slot * ZSL;
-        if (pc.kind == ZP_B) {
+        if (SP && pc.kind == ZP_SPAN) {
+            // the whole block [A | C | B | D] is in the slot; one warp takes it all
+            if (warp == pc.rot) {
+                span_begin(pc);
+                const int r8 = nib * 8;
+                const int pa = round8(pc.len) * r8;              // elements of A (and of C)
+                do_u(zs + 4 * pa, 0, r8);
+                do_units(zs, zs + 2 * pa, pc.len, 0, 1);
+                do_merge();
+                do_D(zs + 4 * pa + 2 * r8 * D, 0, r8);
+            }
+        } else if (pc.kind == ZP_B) {
             if (pc.first) {
-                rS = pc.rS;
-                nib = (rS + 7) >> 3;
+                span_begin(pc);
                 mine = ((pc.len + 31) >> 5) > ((warp - pc.rot) & 3);
-                zh0 = 2 * c < G && ((pc.hm >> (2 * c)) & 1u);
-                zh1 = 2 * c + 1 < G && ((pc.hm >> (2 * c + 1)) & 1u);
-                msp[0] = msp[1] = -INFINITY;
-                lsp[0] = lsp[1] = 0.f;
-#pragma unroll
-                for (int ks = 0; ks < NKS; ++ks) yacc[ks][0] = yacc[ks][1] = yacc[ks][2] = yacc[ks][3] = 0.f;
             }
-            if (mine) {
-                // u for the basis rows of this piece, 16 at a time (two partial sums
-                // over even / odd k-steps keep the mma chains short)
-#pragma unroll
-                for (int ks = 0; ks < NKS; ++ks) {
-                    if (16 * ks < pc.r0 || 16 * ks >= pc.r0 + pc.cnt) continue;
-                    const int ib = (16 * ks - pc.r0) >> 3;             // piece-local 8-row block
-                    const bool two = 16 * ks + 8 < pc.r0 + pc.cnt;
-                    float ua[4] = {0.f, 0.f, 0.f, 0.f}, uv[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        uint32_t ba[4];
-                        ldsm_x4(ba, zs + (((ib + (lj & 1)) * DB + 2 * kk + (lj >> 1)) * 64 + lr * 8) * 2);
-                        if (!two) ba[1] = ba[3] = 0u;
-                        const uint32_t qf[2] = {qb[kk][0], qb[kk][1]};
-                        mma_bf16_16816((kk & 1) ? uv : ua, ba, qf);
-                    }
-                    // rows i >= r_S do not exist: exact zeros (select, not multiply)
-                    const int i0 = 16 * ks + g;
-                    uint32_t h01, l01, h23, l23;
-                    split_bf16x2(i0 < rS ? (ua[0] + uv[0]) * sl2 : 0.f, i0 < rS ? (ua[1] + uv[1]) * sl2 : 0.f, h01, l01);
-                    split_bf16x2(i0 + 8 < rS ? (ua[2] + uv[2]) * sl2 : 0.f, i0 + 8 < rS ? (ua[3] + uv[3]) * sl2 : 0.f,
-                                 h23, l23);
-                    ub[ks][0] = movm_t(h01);
-                    ub[ks][1] = movm_t(h23);
-                    ub[ks][2] = movm_t(l01);
-                    ub[ks][3] = movm_t(l23);
-                }
-            }
+            if (mine) do_u(zs, pc.r0, pc.cnt);
         } else if (pc.kind == ZP_AC) {
-            if (mine) {
-                const unsigned char* As = zs;
-                const unsigned char* Cs = zs + ZSL / 2;
-                const int nv = (pc.cnt + 31) >> 5;
-                for (int v = (warp - pc.rot - (pc.r0 >> 5)) & 3; v < nv; v += 4) {
-                    // token groups 4v .. 4v+3 of the piece; those at or past ngp were not copied
-                    const int ngp = ((pc.cnt + 7) >> 3) - 4 * v;
-                    // s = A u for the unit's 32 tokens (two m-tiles of 16)
-                    float sc[2][4];
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
-                        if (ngp <= 2 * mt) continue;
-#pragma unroll
-                        for (int ks = 0; ks < NKS; ++ks) {
-                            if (2 * ks >= nib) continue;
-                            uint32_t aa[4];
-                            ldsm_x4(aa, As + (((4 * v + 2 * mt + (lj & 1)) * nib + 2 * ks + (lj >> 1)) * 64 + lr * 8) * 2);
-                            if (2 * ks + 1 >= nib) aa[2] = aa[3] = 0u;
-                            const uint32_t uh[2] = {ub[ks][0], ub[ks][1]}, ul[2] = {ub[ks][2], ub[ks][3]};
-                            mma_bf16_16816(sc[mt], aa, uh);
-                            mma_bf16_16816(sc[mt], aa, ul);
-                        }
-                    }
-                    // the span's online softmax for heads 2c, 2c+1 (log2 domain; u carries the scale)
-                    float x[2][4];
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int tk = 32 * v + 16 * mt + g + ((e >> 1) << 3);
-                            const bool zz = (e & 1) ? zh1 : zh0;
-                            x[mt][e] = (zz && tk < pc.cnt) ? sc[mt][e] : -INFINITY;
-                        }
-                    float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
-                    float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
-#pragma unroll
-                    for (int o = 4; o < 32; o <<= 1) {
-                        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, o));
-                        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, o));
-                    }
-                    const float mn0 = fmaxf(msp[0], mx0), mn1 = fmaxf(msp[1], mx1);
-                    const float al0 = (mn0 == -INFINITY) ? 1.f : ex2(msp[0] - mn0);
-                    const float al1 = (mn1 == -INFINITY) ? 1.f : ex2(msp[1] - mn1);
-                    const float r0 = (mn0 == -INFINITY) ? 0.f : mn0, r1 = (mn1 == -INFINITY) ? 0.f : mn1;
-                    float pv[2][4];
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) pv[mt][e] = ex2(x[mt][e] - ((e & 1) ? r1 : r0));
-                    lsp[0] = fmaf(lsp[0], al0, (pv[0][0] + pv[0][2]) + (pv[1][0] + pv[1][2]));
-                    lsp[1] = fmaf(lsp[1], al1, (pv[0][1] + pv[0][3]) + (pv[1][1] + pv[1][3]));
-                    msp[0] = mn0;
-                    msp[1] = mn1;
-                    if (__any_sync(FULL, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
-                        for (int ks = 0; ks < NKS; ++ks) {
-                            yacc[ks][0] *= al0; yacc[ks][1] *= al1;
-                            yacc[ks][2] *= al0; yacc[ks][3] *= al1;
-                        }
-                    }
-                    // y += C^T p: p (k = tokens, n = heads) as B fragments by transposing
-                    // the 8 x 8 (token, head) blocks of the score accumulators
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        if (ngp <= 2 * mt) continue;
-                        const bool g2 = ngp > 2 * mt + 1;          // the m-tile's second token group was copied
-                        const uint32_t pb[2] = {movm_t(pack_bf16(pv[mt][0], pv[mt][1])),
-                                                movm_t(pack_bf16(pv[mt][2], pv[mt][3]))};
-#pragma unroll
-                        for (int js = 0; js < NKS; ++js) {
-                            if (2 * js >= nib) continue;
-                            uint32_t ca[4];
-                            ldsm_x4_t(ca, Cs + (((4 * v + 2 * mt + (lj >> 1)) * nib + 2 * js + (lj & 1)) * 64 + lr * 8) * 2);
-                            if (!g2) ca[2] = ca[3] = 0u;
-                            mma_bf16_16816(yacc[js], ca, pb);
-                        }
-                    }
-                }
-            }
+            if (mine) do_units(zs, zs + ZSL / 2, pc.cnt, (warp - pc.rot - (pc.r0 >> 5)) & 3, 4);
         } else {  // ZP_D
             if (mine) {
-                if (pc.first) {
-                    // merge the span's (max, partial sum) into the stream state of heads
-                    // 2c, 2c+1; keep (beta y) as B fragments in ub (u is dead by now)
-                    float be[2] = {0.f, 0.f};
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const bool zz = hh ? zh1 : zh0;
-                        if (zz && msp[hh] != -INFINITY) {
-                            const float mnew = fmaxf(mh[hh], msp[hh]);
-                            const float alpha = (mh[hh] == -INFINITY) ? 0.f : ex2(mh[hh] - mnew);
-                            be[hh] = ex2(msp[hh] - mnew);
-                            lh[hh] = lh[hh] * alpha + lsp[hh] * be[hh];
-                            mh[hh] = mnew;
-#pragma unroll
-                            for (int mt = 0; mt < D / 16; ++mt) {
-                                oc[mt][hh] *= alpha;
-                                oc[mt][2 + hh] *= alpha;
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int ks = 0; ks < NKS; ++ks) {
-                        const int i0 = 16 * ks + g;
-                        ub[ks][0] = movm_t(pack_bf16(i0 < rS ? yacc[ks][0] * be[0] : 0.f, i0 < rS ? yacc[ks][1] * be[1] : 0.f));
-                        ub[ks][1] = movm_t(pack_bf16(i0 + 8 < rS ? yacc[ks][2] * be[0] : 0.f,
-                                                     i0 + 8 < rS ? yacc[ks][3] * be[1] : 0.f));
-                    }
-                }
-                // O^T += D^T (beta y) over this piece's basis-row blocks
-#pragma unroll
-                for (int ks = 0; ks < NKS; ++ks) {
-                    if (16 * ks < pc.r0 || 16 * ks >= pc.r0 + pc.cnt) continue;
-                    const int ib = (16 * ks - pc.r0) >> 3;
-                    const bool two = 16 * ks + 8 < pc.r0 + pc.cnt;
-                    const uint32_t yb[2] = {ub[ks][0], ub[ks][1]};
-#pragma unroll
-                    for (int mt = 0; mt < D / 16; ++mt) {
-                        uint32_t da[4];
-                        ldsm_x4_t(da, zs + (((ib + (lj >> 1)) * DB + 2 * mt + (lj & 1)) * 64 + lr * 8) * 2);
-                        if (!two) da[2] = da[3] = 0u;
-                        mma_bf16_16816(oc[mt], da, yb);
-                    }
-                }
+                if (pc.first) do_merge();
+                do_D(zs, pc.r0, pc.cnt);
             }
         }
         __syncwarp();
@@ -942,7 +991,9 @@ SEKV_DEV void store_state_lanes(const DecSmem& sm, int idx, int lane, const floa
         for (int k = 0; k < DPL; ++k) sm.st_o[(idx * G + h) * D + lane * DPL + k] = o[h][k];
 }
 
-template <int DT, int D, int G, int RM>
+// SP: the zoom phase may take small spans whole (rank <= 16 only; chosen by the host
+// from the expected zoom count: with few zoomed spans the plain variant is faster)
+template <int DT, int D, int G, int RM, bool SP>
 __global__ void __launch_bounds__((kNW + 1) * 32, 3)
 decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     using C = DecCfg<DT, D, G>;
@@ -1332,8 +1383,8 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         for (int i = lane; i < G * zwords; i += 32) zany = zany || sm.zw[i] != 0u;
         zany = __any_sync(0xffffffffu, zany);
         if (!route_only && zany && *sm.sfail == 0) {     // uniform over the CTA
-            if (warp == kNW) zoom_produce<D, G>(a, sm, lane, b, l, kvh, s0, nwords, zwords);
-            else zoom_consume<D, G, RM>(a, sm, warp, lane, qb, mh, lh, oc);
+            if (warp == kNW) zoom_produce<D, G, SP>(a, sm, lane, b, l, kvh, s0, nwords, zwords);
+            else zoom_consume<D, G, RM, SP>(a, sm, warp, lane, qb, mh, lh, oc);
         }
     } else {
         if (!route_only && warp < kNW && ok) zoom_phase<DT, D, G>(a, sm, warp, lane, b, l, kvh, m_run, l_run, o, m_lane);
@@ -1671,7 +1722,7 @@ static bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int d) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DT, int D, int G, int RM>
+template <int DT, int D, int G, int RM, bool SP>
 static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st,
                             int zin) {
     using C = DecCfg<DT, D, G>;
@@ -1694,7 +1745,7 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     a.zin = zin;
     const size_t smem = decode_smem_bytes<DT, D, G>(a.sch_max, a.qcap);
     if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT, D, G, RM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT, D, G, RM, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     DecMaps maps;
@@ -1712,7 +1763,7 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     const int64_t nblk = (int64_t)p.nsplit * d.Hkv * d.B * Lr;
     if (nblk > 0x7fffffff) return cudaErrorInvalidConfiguration;
     dim3 grid((unsigned)nblk);
-    decode_kernel<DT, D, G, RM><<<grid, (kNW + 1) * 32, smem, st>>>(a, maps);
+    decode_kernel<DT, D, G, RM, SP><<<grid, (kNW + 1) * 32, smem, st>>>(a, maps);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (d.phase != SEKV_ROUTE) {
         merge_kernel<D><<<d.B * Lr * d.Hq, D, 0, st>>>(a.part_o, a.part_ml, d.O, d.lse, p.nsplit, G, d.Hkv,
@@ -1726,9 +1777,11 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
 // CUDA-core path handles any rank up to 64 in one variant
 template <int DT, int D, int G>
 static cudaError_t launch_r(const sekv_decode_desc& d, const DecodePlan& p, void* w, cudaStream_t st, int zin) {
-    if (DT == SEKV_BF16 && d.rank <= 16) return launch_t<DT, D, G, 16>(d, p, w, st, zin);
-    if (DT == SEKV_BF16 && d.rank <= 32) return launch_t<DT, D, G, 32>(d, p, w, st, zin);
-    return launch_t<DT, D, G, 64>(d, p, w, st, zin);
+    if (DT == SEKV_BF16 && d.rank <= 16)
+        return d.zoom_hint >= (int)kSpanModeSpans ? launch_t<DT, D, G, 16, true>(d, p, w, st, zin)
+                                                   : launch_t<DT, D, G, 16, false>(d, p, w, st, zin);
+    if (DT == SEKV_BF16 && d.rank <= 32) return launch_t<DT, D, G, 32, false>(d, p, w, st, zin);
+    return launch_t<DT, D, G, 64, false>(d, p, w, st, zin);
 }
 
 template <int DT, int D>

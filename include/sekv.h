@@ -206,6 +206,12 @@ typedef struct sekv_decode_desc {
                                 the capped mask; ATTEND reads it as input (no re-routing);
                                 FUSED routes, caps, then attends with the capped mask.
                                 Without route_logits the workspace holds the logits.     */
+    int32_t zoom_hint;       /* expected zoomed spans per (b, l, kv head) (e.g. from the
+                                previous step); 0 = unknown. At >= 64 (and rank <= 16) a
+                                decode variant that hands small spans whole to one warp
+                                is used, which is faster when most spans zoom and slower
+                                when few do. Results are the same either way.            */
+    int32_t reserved;
 } sekv_decode_desc;
 
 size_t sekv_decode_workspace_bytes(const sekv_decode_desc* desc);

@@ -304,3 +304,26 @@ def test_empty_cache_rows():
         np.testing.assert_allclose(T.f64(O2[0, 0, h]), vb, atol=1e-5)   # one entry: softmax weight 1
         lo = float(T.f64(q[0, 0, h]) @ kb / math.sqrt(wl.d) + math.log(64))
         assert float(l2[0, 0, h]) == pytest.approx(lo, abs=1e-4)
+
+
+def test_whole_span_variant_matches_oracle():
+    """zoom_hint >= 64 selects the decode variant that hands small zoomed spans whole
+    to one warp (taken per CTA when it holds >= 64 zoomed spans). Every span zoomed,
+    one split, ~240 spans per CTA: both variants must match the oracle."""
+    wl = WORKLOADS["c2"].scaled(n=16384, L=1, Hq=8, Hkv=2)
+    H, K, V, segs, units, q, _, scale = _setup(wl)
+    theta = np.full((wl.L, wl.Hq), -np.inf)
+    c = _cache(wl)
+    T.upload_oracle_cache(c, segs, units)
+    th = torch.full((wl.L, wl.Hq), -math.inf, dtype=torch.float32, device="cuda")
+    assert min(len(s.spans) for s in segs) >= 64
+    outs = []
+    for hint in (0, 10 ** 6):
+        zmask = c.new_zmask()
+        O_gpu, lse_gpu = c.decode(q.cuda(), th, zmask=zmask, nsplit=1, zoom_hint=hint)
+        torch.cuda.synchronize()
+        assert c.read_status() == 0
+        err, lerr, nz = _compare(wl, c, q, theta, scale, segs, units, O_gpu, lse_gpu, zmask)
+        outs.append(O_gpu)
+        print(f"zoom_hint={hint}: max|dO|={err:.2e} max|dlse|={lerr:.2e} zoomed={nz}")
+    assert (outs[0] - outs[1]).abs().max().item() <= 2e-2
