@@ -209,6 +209,17 @@ sekv_status sekv_decode_attn(const sekv_decode_desc* d, sekv_stream_t stream) {
     return SEKV_OK;
 }
 
+sekv_status sekv_merge_partials(const float* O_parts, const float* lse_parts, int32_t nparts, int64_t rows,
+                                int32_t d, float* O, float* lse, sekv_stream_t stream) {
+    SEKV_REQUIRE(O_parts && lse_parts && O && lse, "merge: null pointer");
+    SEKV_REQUIRE(nparts >= 1 && nparts <= 64 && rows >= 0 && rows < (1LL << 31) && d >= 1 && d <= 1024,
+                 "merge: nparts in [1, 64], rows in [0, 2^31), d in [1, 1024]");
+    cudaError_t e = sekv::launch_merge_parts(O_parts, lse_parts, nparts, rows, d, O, lse,
+                                             reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "merge");
+    return SEKV_OK;
+}
+
 sekv_status sekv_decode_attn_static(const sekv_decode_desc* d, sekv_stream_t stream) {
     sekv_status s = check_decode(d, false);
     if (s != SEKV_OK) return s;

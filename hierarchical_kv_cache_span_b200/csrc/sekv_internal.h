@@ -27,6 +27,8 @@ DecodePlan plan_decode(const sekv_decode_desc& d);
 size_t decode_workspace_bytes(const sekv_decode_desc& d);
 bool decode_supported(const sekv_decode_desc& d);
 cudaError_t launch_decode(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st);
+cudaError_t launch_merge_parts(const float* O_parts, const float* lse_parts, int nparts, int64_t rows, int d,
+                               float* O, float* lse, cudaStream_t st);
 size_t decode_static_scratch_bytes();
 void* decode_static_scratch(cudaError_t* err);
 

@@ -84,6 +84,7 @@ _SIGS = {
     "sekv_decode_attn": (_i32, [C.POINTER(sekv_decode_desc), _p]),
     "sekv_decode_attn_static": (_i32, [C.POINTER(sekv_decode_desc), _p]),
     "sekv_fetch_bases": (_i32, [C.POINTER(sekv_fetch_desc), _p, _p, _p]),
+    "sekv_merge_partials": (_i32, [_p, _p, _i32, _i64, _i32, _p, _p, _p]),
     "sekv_status_str": (C.c_char_p, [_i32]),
     "sekv_last_error": (C.c_char_p, []),
     "sekv_desc_size": (C.c_size_t, [_i32]),
@@ -151,6 +152,12 @@ def sekv_decode_attn_static(desc: sekv_decode_desc, stream: int = 0) -> int:
 
 
 SEKV_STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def sekv_merge_partials(O_parts: int, lse_parts: int, nparts: int, rows: int, d: int, O: int, lse: int,
+                        stream: int = 0) -> int:
+    return int(_lib.sekv_merge_partials(C.c_void_p(O_parts), C.c_void_p(lse_parts), nparts, rows, d,
+                                        C.c_void_p(O), C.c_void_p(lse), C.c_void_p(stream or None)))
 
 
 def sekv_fetch_bases(desc: sekv_fetch_desc, compute: int, copy: int, done: int) -> int:

@@ -247,6 +247,21 @@ sekv_status sekv_decode_attn(const sekv_decode_desc* desc, sekv_stream_t stream)
 #define SEKV_STATIC_SCRATCH_BYTES (8u << 20)
 sekv_status sekv_decode_attn_static(const sekv_decode_desc* desc, sekv_stream_t stream);
 
+/*
+ * Merge decode results of disjoint parts of one logit list by log-sum-exp
+ * (SeKV summary, workflow paragraph: Stage 2 is ONE softmax over every entry, so
+ * results of a partition recombine exactly). Used for context-parallel decode:
+ * each rank decodes the anchors and spans of its slice of the context and the
+ * parts are merged after an all-gather.
+ *   O_parts   [nparts][rows][d] fp32 (device), lse_parts [nparts][rows] fp32 (device)
+ *   O         [rows][d] fp32 (device, written), lse [rows] fp32 (device, written)
+ * A part with lse = -inf (no entries) contributes nothing; rows with no entries in
+ * any part get O = 0, lse = -inf. d <= 1024, 1 <= nparts <= 64. Asynchronous on
+ * `stream`; argument errors return SEKV_ERR_INVALID_ARG before any launch.
+ */
+sekv_status sekv_merge_partials(const float* O_parts, const float* lse_parts, int32_t nparts, int64_t rows,
+                                int32_t d, float* O, float* lse, sekv_stream_t stream);
+
 /* ------------------------------------------------------------------------- */
 /* Cold-basis fetch (SeKV summary: zoomed spans' bases fetched from the CPU;  */
 /* SeKV blog Fig. 2)                                                          */
