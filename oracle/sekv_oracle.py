@@ -25,7 +25,8 @@ mu/sigma are the per-sequence mean and population std over all n positions,
 in fp64, with a strict ``>``; the last ``window`` positions are anchors too;
 anchors are not members of any span, and spans are the maximal runs of
 non-anchor positions; the routing projection is the identity (d' = d), so
-the routing summary is ``kbar / ||kbar||``; all attention and routing logits
+the routing summary is ``kbar / ||kbar||``, unless a projection W is given (the
+learned form, Eq. (3) and (5), with the query projected by the same W); all attention and routing logits
 use the scale ``1/sqrt(d)`` and ``+log|S|`` is added after scaling; thresholds
 are compared in logit space (``l > ln(tau/(1-tau))``, which is monotone-equal
 to Eq. (9)); zoomed tokens use the reconstructed ``A_S B_S`` / ``C_S D_S``; a
@@ -44,6 +45,7 @@ __all__ = [
     "to_storage", "tau_to_theta", "Segmentation", "segment", "span_weights",
     "weighted_mean", "span_summaries", "truncated_basis", "span_bases",
     "routing_logits", "zoom_decisions", "decode_unit", "UnitCache", "build_unit",
+    "routing_summary", "routing_summaries", "learned_routing_logits",
 ]
 
 
@@ -180,34 +182,69 @@ def span_summaries(K, V, H, seg: Segmentation, wmode: str, dtype: str):
 
 
 # ---------------------------------------------------------------------------
-# prefill: truncated bases  [SeKV blog 2.2 Eq. (6)-(8), rank gate m_i = 1]
+# prefill: learned-form routing summaries  [SeKV blog 2.2 Eq. (3)]
 # ---------------------------------------------------------------------------
-def truncated_basis(X, r: int, dtype: str):
-    """Rank-r_S truncated SVD of X (|S| x d), r_S = min(r, |S|, d), as two
-    stored factors with A @ B = sum_{i <= r_S} sigma_i u_i v_i^T.
+def routing_summary(Ks, w, W) -> np.ndarray:
+    """Eq. (3) for one span and one (layer, head): every token's key is projected
+    into the routing space, the projections are summed with the span weights and
+    the sum is scaled to unit length: sum_t w_t W K_t / ||sum_t w_t W K_t||_2.
+    A zero sum gives the zero vector (a reading: the pages do not say)."""
+    Ks = np.asarray(Ks, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    proj = Ks @ W.T                     # row t is W K_t
+    y = (w[:, None] * proj).sum(axis=0)
+    nrm = np.sqrt(np.sum(y * y))
+    return y / nrm if nrm > 0.0 else np.zeros_like(y)
 
-    Factor split: if |S| <= d, A = U_r (|S| x r_S) and B = Sigma_r V_r^T;
-    otherwise A = U_r Sigma_r and B = V_r^T (r_S x d).
+
+def routing_summaries(K, H, seg: Segmentation, wmode: str, W_heads, dtype: str) -> np.ndarray:
+    """[G][m][d'] stored routing summaries of every span for the G query heads that
+    share this key head (each head has its own W, [G][d'][d])."""
+    W_heads = np.asarray(W_heads, dtype=np.float64)
+    G, dr = W_heads.shape[0], W_heads.shape[1]
+    out = np.zeros((G, len(seg.spans), dr))
+    for i, (b, e) in enumerate(seg.spans):
+        w = span_weights(np.asarray(H, dtype=np.float64)[b:e], wmode)
+        for g in range(G):
+            out[g, i] = to_storage(routing_summary(np.asarray(K)[b:e], w, W_heads[g]), dtype)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# prefill: truncated bases  [SeKV blog 2.2 Eq. (6)-(8)]
+# ---------------------------------------------------------------------------
+def truncated_basis(X, r: int, dtype: str, gate=None):
+    """Rank-r_S truncated SVD of X (|S| x d), r_S = min(r, |S|, d), as two stored
+    factors with A @ B = sum_{i <= r_S} m_i sigma_i u_i v_i^T (Eq. (6)); the rank
+    gate m (components in descending singular-value order) is 1 when not given.
+
+    Factor split: if |S| <= d, A = U_r (|S| x r_S) and B = M_r Sigma_r V_r^T;
+    otherwise A = U_r Sigma_r and B = M_r V_r^T (r_S x d), M_r = diag(m_1..m_rS).
     """
     X = np.asarray(X, dtype=np.float64)
     ns, d = X.shape
     rs = min(r, ns, d)
     U, s, Vt = np.linalg.svd(X, full_matrices=False)
+    m = np.ones(rs) if gate is None else np.asarray(gate, dtype=np.float64)[:rs]
     if ns <= d:
         A = U[:, :rs]
-        B = s[:rs, None] * Vt[:rs]
+        B = (m * s[:rs])[:, None] * Vt[:rs]
     else:
         A = U[:, :rs] * s[None, :rs]
-        B = Vt[:rs]
+        B = m[:, None] * Vt[:rs]
     return to_storage(A, dtype), to_storage(B, dtype)
 
 
-def span_bases(K, V, seg: Segmentation, r: int, dtype: str):
-    """(A_S, B_S, C_S, D_S) per span: K_S ~ A_S B_S and V_S ~ C_S D_S."""
+def span_bases(K, V, seg: Segmentation, r: int, dtype: str, gates=None):
+    """(A_S, B_S, C_S, D_S) per span: K_S ~ A_S B_S and V_S ~ C_S D_S. ``gates``
+    ([m][2][r], keys then values) is the rank gate of Eq. (6), 1 when absent."""
     out = []
-    for b, e in seg.spans:
-        A, B = truncated_basis(np.asarray(K)[b:e], r, dtype)
-        C, D = truncated_basis(np.asarray(V)[b:e], r, dtype)
+    for i, (b, e) in enumerate(seg.spans):
+        gk = None if gates is None else gates[i][0]
+        gv = None if gates is None else gates[i][1]
+        A, B = truncated_basis(np.asarray(K)[b:e], r, dtype, gk)
+        C, D = truncated_basis(np.asarray(V)[b:e], r, dtype, gv)
         out.append((A, B, C, D))
     return out
 
@@ -219,6 +256,16 @@ def routing_logits(qh, kbar, inv_norm, logS, scale: float) -> np.ndarray:
     """Eq. (5)'s pre-sigmoid logit with W = I: l_S = q . kbar_S / ||kbar_S|| * scale + log|S|."""
     s = np.asarray(kbar, dtype=np.float64) @ np.asarray(qh, dtype=np.float64)
     return s * np.asarray(inv_norm, dtype=np.float64) * scale + np.asarray(logS, dtype=np.float64)
+
+
+def learned_routing_logits(qh, W, kbar_r, logS) -> np.ndarray:
+    """Eq. (5)'s pre-sigmoid logit with a routing projection: the query is projected
+    by the same W as the keys (a reading), q~ = W q, and
+    l_S = q~ . Kbar_S / sqrt(d') + log|S| with Kbar_S the Eq. (3) summaries."""
+    W = np.asarray(W, dtype=np.float64)
+    qt = W @ np.asarray(qh, dtype=np.float64)
+    dr = W.shape[0]
+    return np.asarray(kbar_r, dtype=np.float64) @ qt / np.sqrt(dr) + np.asarray(logS, dtype=np.float64)
 
 
 def zoom_decisions(ell, theta: float, budget=None) -> np.ndarray:
@@ -292,13 +339,21 @@ class UnitCache:
     inv_norm: np.ndarray
     logS: np.ndarray
     bases: Optional[list]
+    W: Optional[np.ndarray] = None        # [G][d'][d] routing projections (learned form)
+    kbar_r: Optional[np.ndarray] = None   # [G][m][d'] routing summaries (learned form)
 
 
 def build_unit(K, V, H, seg: Segmentation, wmode: str, rank: int, dtype: str,
-               with_bases: bool = True) -> UnitCache:
+               with_bases: bool = True, W=None, gates=None) -> UnitCache:
+    """Everything one (sequence, layer, kv head) needs. ``W`` ([G][d'][d]) switches
+    on the learned routing form; ``gates`` ([m][2][r]) is the rank gate."""
     K = np.asarray(K, dtype=np.float64)
     V = np.asarray(V, dtype=np.float64)
     kbar, vbar, inv_norm, logS = span_summaries(K, V, H, seg, wmode, dtype)
-    bases = span_bases(K, V, seg, rank, dtype) if with_bases else None
+    bases = span_bases(K, V, seg, rank, dtype, gates) if with_bases else None
+    kbar_r = None
+    if W is not None:
+        W = np.asarray(W, dtype=np.float64)
+        kbar_r = routing_summaries(K, H, seg, wmode, W, dtype)
     return UnitCache(K[seg.anchor_pos].copy(), V[seg.anchor_pos].copy(), kbar, vbar,
-                     inv_norm, logS, bases)
+                     inv_norm, logS, bases, W, kbar_r)

@@ -189,6 +189,28 @@ def queries(wl: Workload, step: int = 0, device="cpu", seed: Optional[int] = Non
     return q.to(wl.torch_dtype())
 
 
+def route_projection(wl: Workload, dr: int = 32, device="cpu", seed: Optional[int] = None) -> torch.Tensor:
+    """W [L][Hq][dr][d] ~ N(0, dr/d) in the storage dtype: a seeded stand-in for the
+    trained per-(layer, head) routing projections (no trained weights exist). With
+    q ~ N(0, I) each of the dr projected coordinates then has variance dr, so a dot
+    product with a unit vector divided by sqrt(dr) has unit variance, the same order
+    as the spread of log|S| over the spans."""
+    seed = wl.seed if seed is None else seed
+    g = _gen(device, seed, 5, dr)
+    W = torch.randn(wl.L, wl.Hq, dr, wl.d, generator=g, device=device) * (dr / wl.d) ** 0.5
+    return W.to(wl.torch_dtype())
+
+
+def rank_gates(wl: Workload, m_cap: int, device="cpu", seed: Optional[int] = None) -> torch.Tensor:
+    """Gates [B][L][Hkv][m_cap][2][rank] (fp32) for the keys and the values of every
+    span: a seeded stand-in for a rank predictor's output. About 30 % exactly 1,
+    15 % exactly 0 and the rest uniform in (0.15, 0.7)."""
+    seed = wl.seed if seed is None else seed
+    g = _gen(device, seed, 6, m_cap)
+    u = torch.rand(wl.B, wl.L, wl.Hkv, m_cap, 2, wl.rank, generator=g, device=device)
+    return torch.where(u > 0.7, torch.ones_like(u), torch.where(u < 0.15, torch.zeros_like(u), u))
+
+
 def taus(wl: Workload, seed: Optional[int] = None) -> Optional[torch.Tensor]:
     """Return tau [L][Hq] (float64, CPU) or None when the workload calibrates tau."""
     seed = wl.seed if seed is None else seed

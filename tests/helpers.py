@@ -45,20 +45,32 @@ def h_margin_ok(H_row: np.ndarray, seg) -> bool:
     return np.min(np.abs(H_row - seg.thr)) > 1e-9 * max(seg.sigma, 1e-30)
 
 
-def oracle_units(K, V, H, segs, wl, with_bases=True, units=None):
+def oracle_units(K, V, H, segs, wl, with_bases=True, units=None, W=None, gates=None):
+    """oracle caches per (b, l, kv head); W [L][Hq][dr][d] switches on the learned
+    routing form, gates [B][L][Hkv][m_cap][2][rank] the rank gate"""
     out = {}
     B, L, Hkv = K.shape[0], K.shape[1], K.shape[2]
+    G = wl.Hq // wl.Hkv
     todo = units if units is not None else [(b, l, h) for b in range(B) for l in range(L) for h in range(Hkv)]
     for (b, l, h) in todo:
+        Wh = None if W is None else f64(W[l, h * G:(h + 1) * G])
+        gh = None if gates is None else f64(gates[b, l, h, :len(segs[b].spans)])
         out[(b, l, h)] = O.build_unit(f64(K[b, l, h]), f64(V[b, l, h]), f64(H[b]), segs[b], wl.wmode,
-                                      wl.rank, wl.dtype, with_bases=with_bases)
+                                      wl.rank, wl.dtype, with_bases=with_bases, W=Wh, gates=gh)
     return out
+
+
+def unit_route(qh, unit, g, scale):
+    """routing logits of query head g (within its kv head) for one unit: the learned
+    form when the unit has routing summaries, else the identity form"""
+    if unit.kbar_r is not None:
+        return O.learned_routing_logits(qh, unit.W[g], unit.kbar_r[g], unit.logS)
+    return O.routing_logits(qh, unit.kbar, unit.inv_norm, unit.logS, scale)
 
 
 def oracle_route(q_np, unit, scale):
     """routing logits [G][m] for one unit"""
-    return np.stack([O.routing_logits(q_np[h], unit.kbar, unit.inv_norm, unit.logS, scale)
-                     for h in range(q_np.shape[0])])
+    return np.stack([unit_route(q_np[h], unit, h, scale) for h in range(q_np.shape[0])])
 
 
 def calibrate_theta(ell_rows, quantile, delta=DELTA_L):
@@ -153,6 +165,9 @@ def upload_oracle_cache(cache, segs, units, with_bases=True):
             c.vbar[b, l, kvh, :m] = torch.tensor(u.vbar, dtype=c.dt)
             c.inv_norm[b, l, kvh, :m] = torch.tensor(u.inv_norm, dtype=torch.float32)
             c.logS[b, :m] = torch.tensor(u.logS, dtype=torch.float32)
+            if u.kbar_r is not None and c.kbar_r is not None:
+                G = c.Hq // c.Hkv
+                c.kbar_r[b, l, kvh * G:(kvh + 1) * G, :m] = torch.tensor(u.kbar_r, dtype=c.dt)
     if with_bases:
         pack_bases(c, segs, units)
     torch.cuda.synchronize()
@@ -168,7 +183,7 @@ def budget_with_margin(q, units, segs, theta, scale, G, candidates=range(1, 41),
     for (b, l, kvh), u in units.items():
         for g in range(G):
             h = kvh * G + g
-            ell = O.routing_logits(qn[b, l, h], u.kbar, u.inv_norm, u.logS, scale)
+            ell = unit_route(qn[b, l, h], u, g, scale)
             rows.append(np.sort(ell[ell > theta[l, h]])[::-1])
     for k in candidates:
         capped = [r for r in rows if len(r) > k]
@@ -188,7 +203,7 @@ def oracle_decode(q, units, segs, theta, scale, G, budget=None):
         qg = qn[b, l, kvh * G:(kvh + 1) * G]
         z = np.zeros((G, len(segs[b].spans)), bool)
         for g in range(G):
-            ell = O.routing_logits(qg[g], u.kbar, u.inv_norm, u.logS, scale)
+            ell = unit_route(qg[g], u, g, scale)
             z[g] = O.zoom_decisions(ell, theta[l, kvh * G + g], budget=budget)
             zooms[(b, l, kvh * G + g)] = z[g]
         o, ls = O.decode_unit(qg, u.Ka, u.Va, u.kbar, u.vbar, u.logS, z, u.bases, scale)
@@ -215,8 +230,7 @@ def thetas_with_margin(q, units, segs, wl, scale, G, taus=None, quantile=None, m
         for h in range(Hq):
             kvh = h // G
             for attempt in range(max_tries):
-                ells = [O.routing_logits(f64(q[b, l, h]), units[(b, l, kvh)].kbar,
-                                         units[(b, l, kvh)].inv_norm, units[(b, l, kvh)].logS, scale)
+                ells = [unit_route(f64(q[b, l, h]), units[(b, l, kvh)], h % G, scale)
                         for b in range(B) if (b, l, kvh) in units]
                 allv = np.concatenate(ells) if ells else np.zeros(0)
                 if quantile is not None:

@@ -486,3 +486,96 @@ def test_budget_cap_none_is_the_threshold_rule():
         assert capped.sum() == min(7, z.sum()) and not (capped & ~z).any()
         # the kept logits are the 7 largest passing ones
         np.testing.assert_allclose(np.sort(ell[capped]), np.sort(ell[z])[-7:])
+
+
+# ---------------------------------------------------------------------------
+# Learned-form routing (SeKV blog 2.2 Eq. (3), 2.3 Eq. (5)) and the rank gate
+# (SeKV blog 2.2 Eq. (6))
+# ---------------------------------------------------------------------------
+def test_learned_routing_hand_example():
+    g = _gold("learned_routing_example.json")
+    Kb = O.routing_summary(g["K"], g["w"], g["W"])
+    np.testing.assert_allclose(Kb, np.array(g["y"]) / math.sqrt(g["y_norm_sq"]), rtol=0, atol=1e-15)
+    ell = O.learned_routing_logits(g["q"], g["W"], Kb[None, :], np.array([math.log(g["len"])]))
+    expect = g["qW_dot_y"] / math.sqrt(g["y_norm_sq"]) / math.sqrt(3) + math.log(g["len"])
+    assert ell[0] == pytest.approx(expect, abs=1e-14)
+
+
+def test_identity_projection_is_the_degenerate_form():
+    """W = I (d' = d): Eq. (3) is kbar / ||kbar|| and Eq. (5) is the identity-form
+    routing logit with scale 1/sqrt(d) (pinned by its own hand example)."""
+    rng = np.random.default_rng(21)
+    d = 16
+    K = rng.normal(size=(9, d))
+    w = rng.uniform(0.1, 2.0, size=9)
+    kbar = (w[:, None] * K).sum(0) / w.sum()               # weighted mean, written out
+    Kb = O.routing_summary(K, w, np.eye(d))
+    np.testing.assert_allclose(Kb, kbar / np.linalg.norm(kbar), atol=1e-14)
+    q = rng.normal(size=d)
+    logS = np.array([math.log(9)])
+    ell = O.learned_routing_logits(q, np.eye(d), Kb[None, :], logS)
+    ref = O.routing_logits(q, kbar[None, :], np.array([1 / np.linalg.norm(kbar)]), logS, 1 / math.sqrt(d))
+    assert ell[0] == pytest.approx(ref[0], abs=1e-13)
+
+
+def test_routing_summary_invariances():
+    rng = np.random.default_rng(22)
+    d, dr = 12, 5
+    K = rng.normal(size=(7, d))
+    w = rng.uniform(0.1, 1.0, size=7)
+    W = rng.normal(size=(dr, d))
+    Kb = O.routing_summary(K, w, W)
+    assert np.linalg.norm(Kb) == pytest.approx(1.0, abs=1e-14)
+    # positive scalings of W or of the weights cancel in the normalisation
+    np.testing.assert_allclose(O.routing_summary(K, w, 3.5 * W), Kb, atol=1e-14)
+    np.testing.assert_allclose(O.routing_summary(K, 0.2 * w, W), Kb, atol=1e-14)
+    # a rotation of the routing space rotates the summary and leaves the logit unchanged
+    Q = _orth(rng, dr, dr)
+    np.testing.assert_allclose(O.routing_summary(K, w, Q @ W), Q @ Kb, atol=1e-13)
+    q = rng.normal(size=d)
+    l1 = O.learned_routing_logits(q, W, Kb[None, :], np.array([0.7]))
+    l2 = O.learned_routing_logits(q, Q @ W, (Q @ Kb)[None, :], np.array([0.7]))
+    assert l1[0] == pytest.approx(l2[0], abs=1e-13)
+    # a one-token span: the normalised projection of its key
+    np.testing.assert_allclose(O.routing_summary(K[:1], [2.0], W), W @ K[0] / np.linalg.norm(W @ K[0]),
+                               atol=1e-14)
+
+
+def test_zero_projection_leaves_the_size_prior():
+    rng = np.random.default_rng(23)
+    K = rng.normal(size=(4, 8))
+    Kb = O.routing_summary(K, np.ones(4), np.zeros((3, 8)))
+    assert (Kb == 0).all()
+    ell = O.learned_routing_logits(rng.normal(size=8), np.zeros((3, 8)), Kb[None, :], np.array([math.log(4)]))
+    assert ell[0] == pytest.approx(math.log(4), abs=1e-15)
+
+
+@pytest.mark.parametrize("ns,d", [(12, 20), (20, 12)])
+def test_rank_gate_scales_known_components(ns, d):
+    """Eq. (6) on a matrix of known singular structure: the gated reconstruction is
+    sum_i m_i sigma_i u_i v_i^T over the top r components, in descending order."""
+    rng = np.random.default_rng(ns * 7 + d)
+    k = min(ns, d)
+    U, V = _orth(rng, ns, k), _orth(rng, d, k)
+    s = np.linspace(9.0, 1.0, k) ** 1.3
+    X = (U * s) @ V.T
+    r = 5
+    m = np.array([1.0, 0.0, 0.25, 0.9, 0.5])
+    A, B = O.truncated_basis(X, r, "f64", gate=m)
+    expect = (U[:, :r] * (m * s[:r])) @ V[:, :r].T
+    np.testing.assert_allclose(A @ B, expect, rtol=0, atol=1e-10 * s[0])
+    A1, B1 = O.truncated_basis(X, r, "f64", gate=np.ones(r))
+    A0, B0 = O.truncated_basis(X, r, "f64")
+    np.testing.assert_allclose(A1 @ B1, A0 @ B0, atol=1e-12 * s[0])
+    Az, Bz = O.truncated_basis(X, r, "f64", gate=np.zeros(r))
+    assert np.abs(Az @ Bz).max() == 0.0
+
+
+def test_rank_gate_prefix_meets_eckart_young():
+    rng = np.random.default_rng(31)
+    X = rng.normal(size=(24, 16))
+    lam = np.sort(np.linalg.eigvalsh(X.T @ X))[::-1]      # sigma_i^2 from another routine
+    for k in (1, 3, 6):
+        gate = np.r_[np.ones(k), np.zeros(8 - k)]
+        A, B = O.truncated_basis(X, 8, "f64", gate=gate)
+        assert np.sum((X - A @ B) ** 2) == pytest.approx(np.sum(lam[k:]), rel=1e-9)
