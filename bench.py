@@ -52,6 +52,8 @@ def parse_args(argv=None):
     ap.add_argument("--cache", action="store_true",
                     help="cold workloads: keep fetched bases resident in a device cache across steps "
                          "(the configs fetch every step)")
+    ap.add_argument("--route-dim", type=int, default=0, choices=[0, 32, 64],
+                    help="learned-form routing with a seeded d'-dimensional projection (0: identity form)")
     ap.add_argument("--budget", type=int, default=0,
                     help="zoom budget per (layer, query head), keeping the largest routing logits; 0 = none "
                          "(the configs run without one)")
@@ -209,6 +211,25 @@ def attend_bytes(cache, zmask_host, P):
     return total, zoom_units
 
 
+def route_bytes(cache, learned):
+    """Algorithmic bytes of one ROUTE call without a budget. Identity form: per
+    (b, l, kv head) the kbar rows, 1/||kbar|| and log|S| once, the G queries and the
+    G mask rows. Learned form: per (b, l, query head) its dr-wide routing summaries,
+    log|S|, its query and d' x d projection, and its mask row."""
+    c = cache
+    s = 2 if c.dtype_name == "bf16" else 4
+    G = c.Hq // c.Hkv
+    mw = c.m_cap // 32
+    tot = 0
+    for b in range(c.B):
+        m = int(c.m_count[b])
+        if learned:
+            tot += c.L * c.Hq * (m * c.dr * s + m * 4 + c.d * s + c.dr * c.d * s + mw * 4)
+        else:
+            tot += c.L * c.Hkv * (m * c.d * s + 8 * m + G * c.d * s + G * mw * 4)
+    return tot
+
+
 def zoom_rate(cache, zmask_host):
     import numpy as np
     c = cache
@@ -224,31 +245,35 @@ def zoom_rate(cache, zmask_host):
 def _oracle_unit_task(args):
     import numpy as np
     import oracle as O
-    kv_path, H, alpha, window, wmode, rank, dtype, q, theta, quantile, scale, reps, budget = args
+    kv_path, H, alpha, window, wmode, rank, dtype, q, theta, quantile, scale, reps, budget, W = args
     with np.load(kv_path) as f:
         K, V = f["K"].astype(np.float64), f["V"].astype(np.float64)
     seg = O.segment(H, alpha, window)
     t0 = time.perf_counter()
-    u = O.build_unit(K, V, H, seg, wmode, rank, dtype)
+    u = O.build_unit(K, V, H, seg, wmode, rank, dtype, W=W)
     t_build = time.perf_counter() - t0
+
+    def route(g):
+        if W is not None:
+            return O.learned_routing_logits(q[g], u.W[g], u.kbar_r[g], u.logS)
+        return O.routing_logits(q[g], u.kbar, u.inv_norm, u.logS, scale)
+
     if theta is None:             # calibrate on the oracle's own routing logits
         theta = []
         for g in range(q.shape[0]):
-            x = np.sort(O.routing_logits(q[g], u.kbar, u.inv_norm, u.logS, scale))
+            x = np.sort(route(g))
             k = int(round(quantile * (x.size - 1)))
             theta.append(0.5 * (x[min(k, x.size - 1)] + x[min(k + 1, x.size - 1)]))
     times = []
     for _ in range(reps):
         t0 = time.perf_counter()
-        z = np.stack([O.zoom_decisions(O.routing_logits(q[g], u.kbar, u.inv_norm, u.logS, scale), theta[g],
-                                       budget=budget or None)
-                      for g in range(q.shape[0])])
+        z = np.stack([O.zoom_decisions(route(g), theta[g], budget=budget or None) for g in range(q.shape[0])])
         O.decode_unit(q, u.Ka, u.Va, u.kbar, u.vbar, u.logS, z, u.bases, scale)
         times.append(time.perf_counter() - t0)
     return t_build, times
 
 
-def oracle_sample(wl, H, KV_units, q, theta, reps, workers, quantile=None, budget=0):
+def oracle_sample(wl, H, KV_units, q, theta, reps, workers, quantile=None, budget=0, W=None):
     """Time the oracle on the sampled (layer, kv head) units (one per process of a
     spawn pool). K/V of each unit go through a temporary .npz file (float32 holds
     the bf16 values exactly). Returns per-unit build seconds and decode seconds."""
@@ -262,8 +287,9 @@ def oracle_sample(wl, H, KV_units, q, theta, reps, workers, quantile=None, budge
             path = os.path.join(tmp, f"u{i}.npz")
             np.savez(path, K=K, V=V)
             th = None if theta is None else theta[l, h * G:(h + 1) * G]
+            Wu = None if W is None else W[l, h * G:(h + 1) * G]
             tasks.append((path, H, wl.alpha, wl.window, wl.wmode, wl.rank, wl.dtype,
-                          q[l, h * G:(h + 1) * G], th, quantile, scale, reps, budget))
+                          q[l, h * G:(h + 1) * G], th, quantile, scale, reps, budget, Wu))
         ctx = mp.get_context("spawn")
         saved = {k: os.environ.get(k) for k in _BLAS_ENV}
         os.environ.update({k: "1" for k in _BLAS_ENV})      # one BLAS thread per worker process
@@ -320,6 +346,9 @@ def run_sekv(args, rank, world, local_rank):
     K, V = gen.keys_values(wl, spikes, device=dev)
     cache = P.SpanCache(wl.B, wl.L, wl.Hq, wl.Hkv, wl.n, wl.d, wl.dtype, a_cap, m_cap, wl.rank,
                         home=None, device=dev)
+    learned = args.route_dim > 0
+    if learned:
+        cache.set_routing(gen.route_projection(wl, args.route_dim, device=dev))
     # ---- prefill build, timed by step
     ev = lambda: torch.cuda.Event(enable_timing=True)
     seg_e = [ev(), ev()]
@@ -407,7 +436,8 @@ def run_sekv(args, rank, world, local_rank):
     if cold:
         d_route = cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud)
         d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_ATTEND, O=O, lse=lse, slot=fetcher.slot_dev,
-                                   arena=fetcher.arena, zmask=zm if bud else None, budget=bud, zoom_hint=zoom_hint)
+                                   arena=fetcher.arena, zmask=zm if (bud or learned) else None, budget=bud,
+                                   zoom_hint=zoom_hint)
     else:
         d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_FUSED, O=O, lse=lse, zmask=zm, budget=bud,
                                    zoom_hint=zoom_hint)
@@ -511,7 +541,9 @@ def run_sekv(args, rank, world, local_rank):
     if want_cpu:
         qs = qpool[warm].double().cpu().numpy()[0]
         th = theta.double().cpu().numpy()
-        t_build, t_dec = oracle_sample(wl, H0, cpu_units, qs, th, reps=2, workers=workers, budget=args.budget)
+        Wn = cache.route_W.double().cpu().numpy() if learned else None
+        t_build, t_dec = oracle_sample(wl, H0, cpu_units, qs, th, reps=2, workers=workers, budget=args.budget,
+                                       W=Wn)
         per_unit = statistics.mean(min(t) for t in t_dec)
         units_total = wl.B * wl.L * wl.Hkv
         oracle_step_s = per_unit * units_total / workers
@@ -523,7 +555,15 @@ def run_sekv(args, rank, world, local_rank):
 
     # ROUTE + ATTEND + merge (cold) or FUSED + merge (hot); a budget adds the cap
     # kernel, and on the hot path the routing pass before the capped FUSED pass
-    launches_per_step = (3 + (1 if args.budget else 0)) if cold else (2 + (2 if args.budget else 0))
+    # (learned routing: its own routing kernel before the attention pass)
+    if cold:
+        launches_per_step = 3 + (1 if args.budget else 0)
+    elif learned:
+        launches_per_step = 3 + (1 if args.budget else 0)
+    else:
+        launches_per_step = 2 + (2 if args.budget else 0)
+    rb = route_bytes(cache, learned)
+    route_avg = statistics.mean(route_ms)
     from sekv_synth import WORKLOADS as _WL
     full_size = (wl.L, wl.n) == (_WL[wl.name].L, _WL[wl.name].n)
     kv_total = kv_bytes
@@ -538,10 +578,15 @@ def run_sekv(args, rank, world, local_rank):
                    "anchors": int(cache.a_count.sum()), "spans": int(cache.m_count.sum()),
                    "l2": f"inputs larger than L2 ({alg_bytes / 1e6:.0f} MB read per ATTEND)",
                    "parallelism": f"replicas x{world} (no collective)",
-                   **({"budget": args.budget} if args.budget else {})},
+                   **({"budget": args.budget} if args.budget else {}),
+                   **({"routing": f"learned form, d'={args.route_dim} (seeded projection)"} if learned else {})},
         "decode_attn": {"us_per_step": attn_avg * 1e3, "steps_per_s": 1e3 / attn_avg,
                         "alg_bytes_per_step": int(alg_bytes), "GBps": achieved},
-        "route_us": statistics.mean(route_ms) * 1e3,
+        "route_us": route_avg * 1e3,
+        **({"route": {"form": "learned" if learned else "identity", "alg_bytes": rb,
+                      "GBps": rb / (route_avg * 1e-3) / 1e9, "frac": rb / (route_avg * 1e-3) / 1e9 / peak,
+                      "note": "the ROUTE call of the cold path (no budget): summaries, log|S|, queries, "
+                              "projections and mask words"}} if cold and route_avg > 0 else {}),
         "zoom_rate": zr,
         "zoom_hint": zoom_hint,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -594,8 +639,9 @@ def run_reference(args):
     taus = gen.taus(wl)
     theta = O.tau_to_theta(taus.numpy()) if taus is not None else None
     reps = min(5, max(1, args.steps))
+    W = gen.route_projection(wl, args.route_dim).double().numpy() if args.route_dim else None
     t_build, t_dec = oracle_sample(wl, H0, units, q, theta, reps=reps, workers=workers,
-                                   quantile=wl.tau_a, budget=args.budget)
+                                   quantile=wl.tau_a, budget=args.budget, W=W)
     per_unit = [min(t) for t in t_dec]
     units_total = wl.B * wl.L * wl.Hkv
     step_s = statistics.mean(per_unit) * units_total / workers

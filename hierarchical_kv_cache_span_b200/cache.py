@@ -74,6 +74,24 @@ class SpanCache:
             self.alloc_home(home)
         self._bws = None
         self._dws = {}
+        self.route_W = None      # learned-form routing projections [L][Hq][dr][d]
+        self.kbar_r = None       # routing summaries [B][L][Hq][m_cap][dr]
+        self.dr = 0
+        self._zscratch = None
+
+    def set_routing(self, W: Optional[torch.Tensor]):
+        """Learned-form routing (SeKV blog 2.2 Eq. (3), 2.3 Eq. (5)): W [L][Hq][dr][d] in
+        the storage dtype on the cache's device, dr 32 or 64; None returns to the
+        identity form. The summaries are written by the next SUMMARY build step."""
+        if W is None:
+            self.route_W, self.kbar_r, self.dr = None, None, 0
+            return self
+        if tuple(W.shape[:2]) != (self.L, self.Hq) or W.shape[3] != self.d or W.dtype != self.dt:
+            raise ValueError(f"W must be [{self.L}][{self.Hq}][dr][{self.d}] {self.dt}")
+        self.route_W = W.to(self.device).contiguous()
+        self.dr = int(W.shape[2])
+        self.kbar_r = torch.zeros(self.B, self.L, self.Hq, self.m_cap, self.dr, dtype=self.dt, device=self.device)
+        return self
 
     def alloc_home(self, kind: str, region: Optional[int] = None):
         """Allocate the basis home: ``kind`` 'device' (hot) or 'host' (pinned, cold).
@@ -97,7 +115,7 @@ class SpanCache:
 
     # ------------------------------------------------------------------ build
     def build_desc(self, H, K, V, alpha, window, wmode, max_sweeps=15, steps=S.SEKV_BUILD_ALL,
-                   l0=0, l1=None) -> S.sekv_build_desc:
+                   l0=0, l1=None, rank_gate=None) -> S.sekv_build_desc:
         d = S.sekv_build_desc()
         d.H, d.K, d.V = _ptr(H), _ptr(K), _ptr(V)
         d.a_count, d.m_count, d.anchor_pos = _ptr(self.a_count), _ptr(self.m_count), _ptr(self.anchor_pos)
@@ -112,6 +130,12 @@ class SpanCache:
         d.a_cap, d.m_cap, d.window = self.a_cap, self.m_cap, window
         d.wmode = _WMODE[wmode] if isinstance(wmode, str) else int(wmode)
         d.rank, d.max_sweeps, d.steps = self.rank, max_sweeps, steps
+        d.route_W, d.kbar_r, d.Hq, d.dr = _ptr(self.route_W), _ptr(self.kbar_r), self.Hq, self.dr
+        if rank_gate is not None:
+            if tuple(rank_gate.shape) != (self.B, self.L, self.Hkv, self.m_cap, 2, self.rank) or \
+                    rank_gate.dtype != torch.float32 or not rank_gate.is_contiguous():
+                raise ValueError("rank_gate must be contiguous fp32 [B][L][Hkv][m_cap][2][rank]")
+        d.rank_gate = _ptr(rank_gate)
         need = S.sekv_build_workspace_bytes(d)
         if need and (self._bws is None or self._bws.numel() < need):
             self._bws = torch.empty(need, dtype=torch.uint8, device=self.device)
@@ -120,8 +144,8 @@ class SpanCache:
         return d
 
     def build(self, H, K, V, alpha, window, wmode, max_sweeps=15, steps=S.SEKV_BUILD_ALL, l0=0,
-              l1=None, stream=None):
-        d = self.build_desc(H, K, V, alpha, window, wmode, max_sweeps, steps, l0, l1)
+              l1=None, stream=None, rank_gate=None):
+        d = self.build_desc(H, K, V, alpha, window, wmode, max_sweeps, steps, l0, l1, rank_gate)
         S.check(S.sekv_build_spans(d, _stream(stream)), "sekv_build_spans")
         if steps & S.SEKV_BUILD_SCAN:
             self._rows_hint = None          # re-read from the new counts at the next decode_desc
@@ -149,7 +173,13 @@ class SpanCache:
         if arena is None and self.home_kind == "device":
             arena = self.home
         d.arena, d.slot = _ptr(arena), _ptr(slot)
+        if zmask is None and self.route_W is not None:
+            # the learned routing pass hands its decisions to attention through a mask
+            if self._zscratch is None:
+                self._zscratch = self.new_zmask()
+            zmask = self._zscratch
         d.O, d.lse, d.zmask, d.route_logits = _ptr(O), _ptr(lse), _ptr(zmask), _ptr(route_logits)
+        d.route_W, d.kbar_r, d.dr = _ptr(self.route_W), _ptr(self.kbar_r), self.dr
         d.dev_status = _ptr(self.status)
         d.region_elems = self.region
         d.scale = float(1.0 / math.sqrt(self.d) if scale is None else scale)

@@ -68,6 +68,15 @@ sekv_status check_build(const sekv_build_desc* d) {
         SEKV_REQUIRE(aligned(d->Ka, 16) && aligned(d->Va, 16) && aligned(d->kbar, 16) && aligned(d->vbar, 16),
                      "build/summary: Ka, Va, kbar, vbar must be 16-byte aligned");
         SEKV_REQUIRE(d->wmode >= SEKV_W_UNIFORM && d->wmode <= SEKV_W_SOFTMAX, "build: wmode %d", d->wmode);
+        if (d->route_W) {
+            SEKV_REQUIRE(d->kbar_r && aligned(d->route_W, 16) && aligned(d->kbar_r, 16),
+                         "build/summary: route_W needs kbar_r; both 16-byte aligned");
+            if (!sekv::route_summary_supported(*d))
+                return fail(SEKV_ERR_UNSUPPORTED,
+                            "build/summary: routing summaries for Hq=%d, Hkv=%d, dr=%d, d=%d, dtype=%d not "
+                            "supported (Hq a multiple of Hkv, Hq/Hkv <= 8, dr 32 or 64, W within shared memory)",
+                            d->Hq, d->Hkv, d->dr, d->d, d->dtype);
+        }
     }
     if (d->steps & SEKV_BUILD_BASES) {
         SEKV_REQUIRE(d->basis_home && d->blk_off && d->m_count && d->span_beg && d->span_end,
@@ -96,6 +105,12 @@ sekv_status check_decode(const sekv_decode_desc* d, bool with_workspace = true) 
                  "decode: nsplit, rows_hint, budget and zoom_hint must be >= 0");
     SEKV_REQUIRE(d->budget == 0 || d->zmask, "decode: a budget needs the zmask buffer (output of ROUTE / FUSED, "
                                              "input of ATTEND)");
+    if (d->route_W) {
+        SEKV_REQUIRE(d->kbar_r && d->zmask && aligned(d->kbar_r, 16),
+                     "decode: learned routing (route_W) needs kbar_r (16-byte aligned) and the zmask buffer");
+        if (!sekv::route_learned_supported(*d))
+            return fail(SEKV_ERR_UNSUPPORTED, "decode: routing dimension dr = %d (32 or 64)", d->dr);
+    }
     if (!sekv::decode_supported(*d))
         return fail(SEKV_ERR_UNSUPPORTED, "decode: d=%d, Hq/Hkv=%d, rank=%d, dtype=%d not compiled", d->d,
                     d->Hq / d->Hkv, d->rank, d->dtype);

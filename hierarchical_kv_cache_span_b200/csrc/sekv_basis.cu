@@ -2,7 +2,8 @@
 //
 // SeKV blog walkthrough, section 2.2, Eq. (6)-(8): each span's key matrix (and
 // value matrix) is stored as a truncated SVD, K_S ~ sum_{i<=R} m_i sigma_i u_i v_i^T;
-// with the rank gate fixed to m_i = 1 for i <= r this is the rank-r truncation.
+// with the rank gate m_i = 1 for i <= r this is the rank-r truncation; a caller-
+// supplied gate scales component i (row i of the stored B or D factor).
 //
 // Per (sequence, layer, kv head, span, K-or-V) problem with X = the span's rows
 // (|S| x d) and N = min(|S|, d):
@@ -68,6 +69,7 @@ struct BasisArgs {
     const int64_t* blk_off;
     void* home;
     int32_t* status;
+    const float* gate;   // null or [B][L][Hkv][m_cap][2][rank] rank gate m_{S,i} (Eq. (6))
     int64_t region;
     int L, l0, Lr, Hkv, n, d, m_cap, rank, max_sweeps;
 };
@@ -283,6 +285,10 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
         const int r8 = round8(rS);
         const int64_t pa = block_ac_elems(len, rS);
         const bool rows_form = len <= d;            // G = X X^T
+        // rank gate of component j (descending singular value), folded into row j of B / D
+        const float* gate = a.gate ? a.gate + (((((int64_t)b * a.L + l) * a.Hkv + kvh) * a.m_cap + S) * 2 + which) *
+                                                  (int64_t)a.rank
+                                   : nullptr;
         const char* src = reinterpret_cast<const char*>(which ? a.V : a.K) +
                           ((((int64_t)b * a.L + l) * a.Hkv + kvh) * a.n + beg) * (int64_t)d * E::bytes;
         char* blk = reinterpret_cast<char*>(a.home) +
@@ -374,13 +380,14 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
                 const int cj = sel[j];
                 float acc = 0.f;
                 for (int t = 0; t < len; ++t) acc = fmaf(Vm[t * ld + cj], xs(t, k), acc);
-                store1<DT>(fac_col, tile8_index(j, k, d), acc);
+                store1<DT>(fac_col, tile8_index(j, k, d), gate ? acc * gate[j] : acc);
             }
         } else {
             // B[j][k] = V[k][sel j];  A[t][j] = sum_k X[t][k] V[k][sel j]
             for (int i = tid; i < rS * d; i += T) {
                 const int j = i / d, k = i % d;
-                store1<DT>(fac_col, tile8_index(j, k, d), Vm[k * ld + sel[j]]);
+                const float v = Vm[k * ld + sel[j]];
+                store1<DT>(fac_col, tile8_index(j, k, d), gate ? v * gate[j] : v);
             }
             for (int t0 = 0; t0 < len; t0 += kChunkRows) {
                 const int rows = min(kChunkRows, len - t0);
@@ -447,7 +454,8 @@ cudaError_t launch_basis(const sekv_build_desc& d, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     classify_kernel<<<d.B, 256, 0, st>>>(d.m_count, d.span_beg, d.span_end, d.m_cap, d.d, w, cap);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    BasisArgs a{d.m_count, d.K, d.V, d.span_beg, d.span_end, d.blk_off, d.basis_home, d.dev_status, d.region_elems,
+    BasisArgs a{d.m_count, d.K, d.V, d.span_beg, d.span_end, d.blk_off, d.basis_home, d.dev_status, d.rank_gate,
+                d.region_elems,
                 d.L, d.l0, d.l1 - d.l0, d.Hkv, d.n, d.d, d.m_cap, d.rank, d.max_sweeps};
     if (d.dtype == SEKV_F32) {
         if ((e = launch_bucket<SEKV_F32, 32>(a, w, 0, cap, st)) != cudaSuccess) return e;

@@ -1842,19 +1842,27 @@ void* decode_static_scratch(cudaError_t* err) {
 // FUSED then attends with the capped mask as input. ATTEND takes the caller's
 // (capped) mask as input.
 cudaError_t launch_decode(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st) {
-    if (d.budget <= 0) return launch_pass(d, p, partials, st, 0);
-    if (d.phase == SEKV_ATTEND) return launch_pass(d, p, partials, st, 1);
+    const bool learned = d.route_W != nullptr;
+    if (!learned && d.budget <= 0) return launch_pass(d, p, partials, st, 0);
+    // the attention pass takes the (capped / learned) mask as input; with learned
+    // routing it must not overwrite the routing logits with identity-form ones
+    sekv_decode_desc att = d;
+    if (learned) att.route_logits = nullptr;
+    if (d.phase == SEKV_ATTEND) return launch_pass(att, p, partials, st, 1);
     sekv_decode_desc r = d;
     r.phase = SEKV_ROUTE;
-    if (!r.route_logits) r.route_logits = reinterpret_cast<float*>(reinterpret_cast<char*>(partials) + p.partial_bytes);
-    cudaError_t e = launch_pass(r, p, partials, st, 0);
+    if (d.budget > 0 && !r.route_logits)
+        r.route_logits = reinterpret_cast<float*>(reinterpret_cast<char*>(partials) + p.partial_bytes);
+    cudaError_t e = learned ? launch_route_learned(r, st) : launch_pass(r, p, partials, st, 0);
     if (e != cudaSuccess) return e;
-    const int Lr = d.l1 - d.l0;
-    cap_kernel<<<d.B * Lr * d.Hq, 256, 0, st>>>(r.route_logits, d.zmask, d.m_count, d.L, d.l0, Lr, d.Hq, d.m_cap,
-                                                 d.budget);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (d.budget > 0) {
+        const int Lr = d.l1 - d.l0;
+        cap_kernel<<<d.B * Lr * d.Hq, 256, 0, st>>>(r.route_logits, d.zmask, d.m_count, d.L, d.l0, Lr, d.Hq,
+                                                     d.m_cap, d.budget);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if (d.phase == SEKV_ROUTE) return cudaSuccess;
-    return launch_pass(d, p, partials, st, 1);
+    return launch_pass(att, p, partials, st, 1);
 }
 
 }  // namespace sekv

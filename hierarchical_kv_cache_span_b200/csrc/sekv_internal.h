@@ -10,6 +10,7 @@ namespace sekv {
 cudaError_t launch_scan(const sekv_build_desc& d, cudaStream_t st);
 cudaError_t launch_layout(const sekv_build_desc& d, bool check_region, cudaStream_t st);
 cudaError_t launch_summary(const sekv_build_desc& d, cudaStream_t st);
+bool route_summary_supported(const sekv_build_desc& d);   // route_W shapes the summary step handles
 
 // basis build: workspace layout and launch
 size_t basis_workspace_bytes(const sekv_build_desc& d);
@@ -27,6 +28,9 @@ DecodePlan plan_decode(const sekv_decode_desc& d);
 size_t decode_workspace_bytes(const sekv_decode_desc& d);
 bool decode_supported(const sekv_decode_desc& d);
 cudaError_t launch_decode(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st);
+// learned-form routing pass (zoom mask + optional logits); defined with its kernel
+cudaError_t launch_route_learned(const sekv_decode_desc& d, cudaStream_t st);
+bool route_learned_supported(const sekv_decode_desc& d);
 cudaError_t launch_merge_parts(const float* O_parts, const float* lse_parts, int nparts, int64_t rows, int d,
                                float* O, float* lse, cudaStream_t st);
 size_t decode_static_scratch_bytes();

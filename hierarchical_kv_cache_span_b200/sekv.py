@@ -42,10 +42,12 @@ class sekv_build_desc(C.Structure):
         ("logS", _p), ("blk_off", _p), ("stats", _p),
         ("Ka", _p), ("Va", _p), ("kbar", _p), ("vbar", _p), ("inv_norm", _p),
         ("basis_home", _p), ("dev_status", _p), ("workspace", _p),
+        ("route_W", _p), ("kbar_r", _p), ("rank_gate", _p),
         ("region_elems", _i64), ("workspace_bytes", _i64), ("alpha", C.c_double),
         ("B", _i32), ("L", _i32), ("Hkv", _i32), ("n", _i32), ("d", _i32), ("dtype", _i32),
         ("l0", _i32), ("l1", _i32), ("a_cap", _i32), ("m_cap", _i32), ("window", _i32),
-        ("wmode", _i32), ("rank", _i32), ("max_sweeps", _i32), ("steps", _i32), ("reserved", _i32),
+        ("wmode", _i32), ("rank", _i32), ("max_sweeps", _i32), ("steps", _i32), ("Hq", _i32),
+        ("dr", _i32), ("reserved", _i32),
     ]
 
 
@@ -54,12 +56,13 @@ class sekv_decode_desc(C.Structure):
         ("q", _p), ("a_count", _p), ("m_count", _p), ("span_beg", _p), ("span_end", _p),
         ("logS", _p), ("blk_off", _p), ("Ka", _p), ("Va", _p), ("kbar", _p), ("vbar", _p),
         ("inv_norm", _p), ("theta", _p), ("arena", _p), ("slot", _p), ("O", _p), ("lse", _p),
-        ("zmask", _p), ("route_logits", _p), ("dev_status", _p), ("workspace", _p),
+        ("zmask", _p), ("route_logits", _p), ("route_W", _p), ("kbar_r", _p), ("dev_status", _p),
+        ("workspace", _p),
         ("region_elems", _i64), ("workspace_bytes", _i64), ("scale", C.c_float),
         ("B", _i32), ("L", _i32), ("Hq", _i32), ("Hkv", _i32), ("d", _i32), ("dtype", _i32),
         ("l0", _i32), ("l1", _i32), ("a_cap", _i32), ("m_cap", _i32), ("rank", _i32),
         ("phase", _i32), ("nsplit", _i32), ("rows_hint", _i32), ("budget", _i32), ("zoom_hint", _i32),
-        ("reserved", _i32),
+        ("dr", _i32), ("reserved", _i32),
     ]
 
 

@@ -106,7 +106,8 @@ typedef void* sekv_event_t;    /* a cudaEvent_t */
  * conflict-free shared-memory matrix loads; a run of token (or basis-row) groups
  * is one contiguous byte range. Padding is zero. The block size,
  * 2 len8 r8 + 2 r8 d, is a multiple of 64 elements (sekv_block_elems).
- * K_S ~ A B, V_S ~ C D (SeKV blog 2.2, Eq. (6)-(8) with the rank gate fixed to 1).
+ * K_S ~ A B, V_S ~ C D (SeKV blog 2.2, Eq. (6)-(8); the rank gate, 1 unless
+ * sekv_build_desc.rank_gate is given, is folded into B and D).
  */
 int64_t sekv_block_elems(int32_t len, int32_t d, int32_t rank);
 /* An upper bound of the region size for any segmentation with <= m_cap spans of a
@@ -141,6 +142,17 @@ typedef struct sekv_build_desc {
     void* basis_home;        /* [B][L][region_elems]                                       */
     int32_t* dev_status;     /* device int32, required                                     */
     void* workspace;         /* device, sekv_build_workspace_bytes() bytes, 256-B aligned  */
+    /* learned-form routing summaries (SeKV blog 2.2 Eq. (3)); optional, SUMMARY step:
+     *   kbar_r[b][l][h][S] = y / ||y||_2,  y = sum_{t in S} w_t W^(l,h) K_t = (sum w) W^(l,h) kbar_S
+     * for every query head h (its kv head is h / (Hq/Hkv)); the positive weight sum
+     * cancels, so y is formed from the unrounded weighted mean; a zero y gives 0.  */
+    const void* route_W;     /* NULL (identity routing) or [L][Hq][dr][d] W^(l,h) (storage dtype) */
+    void* kbar_r;            /* [B][L][Hq][m_cap][dr] routing summaries (storage dtype, written)  */
+    /* rank gate (SeKV blog 2.2 Eq. (6)): K^_S = sum_i m_i sigma_i u_i v_i^T, same for V.
+     * Optional, BASES step; folded into the stored factors (row i of B / D times m_i). */
+    const float* rank_gate;  /* NULL (all 1) or [B][L][Hkv][m_cap][2][rank]: the key gates then the
+                                value gates of span S, component i in descending singular-value
+                                order (i < rS is used)                                       */
     int64_t region_elems;    /* elements per (b, l) region of basis_home                   */
     int64_t workspace_bytes;
     double alpha;            /* boundary sensitivity: boundary iff H_t > mu + alpha*sigma   */
@@ -152,6 +164,8 @@ typedef struct sekv_build_desc {
     int32_t rank;            /* basis rank r >= 1                                           */
     int32_t max_sweeps;      /* Jacobi sweep limit (e.g. 15)                               */
     int32_t steps;           /* SEKV_BUILD_* mask                                           */
+    int32_t Hq;              /* query heads (with route_W: a multiple of Hkv, Hq/Hkv <= 8)  */
+    int32_t dr;              /* routing dimension d' (with route_W: 32 or 64)               */
     int32_t reserved;
 } sekv_build_desc;
 
@@ -185,6 +199,13 @@ typedef struct sekv_decode_desc {
     uint32_t* zmask;         /* optional [B][L][Hq][m_cap/32] zoom bits (bit S%32 of word   */
                              /* S/32); required for ROUTE. Bits of spans >= m_count are 0  */
     float* route_logits;     /* optional [B][L][Hq][m_cap] routing logits l_S              */
+    /* learned-form routing (SeKV blog 2.3 Eq. (5)); optional. With route_W the routing
+     * logit is l_S = (W^(l,h) q_h) . kbar_r_S / sqrt(dr) + logS_S, computed by a separate
+     * routing pass; zmask is then required in every phase (ROUTE writes it; FUSED
+     * writes it and attends with it; ATTEND reads it as input, no re-routing). The
+     * coarse entries of Stage 2 still use kbar / vbar in the key/value space.       */
+    const void* route_W;     /* NULL (identity routing) or [L][Hq][dr][d] (storage dtype)  */
+    const void* kbar_r;      /* [B][L][Hq][m_cap][dr] routing summaries from the build     */
     int32_t* dev_status;     /* device int32, required                                     */
     void* workspace;         /* device, sekv_decode_workspace_bytes() bytes, 256-B aligned */
     int64_t region_elems;
@@ -211,13 +232,15 @@ typedef struct sekv_decode_desc {
                                 decode variant that hands small spans whole to one warp
                                 is used, which is faster when most spans zoom and slower
                                 when few do. Results are the same either way.            */
+    int32_t dr;              /* routing dimension d' with route_W (32 or 64)                */
     int32_t reserved;
 } sekv_decode_desc;
 
 size_t sekv_decode_workspace_bytes(const sekv_decode_desc* desc);
 /* Enqueue one decode step for layers [l0, l1) on `stream`. Hq/Hkv must be 1, 2, 4
- * or 8 and d 64 or 128. Routing logit per query head h and span S:
- *   l_S = (q_h . kbar_S) * inv_norm_S * scale + logS_S, zoom iff l_S > theta[l][h];
+ * or 8 and d 64 or 128. Routing logit per query head h and span S (identity form):
+ *   l_S = (q_h . kbar_S) * inv_norm_S * scale + logS_S, zoom iff l_S > theta[l][h]
+ * (learned form: see route_W);
  * attention over anchors (q.Ka*scale), non-zoomed spans (q.kbar*scale + logS,
  * value vbar) and the tokens of zoomed spans ((A_S (B_S q))*scale, value C_S^T-
  * weighted D_S rows), all in one softmax. */
