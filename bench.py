@@ -54,6 +54,8 @@ def parse_args(argv=None):
                          "(the configs fetch every step)")
     ap.add_argument("--route-dim", type=int, default=0, choices=[0, 32, 64],
                     help="learned-form routing with a seeded d'-dimensional projection (0: identity form)")
+    ap.add_argument("--latency-form", action="store_true",
+                    help="also time the step as per-layer decode calls replayed from one CUDA graph")
     ap.add_argument("--budget", type=int, default=0,
                     help="zoom budget per (layer, query head), keeping the largest routing logits; 0 = none "
                          "(the configs run without one)")
@@ -581,7 +583,9 @@ def run_sekv(args, rank, world, local_rank):
                    **({"budget": args.budget} if args.budget else {}),
                    **({"routing": f"learned form, d'={args.route_dim} (seeded projection)"} if learned else {})},
         "decode_attn": {"us_per_step": attn_avg * 1e3, "steps_per_s": 1e3 / attn_avg,
-                        "alg_bytes_per_step": int(alg_bytes), "GBps": achieved},
+                        "alg_bytes_per_step": int(alg_bytes), "GBps": achieved,
+                        "us_p10_median_p90": [pct(attn_ms, 10) * 1e3, pct(attn_ms, 50) * 1e3,
+                                              pct(attn_ms, 90) * 1e3]},
         "route_us": route_avg * 1e3,
         **({"route": {"form": "learned" if learned else "identity", "alg_bytes": rb,
                       "GBps": rb / (route_avg * 1e-3) / 1e9, "frac": rb / (route_avg * 1e-3) / 1e9 / peak,
@@ -610,11 +614,101 @@ def run_sekv(args, rank, world, local_rank):
             out["fetch"]["resident_spans_per_step"] = statistics.mean(f["resident"] for f in fetched)
             out["fetch"]["copied_spans_per_step"] = statistics.mean(f["spans"] for f in fetched)
             out["config"]["fetch"] = "cached across steps"
+    if cold:
+        try:
+            pk = h2d_peak(torch, dev)
+            out["fetch"]["h2d_peak_GBps"] = pk
+            out["fetch"]["frac_of_h2d_peak"] = out["fetch"]["GBps"] / pk
+        except Exception as e:                        # context only; never fatal to the line
+            out["fetch"]["h2d_peak_GBps"] = None
+            out["fetch"]["h2d_peak_error"] = f"{type(e).__name__}: {e}"
     if e2e:
         out["e2e"] = e2e
     if cpu:
         out["cpu_baseline"] = cpu
+    if args.latency_form:
+        out["latency_form"] = latency_form(P, torch, cache, wl, q_buf, qpool[warm], theta, O, lse, zm, fetcher,
+                                           cold, learned, bud, zoom_hint, steps)
     return out
+
+
+def pct(xs, p):
+    """p-th percentile (nearest rank) of a list of timings"""
+    ys = sorted(xs)
+    return ys[min(len(ys) - 1, max(0, int(round(p / 100.0 * (len(ys) - 1)))))]
+
+
+def h2d_peak(torch, dev, nbytes=512 << 20):
+    """pinned host -> device copy rate of one large copy (the ceiling the fetch is held to)"""
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        dst.copy_(src, non_blocking=True)
+    best = None
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dst.copy_(src, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1)
+        best = t if best is None else min(best, t)
+    return nbytes / (best * 1e-3) / 1e9
+
+
+def latency_form(P, torch, cache, wl, q_buf, q, theta, O, lse, zm, fetcher, cold, learned, bud, zoom_hint, steps):
+    """The step as L per-layer decode calls (l0 = l, l1 = l + 1) replayed from one CUDA
+    graph. Cold bases: the graph holds the per-layer ATTEND calls after one ROUTE +
+    fetch outside it (the fetch waits on the host and cannot be captured)."""
+    try:
+        q_buf.copy_(q)
+        if cold:
+            dr_ = cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud)
+            P.check(P.sekv.sekv_decode_attn(dr_, torch.cuda.current_stream().cuda_stream), "route")
+            fetcher.fetch(zm)
+            torch.cuda.current_stream().wait_event(fetcher.done)
+        descs = []
+        for l in range(wl.L):
+            if cold:
+                descs.append(cache.decode_desc(q_buf, theta, phase=P.SEKV_ATTEND, O=O, lse=lse,
+                                               slot=fetcher.slot_dev, arena=fetcher.arena,
+                                               zmask=zm if (bud or learned) else None, budget=bud,
+                                               zoom_hint=zoom_hint, l0=l, l1=l + 1))
+            else:
+                descs.append(cache.decode_desc(q_buf, theta, phase=P.SEKV_FUSED, O=O, lse=lse, zmask=zm,
+                                               budget=bud, zoom_hint=zoom_hint, l0=l, l1=l + 1))
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):                 # one eager pass (first-use setup outside the capture)
+            for d_ in descs:
+                P.check(P.sekv.sekv_decode_attn(d_, side.cuda_stream), "per-layer decode")
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            sid = torch.cuda.current_stream().cuda_stream
+            for d_ in descs:
+                P.check(P.sekv.sekv_decode_attn(d_, sid), "per-layer decode (capture)")
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(max(steps, 5)):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        st = cache.read_status()
+        del g
+        return {"us_per_step": statistics.median(ts) * 1e3, "us_p10": pct(ts, 10) * 1e3, "us_p90": pct(ts, 90) * 1e3,
+                "calls_per_step": wl.L, "status": st,
+                "note": ("per-layer ATTEND calls" if cold else "per-layer FUSED calls") +
+                        " captured in one CUDA graph; L2 is not flushed between replays (each replay reads "
+                        "the whole step, far above L2)"}
+    except Exception as e:                            # reported, never fatal to the main line
+        return {"error": f"{type(e).__name__}: {e}"}
 
 
 def run_reference(args):

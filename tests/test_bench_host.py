@@ -56,3 +56,14 @@ def test_reference_arm_json_contract():
     assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["d2h_bytes_per_step"] == 0
     for k in ("metric", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling", "config"):
         assert k in j
+
+
+def test_percentile_and_flags():
+    sys.path.insert(0, ROOT)
+    import bench
+    xs = [5.0, 1.0, 4.0, 2.0, 3.0]
+    assert bench.pct(xs, 0) == 1.0 and bench.pct(xs, 50) == 3.0 and bench.pct(xs, 100) == 5.0
+    assert bench.pct([7.0], 90) == 7.0
+    a = bench.parse_args(["--latency-form", "--route-dim", "32", "--budget", "4"])
+    assert a.latency_form and a.route_dim == 32 and a.budget == 4
+    assert not bench.parse_args([]).latency_form and bench.parse_args([]).route_dim == 0

@@ -150,6 +150,30 @@ def test_split_count_does_not_change_result():
             assert (lse_gpu - ref[1]).abs().max().item() < 2e-5
 
 
+def test_layer_range_calls_equal_one_call():
+    """per-layer calls (l0 = l, l1 = l + 1, each with its own split plan) write the
+    same masks and, up to split-K summation order, the same O / lse as one call
+    over all layers"""
+    wl = WORKLOADS["c2"].scaled(n=2048, L=3)
+    H, K, V, segs, units, q, theta, scale = _setup(wl)
+    c = _cache(wl)
+    T.upload_oracle_cache(c, segs, units)
+    th = torch.tensor(theta, dtype=torch.float32, device="cuda")
+    qd = q.cuda()
+    zm_f = c.new_zmask()
+    O_f, lse_f = c.decode(qd, th, zmask=zm_f)
+    zm_p = c.new_zmask()
+    O_p, lse_p = c.new_outputs()
+    for l in range(wl.L):
+        c.decode(qd, th, O=O_p, lse=lse_p, zmask=zm_p, l0=l, l1=l + 1)
+    torch.cuda.synchronize()
+    assert c.read_status() == 0
+    assert torch.equal(zm_p, zm_f)
+    assert (O_p - O_f).abs().max().item() < 1e-3
+    assert (lse_p - lse_f).abs().max().item() < 2e-5
+    _compare(wl, c, q, theta, scale, segs, units, O_p, lse_p, zm_p)
+
+
 def test_route_fetch_attend_equals_fused():
     """cold bases in pinned host memory: ROUTE, fetch zoomed bases, ATTEND"""
     P = _lib()

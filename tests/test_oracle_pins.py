@@ -492,13 +492,17 @@ def test_budget_cap_none_is_the_threshold_rule():
 # Learned-form routing (SeKV blog 2.2 Eq. (3), 2.3 Eq. (5)) and the rank gate
 # (SeKV blog 2.2 Eq. (6))
 # ---------------------------------------------------------------------------
-def test_learned_routing_hand_example():
+def _pin_learned_hand_example():
     g = _gold("learned_routing_example.json")
     Kb = O.routing_summary(g["K"], g["w"], g["W"])
     np.testing.assert_allclose(Kb, np.array(g["y"]) / math.sqrt(g["y_norm_sq"]), rtol=0, atol=1e-15)
     ell = O.learned_routing_logits(g["q"], g["W"], Kb[None, :], np.array([math.log(g["len"])]))
     expect = g["qW_dot_y"] / math.sqrt(g["y_norm_sq"]) / math.sqrt(3) + math.log(g["len"])
     assert ell[0] == pytest.approx(expect, abs=1e-14)
+
+
+def test_learned_routing_hand_example():
+    _pin_learned_hand_example()
 
 
 def test_identity_projection_is_the_degenerate_form():
@@ -550,8 +554,7 @@ def test_zero_projection_leaves_the_size_prior():
     assert ell[0] == pytest.approx(math.log(4), abs=1e-15)
 
 
-@pytest.mark.parametrize("ns,d", [(12, 20), (20, 12)])
-def test_rank_gate_scales_known_components(ns, d):
+def _pin_rank_gate_known_components(ns, d):
     """Eq. (6) on a matrix of known singular structure: the gated reconstruction is
     sum_i m_i sigma_i u_i v_i^T over the top r components, in descending order."""
     rng = np.random.default_rng(ns * 7 + d)
@@ -571,6 +574,11 @@ def test_rank_gate_scales_known_components(ns, d):
     assert np.abs(Az @ Bz).max() == 0.0
 
 
+@pytest.mark.parametrize("ns,d", [(12, 20), (20, 12)])
+def test_rank_gate_scales_known_components(ns, d):
+    _pin_rank_gate_known_components(ns, d)
+
+
 def test_rank_gate_prefix_meets_eckart_young():
     rng = np.random.default_rng(31)
     X = rng.normal(size=(24, 16))
@@ -579,3 +587,42 @@ def test_rank_gate_prefix_meets_eckart_young():
         gate = np.r_[np.ones(k), np.zeros(8 - k)]
         A, B = O.truncated_basis(X, 8, "f64", gate=gate)
         assert np.sum((X - A @ B) ** 2) == pytest.approx(np.sum(lam[k:]), rel=1e-9)
+
+
+def test_planted_learned_routing_mistakes_are_caught(monkeypatch):
+    """Plausible misreadings of Eq. (3) / (5), planted in the oracle, fail the hand pin."""
+    real_sum, real_logits = O.routing_summary, O.learned_routing_logits
+
+    def per_token_normalised(Ks, w, W):            # normalises each projected key first
+        P = np.asarray(Ks, float) @ np.asarray(W, float).T
+        P = P / np.linalg.norm(P, axis=1, keepdims=True)
+        y = (np.asarray(w, float)[:, None] * P).sum(0)
+        return y / np.linalg.norm(y)
+
+    def unweighted(Ks, w, W):                      # drops the span weights
+        return real_sum(Ks, np.ones(len(w)), W)
+
+    def key_dim_scale(qh, W, kbar_r, logS):         # 1/sqrt(d) instead of 1/sqrt(d')
+        d, dr = np.asarray(W).shape[1], np.asarray(W).shape[0]
+        return (real_logits(qh, W, kbar_r, logS) - np.asarray(logS)) * math.sqrt(dr) / math.sqrt(d) + logS
+
+    for name, bad in (("routing_summary", per_token_normalised), ("routing_summary", unweighted),
+                      ("learned_routing_logits", key_dim_scale)):
+        monkeypatch.setattr(O, name, bad)
+        with pytest.raises(AssertionError):
+            _pin_learned_hand_example()
+        monkeypatch.undo()
+    _pin_learned_hand_example()
+
+
+def test_planted_reversed_rank_gate_is_caught(monkeypatch):
+    """A gate applied in ascending singular-value order fails the Eq. (6) pin."""
+    real = O.truncated_basis
+
+    def reversed_gate(X, r, dtype, gate=None):
+        return real(X, r, dtype, None if gate is None else np.asarray(gate)[:min(r, *np.shape(X))][::-1])
+    monkeypatch.setattr(O, "truncated_basis", reversed_gate)
+    with pytest.raises(AssertionError):
+        _pin_rank_gate_known_components(12, 20)
+    monkeypatch.undo()
+    _pin_rank_gate_known_components(12, 20)
