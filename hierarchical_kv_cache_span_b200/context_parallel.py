@@ -21,7 +21,7 @@ across the whole context. Batch size 1 (each sequence has its own cuts).
 """
 from __future__ import annotations
 
-from typing import List, Tuple
+from typing import List, Optional, Tuple
 
 import torch
 
@@ -66,10 +66,11 @@ class ContextShard:
     plan() first to learn the cuts from the global segmentation."""
 
     def __init__(self, L, Hq, Hkv, n, d, dtype, a_cap, m_cap, rank_basis, rank: int, world: int,
-                 device="cuda"):
+                 device="cuda", route_W: Optional[torch.Tensor] = None):
         self.L, self.Hq, self.Hkv, self.n, self.d, self.dtype = L, Hq, Hkv, n, d, dtype
         self.a_cap, self.m_cap, self.r = a_cap, m_cap, rank_basis
         self.rank, self.world, self.device = rank, world, torch.device(device)
+        self.route_W = route_W          # learned-form routing projections, the same on every rank
         self.cuts = None
         self.cache = None
         self._seg = None
@@ -91,8 +92,27 @@ class ContextShard:
         self.cuts = shard_cuts(ap, sb, self.n, self.world)
         return self.cuts
 
+    def span_range(self):
+        """[k0, k1): the global indices of this rank's spans (spans are ordered by
+        position, so a shard's spans are a contiguous run of them)."""
+        t0, t1 = self.cuts[self.rank], self.cuts[self.rank + 1]
+        sb = torch.as_tensor(self._seg[1], dtype=torch.int64).reshape(-1).cpu().contiguous()
+        k0 = int(torch.searchsorted(sb, torch.tensor(t0, dtype=torch.int64)))
+        k1 = int(torch.searchsorted(sb, torch.tensor(t1, dtype=torch.int64)))
+        return k0, k1
+
+    def shard_gate(self, rank_gate: torch.Tensor) -> torch.Tensor:
+        """A global rank gate [1][L][Hkv][>= m][2][rank] cut to this shard's spans, in
+        the shard cache's [1][L][Hkv][m_cap][2][rank] layout (zero past its spans)."""
+        k0, k1 = self.span_range()
+        out = torch.zeros(1, self.L, self.Hkv, self.m_cap, 2, self.r, dtype=torch.float32,
+                          device=rank_gate.device)
+        out[:, :, :, :k1 - k0] = rank_gate[:, :, :, k0:k1].to(torch.float32)
+        return out
+
     def build(self, H_full: torch.Tensor, K_slice: torch.Tensor, V_slice: torch.Tensor, alpha: float,
-              window: int, wmode: str, max_sweeps: int = 15):
+              window: int, wmode: str, max_sweeps: int = 15, rank_gate: Optional[torch.Tensor] = None):
+        """``rank_gate`` is the sequence's global gate tensor (indexed by global span)."""
         if self.cuts is None:
             self.plan(H_full, alpha, window)
         t0, t1 = self.cuts[self.rank], self.cuts[self.rank + 1]
@@ -105,6 +125,8 @@ class ContextShard:
                              f"{self.a_cap} / {self.m_cap}")
         c = SpanCache(1, self.L, self.Hq, self.Hkv, ns, self.d, self.dtype, self.a_cap, self.m_cap, self.r,
                       home=None, device=self.device)
+        if self.route_W is not None:
+            c.set_routing(self.route_W)
         c.a_count[0], c.m_count[0] = len(a), len(sb)
         if len(a):
             c.anchor_pos[0, :len(a)] = torch.as_tensor(a, dtype=torch.int32)
@@ -116,8 +138,9 @@ class ContextShard:
         torch.cuda.synchronize(self.device)
         c.alloc_home("device", c.exact_region())
         if t1 > t0:
+            gate = None if rank_gate is None else self.shard_gate(rank_gate).to(self.device)
             c.build(H_slice, K_slice, V_slice, alpha, window, wmode, max_sweeps=max_sweeps,
-                    steps=S.SEKV_BUILD_SUMMARY | S.SEKV_BUILD_BASES)
+                    steps=S.SEKV_BUILD_SUMMARY | S.SEKV_BUILD_BASES, rank_gate=gate)
         self.cache = c
         return self
 

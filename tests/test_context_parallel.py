@@ -67,6 +67,32 @@ def test_cuts_partition_without_splitting_spans(world):
         assert na == len(seg.anchor_pos) and ns == len(seg.spans)
 
 
+def test_shard_gate_slices_the_global_span_range():
+    CP = _cp()
+    wl = WORKLOADS["c1"].scaled(n=2000, seed=3)
+    H, _ = gen.surprisal(wl)
+    seg = O.segment(T.f64(H[0]), wl.alpha, wl.window)
+    m = len(seg.spans)
+    L, Hkv, r, m_cap = 2, 3, 4, ((m + 31) // 32) * 32
+    g = torch.arange(L * Hkv * m * 2 * r, dtype=torch.float32).reshape(1, L, Hkv, m, 2, r)
+    world = 3
+    seen = 0
+    for rank in range(world):
+        sh = CP.ContextShard(L, 4, Hkv, wl.n, 64, "f32", 64, m_cap, r, rank=rank, world=world, device="cpu")
+        sh._seg = (seg.anchor_pos, seg.spans[:, 0], seg.spans[:, 1])
+        sh.cuts = CP.shard_cuts(seg.anchor_pos, seg.spans[:, 0], wl.n, world)
+        k0, k1 = sh.span_range()
+        t0, t1 = sh.cuts[rank], sh.cuts[rank + 1]
+        inside = np.flatnonzero((seg.spans[:, 0] >= t0) & (seg.spans[:, 0] < t1))
+        assert (k0, k1) == ((int(inside[0]), int(inside[-1]) + 1) if len(inside) else (k0, k0))
+        sg = sh.shard_gate(g)
+        assert sg.shape == (1, L, Hkv, m_cap, 2, r)
+        assert torch.equal(sg[:, :, :, :k1 - k0], g[:, :, :, k0:k1])
+        assert (sg[:, :, :, k1 - k0:] == 0).all()
+        seen += k1 - k0
+    assert seen == m
+
+
 def _rank_main(rank, world, port, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
@@ -167,6 +193,44 @@ def test_library_shards_merge_to_the_unsharded_decode(world):
     assert int(zm.ne(0).sum()) > 0
     # same entries, same factors (the bases of a span do not depend on the shard);
     # only the split-K / merge summation order differs
+    assert (O_m - O_f).abs().max().item() <= 2e-3
+    assert (lse_m - lse_f).abs().max().item() <= 2e-3
+
+
+@pytest.mark.gpu
+def test_learned_routing_shards_merge_to_the_unsharded_decode():
+    """learned-form routing and a rank gate, split over 2 shards"""
+    import hierarchical_kv_cache_span_b200 as P
+    CP = _cp()
+    wl = WORKLOADS["c2"].scaled(n=4000, L=2, Hq=8, Hkv=2)
+    H, K, V = T.make_inputs(wl)
+    ac, mc = T.caps(wl)
+    W = gen.route_projection(wl, 32).cuda()
+    gates = gen.rank_gates(wl, mc).cuda()
+    Hd, Kd, Vd = H.cuda(), K.cuda(), V.cuda()
+    full = P.SpanCache(1, wl.L, wl.Hq, wl.Hkv, wl.n, wl.d, wl.dtype, ac, mc, wl.rank)
+    full.set_routing(W)
+    full.build(Hd, Kd, Vd, wl.alpha, wl.window, wl.wmode, rank_gate=gates)
+    q = gen.queries(wl).cuda()
+    theta = torch.full((wl.L, wl.Hq), 2.0, dtype=torch.float32, device="cuda")
+    zm = full.new_zmask()
+    O_f, lse_f = full.decode(q, theta, zmask=zm)
+    parts_O, parts_l = [], []
+    for r in range(2):
+        sh = CP.ContextShard(wl.L, wl.Hq, wl.Hkv, wl.n, wl.d, wl.dtype, ac, mc, wl.rank, rank=r, world=2,
+                             route_W=W)
+        cuts = sh.plan(Hd, wl.alpha, wl.window)
+        t0, t1 = cuts[r], cuts[r + 1]
+        sh.build(Hd, Kd[:, :, :, t0:t1].contiguous(), Vd[:, :, :, t0:t1].contiguous(), wl.alpha, wl.window,
+                 wl.wmode, rank_gate=gates)
+        o, l = sh.decode(q, theta)
+        assert sh.cache.read_status() == 0
+        parts_O.append(o)
+        parts_l.append(l)
+    O_m, lse_m = CP.merge_parts(torch.stack(parts_O), torch.stack(parts_l))
+    torch.cuda.synchronize()
+    assert full.read_status() == 0
+    assert int(zm.ne(0).sum()) > 0
     assert (O_m - O_f).abs().max().item() <= 2e-3
     assert (lse_m - lse_f).abs().max().item() <= 2e-3
 
