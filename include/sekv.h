@@ -84,9 +84,12 @@ enum {
     SEKV_BUILD_ALL = 15
 };
 
-/* Decode phases. FUSED: routing + attention in one pass over a hot cache.
- * ROUTE: routing only (writes zmask / route_logits). ATTEND: routing again
- * (bit-identical) + attention, reading bases through the slot table. */
+/* Decode phases. FUSED: routing + attention over a hot cache (one pass for the
+ * identity routing form; with a budget or learned routing, a routing pass and then
+ * attention with its mask). ROUTE: routing only (writes zmask / route_logits).
+ * ATTEND: attention reading bases through the slot table; it routes again
+ * (bit-identical to ROUTE) in the identity form without a budget, and otherwise
+ * takes zmask, as ROUTE wrote it, as input. */
 enum { SEKV_FUSED = 0, SEKV_ROUTE = 1, SEKV_ATTEND = 2 };
 
 typedef void* sekv_stream_t;   /* a cudaStream_t (NULL = legacy default stream) */
