@@ -614,6 +614,10 @@ def run_sekv(args, rank, world, local_rank):
             out["fetch"]["resident_spans_per_step"] = statistics.mean(f["resident"] for f in fetched)
             out["fetch"]["copied_spans_per_step"] = statistics.mean(f["spans"] for f in fetched)
             out["config"]["fetch"] = "cached across steps"
+    try:
+        out["memory"] = memory_model(cache, cold)
+    except Exception as e:                            # context only; never fatal to the line
+        out["memory"] = {"error": f"{type(e).__name__}: {e}"}
     if cold:
         try:
             pk = h2d_peak(torch, dev)
@@ -630,6 +634,36 @@ def run_sekv(args, rank, world, local_rank):
         out["latency_form"] = latency_form(P, torch, cache, wl, q_buf, qpool[warm], theta, O, lse, zm, fetcher,
                                            cold, learned, bud, zoom_hint, steps)
     return out
+
+
+def memory_model(cache, cold: bool):
+    """SeKV blog §2.3 Eq. (17): GPU-resident bytes 2·L·H_kv·d·(a+w)·b (anchors, the
+    window included in a) + 2·L·H·d'·m·b (span summaries), from the realised anchor
+    and span counts, beside the buffers the cache actually holds on the device and
+    the full KV cache of the same context. The summaries here are kbar and vbar per
+    kv head (d' = d, H = H_kv) plus, with learned routing, the d'-wide routing
+    summaries per query head; bases count only when they live on the device."""
+    c = cache
+    s = 2 if c.dtype_name == "bf16" else 4
+    a = int(c.a_count.clamp(max=c.a_cap).sum())
+    m = int(c.m_count.clamp(max=c.m_cap).sum())
+    anchors = 2 * c.L * c.Hkv * c.d * a * s
+    summaries = 2 * c.L * c.Hkv * c.d * m * s
+    routing = c.L * c.Hq * c.dr * m * s if c.kbar_r is not None else 0
+    meta = c.L * c.Hkv * m * 4 + m * 4            # 1/||kbar|| and log|S|
+    bufs = [c.Ka, c.Va, c.kbar, c.vbar, c.inv_norm, c.logS, c.anchor_pos, c.span_beg, c.span_end, c.blk_off]
+    if c.kbar_r is not None:
+        bufs.append(c.kbar_r)
+    allocated = sum(t.numel() * t.element_size() for t in bufs)
+    home = c.home.numel() * c.home.element_size() if c.home is not None else 0
+    full_kv = 2 * c.B * c.L * c.Hkv * c.n * c.d * s
+    eq17 = anchors + summaries + routing + meta
+    return {"eq17_bytes": eq17, "anchors_bytes": anchors, "summaries_bytes": summaries + routing + meta,
+            "allocated_bytes": allocated + (0 if cold else home),
+            "bases_bytes": home, "bases_on": "pinned host" if cold else "device",
+            "full_kv_bytes": full_kv, "eq17_over_full_kv": eq17 / full_kv,
+            "note": "allocated = the cache's device buffers at their capacities (a_cap, m_cap)"
+                    + ("" if cold else " plus the device-resident bases")}
 
 
 def pct(xs, p):

@@ -67,3 +67,29 @@ def test_percentile_and_flags():
     a = bench.parse_args(["--latency-form", "--route-dim", "32", "--budget", "4"])
     assert a.latency_form and a.route_dim == 32 and a.budget == 4
     assert not bench.parse_args([]).latency_form and bench.parse_args([]).route_dim == 0
+
+
+def test_eq17_memory_model_arithmetic():
+    """Eq. (17) from realised counts on a fake cache: hand-computed byte counts"""
+    from types import SimpleNamespace
+    sys.path.insert(0, ROOT)
+    import bench
+    B, L, Hq, Hkv, n, d, a_cap, m_cap = 1, 2, 4, 2, 1000, 8, 64, 64
+    z = lambda *sh, dt=torch.bfloat16: torch.zeros(*sh, dtype=dt)
+    c = SimpleNamespace(B=B, L=L, Hq=Hq, Hkv=Hkv, n=n, d=d, a_cap=a_cap, m_cap=m_cap, dr=0, dtype_name="bf16",
+                        a_count=torch.tensor([40], dtype=torch.int32), m_count=torch.tensor([30], dtype=torch.int32),
+                        Ka=z(B, L, Hkv, a_cap, d), Va=z(B, L, Hkv, a_cap, d), kbar=z(B, L, Hkv, m_cap, d),
+                        vbar=z(B, L, Hkv, m_cap, d), inv_norm=z(B, L, Hkv, m_cap, dt=torch.float32),
+                        logS=z(B, m_cap, dt=torch.float32), anchor_pos=z(B, a_cap, dt=torch.int32),
+                        span_beg=z(B, m_cap, dt=torch.int32), span_end=z(B, m_cap, dt=torch.int32),
+                        blk_off=z(B, m_cap + 1, dt=torch.int64), kbar_r=None, home=z(B, L, 512))
+    r = bench.memory_model(c, cold=True)
+    assert r["anchors_bytes"] == 2 * 2 * 2 * 8 * 40 * 2
+    assert r["eq17_bytes"] == 2 * 2 * 2 * 8 * 40 * 2 + 2 * 2 * 2 * 8 * 30 * 2 + 2 * 2 * 30 * 4 + 30 * 4
+    assert r["full_kv_bytes"] == 2 * 2 * 2 * 1000 * 8 * 2
+    assert r["allocated_bytes"] == (2 * 2 * 2 * 64 * 8 * 2 + 2 * 2 * 2 * 64 * 8 * 2 + 2 * 2 * 64 * 4 + 64 * 4
+                                    + 64 * 4 * 3 + 65 * 8)
+    c.dr, c.kbar_r = 32, z(B, L, Hq, m_cap, 32)
+    r2 = bench.memory_model(c, cold=False)
+    assert r2["eq17_bytes"] - r["eq17_bytes"] == 2 * 4 * 32 * 30 * 2
+    assert r2["allocated_bytes"] - r["allocated_bytes"] == 2 * 4 * 64 * 32 * 2 + 2 * 512 * 2
