@@ -20,7 +20,7 @@ Sources (cited by page title and section):
   summary, Fig. 2, Eq. (6)-(8) truncated SVD; section 2.3 Eq. (5) routing gate,
   Eq. (9) zoom decision; section 3.1 hyperparameters.
 
-Readings fixed where the pages are silent (each is listed in the design doc):
+Readings fixed where the pages are silent:
 mu/sigma are the per-sequence mean and population std over all n positions,
 in fp64, with a strict ``>``; the last ``window`` positions are anchors too;
 anchors are not members of any span, and spans are the maximal runs of
