@@ -39,7 +39,10 @@ class SpanCache:
 
     Device: segmentation (counts, anchor positions, span bounds, log|S|, basis
     block offsets), anchors Ka/Va, summaries kbar/vbar + 1/||kbar||. Bases live
-    in ``home``: device memory (hot) or pinned host memory (cold).
+    in ``home``: device memory (hot) or pinned host memory (cold). With
+    ``set_routing(W)`` the summary step also writes per-query-head routing
+    summaries ``kbar_r`` and decode routes with them; ``build(..., rank_gate=g)``
+    folds a rank gate into the bases.
     """
 
     def __init__(self, B, L, Hq, Hkv, n, d, dtype, a_cap, m_cap, rank, home="device",
