@@ -780,7 +780,10 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{wl.name}: {wl.n // 1024}K ctx, {wl.L} layers, {wl.Hq}q/{wl.Hkv}kv, "
-                                   f"d={wl.d}, rank {wl.rank} (fp64 oracle)"},
+                                   f"d={wl.d}, rank {wl.rank} (fp64 oracle)",
+                       **({"budget": args.budget} if args.budget else {}),
+                       **({"routing": f"learned form, d'={args.route_dim} (seeded projection)"}
+                          if args.route_dim else {})},
             "cpu_baseline": {"value": v, "unit": "steps/s", "cores": workers, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
