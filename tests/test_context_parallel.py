@@ -67,6 +67,27 @@ def test_cuts_partition_without_splitting_spans(world):
         assert na == len(seg.anchor_pos) and ns == len(seg.spans)
 
 
+def test_cuts_edge_cases():
+    CP = _cp()
+    # more ranks than places to cut: some shards are empty, cuts stay monotone
+    cuts = CP.shard_cuts([0, 1, 50], [2, 51], 60, 8)
+    assert cuts[0] == 0 and cuts[-1] == 60 and all(a <= b for a, b in zip(cuts, cuts[1:]))
+    assert set(cuts[1:-1]) <= {0, 1, 2, 50, 51, 60}
+    for r in range(8):
+        a, sb, se = CP.shard_segmentation([0, 1, 50], [2, 51], [50, 60], cuts[r], cuts[r + 1])
+        assert (se <= cuts[r + 1] - cuts[r]).all()
+    # every token an anchor (no spans): cuts fall on anchors
+    cuts = CP.shard_cuts(list(range(10)), [], 10, 3)
+    assert cuts == [0, 3, 6, 10]
+    # one span and nothing else: a single cut point, the other shards empty
+    cuts = CP.shard_cuts([], [0], 100, 4)
+    assert cuts == [0, 100, 100, 100, 100]
+    a, sb, se = CP.shard_segmentation([], [0], [100], 0, 100)
+    assert len(a) == 0 and sb.tolist() == [0] and se.tolist() == [100]
+    with pytest.raises(ValueError):
+        CP.shard_segmentation([], [0], [100], 0, 50)      # a cut inside a span is refused
+
+
 def test_shard_gate_slices_the_global_span_range():
     CP = _cp()
     wl = WORKLOADS["c1"].scaled(n=2000, seed=3)
