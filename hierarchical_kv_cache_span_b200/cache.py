@@ -25,13 +25,13 @@ def _stream(stream) -> int:
 
 
 def tau_to_theta(tau: torch.Tensor) -> torch.Tensor:
-    """Eq. (9) threshold in logit space, theta = ln(tau / (1 - tau)) (fp64 on the
-    host, passed to the kernels as fp32; tau <= 0 -> -inf, tau >= 1 -> +inf)."""
-    t = tau.detach().to("cpu", torch.float64)
-    th = torch.log(t / (1.0 - t))
-    th = torch.where(t <= 0.0, torch.full_like(th, -math.inf), th)
-    th = torch.where(t >= 1.0, torch.full_like(th, math.inf), th)
-    return th.to(torch.float32)
+    """Zoom thresholds in logit space from tau (SeKV blog 2.3, Eq. (9)), computed by
+    the library's ``sekv_tau_to_theta``: marshals tau as host fp64 and returns the
+    host fp32 theta table of the same shape."""
+    t = tau.detach().to("cpu", torch.float64).contiguous()
+    th = torch.empty(t.shape, dtype=torch.float32)
+    S.check(S.sekv_tau_to_theta(t.data_ptr(), th.data_ptr(), t.numel()), "sekv_tau_to_theta")
+    return th
 
 
 class SpanCache:

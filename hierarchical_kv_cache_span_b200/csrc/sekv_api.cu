@@ -1,6 +1,7 @@
 // C ABI of the SeKV span-cache library: argument checks, workspace carving,
 // launches, and the host side of the cold-basis fetch.
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -250,6 +251,18 @@ sekv_status sekv_decode_attn_static(const sekv_decode_desc* d, sekv_stream_t str
     if (!scratch) return cuda_fail(e, "decode_static: address of the static scratch");
     e = sekv::launch_decode(*d, p, scratch, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "decode_static");
+    return SEKV_OK;
+}
+
+sekv_status sekv_tau_to_theta(const double* tau, float* theta, int64_t n) {
+    SEKV_REQUIRE(n >= 0 && (n == 0 || (tau && theta)), "tau_to_theta: n >= 0 and non-null tau, theta required");
+    for (int64_t i = 0; i < n; ++i)
+        SEKV_REQUIRE(!std::isnan(tau[i]), "tau_to_theta: tau[%lld] is NaN", (long long)i);
+    // sigma(l) > tau  <=>  l > ln(tau / (1 - tau)) for 0 < tau < 1 (SeKV blog 2.3, Eq. (9))
+    for (int64_t i = 0; i < n; ++i) {
+        const double t = tau[i];
+        theta[i] = t <= 0.0 ? -INFINITY : (t >= 1.0 ? INFINITY : (float)std::log(t / (1.0 - t)));
+    }
     return SEKV_OK;
 }
 

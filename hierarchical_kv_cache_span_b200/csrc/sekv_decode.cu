@@ -1812,19 +1812,43 @@ static __device__ __align__(256) unsigned char g_decode_scratch[SEKV_STATIC_SCRA
 size_t decode_static_scratch_bytes() { return SEKV_STATIC_SCRATCH_BYTES; }
 
 // Device address of g_decode_scratch on the current device. In host code the
-// array's name only stands in for it, so the address is looked up once per
-// device (with that device current) and cached.
+// array's name only stands in for it, so the address is looked up with the
+// device current and cached per device, together with the context it belongs
+// to: after a cudaDeviceReset the device gets a new primary context (and a new
+// copy of the array), which the cache notices and looks the address up again.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+static CtxGetCurrentFn ctx_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    }
+    return fn;
+}
+
 void* decode_static_scratch(cudaError_t* err) {
     static std::mutex mu;
     static void* addr[256] = {nullptr};
+    static CUcontext owner[256] = {nullptr};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 256) {
         *err = e != cudaSuccess ? e : cudaErrorInvalidDevice;
         return nullptr;
     }
+    CtxGetCurrentFn cur = ctx_current_fn();
+    auto current = [&]() -> CUcontext {
+        CUcontext c = nullptr;
+        return (cur && cur(&c) == CUDA_SUCCESS) ? c : nullptr;
+    };
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    const CUcontext ctx = current();
+    if (!addr[dev] || !ctx || owner[dev] != ctx) {
+        // the lookup binds the device's context if the thread has none yet
         void* ptr = nullptr;
         e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
         if (e != cudaSuccess || !ptr) {
@@ -1832,6 +1856,7 @@ void* decode_static_scratch(cudaError_t* err) {
             return nullptr;
         }
         addr[dev] = ptr;
+        owner[dev] = current();
     }
     *err = cudaSuccess;
     return addr[dev];

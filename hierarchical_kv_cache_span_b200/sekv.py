@@ -88,6 +88,7 @@ _SIGS = {
     "sekv_decode_attn_static": (_i32, [C.POINTER(sekv_decode_desc), _p]),
     "sekv_fetch_bases": (_i32, [C.POINTER(sekv_fetch_desc), _p, _p, _p]),
     "sekv_merge_partials": (_i32, [_p, _p, _i32, _i64, _i32, _p, _p, _p]),
+    "sekv_tau_to_theta": (_i32, [_p, _p, _i64]),
     "sekv_status_str": (C.c_char_p, [_i32]),
     "sekv_last_error": (C.c_char_p, []),
     "sekv_desc_size": (C.c_size_t, [_i32]),
@@ -166,6 +167,10 @@ def sekv_merge_partials(O_parts: int, lse_parts: int, nparts: int, rows: int, d:
 def sekv_fetch_bases(desc: sekv_fetch_desc, compute: int, copy: int, done: int) -> int:
     return int(_lib.sekv_fetch_bases(C.byref(desc), C.c_void_p(compute or None),
                                      C.c_void_p(copy or None), C.c_void_p(done or None)))
+
+
+def sekv_tau_to_theta(tau: int, theta: int, n: int) -> int:
+    return int(_lib.sekv_tau_to_theta(C.c_void_p(tau), C.c_void_p(theta), n))
 
 
 def sekv_status_str(status: int) -> str:

@@ -263,8 +263,10 @@ sekv_status sekv_decode_attn(const sekv_decode_desc* desc, sekv_stream_t stream)
  *     rejected with SEKV_ERR_CAPACITY and launches nothing.
  *   - No cudaMalloc, cudaFree or allocating library routine is called. The first
  *     call on a device looks up the array's device address (cudaGetSymbolAddress,
- *     with that device current) and caches it: make that first call before any
- *     stream capture.
+ *     with that device current) and caches it with the device's current context:
+ *     make that first call before any stream capture. A call made under another
+ *     context of the device (for example after cudaDeviceReset) looks the address
+ *     up again, so it too should come before any capture.
  *   - Every call uses the same array, which keeps the last call's contents; each
  *     call writes all the scratch it reads, so nothing has to start at zero.
  *     Calls whose kernels can overlap on the GPU (different streams without an
@@ -332,6 +334,19 @@ typedef struct sekv_fetch_desc {
  * SEKV_ERR_CAPACITY (nothing copied) if the zoomed bases exceed arena_elems. */
 sekv_status sekv_fetch_bases(const sekv_fetch_desc* desc, sekv_stream_t compute,
                              sekv_stream_t copy, sekv_event_t done);
+
+/* ------------------------------------------------------------------------- */
+/* Zoom thresholds (SeKV blog 2.3, Eq. (9))                                   */
+/* ------------------------------------------------------------------------- */
+/* Eq. (9) zooms span S for a head when sigma(l_S) > tau^(l,h). The decode compares
+ * in logit space instead, l_S > theta with theta = ln(tau / (1 - tau)), which is
+ * the same decision without the sigmoid's saturation. This fills theta (host,
+ * n floats, e.g. the [L][Hq] table that sekv_decode_desc.theta points at once it
+ * is copied to the device) from tau (host, n doubles): computed in double,
+ * rounded to float; tau <= 0 gives -inf (every span zooms) and tau >= 1 gives
+ * +inf (none does). A NaN tau, a null pointer with n > 0, or n < 0 returns
+ * SEKV_ERR_INVALID_ARG before anything is written. Synchronous, no GPU work. */
+sekv_status sekv_tau_to_theta(const double* tau, float* theta, int64_t n);
 
 /* ------------------------------------------------------------------------- */
 const char* sekv_status_str(int32_t status);

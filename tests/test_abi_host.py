@@ -122,3 +122,27 @@ def test_product_path_has_no_oracle_or_cpu_fallback():
             src = open(os.path.join(pkg, fn)).read()
             assert "oracle" not in src.replace("no oracle", ""), fn
             assert "import numpy" not in src, fn
+
+
+def test_tau_to_theta_through_the_abi_matches_the_oracle():
+    """sekv_tau_to_theta (SeKV blog 2.3, Eq. (9) in logit space) against the oracle's
+    fp64 conversion rounded to fp32, including tau <= 0, tau >= 1 and interior values."""
+    import torch
+    import oracle as O
+    from hierarchical_kv_cache_span_b200 import cache, sekv as S
+    rng = np.random.default_rng(5)
+    tau = np.r_[0.0, -0.3, 1.0, 1.7, 0.5, 1e-12, 1 - 1e-12, rng.uniform(0.3, 0.9, 61)]
+    th = cache.tau_to_theta(torch.tensor(tau, dtype=torch.float64)).numpy()
+    assert th.dtype == np.float32
+    np.testing.assert_array_equal(th, O.tau_to_theta(tau).astype(np.float32))
+    assert th[0] == -np.inf and th[1] == -np.inf and th[2] == np.inf and th[3] == np.inf and th[4] == 0.0
+    # the shape of the table is kept ([L][Hq])
+    t2 = torch.full((3, 4), 0.75, dtype=torch.float64)
+    assert tuple(cache.tau_to_theta(t2).shape) == (3, 4)
+    # NaN or null pointers: rejected before anything is written
+    out = np.full(2, 7.0, np.float32)
+    bad = np.array([0.5, np.nan])
+    assert S.sekv_tau_to_theta(bad.ctypes.data, out.ctypes.data, 2) == S.SEKV_ERR_INVALID_ARG
+    assert (out == 7.0).all()
+    assert S.sekv_tau_to_theta(0, 0, 3) == S.SEKV_ERR_INVALID_ARG
+    assert S.sekv_tau_to_theta(0, 0, 0) == S.SEKV_OK

@@ -626,3 +626,110 @@ def test_planted_reversed_rank_gate_is_caught(monkeypatch):
         _pin_rank_gate_known_components(12, 20)
     monkeypatch.undo()
     _pin_rank_gate_known_components(12, 20)
+
+
+# ---------------------------------------------------------------------------
+# Per-head routing summaries of a key head's spans (SeKV blog 2.2 Eq. (2), (3)):
+# each query head uses its own W, each span its own weights
+# ---------------------------------------------------------------------------
+def _pin_routing_summaries():
+    g = _gold("routing_summaries_example.json")
+    seg = O.segment(g["H"], 1.0, 0)
+    assert seg.spans.tolist() == g["spans"] and seg.anchor_pos.tolist() == g["anchors"]
+    out = O.routing_summaries(g["K"], g["H"], seg, "surprisal", g["W"], "f64")
+    assert out.shape == (2, 2, 3)
+    for h in range(2):
+        for s in range(2):
+            expect = np.array(g["direction"][h][s]) / math.sqrt(g["norm_sq"][h][s])
+            np.testing.assert_allclose(out[h, s], expect, rtol=0, atol=1e-15)
+
+
+def test_routing_summaries_hand_example():
+    _pin_routing_summaries()
+
+
+def test_planted_routing_summaries_mistakes_are_caught(monkeypatch):
+    """A swapped head index, or a span read one token too far (into the anchor that
+    follows it), planted in the oracle, fails the hand pin."""
+    real = O.routing_summaries
+
+    def swapped_heads(K, H, seg, wmode, W_heads, dtype):
+        return real(K, H, seg, wmode, np.asarray(W_heads)[::-1], dtype)
+
+    def span_plus_one(K, H, seg, wmode, W_heads, dtype):
+        W_heads = np.asarray(W_heads, dtype=np.float64)
+        out = np.zeros((W_heads.shape[0], len(seg.spans), W_heads.shape[1]))
+        for i, (b, e) in enumerate(seg.spans):
+            w = O.span_weights(np.asarray(H, float)[b:e + 1], wmode)
+            for h in range(W_heads.shape[0]):
+                out[h, i] = O.routing_summary(np.asarray(K, float)[b:e + 1], w, W_heads[h])
+        return out
+
+    for bad in (swapped_heads, span_plus_one):
+        monkeypatch.setattr(O, "routing_summaries", bad)
+        with pytest.raises(AssertionError):
+            _pin_routing_summaries()
+        monkeypatch.undo()
+    _pin_routing_summaries()
+
+
+# ---------------------------------------------------------------------------
+# Rank gates routed per span and per side (SeKV blog 2.2 Eq. (6)): gates[S][0]
+# scales the key truncation of span S, gates[S][1] its value truncation
+# ---------------------------------------------------------------------------
+def _known_matrix(rng, ns, d, top):
+    k = min(ns, d)
+    U, V = _orth(rng, ns, k), _orth(rng, d, k)
+    s = np.linspace(top, 1.0, k)
+    return U, s, V, (U * s) @ V.T
+
+
+def _pin_span_bases_gates():
+    rng = np.random.default_rng(41)
+    d, r = 10, 4
+    lens = (6, 14)                         # one span shorter than d, one longer
+    spans = [(0, lens[0]), (lens[0] + 1, lens[0] + 1 + lens[1])]
+    n = spans[1][1]
+    K = rng.normal(size=(n, d))            # the anchor row between the spans is noise
+    V = rng.normal(size=(n, d))
+    known = []
+    for (b, e), top in zip(spans, (9.0, 7.0)):
+        kk = _known_matrix(rng, e - b, d, top)
+        vv = _known_matrix(rng, e - b, d, top + 3.0)
+        K[b:e], V[b:e] = kk[3], vv[3]
+        known.append((kk, vv))
+    anchor = np.zeros(n, bool)
+    anchor[lens[0]] = True
+    seg = O.Segmentation(0.0, 0.0, 0.0, anchor, np.array([lens[0]]), np.array(spans))
+    gates = np.array([[[1.0, 0.0, 0.5, 0.25], [0.75, 1.0, 0.0, 0.5]],
+                      [[0.0, 0.5, 1.0, 1.0], [1.0, 0.25, 0.75, 0.0]]])
+    out = O.span_bases(K, V, seg, r, "f64", gates)
+    for i, ((Uk, sk, Vk, _), (Uv, sv, Vv, _)) in enumerate(known):
+        A, B, C, D = out[i]
+        # sum_j m_j sigma_j u_j v_j^T over the top r components, written from the construction
+        np.testing.assert_allclose(A @ B, (Uk[:, :r] * (gates[i, 0] * sk[:r])) @ Vk[:, :r].T, rtol=0, atol=1e-10)
+        np.testing.assert_allclose(C @ D, (Uv[:, :r] * (gates[i, 1] * sv[:r])) @ Vv[:, :r].T, rtol=0, atol=1e-10)
+
+
+def test_span_bases_route_key_and_value_gates():
+    _pin_span_bases_gates()
+
+
+def test_planted_span_bases_gate_mistakes_are_caught(monkeypatch):
+    """Key and value gates swapped, or the first span's gates used for every span,
+    planted in the oracle, fail the pin."""
+    real = O.span_bases
+
+    def swapped_sides(K, V, seg, r, dtype, gates=None):
+        return real(K, V, seg, r, dtype, None if gates is None else np.asarray(gates)[:, ::-1])
+
+    def first_span_only(K, V, seg, r, dtype, gates=None):
+        g = None if gates is None else np.repeat(np.asarray(gates)[:1], len(seg.spans), axis=0)
+        return real(K, V, seg, r, dtype, g)
+
+    for bad in (swapped_sides, first_span_only):
+        monkeypatch.setattr(O, "span_bases", bad)
+        with pytest.raises(AssertionError):
+            _pin_span_bases_gates()
+        monkeypatch.undo()
+    _pin_span_bases_gates()

@@ -3,24 +3,20 @@ allocate device memory on the decode path (a serving loop inside a memory pool i
 does not own, a plugin whose host framework forbids allocations after start-up,
 code that must not call cudaMalloc because it can synchronize the device).
 
-It must give the same result as sekv_decode_attn with a caller workspace, on
-every call: the static scratch array keeps the previous call's contents, so the
-check runs two calls in a row. This file is collected last so that a failure here
-stops a `-x` run only after every other test has run; it also passes on its own
-in a fresh process.
+It must give the same result as sekv_decode_attn with a caller workspace, bit for
+bit, on every call: the static scratch array keeps the previous call's contents,
+so the check runs calls in a row with different inputs. This file is collected
+last so that a failure here stops a `-x` run only after every other test has run;
+it also passes on its own in a fresh process.
 """
-import ctypes
 import math
 
-import numpy as np
 import pytest
 import torch
 
 from sekv_synth import WORKLOADS, gen
 
 pytestmark = pytest.mark.gpu
-
-TOL = 2e-2          # the bf16 tolerance the parity tests use
 
 
 def _lib():
@@ -41,33 +37,71 @@ def _built_cache(wl):
     return c
 
 
-def test_static_scratch_decode_matches_workspace_decode():
+def _static_call(c, q, theta, zm, budget=0):
     P = _lib()
     S = P.sekv
+    O, lse = c.new_outputs()
+    O.fill_(float("nan"))
+    lse.fill_(float("nan"))
+    d = c.decode_desc(q, theta, O=O, lse=lse, zmask=zm, budget=budget)
+    d.workspace, d.workspace_bytes = None, 0          # the static entry point needs none
+    S.check(S.sekv_decode_attn_static(d, torch.cuda.current_stream().cuda_stream), "sekv_decode_attn_static")
+    return O, lse
+
+
+def _workspace_call(c, q, theta, zm, budget=0):
+    return c.decode(q, theta, zmask=zm, budget=budget)
+
+
+def _draws(wl):
+    """two (query, threshold) pairs with different zoom sets: the first zooms a
+    good share of the spans, the second almost none, so the two calls write
+    different split-K partials into the same static array"""
+    q1 = gen.queries(wl).cuda()
+    g = torch.Generator().manual_seed(gen.unit_seed(wl.seed, 7, 0, 0, 1))
+    q2 = torch.randn(q1.shape, generator=g).to(q1.dtype).cuda()
+    th1 = torch.full((wl.L, wl.Hq), 3.5, dtype=torch.float32, device="cuda")
+    th2 = torch.full((wl.L, wl.Hq), 5.5, dtype=torch.float32, device="cuda")
+    return (q1, th1), (q2, th2)
+
+
+@pytest.mark.parametrize("budget", [0, 3])
+def test_static_scratch_decode_matches_workspace_decode(budget):
+    """Two static calls in a row with different inputs; each must equal the
+    workspace decode of the same inputs bit for bit (same kernels, same split plan),
+    so partials left in the static array by the earlier call cannot leak into a
+    later result. With a budget and no route_logits buffer, the routing logits of
+    the cap live in the static array too."""
     wl = WORKLOADS["c2"].scaled(n=4096, L=2)
     c = _built_cache(wl)
-    q = gen.queries(wl).cuda()
-    # thresholds low enough that a good share of spans zoom (the zoom path runs too)
-    theta = torch.full((wl.L, wl.Hq), 3.5, dtype=torch.float32, device="cuda")
-    zm_ref = c.new_zmask()
-    O_ref, lse_ref = c.decode(q, theta, zmask=zm_ref)
-    torch.cuda.synchronize()
-    assert c.read_status() == 0
-    assert int(zm_ref.ne(0).sum()) > 0
-    stream = torch.cuda.current_stream().cuda_stream
-    for call in range(2):
-        O = torch.full_like(O_ref, float("nan"))
-        lse = torch.full_like(lse_ref, float("nan"))
+    draws = _draws(wl)
+    refs = []
+    for q, th in draws:
         zm = c.new_zmask()
-        d = c.decode_desc(q, theta, O=O, lse=lse, zmask=zm)
-        d.workspace, d.workspace_bytes = None, 0          # the static entry point needs none
-        S.check(S.sekv_decode_attn_static(d, stream), "sekv_decode_attn_static")
+        O, lse = _workspace_call(c, q, th, zm, budget)
         torch.cuda.synchronize()
         assert c.read_status() == 0
-        assert torch.equal(zm, zm_ref)
-        assert torch.isfinite(O).all() and torch.isfinite(lse).all()
-        assert (O - O_ref).abs().max().item() <= TOL
-        assert (lse - lse_ref).abs().max().item() <= TOL
+        refs.append((O, lse, zm))
+    assert int(refs[0][2].ne(0).sum()) > int(refs[1][2].ne(0).sum())
+    assert int(refs[0][2].ne(0).sum()) > 0
+    if budget:
+        assert not torch.equal(refs[0][2], _no_cap_mask(c, *draws[0]))   # the cap actually bites
+    for rep in range(2):
+        for (q, th), (O_ref, lse_ref, zm_ref) in zip(draws, refs):
+            zm = c.new_zmask()
+            O, lse = _static_call(c, q, th, zm, budget)
+            torch.cuda.synchronize()
+            assert c.read_status() == 0
+            assert torch.equal(zm, zm_ref)
+            assert torch.equal(O, O_ref), (O - O_ref).abs().max().item()
+            assert torch.equal(lse, lse_ref), (lse - lse_ref).abs().max().item()
+
+
+def _no_cap_mask(c, q, th):
+    zm = c.new_zmask()
+    c.decode(q, th, zmask=zm)
+    torch.cuda.synchronize()
+    return zm
 
 
 def test_static_scratch_rejects_oversized_calls():
