@@ -97,6 +97,18 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (earlier measurement on this pool)"
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms during a region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -211,6 +223,36 @@ def attend_bytes(cache, zmask_host, P):
         total += base * c.L * c.Hkv + int((bits * blk[None, None, :]).sum())
         zoom_units += int(bits.sum())
     return total, zoom_units
+
+
+FP32_LANES_PER_SM = 128      # B200: 4 SM sub-partitions x 32 fp32 FMA lanes
+
+
+def basis_work(cache, layers, P):
+    """Operation counts of the basis build (BASES step) from the realised span
+    lengths, per the algorithm the kernel runs (one problem per span, kv head, layer
+    and side K / V; X is |S| x d, N = min(|S|, d), rS = min(r, |S|, d)):
+    Gram 2 N^2 max(|S|, d) (tensor cores); Householder tridiagonalisation 4/3 N^3;
+    back-transformation of rS vectors 2 rS N^2; factors 2 rS |S| d (fp32). The
+    eigenvalue / eigenvector steps on the tridiagonal are O(rS N) and left out.
+    Also the bytes the step must move: K, V read once, factors written."""
+    import numpy as np
+    c = cache
+    s = 2 if c.dtype_name == "bf16" else 4
+    ln = (c.span_end - c.span_beg).cpu().numpy().astype(np.float64)
+    m = c.m_count.cpu().numpy()
+    gram = f32 = 0.0
+    wbytes = 0
+    for b in range(c.B):
+        L_ = ln[b, :int(m[b])]
+        N = np.minimum(L_, c.d)
+        rS = np.minimum(np.minimum(L_, c.d), c.rank)
+        gram += float(np.sum(2 * N ** 2 * np.maximum(L_, c.d)))
+        f32 += float(np.sum(4.0 / 3.0 * N ** 3 + 2 * rS * N ** 2 + 2 * rS * L_ * c.d))
+        wbytes += int(sum(c.Hkv * P.sekv.sekv_block_elems(int(x), c.d, c.rank) for x in L_)) * s
+    per = 2 * layers * c.Hkv                 # K and V, every layer and kv head
+    return {"tensor_flops": gram * per, "fp32_flops": f32 * per,
+            "bytes": int(2 * c.B * layers * c.Hkv * c.n * c.d * s + wbytes * layers)}
 
 
 def route_bytes(cache, learned):
@@ -384,6 +426,21 @@ def run_sekv(args, rank, world, local_rank):
         "not_converged_warning": st == P.sekv.SEKV_WARN_NOT_CONVERGED,
     }
     build["total_ms"] = build["segment_ms"] + build["summary_ms"] + build["bases_ms"]
+    try:
+        bw = basis_work(cache, wl.L, P)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        sec = build["bases_ms"] * 1e-3
+        build["bases_work"] = {
+            "fp32_tflop": bw["fp32_flops"] / 1e12, "tensor_tflop": bw["tensor_flops"] / 1e12,
+            "fp32_TFLOPs": bw["fp32_flops"] / sec / 1e12, "tensor_TFLOPs": bw["tensor_flops"] / sec / 1e12,
+            "GBps": bw["bytes"] / sec / 1e9,
+            "fp32_peak_TFLOPs": sms * FP32_LANES_PER_SM * 2 * 1.965e9 / 1e12,
+            "note": "counts from the realised span lengths (Gram on tensor cores; tridiagonalisation, "
+                    "back-transformation and factors in fp32); fp32 peak = SMs x 128 lanes x 2 x 1965 MHz "
+                    "(nominal, from unit counts and the maximum clock)"}
+        build["bases_work"]["fp32_frac"] = build["bases_work"]["fp32_TFLOPs"] / build["bases_work"]["fp32_peak_TFLOPs"]
+    except Exception as e:                            # context only; never fatal to the line
+        build["bases_work"] = {"error": f"{type(e).__name__}: {e}"}
 
     # sample units for the CPU oracle before K/V are freed
     cpu_units = {}
@@ -438,8 +495,7 @@ def run_sekv(args, rank, world, local_rank):
     if cold:
         d_route = cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud)
         d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_ATTEND, O=O, lse=lse, slot=fetcher.slot_dev,
-                                   arena=fetcher.arena, zmask=zm if (bud or learned) else None, budget=bud,
-                                   zoom_hint=zoom_hint)
+                                   arena=fetcher.arena, zmask=zm, budget=bud, zoom_hint=zoom_hint)
     else:
         d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_FUSED, O=O, lse=lse, zmask=zm, budget=bud,
                                    zoom_hint=zoom_hint)
@@ -550,6 +606,7 @@ def run_sekv(args, rank, world, local_rank):
         units_total = wl.B * wl.L * wl.Hkv
         oracle_step_s = per_unit * units_total / workers
         cpu = {"value": 1.0 / oracle_step_s, "unit": "steps/s", "cores": workers, "kind": "oracle",
+               "cpu_model": cpu_model(),
                "sample": f"{workers} (layer, kv-head) units of one decode step, one unit per process "
                          f"(spawn pool, 1 BLAS thread each); per-unit decode time x {units_total} units / "
                          f"{workers} cores. Oracle build of those units: mean {statistics.mean(t_build):.2f} s/unit",
@@ -705,8 +762,7 @@ def latency_form(P, torch, cache, wl, q_buf, q, theta, O, lse, zm, fetcher, cold
         for l in range(wl.L):
             if cold:
                 descs.append(cache.decode_desc(q_buf, theta, phase=P.SEKV_ATTEND, O=O, lse=lse,
-                                               slot=fetcher.slot_dev, arena=fetcher.arena,
-                                               zmask=zm if (bud or learned) else None, budget=bud,
+                                               slot=fetcher.slot_dev, arena=fetcher.arena, zmask=zm, budget=bud,
                                                zoom_hint=zoom_hint, l0=l, l1=l + 1))
             else:
                 descs.append(cache.decode_desc(q_buf, theta, phase=P.SEKV_FUSED, O=O, lse=lse, zmask=zm,
@@ -746,7 +802,12 @@ def latency_form(P, torch, cache, wl, q_buf, q, theta, O, lse, zm, fetcher, cold
 
 
 def run_reference(args):
-    """The fp64 oracle as the reference arm: same workload recipe, bounded sample."""
+    """The fp64 oracle as the reference arm, on the host cores. Each step is a
+    bounded sample of the workload's decode step: one (layer, kv head) unit per
+    worker process, decoded once per step (W warm-up steps, then K timed steps).
+    `ms_per_step` and `steps` describe that sample as it ran; `value` scales the
+    sample to the whole step (units_total / units per sample), which the
+    `extrapolation` field states."""
     import numpy as np
     import torch
     from sekv_synth import gen
@@ -766,25 +827,33 @@ def run_reference(args):
     import oracle as O
     taus = gen.taus(wl)
     theta = O.tau_to_theta(taus.numpy()) if taus is not None else None
-    reps = min(5, max(1, args.steps))
     W = gen.route_projection(wl, args.route_dim).double().numpy() if args.route_dim else None
-    t_build, t_dec = oracle_sample(wl, H0, units, q, theta, reps=reps, workers=workers,
+    steps, warm = max(1, args.steps), max(0, args.warmup)
+    t_build, t_dec = oracle_sample(wl, H0, units, q, theta, reps=warm + steps, workers=workers,
                                    quantile=wl.tau_a, budget=args.budget, W=W)
-    per_unit = [min(t) for t in t_dec]
+    # a sampled step runs the workers' units side by side: its time is the slowest unit's
+    sample_ms = [1e3 * max(t[warm + i] for t in t_dec) for i in range(steps)]
+    ms = statistics.mean(sample_ms)
     units_total = wl.B * wl.L * wl.Hkv
-    step_s = statistics.mean(per_unit) * units_total / workers
-    v = 1.0 / step_s
-    sample = (f"{workers} (layer, kv-head) units of one decode step on {workers} host cores (spawn pool), "
-              f"scaled to {units_total} units")
+    scale_up = units_total / workers
+    v = 1.0 / (ms * 1e-3 * scale_up)
+    sample = (f"{workers} (layer, kv-head) units of one decode step per timed step, one unit per process on "
+              f"{workers} host cores (spawn pool, 1 BLAS thread each); oracle build of the units outside the "
+              f"timed steps (mean {statistics.mean(t_build):.2f} s per unit)")
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "steps": steps, "warmup": warm, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{wl.name}: {wl.n // 1024}K ctx, {wl.L} layers, {wl.Hq}q/{wl.Hkv}kv, "
                                    f"d={wl.d}, rank {wl.rank} (fp64 oracle)",
                        **({"budget": args.budget} if args.budget else {}),
                        **({"routing": f"learned form, d'={args.route_dim} (seeded projection)"}
                           if args.route_dim else {})},
-            "cpu_baseline": {"value": v, "unit": "steps/s", "cores": workers, "kind": "oracle", "sample": sample},
+            "extrapolation": {"units_per_timed_step": workers, "units_per_full_step": units_total,
+                              "full_step_ms": ms * scale_up,
+                              "note": "ms_per_step and steps are the sampled steps that ran; value = 1 / "
+                                      "full_step_ms, the sample scaled to every (layer, kv head) unit"},
+            "cpu_baseline": {"value": v, "unit": "steps/s", "cores": workers, "kind": "oracle", "sample": sample,
+                             "cpu_model": cpu_model()},
             "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 

@@ -166,13 +166,22 @@ def merge_parts(O_parts: torch.Tensor, lse_parts: torch.Tensor, stream=None) -> 
 
 
 def context_parallel_decode(shard: ContextShard, q: torch.Tensor, theta: torch.Tensor, group=None, **kw):
-    """Every rank decodes its shard, the parts are all-gathered (NCCL on GPUs) and
-    merged; every rank returns the full (O, lse)."""
+    """Every rank decodes its shard, the parts are all-gathered and merged on the
+    device; every rank returns the full (O, lse). With NCCL the gather runs on the
+    device tensors; a host-side group (gloo) gathers host copies of them."""
     import torch.distributed as dist
     O_r, lse_r = shard.decode(q, theta, **kw)
     world = dist.get_world_size(group)
-    O_all = torch.empty((world,) + tuple(O_r.shape), dtype=O_r.dtype, device=O_r.device)
-    lse_all = torch.empty((world,) + tuple(lse_r.shape), dtype=lse_r.dtype, device=lse_r.device)
-    dist.all_gather_into_tensor(O_all, O_r.contiguous(), group=group)
-    dist.all_gather_into_tensor(lse_all, lse_r.contiguous(), group=group)
-    return merge_parts(O_all, lse_all)
+    on_host = dist.get_backend(group) == "gloo"
+    dev = O_r.device
+    src_O = O_r.contiguous().cpu() if on_host else O_r.contiguous()
+    src_l = lse_r.contiguous().cpu() if on_host else lse_r.contiguous()
+    O_all = torch.empty((world,) + tuple(O_r.shape), dtype=O_r.dtype, device=src_O.device)
+    lse_all = torch.empty((world,) + tuple(lse_r.shape), dtype=lse_r.dtype, device=src_l.device)
+    if on_host:
+        dist.all_gather(list(O_all.unbind(0)), src_O, group=group)
+        dist.all_gather(list(lse_all.unbind(0)), src_l, group=group)
+    else:
+        dist.all_gather_into_tensor(O_all, src_O, group=group)
+        dist.all_gather_into_tensor(lse_all, src_l, group=group)
+    return merge_parts(O_all.to(dev), lse_all.to(dev))

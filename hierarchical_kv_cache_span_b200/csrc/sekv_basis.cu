@@ -10,14 +10,29 @@
 //   |S| <= d: G = X X^T (N x N), top-rS eigenvectors U_r, A = U_r, B = U_r^T X
 //   |S| >  d: G = X^T X (N x N), top-rS eigenvectors V_r, A = X V_r, B = V_r^T
 // so A B is the projection of X on its top-rS singular subspace (Eckart-Young).
-// The symmetric eigenproblem is solved by the parallel cyclic Jacobi method
-// (round-robin pairing, N/2 disjoint rotations per round) in shared memory, fp32.
+//
+// Only the top rS of the N eigenpairs are needed, so the symmetric eigenproblem is
+// solved the way a selected-eigenvector solver does it rather than by a full
+// diagonalisation (whose cost is ~N^3 per sweep over many sweeps):
+//   1. Householder tridiagonalisation G = Q T Q^T in shared memory (N - 2
+//      reflectors; each step is a symmetric matrix-vector product and a rank-2
+//      update of the trailing block);
+//   2. the rS largest eigenvalues of T by multisection on Sturm counts (several
+//      threads probe one eigenvalue's bracket at once);
+//   3. their eigenvectors by inverse iteration on T - lambda I (one thread per
+//      eigenvalue, pseudo-random start vectors), then modified Gram-Schmidt twice in
+//      descending eigenvalue order, so that vectors of clustered eigenvalues come
+//      out orthonormal and span their cluster;
+//   4. back-transformation by the reflectors (u = Q z), one warp per vector.
+// T is scaled to unit norm before steps 2-3 (eigenvectors do not change).
 // The Gram contraction runs on the tensor cores (mma.sync m16n8k16 bf16 -> fp32)
 // for bf16 inputs and on the FMA pipes for fp32 inputs.
 //
 // Problems are bucketed by N (<= 32, <= 64, <= 128) so each bucket gets a
 // shared-memory footprint and CTA size that fit it; each bucket is a persistent
 // launch that pulls work items from an atomic counter.
+#include <cfloat>
+
 #include "sekv_common.cuh"
 #include "sekv_internal.h"
 
@@ -25,6 +40,7 @@ namespace sekv {
 
 constexpr int kBuckets = 3;
 constexpr int kChunkRows = 32;    // rows of X staged per step when |S| > d
+constexpr int kInvIters = 3;      // inverse-iteration steps per eigenvector
 
 struct BasisWork {
     int* bucket_count;   // [kBuckets]
@@ -71,7 +87,7 @@ struct BasisArgs {
     int32_t* status;
     const float* gate;   // null or [B][L][Hkv][m_cap][2][rank] rank gate m_{S,i} (Eq. (6))
     int64_t region;
-    int L, l0, Lr, Hkv, n, d, m_cap, rank, max_sweeps;
+    int L, l0, Lr, Hkv, n, d, m_cap, rank;
 };
 
 // ---------------------------------------------------------------------------
@@ -145,118 +161,370 @@ SEKV_DEV void gram_cols_mma(float* G, int ldg, const __nv_bfloat16* Xb, int ldb,
 }
 
 // ---------------------------------------------------------------------------
-// parallel cyclic Jacobi on the symmetric Ne x Ne matrix G (Ne even); Vm <- eigenvectors
-// returns true when ||off||_F^2 <= tol2 * ||diag||_F^2
+// Householder tridiagonalisation of the symmetric N x N matrix in G (row stride
+// ld, full storage). Afterwards dg[0..N-1] holds the diagonal of T, eo[0..N-2] its
+// off-diagonal, and reflector k (k = 0 .. N-3), H_k = I - tk[k] v v^T acting on
+// coordinates k+1 .. N-1, is stored with v in row k of G at columns k+1 .. N-1
+// (v[k+1] = 1), so that G = Q T Q^T with Q = H_0 H_1 ... H_{N-3}.
+// Scratch: pv[ld] (the vector p), red[>= 64].
 // ---------------------------------------------------------------------------
-SEKV_DEV bool jacobi(float* G, float* Vm, int ld, int Ne, int max_sweeps, int* rp, int* rq, float* rc,
-                     float* rs, float* red, float tol2) {
-    const int tid = threadIdx.x, T = blockDim.x;
-    const int half = Ne >> 1;
-    for (int i = tid; i < Ne * Ne; i += T) Vm[(i / Ne) * ld + (i % Ne)] = (i / Ne == i % Ne) ? 1.f : 0.f;
-    bool converged = false;
-    for (int sweep = 0; sweep <= max_sweeps; ++sweep) {
-        // convergence test
-        float off = 0.f, dia = 0.f;
-        for (int i = tid; i < Ne * Ne; i += T) {
-            const int r = i / Ne, c = i % Ne;
-            const float g = G[r * ld + c];
-            if (r == c) dia = fmaf(g, g, dia); else off = fmaf(g, g, off);
+SEKV_DEV void tridiagonalize(float* G, int ld, int N, float* dg, float* eo, float* tk, float* pv, float* red) {
+    const int tid = threadIdx.x, T = blockDim.x, lane = tid & 31, wid = tid >> 5;
+    // column c, partition part: the symmetric product splits each column's sum over R parts
+    const int R = T / ld >= 1 ? T / ld : 1;
+    float* part = red + 64;      // [R][ld] partial column sums (caller sized)
+    for (int k = 0; k + 2 < N; ++k) {
+        const int m = N - k - 1;              // trailing block: coordinates k+1 .. N-1
+        float* row = G + (size_t)k * ld;
+        // (a) reflector of x = row k, columns k+1 .. N-1 (warp 0)
+        if (wid == 0) {
+            float s = 0.f;
+            for (int i = k + 2 + lane; i < N; i += 32) s = fmaf(row[i], row[i], s);
+            s = warp_sum(s);
+            const float alpha = row[k + 1];
+            float tau = 0.f, beta = alpha, scl = 0.f;
+            if (s > 0.f) {
+                const float nrm = sqrtf(fmaf(alpha, alpha, s));
+                beta = alpha >= 0.f ? -nrm : nrm;
+                tau = (beta - alpha) / beta;
+                scl = 1.f / (alpha - beta);
+            }
+            for (int i = k + 2 + lane; i < N; i += 32) row[i] *= scl;   // tau = 0: v = e1, tail unused
+            if (lane == 0) {
+                row[k + 1] = 1.f;
+                dg[k] = row[k];
+                eo[k] = beta;
+                tk[k] = tau;
+            }
         }
-        off = warp_sum(off);
-        dia = warp_sum(dia);
-        if ((tid & 31) == 0) { red[2 * (tid >> 5)] = off; red[2 * (tid >> 5) + 1] = dia; }
         __syncthreads();
-        float o = 0.f, dd = 0.f;
-        for (int w = 0; w < (T >> 5); ++w) { o += red[2 * w]; dd += red[2 * w + 1]; }
-        __syncthreads();
-        if (o <= tol2 * dd) { converged = true; break; }
-        if (sweep == max_sweeps) break;
-        for (int rho = 0; rho < Ne - 1; ++rho) {
-            if (tid < half) {
-                const int k = tid;
-                auto pos = [&](int i) { return i == 0 ? 0 : 1 + (i - 1 + rho) % (Ne - 1); };
-                int p = pos(k), q = pos(Ne - 1 - k);
-                if (p > q) { int t = p; p = q; q = t; }
-                const float app = G[p * ld + p], aqq = G[q * ld + q], apq = G[p * ld + q];
-                float c = 1.f, s = 0.f;
-                if (fabsf(apq) > 1e-30f && fabsf(apq) > 1e-9f * sqrtf(fabsf(app * aqq))) {
-                    const float zeta = (aqq - app) / (2.f * apq);
-                    float t;
-                    if (fabsf(zeta) > 1e15f) {
-                        t = 0.5f / zeta;
-                    } else {
-                        t = 1.f / (fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
-                        if (zeta < 0.f) t = -t;
-                    }
-                    c = rsqrtf(fmaf(t, t, 1.f));
-                    s = t * c;
+        const float tau = tk[k];
+        if (tau != 0.f) {
+            // (b) p = tau A v over the trailing block (A symmetric: column sums, conflict-free rows)
+            {
+                const int c = tid % ld, pr = tid / ld;
+                if (pr < R && c < m) {
+                    const int i = k + 1 + c;
+                    const int per = (m + R - 1) / R;
+                    const int j0 = pr * per, j1 = min(m, j0 + per);
+                    float acc = 0.f;
+                    for (int j = j0; j < j1; ++j) acc = fmaf(G[(size_t)(k + 1 + j) * ld + i], row[k + 1 + j], acc);
+                    part[pr * ld + c] = acc;
                 }
-                rp[k] = p; rq[k] = q; rc[k] = c; rs[k] = s;
             }
             __syncthreads();
-            // columns of G and of Vm: [x_p, x_q] <- [c x_p - s x_q, s x_p + c x_q]
-            for (int i = tid; i < Ne * half; i += T) {
-                const int r = i % Ne, k = i / Ne;
-                const int p = rp[k], q = rq[k];
-                const float c = rc[k], s = rs[k];
-                float* g = G + r * ld;
-                const float gp = g[p], gq = g[q];
-                g[p] = c * gp - s * gq;
-                g[q] = s * gp + c * gq;
-                float* v = Vm + r * ld;
-                const float vp = v[p], vq = v[q];
-                v[p] = c * vp - s * vq;
-                v[q] = s * vp + c * vq;
+            // (c) p, and p . v
+            float dot = 0.f;
+            for (int c = tid; c < m; c += T) {
+                float p = 0.f;
+                for (int r = 0; r < R; ++r) p += part[r * ld + c];
+                p *= tau;
+                pv[c] = p;
+                dot = fmaf(p, row[k + 1 + c], dot);
             }
+            dot = warp_sum(dot);
+            if (lane == 0) red[wid] = dot;
             __syncthreads();
-            // rows of G: [G_p., G_q.] <- [c G_p. - s G_q., s G_p. + c G_q.]
-            for (int i = tid; i < Ne * half; i += T) {
-                const int j = i % Ne, k = i / Ne;
-                const int p = rp[k], q = rq[k];
-                const float c = rc[k], s = rs[k];
-                const float gp = G[p * ld + j], gq = G[q * ld + j];
-                float np = c * gp - s * gq, nq = s * gp + c * gq;
-                if (j == q) np = 0.f;      // the annihilated pair
-                if (j == p) nq = 0.f;
-                G[p * ld + j] = np;
-                G[q * ld + j] = nq;
+            float pvd = 0.f;
+            for (int w = 0; w < (T >> 5); ++w) pvd += red[w];
+            const float Kc = 0.5f * tau * pvd;
+            // (d) A -= v w^T + w v^T with w = p - Kc v
+            {
+                const int c = tid % ld, r0 = tid / ld;
+                if (c < m) {
+                    const float vj = row[k + 1 + c];
+                    const float wj = pv[c] - Kc * vj;
+                    for (int r = r0; r < m; r += R) {
+                        const float vi = row[k + 1 + r];
+                        const float wi = pv[r] - Kc * vi;
+                        float* g = G + (size_t)(k + 1 + r) * ld + (k + 1 + c);
+                        *g = fmaf(-vi, wj, fmaf(-wi, vj, *g));
+                    }
+                }
             }
-            __syncthreads();
+        }
+        __syncthreads();
+    }
+    if (tid == 0) {
+        if (N >= 2) {
+            dg[N - 2] = G[(size_t)(N - 2) * ld + N - 2];
+            eo[N - 2] = G[(size_t)(N - 2) * ld + N - 1];
+        }
+        dg[N - 1] = G[(size_t)(N - 1) * ld + N - 1];
+    }
+    __syncthreads();
+}
+
+// number of eigenvalues of T (diagonal dg, squared off-diagonal e2) below x
+// (Sturm count of the LDL^T pivots; a pivot smaller than pivmin counts as -pivmin)
+SEKV_DEV int sturm_count(const float* dg, const float* e2, int N, float x, float pivmin) {
+    float q = dg[0] - x;
+    if (fabsf(q) < pivmin) q = -pivmin;
+    int c = q < 0.f;
+    for (int i = 1; i < N; ++i) {
+        q = (dg[i] - x) - __fdividef(e2[i - 1], q);
+        if (fabsf(q) < pivmin) q = -pivmin;
+        c += q < 0.f;
+    }
+    return c;
+}
+
+// deterministic start vectors for inverse iteration: a hash of (vector, row) in [-1, 1)
+SEKV_DEV float start_entry(int j, int i) {
+    uint32_t h = (uint32_t)(j * 0x9E3779B1u) ^ (uint32_t)(i * 0x85EBCA77u) ^ 0x27D4EB2Fu;
+    h ^= h >> 15; h *= 0x2C1B3C6Du; h ^= h >> 12; h *= 0x297A2D39u; h ^= h >> 15;
+    return (float)(h >> 8) * (2.f / 16777216.f) - 1.f;
+}
+
+// ---------------------------------------------------------------------------
+// The rS largest eigenpairs of the tridiagonal T (dg, eo; N x N), eigenvectors
+// written to Z[j][0..N-1] (row stride ldz) in descending eigenvalue order, j < rS.
+// Scratch: Dw[rS][ldz] (pivots of the solves), e2[N], lam[rS], red[>= 64].
+// Returns false (uniform over the CTA) when a solve produced no usable vector.
+// ---------------------------------------------------------------------------
+SEKV_DEV bool top_eigvecs_tridiag(float* dg, float* eo, float* e2, int N, int rS, float* Z, int ldz, float* Dw,
+                                  float* lam, float* red, int* lost) {
+    const int tid = threadIdx.x, T = blockDim.x, lane = tid & 31, wid = tid >> 5, nw = T >> 5;
+    // Gershgorin bound of ||T||; scale T to unit norm
+    float tn = 0.f;
+    for (int i = tid; i < N; i += T) {
+        const float el = i > 0 ? fabsf(eo[i - 1]) : 0.f, er = i + 1 < N ? fabsf(eo[i]) : 0.f;
+        tn = fmaxf(tn, fabsf(dg[i]) + el + er);
+    }
+    tn = warp_max(tn);
+    if (lane == 0) red[wid] = tn;
+    __syncthreads();
+    tn = 0.f;
+    for (int w = 0; w < nw; ++w) tn = fmaxf(tn, red[w]);
+    __syncthreads();
+    if (!(tn > 0.f) || !isfinite(tn)) {
+        // T = 0: every vector is an eigenvector; take the coordinate axes
+        for (int i = tid; i < rS * ldz; i += T) Z[i] = ((i % ldz) == (i / ldz)) ? 1.f : 0.f;
+        __syncthreads();
+        return isfinite(tn);
+    }
+    const float inv = 1.f / tn;
+    for (int i = tid; i < N; i += T) {
+        dg[i] *= inv;
+        if (i + 1 < N) {
+            eo[i] *= inv;
+            e2[i] = eo[i] * eo[i];
         }
     }
-    return converged;
+    __syncthreads();
+    // ---- multisection: S threads per eigenvalue (S a power of two, <= 8)
+    const float pivmin = 1e-30f;
+    int S = 8;
+    while (S > 1 && S * rS > T) S >>= 1;
+    const int groups = T / S;
+    const int g = tid / S, s = tid % S;
+    const float tol = 4.f * FLT_EPSILON;
+    for (int j0 = 0; j0 < rS; j0 += groups) {
+        const int j = j0 + g;
+        const int k = N - 1 - (j < rS ? j : rS - 1);    // ascending index of the j-th largest
+        float lo = -1.f - 2.f * tol, hi = 1.f + 2.f * tol;    // contains every eigenvalue of the scaled T
+        // every lane of the warp runs the same iterations (the shuffles below need
+        // them all); a finished bracket only keeps shrinking
+        for (int it = 0; it < 64 && __any_sync(0xffffffffu, hi - lo > tol); ++it) {
+            const float x = lo + (float)(s + 1) * ((hi - lo) / (float)(S + 1));
+            const int c = sturm_count(dg, e2, N, x, pivmin);
+            // the largest probe with count <= k is the new lo, the smallest with count > k the new hi
+            float nlo = (c <= k) ? x : -INFINITY, nhi = (c > k) ? x : INFINITY;
+            for (int o = 1; o < S; o <<= 1) {
+                nlo = fmaxf(nlo, __shfl_xor_sync(0xffffffffu, nlo, o));
+                nhi = fminf(nhi, __shfl_xor_sync(0xffffffffu, nhi, o));
+            }
+            lo = fmaxf(lo, nlo);
+            hi = fminf(hi, nhi);
+        }
+        if (j < rS && s == 0) lam[j] = 0.5f * (lo + hi);
+    }
+    __syncthreads();
+    // ---- inverse iteration, one thread per eigenvalue: (T - lam I) x = b by the LDL^T
+    // recurrence; a pivot below eps (|T| = 1) is set to +-eps, i.e. the shift is
+    // perturbed by at most eps, which inverse iteration tolerates
+    bool good = true;
+    if (tid < rS) {
+        const int j = tid;
+        float* z = Z + (size_t)j * ldz;
+        float* D = Dw + (size_t)j * ldz;
+        const float lj = lam[j];
+        const float pv = FLT_EPSILON;
+        float nrm = 0.f;
+        for (int i = 0; i < N; ++i) {
+            z[i] = start_entry(j, i);
+            nrm = fmaf(z[i], z[i], nrm);
+        }
+        float sc = rsqrtf(fmaxf(nrm, 1e-30f));
+        for (int it = 0; it < kInvIters; ++it) {
+            // forward: D_i and y = L^{-1} (sc * b)
+            float Dp = dg[0] - lj;
+            if (fabsf(Dp) < pv) Dp = Dp < 0.f ? -pv : pv;
+            D[0] = Dp;
+            float y = z[0] * sc;
+            z[0] = y;
+            for (int i = 1; i < N; ++i) {
+                const float l = __fdividef(eo[i - 1], Dp);
+                float Dn = (dg[i] - lj) - l * eo[i - 1];
+                if (fabsf(Dn) < pv) Dn = Dn < 0.f ? -pv : pv;
+                y = fmaf(-l, y, z[i] * sc);
+                z[i] = y;
+                D[i] = Dn;
+                Dp = Dn;
+            }
+            // backward: x_i = y_i / D_i - (e_i / D_i) x_{i+1}
+            float x = __fdividef(z[N - 1], D[N - 1]);
+            z[N - 1] = x;
+            float mx = fabsf(x);
+            for (int i = N - 2; i >= 0; --i) {
+                x = __fdividef(fmaf(-eo[i], x, z[i]), D[i]);
+                z[i] = x;
+                mx = fmaxf(mx, fabsf(x));
+            }
+            // rescale by the largest entry first (no overflow in the norm), then normalise
+            const float im = mx > 0.f && isfinite(mx) ? 1.f / mx : 0.f;
+            nrm = 0.f;
+            for (int i = 0; i < N; ++i) {
+                const float v = z[i] * im;
+                z[i] = v;
+                nrm = fmaf(v, v, nrm);
+            }
+            if (!(nrm > 0.f) || !isfinite(nrm)) {
+                for (int i = 0; i < N; ++i) z[i] = start_entry(j + 977, i);     // restart from another vector
+                nrm = 0.f;
+                for (int i = 0; i < N; ++i) nrm = fmaf(z[i], z[i], nrm);
+                good = false;
+            }
+            sc = rsqrtf(nrm);
+        }
+        for (int i = 0; i < N; ++i) z[i] *= sc;
+    }
+    good = __syncthreads_and(good);
+    // ---- modified Gram-Schmidt, twice, in descending eigenvalue order. Vector j is
+    // final after step j - 1; warp w updates vectors j + 1 + w, j + 1 + w + nw, ...
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int j = 0; j < rS; ++j) {
+            const float* zj = Z + (size_t)j * ldz;
+            if (j == 0 && wid == 0) {                  // vector 0 only needs normalising
+                float nn = 0.f;
+                for (int i = lane; i < N; i += 32) nn = fmaf(zj[i], zj[i], nn);
+                nn = warp_sum(nn);
+                const float r = nn > 0.f ? rsqrtf(nn) : 0.f;
+                for (int i = lane; i < N; i += 32) Z[i] *= r;
+            }
+            __syncthreads();
+            for (int kv = j + 1 + wid; kv < rS; kv += nw) {
+                float* zk = Z + (size_t)kv * ldz;
+                float dt = 0.f;
+                for (int i = lane; i < N; i += 32) dt = fmaf(zj[i], zk[i], dt);
+                dt = warp_sum(dt);
+                float nn = 0.f;
+                for (int i = lane; i < N; i += 32) {
+                    const float v = fmaf(-dt, zj[i], zk[i]);
+                    zk[i] = v;
+                    nn = fmaf(v, v, nn);
+                }
+                if (kv == j + 1) {                     // normalise the next vector here
+                    nn = warp_sum(nn);
+                    const float r = nn > 1e-30f ? rsqrtf(nn) : 0.f;
+                    if (r == 0.f && lane == 0) *lost = 1;      // dependent vectors: reported
+                    for (int i = lane; i < N; i += 32) zk[i] *= r;
+                }
+            }
+        }
+        __syncthreads();
+    }
+    return good && *lost == 0;
+}
+
+// u = Q z for the rS vectors in Z (row stride ldz), with the reflectors stored by
+// tridiagonalize in G; one warp per vector, no block barrier inside
+SEKV_DEV void back_transform(const float* G, int ld, const float* tk, int N, int rS, float* Z, int ldz) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int j = wid; j < rS; j += nw) {
+        float* z = Z + (size_t)j * ldz;
+        for (int k = N - 3; k >= 0; --k) {
+            const float tau = tk[k];
+            if (tau == 0.f) continue;
+            const float* v = G + (size_t)k * ld;
+            float s = 0.f;
+            for (int i = k + 1 + lane; i < N; i += 32) s = fmaf(v[i], z[i], s);
+            s = warp_sum(s) * tau;
+            for (int i = k + 1 + lane; i < N; i += 32) z[i] = fmaf(-s, v[i], z[i]);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+}
+
+// threads per CTA of a bucket
+template <int NB> struct BasisThreads { static constexpr int value = NB >= 128 ? 256 : (NB >= 64 ? 128 : 64); };
+
+// shared-memory carve-up (bytes), shared by the kernel and its launcher:
+//   [ G: NB x NB fp32 | XA | small arrays ]
+// XA holds X for the Gram (|S| <= d: up to NB rows; |S| > d: 32-row chunks), then,
+// during the eigensolve, the solve pivots at offset 0 and the vectors at z_off. In
+// the factor stage X is streamed again in 32-row chunks from the start of G, which
+// may run past G into the (dead) pivots but stops before z_off.
+struct BasisSmem {
+    size_t g, xa, z_off, small, total;
+    int ldx, ldz, rsmax, R;
+};
+
+template <int DT, int NB>
+__host__ __device__ inline BasisSmem basis_smem_layout(int d, int rank) {
+    BasisSmem s;
+    constexpr int T = BasisThreads<NB>::value;
+    const int esz = DT == SEKV_BF16 ? 2 : 4;
+    s.rsmax = rank < NB ? rank : NB;
+    s.ldx = (DT == SEKV_BF16) ? d + 8 : d + 1;
+    s.ldz = NB + 1;
+    s.R = T / NB >= 1 ? T / NB : 1;
+    const int xrows = NB > kChunkRows ? NB : kChunkRows;
+    s.g = (size_t)NB * NB * 4;
+    const size_t xbytes = (size_t)xrows * s.ldx * esz;
+    const size_t chunk = (size_t)kChunkRows * s.ldx * esz;
+    const size_t zbytes = (size_t)s.rsmax * s.ldz * 4;
+    const size_t past_g = chunk > s.g ? chunk - s.g : 0;
+    s.z_off = round_up(zbytes > past_g ? zbytes : past_g, 16);
+    const size_t need = s.z_off + zbytes;
+    s.xa = round_up(xbytes > need ? xbytes : need, 16);
+    // dg, eo, e2, tk, pv: 5 x NB floats; lam: rsmax; red: 64 + R * NB floats
+    s.small = round_up((size_t)(5 * NB + s.rsmax + 64 + s.R * NB) * 4, 16);
+    s.total = s.g + s.xa + s.small;
+    return s;
 }
 
 template <int DT, int NB>
-__global__ void __launch_bounds__(NB * 4)
+__global__ void __launch_bounds__(BasisThreads<NB>::value)
 basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
     using E = Elt<DT>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int tid = threadIdx.x, T = blockDim.x;
     const int d = a.d;
-    const int ld = NB + 1;           // fp32 G / Vm row stride
-    // X staging: fp32 rows (stride d+1) for fp32 inputs, bf16 rows (stride d+8,
-    // 16-byte aligned for ldmatrix) for bf16 inputs; bf16 values are exact in fp32.
-    const int ldx = (DT == SEKV_BF16) ? d + 8 : d + 1;
-    const int xrows = NB > kChunkRows ? NB : kChunkRows;
+    constexpr int ld = NB;                          // fp32 G row stride
+    const BasisSmem L = basis_smem_layout<DT, NB>(d, a.rank);
+    const int ldx = L.ldx, ldz = L.ldz;
     float* G = reinterpret_cast<float*>(smem_raw);
-    float* Vm = G + NB * ld;
-    float* X = Vm + NB * ld;
-    __nv_bfloat16* Xb = reinterpret_cast<__nv_bfloat16*>(X);
+    unsigned char* xa = smem_raw + L.g;
+    float* X = reinterpret_cast<float*>(xa);
+    __nv_bfloat16* Xb = reinterpret_cast<__nv_bfloat16*>(xa);
+    float* Dw = reinterpret_cast<float*>(xa);                  // solve pivots
+    float* Z = reinterpret_cast<float*>(xa + L.z_off);         // eigenvectors
+    float* dg = reinterpret_cast<float*>(smem_raw + L.g + L.xa);
+    float* eo = dg + NB;
+    float* e2 = eo + NB;
+    float* tk = e2 + NB;
+    float* pv = tk + NB;
+    float* lam = pv + NB;
+    float* red = lam + L.rsmax;                    // 64 + R * NB floats
     auto xs = [&](int r, int c) -> float {
         return (DT == SEKV_BF16) ? __bfloat162float(Xb[r * ldx + c]) : X[r * ldx + c];
     };
     auto xput = [&](int r, int c, float v) {
         if (DT == SEKV_BF16) Xb[r * ldx + c] = __float2bfloat16_rn(v); else X[r * ldx + c] = v;
     };
-    int* rp = reinterpret_cast<int*>(smem_raw + round_up((size_t)2 * NB * ld * 4 +
-                                                          (size_t)xrows * ldx * (DT == SEKV_BF16 ? 2 : 4), 16));
-    int* rq = rp + NB / 2;
-    float* rc = reinterpret_cast<float*>(rq + NB / 2);
-    float* rs = rc + NB / 2;
-    float* red = rs + NB / 2;        // 2 * 32 floats
-    int* sel = reinterpret_cast<int*>(red + 64);
-    __shared__ int item_s;
+    __shared__ int item_s, lost_s;
 
     const int per_entry = a.Lr * a.Hkv * 2;
     const int total = w.bucket_count[bucket] * per_entry;
@@ -280,7 +548,6 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
             continue;   // uniform across the CTA: the loop head re-synchronises
         }
         const int N = min(len, d);
-        const int Ne = N + (N & 1);
         const int rS = block_rank(len, d, a.rank);
         const int r8 = round8(rS);
         const int64_t pa = block_ac_elems(len, rS);
@@ -339,54 +606,72 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
             }
         }
         __syncthreads();
-        // zero the padding row/column of odd N
-        if (Ne > N) {
-            for (int i = tid; i < Ne; i += T) { G[N * ld + i] = 0.f; G[i * ld + N] = 0.f; }
-        }
-        __syncthreads();
 
-        // ---- eigenvectors ---------------------------------------------------------
-        bool conv = true;
-        // bf16 factors (precision 2^-9): stop at ||off|| <= 1e-5 ||diag|| (fp32 rounding
-        // leaves ~1e-7 per element, so a much tighter test is never met, and with
-        // quadratic convergence the eigenvectors are then far more accurate than the
-        // factors are stored); fp32 factors keep the strict test (max_sweeps bounds it)
-        const float tol2 = (DT == SEKV_BF16) ? 1e-10f : 1e-12f;
-        if (Ne >= 2) conv = jacobi(G, Vm, ld, Ne, a.max_sweeps, rp, rq, rc, rs, red, tol2);
-        else if (tid == 0) Vm[0] = 1.f;
-        __syncthreads();
-        if (!conv && tid == 0) set_status(a.status, SEKV_WARN_NOT_CONVERGED);
-        // top-rS by descending eigenvalue (ties: lower index first), over the real N
-        for (int i = tid; i < N; i += T) {
-            const float li = G[i * ld + i];
-            int rank = 0;
-            for (int j = 0; j < N; ++j) {
-                const float lj = G[j * ld + j];
-                rank += (lj > li) || (lj == li && j < i);
-            }
-            if (rank < rS) sel[rank] = i;
-        }
-        __syncthreads();
+        // ---- top-rS eigenvectors of G ------------------------------------------
+        if (tid == 0) lost_s = 0;
+        tridiagonalize(G, ld, N, dg, eo, tk, pv, red);
+        const bool good = top_eigvecs_tridiag(dg, eo, e2, N, rS, Z, ldz, Dw, lam, red, &lost_s);
+        if (!good && tid == 0) set_status(a.status, SEKV_WARN_NOT_CONVERGED);
+        back_transform(G, ld, tk, N, rS, Z, ldz);
 
         // ---- factors ----------------------------------------------------------------
+        // X is streamed again in chunks of 32 rows into G's space (G is dead now)
+        __nv_bfloat16* Xc = reinterpret_cast<__nv_bfloat16*>(G);
+        float* Xf = G;
+        auto xcs = [&](int r, int c) -> float {
+            return (DT == SEKV_BF16) ? __bfloat162float(Xc[r * ldx + c]) : Xf[r * ldx + c];
+        };
+        auto xcput = [&](int r, int c, float v) {
+            if (DT == SEKV_BF16) Xc[r * ldx + c] = __float2bfloat16_rn(v); else Xf[r * ldx + c] = v;
+        };
         if (rows_form) {
-            // A[t][j] = U[t][sel j];  B[j][k] = sum_t U[t][sel j] X[t][k]
+            // A[t][j] = U[t][j];  B[j][k] = sum_t U[t][j] X[t][k]
             for (int i = tid; i < len * rS; i += T) {
                 const int t = i / rS, j = i % rS;
-                store1<DT>(fac_row, tile8_index(t, j, r8), Vm[t * ld + sel[j]]);
+                store1<DT>(fac_row, tile8_index(t, j, r8), Z[(size_t)j * ldz + t]);
             }
-            for (int i = tid; i < rS * d; i += T) {
-                const int j = i / d, k = i % d;
-                const int cj = sel[j];
-                float acc = 0.f;
-                for (int t = 0; t < len; ++t) acc = fmaf(Vm[t * ld + cj], xs(t, k), acc);
-                store1<DT>(fac_col, tile8_index(j, k, d), gate ? acc * gate[j] : acc);
+            // each thread owns outputs (j, k) = i, i + T, ... of the rS x d product, in
+            // blocks of kMaxOut (X is streamed once per block)
+            constexpr int kMaxOut = 16;
+            const int nout = (rS * d + T - 1) / T;
+            for (int q0 = 0; q0 < nout; q0 += kMaxOut) {
+                float acc[kMaxOut];
+#pragma unroll
+                for (int q = 0; q < kMaxOut; ++q) acc[q] = 0.f;
+                for (int t0 = 0; t0 < len; t0 += kChunkRows) {
+                    const int rows = min(kChunkRows, len - t0);
+                    __syncthreads();
+                    for (int i = tid; i < rows * d; i += T) {
+                        const int r = i / d, c = i % d;
+                        xcput(r, c, load1<DT>(src, (int64_t)(t0 + r) * d + c));
+                    }
+                    __syncthreads();
+#pragma unroll
+                    for (int q = 0; q < kMaxOut; ++q) {
+                        const int i = tid + (q0 + q) * T;
+                        if (q0 + q < nout && i < rS * d) {
+                            const int j = i / d, k = i % d;
+                            const float* zj = Z + (size_t)j * ldz + t0;
+                            float s = acc[q];
+                            for (int t = 0; t < rows; ++t) s = fmaf(zj[t], xcs(t, k), s);
+                            acc[q] = s;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < kMaxOut; ++q) {
+                    const int i = tid + (q0 + q) * T;
+                    if (q0 + q < nout && i < rS * d) {
+                        const int j = i / d, k = i % d;
+                        store1<DT>(fac_col, tile8_index(j, k, d), gate ? acc[q] * gate[j] : acc[q]);
+                    }
+                }
             }
         } else {
-            // B[j][k] = V[k][sel j];  A[t][j] = sum_k X[t][k] V[k][sel j]
+            // B[j][k] = V[k][j];  A[t][j] = sum_k X[t][k] V[k][j]
             for (int i = tid; i < rS * d; i += T) {
                 const int j = i / d, k = i % d;
-                const float v = Vm[k * ld + sel[j]];
+                const float v = Z[(size_t)j * ldz + k];
                 store1<DT>(fac_col, tile8_index(j, k, d), gate ? v * gate[j] : v);
             }
             for (int t0 = 0; t0 < len; t0 += kChunkRows) {
@@ -394,14 +679,14 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
                 __syncthreads();
                 for (int i = tid; i < rows * d; i += T) {
                     const int r = i / d, c = i % d;
-                    xput(r, c, load1<DT>(src, (int64_t)(t0 + r) * d + c));
+                    xcput(r, c, load1<DT>(src, (int64_t)(t0 + r) * d + c));
                 }
                 __syncthreads();
                 for (int i = tid; i < rows * rS; i += T) {
                     const int r = i / rS, j = i % rS;
-                    const int cj = sel[j];
+                    const float* zj = Z + (size_t)j * ldz;
                     float acc = 0.f;
-                    for (int k = 0; k < d; ++k) acc = fmaf(xs(r, k), Vm[k * ld + cj], acc);
+                    for (int k = 0; k < d; ++k) acc = fmaf(xcs(r, k), zj[k], acc);
                     store1<DT>(fac_row, tile8_index(t0 + r, j, r8), acc);
                 }
             }
@@ -419,31 +704,21 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
 }
 
 template <int DT, int NB>
-static size_t basis_smem(int d) {
-    const int xrows = NB > kChunkRows ? NB : kChunkRows;
-    size_t s = 2 * (size_t)NB * (NB + 1) * 4;              // G, Vm
-    s += (DT == SEKV_BF16) ? (size_t)xrows * (d + 8) * 2   // X bf16
-                           : (size_t)xrows * (d + 1) * 4;  // X fp32
-    s = round_up(s, 16);
-    s += 4 * (size_t)(NB / 2) * 4;                         // rp, rq, rc, rs
-    s += 64 * 4 + (size_t)NB * 4;                          // red, sel
-    return round_up(s, 16);
-}
-
-template <int DT, int NB>
 static cudaError_t launch_bucket(const BasisArgs& a, const BasisWork& w, int bucket, size_t cap,
                                  cudaStream_t st) {
-    const size_t smem = basis_smem<DT, NB>(a.d);
+    constexpr int T = BasisThreads<NB>::value;
+    const BasisSmem L = basis_smem_layout<DT, NB>(a.d, a.rank);
+    if (L.total > 227 * 1024) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(basis_kernel<DT, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+                                         (int)L.total);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, basis_kernel<DT, NB>, NB * 4, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, basis_kernel<DT, NB>, T, L.total);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
-    basis_kernel<DT, NB><<<sms * per_sm, NB * 4, smem, st>>>(a, w, bucket, cap);
+    basis_kernel<DT, NB><<<sms * per_sm, T, L.total, st>>>(a, w, bucket, cap);
     return cudaGetLastError();
 }
 
@@ -456,7 +731,7 @@ cudaError_t launch_basis(const sekv_build_desc& d, cudaStream_t st) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     BasisArgs a{d.m_count, d.K, d.V, d.span_beg, d.span_end, d.blk_off, d.basis_home, d.dev_status, d.rank_gate,
                 d.region_elems,
-                d.L, d.l0, d.l1 - d.l0, d.Hkv, d.n, d.d, d.m_cap, d.rank, d.max_sweeps};
+                d.L, d.l0, d.l1 - d.l0, d.Hkv, d.n, d.d, d.m_cap, d.rank};
     if (d.dtype == SEKV_F32) {
         if ((e = launch_bucket<SEKV_F32, 32>(a, w, 0, cap, st)) != cudaSuccess) return e;
         if ((e = launch_bucket<SEKV_F32, 64>(a, w, 1, cap, st)) != cudaSuccess) return e;

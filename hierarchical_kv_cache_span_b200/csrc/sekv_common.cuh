@@ -145,13 +145,14 @@ SEKV_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait: gives up after ~2^22 polls with back-off (far above any
 // legitimate wait, well under a second of wall time).
 constexpr uint32_t kWaitPolls = 1u << 22;
-SEKV_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+SEKV_DEV bool mbar_wait_n(uint64_t* bar, uint32_t parity, uint32_t polls) {
+    for (uint32_t i = 0; i < polls; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if (i > 64) __nanosleep(64);
     }
     return false;
 }
+SEKV_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) { return mbar_wait_n(bar, parity, kWaitPolls); }
 SEKV_DEV void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"

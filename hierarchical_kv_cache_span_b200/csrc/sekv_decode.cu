@@ -42,6 +42,7 @@ namespace sekv {
 constexpr int kNW = 4;          // consumer warps per CTA
 constexpr unsigned kSpanModeSpans = 64;   // zoomed spans in a CTA for whole-span pieces
 constexpr int kRMax = 64;       // largest basis rank the decode accepts
+constexpr size_t kBalMaskBytes = 5632;   // largest unit mask (G x m_cap / 32 words) dealt by rank
 
 template <int DT, int D, int G>
 struct DecCfg {
@@ -107,6 +108,11 @@ struct DecArgs {
     float scale;
     int B, L, l0, Lr, Hq, Hkv, a_cap, m_cap, rank, phase, nsplit, sch_max, qcap, mw;
     int zin;          // zoom decisions come from zmask (a capped mask) instead of l > theta
+    int bal;          // zin and the unit's whole mask fits shared memory: zoomed spans are dealt
+                      // over the unit's splits by rank instead of staying with their own split
+    int zwords;       // zoom-mask words per head in shared memory (the split's range, or the unit's)
+    uint32_t polls;   // poll limit of every bounded barrier wait
+    int starve;       // test hook: the producer issues no copy, so every wait runs out
 };
 
 // zoom bit of span S for query head hq of (b, l) in a caller-supplied (capped) mask
@@ -122,12 +128,12 @@ struct DecMaps {
 };
 
 template <int DT, int D, int G>
-static size_t decode_smem_bytes(int sch_max, int qcap) {
+static size_t decode_smem_bytes(int zwords, int qcap) {
     using C = DecCfg<DT, D, G>;
     size_t s = C::HDR;
     s += (size_t)C::RING;
     s += (size_t)kNW * qcap * 4;                               // zoom queues
-    s += (size_t)G * (sch_max / 32) * 4;                       // zoom-mask words
+    s += (size_t)G * zwords * 4;                               // zoom-mask words
     s += (size_t)kNW * C::WSCR * 4;                            // per-warp scratch
     s = round_up(s, 16) + (size_t)G * C::ROWB;                 // the group's query rows
     return round_up(s, 128) + 1024;                            // + alignment slack
@@ -343,7 +349,7 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
         for (int k = 0; k < total; ++k) {
             issue();
             const int slot = ncons % C::ZNS;
-            if (!mbar_wait(&zb[slot], (ncons / C::ZNS) & 1)) {
+            if (!mbar_wait_n(&zb[slot], (ncons / C::ZNS) & 1, a.polls)) {
                 set_status(a.status, SEKV_ERR_TIMEOUT);
                 zok = false;
                 break;
@@ -544,7 +550,7 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
     }
     // drain anything still in flight (only after an error)
     while (ncons < nis) {
-        if (!mbar_wait(&zb[ncons % C::ZNS], (ncons / C::ZNS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
+        if (!mbar_wait_n(&zb[ncons % C::ZNS], (ncons / C::ZNS) & 1, a.polls)) set_status(a.status, SEKV_ERR_TIMEOUT);
         ++ncons;
     }
 }
@@ -618,7 +624,7 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
         int okk = 1;
         if (lane == 0) {
             const int slot = (int)(np % ZNS);
-            if (np >= (uint32_t)ZNS && !mbar_wait(&sm.zempty[slot], ((np / ZNS) - 1) & 1)) okk = 0;
+            if (np >= (uint32_t)ZNS && !mbar_wait_n(&sm.zempty[slot], ((np / ZNS) - 1) & 1, a.polls)) okk = 0;
             if (okk) {
                 sm.zmeta[slot] = pc;
                 unsigned char* dst = sm.stages + (size_t)slot * ZSL;
@@ -734,7 +740,7 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
     if (lane == 0) {
         const uint32_t lo = np > (uint32_t)ZNS ? np - ZNS : 0u;
         for (uint32_t i = lo; i < np; ++i)
-            if (!mbar_wait(&sm.zfull[i % ZNS], (i / ZNS) & 1)) set_status(a.status, SEKV_ERR_TIMEOUT);
+            if (!mbar_wait_n(&sm.zfull[i % ZNS], (i / ZNS) & 1, a.polls)) set_status(a.status, SEKV_ERR_TIMEOUT);
     }
 }
 
@@ -931,7 +937,7 @@ SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int la
 
     for (uint32_t k = 0;; ++k) {
         const int slot = (int)(k % ZNS);
-        if (!mbar_wait(&sm.zfull[slot], (k / ZNS) & 1)) {
+        if (!mbar_wait_n(&sm.zfull[slot], (k / ZNS) & 1, a.polls)) {
             set_status(a.status, SEKV_ERR_TIMEOUT);
             break;
         }
@@ -1000,7 +1006,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     constexpr int DPL = C::DPL, R = C::R, TR = C::TR, NS = C::NS;
     extern __shared__ __align__(1024) unsigned char sm_raw[];
     unsigned char* base = sm_raw + ((1024 - (smem_u32(sm_raw) & 1023)) & 1023);
-    const int zwords = a.sch_max / 32;
+    const int zwords = a.zwords;
     const DecSmem sm = carve_smem<C, G, D>(base, a.qcap, zwords);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1032,7 +1038,55 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     const int nts = s1 > s0 ? (s1 - s0 + TR - 1) / TR : 0;
     const int ntiles = nta + nts;
 
-    if (tid == 0) {
+    // issue stream tile i into its ring stage (producer lane 0)
+    auto issue_tile = [&](int i) {
+        const int s = i % NS;
+        unsigned char* st = sm.stages + (size_t)s * C::STAGE;
+        if (i < nta) {
+            const int r0 = a0 + i * TR;
+            if constexpr (C::MMA) {
+                const int y = (int)(unit * a.a_cap + r0);
+                mbar_arrive_expect_tx(&sm.full[s], 2 * C::NBOX * 8192);
+#pragma unroll
+                for (int h = 0; h < C::NBOX; ++h) {
+                    tma_load_2d(st + h * 8192, &maps.Ka, 64 * h, y, &sm.full[s]);
+                    tma_load_2d(st + C::TILE + h * 8192, &maps.Va, 64 * h, y, &sm.full[s]);
+                }
+            } else {
+                const uint32_t bytes = (uint32_t)min(TR, a1 - r0) * C::ROWB;
+                mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
+                const int64_t off = (unit * a.a_cap + r0) * C::ROWB;
+                bulk_g2s(st, a.Ka + off, bytes, &sm.full[s]);
+                bulk_g2s(st + C::TILE, a.Va + off, bytes, &sm.full[s]);
+            }
+        } else {
+            const int S0 = s0 + (i - nta) * TR;
+            const int rows = min(TR, s1 - S0);
+            const uint32_t mbytes = (uint32_t)((rows + 3) & ~3) * 4;
+            if constexpr (C::MMA) {
+                const int y = (int)(unit * a.m_cap + S0);
+                mbar_arrive_expect_tx(&sm.full[s], (route_only ? 1 : 2) * C::NBOX * 8192 + 2 * mbytes);
+#pragma unroll
+                for (int h = 0; h < C::NBOX; ++h) {
+                    tma_load_2d(st + h * 8192, &maps.kbar, 64 * h, y, &sm.full[s]);
+                    if (!route_only) tma_load_2d(st + C::TILE + h * 8192, &maps.vbar, 64 * h, y, &sm.full[s]);
+                }
+            } else {
+                const uint32_t bytes = (uint32_t)rows * C::ROWB;
+                mbar_arrive_expect_tx(&sm.full[s], (route_only ? bytes : 2 * bytes) + 2 * mbytes);
+                const int64_t off = (unit * a.m_cap + S0) * C::ROWB;
+                bulk_g2s(st, a.kbar + off, bytes, &sm.full[s]);
+                if (!route_only) bulk_g2s(st + C::TILE, a.vbar + off, bytes, &sm.full[s]);
+            }
+            bulk_g2s(st + 2 * C::TILE, a.inv_norm + unit * a.m_cap + S0, mbytes, &sm.full[s]);
+            bulk_g2s(st + 2 * C::TILE + TR * 4, a.logS + (int64_t)b * a.m_cap + S0, mbytes, &sm.full[s]);
+        }
+    };
+
+    // The producer initialises the barriers and issues the first ring stages before
+    // the CTA-wide barrier, so their latency overlaps the query and mask loads.
+    const int early = min(NS, ntiles);
+    if (tid == kNW * 32) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kNW);
@@ -1048,13 +1102,32 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         *sm.zq_next = 0;
         *sm.sfail = 0;
         fence_barrier_init();
+        if (!a.starve)
+            for (int i = 0; i < early; ++i) issue_tile(i);
     }
-    for (int i = tid; i < G * zwords; i += blockDim.x) sm.zw[i] = 0u;
+    // zoom-mask words: zeros, or (balanced mode) the unit's whole mask as given, bits
+    // of spans >= m_count cleared
+    const int mw_used = (mb + 31) >> 5;
+    for (int i = tid; i < G * zwords; i += blockDim.x) {
+        const int h = i / zwords, w = i % zwords;
+        uint32_t v = 0u;
+        if (a.bal && w < mw_used) {
+            v = a.zmask[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.mw + w];
+            if (w == mw_used - 1 && (mb & 31)) v &= (1u << (mb & 31)) - 1u;
+        }
+        sm.zw[i] = v;
+    }
     {
         const uint4* qg = reinterpret_cast<const uint4*>(a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB);
         for (int i = tid; i < G * C::ROWB / 16; i += blockDim.x) reinterpret_cast<uint4*>(sm.qs)[i] = qg[i];
     }
     __syncthreads();
+    // balanced mode: does the unit zoom any span at all (the same answer in every warp)
+    bool unit_zooms = false;
+    if (a.bal) {
+        for (int i = lane; i < G * mw_used; i += 32) unit_zooms = unit_zooms || sm.zw[(i / mw_used) * zwords + i % mw_used] != 0u;
+        unit_zooms = __any_sync(0xffffffffu, unit_zooms);
+    }
 
     const float sl2 = a.scale * kLog2e;
     bool ok = true;
@@ -1082,59 +1155,20 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     if (warp == kNW) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            int issued = 0;
-            for (int i = 0; i < ntiles; ++i) {
+            int issued = a.starve ? 0 : early;
+            for (int i = early; i < ntiles && !a.starve; ++i) {
                 const int s = i % NS;
-                if (i >= NS && !mbar_wait(&sm.empty[s], ((i / NS) - 1) & 1)) {
+                if (!mbar_wait_n(&sm.empty[s], ((i / NS) - 1) & 1, a.polls)) {
                     set_status(a.status, SEKV_ERR_TIMEOUT);
                     *sm.sfail = 1;
                     break;
                 }
-                unsigned char* st = sm.stages + (size_t)s * C::STAGE;
-                if (i < nta) {
-                    const int r0 = a0 + i * TR;
-                    if constexpr (C::MMA) {
-                        const int y = (int)(unit * a.a_cap + r0);
-                        mbar_arrive_expect_tx(&sm.full[s], 2 * C::NBOX * 8192);
-#pragma unroll
-                        for (int h = 0; h < C::NBOX; ++h) {
-                            tma_load_2d(st + h * 8192, &maps.Ka, 64 * h, y, &sm.full[s]);
-                            tma_load_2d(st + C::TILE + h * 8192, &maps.Va, 64 * h, y, &sm.full[s]);
-                        }
-                    } else {
-                        const uint32_t bytes = (uint32_t)min(TR, a1 - r0) * C::ROWB;
-                        mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
-                        const int64_t off = (unit * a.a_cap + r0) * C::ROWB;
-                        bulk_g2s(st, a.Ka + off, bytes, &sm.full[s]);
-                        bulk_g2s(st + C::TILE, a.Va + off, bytes, &sm.full[s]);
-                    }
-                } else {
-                    const int S0 = s0 + (i - nta) * TR;
-                    const int rows = min(TR, s1 - S0);
-                    const uint32_t mbytes = (uint32_t)((rows + 3) & ~3) * 4;
-                    if constexpr (C::MMA) {
-                        const int y = (int)(unit * a.m_cap + S0);
-                        mbar_arrive_expect_tx(&sm.full[s], (route_only ? 1 : 2) * C::NBOX * 8192 + 2 * mbytes);
-#pragma unroll
-                        for (int h = 0; h < C::NBOX; ++h) {
-                            tma_load_2d(st + h * 8192, &maps.kbar, 64 * h, y, &sm.full[s]);
-                            if (!route_only) tma_load_2d(st + C::TILE + h * 8192, &maps.vbar, 64 * h, y, &sm.full[s]);
-                        }
-                    } else {
-                        const uint32_t bytes = (uint32_t)rows * C::ROWB;
-                        mbar_arrive_expect_tx(&sm.full[s], (route_only ? bytes : 2 * bytes) + 2 * mbytes);
-                        const int64_t off = (unit * a.m_cap + S0) * C::ROWB;
-                        bulk_g2s(st, a.kbar + off, bytes, &sm.full[s]);
-                        if (!route_only) bulk_g2s(st + C::TILE, a.vbar + off, bytes, &sm.full[s]);
-                    }
-                    bulk_g2s(st + 2 * C::TILE, a.inv_norm + unit * a.m_cap + S0, mbytes, &sm.full[s]);
-                    bulk_g2s(st + 2 * C::TILE + TR * 4, a.logS + (int64_t)b * a.m_cap + S0, mbytes, &sm.full[s]);
-                }
+                issue_tile(i);
                 issued = i + 1;
             }
             // drain: every issued copy has landed before the ring is reused
             for (int i = max(0, issued - NS); i < issued; ++i)
-                if (!mbar_wait(&sm.full[i % NS], (i / NS) & 1)) {
+                if (!mbar_wait_n(&sm.full[i % NS], (i / NS) & 1, a.polls)) {
                     set_status(a.status, SEKV_ERR_TIMEOUT);
                     *sm.sfail = 1;
                 }
@@ -1164,7 +1198,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         const int vrow = rbase + lr + ((lj >> 1) << 3);   // ... and for V
         for (int i = 0; i < ntiles && ok; ++i) {
             const int s = i % NS;
-            if (!mbar_wait(&sm.full[s], (i / NS) & 1)) {
+            if (!mbar_wait_n(&sm.full[s], (i / NS) & 1, a.polls)) {
                 set_status(a.status, SEKV_ERR_TIMEOUT);
                 ok = false;
                 break;
@@ -1208,11 +1242,12 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                             const bool valid = rv && h < G;
                             const float x = sa[e] + sb[e];
                             const float ell = fmaf(x * inv, a.scale, ls);          // Eq. (5) pre-sigmoid
-                            const bool z = valid && (a.zin ? zmask_bit(a, b, l, kvh * G + h, SL)
-                                                           : (ell > (hh ? th1 : th0)));   // Eq. (9)
+                            const bool z = valid && (a.bal ? ((sm.zw[h * zwords + (SL >> 5)] >> (SL & 31)) & 1u)
+                                                     : a.zin ? zmask_bit(a, b, l, kvh * G + h, SL)
+                                                             : (ell > (hh ? th1 : th0)));   // Eq. (9)
                             if (valid && a.route_logits)
                                 a.route_logits[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.m_cap + SL] = ell;
-                            if (z) atomicOr(&sm.zw[h * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
+                            if (z && !a.bal) atomicOr(&sm.zw[h * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
                             lg[e] = (valid && !z) ? fmaf(x, a.scale, ls) * kLog2e : -INFINITY;
                         }
                     }
@@ -1274,7 +1309,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         const int rbase = warp * R;
         for (int i = 0; i < ntiles && ok; ++i) {
             const int s = i % NS;
-            if (!mbar_wait(&sm.full[s], (i / NS) & 1)) {
+            if (!mbar_wait_n(&sm.full[s], (i / NS) & 1, a.polls)) {
                 set_status(a.status, SEKV_ERR_TIMEOUT);
                 ok = false;
                 break;
@@ -1377,14 +1412,54 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     __syncthreads();    // the stream is done: the stage ring is free, the zoom queues are complete
 
     if constexpr (C::MMA) {
-        // any zoomed span in this CTA's range (the same answer in every warp)
-        const int nwords = s1 > s0 ? (s1 - s0 + 31) >> 5 : 0;
-        bool zany = false;
-        for (int i = lane; i < G * zwords; i += 32) zany = zany || sm.zw[i] != 0u;
-        zany = __any_sync(0xffffffffu, zany);
-        if (!route_only && zany && *sm.sfail == 0) {     // uniform over the CTA
-            if (warp == kNW) zoom_produce<D, G, SP>(a, sm, lane, b, l, kvh, s0, nwords, zwords);
-            else zoom_consume<D, G, RM, SP>(a, sm, warp, lane, qb, mh, lh, oc);
+        if (a.bal) {
+            // The unit's zoomed spans (any head of the group) ranked in span order; this
+            // split takes ranks split, split + nsplit, ... wherever the spans sit, so
+            // every split of the unit gets an even share of the zoom work. Every split
+            // ranks the same mask, so each zoomed span is taken exactly once.
+            if (!route_only && unit_zooms && *sm.sfail == 0) {   // uniform over the CTA
+                if (warp == kNW) {
+                    int carry = 0;
+                    for (int w0 = 0; w0 < mw_used; w0 += 32) {
+                        const int w = w0 + lane;
+                        uint32_t u = 0u;
+                        if (w < mw_used) {
+#pragma unroll
+                            for (int h = 0; h < G; ++h) u |= sm.zw[h * zwords + w];
+                        }
+                        const int cnt = __popc(u);
+                        int inc = cnt;
+#pragma unroll
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const int t = __shfl_up_sync(0xffffffffu, inc, o);
+                            if (lane >= o) inc += t;
+                        }
+                        const int first = carry + inc - cnt;          // rank of this word's first zoomed span
+                        uint32_t keep = 0u;
+                        for (int k = ((split - first) % a.nsplit + a.nsplit) % a.nsplit; k < cnt; k += a.nsplit)
+                            keep |= 1u << (__fns(u, 0u, k + 1));
+                        if (w < mw_used) {
+#pragma unroll
+                            for (int h = 0; h < G; ++h) sm.zw[h * zwords + w] &= keep;
+                        }
+                        carry += __shfl_sync(0xffffffffu, inc, 31);
+                    }
+                    __syncwarp();
+                    zoom_produce<D, G, SP>(a, sm, lane, b, l, kvh, 0, mw_used, zwords);
+                } else {
+                    zoom_consume<D, G, RM, SP>(a, sm, warp, lane, qb, mh, lh, oc);
+                }
+            }
+        } else {
+            // any zoomed span in this CTA's range (the same answer in every warp)
+            const int nwords = s1 > s0 ? (s1 - s0 + 31) >> 5 : 0;
+            bool zany = false;
+            for (int i = lane; i < G * zwords; i += 32) zany = zany || sm.zw[i] != 0u;
+            zany = __any_sync(0xffffffffu, zany);
+            if (!route_only && zany && *sm.sfail == 0) {     // uniform over the CTA
+                if (warp == kNW) zoom_produce<D, G, SP>(a, sm, lane, b, l, kvh, s0, nwords, zwords);
+                else zoom_consume<D, G, RM, SP>(a, sm, warp, lane, qb, mh, lh, oc);
+            }
         }
     } else {
         if (!route_only && warp < kNW && ok) zoom_phase<DT, D, G>(a, sm, warp, lane, b, l, kvh, m_run, l_run, o, m_lane);
@@ -1743,7 +1818,14 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     a.qcap = C::MMA ? 0 : ((p.span_chunk + C::TR - 1) / C::TR) * C::R;   // the tensor-core path reads the bitmask
     a.mw = d.m_cap / 32;
     a.zin = zin;
-    const size_t smem = decode_smem_bytes<DT, D, G>(a.sch_max, a.qcap);
+    // test hook (sekv_decode_desc.test_flags bit 0): no copies and short waits
+    a.starve = (d.test_flags & 1) ? 1 : 0;
+    a.polls = a.starve ? 4096u : kWaitPolls;
+    // balanced zoom dealing needs the unit's whole mask in shared memory; it is used
+    // while that keeps three CTAs per SM (the mask words beside the ~70 KB ring)
+    a.bal = (C::MMA && zin && d.phase != SEKV_ROUTE && (size_t)G * a.mw * 4 <= kBalMaskBytes) ? 1 : 0;
+    a.zwords = a.bal ? a.mw : a.sch_max / 32;
+    const size_t smem = decode_smem_bytes<DT, D, G>(a.zwords, a.qcap);
     if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT, D, G, RM, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -1868,7 +1950,9 @@ void* decode_static_scratch(cudaError_t* err) {
 // (capped) mask as input.
 cudaError_t launch_decode(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st) {
     const bool learned = d.route_W != nullptr;
-    if (!learned && d.budget <= 0) return launch_pass(d, p, partials, st, 0);
+    // identity routing without a budget: FUSED and ROUTE route in the kernel; ATTEND
+    // takes the mask ROUTE wrote when the caller passes it (and routes again if not)
+    if (!learned && d.budget <= 0) return launch_pass(d, p, partials, st, d.phase == SEKV_ATTEND && d.zmask ? 1 : 0);
     // the attention pass takes the (capped / learned) mask as input; with learned
     // routing it must not overwrite the routing logits with identity-form ones
     sekv_decode_desc att = d;

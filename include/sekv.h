@@ -87,9 +87,11 @@ enum {
 /* Decode phases. FUSED: routing + attention over a hot cache (one pass for the
  * identity routing form; with a budget or learned routing, a routing pass and then
  * attention with its mask). ROUTE: routing only (writes zmask / route_logits).
- * ATTEND: attention reading bases through the slot table; it routes again
- * (bit-identical to ROUTE) in the identity form without a budget, and otherwise
- * takes zmask, as ROUTE wrote it, as input. */
+ * ATTEND: attention reading bases through the slot table; it takes zmask, as ROUTE
+ * wrote it, as input (required with a budget or learned routing; in the identity
+ * form without a budget a NULL zmask makes ATTEND route again, bit-identical to
+ * ROUTE). With the mask as input the zoom work of each (b, l, kv head) is dealt
+ * evenly over its CTAs. */
 enum { SEKV_FUSED = 0, SEKV_ROUTE = 1, SEKV_ATTEND = 2 };
 
 typedef void* sekv_stream_t;   /* a cudaStream_t (NULL = legacy default stream) */
@@ -200,7 +202,8 @@ typedef struct sekv_decode_desc {
     float* O;                /* [B][L][Hq][d] attention output (FUSED/ATTEND)              */
     float* lse;              /* [B][L][Hq] natural-log partition (FUSED/ATTEND)            */
     uint32_t* zmask;         /* optional [B][L][Hq][m_cap/32] zoom bits (bit S%32 of word   */
-                             /* S/32); required for ROUTE. Bits of spans >= m_count are 0  */
+                             /* S/32); required for ROUTE; input of ATTEND. Bits of spans  */
+                             /* >= m_count are 0 (ignored on input)                        */
     float* route_logits;     /* optional [B][L][Hq][m_cap] routing logits l_S              */
     /* learned-form routing (SeKV blog 2.3 Eq. (5)); optional. With route_W the routing
      * logit is l_S = (W^(l,h) q_h) . kbar_r_S / sqrt(dr) + logS_S, computed by a separate
@@ -236,7 +239,10 @@ typedef struct sekv_decode_desc {
                                 is used, which is faster when most spans zoom and slower
                                 when few do. Results are the same either way.            */
     int32_t dr;              /* routing dimension d' with route_W (32 or 64)                */
-    int32_t reserved;
+    int32_t test_flags;      /* 0 in normal use. Bit 0 (testing the error path): the decode
+                                kernels issue no copy and give every bounded wait ~4096 polls,
+                                so the waits run out, *dev_status reads SEKV_ERR_TIMEOUT and the
+                                kernels return with nothing in flight (O = 0, lse = -inf).   */
 } sekv_decode_desc;
 
 size_t sekv_decode_workspace_bytes(const sekv_decode_desc* desc);

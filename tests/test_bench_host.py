@@ -56,6 +56,12 @@ def test_reference_arm_json_contract():
     assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["d2h_bytes_per_step"] == 0
     for k in ("metric", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling", "config"):
         assert k in j
+    # steps x ms_per_step is the sampled work that ran; the full-step figure is labelled
+    ex = j["extrapolation"]
+    assert j["steps"] == 1 and ex["units_per_timed_step"] == j["cpu_baseline"]["cores"]
+    assert ex["full_step_ms"] == pytest.approx(j["ms_per_step"] * ex["units_per_full_step"] / ex["units_per_timed_step"])
+    assert j["value"] == pytest.approx(1e3 / ex["full_step_ms"])
+    assert j["cpu_baseline"]["cpu_model"]
 
 
 def test_percentile_and_flags():

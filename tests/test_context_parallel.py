@@ -270,3 +270,92 @@ def test_merge_partials_edge_cases():
     assert np.abs(Om[:4].double().cpu().numpy() - Oo).max() <= 1e-5
     assert np.abs(lm[:4].double().cpu().numpy() - lo).max() <= 1e-5
     assert (Om[4] == 0).all() and lm[4].item() == -math.inf
+
+
+# ---------------------------------------------------------------------------
+# The exchange path itself: two processes on the one GPU, a gloo group, and
+# context_parallel_decode (library decode of each shard, all-gather, library
+# merge) against the oracle over the whole context. The two ranks' kernels never
+# wait on each other: the exchange is a host-side collective between launches.
+# ---------------------------------------------------------------------------
+def _cp_case():
+    wl = WORKLOADS["c2"].scaled(n=4096, L=2, Hq=8, Hkv=2)
+    return wl
+
+
+def _cp_gpu_rank(rank, world, port, theta, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from hierarchical_kv_cache_span_b200 import context_parallel as CP
+        torch.cuda.set_device(0)
+        wl = _cp_case()
+        H, K, V = (x.cuda() for x in T.make_inputs(wl))      # the parent's inputs (CPU draws)
+        ac, mc = T.caps(wl)
+        sh = CP.ContextShard(wl.L, wl.Hq, wl.Hkv, wl.n, wl.d, wl.dtype, ac, mc, wl.rank, rank=rank, world=world)
+        cuts = sh.plan(H, wl.alpha, wl.window)
+        t0, t1 = cuts[rank], cuts[rank + 1]
+        sh.build(H, K[:, :, :, t0:t1].contiguous(), V[:, :, :, t0:t1].contiguous(), wl.alpha, wl.window, wl.wmode)
+        q = gen.queries(wl).cuda()
+        th = torch.tensor(theta, dtype=torch.float32, device="cuda")
+        zm = sh.cache.new_zmask()
+        O_m, lse_m = CP.context_parallel_decode(sh, q, th, zmask=zm)
+        torch.cuda.synchronize()
+        st = sh.cache.read_status()
+        k0, k1 = sh.span_range()
+        out.put((rank, st, cuts, k0, k1, O_m.double().cpu().numpy(), lse_m.double().cpu().numpy(),
+                 zm.cpu().numpy()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_context_parallel_decode_over_gloo_matches_the_oracle():
+    wl = _cp_case()
+    scale = 1.0 / math.sqrt(wl.d)
+    G = wl.Hq // wl.Hkv
+    H, K, V = T.make_inputs(wl)
+    segs = T.oracle_segments(H, wl)
+    units = T.oracle_units(K, V, H, segs, wl)
+    q = gen.queries(wl)
+    # thresholds in gaps of the oracle's routing logits (~10 % zoom); q stays as drawn
+    theta = np.zeros((wl.L, wl.Hq))
+    qn = T.f64(q)
+    for (b, l, kvh), u in units.items():
+        for g in range(G):
+            ell = T.unit_route(qn[b, l, kvh * G + g], u, g, scale)
+            th = T.calibrate_theta(ell, 0.9)
+            assert T.margin(ell, th) > T.DELTA_L
+            theta[l, kvh * G + g] = th
+    Oo, lo, zooms = T.oracle_decode(q, units, segs, theta, scale, G)
+
+    world, port = 2, 29547
+    ctx = tmp.get_context("spawn")
+    qq = ctx.Queue()
+    procs = [ctx.Process(target=_cp_gpu_rank, args=(r, world, port, theta, qq)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted([qq.get(timeout=900) for _ in range(world)], key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    m = len(segs[0].spans)
+    zoomed = 0
+    for rank, st, cuts, k0, k1, O_m, lse_m, zm in res:
+        assert st == 0
+        assert 0 < cuts[1] < cuts[2]
+        # every rank returns the merged whole-context result
+        assert np.abs(O_m[0] - Oo[0]).max() <= 2e-2
+        assert np.abs(lse_m[0] - lo[0]).max() <= 2e-2
+        # this rank's zoom bits are the oracle's for its run of global spans
+        for l in range(wl.L):
+            for h in range(wl.Hq):
+                w = zm[0, l, h].astype(np.uint32)
+                bits = ((w[:, None] >> np.arange(32, dtype=np.uint32)[None, :]) & 1).reshape(-1).astype(bool)
+                np.testing.assert_array_equal(bits[:k1 - k0], zooms[(0, l, h)][k0:k1])
+                zoomed += int(bits[:k1 - k0].sum())
+    assert sum(r[4] - r[3] for r in res) == m
+    assert zoomed > 0
+    assert np.abs(res[0][5] - res[1][5]).max() == 0.0

@@ -105,3 +105,134 @@ def test_full_size_cold_step_on_sampled_units():
         assert err <= 2e-2, (l, kvh, err)
         assert lerr <= 2e-2, (l, kvh, lerr)
     assert zoomed > 0
+
+
+# ---------------------------------------------------------------------------
+# The other Llama-shaped configs at their own full size, each in its benchmark
+# launch configuration (hot bases, one FUSED call with the automatic split plan
+# and the zoom hint from a routing pass with another query).
+#
+# Threshold margin. The kernel's routing logit differs from the oracle's fp64 one
+# only by the fp32 dot product q . kbar (128 bf16 products, fp32 accumulation:
+# |error| <= 128 * 2^-24 * sum |q_i kbar_i|, below 1e-5 after the 1/||kbar|| and
+# 1/sqrt(d) factors for these inputs); inv_norm and log|S| are the same stored fp32
+# values on both sides. With thousands of spans per head a 1e-2 gap is rare at
+# full size, so the sampled heads keep every logit >= 1e-3 from theta (100x that
+# bound): quantile thresholds move into such a gap, drawn tau keep their value and
+# the sampled heads' queries are redrawn instead.
+# ---------------------------------------------------------------------------
+DELTA_FULL = 1e-3
+
+
+def _hot_full_size_case(name, sampled):
+    import bench
+    import hierarchical_kv_cache_span_b200 as P
+    wl = WORKLOADS[name]
+    dev = torch.device("cuda")
+    G = wl.Hq // wl.Hkv
+    scale = 1.0 / math.sqrt(wl.d)
+    H, spikes = gen.surprisal(wl, device=dev)
+    K, V = gen.keys_values(wl, spikes, device=dev)
+    a_cap, m_cap = bench.caps_for(wl)
+    c = P.SpanCache(wl.B, wl.L, wl.Hq, wl.Hkv, wl.n, wl.d, wl.dtype, a_cap, m_cap, wl.rank, home=None,
+                    device=dev)
+    c.build(H, None, None, wl.alpha, wl.window, wl.wmode, steps=P.SEKV_BUILD_SCAN | P.SEKV_BUILD_LAYOUT)
+    torch.cuda.synchronize()
+    assert c.read_status() == 0
+    c.alloc_home("device", c.exact_region())
+    c.build(H, K, V, wl.alpha, wl.window, wl.wmode, steps=P.SEKV_BUILD_SUMMARY | P.SEKV_BUILD_BASES)
+    torch.cuda.synchronize()
+    assert c.read_status() == 0, P.sekv.sekv_status_str(c.read_status())
+
+    segs = {}
+    units = {}
+    for (b, l, kvh) in sampled:
+        if b not in segs:
+            Hn = T.f64(H[b])
+            segs[b] = O.segment(Hn, wl.alpha, wl.window)
+            assert T.h_margin_ok(Hn, segs[b])
+            assert int(c.a_count[b]) == len(segs[b].anchor_pos) and int(c.m_count[b]) == len(segs[b].spans)
+        units[(b, l, kvh)] = O.build_unit(T.f64(K[b, l, kvh]), T.f64(V[b, l, kvh]), T.f64(H[b]), segs[b],
+                                          wl.wmode, wl.rank, wl.dtype)
+    del K, V, spikes
+    torch.cuda.empty_cache()
+
+    q = gen.queries(wl, step=0, device=dev)
+    if wl.tau_kind == "quantile":
+        theta = bench.calibrate_theta(c, gen.queries(wl, step=10 ** 6, device=dev), wl.tau_a, P, torch)
+        theta = theta.double().cpu().numpy()
+    else:
+        theta = O.tau_to_theta(gen.taus(wl).numpy())
+    # margins on the sampled heads (every sequence of the batch shares a head's theta)
+    heads = sorted({(l, kvh * G + g) for (_, l, kvh) in sampled for g in range(G)})
+    for (l, h) in heads:
+        kvh = h // G
+        for attempt in range(200):
+            qn = T.f64(q)
+            ell = np.concatenate([T.unit_route(qn[b, l, h], u, h % G, scale)
+                                  for (b, l2, k2), u in units.items() if l2 == l and k2 == kvh])
+            if wl.tau_kind == "quantile":
+                for qt in (wl.tau_a, wl.tau_a - 0.005, wl.tau_a + 0.005, wl.tau_a - 0.01, wl.tau_a + 0.01):
+                    th = T.calibrate_theta(ell, qt, delta=DELTA_FULL)
+                    if T.margin(ell, th) > DELTA_FULL:
+                        break
+            else:
+                th = theta[l, h]
+            if T.margin(ell, th) > DELTA_FULL:
+                theta[l, h] = th
+                break
+            g_ = torch.Generator().manual_seed(gen.unit_seed(wl.seed, 98, l, h, attempt))
+            q[:, l, h] = torch.randn(wl.B, wl.d, generator=g_).to(q.dtype).to(dev)
+        else:
+            raise AssertionError(f"no margin for layer {l} head {h}")
+    th_d = torch.tensor(theta, dtype=torch.float32, device=dev)
+
+    zm = c.new_zmask()
+    c.decode(gen.queries(wl, step=10 ** 6 + 1, device=dev), th_d, phase=P.SEKV_ROUTE, zmask=zm)
+    zw = zm.cpu().numpy().view(np.uint32).reshape(wl.B, wl.L, wl.Hkv, G, -1)
+    zoom_hint = int(np.unpackbits(np.bitwise_or.reduce(zw, axis=3).view(np.uint8), axis=-1).sum()
+                    // (wl.B * wl.L * wl.Hkv))
+    zm.zero_()
+    O_g, lse_g = c.decode(q, th_d, phase=P.SEKV_FUSED, zmask=zm, zoom_hint=zoom_hint)
+    torch.cuda.synchronize()
+    assert c.read_status() == 0, P.sekv.sekv_status_str(c.read_status())
+
+    qn = T.f64(q)
+    zoomed, worst_o, worst_l = 0, 0.0, 0.0
+    for (b, l, kvh), u in units.items():
+        m = len(segs[b].spans)
+        qg = qn[b, l, kvh * G:(kvh + 1) * G]
+        z = np.stack([O.zoom_decisions(T.unit_route(qg[g], u, g, scale), theta[l, kvh * G + g])
+                      for g in range(G)])
+        for g in range(G):
+            np.testing.assert_array_equal(T.zmask_bits(zm, b, l, kvh * G + g, m), z[g],
+                                          err_msg=str((b, l, kvh, g)))
+        zoomed += int(z.sum())
+        o, ls = O.decode_unit(qg, u.Ka, u.Va, u.kbar, u.vbar, u.logS, z, u.bases, scale)
+        err = float(np.abs(T.f64(O_g[b, l, kvh * G:(kvh + 1) * G]) - o).max())
+        lerr = float(np.abs(T.f64(lse_g[b, l, kvh * G:(kvh + 1) * G]) - ls).max())
+        worst_o, worst_l = max(worst_o, err), max(worst_l, lerr)
+        assert err <= 2e-2, (b, l, kvh, err)
+        assert lerr <= 2e-2, (b, l, kvh, lerr)
+    assert zoomed > 0
+    print(f"{name}: zoom_hint {zoom_hint}, sampled zoom entries {zoomed}, max |dO| {worst_o:.2e}, "
+          f"max |dlse| {worst_l:.2e}")
+    return zoom_hint
+
+
+def test_full_size_c2_fused_on_sampled_units():
+    """32K context, 32 layers, ~2 % zoom (quantile thresholds)."""
+    _hot_full_size_case("c2", [(0, 0, 0), (0, 17, 3), (0, 31, 7)])
+
+
+def test_full_size_c4_batch8_mixed_tau_on_sampled_units():
+    """8 x 32K, tau ~ U(0.3, 0.9) per (layer, head): a zoom-dense step that runs the
+    whole-span zoom variant (its zoom hint is far above the switch point)."""
+    hint = _hot_full_size_case("c4", [(0, 0, 0), (3, 9, 2), (5, 20, 5), (7, 31, 7)])
+    assert hint >= 64
+
+
+def test_full_size_c5_rank32_quarter_zoom_on_sampled_units():
+    """128K context: the rank-32 build of all 32 layers, then a FUSED decode with ~25 %
+    of the spans zoomed."""
+    _hot_full_size_case("c5", [(0, 0, 0), (0, 16, 4), (0, 31, 7)])
