@@ -690,6 +690,10 @@ def run_sekv(args, rank, world, local_rank):
     if args.latency_form:
         out["latency_form"] = latency_form(P, torch, cache, wl, q_buf, qpool[warm], theta, O, lse, zm, fetcher,
                                            cold, learned, bud, zoom_hint, steps)
+        if cold and args.cache:
+            out["latency_form"]["prefetch_pipeline"] = prefetch_pipeline(
+                P, torch, cache, wl, q_buf, qpool, theta, O, lse, zm, fetcher.arena.numel(), bud, zoom_hint,
+                steps, warm)
     return out
 
 
@@ -797,6 +801,67 @@ def latency_form(P, torch, cache, wl, q_buf, q, theta, O, lse, zm, fetcher, cold
                 "note": ("per-layer ATTEND calls" if cold else "per-layer FUSED calls") +
                         " captured in one CUDA graph; L2 is not flushed between replays (each replay reads "
                         "the whole step, far above L2)"}
+    except Exception as e:                            # reported, never fatal to the main line
+        return {"error": f"{type(e).__name__}: {e}"}
+
+
+def prefetch_pipeline(P, torch, cache, wl, q_buf, qpool, theta, O, lse, zm, arena_elems, bud, zoom_hint, steps,
+                      warm):
+    """The serving loop's cold step, layer by layer, with the fetch overlapped: layer
+    l + 1 is routed before layer l attends, and its zoomed bases are fetched on the
+    copy stream (after that routing event, into the keep-mode device cache) while
+    layer l attends. The host takes part in every layer (the fetch reads the routing
+    result), so the step is timed with events around the whole loop, not replayed
+    from a graph."""
+    try:
+        fetcher = P.ColdFetcher(cache, arena_elems=arena_elems, keep=True)
+        comp = torch.cuda.current_stream()
+        sid = comp.cuda_stream
+        route = [cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud, l0=l, l1=l + 1)
+                 for l in range(wl.L)]
+        attend = [cache.decode_desc(q_buf, theta, phase=P.SEKV_ATTEND, O=O, lse=lse, slot=fetcher.slot_dev,
+                                    arena=fetcher.arena, zmask=zm, budget=bud, zoom_hint=zoom_hint, l0=l, l1=l + 1)
+                  for l in range(wl.L)]
+        evs = [torch.cuda.Event() for _ in range(wl.L)]
+        stats = {"bytes": 0, "copies": 0, "resident": 0, "spans": 0, "evicted": 0}
+
+        def step(t, q, count):
+            q_buf.copy_(q, non_blocking=True)
+            P.check(P.sekv.sekv_decode_attn(route[0], sid), "route")
+            evs[0].record(comp)
+            infos = [fetcher.fetch(zm, l0=0, l1=1, step=t, route_done=evs[0])]
+            for l in range(wl.L):
+                if l + 1 < wl.L:
+                    P.check(P.sekv.sekv_decode_attn(route[l + 1], sid), "route")
+                    evs[l + 1].record(comp)
+                comp.wait_event(fetcher.done)
+                P.check(P.sekv.sekv_decode_attn(attend[l], sid), "attend")
+                if l + 1 < wl.L:
+                    infos.append(fetcher.fetch(zm, l0=l + 1, l1=l + 2, step=t, route_done=evs[l + 1]))
+            if count:
+                for i in infos:
+                    for k in stats:
+                        stats[k] += i[k]
+
+        for t in range(warm):
+            step(t, qpool[t], False)
+        torch.cuda.synchronize()
+        ts = []
+        for i in range(steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(comp)
+            step(warm + i, qpool[warm + i], True)
+            e1.record(comp)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        st = cache.read_status()
+        return {"us_per_step": statistics.median(ts) * 1e3, "us_p10": pct(ts, 10) * 1e3,
+                "us_p90": pct(ts, 90) * 1e3, "steps_per_s": 1e3 / statistics.median(ts), "status": st,
+                "fetch_bytes_per_step": stats["bytes"] / steps, "copies_per_step": stats["copies"] / steps,
+                "resident_spans_per_step": stats["resident"] / steps,
+                "copied_spans_per_step": stats["spans"] / steps, "evicted_per_step": stats["evicted"] / steps,
+                "note": "per layer: ROUTE(l+1), ATTEND(l), fetch(l+1) on the copy stream after ROUTE(l+1) "
+                        "(keep-mode cache, arena as the main line's); i.i.d. queries"}
     except Exception as e:                            # reported, never fatal to the main line
         return {"error": f"{type(e).__name__}: {e}"}
 

@@ -230,8 +230,12 @@ class ColdFetcher:
     """Pinned mirrors, device arena and slot table for fetching cold bases.
 
     keep=False: every fetch refills the arena with the step's zoomed spans.
-    keep=True: the arena is a device cache across fetches (resident spans are not
-    copied again; a full arena is flushed and refilled)."""
+    keep=True: the arena is a device cache across fetches: resident spans are not
+    copied again, misses go to free space, and the least recently used spans not
+    needed by this step or the previous one are evicted when space runs out.
+    ``step`` (keep mode) is the caller's decode-step counter; ``route_done`` (keep
+    mode) an event recorded after the ROUTE call whose mask is fetched, so that the
+    copies may overlap work queued after it (the previous layer's ATTEND)."""
 
     def __init__(self, cache: SpanCache, arena_elems: int, keep: bool = False):
         self.c = cache
@@ -242,10 +246,11 @@ class ColdFetcher:
         self.arena = torch.zeros(max(arena_elems, 64), dtype=cache.dt, device=dev)
         self.slot_dev = torch.full((B, L, m_cap), -1, dtype=torch.int64, device=dev)
         self.slot_host = torch.full((B, L, m_cap), -1, dtype=torch.int64, pin_memory=True)
+        self.last_use = torch.full((B, L, m_cap), -1, dtype=torch.int64)
         self.zmask_host = torch.zeros(B, L, Hq, m_cap // 32, dtype=torch.int32, pin_memory=True)
         self.m_count_host = cache.m_count.to("cpu")
         self.blk_off_host = cache.blk_off.to("cpu")
-        self.stats = torch.zeros(4, dtype=torch.int64)
+        self.stats = torch.zeros(5, dtype=torch.int64)
         self.copy_stream = torch.cuda.Stream(device=dev)
         self.done = torch.cuda.Event()
         self.done.record(self.copy_stream)
@@ -254,19 +259,21 @@ class ColdFetcher:
         self.m_count_host = self.c.m_count.to("cpu")
         self.blk_off_host = self.c.blk_off.to("cpu")
 
-    def fetch(self, zmask: torch.Tensor, l0=0, l1=None, compute=None):
+    def fetch(self, zmask: torch.Tensor, l0=0, l1=None, compute=None, step=0, route_done=None):
         c = self.c
         d = S.sekv_fetch_desc()
         d.zmask_dev, d.zmask_host = _ptr(zmask), _ptr(self.zmask_host)
         d.m_count_host, d.blk_off_host = _ptr(self.m_count_host), _ptr(self.blk_off_host)
         d.home, d.arena = _ptr(c.home), _ptr(self.arena)
         d.slot_dev, d.slot_host, d.stats = _ptr(self.slot_dev), _ptr(self.slot_host), _ptr(self.stats)
-        d.region_elems, d.arena_elems = c.region, self.arena.numel()
+        d.arena_used, d.last_use = _ptr(self.arena_used), _ptr(self.last_use) if self.keep else None
+        d.route_done = route_done.cuda_event if route_done is not None else None
+        d.region_elems, d.arena_elems, d.step = c.region, self.arena.numel(), int(step)
         d.B, d.L, d.Hq, d.Hkv, d.d, d.dtype = c.B, c.L, c.Hq, c.Hkv, c.d, c.code
         d.l0, d.l1, d.m_cap, d.rank = l0, c.L if l1 is None else l1, c.m_cap, c.rank
-        d.keep, d.arena_used = int(self.keep), _ptr(self.arena_used)
+        d.keep = int(self.keep)
         cs = _stream(compute)
         st = S.sekv_fetch_bases(d, cs, self.copy_stream.cuda_stream, self.done.cuda_event)
         S.check(st, "sekv_fetch_bases")
         return dict(bytes=int(self.stats[0]), spans=int(self.stats[1]), copies=int(self.stats[2]),
-                    resident=int(self.stats[3]))
+                    resident=int(self.stats[3]), evicted=int(self.stats[4]))

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <string>
 #include <vector>
 
@@ -159,7 +160,7 @@ const char* sekv_status_str(int32_t s) {
         case SEKV_ERR_COLD_SPAN: return "zoomed span has no resident bases";
         case SEKV_ERR_TIMEOUT: return "bounded device wait ran out";
         case SEKV_ERR_UNSUPPORTED: return "unsupported shape";
-        case SEKV_WARN_NOT_CONVERGED: return "Jacobi solve hit max_sweeps";
+        case SEKV_WARN_NOT_CONVERGED: return "basis eigenvector solve failed";
         default: return "unknown status";
     }
 }
@@ -266,6 +267,166 @@ sekv_status sekv_tau_to_theta(const double* tau, float* theta, int64_t n) {
     return SEKV_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Keep mode: the arena as a cache of span entries across calls. Entry (b, l, S)
+// holds span S's Hkv blocks of layer l at [slot, slot + blk_off[S+1] - blk_off[S]).
+// Misses are placed first-fit in the free gaps; when none is large enough, entries
+// are evicted least recently used first (by last_use, then (b, l, S)) among those
+// that neither this call nor the calls of this step or the previous one needed:
+// an ATTEND of those steps may still be reading them. Nothing is changed on the
+// host or the device unless every miss finds room.
+struct KeepPlan {
+    struct Copy { int64_t src, dst, width; int b, l; };
+    std::vector<int64_t> hit;                           // slot-table indices of the hits
+    std::vector<Copy> copies;
+    std::vector<std::pair<int64_t, int64_t>> evict;     // (index into the slot table, unused)
+    std::vector<std::pair<int64_t, int64_t>> place;     // (index into the slot table, slot)
+    std::vector<uint8_t> dirty;                         // per layer: slot rows to upload
+    int64_t hits = 0, spans = 0, bytes_elems = 0, used = 0;
+};
+
+bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
+    const int mw = d->m_cap / 32;
+    const int64_t step = d->step;
+    auto idx = [&](int b, int l, int S) { return ((int64_t)b * d->L + l) * d->m_cap + S; };
+    auto size_of = [&](int b, int S) {
+        const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
+        return bo[S + 1] - bo[S];
+    };
+    // spans this call needs: any head of (b, l) zooms them (rows of [l0, l1) only)
+    const int Lr = d->l1 - d->l0;
+    std::vector<uint32_t> needw((size_t)d->B * Lr * mw, 0u);
+    int64_t misses = 0;
+    for (int b = 0; b < d->B; ++b) {
+        const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
+        for (int l = d->l0; l < d->l1; ++l) {
+            uint32_t* uni = needw.data() + ((size_t)b * Lr + (l - d->l0)) * mw;
+            const uint32_t* zm = d->zmask_host + ((int64_t)b * d->L + l) * d->Hq * mw;
+            for (int h = 0; h < d->Hq; ++h)
+                for (int w = 0; w < mw; ++w) uni[w] |= zm[h * mw + w];
+            if (m < d->m_cap) {                                   // bits of spans >= m_count are ignored
+                for (int w = m >> 5; w < mw; ++w) uni[w] &= (w == (m >> 5)) ? ((1u << (m & 31)) - 1u) : 0u;
+            }
+            for (int w = 0; w < mw; ++w)
+                for (uint32_t bits = uni[w]; bits; bits &= bits - 1u) {
+                    const int S = (w << 5) + __builtin_ctz(bits);
+                    if (d->slot_host[idx(b, l, S)] >= 0) kp.hit.push_back(idx(b, l, S));
+                    else ++misses;
+                }
+        }
+    }
+    auto needed = [&](int b, int l, int S) {
+        if (l < d->l0 || l >= d->l1) return false;
+        return ((needw[((size_t)b * Lr + (l - d->l0)) * mw + (S >> 5)] >> (S & 31)) & 1u) != 0u;
+    };
+    kp.hits = (int64_t)kp.hit.size();
+    kp.dirty.assign(d->L, 0);
+    if (misses == 0) {                                    // nothing to place: no scan of the arena
+        kp.used = d->arena_used ? *d->arena_used : 0;
+        return true;
+    }
+    // resident entries: the occupied intervals and the eviction candidates
+    struct Ent { int64_t last, off, size, id; int b, l; };
+    std::vector<Ent> occ, cand;
+    for (int b = 0; b < d->B; ++b) {
+        const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
+        for (int l = 0; l < d->L; ++l)
+            for (int S = 0; S < m; ++S) {
+                const int64_t i = idx(b, l, S), off = d->slot_host[i];
+                if (off < 0) continue;
+                const Ent e{d->last_use[i], off, size_of(b, S), i, b, l};
+                occ.push_back(e);
+                if (!needed(b, l, S) && e.last < step - 1) cand.push_back(e);
+            }
+    }
+    std::sort(occ.begin(), occ.end(), [](const Ent& x, const Ent& y) { return x.off < y.off; });
+    std::sort(cand.begin(), cand.end(), [](const Ent& x, const Ent& y) {
+        return x.last != y.last ? x.last < y.last : x.id < y.id;
+    });
+    std::map<int64_t, int64_t> gaps;                    // offset -> elements
+    int64_t cur = 0;
+    for (const Ent& e : occ) {
+        if (e.off > cur) gaps[cur] = e.off - cur;
+        cur = std::max(cur, e.off + e.size);
+        kp.used += e.size;
+    }
+    if (d->arena_elems > cur) gaps[cur] = d->arena_elems - cur;
+    auto release = [&](int64_t off, int64_t size) {
+        auto nx = gaps.lower_bound(off);
+        if (nx != gaps.end() && nx->first == off + size) {
+            size += nx->second;
+            nx = gaps.erase(nx);
+        }
+        if (nx != gaps.begin()) {
+            auto pv = std::prev(nx);
+            if (pv->first + pv->second == off) {
+                pv->second += size;
+                return;
+            }
+        }
+        gaps[off] = size;
+    };
+    size_t next_victim = 0;
+    auto alloc = [&](int64_t size) -> int64_t {
+        for (;;) {
+            for (auto it = gaps.begin(); it != gaps.end(); ++it) {
+                if (it->second < size) continue;
+                const int64_t off = it->first, rest = it->second - size;
+                gaps.erase(it);
+                if (rest > 0) gaps[off + size] = rest;
+                return off;
+            }
+            if (next_victim >= cand.size()) return -1;
+            const Ent& v = cand[next_victim++];
+            kp.evict.push_back({v.id, 0});
+            kp.dirty[v.l] = 1;
+            kp.used -= v.size;
+            release(v.off, v.size);
+        }
+    };
+    for (int b = 0; b < d->B; ++b) {
+        const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
+        const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
+        for (int l = d->l0; l < d->l1; ++l) {
+            int S = 0;
+            while (S < m) {
+                const int64_t i = idx(b, l, S);
+                if (!needed(b, l, S) || d->slot_host[i] >= 0) { ++S; continue; }
+                const int Sa = S;                        // a run of consecutive misses
+                while (S < m && needed(b, l, S) && d->slot_host[idx(b, l, S)] < 0) ++S;
+                const int64_t width = bo[S] - bo[Sa];
+                const int64_t src = ((int64_t)b * d->L + l) * d->region_elems + bo[Sa];
+                int64_t off = alloc(width);
+                if (off >= 0) {
+                    for (int t = Sa; t < S; ++t) kp.place.push_back({idx(b, l, t), off + (bo[t] - bo[Sa])});
+                    kp.copies.push_back({src, off, width, b, l});
+                } else {
+                    // no room for the whole run: place its spans one by one
+                    for (int t = Sa; t < S; ++t) {
+                        const int64_t w1 = bo[t + 1] - bo[t];
+                        const int64_t o1 = alloc(w1);
+                        if (o1 < 0) return false;
+                        kp.place.push_back({idx(b, l, t), o1});
+                        kp.copies.push_back({src + (bo[t] - bo[Sa]), o1, w1, b, l});
+                    }
+                }
+                kp.spans += S - Sa;
+                kp.bytes_elems += width;
+                kp.used += width;
+                kp.dirty[l] = 1;
+            }
+        }
+    }
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
 sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, sekv_stream_t copy,
                              sekv_event_t done) {
     SEKV_REQUIRE(d, "fetch: null descriptor");
@@ -276,9 +437,11 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
                      d->l1 <= d->L && d->m_cap >= 32 && d->m_cap % 32 == 0 && d->region_elems > 0 &&
                      d->arena_elems >= 0 && (d->dtype == SEKV_F32 || d->dtype == SEKV_BF16),
                  "fetch: bad shape");
-    SEKV_REQUIRE(d->keep == 0 || (d->keep == 1 && d->arena_used && *d->arena_used >= 0 &&
-                                  *d->arena_used <= d->arena_elems),
-                 "fetch: keep must be 0 or 1, and keep mode needs arena_used in [0, arena_elems]");
+    SEKV_REQUIRE(d->keep == 0 || (d->keep == 1 && d->last_use && d->step >= 0),
+                 "fetch: keep must be 0 or 1, and keep mode needs last_use and a step >= 0");
+    SEKV_REQUIRE(!d->route_done || d->keep == 1,
+                 "fetch: route_done (a fetch that overlaps earlier ATTEND calls) needs keep mode: a refill "
+                 "would overwrite bases those calls may still read");
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(compute);
     cudaStream_t xs = reinterpret_cast<cudaStream_t>(copy);
     cudaEvent_t ev = reinterpret_cast<cudaEvent_t>(done);
@@ -287,21 +450,71 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
     cudaError_t e;
     // the previous call's slot upload must be finished before the mirror is rewritten
     if ((e = cudaEventSynchronize(ev)) != cudaSuccess) return cuda_fail(e, "fetch: previous done event");
+    // the routing result: after route_done on the copy stream (the compute stream may
+    // already hold later work), else on the compute stream after all its work
+    cudaStream_t rs = cs;
+    if (d->route_done) {
+        if ((e = cudaStreamWaitEvent(xs, reinterpret_cast<cudaEvent_t>(d->route_done), 0)) != cudaSuccess)
+            return cuda_fail(e, "fetch: wait for route_done");
+        rs = xs;
+    }
     for (int b = 0; b < d->B; ++b) {
         const int64_t w0 = ((int64_t)b * d->L + d->l0) * d->Hq * mw;
         if ((e = cudaMemcpyAsync(d->zmask_host + w0, d->zmask_dev + w0, sizeof(uint32_t) * Lr * d->Hq * mw,
-                                 cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+                                 cudaMemcpyDeviceToHost, rs)) != cudaSuccess)
             return cuda_fail(e, "fetch: zmask readback");
     }
-    // the host needs the routing result; this also orders the copies after the
-    // previous step's ATTEND (which ran earlier on `compute`)
-    if ((e = cudaStreamSynchronize(cs)) != cudaSuccess) return cuda_fail(e, "fetch: compute stream");
+    // the host needs the routing result; without route_done this also orders the
+    // copies after the previous step's ATTEND (which ran earlier on `compute`)
+    if ((e = cudaStreamSynchronize(rs)) != cudaSuccess) return cuda_fail(e, "fetch: routing result");
+    const char* home = reinterpret_cast<const char*>(d->home);
+    char* arena = reinterpret_cast<char*>(d->arena);
 
-    // A span's blocks sit at the same offset blk_off[b][S] of every layer's region,
-    // so a run of consecutive spans zoomed in a run of consecutive layers is one
-    // pitched rectangle of the home: width = the spans' blocks, height = the
-    // layers, source pitch = the region. The copy engine pays a fixed cost per
-    // copy (a few microseconds), so one rectangle per (span run, layer run)
+    if (d->keep == 1) {
+        KeepPlan kp;
+        if (!plan_keep(d, kp)) {
+            if ((e = cudaEventRecord(ev, xs)) != cudaSuccess) return cuda_fail(e, "fetch: record");
+            return fail(SEKV_ERR_CAPACITY,
+                        "fetch: the zoomed bases that are not resident do not fit the arena of %lld elements "
+                        "even after evicting every span this step and the previous one do not need",
+                        (long long)d->arena_elems);
+        }
+        for (const auto& v : kp.evict) d->slot_host[v.first] = -1;
+        for (const auto& p : kp.place) {
+            d->slot_host[p.first] = p.second;
+            d->last_use[p.first] = d->step;
+        }
+        for (const int64_t i : kp.hit) d->last_use[i] = d->step;     // hits are stamped too
+        for (const auto& c : kp.copies)
+            if ((e = cudaMemcpyAsync(arena + c.dst * es, home + c.src * es, c.width * es, cudaMemcpyHostToDevice,
+                                     xs)) != cudaSuccess)
+                return cuda_fail(e, "fetch: basis copy");
+        for (int l = 0; l < d->L; ++l) {
+            if (!kp.dirty[l]) continue;
+            for (int b = 0; b < d->B; ++b) {
+                const int64_t o = ((int64_t)b * d->L + l) * d->m_cap;
+                if ((e = cudaMemcpyAsync(d->slot_dev + o, d->slot_host + o, sizeof(int64_t) * d->m_cap,
+                                         cudaMemcpyHostToDevice, xs)) != cudaSuccess)
+                    return cuda_fail(e, "fetch: slot upload");
+            }
+        }
+        if (d->stats) {
+            d->stats[0] = kp.bytes_elems * es;
+            d->stats[1] = kp.spans;
+            d->stats[2] = (int64_t)kp.copies.size();
+            d->stats[3] = kp.hits;
+            d->stats[4] = (int64_t)kp.evict.size();
+        }
+        if (d->arena_used) *d->arena_used = kp.used;
+        if ((e = cudaEventRecord(ev, xs)) != cudaSuccess) return cuda_fail(e, "fetch: record");
+        return SEKV_OK;
+    }
+
+    // Refill mode. A span's blocks sit at the same offset blk_off[b][S] of every
+    // layer's region, so a run of consecutive spans zoomed in a run of consecutive
+    // layers is one pitched rectangle of the home: width = the spans' blocks,
+    // height = the layers, source pitch = the region. The copy engine pays a fixed
+    // cost per copy (a few microseconds), so one rectangle per (span run, layer run)
     // instead of one copy per (span run, layer) is what keeps the fetch near the
     // PCIe rate.
     struct Rect { int64_t src, dst, width, height; };
@@ -313,107 +526,72 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
         cudaDeviceGetAttribute(&max_pitch, cudaDevAttrMaxPitch, dev) != cudaSuccess)
         max_pitch = 0;
     const bool pitched = (int64_t)max_pitch >= d->region_elems * es;
-    const bool keep = d->keep == 1;
-    int64_t bump = 0, spans = 0, hits = 0;
-    // Plan the copies of every zoomed (b, l, S) that is not resident, appending at
-    // `start`; fill the host slot mirror. Returns the arena end.
-    auto plan = [&](int64_t start) -> int64_t {
-        rects.clear();
-        spans = hits = 0;
-        int64_t end = start;
-        for (int b = 0; b < d->B; ++b) {
-            const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
-            const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
-            if (!keep) {
-                for (int l = d->l0; l < d->l1; ++l) {
-                    int64_t* sl = d->slot_host + ((int64_t)b * d->L + l) * d->m_cap;
-                    for (int S = 0; S < d->m_cap; ++S) sl[S] = -1;
-                }
+    int64_t end = 0, spans = 0;
+    for (int b = 0; b < d->B; ++b) {
+        const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
+        const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
+        for (int l = d->l0; l < d->l1; ++l) {
+            int64_t* sl = d->slot_host + ((int64_t)b * d->L + l) * d->m_cap;
+            for (int S = 0; S < d->m_cap; ++S) sl[S] = -1;
+        }
+        // layers in chunks of 64: lmask[S] bit j = span S zoomed (by any head) in layer lc + j
+        for (int lc = d->l0; lc < d->l1; lc += 64) {
+            const int nl = d->l1 - lc < 64 ? d->l1 - lc : 64;
+            lmask.assign(m, 0ull);
+            uni.assign(mw, 0u);
+            for (int j = 0; j < nl; ++j) {
+                std::fill(uni.begin(), uni.end(), 0u);
+                const uint32_t* zm = d->zmask_host + ((int64_t)b * d->L + lc + j) * d->Hq * mw;
+                for (int h = 0; h < d->Hq; ++h)
+                    for (int w = 0; w < mw; ++w) uni[w] |= zm[h * mw + w];
+                for (int S = 0; S < m; ++S)
+                    if ((uni[S >> 5] >> (S & 31)) & 1u) lmask[S] |= 1ull << j;
             }
-            // layers in chunks of 64: lmask[S] bit j = span S zoomed (by any head) in
-            // layer lc + j and not resident
-            for (int lc = d->l0; lc < d->l1; lc += 64) {
-                const int nl = d->l1 - lc < 64 ? d->l1 - lc : 64;
-                lmask.assign(m, 0ull);
-                uni.assign(mw, 0u);
-                for (int j = 0; j < nl; ++j) {
-                    std::fill(uni.begin(), uni.end(), 0u);
-                    const uint32_t* zm = d->zmask_host + ((int64_t)b * d->L + lc + j) * d->Hq * mw;
-                    for (int h = 0; h < d->Hq; ++h)
-                        for (int w = 0; w < mw; ++w) uni[w] |= zm[h * mw + w];
-                    const int64_t* sl = d->slot_host + ((int64_t)b * d->L + lc + j) * d->m_cap;
-                    for (int S = 0; S < m; ++S)
-                        if ((uni[S >> 5] >> (S & 31)) & 1u) {
-                            if (keep && sl[S] >= 0) ++hits;
-                            else lmask[S] |= 1ull << j;
-                        }
-                }
-                int S = 0;
-                while (S < m) {
-                    if (!lmask[S]) { ++S; continue; }
-                    const int Sa = S;
-                    const uint64_t mk = lmask[S];
-                    while (S < m && lmask[S] == mk) ++S;      // spans [Sa, S) share the layer set
-                    const int64_t width = bo[S] - bo[Sa];
-                    spans += (int64_t)(S - Sa) * __builtin_popcountll(mk);
-                    int j = 0;
-                    while (j < nl) {
-                        if (!((mk >> j) & 1ull)) { ++j; continue; }
-                        const int ja = j;
-                        while (j < nl && ((mk >> j) & 1ull)) ++j;   // layers [lc + ja, lc + j)
-                        const int hgt = j - ja;
-                        for (int q = 0; q < hgt; ++q) {
-                            int64_t* sl = d->slot_host + ((int64_t)b * d->L + lc + ja + q) * d->m_cap;
-                            for (int t = Sa; t < S; ++t) sl[t] = end + (int64_t)q * width + (bo[t] - bo[Sa]);
-                        }
-                        const int64_t src = ((int64_t)b * d->L + lc + ja) * d->region_elems + bo[Sa];
-                        if (pitched) {
-                            rects.push_back({src, end, width, hgt});
-                        } else {
-                            for (int q = 0; q < hgt; ++q)
-                                rects.push_back({src + (int64_t)q * d->region_elems, end + (int64_t)q * width, width, 1});
-                        }
-                        end += (int64_t)hgt * width;
+            int S = 0;
+            while (S < m) {
+                if (!lmask[S]) { ++S; continue; }
+                const int Sa = S;
+                const uint64_t mk = lmask[S];
+                while (S < m && lmask[S] == mk) ++S;      // spans [Sa, S) share the layer set
+                const int64_t width = bo[S] - bo[Sa];
+                spans += (int64_t)(S - Sa) * __builtin_popcountll(mk);
+                int j = 0;
+                while (j < nl) {
+                    if (!((mk >> j) & 1ull)) { ++j; continue; }
+                    const int ja = j;
+                    while (j < nl && ((mk >> j) & 1ull)) ++j;   // layers [lc + ja, lc + j)
+                    const int hgt = j - ja;
+                    for (int q = 0; q < hgt; ++q) {
+                        int64_t* sl = d->slot_host + ((int64_t)b * d->L + lc + ja + q) * d->m_cap;
+                        for (int t = Sa; t < S; ++t) sl[t] = end + (int64_t)q * width + (bo[t] - bo[Sa]);
                     }
+                    const int64_t src = ((int64_t)b * d->L + lc + ja) * d->region_elems + bo[Sa];
+                    if (pitched) {
+                        rects.push_back({src, end, width, hgt});
+                    } else {
+                        for (int q = 0; q < hgt; ++q)
+                            rects.push_back({src + (int64_t)q * d->region_elems, end + (int64_t)q * width, width, 1});
+                    }
+                    end += (int64_t)hgt * width;
                 }
             }
         }
-        return end;
-    };
-    auto reset_slots = [&]() {
-        for (int b = 0; b < d->B; ++b)
-            for (int l = d->l0; l < d->l1; ++l) {
-                int64_t* sl = d->slot_host + ((int64_t)b * d->L + l) * d->m_cap;
-                for (int S = 0; S < d->m_cap; ++S) sl[S] = -1;
-            }
-    };
-    bump = plan(keep ? *d->arena_used : 0);
-    if (keep && bump > d->arena_elems) {
-        // the misses do not fit behind the resident spans: flush and refill
-        reset_slots();
-        bump = plan(0);
     }
     if (d->stats) {
         d->stats[0] = 0;
         for (const Rect& r : rects) d->stats[0] += r.width * r.height * es;
         d->stats[1] = spans;
         d->stats[2] = (int64_t)rects.size();
-        d->stats[3] = hits;
+        d->stats[3] = 0;
+        d->stats[4] = 0;
     }
-    if (bump > d->arena_elems) {
-        // nothing is copied and the device slot table stays as it was; a keep-mode
-        // cache is emptied on the host side
-        if (keep) {
-            reset_slots();
-            *d->arena_used = 0;
-        }
+    if (end > d->arena_elems) {
+        // nothing is copied and the device slot table stays as it was
         if ((e = cudaEventRecord(ev, xs)) != cudaSuccess) return cuda_fail(e, "fetch: record");
         return fail(SEKV_ERR_CAPACITY, "fetch: zoomed bases need %lld elements, arena holds %lld",
-                    (long long)bump, (long long)d->arena_elems);
+                    (long long)end, (long long)d->arena_elems);
     }
-    if (keep) *d->arena_used = bump;
-    const char* home = reinterpret_cast<const char*>(d->home);
-    char* arena = reinterpret_cast<char*>(d->arena);
+    if (d->arena_used) *d->arena_used = end;
     for (const Rect& r : rects) {
         if (r.height == 1)
             e = cudaMemcpyAsync(arena + r.dst * es, home + r.src * es, r.width * es, cudaMemcpyHostToDevice, xs);

@@ -41,10 +41,13 @@ namespace sekv {
 constexpr int kBuckets = 3;
 constexpr int kChunkRows = 32;    // rows of X staged per step when |S| > d
 constexpr int kInvIters = 3;      // inverse-iteration steps per eigenvector
+constexpr float kBig = 1e20f;     // rescaling threshold of the tridiagonal solves
+constexpr float kSmall = 1e-20f;
 
 struct BasisWork {
     int* bucket_count;   // [kBuckets]
     int* work_next;      // [kBuckets]
+    int* failures;       // [2]: eigenvectors restarted after a failed solve; vectors lost in Gram-Schmidt
     int2* list;          // [kBuckets][B * m_cap]  (b, S)
 };
 
@@ -59,6 +62,7 @@ static BasisWork carve(const sekv_build_desc& d) {
     char* p = reinterpret_cast<char*>(d.workspace);
     w.bucket_count = reinterpret_cast<int*>(p);
     w.work_next = reinterpret_cast<int*>(p + 64);
+    w.failures = reinterpret_cast<int*>(p + 128);
     w.list = reinterpret_cast<int2*>(p + 256);
     return w;
 }
@@ -283,7 +287,7 @@ SEKV_DEV float start_entry(int j, int i) {
 // Returns false (uniform over the CTA) when a solve produced no usable vector.
 // ---------------------------------------------------------------------------
 SEKV_DEV bool top_eigvecs_tridiag(float* dg, float* eo, float* e2, int N, int rS, float* Z, int ldz, float* Dw,
-                                  float* lam, float* red, int* lost) {
+                                  float* lam, float* red, int* lost, int* failures) {
     const int tid = threadIdx.x, T = blockDim.x, lane = tid & 31, wid = tid >> 5, nw = T >> 5;
     // Gershgorin bound of ||T||; scale T to unit norm
     float tn = 0.f;
@@ -340,76 +344,28 @@ SEKV_DEV bool top_eigvecs_tridiag(float* dg, float* eo, float* e2, int N, int rS
         if (j < rS && s == 0) lam[j] = 0.5f * (lo + hi);
     }
     __syncthreads();
-    // ---- inverse iteration, one thread per eigenvalue: (T - lam I) x = b by the LDL^T
-    // recurrence; a pivot below eps (|T| = 1) is set to +-eps, i.e. the shift is
-    // perturbed by at most eps, which inverse iteration tolerates
-    bool good = true;
-    if (tid < rS) {
-        const int j = tid;
-        float* z = Z + (size_t)j * ldz;
-        float* D = Dw + (size_t)j * ldz;
-        const float lj = lam[j];
-        const float pv = FLT_EPSILON;
-        float nrm = 0.f;
-        for (int i = 0; i < N; ++i) {
-            z[i] = start_entry(j, i);
-            nrm = fmaf(z[i], z[i], nrm);
-        }
-        float sc = rsqrtf(fmaxf(nrm, 1e-30f));
-        for (int it = 0; it < kInvIters; ++it) {
-            // forward: D_i and y = L^{-1} (sc * b)
-            float Dp = dg[0] - lj;
-            if (fabsf(Dp) < pv) Dp = Dp < 0.f ? -pv : pv;
-            D[0] = Dp;
-            float y = z[0] * sc;
-            z[0] = y;
-            for (int i = 1; i < N; ++i) {
-                const float l = __fdividef(eo[i - 1], Dp);
-                float Dn = (dg[i] - lj) - l * eo[i - 1];
-                if (fabsf(Dn) < pv) Dn = Dn < 0.f ? -pv : pv;
-                y = fmaf(-l, y, z[i] * sc);
-                z[i] = y;
-                D[i] = Dn;
-                Dp = Dn;
-            }
-            // backward: x_i = y_i / D_i - (e_i / D_i) x_{i+1}
-            float x = __fdividef(z[N - 1], D[N - 1]);
-            z[N - 1] = x;
-            float mx = fabsf(x);
-            for (int i = N - 2; i >= 0; --i) {
-                x = __fdividef(fmaf(-eo[i], x, z[i]), D[i]);
-                z[i] = x;
-                mx = fmaxf(mx, fabsf(x));
-            }
-            // rescale by the largest entry first (no overflow in the norm), then normalise
-            const float im = mx > 0.f && isfinite(mx) ? 1.f / mx : 0.f;
-            nrm = 0.f;
-            for (int i = 0; i < N; ++i) {
-                const float v = z[i] * im;
-                z[i] = v;
-                nrm = fmaf(v, v, nrm);
-            }
-            if (!(nrm > 0.f) || !isfinite(nrm)) {
-                for (int i = 0; i < N; ++i) z[i] = start_entry(j + 977, i);     // restart from another vector
-                nrm = 0.f;
-                for (int i = 0; i < N; ++i) nrm = fmaf(z[i], z[i], nrm);
-                good = false;
-            }
-            sc = rsqrtf(nrm);
-        }
-        for (int i = 0; i < N; ++i) z[i] *= sc;
-    }
-    good = __syncthreads_and(good);
-    // ---- modified Gram-Schmidt, twice, in descending eigenvalue order. Vector j is
-    // final after step j - 1; warp w updates vectors j + 1 + w, j + 1 + w + nw, ...
-    for (int pass = 0; pass < 2; ++pass) {
+    // ---- block inverse iteration: every step solves (T - lam_j I) x_j = z_j for all j
+    // in parallel (one thread per eigenvalue, LDL^T recurrence; a pivot below eps,
+    // with |T| = 1, is set to +-eps, i.e. the shift moves by at most eps, which
+    // inverse iteration tolerates) and then orthonormalises the block by modified
+    // Gram-Schmidt in descending eigenvalue order. The orthonormalisation inside the
+    // iteration makes the vectors of eigenvalues closer than the bisection
+    // tolerance converge to different directions of their cluster instead of all to
+    // the same one.
+    // modified Gram-Schmidt over the block: vector j is final after step j - 1; warp w
+    // updates vectors j + 1 + w, j + 1 + w + nw, ...; a vector that vanishes is flagged
+    auto mgs = [&]() {
         for (int j = 0; j < rS; ++j) {
             const float* zj = Z + (size_t)j * ldz;
             if (j == 0 && wid == 0) {                  // vector 0 only needs normalising
                 float nn = 0.f;
                 for (int i = lane; i < N; i += 32) nn = fmaf(zj[i], zj[i], nn);
                 nn = warp_sum(nn);
-                const float r = nn > 0.f ? rsqrtf(nn) : 0.f;
+                const float r = nn > 1e-30f ? rsqrtf(nn) : 0.f;
+                if (r == 0.f && lane == 0) {
+                    *lost = 1;
+                    if (failures) atomicAdd(&failures[1], 1);
+                }
                 for (int i = lane; i < N; i += 32) Z[i] *= r;
             }
             __syncthreads();
@@ -427,13 +383,96 @@ SEKV_DEV bool top_eigvecs_tridiag(float* dg, float* eo, float* e2, int N, int rS
                 if (kv == j + 1) {                     // normalise the next vector here
                     nn = warp_sum(nn);
                     const float r = nn > 1e-30f ? rsqrtf(nn) : 0.f;
-                    if (r == 0.f && lane == 0) *lost = 1;      // dependent vectors: reported
+                    if (r == 0.f && lane == 0) {       // dependent vectors: reported
+                        *lost = 1;
+                        if (failures) atomicAdd(&failures[1], 1);
+                    }
                     for (int i = lane; i < N; i += 32) zk[i] *= r;
                 }
             }
         }
         __syncthreads();
+    };
+    bool good = true;
+    if (tid < rS) {
+        float* z = Z + (size_t)tid * ldz;
+        float nrm = 0.f;
+        for (int i = 0; i < N; ++i) {
+            z[i] = start_entry(tid, i);
+            nrm = fmaf(z[i], z[i], nrm);
+        }
+        const float r = rsqrtf(nrm);
+        for (int i = 0; i < N; ++i) z[i] *= r;
     }
+    __syncthreads();
+    for (int it = 0; it < kInvIters; ++it) {
+        if (tid < rS) {
+            const int j = tid;
+            float* z = Z + (size_t)j * ldz;
+            float* D = Dw + (size_t)j * ldz;
+            const float lj = lam[j];
+            const float pv = FLT_EPSILON;
+            // forward: D_i and y = L^{-1} (rs * z). The unpivoted elimination can grow
+            // by up to 1/eps per step; when |y| passes kBig, the partial solution and
+            // the multiplier of the remaining right-hand side are scaled down together,
+            // which scales the whole system and keeps it exact.
+            float rs = 1.f;
+            float Dp = dg[0] - lj;
+            if (fabsf(Dp) < pv) Dp = Dp < 0.f ? -pv : pv;
+            D[0] = Dp;
+            float y = z[0];
+            for (int i = 1; i < N; ++i) {
+                const float l = __fdividef(eo[i - 1], Dp);
+                float Dn = (dg[i] - lj) - l * eo[i - 1];
+                if (fabsf(Dn) < pv) Dn = Dn < 0.f ? -pv : pv;
+                y = fmaf(-l, y, z[i] * rs);
+                if (fabsf(y) > kBig) {
+                    for (int k = 0; k < i; ++k) z[k] *= kSmall;
+                    y *= kSmall;
+                    rs *= kSmall;
+                }
+                z[i] = y;
+                D[i] = Dn;
+                Dp = Dn;
+            }
+            // backward: x_i = (y_i - e_i x_{i+1}) / D_i, rescaled the same way (the
+            // x found so far and the y still to use)
+            float x = __fdividef(z[N - 1], D[N - 1]);
+            if (fabsf(x) > kBig) {
+                for (int k = 0; k < N - 1; ++k) z[k] *= kSmall;
+                x *= kSmall;
+            }
+            z[N - 1] = x;
+            float mx = fabsf(x);
+            for (int i = N - 2; i >= 0; --i) {
+                x = __fdividef(fmaf(-eo[i], x, z[i]), D[i]);
+                if (fabsf(x) > kBig) {
+                    for (int k = 0; k < N; ++k)
+                        if (k != i) z[k] *= kSmall;
+                    x *= kSmall;
+                    mx *= kSmall;
+                }
+                z[i] = x;
+                mx = fmaxf(mx, fabsf(x));
+            }
+            // scale by the largest entry (no overflow in the later norms)
+            const float im = mx > 0.f && isfinite(mx) ? 1.f / mx : 0.f;
+            bool finite = im > 0.f;
+            for (int i = 0; i < N; ++i) {
+                z[i] *= im;
+                finite = finite && isfinite(z[i]);
+            }
+            if (!finite) {
+                if (failures) atomicAdd(&failures[0], 1);
+                for (int i = 0; i < N; ++i) z[i] = start_entry(j + 977, i);     // restart from another vector
+                good = false;
+            }
+        }
+        __syncthreads();
+        mgs();
+    }
+    mgs();                                             // a second pass: orthogonal to rounding
+    good = __syncthreads_and(good);
     return good && *lost == 0;
 }
 
@@ -495,8 +534,31 @@ __host__ __device__ inline BasisSmem basis_smem_layout(int d, int rank) {
     return s;
 }
 
+// Stage rows [0, fill) of a row-padded copy of X in shared memory (row stride ldx
+// elements): rows < rows come from src (row stride d elements), the rest are zero.
+// bf16 rows move as 16-byte vectors (d and ldx are multiples of 8, rows of X are
+// 16-byte aligned); fp32 element by element.
+template <int DT>
+SEKV_DEV void stage_rows(void* dst, int ldx, const char* src, int d, int rows, int fill) {
+    const int tid = threadIdx.x, T = blockDim.x;
+    if constexpr (DT == SEKV_BF16) {
+        const int vpr = d / 8;                                       // 16-byte vectors per row
+        for (int i = tid; i < fill * vpr; i += T) {
+            const int r = i / vpr, c = (i % vpr) * 8;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (r < rows) v = *reinterpret_cast<const uint4*>(src + ((int64_t)r * d + c) * 2);
+            *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(dst) + (size_t)r * ldx + c) = v;
+        }
+    } else {
+        for (int i = tid; i < fill * d; i += T) {
+            const int r = i / d, c = i % d;
+            reinterpret_cast<float*>(dst)[(size_t)r * ldx + c] = r < rows ? load1<DT>(src, (int64_t)r * d + c) : 0.f;
+        }
+    }
+}
+
 template <int DT, int NB>
-__global__ void __launch_bounds__(BasisThreads<NB>::value)
+__global__ void __launch_bounds__(BasisThreads<NB>::value, NB >= 128 ? 2 : 4)
 basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
     using E = Elt<DT>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -518,12 +580,6 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
     float* pv = tk + NB;
     float* lam = pv + NB;
     float* red = lam + L.rsmax;                    // 64 + R * NB floats
-    auto xs = [&](int r, int c) -> float {
-        return (DT == SEKV_BF16) ? __bfloat162float(Xb[r * ldx + c]) : X[r * ldx + c];
-    };
-    auto xput = [&](int r, int c, float v) {
-        if (DT == SEKV_BF16) Xb[r * ldx + c] = __float2bfloat16_rn(v); else X[r * ldx + c] = v;
-    };
     __shared__ int item_s, lost_s;
 
     const int per_entry = a.Lr * a.Hkv * 2;
@@ -568,10 +624,7 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
         const int Mp = (N + 15) & ~15;              // padded for the MMA tiles
         for (int i = tid; i < Mp * ld; i += T) G[i] = 0.f;
         if (rows_form) {
-            for (int i = tid; i < Mp * d; i += T) {
-                const int r = i / d, c = i % d;
-                xput(r, c, r < len ? load1<DT>(src, (int64_t)r * d + c) : 0.f);
-            }
+            stage_rows<DT>(xa, ldx, src, d, len, Mp);
             __syncthreads();
             if (DT == SEKV_BF16) {
                 gram_rows_mma(G, ld, Xb, ldx, Mp, d, false);
@@ -587,10 +640,7 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
             __syncthreads();
             for (int t0 = 0; t0 < len; t0 += kChunkRows) {
                 const int rows = min(kChunkRows, len - t0);
-                for (int i = tid; i < kChunkRows * d; i += T) {
-                    const int r = i / d, c = i % d;
-                    xput(r, c, r < rows ? load1<DT>(src, (int64_t)(t0 + r) * d + c) : 0.f);
-                }
+                stage_rows<DT>(xa, ldx, src + (int64_t)t0 * d * E::bytes, d, rows, kChunkRows);
                 __syncthreads();
                 if (DT == SEKV_BF16) {
                     gram_cols_mma(G, ld, Xb, ldx, Mp, kChunkRows, true);
@@ -610,7 +660,7 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
         // ---- top-rS eigenvectors of G ------------------------------------------
         if (tid == 0) lost_s = 0;
         tridiagonalize(G, ld, N, dg, eo, tk, pv, red);
-        const bool good = top_eigvecs_tridiag(dg, eo, e2, N, rS, Z, ldz, Dw, lam, red, &lost_s);
+        const bool good = top_eigvecs_tridiag(dg, eo, e2, N, rS, Z, ldz, Dw, lam, red, &lost_s, w.failures);
         if (!good && tid == 0) set_status(a.status, SEKV_WARN_NOT_CONVERGED);
         back_transform(G, ld, tk, N, rS, Z, ldz);
 
@@ -620,9 +670,6 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
         float* Xf = G;
         auto xcs = [&](int r, int c) -> float {
             return (DT == SEKV_BF16) ? __bfloat162float(Xc[r * ldx + c]) : Xf[r * ldx + c];
-        };
-        auto xcput = [&](int r, int c, float v) {
-            if (DT == SEKV_BF16) Xc[r * ldx + c] = __float2bfloat16_rn(v); else Xf[r * ldx + c] = v;
         };
         if (rows_form) {
             // A[t][j] = U[t][j];  B[j][k] = sum_t U[t][j] X[t][k]
@@ -641,10 +688,7 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
                 for (int t0 = 0; t0 < len; t0 += kChunkRows) {
                     const int rows = min(kChunkRows, len - t0);
                     __syncthreads();
-                    for (int i = tid; i < rows * d; i += T) {
-                        const int r = i / d, c = i % d;
-                        xcput(r, c, load1<DT>(src, (int64_t)(t0 + r) * d + c));
-                    }
+                    stage_rows<DT>(G, ldx, src + (int64_t)t0 * d * E::bytes, d, rows, rows);
                     __syncthreads();
 #pragma unroll
                     for (int q = 0; q < kMaxOut; ++q) {
@@ -677,10 +721,7 @@ basis_kernel(BasisArgs a, BasisWork w, int bucket, size_t cap) {
             for (int t0 = 0; t0 < len; t0 += kChunkRows) {
                 const int rows = min(kChunkRows, len - t0);
                 __syncthreads();
-                for (int i = tid; i < rows * d; i += T) {
-                    const int r = i / d, c = i % d;
-                    xcput(r, c, load1<DT>(src, (int64_t)(t0 + r) * d + c));
-                }
+                stage_rows<DT>(G, ldx, src + (int64_t)t0 * d * E::bytes, d, rows, rows);
                 __syncthreads();
                 for (int i = tid; i < rows * rS; i += T) {
                     const int r = i / rS, j = i % rS;

@@ -42,7 +42,6 @@ namespace sekv {
 constexpr int kNW = 4;          // consumer warps per CTA
 constexpr unsigned kSpanModeSpans = 64;   // zoomed spans in a CTA for whole-span pieces
 constexpr int kRMax = 64;       // largest basis rank the decode accepts
-constexpr size_t kBalMaskBytes = 5632;   // largest unit mask (G x m_cap / 32 words) dealt by rank
 
 template <int DT, int D, int G>
 struct DecCfg {
@@ -67,8 +66,8 @@ struct DecCfg {
     static constexpr int ZSLOT = 4096;
     static constexpr int RB = ZSLOT / ROWB;                 // B / D rows per slot (a multiple of 8)
     static constexpr int ZBYTES = kNW * ZNS * ZSLOT;
-    // tensor-core zoom phase: one CTA-wide ring of ZNSC slots of ZSLOTC bytes, filled
-    // by the producer warp and read by all consumer warps
+    // tensor-core zoom phase: one CTA-wide ring of slots (ZRing below) filled by the
+    // producer warp and read by all consumer warps, sized here for the largest slot
     static constexpr int ZSLOTC = 16384;
     static constexpr int RBC = ZSLOTC / ROWB;               // B / D rows per piece (a multiple of 16)
     static constexpr int ZNSC0 = (NS * STAGE) / ZSLOTC;
@@ -81,6 +80,21 @@ struct DecCfg {
     static constexpr int RING1 = ZRING > SBYTES ? ZRING : SBYTES;
     static constexpr int RING = RING0 > RING1 ? RING0 : RING1;
     static constexpr int HDR = 1024;                        // mbarriers + counters (keeps stages 1 KB aligned)
+};
+
+// The tensor-core zoom ring in the stream stages' memory: 16 KB slots (measured on
+// B200 against 8 KB slots, which keep twice as many pieces in flight: the 128K
+// default workload's ATTEND call was ~3 % faster with 16 KB). The variant that hands
+// small spans whole to one warp needs a span's block in one slot as well.
+constexpr int kMaxZSlots = 16;   // zfull / zempty barriers and piece descriptors in the header
+template <class C, bool SP>
+struct ZRing {
+    static constexpr int SLOT = 16384;
+    static constexpr int RB = SLOT / C::ROWB;               // B / D rows per piece (a multiple of 16)
+    static constexpr int NS0 = C::RING0 / SLOT;
+    static constexpr int NS = NS0 > kMaxZSlots ? kMaxZSlots : NS0;
+    static_assert(NS * SLOT <= C::RING, "zoom ring exceeds the stage memory");
+    static_assert(RB % 16 == 0, "B / D pieces must hold whole 16-row blocks");
 };
 
 struct DecArgs {
@@ -108,9 +122,7 @@ struct DecArgs {
     float scale;
     int B, L, l0, Lr, Hq, Hkv, a_cap, m_cap, rank, phase, nsplit, sch_max, qcap, mw;
     int zin;          // zoom decisions come from zmask (a capped mask) instead of l > theta
-    int bal;          // zin and the unit's whole mask fits shared memory: zoomed spans are dealt
-                      // over the unit's splits by rank instead of staying with their own split
-    int zwords;       // zoom-mask words per head in shared memory (the split's range, or the unit's)
+    int zwords;       // zoom-mask words per head in shared memory (the split's span range)
     uint32_t polls;   // poll limit of every bounded barrier wait
     int starve;       // test hook: the producer issues no copy, so every wait runs out
 };
@@ -153,12 +165,18 @@ struct ZSpan {
 // the producer before it arms the slot's full barrier (a release), read by the
 // consumers after their wait on it (an acquire).
 // ZP_SPAN: a whole span's block [A | C | B | D] in one slot, handled by one warp.
-enum : int { ZP_B = 0, ZP_AC = 1, ZP_D = 2, ZP_END = 3, ZP_SPAN = 4 };
+// ZP_MIX: parts of one span packed into a slot, in order: the whole B (flag 1,
+// at offset 0), the A and C rows of tokens [r0, r0 + cnt) (each part reserved for
+// roundup(cnt, 32) tokens), the whole D (flag 2, reserved for roundup(r8, 16) rows).
+// ZP_B / ZP_D: chunks of B or D rows in slots of their own (for ranks whose B or D
+// takes more than half a slot).
+enum : int { ZP_B = 0, ZP_D = 2, ZP_END = 3, ZP_SPAN = 4, ZP_MIX = 5 };
+constexpr int kMixB = 1, kMixD = 2;
 struct __align__(16) ZPiece {
     int kind;
-    int first;           // first B (or D) piece of its span
-    int r0;              // B / D: first basis row; AC: first token (span-local, a multiple of 32)
-    int cnt;             // B / D: basis rows (a multiple of 8); AC: tokens
+    int first;           // B / D chunks: first chunk of its span; MIX: kMixB | kMixD flags
+    int r0;              // B / D: first basis row; MIX: first token (span-local, a multiple of 32)
+    int cnt;             // B / D: basis rows (a multiple of 8); MIX: tokens (may be 0)
     int len, rS;
     uint32_t hm;         // query heads of the group that zoom the span
     int rot;             // B / AC / D: the span's 32-token unit j belongs to consumer warp
@@ -572,12 +590,6 @@ SEKV_DEV void zoom_phase(const DecArgs& a, const DecSmem& sm, int warp, int lane
 // hi + lo bf16 pair (about 16 significant bits); p and beta*y are rounded to
 // bf16 as p on the stream path.
 // ---------------------------------------------------------------------------
-// tokens of an A/C piece: both halves fit ZSLOTC / 2, a multiple of 32, at most 256
-SEKV_DEV int zoom_piece_tokens(int r8, int zslot) {
-    int t = ((zslot / 2) / (r8 * 2)) & ~31;
-    return t > 256 ? 256 : t;
-}
-
 // split v0, v1 into a hi + lo bf16x2 pair
 SEKV_DEV void split_bf16x2(float v0, float v1, uint32_t& hi, uint32_t& lo) {
     hi = pack_bf16(v0, v1);
@@ -597,7 +609,8 @@ template <int D, int G, bool SP>
 SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b, int l, int kvh, int s0, int nwords,
                            int zwords) {
     using C = DecCfg<SEKV_BF16, D, G>;
-    constexpr int ZNS = C::ZNSC, ZSL = C::ZSLOTC, RBC = C::RBC;
+    using Z = ZRing<C, SP>;
+    constexpr int ZNS = Z::NS, ZSL = Z::SLOT, RBC = Z::RB;
     constexpr uint32_t FULL = 0xffffffffu;
     uint32_t np = 0;          // pieces armed
     bool good = true;
@@ -619,8 +632,10 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
     }
     // the slots were last read through the generic proxy (stream phase)
     fence_proxy_async();
-    // arm the next slot with piece pc and up to two bulk copies (lane 0 issues)
-    auto emit = [&](const ZPiece& pc, const char* src0, uint32_t n0, const char* src1, uint32_t n1) {
+    // arm the next slot with piece pc and up to four bulk copies (lane 0 issues):
+    // part k lands at byte offset off[k] of the slot
+    auto emit = [&](const ZPiece& pc, int nparts, const uint32_t (&off)[4], const char* const (&src)[4],
+                    const uint32_t (&bytes)[4]) {
         int okk = 1;
         if (lane == 0) {
             const int slot = (int)(np % ZNS);
@@ -628,12 +643,14 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
             if (okk) {
                 sm.zmeta[slot] = pc;
                 unsigned char* dst = sm.stages + (size_t)slot * ZSL;
-                if (n0 + n1 == 0) {
+                uint32_t tot = 0;
+                for (int k = 0; k < nparts; ++k) tot += bytes[k];
+                if (tot == 0) {
                     mbar_arrive(&sm.zfull[slot]);
                 } else {
-                    mbar_arrive_expect_tx(&sm.zfull[slot], n0 + n1);
-                    if (n0) bulk_g2s(dst, src0, n0, &sm.zfull[slot]);
-                    if (n1) bulk_g2s(dst + ZSL / 2, src1, n1, &sm.zfull[slot]);
+                    mbar_arrive_expect_tx(&sm.zfull[slot], tot);
+                    for (int k = 0; k < nparts; ++k)
+                        if (bytes[k]) bulk_g2s(dst + off[k], src[k], bytes[k], &sm.zfull[slot]);
                 }
             } else {
                 set_status(a.status, SEKV_ERR_TIMEOUT);
@@ -642,6 +659,11 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
         okk = __shfl_sync(FULL, okk, 0);
         if (okk) ++np;
         good = good && okk;
+    };
+    auto emit1 = [&](const ZPiece& pc, const char* src0, uint32_t n0) {
+        const uint32_t off[4] = {0u, 0u, 0u, 0u}, by[4] = {n0, 0u, 0u, 0u};
+        const char* const sr[4] = {src0, nullptr, nullptr, nullptr};
+        emit(pc, 1, off, sr, by);
     };
     for (int w0 = 0; w0 < nwords && good; w0 += 32) {
         // lane j takes word w0 + j: spans zoomed by any head, counted and scanned
@@ -697,7 +719,6 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
                 const int64_t pa = block_ac_elems(jl, rS);
                 const int64_t be = 2 * pa + 2 * (int64_t)r8 * D;
                 const char* blk = a.arena + ((int64_t)jo + (int64_t)kvh * be) * 2;
-                const int tcz = zoom_piece_tokens(r8, ZSL);
                 ZPiece pc;
                 pc.len = jl;
                 pc.rS = rS;
@@ -707,24 +728,52 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
                     // the whole block fits one slot (with room for the D projection's
                     // read of one 8-row block past D): one piece, one owner warp
                     pc.kind = ZP_SPAN; pc.first = 1; pc.r0 = 0; pc.cnt = jl;
-                    emit(pc, blk, (uint32_t)(be * 2), nullptr, 0u);
+                    emit1(pc, blk, (uint32_t)(be * 2));
                     rot = (rot + 1) & 3;
                     continue;
                 }
-                for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
-                    pc.kind = ZP_B; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
-                    emit(pc, blk + (2 * pa + (int64_t)r0 * D) * 2, (uint32_t)pc.cnt * C::ROWB, nullptr, 0u);
+                // B, then the A / C rows of the tokens, then D, packed into as few slots
+                // as they fit (B or D of more than half a slot travel in chunks of their
+                // own). Every part is reserved with the rows its fragment loads read:
+                // tokens up to a multiple of 32, basis rows up to a multiple of 16.
+                const uint32_t bsz = (uint32_t)r8 * D * 2;                 // bytes of B (and of D)
+                const uint32_t dres = (uint32_t)((r8 + 15) & ~15) * D * 2;
+                const uint32_t tokb = 4u * r8;                              // A + C bytes per token
+                const bool pack = bsz <= (uint32_t)ZSL / 2;
+                const char* srcB = blk + (2 * pa) * 2;
+                const char* srcD = blk + (2 * pa + (int64_t)r8 * D) * 2;
+                if (!pack) {
+                    for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
+                        pc.kind = ZP_B; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
+                        emit1(pc, srcB + (int64_t)r0 * D * 2, (uint32_t)pc.cnt * C::ROWB);
+                    }
                 }
-                for (int t0 = 0; t0 < jl && good; t0 += tcz) {
-                    pc.kind = ZP_AC; pc.first = t0 == 0; pc.r0 = t0; pc.cnt = min(tcz, jl - t0);
-                    const uint32_t nb = (uint32_t)round8(pc.cnt) * r8 * 2;
-                    const int64_t to = (int64_t)t0 * r8 * 2;
-                    emit(pc, blk + to, nb, blk + pa * 2 + to, nb);
+                bool with_b = pack;
+                for (int t0 = 0; t0 < jl && good;) {
+                    const uint32_t room = (uint32_t)ZSL - (with_b ? bsz : 0u);
+                    const int tmax = (int)(room / tokb) & ~31;
+                    const int cnt = min(tmax, jl - t0);
+                    const uint32_t res = (uint32_t)((cnt + 31) & ~31) * r8 * 2;   // bytes reserved for A (and C)
+                    const bool last = t0 + cnt >= jl;
+                    const bool with_d = pack && last && room >= 2 * res + dres;
+                    pc.kind = ZP_MIX; pc.first = (with_b ? kMixB : 0) | (with_d ? kMixD : 0); pc.r0 = t0; pc.cnt = cnt;
+                    const uint32_t oa = with_b ? bsz : 0u, ab = (uint32_t)round8(cnt) * r8 * 2;
+                    const uint32_t off[4] = {0u, oa, oa + res, oa + 2 * res};
+                    const char* const sr[4] = {srcB, blk + (int64_t)t0 * r8 * 2, blk + (pa + (int64_t)t0 * r8) * 2, srcD};
+                    const uint32_t by[4] = {with_b ? bsz : 0u, ab, ab, with_d ? bsz : 0u};
+                    emit(pc, 4, off, sr, by);
+                    t0 += cnt;
+                    with_b = false;
+                    if (last && pack && !with_d && good) {                 // D in a slot of its own
+                        pc.kind = ZP_MIX; pc.first = kMixD; pc.r0 = t0; pc.cnt = 0;
+                        emit1(pc, srcD, bsz);
+                    }
                 }
-                for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
-                    pc.kind = ZP_D; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
-                    emit(pc, blk + (2 * pa + (int64_t)r8 * D + (int64_t)r0 * D) * 2, (uint32_t)pc.cnt * C::ROWB,
-                         nullptr, 0u);
+                if (!pack) {
+                    for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
+                        pc.kind = ZP_D; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
+                        emit1(pc, srcD + (int64_t)r0 * D * 2, (uint32_t)pc.cnt * C::ROWB);
+                    }
                 }
                 rot = (rot + ((jl + 31) >> 5)) & 3;
             }
@@ -733,7 +782,7 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
     if (good) {
         ZPiece pc;
         pc.kind = ZP_END; pc.first = 0; pc.r0 = 0; pc.cnt = 0; pc.len = 0; pc.rS = 0; pc.hm = 0u; pc.rot = 0;
-        emit(pc, nullptr, 0u, nullptr, 0u);
+        emit1(pc, nullptr, 0u);
     }
     // every copy this warp started has landed before the CTA moves on (the full
     // barrier of a slot is re-armed only by this warp, so its last phase is stable)
@@ -751,7 +800,8 @@ template <int D, int G, int RM, bool SP>
 SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int lane, const uint32_t (&qb)[D / 16][2],
                            float (&mh)[2], float (&lh)[2], float (&oc)[D / 16][4]) {
     using C = DecCfg<SEKV_BF16, D, G>;
-    constexpr int ZNS = C::ZNSC, ZSL = C::ZSLOTC;
+    using Z = ZRing<C, SP>;
+    constexpr int ZNS = Z::NS, ZSL = Z::SLOT;
     constexpr int NKS = RM / 16;         // groups of 16 basis rows (m-tiles of u, y; k-steps of s, O)
     constexpr int DB = D / 8;            // column blocks of 8 in B / D rows
     constexpr uint32_t FULL = 0xffffffffu;
@@ -960,14 +1010,26 @@ SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int la
                 do_merge();
                 do_D(zs + 4 * pa + 2 * r8 * D, 0, r8);
             }
+        } else if (pc.kind == ZP_MIX) {
+            const int r8 = round8(pc.rS);
+            const int oa = (pc.first & kMixB) ? r8 * D * 2 : 0;
+            const int res = ((pc.cnt + 31) & ~31) * r8 * 2;
+            if (pc.first & kMixB) {
+                span_begin(pc);
+                mine = ((pc.len + 31) >> 5) > ((warp - pc.rot) & 3);
+                if (mine) do_u(zs, 0, r8);
+            }
+            if (mine && pc.cnt > 0) do_units(zs + oa, zs + oa + res, pc.cnt, (warp - pc.rot - (pc.r0 >> 5)) & 3, 4);
+            if (mine && (pc.first & kMixD)) {
+                do_merge();
+                do_D(zs + oa + 2 * res, 0, r8);
+            }
         } else if (pc.kind == ZP_B) {
             if (pc.first) {
                 span_begin(pc);
                 mine = ((pc.len + 31) >> 5) > ((warp - pc.rot) & 3);
             }
             if (mine) do_u(zs, pc.r0, pc.cnt);
-        } else if (pc.kind == ZP_AC) {
-            if (mine) do_units(zs, zs + ZSL / 2, pc.cnt, (warp - pc.rot - (pc.r0 >> 5)) & 3, 4);
         } else {  // ZP_D
             if (mine) {
                 if (pc.first) do_merge();
@@ -1092,7 +1154,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
             mbar_init(&sm.empty[s], kNW);
         }
         if constexpr (C::MMA) {
-            for (int s = 0; s < C::ZNSC; ++s) {
+            for (int s = 0; s < kMaxZSlots; ++s) {
                 mbar_init(&sm.zfull[s], 1);
                 mbar_init(&sm.zempty[s], kNW);
             }
@@ -1105,29 +1167,12 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         if (!a.starve)
             for (int i = 0; i < early; ++i) issue_tile(i);
     }
-    // zoom-mask words: zeros, or (balanced mode) the unit's whole mask as given, bits
-    // of spans >= m_count cleared
-    const int mw_used = (mb + 31) >> 5;
-    for (int i = tid; i < G * zwords; i += blockDim.x) {
-        const int h = i / zwords, w = i % zwords;
-        uint32_t v = 0u;
-        if (a.bal && w < mw_used) {
-            v = a.zmask[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.mw + w];
-            if (w == mw_used - 1 && (mb & 31)) v &= (1u << (mb & 31)) - 1u;
-        }
-        sm.zw[i] = v;
-    }
+    for (int i = tid; i < G * zwords; i += blockDim.x) sm.zw[i] = 0u;
     {
         const uint4* qg = reinterpret_cast<const uint4*>(a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB);
         for (int i = tid; i < G * C::ROWB / 16; i += blockDim.x) reinterpret_cast<uint4*>(sm.qs)[i] = qg[i];
     }
     __syncthreads();
-    // balanced mode: does the unit zoom any span at all (the same answer in every warp)
-    bool unit_zooms = false;
-    if (a.bal) {
-        for (int i = lane; i < G * mw_used; i += 32) unit_zooms = unit_zooms || sm.zw[(i / mw_used) * zwords + i % mw_used] != 0u;
-        unit_zooms = __any_sync(0xffffffffu, unit_zooms);
-    }
 
     const float sl2 = a.scale * kLog2e;
     bool ok = true;
@@ -1242,12 +1287,11 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                             const bool valid = rv && h < G;
                             const float x = sa[e] + sb[e];
                             const float ell = fmaf(x * inv, a.scale, ls);          // Eq. (5) pre-sigmoid
-                            const bool z = valid && (a.bal ? ((sm.zw[h * zwords + (SL >> 5)] >> (SL & 31)) & 1u)
-                                                     : a.zin ? zmask_bit(a, b, l, kvh * G + h, SL)
-                                                             : (ell > (hh ? th1 : th0)));   // Eq. (9)
+                            const bool z = valid && (a.zin ? zmask_bit(a, b, l, kvh * G + h, SL)
+                                                           : (ell > (hh ? th1 : th0)));   // Eq. (9)
                             if (valid && a.route_logits)
                                 a.route_logits[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.m_cap + SL] = ell;
-                            if (z && !a.bal) atomicOr(&sm.zw[h * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
+                            if (z) atomicOr(&sm.zw[h * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
                             lg[e] = (valid && !z) ? fmaf(x, a.scale, ls) * kLog2e : -INFINITY;
                         }
                     }
@@ -1412,54 +1456,14 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     __syncthreads();    // the stream is done: the stage ring is free, the zoom queues are complete
 
     if constexpr (C::MMA) {
-        if (a.bal) {
-            // The unit's zoomed spans (any head of the group) ranked in span order; this
-            // split takes ranks split, split + nsplit, ... wherever the spans sit, so
-            // every split of the unit gets an even share of the zoom work. Every split
-            // ranks the same mask, so each zoomed span is taken exactly once.
-            if (!route_only && unit_zooms && *sm.sfail == 0) {   // uniform over the CTA
-                if (warp == kNW) {
-                    int carry = 0;
-                    for (int w0 = 0; w0 < mw_used; w0 += 32) {
-                        const int w = w0 + lane;
-                        uint32_t u = 0u;
-                        if (w < mw_used) {
-#pragma unroll
-                            for (int h = 0; h < G; ++h) u |= sm.zw[h * zwords + w];
-                        }
-                        const int cnt = __popc(u);
-                        int inc = cnt;
-#pragma unroll
-                        for (int o = 1; o < 32; o <<= 1) {
-                            const int t = __shfl_up_sync(0xffffffffu, inc, o);
-                            if (lane >= o) inc += t;
-                        }
-                        const int first = carry + inc - cnt;          // rank of this word's first zoomed span
-                        uint32_t keep = 0u;
-                        for (int k = ((split - first) % a.nsplit + a.nsplit) % a.nsplit; k < cnt; k += a.nsplit)
-                            keep |= 1u << (__fns(u, 0u, k + 1));
-                        if (w < mw_used) {
-#pragma unroll
-                            for (int h = 0; h < G; ++h) sm.zw[h * zwords + w] &= keep;
-                        }
-                        carry += __shfl_sync(0xffffffffu, inc, 31);
-                    }
-                    __syncwarp();
-                    zoom_produce<D, G, SP>(a, sm, lane, b, l, kvh, 0, mw_used, zwords);
-                } else {
-                    zoom_consume<D, G, RM, SP>(a, sm, warp, lane, qb, mh, lh, oc);
-                }
-            }
-        } else {
-            // any zoomed span in this CTA's range (the same answer in every warp)
-            const int nwords = s1 > s0 ? (s1 - s0 + 31) >> 5 : 0;
-            bool zany = false;
-            for (int i = lane; i < G * zwords; i += 32) zany = zany || sm.zw[i] != 0u;
-            zany = __any_sync(0xffffffffu, zany);
-            if (!route_only && zany && *sm.sfail == 0) {     // uniform over the CTA
-                if (warp == kNW) zoom_produce<D, G, SP>(a, sm, lane, b, l, kvh, s0, nwords, zwords);
-                else zoom_consume<D, G, RM, SP>(a, sm, warp, lane, qb, mh, lh, oc);
-            }
+        // any zoomed span in this CTA's range (the same answer in every warp)
+        const int nwords = s1 > s0 ? (s1 - s0 + 31) >> 5 : 0;
+        bool zany = false;
+        for (int i = lane; i < G * zwords; i += 32) zany = zany || sm.zw[i] != 0u;
+        zany = __any_sync(0xffffffffu, zany);
+        if (!route_only && zany && *sm.sfail == 0) {     // uniform over the CTA
+            if (warp == kNW) zoom_produce<D, G, SP>(a, sm, lane, b, l, kvh, s0, nwords, zwords);
+            else zoom_consume<D, G, RM, SP>(a, sm, warp, lane, qb, mh, lh, oc);
         }
     } else {
         if (!route_only && warp < kNW && ok) zoom_phase<DT, D, G>(a, sm, warp, lane, b, l, kvh, m_run, l_run, o, m_lane);
@@ -1722,7 +1726,9 @@ DecodePlan plan_decode(const sekv_decode_desc& d) {
             // Makespan model over ns: the grid is units * ns CTAs of rows / ns rows
             // each plus a fixed cost (setup, partial write, merge; ~64 rows' worth),
             // scheduled dynamically onto the resident slots, plus half a CTA of tail.
-            const double rows = (double)d.rows_hint;
+            // A routing pass reads only the span rows' keys (about a quarter of the
+            // bytes of an anchor + span row pair), so it counts a quarter of the rows.
+            const double rows = d.phase == SEKV_ROUTE ? 0.25 * d.rows_hint : (double)d.rows_hint;
             const double o = 64.0;
             int best = 1;
             double best_t = 1e300;
@@ -1821,10 +1827,7 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     // test hook (sekv_decode_desc.test_flags bit 0): no copies and short waits
     a.starve = (d.test_flags & 1) ? 1 : 0;
     a.polls = a.starve ? 4096u : kWaitPolls;
-    // balanced zoom dealing needs the unit's whole mask in shared memory; it is used
-    // while that keeps three CTAs per SM (the mask words beside the ~70 KB ring)
-    a.bal = (C::MMA && zin && d.phase != SEKV_ROUTE && (size_t)G * a.mw * 4 <= kBalMaskBytes) ? 1 : 0;
-    a.zwords = a.bal ? a.mw : a.sch_max / 32;
+    a.zwords = a.sch_max / 32;
     const size_t smem = decode_smem_bytes<DT, D, G>(a.zwords, a.qcap);
     if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT, D, G, RM, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1950,9 +1953,7 @@ void* decode_static_scratch(cudaError_t* err) {
 // (capped) mask as input.
 cudaError_t launch_decode(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st) {
     const bool learned = d.route_W != nullptr;
-    // identity routing without a budget: FUSED and ROUTE route in the kernel; ATTEND
-    // takes the mask ROUTE wrote when the caller passes it (and routes again if not)
-    if (!learned && d.budget <= 0) return launch_pass(d, p, partials, st, d.phase == SEKV_ATTEND && d.zmask ? 1 : 0);
+    if (!learned && d.budget <= 0) return launch_pass(d, p, partials, st, 0);
     // the attention pass takes the (capped / learned) mask as input; with learned
     // routing it must not overwrite the routing logits with identity-form ones
     sekv_decode_desc att = d;

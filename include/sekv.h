@@ -6,7 +6,7 @@
  *
  *   prefill  sekv_build_spans   surprisal boundary scan -> anchors and spans,
  *                               anchor gather, per-span weighted-mean key/value,
- *                               per-span rank-r bases (Gram + Jacobi);
+ *                               per-span rank-r bases (Gram + top-r eigenpairs);
  *   decode   sekv_decode_attn   per-head routing over span summaries, zoom mask,
  *                               one softmax over anchors, summaries (+log|S|) and
  *                               low-rank reconstructed tokens of zoomed spans;
@@ -35,7 +35,7 @@
  *     returns SEKV_ERR_INVALID_ARG / SEKV_ERR_UNSUPPORTED and launches nothing.
  *     A CUDA launch error returns SEKV_ERR_CUDA (text: sekv_last_error()).
  *     Errors found on the device (capacity overflow, a cold span in ATTEND, a
- *     bounded wait that ran out, a Jacobi solve that did not converge) are
+ *     bounded wait that ran out, an eigenvector solve that failed) are
  *     written to *dev_status (device int32; first error wins; 0 = ok); kernels
  *     then skip the offending work and return, they never trap.
  *   - Work is enqueued on the given stream; calls do not synchronise unless
@@ -63,7 +63,7 @@ typedef enum {
     SEKV_ERR_COLD_SPAN = 4,     /* ATTEND met a zoomed span whose bases are cold */
     SEKV_ERR_TIMEOUT = 5,       /* a bounded device wait ran out                  */
     SEKV_ERR_UNSUPPORTED = 6,   /* shape outside the compiled variants            */
-    SEKV_WARN_NOT_CONVERGED = 7 /* a Jacobi solve hit max_sweeps (result kept)    */
+    SEKV_WARN_NOT_CONVERGED = 7 /* a basis eigenvector solve failed (result kept) */
 } sekv_status;
 
 enum { SEKV_F32 = 0, SEKV_BF16 = 1 };
@@ -87,11 +87,9 @@ enum {
 /* Decode phases. FUSED: routing + attention over a hot cache (one pass for the
  * identity routing form; with a budget or learned routing, a routing pass and then
  * attention with its mask). ROUTE: routing only (writes zmask / route_logits).
- * ATTEND: attention reading bases through the slot table; it takes zmask, as ROUTE
- * wrote it, as input (required with a budget or learned routing; in the identity
- * form without a budget a NULL zmask makes ATTEND route again, bit-identical to
- * ROUTE). With the mask as input the zoom work of each (b, l, kv head) is dealt
- * evenly over its CTAs. */
+ * ATTEND: attention reading bases through the slot table; it routes again
+ * (bit-identical to ROUTE) in the identity form without a budget, and otherwise
+ * takes zmask, as ROUTE wrote it, as input. */
 enum { SEKV_FUSED = 0, SEKV_ROUTE = 1, SEKV_ATTEND = 2 };
 
 typedef void* sekv_stream_t;   /* a cudaStream_t (NULL = legacy default stream) */
@@ -167,7 +165,7 @@ typedef struct sekv_build_desc {
     int32_t window;          /* the last `window` positions are anchors                    */
     int32_t wmode;           /* SEKV_W_*                                                    */
     int32_t rank;            /* basis rank r >= 1                                           */
-    int32_t max_sweeps;      /* Jacobi sweep limit (e.g. 15)                               */
+    int32_t max_sweeps;      /* >= 1; kept for compatibility (the solver's steps are fixed) */
     int32_t steps;           /* SEKV_BUILD_* mask                                           */
     int32_t Hq;              /* query heads (with route_W: a multiple of Hkv, Hq/Hkv <= 8)  */
     int32_t dr;              /* routing dimension d' (with route_W: 32 or 64)               */
@@ -175,7 +173,13 @@ typedef struct sekv_build_desc {
 } sekv_build_desc;
 
 size_t sekv_build_workspace_bytes(const sekv_build_desc* desc);
-/* Enqueue the requested build steps on `stream`. d must be 64 or 128. */
+/* Enqueue the requested build steps on `stream`. d must be 64 or 128. BASES solves,
+ * per span, key or value matrix X (|S| x d) and N = min(|S|, d), the symmetric
+ * eigenproblem of the N x N Gram matrix (X X^T or X^T X, tensor cores for bf16)
+ * for its top rS eigenpairs only: Householder tridiagonalisation, multisection on
+ * Sturm counts, 3 steps of block inverse iteration with Gram-Schmidt, then the
+ * reflectors' back-transformation (fp32). A solve that fails (a vector that vanishes
+ * or a non-finite solve, none expected) raises SEKV_WARN_NOT_CONVERGED. */
 sekv_status sekv_build_spans(const sekv_build_desc* desc, sekv_stream_t stream);
 
 /* ------------------------------------------------------------------------- */
@@ -202,8 +206,7 @@ typedef struct sekv_decode_desc {
     float* O;                /* [B][L][Hq][d] attention output (FUSED/ATTEND)              */
     float* lse;              /* [B][L][Hq] natural-log partition (FUSED/ATTEND)            */
     uint32_t* zmask;         /* optional [B][L][Hq][m_cap/32] zoom bits (bit S%32 of word   */
-                             /* S/32); required for ROUTE; input of ATTEND. Bits of spans  */
-                             /* >= m_count are 0 (ignored on input)                        */
+                             /* S/32); required for ROUTE. Bits of spans >= m_count are 0  */
     float* route_logits;     /* optional [B][L][Hq][m_cap] routing logits l_S              */
     /* learned-form routing (SeKV blog 2.3 Eq. (5)); optional. With route_W the routing
      * logit is l_S = (W^(l,h) q_h) . kbar_r_S / sqrt(dr) + logS_S, computed by a separate
@@ -309,35 +312,49 @@ typedef struct sekv_fetch_desc {
     void* arena;                  /* device arena, arena_elems elements                      */
     int64_t* slot_dev;            /* [B][L][m_cap] device slot table (written on `copy`)     */
     int64_t* slot_host;           /* pinned host mirror of the slot table                    */
-    int64_t* stats;               /* optional host [4]: bytes copied, spans copied, copies,
-                                     spans already resident (keep mode)                      */
-    int64_t* arena_used;          /* host, keep mode only: elements of the arena in use; the
-                                     caller sets it to 0 (and slot_host to -1) once            */
+    int64_t* stats;               /* optional host [5]: bytes copied, spans copied, copies,
+                                     spans already resident (keep mode), spans evicted       */
+    int64_t* arena_used;          /* optional host [1], written: arena elements holding bases
+                                     after the call                                          */
+    int64_t* last_use;            /* keep mode: host [B][L][m_cap], the step at which each
+                                     resident span was last needed; the caller sets it to -1
+                                     (and slot_host to -1) once, the library keeps it        */
+    sekv_event_t route_done;      /* optional (keep mode only): an event recorded right after
+                                     the ROUTE call that wrote zmask_dev. The routing result is
+                                     then read after this event on `copy`, so the caller may
+                                     have queued later work (the previous layer's ATTEND) on
+                                     `compute` and the copies overlap it. NULL: the result is
+                                     read on `compute` after all work queued there.          */
     int64_t region_elems;
     int64_t arena_elems;
+    int64_t step;                 /* keep mode: the caller's decode-step counter (>= 0, the
+                                     same for every layer range of one step, increasing)     */
     int32_t B, L, Hq, Hkv, d, dtype;
     int32_t l0, l1, m_cap, rank;
-    int32_t keep;                 /* 0: every call refills the arena (the zoomed spans of the
-                                     step only). 1: a device cache across calls: spans whose
-                                     slot (host mirror) is set stay resident and are not
-                                     copied again; misses are appended; when they do not fit,
-                                     the arena is flushed (every slot of [l0, l1) reset) and
-                                     refilled with this step's spans                         */
+    int32_t keep;                 /* 0: every call refills the arena with the zoomed spans of
+                                     [l0, l1) (each as one copy per rectangle of consecutive
+                                     spans x consecutive layers).
+                                     1: the arena is a device cache across calls: spans zoomed
+                                     again are not copied again. Misses are placed first-fit in
+                                     free space;
+                                     when none fits, spans are evicted least recently used
+                                     first, never one needed by this call or stamped with this
+                                     step or the previous one (ATTEND calls of those steps may
+                                     still be reading it; the caller must have finished every
+                                     ATTEND of older steps).                                 */
     int32_t reserved;
 } sekv_fetch_desc;
 
 /* Copy the bases of every span that any query head of (b, l) zooms, for layers
- * [l0, l1), into the arena, and point the slot table at them (-1 elsewhere; in
- * keep mode resident spans keep their slots).
- * Order: zmask is read back on `compute` (the host waits for it); the copies
- * and the slot-table upload go on `copy`; `done` is recorded on `copy`. The
- * caller makes `compute` wait on `done` before ATTEND. A run of consecutive
- * spans zoomed in the same layers is one rectangle of the home (its blocks sit
- * at the same offset of every layer's region); each rectangle is one
- * cudaMemcpy2DAsync (cudaMemcpyAsync for a single layer, or per layer when the
- * region pitch exceeds the device's maximum copy pitch). stats[2] counts the
- * copies. Arena contents from earlier calls are overwritten. Returns
- * SEKV_ERR_CAPACITY (nothing copied) if the zoomed bases exceed arena_elems. */
+ * [l0, l1), into the arena, and point the slot table at them (refill mode: -1
+ * elsewhere in [l0, l1); keep mode: resident spans keep their slots, evicted ones
+ * get -1). The routing result is read back first (see route_done; the host waits
+ * for it); the copies and the slot-table upload go on `copy`; `done` is recorded on
+ * `copy`. The caller makes `compute` wait on `done` before ATTEND. stats[2] counts
+ * the copies (cudaMemcpyAsync, or cudaMemcpy2DAsync for a rectangle). Returns
+ * SEKV_ERR_CAPACITY, with nothing copied and both slot tables as they were, when
+ * the zoomed bases that are not resident do not fit (keep mode: after every
+ * allowed eviction). */
 sekv_status sekv_fetch_bases(const sekv_fetch_desc* desc, sekv_stream_t compute,
                              sekv_stream_t copy, sekv_event_t done);
 

@@ -117,7 +117,7 @@ def test_decode_all_zoom_matches_oracle(name, over):
 
 @pytest.mark.parametrize("name,over", [("c1", dict()), ("c2", dict(n=4096, L=2)), ("c5", dict(n=2048, L=1))])
 def test_decode_end_to_end(name, over):
-    """library build (scan, summaries, Jacobi bases) + decode vs oracle build + decode"""
+    """library build (scan, summaries, bases) + decode vs oracle build + decode"""
     wl = WORKLOADS[name].scaled(**over)
     H, K, V, segs, units, q, theta, scale = _setup(wl)
     c = _cache(wl)
