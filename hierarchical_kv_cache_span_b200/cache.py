@@ -81,6 +81,7 @@ class SpanCache:
         self.kbar_r = None       # routing summaries [B][L][Hq][m_cap][dr]
         self.dr = 0
         self._zscratch = None
+        self._arrive = None             # arrival counters of the in-kernel split merge
 
     def set_routing(self, W: Optional[torch.Tensor]):
         """Learned-form routing (SeKV blog 2.2 Eq. (3), 2.3 Eq. (5)): W [L][Hq][dr][d] in
@@ -201,6 +202,11 @@ class SpanCache:
                 self._dws[key] = ws
             workspace = ws
         d.workspace, d.workspace_bytes = _ptr(workspace), workspace.numel()
+        if phase != S.SEKV_ROUTE:
+            # arrival counters: the last CTA of each (b, l, kv head) merges the splits
+            if self._arrive is None:
+                self._arrive = torch.zeros(self.B * self.L * self.Hkv, dtype=torch.int32, device=self.device)
+            d.arrive = _ptr(self._arrive)
         return d
 
     def new_outputs(self, l0=0, l1=None):

@@ -42,6 +42,7 @@ namespace sekv {
 constexpr int kNW = 4;          // consumer warps per CTA
 constexpr unsigned kSpanModeSpans = 64;   // zoomed spans in a CTA for whole-span pieces
 constexpr int kRMax = 64;       // largest basis rank the decode accepts
+constexpr size_t kDealMaskBytes = 5632;   // largest unit mask + unit table ((G + 1) x m_cap / 32 words) for dealing
 
 template <int DT, int D, int G>
 struct DecCfg {
@@ -122,9 +123,14 @@ struct DecArgs {
     float scale;
     int B, L, l0, Lr, Hq, Hkv, a_cap, m_cap, rank, phase, nsplit, sch_max, qcap, mw;
     int zin;          // zoom decisions come from zmask (a capped mask) instead of l > theta
+    int deal;         // zin, tensor-core path: the unit's whole mask is in shared memory and
+                      // every split takes an even share of the unit's zoomed token units
     int zwords;       // zoom-mask words per head in shared memory (the split's span range)
     uint32_t polls;   // poll limit of every bounded barrier wait
     int starve;       // test hook: the producer issues no copy, so every wait runs out
+    uint32_t* arrive; // [B][L][Hkv] arrival counters (the last CTA of a unit merges), or null
+    float* O;         // [B][L][Hq][D] and [B][L][Hq]: written by the merging CTA
+    float* lse;
 };
 
 // zoom bit of span S for query head hq of (b, l) in a caller-supplied (capped) mask
@@ -140,12 +146,13 @@ struct DecMaps {
 };
 
 template <int DT, int D, int G>
-static size_t decode_smem_bytes(int zwords, int qcap) {
+static size_t decode_smem_bytes(int zwords, int qcap, int deal) {
     using C = DecCfg<DT, D, G>;
     size_t s = C::HDR;
     s += (size_t)C::RING;
     s += (size_t)kNW * qcap * 4;                               // zoom queues
     s += (size_t)G * zwords * 4;                               // zoom-mask words
+    s += deal ? (size_t)zwords * 4 : 0;                        // zoomed token units per word
     s += (size_t)kNW * C::WSCR * 4;                            // per-warp scratch
     s = round_up(s, 16) + (size_t)G * C::ROWB;                 // the group's query rows
     return round_up(s, 128) + 1024;                            // + alignment slack
@@ -193,10 +200,12 @@ struct DecSmem {
     int* qcnt;           // [kNW]
     int* zq_next;
     int* sfail;          // set when any warp gave up during the stream phase
+    int* last;           // this CTA is the unit's last to finish (it merges the splits)
     ZPiece* zmeta;       // tensor-core zoom: [ZNSC]
     unsigned char* stages;
     int* zq;             // [kNW][qcap]
     uint32_t* zw;        // [G][zwords]
+    int* zu;             // deal: [zwords] zoomed 32-token units of the spans of each mask word
     float* wscr;         // [kNW][WSCR]
     unsigned char* qs;   // [G][D] query rows of the kv head's group (storage dtype)
     float* st_m;         // [NSTATE][G]   (in the ring, once the zoom phase is over)
@@ -208,7 +217,7 @@ struct DecSmem {
 // counters @384, zmeta @512 (tensor-core path; the fp32 path keeps its per-warp
 // p tiles there)
 template <class C, int G, int D>
-SEKV_DEV DecSmem carve_smem(unsigned char* base, int qcap, int zwords) {
+SEKV_DEV DecSmem carve_smem(unsigned char* base, int qcap, int zwords, int deal) {
     DecSmem s;
     s.full = reinterpret_cast<uint64_t*>(base);
     s.empty = s.full + 8;
@@ -218,11 +227,13 @@ SEKV_DEV DecSmem carve_smem(unsigned char* base, int qcap, int zwords) {
     s.qcnt = reinterpret_cast<int*>(base + 384);
     s.zq_next = s.qcnt + kNW;
     s.sfail = s.zq_next + 1;
+    s.last = s.sfail + 1;
     s.zmeta = reinterpret_cast<ZPiece*>(base + 512);
     s.stages = base + C::HDR;
     s.zq = reinterpret_cast<int*>(s.stages + C::RING);
     s.zw = reinterpret_cast<uint32_t*>(s.zq + kNW * qcap);
-    s.wscr = reinterpret_cast<float*>(s.zw + G * zwords);
+    s.zu = reinterpret_cast<int*>(s.zw + G * zwords);
+    s.wscr = reinterpret_cast<float*>(s.zu + (deal ? zwords : 0));
     s.qs = reinterpret_cast<unsigned char*>(
         round_up(reinterpret_cast<uintptr_t>(s.wscr + kNW * C::WSCR), 16));
     s.st_m = reinterpret_cast<float*>(s.stages);             // written after the zoom phase
@@ -603,11 +614,16 @@ SEKV_DEV float ex2(float x) {
     return y;
 }
 
-// zoomed spans of the CTA: word w of zw[h] holds heads h's bits for spans
-// s0 + 32 w .. s0 + 32 w + 31; nwords words are in use
+// zoomed spans of the CTA: word w of zw[h] holds head h's bits for spans
+// s0 + 32 w .. s0 + 32 w + 31; nwords words are in use. With a.deal the words are
+// the unit's (s0 = 0) and this split takes an even share of the unit's zoomed
+// 32-token units: the zoomed spans (any head of the group) in span order, span S
+// contributing ceil(|S| / 32) units, split j the units [U j / nsplit, U (j + 1) / nsplit).
+// A span cut between splits is attended in parts (each part its own u = B q and
+// D projection): the parts are disjoint subsets of the one softmax's entries.
 template <int D, int G, bool SP>
 SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b, int l, int kvh, int s0, int nwords,
-                           int zwords) {
+                           int zwords, int split) {
     using C = DecCfg<SEKV_BF16, D, G>;
     using Z = ZRing<C, SP>;
     constexpr int ZNS = Z::NS, ZSL = Z::SLOT, RBC = Z::RB;
@@ -620,7 +636,7 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
     // with different spans; with few, sharing each span's units across the warps
     // keeps the critical path shorter.
     bool span_mode = false;
-    if (SP) {
+    if (SP && !a.deal) {
         unsigned nz = 0;
         for (int w = lane; w < nwords; w += 32) {
             uint32_t m = 0u;
@@ -665,118 +681,203 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
         const char* const sr[4] = {src0, nullptr, nullptr, nullptr};
         emit(pc, 1, off, sr, by);
     };
-    for (int w0 = 0; w0 < nwords && good; w0 += 32) {
-        // lane j takes word w0 + j: spans zoomed by any head, counted and scanned
-        const int wi = w0 + lane;
-        uint32_t m = 0u;
-        if (wi < nwords) {
-#pragma unroll
-            for (int h = 0; h < G; ++h) m |= sm.zw[h * zwords + wi];
+    // the pieces of tokens [tb, te) of a zoomed span of jl tokens whose Hkv blocks start
+    // at element jo of the arena (tb a multiple of 32; the whole span: 0, jl)
+    auto emit_span = [&](int jl, uint32_t jhm, long long jo, int tb, int te) {
+        const int rS = block_rank(jl, D, a.rank), r8 = round8(rS);
+        const int64_t pa = block_ac_elems(jl, rS);
+        const int64_t be = 2 * pa + 2 * (int64_t)r8 * D;
+        const char* blk = a.arena + ((int64_t)jo + (int64_t)kvh * be) * 2;
+        ZPiece pc;
+        pc.len = te - tb;
+        pc.rS = rS;
+        pc.hm = jhm;
+        pc.rot = rot;
+        if (span_mode && tb == 0 && te == jl && be * 2 + D * 16 <= ZSL) {
+            // the whole block fits one slot (with room for the D projection's
+            // read of one 8-row block past D): one piece, one owner warp
+            pc.kind = ZP_SPAN; pc.first = 1; pc.r0 = 0; pc.cnt = jl;
+            emit1(pc, blk, (uint32_t)(be * 2));
+            rot = (rot + 1) & 3;
+            return;
         }
-        const int cnt = __popc(m);
-        int inc = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(FULL, inc, o);
-            if (lane >= o) inc += t;
-        }
-        const int total = __shfl_sync(FULL, inc, 31);
-        for (int e0 = 0; e0 < total && good; e0 += 32) {
-            // lane j resolves entry e0 + j: its word, bit, heads and block offset
-            const int e = e0 + lane;
-            int k = 0;
-            for (int j = 0; j < 32; ++j) k += (__shfl_sync(FULL, inc, j) <= e) ? 1 : 0;
-            const int kw = k < 32 ? k : 31;
-            const int inck = __shfl_sync(FULL, inc, kw), cntk = __shfl_sync(FULL, cnt, kw);
-            const uint32_t mk = __shfl_sync(FULL, m, kw);
-            int len = 0;
-            uint32_t hm = 0u;
-            long long off = -1;
-            if (e < total) {
-                const int bit = (int)__fns(mk, 0u, e - (inck - cntk) + 1);
-                const int S = s0 + (w0 + kw) * 32 + bit;
-#pragma unroll
-                for (int h = 0; h < G; ++h) hm |= ((sm.zw[h * zwords + w0 + kw] >> bit) & 1u) << h;
-                const int beg = a.span_beg[(int64_t)b * a.m_cap + S];
-                len = a.span_end[(int64_t)b * a.m_cap + S] - beg;
-                if (len < 1) {
-                    set_status(a.status, SEKV_ERR_INVALID_ARG);
-                    len = 0;
-                } else if (a.slot) {
-                    off = a.slot[((int64_t)b * a.L + l) * a.m_cap + S];
-                    if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
-                } else {
-                    off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S];
-                }
+        // B, then the A / C rows of the tokens, then D, packed into as few slots
+        // as they fit (B or D of more than half a slot travel in chunks of their
+        // own). Every part is reserved with the rows its fragment loads read:
+        // tokens up to a multiple of 32, basis rows up to a multiple of 16.
+        const uint32_t bsz = (uint32_t)r8 * D * 2;                 // bytes of B (and of D)
+        const uint32_t dres = (uint32_t)((r8 + 15) & ~15) * D * 2;
+        const uint32_t tokb = 4u * r8;                              // A + C bytes per token
+        const bool pack = bsz <= (uint32_t)ZSL / 2;
+        const char* srcB = blk + (2 * pa) * 2;
+        const char* srcD = blk + (2 * pa + (int64_t)r8 * D) * 2;
+        if (!pack) {
+            for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
+                pc.kind = ZP_B; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
+                emit1(pc, srcB + (int64_t)r0 * D * 2, (uint32_t)pc.cnt * C::ROWB);
             }
-            const int cntb = min(32, total - e0);
-            for (int j = 0; j < cntb && good; ++j) {
+        }
+        bool with_b = pack;
+        for (int t0 = tb; t0 < te && good;) {
+            const uint32_t room = (uint32_t)ZSL - (with_b ? bsz : 0u);
+            const int tmax = (int)(room / tokb) & ~31;
+            const int cnt = min(tmax, te - t0);
+            const uint32_t res = (uint32_t)((cnt + 31) & ~31) * r8 * 2;   // bytes reserved for A (and C)
+            const bool last = t0 + cnt >= te;
+            const bool with_d = pack && last && room >= 2 * res + dres;
+            pc.kind = ZP_MIX; pc.first = (with_b ? kMixB : 0) | (with_d ? kMixD : 0); pc.r0 = t0 - tb; pc.cnt = cnt;
+            const uint32_t oa = with_b ? bsz : 0u, ab = (uint32_t)round8(cnt) * r8 * 2;
+            const uint32_t off[4] = {0u, oa, oa + res, oa + 2 * res};
+            const char* const sr[4] = {srcB, blk + (int64_t)t0 * r8 * 2, blk + (pa + (int64_t)t0 * r8) * 2, srcD};
+            const uint32_t by[4] = {with_b ? bsz : 0u, ab, ab, with_d ? bsz : 0u};
+            emit(pc, 4, off, sr, by);
+            t0 += cnt;
+            with_b = false;
+            if (last && pack && !with_d && good) {                 // D in a slot of its own
+                pc.kind = ZP_MIX; pc.first = kMixD; pc.r0 = t0 - tb; pc.cnt = 0;
+                emit1(pc, srcD, bsz);
+            }
+        }
+        if (!pack) {
+            for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
+                pc.kind = ZP_D; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
+                emit1(pc, srcD + (int64_t)r0 * D * 2, (uint32_t)pc.cnt * C::ROWB);
+            }
+        }
+        rot = (rot + ((te - tb + 31) >> 5)) & 3;
+    };
+    // Walk the zoomed spans (any head of the group) in span order, up to 32 at a time:
+    // visit(len, hm, off, n) gets this lane's span of the batch (len 0: none or
+    // invalid; off < 0: cold) and the batch size n (warp-uniform); it returns false
+    // to stop the walk.
+    auto walk = [&](auto&& visit) {
+        for (int w0 = 0; w0 < nwords && good; w0 += 32) {
+            // lane j takes word w0 + j: spans zoomed by any head, counted and scanned
+            const int wi = w0 + lane;
+            uint32_t m = 0u;
+            if (wi < nwords) {
+#pragma unroll
+                for (int h = 0; h < G; ++h) m |= sm.zw[h * zwords + wi];
+            }
+            const int cnt = __popc(m);
+            int inc = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(FULL, inc, o);
+                if (lane >= o) inc += t;
+            }
+            const int total = __shfl_sync(FULL, inc, 31);
+            for (int e0 = 0; e0 < total && good; e0 += 32) {
+                // lane j resolves entry e0 + j: its word, bit, heads and block offset
+                const int e = e0 + lane;
+                int k = 0;
+                for (int j = 0; j < 32; ++j) k += (__shfl_sync(FULL, inc, j) <= e) ? 1 : 0;
+                const int kw = k < 32 ? k : 31;
+                const int inck = __shfl_sync(FULL, inc, kw), cntk = __shfl_sync(FULL, cnt, kw);
+                const uint32_t mk = __shfl_sync(FULL, m, kw);
+                int len = 0;
+                uint32_t hm = 0u;
+                long long off = -1;
+                if (e < total) {
+                    const int bit = (int)__fns(mk, 0u, e - (inck - cntk) + 1);
+                    const int S = s0 + (w0 + kw) * 32 + bit;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) hm |= ((sm.zw[h * zwords + w0 + kw] >> bit) & 1u) << h;
+                    const int beg = a.span_beg[(int64_t)b * a.m_cap + S];
+                    len = a.span_end[(int64_t)b * a.m_cap + S] - beg;
+                    if (len < 1) {
+                        set_status(a.status, SEKV_ERR_INVALID_ARG);
+                        len = 0;
+                    } else if (a.slot) {
+                        off = a.slot[((int64_t)b * a.L + l) * a.m_cap + S];
+                        if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
+                    } else {
+                        off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S];
+                    }
+                }
+                if (!visit(len, hm, off, min(32, total - e0))) return;
+            }
+        }
+    };
+    if (!a.deal) {
+        walk([&](int len, uint32_t hm, long long off, int n) {
+            for (int j = 0; j < n && good; ++j) {
                 const int jl = __shfl_sync(FULL, len, j);
                 const uint32_t jhm = __shfl_sync(FULL, hm, j);
                 const long long jo = __shfl_sync(FULL, off, j);
-                if (jl < 1 || jo < 0) continue;
-                const int rS = block_rank(jl, D, a.rank), r8 = round8(rS);
-                const int64_t pa = block_ac_elems(jl, rS);
-                const int64_t be = 2 * pa + 2 * (int64_t)r8 * D;
-                const char* blk = a.arena + ((int64_t)jo + (int64_t)kvh * be) * 2;
-                ZPiece pc;
-                pc.len = jl;
-                pc.rS = rS;
-                pc.hm = jhm;
-                pc.rot = rot;
-                if (span_mode && be * 2 + D * 16 <= ZSL) {
-                    // the whole block fits one slot (with room for the D projection's
-                    // read of one 8-row block past D): one piece, one owner warp
-                    pc.kind = ZP_SPAN; pc.first = 1; pc.r0 = 0; pc.cnt = jl;
-                    emit1(pc, blk, (uint32_t)(be * 2));
-                    rot = (rot + 1) & 3;
-                    continue;
-                }
-                // B, then the A / C rows of the tokens, then D, packed into as few slots
-                // as they fit (B or D of more than half a slot travel in chunks of their
-                // own). Every part is reserved with the rows its fragment loads read:
-                // tokens up to a multiple of 32, basis rows up to a multiple of 16.
-                const uint32_t bsz = (uint32_t)r8 * D * 2;                 // bytes of B (and of D)
-                const uint32_t dres = (uint32_t)((r8 + 15) & ~15) * D * 2;
-                const uint32_t tokb = 4u * r8;                              // A + C bytes per token
-                const bool pack = bsz <= (uint32_t)ZSL / 2;
-                const char* srcB = blk + (2 * pa) * 2;
-                const char* srcD = blk + (2 * pa + (int64_t)r8 * D) * 2;
-                if (!pack) {
-                    for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
-                        pc.kind = ZP_B; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
-                        emit1(pc, srcB + (int64_t)r0 * D * 2, (uint32_t)pc.cnt * C::ROWB);
-                    }
-                }
-                bool with_b = pack;
-                for (int t0 = 0; t0 < jl && good;) {
-                    const uint32_t room = (uint32_t)ZSL - (with_b ? bsz : 0u);
-                    const int tmax = (int)(room / tokb) & ~31;
-                    const int cnt = min(tmax, jl - t0);
-                    const uint32_t res = (uint32_t)((cnt + 31) & ~31) * r8 * 2;   // bytes reserved for A (and C)
-                    const bool last = t0 + cnt >= jl;
-                    const bool with_d = pack && last && room >= 2 * res + dres;
-                    pc.kind = ZP_MIX; pc.first = (with_b ? kMixB : 0) | (with_d ? kMixD : 0); pc.r0 = t0; pc.cnt = cnt;
-                    const uint32_t oa = with_b ? bsz : 0u, ab = (uint32_t)round8(cnt) * r8 * 2;
-                    const uint32_t off[4] = {0u, oa, oa + res, oa + 2 * res};
-                    const char* const sr[4] = {srcB, blk + (int64_t)t0 * r8 * 2, blk + (pa + (int64_t)t0 * r8) * 2, srcD};
-                    const uint32_t by[4] = {with_b ? bsz : 0u, ab, ab, with_d ? bsz : 0u};
-                    emit(pc, 4, off, sr, by);
-                    t0 += cnt;
-                    with_b = false;
-                    if (last && pack && !with_d && good) {                 // D in a slot of its own
-                        pc.kind = ZP_MIX; pc.first = kMixD; pc.r0 = t0; pc.cnt = 0;
-                        emit1(pc, srcD, bsz);
-                    }
-                }
-                if (!pack) {
-                    for (int r0 = 0; r0 < r8 && good; r0 += RBC) {
-                        pc.kind = ZP_D; pc.first = r0 == 0; pc.r0 = r0; pc.cnt = min(RBC, r8 - r0);
-                        emit1(pc, srcD + (int64_t)r0 * D * 2, (uint32_t)pc.cnt * C::ROWB);
-                    }
-                }
-                rot = (rot + ((jl + 31) >> 5)) & 3;
+                if (jl >= 1 && jo >= 0) emit_span(jl, jhm, jo, 0, jl);
             }
+            return true;
+        });
+    } else {
+        // the unit's zoomed token units (the per-word table), this split's share of
+        // them, and the words that hold it
+        unsigned tot = 0;
+        for (int w = lane; w < nwords; w += 32) tot += (unsigned)sm.zu[w];
+        const long long U = (long long)warp_sum_u(tot);
+        const long long lo = U * split / a.nsplit, hi = U * (split + 1) / a.nsplit;
+        long long base = 0;               // units of the words before the batch
+        for (int w0 = 0; w0 < nwords && good && base < hi; w0 += 32) {
+            const int w = w0 + lane;
+            const int u = w < nwords ? sm.zu[w] : 0;
+            int inc = u;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(FULL, inc, o);
+                if (lane >= o) inc += t;
+            }
+            const long long cw = base + inc - u;          // units before word w
+            uint32_t hits = __ballot_sync(FULL, u > 0 && cw < hi && cw + u > lo);
+            while (hits && good) {
+                const int k = __ffs(hits) - 1;
+                hits &= hits - 1u;
+                const int wk = w0 + k;
+                const long long cu = base + __shfl_sync(FULL, inc - u, k);
+                uint32_t m = 0u;
+#pragma unroll
+                for (int h = 0; h < G; ++h) m |= sm.zw[h * zwords + wk];
+                // lane j resolves the word's j-th zoomed span
+                const int cnt = __popc(m);
+                int len = 0;
+                uint32_t hm = 0u;
+                long long off = -1;
+                if (lane < cnt) {
+                    const int bit = (int)__fns(m, 0u, lane + 1);
+                    const int S = s0 + wk * 32 + bit;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) hm |= ((sm.zw[h * zwords + wk] >> bit) & 1u) << h;
+                    len = a.span_end[(int64_t)b * a.m_cap + S] - a.span_beg[(int64_t)b * a.m_cap + S];
+                    if (len < 1) {
+                        set_status(a.status, SEKV_ERR_INVALID_ARG);
+                        len = 0;
+                    } else if (a.slot) {
+                        off = a.slot[((int64_t)b * a.L + l) * a.m_cap + S];
+                        if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
+                    } else {
+                        off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S];
+                    }
+                }
+                const int nu = len >= 1 ? (len + 31) >> 5 : 0;
+                int ex = nu;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(FULL, ex, o);
+                    if (lane >= o) ex += t;
+                }
+                ex -= nu;
+                for (int j = 0; j < cnt && good; ++j) {
+                    const long long jc = cu + __shfl_sync(FULL, ex, j);
+                    if (jc >= hi) break;
+                    const int jl = __shfl_sync(FULL, len, j);
+                    const int jn = __shfl_sync(FULL, nu, j);
+                    const uint32_t jhm = __shfl_sync(FULL, hm, j);
+                    const long long jo = __shfl_sync(FULL, off, j);
+                    const long long u0 = lo > jc ? lo - jc : 0, u1 = hi - jc < jn ? hi - jc : jn;
+                    if (jl >= 1 && jo >= 0 && u0 < u1)
+                        emit_span(jl, jhm, jo, (int)(32 * u0), (int)min((long long)jl, 32 * u1));
+                }
+            }
+            base += __shfl_sync(FULL, inc, 31);
         }
     }
     if (good) {
@@ -791,6 +892,58 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
         for (uint32_t i = lo; i < np; ++i)
             if (!mbar_wait_n(&sm.zfull[i % ZNS], (i / ZNS) & 1, a.polls)) set_status(a.status, SEKV_ERR_TIMEOUT);
     }
+}
+
+// The table the zoom producer deals from (deal mode; producer warp): zu[w] = the
+// zoomed 32-token units of the spans of mask word w (spans zoomed by any head of
+// the group). The zoomed spans are gathered 32 at a time across words, so the span
+// lengths cost one round of loads per 32 zoomed spans.
+template <int G>
+SEKV_DEV void deal_table(const DecArgs& a, const DecSmem& sm, int lane, int b, int mb, int zwords) {
+    constexpr uint32_t FULL = 0xffffffffu;
+    const int nwords = (mb + 31) >> 5;
+    int pend = -1;           // this lane's gathered span
+    int p = 0;               // lanes [0, p) hold gathered spans
+    auto flush = [&]() {
+        if (lane < p) {
+            const int len = a.span_end[(int64_t)b * a.m_cap + pend] - a.span_beg[(int64_t)b * a.m_cap + pend];
+            if (len >= 1) atomicAdd(&sm.zu[pend >> 5], (len + 31) >> 5);
+        }
+        p = 0;
+    };
+    for (int w0 = 0; w0 < nwords; w0 += 32) {
+        const int wi = w0 + lane;
+        uint32_t m = 0u;
+        if (wi < nwords) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) m |= sm.zw[h * zwords + wi];
+        }
+        const int cnt = __popc(m);
+        int inc = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(FULL, inc, o);
+            if (lane >= o) inc += t;
+        }
+        const int total = __shfl_sync(FULL, inc, 31);
+        for (int done = 0; done < total;) {
+            const int take = min(32 - p, total - done);
+            // lane p + i takes the batch's entry done + i
+            const int e = done + lane - p;
+            int k = 0;
+            for (int j = 0; j < 32; ++j) k += (__shfl_sync(FULL, inc, j) <= e) ? 1 : 0;
+            const int kw = k < 32 ? k : 31;
+            const int inck = __shfl_sync(FULL, inc, kw), cntk = __shfl_sync(FULL, cnt, kw);
+            const uint32_t mk = __shfl_sync(FULL, m, kw);
+            if (lane >= p && lane < p + take)
+                pend = (w0 + kw) * 32 + (int)__fns(mk, 0u, e - (inck - cntk) + 1);
+            p += take;
+            done += take;
+            if (p == 32) flush();
+        }
+    }
+    flush();
+    __syncwarp();
 }
 
 // RM: the largest basis rank this instantiation handles (16, 32 or 64), which
@@ -1059,6 +1212,82 @@ SEKV_DEV void store_state_lanes(const DecSmem& sm, int idx, int lane, const floa
         for (int k = 0; k < DPL; ++k) sm.st_o[(idx * G + h) * D + lane * DPL + k] = o[h][k];
 }
 
+// The unit's last CTA merges the nsplit partial states of every head by
+// log-sum-exp, in split order, with the arithmetic of merge_kernel below (so the
+// two forms give the same bits): M = max_j m_j, L = sum_j l_j 2^(m_j - M),
+// O = sum_j o_j 2^(m_j - M) / L, lse = (M + log2 L) ln 2. The partials of the
+// other CTAs are read past L1 (they were written by other SMs).
+template <int D, int G>
+SEKV_DEV void merge_unit(const DecArgs& a, const DecSmem& sm, int64_t lunit, int b, int l, int kvh, int tid) {
+    constexpr int NT = (kNW + 1) * 32;
+    const int ns = a.nsplit;
+    const int lane = tid & 31, warp = tid >> 5;
+    float* fac = reinterpret_cast<float*>(sm.stages);          // [G][ns] m_j, then 2^(m_j - M) (the ring is free)
+    float* lsv = fac + G * ns;                                  // [G][ns] l_j
+    float* Mh = lsv + G * ns;                                   // [G]
+    float* Lh = Mh + G;                                         // [G]
+    // every (head, split) pair's (m, l) in one round of loads
+    const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + lunit * G * ns;
+    for (int i = tid; i < G * ns; i += NT) {
+        const float2 v = __ldcg(ml + i);
+        fac[i] = v.x;
+        lsv[i] = v.y;
+    }
+    __syncthreads();
+    // per head (one warp each): M, the factors, and L summed in split order
+    for (int h = warp; h < G; h += kNW + 1) {
+        float* fh = fac + h * ns;
+        float M = -INFINITY;
+        for (int j = lane; j < ns; j += 32) M = fmaxf(M, fh[j]);
+        M = warp_max(M);
+        for (int j = lane; j < ns; j += 32) fh[j] = (M == -INFINITY) ? 0.f : exp2f(fh[j] - M);
+        __syncwarp();
+        if (lane == 0) {
+            float Ls = 0.f;
+            if (M != -INFINITY)
+                for (int j = 0; j < ns; ++j) Ls = fmaf(lsv[h * ns + j], fh[j], Ls);
+            Mh[h] = M;
+            Lh[h] = Ls;
+        }
+    }
+    __syncthreads();
+    // four output dims per thread: O = sum_j o_j f_j / L
+    for (int i = tid; i < G * D / 4; i += NT) {
+        const int h = i / (D / 4), k4 = i % (D / 4);
+        const float M = Mh[h], Ls = Lh[h];
+        const float* fj = fac + h * ns;
+        const float4* po = reinterpret_cast<const float4*>(a.part_o + (lunit * G + h) * ns * D) + k4;
+        float4 os = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (M != -INFINITY) {
+            // 16 splits' loads in flight at a time, summed in split order
+            constexpr int KB = 16;
+            for (int j0 = 0; j0 < ns; j0 += KB) {
+                float4 v[KB];
+#pragma unroll
+                for (int k = 0; k < KB; ++k)
+                    v[k] = j0 + k < ns ? __ldcg(po + (int64_t)(j0 + k) * (D / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int k = 0; k < KB; ++k) {
+                    if (j0 + k < ns) {
+                        const float f = fj[j0 + k];
+                        os.x = fmaf(v[k].x, f, os.x);
+                        os.y = fmaf(v[k].y, f, os.y);
+                        os.z = fmaf(v[k].z, f, os.z);
+                        os.w = fmaf(v[k].w, f, os.w);
+                    }
+                }
+            }
+        }
+        const int64_t out = ((int64_t)b * a.L + l) * a.Hq + kvh * G + h;
+        float* o = a.O + out * D + 4 * k4;
+        o[0] = Ls > 0.f ? os.x / Ls : 0.f;
+        o[1] = Ls > 0.f ? os.y / Ls : 0.f;
+        o[2] = Ls > 0.f ? os.z / Ls : 0.f;
+        o[3] = Ls > 0.f ? os.w / Ls : 0.f;
+        if (k4 == 0) a.lse[out] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
+    }
+}
+
 // SP: the zoom phase may take small spans whole (rank <= 16 only; chosen by the host
 // from the expected zoom count: with few zoomed spans the plain variant is faster)
 template <int DT, int D, int G, int RM, bool SP>
@@ -1069,7 +1298,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     extern __shared__ __align__(1024) unsigned char sm_raw[];
     unsigned char* base = sm_raw + ((1024 - (smem_u32(sm_raw) & 1023)) & 1023);
     const int zwords = a.zwords;
-    const DecSmem sm = carve_smem<C, G, D>(base, a.qcap, zwords);
+    const DecSmem sm = carve_smem<C, G, D>(base, a.qcap, zwords, a.deal);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // one CTA per (split, kv head, sequence x layer); the split index varies
@@ -1167,11 +1396,29 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         if (!a.starve)
             for (int i = 0; i < early; ++i) issue_tile(i);
     }
-    for (int i = tid; i < G * zwords; i += blockDim.x) sm.zw[i] = 0u;
+    // zoom-mask words: routed in this kernel (zero here, bits or-ed in by the stream),
+    // or (tensor-core path, zin) the caller's mask: the split's words, or with deal the
+    // unit's, bits of spans outside them cleared
+    const int zbase = a.deal ? 0 : s0;          // span of bit 0 of word 0
+    const int zend = a.deal ? mb : s1;          // spans >= zend are not in the words
+    for (int i = tid; i < G * zwords; i += blockDim.x) {
+        uint32_t v = 0u;
+        if (C::MMA && a.zin) {
+            const int h = i / zwords, w = i % zwords;
+            const int S = zbase + 32 * w;
+            if (S < zend) {
+                v = a.zmask[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.mw + (S >> 5)];
+                if (zend - S < 32) v &= (1u << (zend - S)) - 1u;
+            }
+        }
+        sm.zw[i] = v;
+    }
     {
         const uint4* qg = reinterpret_cast<const uint4*>(a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB);
         for (int i = tid; i < G * C::ROWB / 16; i += blockDim.x) reinterpret_cast<uint4*>(sm.qs)[i] = qg[i];
     }
+    if (C::MMA && a.deal)
+        for (int w = tid; w < zwords; w += blockDim.x) sm.zu[w] = 0;
     __syncthreads();
 
     const float sl2 = a.scale * kLog2e;
@@ -1199,8 +1446,9 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
 
     if (warp == kNW) {
         // ------------------------------------------------------------ producer
+        int issued = 0;
         if (lane == 0) {
-            int issued = a.starve ? 0 : early;
+            issued = a.starve ? 0 : early;
             for (int i = early; i < ntiles && !a.starve; ++i) {
                 const int s = i % NS;
                 if (!mbar_wait_n(&sm.empty[s], ((i / NS) - 1) & 1, a.polls)) {
@@ -1211,6 +1459,11 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                 issue_tile(i);
                 issued = i + 1;
             }
+        }
+        // every stream tile is issued: while the consumers work through the last ones,
+        // the warp builds the table the zoom producer deals from
+        if (C::MMA && a.deal) deal_table<G>(a, sm, lane, b, mb, zwords);
+        if (lane == 0) {
             // drain: every issued copy has landed before the ring is reused
             for (int i = max(0, issued - NS); i < issued; ++i)
                 if (!mbar_wait_n(&sm.full[i % NS], (i / NS) & 1, a.polls)) {
@@ -1287,11 +1540,12 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                             const bool valid = rv && h < G;
                             const float x = sa[e] + sb[e];
                             const float ell = fmaf(x * inv, a.scale, ls);          // Eq. (5) pre-sigmoid
-                            const bool z = valid && (a.zin ? zmask_bit(a, b, l, kvh * G + h, SL)
+                            const int zwi = h * zwords + ((SL - zbase) >> 5);
+                            const bool z = valid && (a.zin ? ((sm.zw[zwi] >> (SL & 31)) & 1u) != 0u
                                                            : (ell > (hh ? th1 : th0)));   // Eq. (9)
                             if (valid && a.route_logits)
                                 a.route_logits[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.m_cap + SL] = ell;
-                            if (z) atomicOr(&sm.zw[h * zwords + ((SL - s0) >> 5)], 1u << (SL & 31));
+                            if (z && !a.zin) atomicOr(&sm.zw[zwi], 1u << (SL & 31));
                             lg[e] = (valid && !z) ? fmaf(x, a.scale, ls) * kLog2e : -INFINITY;
                         }
                     }
@@ -1457,12 +1711,12 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
 
     if constexpr (C::MMA) {
         // any zoomed span in this CTA's range (the same answer in every warp)
-        const int nwords = s1 > s0 ? (s1 - s0 + 31) >> 5 : 0;
+        const int nwords = a.deal ? zwords : (s1 > s0 ? (s1 - s0 + 31) >> 5 : 0);
         bool zany = false;
         for (int i = lane; i < G * zwords; i += 32) zany = zany || sm.zw[i] != 0u;
         zany = __any_sync(0xffffffffu, zany);
         if (!route_only && zany && *sm.sfail == 0) {     // uniform over the CTA
-            if (warp == kNW) zoom_produce<D, G, SP>(a, sm, lane, b, l, kvh, s0, nwords, zwords);
+            if (warp == kNW) zoom_produce<D, G, SP>(a, sm, lane, b, l, kvh, zbase, nwords, zwords, split);
             else zoom_consume<D, G, RM, SP>(a, sm, warp, lane, qb, mh, lh, oc);
         }
     } else {
@@ -1534,6 +1788,24 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
             a.part_ml[pidx * 2 + 1] = Ls;
         }
     }
+    if (!a.arrive) return;      // a second kernel merges the splits
+
+    // ------------------------------------------------ the unit's last CTA merges its splits
+    // One thread counts the CTA in with an acquire-release add at GPU scope after the
+    // CTA barrier, so the whole CTA's partial is visible before the count and the
+    // other CTAs' partials are visible to the last one after it; the last one resets
+    // the counter for the next call.
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t old;
+        asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(a.arrive + unit) : "memory");
+        const int last = old + 1u == (uint32_t)a.nsplit;
+        if (last) atomicExch(&a.arrive[unit], 0u);
+        *sm.last = last;
+    }
+    __syncthreads();
+    if (!*sm.last) return;
+    merge_unit<D, G>(a, sm, lunit, b, l, kvh, tid);
 }
 
 // one CTA of D threads per (b, l, query head)
@@ -1827,8 +2099,19 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     // test hook (sekv_decode_desc.test_flags bit 0): no copies and short waits
     a.starve = (d.test_flags & 1) ? 1 : 0;
     a.polls = a.starve ? 4096u : kWaitPolls;
-    a.zwords = a.sch_max / 32;
-    const size_t smem = decode_smem_bytes<DT, D, G>(a.zwords, a.qcap);
+    a.arrive = d.phase != SEKV_ROUTE ? d.arrive : nullptr;
+    a.O = d.O;
+    a.lse = d.lse;
+    // Dealing the unit's zoom work evenly over its splits shortens the longest CTA;
+    // it pays when the grid is about one wave (e.g. a call for one layer), where the
+    // call lasts as long as its longest CTA. With several waves the CTAs that hold no
+    // zoom work fill in around the others, and keeping zoom work with its own split
+    // measured faster. It needs the zoom decisions up front (zin) and the unit's
+    // whole mask beside the ring in shared memory.
+    const int64_t ctas = units * p.nsplit;
+    a.deal = (C::MMA && zin && ctas <= 3 * (int64_t)num_sms() && (size_t)(G + 1) * a.mw * 4 <= kDealMaskBytes) ? 1 : 0;
+    a.zwords = a.deal ? a.mw : a.sch_max / 32;
+    const size_t smem = decode_smem_bytes<DT, D, G>(a.zwords, a.qcap, a.deal);
     if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT, D, G, RM, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -1850,7 +2133,7 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     dim3 grid((unsigned)nblk);
     decode_kernel<DT, D, G, RM, SP><<<grid, (kNW + 1) * 32, smem, st>>>(a, maps);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (d.phase != SEKV_ROUTE) {
+    if (d.phase != SEKV_ROUTE && !a.arrive) {
         merge_kernel<D><<<d.B * Lr * d.Hq, D, 0, st>>>(a.part_o, a.part_ml, d.O, d.lse, p.nsplit, G, d.Hkv,
                                                         d.L, d.l0, Lr, d.Hq);
         e = cudaGetLastError();
@@ -1947,13 +2230,14 @@ void* decode_static_scratch(cudaError_t* err) {
     return addr[dev];
 }
 
-// Without a budget: one pass (FUSED / ROUTE / ATTEND). With a budget: ROUTE and
+// Without a budget: one pass (FUSED / ROUTE / ATTEND; ATTEND reads the caller's
+// mask when one is given, and routes again otherwise). With a budget: ROUTE and
 // FUSED run the routing pass (threshold mask + routing logits), then the cap;
 // FUSED then attends with the capped mask as input. ATTEND takes the caller's
 // (capped) mask as input.
 cudaError_t launch_decode(const sekv_decode_desc& d, const DecodePlan& p, void* partials, cudaStream_t st) {
     const bool learned = d.route_W != nullptr;
-    if (!learned && d.budget <= 0) return launch_pass(d, p, partials, st, 0);
+    if (!learned && d.budget <= 0) return launch_pass(d, p, partials, st, d.phase == SEKV_ATTEND && d.zmask ? 1 : 0);
     // the attention pass takes the (capped / learned) mask as input; with learned
     // routing it must not overwrite the routing logits with identity-form ones
     sekv_decode_desc att = d;

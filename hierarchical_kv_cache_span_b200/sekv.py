@@ -57,7 +57,7 @@ class sekv_decode_desc(C.Structure):
         ("logS", _p), ("blk_off", _p), ("Ka", _p), ("Va", _p), ("kbar", _p), ("vbar", _p),
         ("inv_norm", _p), ("theta", _p), ("arena", _p), ("slot", _p), ("O", _p), ("lse", _p),
         ("zmask", _p), ("route_logits", _p), ("route_W", _p), ("kbar_r", _p), ("dev_status", _p),
-        ("workspace", _p),
+        ("workspace", _p), ("arrive", _p),
         ("region_elems", _i64), ("workspace_bytes", _i64), ("scale", C.c_float),
         ("B", _i32), ("L", _i32), ("Hq", _i32), ("Hkv", _i32), ("d", _i32), ("dtype", _i32),
         ("l0", _i32), ("l1", _i32), ("a_cap", _i32), ("m_cap", _i32), ("rank", _i32),

@@ -87,9 +87,9 @@ enum {
 /* Decode phases. FUSED: routing + attention over a hot cache (one pass for the
  * identity routing form; with a budget or learned routing, a routing pass and then
  * attention with its mask). ROUTE: routing only (writes zmask / route_logits).
- * ATTEND: attention reading bases through the slot table; it routes again
- * (bit-identical to ROUTE) in the identity form without a budget, and otherwise
- * takes zmask, as ROUTE wrote it, as input. */
+ * ATTEND: attention reading bases through the slot table; it takes zmask, as ROUTE
+ * wrote it for the same q and theta, as input; without zmask (identity form, no
+ * budget) it routes again, bit-identical to ROUTE. */
 enum { SEKV_FUSED = 0, SEKV_ROUTE = 1, SEKV_ATTEND = 2 };
 
 typedef void* sekv_stream_t;   /* a cudaStream_t (NULL = legacy default stream) */
@@ -217,6 +217,13 @@ typedef struct sekv_decode_desc {
     const void* kbar_r;      /* [B][L][Hq][m_cap][dr] routing summaries from the build     */
     int32_t* dev_status;     /* device int32, required                                     */
     void* workspace;         /* device, sekv_decode_workspace_bytes() bytes, 256-B aligned */
+    uint32_t* arrive;        /* optional [B][L][Hkv] device arrival counters, all zero before
+                                the first call that gets them; every FUSED / ATTEND call leaves
+                                them zero again. With them the last CTA of each (b, l, kv head)
+                                to finish merges the split-K partials (no second kernel);
+                                NULL = a separate merge kernel. The results are the same bits
+                                either way. Calls in flight at the same time must not decode
+                                the same (b, l, kv head) with the same counters.            */
     int64_t region_elems;
     int64_t workspace_bytes;
     float scale;             /* logit scale, normally 1/sqrt(d) (routing uses it too, d'=d) */

@@ -150,6 +150,64 @@ def test_split_count_does_not_change_result():
             assert (lse_gpu - ref[1]).abs().max().item() < 2e-5
 
 
+@pytest.mark.parametrize("name,over,phase", [("c2", dict(n=4096, L=2), "fused"),
+                                             ("c1", dict(), "fused"),
+                                             ("c3", dict(n=8192, L=2), "attend")])
+def test_in_kernel_merge_equals_merge_kernel(name, over, phase):
+    """with arrival counters the last CTA of each (b, l, kv head) merges the split-K
+    partials; on the tensor-core path the result has the same bits as the separate
+    merge kernel (arrive = NULL), for several split counts and for per-layer calls,
+    and the counters are zero again after every call"""
+    P = _lib()
+    S = P.sekv
+    wl = WORKLOADS[name].scaled(**over)
+    H, K, V, segs, units, q, theta, scale = _setup(wl, quantile=0.9 if phase == "attend" else None)
+    c = _cache(wl, home="device" if phase == "fused" else "host")
+    T.upload_oracle_cache(c, segs, units)
+    th = torch.tensor(theta, dtype=torch.float32, device="cuda")
+    qd = q.cuda()
+    kw = {}
+    if phase == "attend":
+        zr = c.new_zmask()
+        c.decode(qd, th, phase=S.SEKV_ROUTE, zmask=zr)
+        fetch = P.ColdFetcher(c, arena_elems=c.region * wl.L)
+        info = fetch.fetch(zr)
+        torch.cuda.current_stream().wait_event(fetch.done)
+        assert info["spans"] > 0
+        kw = dict(phase=S.SEKV_ATTEND, slot=fetch.slot_dev, arena=fetch.arena)
+    stream = torch.cuda.current_stream().cuda_stream
+    refs = []
+    for ns in (1, 3, 0):
+        for lr in ((0, wl.L),) + tuple((l, l + 1) for l in range(wl.L)):
+            outs = []
+            for with_counters in (True, False):
+                O_g, lse_g = c.new_outputs()
+                O_g.fill_(float("nan"))
+                zm = c.new_zmask() if phase == "fused" else zr      # ATTEND reads ROUTE's mask
+                d = c.decode_desc(qd, th, O=O_g, lse=lse_g, zmask=zm, nsplit=ns, l0=lr[0], l1=lr[1], **kw)
+                assert d.arrive
+                if not with_counters:
+                    d.arrive = None
+                S.check(S.sekv_decode_attn(d, stream), "decode")
+                torch.cuda.synchronize()
+                outs.append((O_g[:, lr[0]:lr[1]].clone(), lse_g[:, lr[0]:lr[1]].clone(), zm))
+            assert c.read_status() == 0
+            assert int(c._arrive.abs().sum()) == 0
+            if wl.dtype == "bf16":
+                assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1]), (ns, lr)
+            else:
+                # the fp32 path hands zoomed spans to its warps in arrival order, so the
+                # CTA's sum order (and the last bits) vary from call to call
+                assert (outs[0][0] - outs[1][0]).abs().max().item() <= 1e-6, (ns, lr)
+                assert (outs[0][1] - outs[1][1]).abs().max().item() <= 1e-6, (ns, lr)
+            if lr == (0, wl.L):
+                refs.append(outs[0])
+    # every split count against the oracle (with a mask given, ATTEND deals the zoomed
+    # token units of a unit over its splits, cutting spans between them)
+    for O_r, lse_r, zm_r in refs:
+        _compare(wl, c, q, theta, scale, segs, units, O_r, lse_r, zm_r)
+
+
 def test_layer_range_calls_equal_one_call():
     """per-layer calls (l0 = l, l1 = l + 1, each with its own split plan) write the
     same masks and, up to split-K summation order, the same O / lse as one call
