@@ -1220,12 +1220,22 @@ SEKV_DEV void store_state_lanes(const DecSmem& sm, int idx, int lane, const floa
 template <int D, int G>
 SEKV_DEV void merge_unit(const DecArgs& a, const DecSmem& sm, int64_t lunit, int b, int l, int kvh, int tid) {
     constexpr int NT = (kNW + 1) * 32;
+    constexpr int KB = 16;                                      // splits' loads in flight per thread
     const int ns = a.nsplit;
     const int lane = tid & 31, warp = tid >> 5;
     float* fac = reinterpret_cast<float*>(sm.stages);          // [G][ns] m_j, then 2^(m_j - M) (the ring is free)
     float* lsv = fac + G * ns;                                  // [G][ns] l_j
     float* Mh = lsv + G * ns;                                   // [G]
     float* Lh = Mh + G;                                         // [G]
+    // this thread's first output quad: its first KB splits are loaded now, so they
+    // arrive while the factors are formed
+    constexpr int K0 = 8;
+    const int i0 = tid;
+    const float4* po0 = reinterpret_cast<const float4*>(a.part_o + (lunit * G + i0 / (D / 4)) * ns * D) + i0 % (D / 4);
+    float4 v0[K0];
+#pragma unroll
+    for (int k = 0; k < K0; ++k)
+        v0[k] = (i0 < G * D / 4 && k < ns) ? __ldcg(po0 + (int64_t)k * (D / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
     // every (head, split) pair's (m, l) in one round of loads
     const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + lunit * G * ns;
     for (int i = tid; i < G * ns; i += NT) {
@@ -1251,17 +1261,29 @@ SEKV_DEV void merge_unit(const DecArgs& a, const DecSmem& sm, int64_t lunit, int
         }
     }
     __syncthreads();
-    // four output dims per thread: O = sum_j o_j f_j / L
+    // four output dims per thread: O = sum_j o_j f_j / L, summed in split order
     for (int i = tid; i < G * D / 4; i += NT) {
         const int h = i / (D / 4), k4 = i % (D / 4);
         const float M = Mh[h], Ls = Lh[h];
         const float* fj = fac + h * ns;
         const float4* po = reinterpret_cast<const float4*>(a.part_o + (lunit * G + h) * ns * D) + k4;
         float4 os = make_float4(0.f, 0.f, 0.f, 0.f);
+        int js = 0;
+        if (M != -INFINITY && i == i0) {
+#pragma unroll
+            for (int k = 0; k < K0; ++k) {
+                if (k < ns) {
+                    const float f = fj[k];
+                    os.x = fmaf(v0[k].x, f, os.x);
+                    os.y = fmaf(v0[k].y, f, os.y);
+                    os.z = fmaf(v0[k].z, f, os.z);
+                    os.w = fmaf(v0[k].w, f, os.w);
+                }
+            }
+            js = K0;
+        }
         if (M != -INFINITY) {
-            // 16 splits' loads in flight at a time, summed in split order
-            constexpr int KB = 16;
-            for (int j0 = 0; j0 < ns; j0 += KB) {
+            for (int j0 = js; j0 < ns; j0 += KB) {
                 float4 v[KB];
 #pragma unroll
                 for (int k = 0; k < KB; ++k)
@@ -1295,6 +1317,12 @@ __global__ void __launch_bounds__((kNW + 1) * 32, 3)
 decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     using C = DecCfg<DT, D, G>;
     constexpr int DPL = C::DPL, R = C::R, TR = C::TR, NS = C::NS;
+    // Programmatic dependent launch: the grid may be scheduled while the previous
+    // kernel on the stream finishes; nothing is read before that kernel has
+    // completed and its writes are visible. Once every CTA of this grid has started,
+    // the next kernel may be scheduled likewise.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ __align__(1024) unsigned char sm_raw[];
     unsigned char* base = sm_raw + ((1024 - (smem_u32(sm_raw) & 1023)) & 1023);
     const int zwords = a.zwords;
@@ -1330,9 +1358,22 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     const int ntiles = nta + nts;
 
     // issue stream tile i into its ring stage (producer lane 0)
+    // Ring positions: one per stage, except in a routing pass on the tensor-core path,
+    // which loads key tiles only: then every stage holds two positions (key rows in
+    // its K or V half, the span scalars in the first or second 512 bytes past the two
+    // tiles), so twice as many tiles are in flight.
+    static_assert(!C::MMA || 2 * C::TILE + 2 * C::META <= C::STAGE, "two key tiles per stage");
+    const int NP = (C::MMA && route_only) ? 2 * NS : NS;
+    auto pos_key = [&](int s) -> unsigned char* {
+        return NP == NS ? sm.stages + (size_t)s * C::STAGE : sm.stages + (size_t)(s >> 1) * C::STAGE + (s & 1) * C::TILE;
+    };
+    auto pos_meta = [&](int s) -> unsigned char* {
+        return NP == NS ? sm.stages + (size_t)s * C::STAGE + 2 * C::TILE
+                        : sm.stages + (size_t)(s >> 1) * C::STAGE + 2 * C::TILE + (s & 1) * C::META;
+    };
     auto issue_tile = [&](int i) {
-        const int s = i % NS;
-        unsigned char* st = sm.stages + (size_t)s * C::STAGE;
+        const int s = i % NP;
+        unsigned char* st = pos_key(s);
         if (i < nta) {
             const int r0 = a0 + i * TR;
             if constexpr (C::MMA) {
@@ -1369,16 +1410,16 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                 bulk_g2s(st, a.kbar + off, bytes, &sm.full[s]);
                 if (!route_only) bulk_g2s(st + C::TILE, a.vbar + off, bytes, &sm.full[s]);
             }
-            bulk_g2s(st + 2 * C::TILE, a.inv_norm + unit * a.m_cap + S0, mbytes, &sm.full[s]);
-            bulk_g2s(st + 2 * C::TILE + TR * 4, a.logS + (int64_t)b * a.m_cap + S0, mbytes, &sm.full[s]);
+            bulk_g2s(pos_meta(s), a.inv_norm + unit * a.m_cap + S0, mbytes, &sm.full[s]);
+            bulk_g2s(pos_meta(s) + TR * 4, a.logS + (int64_t)b * a.m_cap + S0, mbytes, &sm.full[s]);
         }
     };
 
     // The producer initialises the barriers and issues the first ring stages before
     // the CTA-wide barrier, so their latency overlaps the query and mask loads.
-    const int early = min(NS, ntiles);
+    const int early = min(NP, ntiles);
     if (tid == kNW * 32) {
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < NP; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kNW);
         }
@@ -1446,12 +1487,15 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
 
     if (warp == kNW) {
         // ------------------------------------------------------------ producer
+        // with the first stages in flight, the warp builds the table the zoom
+        // producer deals from (its loads overlap the consumers' first tiles)
+        if (C::MMA && a.deal) deal_table<G>(a, sm, lane, b, mb, zwords);
         int issued = 0;
         if (lane == 0) {
             issued = a.starve ? 0 : early;
             for (int i = early; i < ntiles && !a.starve; ++i) {
-                const int s = i % NS;
-                if (!mbar_wait_n(&sm.empty[s], ((i / NS) - 1) & 1, a.polls)) {
+                const int s = i % NP;
+                if (!mbar_wait_n(&sm.empty[s], ((i / NP) - 1) & 1, a.polls)) {
                     set_status(a.status, SEKV_ERR_TIMEOUT);
                     *sm.sfail = 1;
                     break;
@@ -1460,13 +1504,10 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                 issued = i + 1;
             }
         }
-        // every stream tile is issued: while the consumers work through the last ones,
-        // the warp builds the table the zoom producer deals from
-        if (C::MMA && a.deal) deal_table<G>(a, sm, lane, b, mb, zwords);
         if (lane == 0) {
             // drain: every issued copy has landed before the ring is reused
-            for (int i = max(0, issued - NS); i < issued; ++i)
-                if (!mbar_wait_n(&sm.full[i % NS], (i / NS) & 1, a.polls)) {
+            for (int i = max(0, issued - NP); i < issued; ++i)
+                if (!mbar_wait_n(&sm.full[i % NP], (i / NP) & 1, a.polls)) {
                     set_status(a.status, SEKV_ERR_TIMEOUT);
                     *sm.sfail = 1;
                 }
@@ -1495,13 +1536,13 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         const int krow = rbase + lr + ((lj & 1) << 3);    // this lane's ldmatrix row for K
         const int vrow = rbase + lr + ((lj >> 1) << 3);   // ... and for V
         for (int i = 0; i < ntiles && ok; ++i) {
-            const int s = i % NS;
-            if (!mbar_wait_n(&sm.full[s], (i / NS) & 1, a.polls)) {
+            const int s = i % NP;
+            if (!mbar_wait_n(&sm.full[s], (i / NP) & 1, a.polls)) {
                 set_status(a.status, SEKV_ERR_TIMEOUT);
                 ok = false;
                 break;
             }
-            const unsigned char* st = sm.stages + (size_t)s * C::STAGE;
+            const unsigned char* st = pos_key(s);
             const bool anchor_tile = i < nta;
             const int S0 = s0 + (i - nta) * TR;
             const int trows = anchor_tile ? min(TR, a1 - (a0 + i * TR)) : min(TR, s1 - S0);
@@ -1525,7 +1566,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                         lg[e] = (2 * c + (e & 1) < G && tk < trows) ? (sa[e] + sb[e]) * sl2 : -INFINITY;
                     }
                 } else {
-                    const float* invn = reinterpret_cast<const float*>(st + 2 * C::TILE);
+                    const float* invn = reinterpret_cast<const float*>(pos_meta(s));
                     const float* lsv = invn + TR;
 #pragma unroll
                     for (int rr = 0; rr < 2; ++rr) {
@@ -2131,7 +2172,20 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     const int64_t nblk = (int64_t)p.nsplit * d.Hkv * d.B * Lr;
     if (nblk > 0x7fffffff) return cudaErrorInvalidConfiguration;
     dim3 grid((unsigned)nblk);
-    decode_kernel<DT, D, G, RM, SP><<<grid, (kNW + 1) * 32, smem, st>>>(a, maps);
+    // launched with programmatic stream serialization: its launch overlaps the end of
+    // the previous kernel on the stream (the kernel waits for that kernel's writes)
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3((kNW + 1) * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, decode_kernel<DT, D, G, RM, SP>, a, maps)) != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (d.phase != SEKV_ROUTE && !a.arrive) {
         merge_kernel<D><<<d.B * Lr * d.Hq, D, 0, st>>>(a.part_o, a.part_ml, d.O, d.lse, p.nsplit, G, d.Hkv,
