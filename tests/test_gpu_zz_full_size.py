@@ -3,7 +3,8 @@
 The default benchmark workload (one 128K-token sequence, 32 layers, 32 query / 8
 kv heads, d = 128, bf16, rank 16, bases in pinned host memory) is built by the
 library and decoded as the benchmark does it: ROUTE, fetch of the zoomed bases,
-ATTEND with the automatic split plan and the zoom hint. The oracle cannot redo the
+ATTEND with ROUTE's mask, the automatic split plan and the zoom hint, and again as
+per-layer ATTEND calls (the latency form). The oracle cannot redo the
 whole step, so it builds and decodes three sampled (layer, kv head) units from
 the same device-generated inputs; for those units the zoom masks must be
 bit-exact (their heads' thresholds sit >= DELTA_L from every routing logit) and
@@ -84,8 +85,14 @@ def test_full_size_cold_step_on_sampled_units():
     fetch = P.ColdFetcher(c, arena_elems=c.region * wl.L)
     info = fetch.fetch(zm)
     torch.cuda.current_stream().wait_event(fetch.done)
-    O_g, lse_g = c.decode(q, th_d, phase=P.SEKV_ATTEND, slot=fetch.slot_dev, arena=fetch.arena,
+    O_g, lse_g = c.decode(q, th_d, phase=P.SEKV_ATTEND, slot=fetch.slot_dev, arena=fetch.arena, zmask=zm,
                           zoom_hint=zoom_hint)
+    # the per-layer form of the same step (one call per layer: a one-wave grid, which
+    # deals each unit's zoomed token units evenly over its splits)
+    O_p, lse_p = c.new_outputs()
+    for l in sorted({l for (l, _) in SAMPLED}):
+        c.decode(q, th_d, phase=P.SEKV_ATTEND, O=O_p, lse=lse_p, slot=fetch.slot_dev, arena=fetch.arena, zmask=zm,
+                 zoom_hint=zoom_hint, l0=l, l1=l + 1)
     torch.cuda.synchronize()
     assert c.read_status() == 0, P.sekv.sekv_status_str(c.read_status())
     assert info["spans"] > 0
@@ -100,10 +107,11 @@ def test_full_size_cold_step_on_sampled_units():
             np.testing.assert_array_equal(T.zmask_bits(zm, b, l, kvh * G + g, m), z[g], err_msg=str((l, kvh, g)))
         zoomed += int(z.sum())
         o, ls = O.decode_unit(qg, u.Ka, u.Va, u.kbar, u.vbar, u.logS, z, u.bases, scale)
-        err = np.abs(T.f64(O_g[b, l, kvh * G:(kvh + 1) * G]) - o).max()
-        lerr = np.abs(T.f64(lse_g[b, l, kvh * G:(kvh + 1) * G]) - ls).max()
-        assert err <= 2e-2, (l, kvh, err)
-        assert lerr <= 2e-2, (l, kvh, lerr)
+        for form, (Of, lf) in (("all layers", (O_g, lse_g)), ("per layer", (O_p, lse_p))):
+            err = np.abs(T.f64(Of[b, l, kvh * G:(kvh + 1) * G]) - o).max()
+            lerr = np.abs(T.f64(lf[b, l, kvh * G:(kvh + 1) * G]) - ls).max()
+            assert err <= 2e-2, (form, l, kvh, err)
+            assert lerr <= 2e-2, (form, l, kvh, lerr)
     assert zoomed > 0
 
 
