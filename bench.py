@@ -612,15 +612,14 @@ def run_sekv(args, rank, world, local_rank):
                          f"{workers} cores. Oracle build of those units: mean {statistics.mean(t_build):.2f} s/unit",
                "oracle_build_s_per_unit": statistics.mean(t_build)}
 
-    # ROUTE + ATTEND + merge (cold) or FUSED + merge (hot); a budget adds the cap
-    # kernel, and on the hot path the routing pass before the capped FUSED pass
-    # (learned routing: its own routing kernel before the attention pass)
-    if cold:
-        launches_per_step = 3 + (1 if args.budget else 0)
-    elif learned:
-        launches_per_step = 3 + (1 if args.budget else 0)
+    # ROUTE + ATTEND (cold) or FUSED (hot), each one decode_kernel launch (the split-K
+    # merge runs in its last CTA per unit); a budget adds the cap kernel, and on the
+    # hot path the routing pass before the capped FUSED pass (learned routing: its own
+    # routing kernel before the attention pass)
+    if cold or learned:
+        launches_per_step = 2 + (1 if args.budget else 0)
     else:
-        launches_per_step = 2 + (2 if args.budget else 0)
+        launches_per_step = 1 + (2 if args.budget else 0)
     rb = route_bytes(cache, learned)
     route_avg = statistics.mean(route_ms)
     from sekv_synth import WORKLOADS as _WL
@@ -654,7 +653,7 @@ def run_sekv(args, rank, world, local_rank):
                      "frac": achieved / peak,
                      "traffic": profiled_traffic(wl.name) if full_size else None,
                      "traffic_unit": "DRAM bytes read + written per ATTEND launch (ncu, profiles/)",
-                     "kernel": "sekv_decode_attn ATTEND call (decode_kernel + merge_kernel)",
+                     "kernel": "sekv_decode_attn ATTEND call (one decode_kernel launch; the split-K merge runs in its last CTA per unit)",
                      "peak_source": peak_src, "frac_of_8TBps_nominal": achieved / 8000.0},
         "prefill_build": build,
         "gpu_launches": launches_per_step * steps,
