@@ -299,7 +299,9 @@ bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
     // spans this call needs: any head of (b, l) zooms them (rows of [l0, l1) only)
     const int Lr = d->l1 - d->l0;
     std::vector<uint32_t> needw((size_t)d->B * Lr * mw, 0u);
-    int64_t misses = 0;
+    int64_t misses = 0, need = 0;                     // spans to place and their elements
+    struct Miss { int b, l, S; };
+    std::vector<Miss> miss;                             // in (b, l, S) order
     for (int b = 0; b < d->B; ++b) {
         const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
         for (int l = d->l0; l < d->l1; ++l) {
@@ -313,8 +315,13 @@ bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
             for (int w = 0; w < mw; ++w)
                 for (uint32_t bits = uni[w]; bits; bits &= bits - 1u) {
                     const int S = (w << 5) + __builtin_ctz(bits);
-                    if (d->slot_host[idx(b, l, S)] >= 0) kp.hit.push_back(idx(b, l, S));
-                    else ++misses;
+                    if (d->slot_host[idx(b, l, S)] >= 0) {
+                        kp.hit.push_back(idx(b, l, S));
+                    } else {
+                        ++misses;
+                        need += size_of(b, S);
+                        miss.push_back({b, l, S});
+                    }
                 }
         }
     }
@@ -327,6 +334,46 @@ bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
     if (misses == 0) {                                    // nothing to place: no scan of the arena
         kp.used = d->arena_used ? *d->arena_used : 0;
         return true;
+    }
+    // Fast path: the end of the highest resident entry, and the misses placed one
+    // after another above it when they fit there (nothing is evicted then; only when
+    // they do not fit are the gaps searched and entries evicted).
+    {
+        int64_t top = 0, held = 0;
+        for (int b = 0; b < d->B; ++b) {
+            const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
+            const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
+            for (int l = 0; l < d->L; ++l) {
+                const int64_t* sl = d->slot_host + idx(b, l, 0);
+                for (int S = 0; S < m; ++S) {             // branch-free: vectorises
+                    const int64_t sz = bo[S + 1] - bo[S];
+                    const bool r = sl[S] >= 0;
+                    top = std::max(top, r ? sl[S] + sz : 0);
+                    held += r ? sz : 0;
+                }
+            }
+        }
+        if (top + need <= d->arena_elems) {
+            kp.used = held;
+            for (size_t i = 0; i < miss.size();) {
+                const int b = miss[i].b, l = miss[i].l, Sa = miss[i].S;
+                size_t j = i + 1;                        // a run of consecutive missing spans
+                while (j < miss.size() && miss[j].b == b && miss[j].l == l && miss[j].S == Sa + (int)(j - i)) ++j;
+                const int Se = Sa + (int)(j - i);
+                const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
+                const int64_t width = bo[Se] - bo[Sa];
+                const int64_t src = ((int64_t)b * d->L + l) * d->region_elems + bo[Sa];
+                for (int t = Sa; t < Se; ++t) kp.place.push_back({idx(b, l, t), top + (bo[t] - bo[Sa])});
+                kp.copies.push_back({src, top, width, b, l});
+                top += width;
+                kp.spans += Se - Sa;
+                kp.bytes_elems += width;
+                kp.used += width;
+                kp.dirty[l] = 1;
+                i = j;
+            }
+            return true;
+        }
     }
     // resident entries: the occupied intervals and the eviction candidates
     struct Ent { int64_t last, off, size, id; int b, l; };
@@ -489,14 +536,20 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
             if ((e = cudaMemcpyAsync(arena + c.dst * es, home + c.src * es, c.width * es, cudaMemcpyHostToDevice,
                                      xs)) != cudaSuccess)
                 return cuda_fail(e, "fetch: basis copy");
-        for (int l = 0; l < d->L; ++l) {
-            if (!kp.dirty[l]) continue;
-            for (int b = 0; b < d->B; ++b) {
-                const int64_t o = ((int64_t)b * d->L + l) * d->m_cap;
-                if ((e = cudaMemcpyAsync(d->slot_dev + o, d->slot_host + o, sizeof(int64_t) * d->m_cap,
-                                         cudaMemcpyHostToDevice, xs)) != cudaSuccess)
-                    return cuda_fail(e, "fetch: slot upload");
+        // the slot rows of the layers that changed: one copy per sequence over the
+        // range from the first to the last such layer (the copy engine's fixed cost
+        // per copy outweighs the few unchanged rows in between)
+        int lf = d->L, ll = -1;
+        for (int l = 0; l < d->L; ++l)
+            if (kp.dirty[l]) {
+                lf = std::min(lf, l);
+                ll = l;
             }
+        for (int b = 0; b < d->B && ll >= lf; ++b) {
+            const int64_t o = ((int64_t)b * d->L + lf) * d->m_cap;
+            if ((e = cudaMemcpyAsync(d->slot_dev + o, d->slot_host + o, sizeof(int64_t) * d->m_cap * (ll - lf + 1),
+                                     cudaMemcpyHostToDevice, xs)) != cudaSuccess)
+                return cuda_fail(e, "fetch: slot upload");
         }
         if (d->stats) {
             d->stats[0] = kp.bytes_elems * es;
