@@ -92,6 +92,38 @@ def test_decode_kernel_level(name, over):
     print(f"{name} {over}: max|dO|={err:.2e} max|dlse|={lerr:.2e} zoomed={nz}")
 
 
+@pytest.mark.parametrize("name,over", KERNEL_CASES)
+def test_attend_with_mask_matches_oracle(name, over):
+    """ROUTE -> fetch -> ATTEND with ROUTE's mask as input, for every kernel-level
+    shape: all layers in one call at two split counts, and one call per layer (a
+    one-wave grid: the tensor-core path deals each unit's zoomed token units over
+    its splits, cutting spans between them); every result against the oracle"""
+    P = _lib()
+    wl = WORKLOADS[name].scaled(**over)
+    H, K, V, segs, units, q, theta, scale = _setup(wl)
+    c = _cache(wl, home="host")
+    T.upload_oracle_cache(c, segs, units)
+    th = torch.tensor(theta, dtype=torch.float32, device="cuda")
+    qd = q.cuda()
+    zm = c.new_zmask()
+    c.decode(qd, th, phase=P.SEKV_ROUTE, zmask=zm)
+    fetch = P.ColdFetcher(c, arena_elems=c.region * wl.L)
+    fetch.fetch(zm)
+    torch.cuda.current_stream().wait_event(fetch.done)
+    kw = dict(phase=P.SEKV_ATTEND, slot=fetch.slot_dev, arena=fetch.arena, zmask=zm)
+    results = []
+    for ns in (0, 5):
+        results.append(c.decode(qd, th, nsplit=ns, **kw))
+    O_p, lse_p = c.new_outputs()
+    for l in range(wl.L):
+        c.decode(qd, th, O=O_p, lse=lse_p, l0=l, l1=l + 1, **kw)
+    results.append((O_p, lse_p))
+    torch.cuda.synchronize()
+    assert c.read_status() == 0
+    for O_gpu, lse_gpu in results:
+        _compare(wl, c, q, theta, scale, segs, units, O_gpu, lse_gpu, zm)
+
+
 @pytest.mark.parametrize("name,over", [
     ("c2", dict(n=2048, L=1, Hq=8, Hkv=2)),                 # r = 16
     ("c5", dict(n=1536, L=1, Hq=8, Hkv=2, rank=40)),        # r8 = 40: two B / D pieces, odd blocks
