@@ -186,8 +186,10 @@ struct __align__(16) ZPiece {
     int cnt;             // B / D: basis rows (a multiple of 8); MIX: tokens (may be 0)
     int len, rS;
     uint32_t hm;         // query heads of the group that zoom the span
-    int rot;             // B / AC / D: the span's 32-token unit j belongs to consumer warp
-                         // (j + rot) % 4; SPAN: the warp that handles the whole span
+    int rot;             // B / MIX / D: the span's 32-token unit j belongs to consumer warp
+                         // (j + rot) % 4 for ranks <= 16, and to 2 (rot / 2) + (j + rot) % 2
+                         // (one pair of warps per span) above; SPAN: the warp that handles
+                         // the whole span
 };
 
 // shared-memory carve-up common to both paths
@@ -630,7 +632,16 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
     constexpr uint32_t FULL = 0xffffffffu;
     uint32_t np = 0;          // pieces armed
     bool good = true;
-    int rot = 0;
+    // Shared spans: for ranks <= 16 a span's units are dealt round-robin over the four
+    // consumer warps, continuing across spans. Above, u = B q and the D projection
+    // (done by every warp that takes part in a span) cost more, so a span goes to one
+    // of two pairs of warps, its units alternating between the pair's warps: two
+    // spans in flight at once, and half the u / D work (C5, rank 32: -8 % per call;
+    // at rank 16 the two forms measured within 2 %). A span goes to the pair with less
+    // work queued (its units + ~4 units' worth for u and D); each pair's next span
+    // continues its unit parity. Whole-span pieces rotate over the warps.
+    const bool pairs = a.rank > 16;
+    int owner = 0, rot = 0, pw[2] = {0, 0}, ps[2] = {0, 0};
     // Whole-span pieces (one warp per small span, no repeated u / D work) pay off
     // when the CTA has enough zoomed spans to keep the four consumer warps busy
     // with different spans; with few, sharing each span's units across the warps
@@ -692,19 +703,31 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
         pc.len = te - tb;
         pc.rS = rS;
         pc.hm = jhm;
-        pc.rot = rot;
         if (span_mode && tb == 0 && te == jl && be * 2 + D * 16 <= ZSL) {
             // the whole block fits one slot (with room for the D projection's
             // read of one 8-row block past D): one piece, one owner warp
+            pc.rot = owner;
             pc.kind = ZP_SPAN; pc.first = 1; pc.r0 = 0; pc.cnt = jl;
             emit1(pc, blk, (uint32_t)(be * 2));
-            rot = (rot + 1) & 3;
+            owner = (owner + 1) & 3;
             return;
         }
         // B, then the A / C rows of the tokens, then D, packed into as few slots
         // as they fit (B or D of more than half a slot travel in chunks of their
         // own). Every part is reserved with the rows its fragment loads read:
         // tokens up to a multiple of 32, basis rows up to a multiple of 16.
+        {
+            const int nu = (te - tb + 31) >> 5;
+            if (pairs) {
+                const int pr = pw[1] < pw[0] ? 1 : 0;
+                pc.rot = 2 * pr + ps[pr];
+                ps[pr] = (ps[pr] + nu) & 1;
+                pw[pr] += nu + 4;
+            } else {
+                pc.rot = rot;
+                rot = (rot + nu) & 3;
+            }
+        }
         const uint32_t bsz = (uint32_t)r8 * D * 2;                 // bytes of B (and of D)
         const uint32_t dres = (uint32_t)((r8 + 15) & ~15) * D * 2;
         const uint32_t tokb = 4u * r8;                              // A + C bytes per token
@@ -744,7 +767,6 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
                 emit1(pc, srcD + (int64_t)r0 * D * 2, (uint32_t)pc.cnt * C::ROWB);
             }
         }
-        rot = (rot + ((te - tb + 31) >> 5)) & 3;
     };
     // Walk the zoomed spans (any head of the group) in span order, up to 32 at a time:
     // visit(len, hm, off, n) gets this lane's span of the batch (len 0: none or
@@ -1138,6 +1160,14 @@ SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int la
         }
     };
 
+    // does this warp take any unit of the span? (ranks above 16: the span's pair of
+    // warps, units alternating within the pair; else all four warps in turn)
+    constexpr bool PAIRS = RM > 16;
+    constexpr int WSTEP = PAIRS ? 2 : 4;
+    auto owns = [&](const ZPiece& pc) {
+        if (PAIRS) return (warp >> 1) == (pc.rot >> 1) && ((pc.len + 31) >> 5) > ((warp - pc.rot) & 1);
+        return ((pc.len + 31) >> 5) > ((warp - pc.rot) & 3);
+    };
     for (uint32_t k = 0;; ++k) {
         const int slot = (int)(k % ZNS);
         if (!mbar_wait_n(&sm.zfull[slot], (k / ZNS) & 1, a.polls)) {
@@ -1169,10 +1199,10 @@ SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int la
             const int res = ((pc.cnt + 31) & ~31) * r8 * 2;
             if (pc.first & kMixB) {
                 span_begin(pc);
-                mine = ((pc.len + 31) >> 5) > ((warp - pc.rot) & 3);
+                mine = owns(pc);
                 if (mine) do_u(zs, 0, r8);
             }
-            if (mine && pc.cnt > 0) do_units(zs + oa, zs + oa + res, pc.cnt, (warp - pc.rot - (pc.r0 >> 5)) & 3, 4);
+            if (mine && pc.cnt > 0) do_units(zs + oa, zs + oa + res, pc.cnt, (warp - pc.rot - (pc.r0 >> 5)) & (WSTEP - 1), WSTEP);
             if (mine && (pc.first & kMixD)) {
                 do_merge();
                 do_D(zs + oa + 2 * res, 0, r8);
@@ -1180,7 +1210,7 @@ SEKV_DEV void zoom_consume(const DecArgs& a, const DecSmem& sm, int warp, int la
         } else if (pc.kind == ZP_B) {
             if (pc.first) {
                 span_begin(pc);
-                mine = ((pc.len + 31) >> 5) > ((warp - pc.rot) & 3);
+                mine = owns(pc);
             }
             if (mine) do_u(zs, pc.r0, pc.cnt);
         } else {  // ZP_D
