@@ -2070,9 +2070,11 @@ DecodePlan plan_decode(const sekv_decode_desc& d) {
             // each plus a fixed cost (setup, partial write, merge; ~64 rows' worth),
             // scheduled dynamically onto the resident slots, plus half a CTA of tail.
             // A routing pass reads only the span rows' keys (about a quarter of the
-            // bytes of an anchor + span row pair), so it counts a quarter of the rows.
+            // bytes of an anchor + span row pair), so it counts a quarter of the rows,
+            // and its fixed cost per CTA weighs twice as much against them (fitted on
+            // a B200 at 128K: 2, 3, 4, 6 splits took 42.7, 35.9, 38.9, 40.2 us).
             const double rows = d.phase == SEKV_ROUTE ? 0.25 * d.rows_hint : (double)d.rows_hint;
-            const double o = 64.0;
+            const double o = d.phase == SEKV_ROUTE ? 128.0 : 64.0;
             int best = 1;
             double best_t = 1e300;
             for (int c = 1; c <= lim; ++c) {
