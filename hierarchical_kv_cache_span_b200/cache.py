@@ -247,6 +247,7 @@ class ColdFetcher:
         self.c = cache
         self.keep = bool(keep)
         self.arena_used = torch.zeros(1, dtype=torch.int64)
+        self.arena_top = torch.zeros(1, dtype=torch.int64)     # keep mode: end of the highest entry
         B, L, Hq, m_cap = cache.B, cache.L, cache.Hq, cache.m_cap
         dev = cache.device
         self.arena = torch.zeros(max(arena_elems, 64), dtype=cache.dt, device=dev)
@@ -273,6 +274,7 @@ class ColdFetcher:
         d.home, d.arena = _ptr(c.home), _ptr(self.arena)
         d.slot_dev, d.slot_host, d.stats = _ptr(self.slot_dev), _ptr(self.slot_host), _ptr(self.stats)
         d.arena_used, d.last_use = _ptr(self.arena_used), _ptr(self.last_use) if self.keep else None
+        d.arena_top = _ptr(self.arena_top) if self.keep else None
         d.route_done = route_done.cuda_event if route_done is not None else None
         d.region_elems, d.arena_elems, d.step = c.region, self.arena.numel(), int(step)
         d.B, d.L, d.Hq, d.Hkv, d.d, d.dtype = c.B, c.L, c.Hq, c.Hkv, c.d, c.code

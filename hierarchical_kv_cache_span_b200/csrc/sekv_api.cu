@@ -286,6 +286,7 @@ struct KeepPlan {
     std::vector<std::pair<int64_t, int64_t>> place;     // (index into the slot table, slot)
     std::vector<uint8_t> dirty;                         // per layer: slot rows to upload
     int64_t hits = 0, spans = 0, bytes_elems = 0, used = 0;
+    int64_t top = -1;                                   // end of the highest entry after the plan
 };
 
 bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
@@ -340,20 +341,25 @@ bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
     // they do not fit are the gaps searched and entries evicted).
     {
         int64_t top = 0, held = 0;
-        for (int b = 0; b < d->B; ++b) {
-            const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
-            const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
-            for (int l = 0; l < d->L; ++l) {
-                const int64_t* sl = d->slot_host + idx(b, l, 0);
-                for (int S = 0; S < m; ++S) {             // branch-free: vectorises
-                    const int64_t sz = bo[S + 1] - bo[S];
-                    const bool r = sl[S] >= 0;
-                    top = std::max(top, r ? sl[S] + sz : 0);
-                    held += r ? sz : 0;
+        if (d->arena_top) {
+            top = *d->arena_top;                          // the caller keeps it with the slot table
+            held = d->arena_used ? *d->arena_used : 0;
+        } else {
+            for (int b = 0; b < d->B; ++b) {
+                const int m = d->m_count_host[b] < d->m_cap ? d->m_count_host[b] : d->m_cap;
+                const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
+                for (int l = 0; l < d->L; ++l) {
+                    const int64_t* sl = d->slot_host + idx(b, l, 0);
+                    for (int S = 0; S < m; ++S) {         // branch-free: vectorises
+                        const int64_t sz = bo[S + 1] - bo[S];
+                        const bool r = sl[S] >= 0;
+                        top = std::max(top, r ? sl[S] + sz : 0);
+                        held += r ? sz : 0;
+                    }
                 }
             }
         }
-        if (top + need <= d->arena_elems) {
+        if (top >= 0 && top + need <= d->arena_elems) {
             kp.used = held;
             for (size_t i = 0; i < miss.size();) {
                 const int b = miss[i].b, l = miss[i].l, Sa = miss[i].S;
@@ -372,6 +378,7 @@ bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
                 kp.dirty[l] = 1;
                 i = j;
             }
+            kp.top = top;
             return true;
         }
     }
@@ -417,6 +424,8 @@ bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
         gaps[off] = size;
     };
     size_t next_victim = 0;
+    std::vector<char> gone((size_t)d->B * d->L * d->m_cap, 0);   // evicted by this plan
+    int64_t top = 0;                                   // end of the highest entry after the plan
     auto alloc = [&](int64_t size) -> int64_t {
         for (;;) {
             for (auto it = gaps.begin(); it != gaps.end(); ++it) {
@@ -428,6 +437,7 @@ bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
             }
             if (next_victim >= cand.size()) return -1;
             const Ent& v = cand[next_victim++];
+            gone[v.id] = 1;
             kp.evict.push_back({v.id, 0});
             kp.dirty[v.l] = 1;
             kp.used -= v.size;
@@ -450,6 +460,7 @@ bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
                 if (off >= 0) {
                     for (int t = Sa; t < S; ++t) kp.place.push_back({idx(b, l, t), off + (bo[t] - bo[Sa])});
                     kp.copies.push_back({src, off, width, b, l});
+                    top = std::max(top, off + width);
                 } else {
                     // no room for the whole run: place its spans one by one
                     for (int t = Sa; t < S; ++t) {
@@ -458,6 +469,7 @@ bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
                         if (o1 < 0) return false;
                         kp.place.push_back({idx(b, l, t), o1});
                         kp.copies.push_back({src + (bo[t] - bo[Sa]), o1, w1, b, l});
+                        top = std::max(top, o1 + w1);
                     }
                 }
                 kp.spans += S - Sa;
@@ -467,6 +479,9 @@ bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
             }
         }
     }
+    for (const Ent& e : occ)
+        if (!gone[e.id]) top = std::max(top, e.off + e.size);
+    kp.top = top;
     return true;
 }
 
@@ -559,6 +574,7 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
             d->stats[4] = (int64_t)kp.evict.size();
         }
         if (d->arena_used) *d->arena_used = kp.used;
+        if (d->arena_top && kp.top >= 0) *d->arena_top = kp.top;
         if ((e = cudaEventRecord(ev, xs)) != cudaSuccess) return cuda_fail(e, "fetch: record");
         return SEKV_OK;
     }

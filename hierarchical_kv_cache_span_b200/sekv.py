@@ -70,7 +70,7 @@ class sekv_fetch_desc(C.Structure):
     _fields_ = [
         ("zmask_dev", _p), ("zmask_host", _p), ("m_count_host", _p), ("blk_off_host", _p),
         ("home", _p), ("arena", _p), ("slot_dev", _p), ("slot_host", _p), ("stats", _p),
-        ("arena_used", _p), ("last_use", _p), ("route_done", _p),
+        ("arena_used", _p), ("arena_top", _p), ("last_use", _p), ("route_done", _p),
         ("region_elems", _i64), ("arena_elems", _i64), ("step", _i64),
         ("B", _i32), ("L", _i32), ("Hq", _i32), ("Hkv", _i32), ("d", _i32), ("dtype", _i32),
         ("l0", _i32), ("l1", _i32), ("m_cap", _i32), ("rank", _i32), ("keep", _i32), ("reserved", _i32),

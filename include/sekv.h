@@ -323,6 +323,11 @@ typedef struct sekv_fetch_desc {
                                      spans already resident (keep mode), spans evicted       */
     int64_t* arena_used;          /* optional host [1], written: arena elements holding bases
                                      after the call                                          */
+    int64_t* arena_top;           /* optional host [1], keep mode: the end (elements) of the
+                                     highest entry placed so far, read and written by every
+                                     call; the caller sets it to 0 together with slot_host.
+                                     Misses that fit above it are placed there without a
+                                     pass over the slot table. NULL: found by that pass.     */
     int64_t* last_use;            /* keep mode: host [B][L][m_cap], the step at which each
                                      resident span was last needed; the caller sets it to -1
                                      (and slot_host to -1) once, the library keeps it        */
@@ -342,8 +347,9 @@ typedef struct sekv_fetch_desc {
                                      [l0, l1) (each as one copy per rectangle of consecutive
                                      spans x consecutive layers).
                                      1: the arena is a device cache across calls: spans zoomed
-                                     again are not copied again. Misses are placed first-fit in
-                                     free space;
+                                     again are not copied again. Misses are placed above the
+                                     highest entry while they fit there, else first-fit in the
+                                     free space below;
                                      when none fits, spans are evicted least recently used
                                      first, never one needed by this call or stamped with this
                                      step or the previous one (ATTEND calls of those steps may
