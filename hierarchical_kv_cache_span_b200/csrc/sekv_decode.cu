@@ -14,20 +14,25 @@
 // shared-memory stages:
 //   bf16: 2-D TMA tensor copies with 128-byte swizzle; each consumer warp takes
 //         16 rows of a 64-row tile and runs q.K^T and p.V on the tensor cores
-//         (mma.sync m16n8k16, the G query heads of the kv head padded to M = 16:
-//         GQA, one K/V read serves all G heads). The q.kbar accumulator of a span
-//         row is both its routing logit and its coarse attention logit.
+//         (mma.sync m16n8k16, the rows on M and the G query heads of the kv head
+//         on N, padded to 8: GQA, one K/V read serves all G heads). The q.kbar
+//         accumulator of a span row is both its routing logit and its coarse
+//         attention logit. A routing pass loads key tiles only, two per stage.
 //   fp32: 1-D bulk copies and CUDA-core dot products (each lane owns d/32 dims,
 //         a 32-way transpose-reduce finishes the dots).
 // Spans zoomed by any head of the group are queued. Phase 2 attends them without
 // materialising K_S (u = B_S q, scores A_S u, y = C_S^T p, contribution y^T D_S):
 //   bf16: the producer warp streams each queued span's factor pieces through one
-//         CTA-wide ring; the four consumer warps share every span, 16 tokens at a
-//         time, on the tensor cores with u, p and y held in registers.
+//         CTA-wide ring; the consumer warps share every span (all four, or one
+//         pair for ranks above 16), 32 tokens at a time, on the tensor cores with
+//         u, p and y held in registers. With the mask given and a grid of about
+//         one wave, the unit's zoomed token units are dealt evenly over its splits
+//         instead.
 //   fp32: each consumer warp pulls whole spans and streams them through its own
 //         3-slot ring, on the CUDA cores.
-// Softmax state is kept in the log2 domain; the CTA merges its warps' states, a
-// second small kernel merges the splits by log-sum-exp.
+// Softmax state is kept in the log2 domain; the CTA merges its warps' states, and
+// the last CTA of each (b, l, kv head) to finish merges the splits by log-sum-exp
+// (arrival counters; without them a second small kernel does).
 #include <cuda.h>
 
 #include <cmath>
