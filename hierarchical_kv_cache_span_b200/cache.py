@@ -271,6 +271,7 @@ class ColdFetcher:
         d = S.sekv_fetch_desc()
         d.zmask_dev, d.zmask_host = _ptr(zmask), _ptr(self.zmask_host)
         d.m_count_host, d.blk_off_host = _ptr(self.m_count_host), _ptr(self.blk_off_host)
+        d.blk_off_dev = _ptr(c.blk_off)
         d.home, d.arena = _ptr(c.home), _ptr(self.arena)
         d.slot_dev, d.slot_host, d.stats = _ptr(self.slot_dev), _ptr(self.slot_host), _ptr(self.stats)
         d.arena_used, d.last_use = _ptr(self.arena_used), _ptr(self.last_use) if self.keep else None

@@ -269,6 +269,59 @@ sekv_status sekv_tau_to_theta(const double* tau, float* theta, int64_t n) {
 
 }  // extern "C"
 
+namespace sekv {
+
+// Refill-mode gather (SeKV summary, workflow paragraph: the bases of the zoomed
+// spans are fetched from the CPU). One CTA per (b, layer, kv head) and
+// chunk: the spans zoomed by any query head of the kv head's group, in span order,
+// are dealt over the unit's nch chunks; a CTA copies the kv head's block of each of
+// its spans from the home (pinned host memory read through unified addressing) to
+// the span's arena slot. Blocks are multiples of 128 bytes (64 elements) and start
+// at multiples of 64 elements, so 16-byte vectors cover them exactly.
+__global__ void __launch_bounds__(256) fetch_gather_kernel(const uint32_t* zmask, const int64_t* blk_off,
+                                                           const int64_t* slot, const char* home, char* arena,
+                                                           int64_t region, int L, int l0, int Lr, int Hq, int Hkv,
+                                                           int m_cap, int es, int nch) {
+    const int unit = blockIdx.x / nch, ch = blockIdx.x % nch;
+    const int kvh = unit % Hkv, bl = unit / Hkv, b = bl / Lr, l = l0 + bl % Lr;
+    const int G = Hq / Hkv, mw = m_cap / 32;
+    const uint32_t* zm = zmask + (((int64_t)b * L + l) * Hq + (int64_t)kvh * G) * mw;
+    const int64_t* bo = blk_off + (int64_t)b * (m_cap + 1);
+    const int64_t* sl = slot + ((int64_t)b * L + l) * m_cap;
+    const int64_t rbase = ((int64_t)b * L + l) * region;
+    constexpr int U = 4;                                    // 16-byte vectors in flight per thread
+    int rank = 0;                                           // zoomed spans passed so far
+    for (int w = 0; w < mw; ++w) {
+        uint32_t u = 0u;
+        for (int g = 0; g < G; ++g) u |= zm[(int64_t)g * mw + w];
+        for (; u; u &= u - 1u) {
+            const int S = w * 32 + __ffs(u) - 1;
+            if (rank++ % nch != ch) continue;
+            const int64_t off = sl[S];
+            if (off < 0) continue;
+            const int64_t be = (bo[S + 1] - bo[S]) / Hkv;   // elements of one kv head's block
+            const uint4* src = reinterpret_cast<const uint4*>(home + (rbase + bo[S] + kvh * be) * es);
+            uint4* dst = reinterpret_cast<uint4*>(arena + (off + kvh * be) * es);
+            const int64_t n16 = be * es / 16;
+            for (int64_t i = threadIdx.x; i < n16; i += (int64_t)U * blockDim.x) {
+                uint4 v[U];
+#pragma unroll
+                for (int k = 0; k < U; ++k) {
+                    const int64_t j = i + (int64_t)k * blockDim.x;
+                    v[k] = j < n16 ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int k = 0; k < U; ++k) {
+                    const int64_t j = i + (int64_t)k * blockDim.x;
+                    if (j < n16) dst[j] = v[k];
+                }
+            }
+        }
+    }
+}
+
+}  // namespace sekv
+
 namespace {
 
 // Keep mode: the arena as a cache of span entries across calls. Entry (b, l, S)
@@ -661,6 +714,63 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
                     (long long)end, (long long)d->arena_elems);
     }
     if (d->arena_used) *d->arena_used = end;
+    // With the device block offsets and a home the device can address, one gather
+    // kernel moves only the kv-head blocks the kv groups zoom (the copy engine would
+    // move every zoomed span's Hkv blocks, and pays a fixed cost per copy).
+    const char* home_dev = nullptr;
+    if (d->blk_off_dev) {
+        cudaPointerAttributes pa;
+        if (cudaPointerGetAttributes(&pa, d->home) == cudaSuccess) {
+            if (pa.type == cudaMemoryTypeHost && pa.devicePointer) home_dev = reinterpret_cast<const char*>(pa.devicePointer);
+            else if (pa.type == cudaMemoryTypeDevice || pa.type == cudaMemoryTypeManaged) home_dev = home;
+        } else {
+            (void)cudaGetLastError();                   // an unregistered host pointer: not an error here
+        }
+    }
+    if (home_dev) {
+        for (int b = 0; b < d->B; ++b) {
+            const int64_t o = ((int64_t)b * d->L + d->l0) * d->m_cap;
+            if ((e = cudaMemcpyAsync(d->slot_dev + o, d->slot_host + o, sizeof(int64_t) * Lr * d->m_cap,
+                                     cudaMemcpyHostToDevice, xs)) != cudaSuccess)
+                return cuda_fail(e, "fetch: slot upload");
+        }
+        const int G = d->Hq / d->Hkv;
+        int64_t blocks = 0, bytes = 0;
+        for (int b = 0; b < d->B; ++b) {
+            const int64_t* bo = d->blk_off_host + (int64_t)b * (d->m_cap + 1);
+            for (int l = d->l0; l < d->l1; ++l)
+                for (int kvh = 0; kvh < d->Hkv; ++kvh) {
+                    const uint32_t* zm = d->zmask_host + (((int64_t)b * d->L + l) * d->Hq + (int64_t)kvh * G) * mw;
+                    const int64_t* sl = d->slot_host + ((int64_t)b * d->L + l) * d->m_cap;
+                    for (int w = 0; w < mw; ++w) {
+                        uint32_t u = 0u;
+                        for (int g = 0; g < G; ++g) u |= zm[(int64_t)g * mw + w];
+                        for (; u; u &= u - 1u) {
+                            const int S = (w << 5) + __builtin_ctz(u);
+                            if (sl[S] < 0) continue;
+                            ++blocks;
+                            bytes += (bo[S + 1] - bo[S]) / d->Hkv * es;
+                        }
+                    }
+                }
+        }
+        if (d->stats) {
+            d->stats[0] = bytes;
+            d->stats[2] = blocks;
+        }
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            sms = 148;
+        const int64_t units = (int64_t)d->B * Lr * d->Hkv;
+        const int nch = (int)std::max<int64_t>(1, std::min<int64_t>(32, (8 * (int64_t)sms + units - 1) / units));
+        if (units * nch > 0x7fffffff) return fail(SEKV_ERR_INVALID_ARG, "fetch: too many (b, layer, kv head) units");
+        sekv::fetch_gather_kernel<<<(unsigned)(units * nch), 256, 0, xs>>>(
+            d->zmask_dev, d->blk_off_dev, d->slot_dev, home_dev, arena, d->region_elems, d->L, d->l0, Lr, d->Hq,
+            d->Hkv, d->m_cap, (int)es, nch);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "fetch: gather");
+        if ((e = cudaEventRecord(ev, xs)) != cudaSuccess) return cuda_fail(e, "fetch: record");
+        return SEKV_OK;
+    }
     for (const Rect& r : rects) {
         if (r.height == 1)
             e = cudaMemcpyAsync(arena + r.dst * es, home + r.src * es, r.width * es, cudaMemcpyHostToDevice, xs);

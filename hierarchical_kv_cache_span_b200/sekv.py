@@ -68,7 +68,7 @@ class sekv_decode_desc(C.Structure):
 
 class sekv_fetch_desc(C.Structure):
     _fields_ = [
-        ("zmask_dev", _p), ("zmask_host", _p), ("m_count_host", _p), ("blk_off_host", _p),
+        ("zmask_dev", _p), ("zmask_host", _p), ("m_count_host", _p), ("blk_off_host", _p), ("blk_off_dev", _p),
         ("home", _p), ("arena", _p), ("slot_dev", _p), ("slot_host", _p), ("stats", _p),
         ("arena_used", _p), ("arena_top", _p), ("last_use", _p), ("route_done", _p),
         ("region_elems", _i64), ("arena_elems", _i64), ("step", _i64),

@@ -315,6 +315,13 @@ typedef struct sekv_fetch_desc {
     uint32_t* zmask_host;         /* pinned host staging of the same shape                   */
     const int32_t* m_count_host;  /* [B] host copy of m_count                                */
     const int64_t* blk_off_host;  /* [B][m_cap+1] host copy of blk_off                       */
+    const int64_t* blk_off_dev;   /* optional [B][m_cap+1] device blk_off. Refill mode with it:
+                                     one gather kernel reads the home through unified
+                                     addressing and copies, for each (b, l, kv head), only
+                                     that kv head's block of the spans its query heads zoom
+                                     (the slot table still reserves a span's Hkv blocks). NULL,
+                                     or a home the device cannot address: copy-engine copies
+                                     of every zoomed span's Hkv blocks.                      */
     const void* home;             /* pinned host basis home [B][L][region_elems]             */
     void* arena;                  /* device arena, arena_elems elements                      */
     int64_t* slot_dev;            /* [B][L][m_cap] device slot table (written on `copy`)     */
@@ -364,7 +371,8 @@ typedef struct sekv_fetch_desc {
  * get -1). The routing result is read back first (see route_done; the host waits
  * for it); the copies and the slot-table upload go on `copy`; `done` is recorded on
  * `copy`. The caller makes `compute` wait on `done` before ATTEND. stats[2] counts
- * the copies (cudaMemcpyAsync, or cudaMemcpy2DAsync for a rectangle). Returns
+ * the copies (cudaMemcpyAsync, or cudaMemcpy2DAsync for a rectangle; with the gather
+ * kernel, the kv-head blocks it moves). Returns
  * SEKV_ERR_CAPACITY, with nothing copied and both slot tables as they were, when
  * the zoomed bases that are not resident do not fit (keep mode: after every
  * allowed eviction). */
