@@ -320,6 +320,37 @@ __global__ void __launch_bounds__(256) fetch_gather_kernel(const uint32_t* zmask
     }
 }
 
+// Keep-mode gather: up to kGatherRuns contiguous runs (whole entries: every kv
+// head's block of consecutive spans of one (b, l)) per launch, passed by value;
+// nch CTAs share a run, each a contiguous share of its 16-byte vectors.
+constexpr int kGatherRuns = 256;
+struct GatherRuns {
+    int64_t src[kGatherRuns], dst[kGatherRuns], n16[kGatherRuns];   // byte offsets / 16, vector counts
+    int count;
+};
+__global__ void __launch_bounds__(256) run_gather_kernel(const __grid_constant__ GatherRuns gr, const char* home,
+                                                         char* arena, int nch) {
+    const int r = blockIdx.x / nch, ch = blockIdx.x % nch;
+    if (r >= gr.count) return;
+    const int64_t n = gr.n16[r], per = (n + nch - 1) / nch, i0 = ch * per, i1 = min(n, i0 + per);
+    const uint4* src = reinterpret_cast<const uint4*>(home) + gr.src[r];
+    uint4* dst = reinterpret_cast<uint4*>(arena) + gr.dst[r];
+    constexpr int U = 4;
+    for (int64_t i = i0 + threadIdx.x; i < i1; i += (int64_t)U * blockDim.x) {
+        uint4 v[U];
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int64_t j = i + (int64_t)k * blockDim.x;
+            v[k] = j < i1 ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const int64_t j = i + (int64_t)k * blockDim.x;
+            if (j < i1) dst[j] = v[k];
+        }
+    }
+}
+
 }  // namespace sekv
 
 namespace {
@@ -542,6 +573,19 @@ bool plan_keep(const sekv_fetch_desc* d, KeepPlan& kp) {
 
 extern "C" {
 
+// The home's device address when the device can read it (pinned or registered host
+// memory through unified addressing, or device memory), else null.
+static const char* device_home(const void* home) {
+    cudaPointerAttributes pa;
+    if (cudaPointerGetAttributes(&pa, home) != cudaSuccess) {
+        (void)cudaGetLastError();                       // an unregistered host pointer: not an error here
+        return nullptr;
+    }
+    if (pa.type == cudaMemoryTypeHost && pa.devicePointer) return reinterpret_cast<const char*>(pa.devicePointer);
+    if (pa.type == cudaMemoryTypeDevice || pa.type == cudaMemoryTypeManaged) return reinterpret_cast<const char*>(home);
+    return nullptr;
+}
+
 sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, sekv_stream_t copy,
                              sekv_event_t done) {
     SEKV_REQUIRE(d, "fetch: null descriptor");
@@ -600,10 +644,33 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
             d->last_use[p.first] = d->step;
         }
         for (const int64_t i : kp.hit) d->last_use[i] = d->step;     // hits are stamped too
-        for (const auto& c : kp.copies)
-            if ((e = cudaMemcpyAsync(arena + c.dst * es, home + c.src * es, c.width * es, cudaMemcpyHostToDevice,
-                                     xs)) != cudaSuccess)
-                return cuda_fail(e, "fetch: basis copy");
+        // the placed runs: by a gather kernel when the device can read the home (no
+        // fixed cost per run), else one copy-engine copy each
+        const char* hd = kp.copies.empty() ? nullptr : device_home(d->home);
+        if (hd) {
+            int dev = 0, sms = 148;
+            if (cudaGetDevice(&dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                sms = 148;
+            for (size_t c0 = 0; c0 < kp.copies.size(); c0 += sekv::kGatherRuns) {
+                sekv::GatherRuns gr;
+                gr.count = (int)std::min<size_t>(sekv::kGatherRuns, kp.copies.size() - c0);
+                for (int k = 0; k < gr.count; ++k) {
+                    const auto& c = kp.copies[c0 + k];
+                    gr.src[k] = c.src * es / 16;
+                    gr.dst[k] = c.dst * es / 16;
+                    gr.n16[k] = c.width * es / 16;
+                }
+                const int nch = std::max(1, std::min(16, (4 * sms + gr.count - 1) / gr.count));
+                sekv::run_gather_kernel<<<gr.count * nch, 256, 0, xs>>>(gr, hd, arena, nch);
+                if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "fetch: gather");
+            }
+        } else {
+            for (const auto& c : kp.copies)
+                if ((e = cudaMemcpyAsync(arena + c.dst * es, home + c.src * es, c.width * es, cudaMemcpyHostToDevice,
+                                         xs)) != cudaSuccess)
+                    return cuda_fail(e, "fetch: basis copy");
+        }
         // the slot rows of the layers that changed: one copy per sequence over the
         // range from the first to the last such layer (the copy engine's fixed cost
         // per copy outweighs the few unchanged rows in between)
@@ -717,16 +784,7 @@ sekv_status sekv_fetch_bases(const sekv_fetch_desc* d, sekv_stream_t compute, se
     // With the device block offsets and a home the device can address, one gather
     // kernel moves only the kv-head blocks the kv groups zoom (the copy engine would
     // move every zoomed span's Hkv blocks, and pays a fixed cost per copy).
-    const char* home_dev = nullptr;
-    if (d->blk_off_dev) {
-        cudaPointerAttributes pa;
-        if (cudaPointerGetAttributes(&pa, d->home) == cudaSuccess) {
-            if (pa.type == cudaMemoryTypeHost && pa.devicePointer) home_dev = reinterpret_cast<const char*>(pa.devicePointer);
-            else if (pa.type == cudaMemoryTypeDevice || pa.type == cudaMemoryTypeManaged) home_dev = home;
-        } else {
-            (void)cudaGetLastError();                   // an unregistered host pointer: not an error here
-        }
-    }
+    const char* home_dev = d->blk_off_dev ? device_home(d->home) : nullptr;
     if (home_dev) {
         for (int b = 0; b < d->B; ++b) {
             const int64_t o = ((int64_t)b * d->L + d->l0) * d->m_cap;
