@@ -114,7 +114,7 @@ __host__ __device__ __forceinline__ int64_t tile8_index(int64_t r, int c, int w8
 }
 
 // ---------------------------------------------------------------------------
-// mbarrier + bulk copy (1-D, global -> shared, no multicast)
+// mbarrier + bulk copy (1-D, global -> this CTA's shared memory)
 // ---------------------------------------------------------------------------
 SEKV_DEV uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -212,7 +212,7 @@ SEKV_DEV uint32_t pack_bf16(float lo, float hi) {
     return r;
 }
 
-// 2-D tensor-map bulk copy (TMA) global -> shared, no multicast
+// 2-D tensor-map bulk copy (TMA) global -> this CTA's shared memory
 SEKV_DEV void tma_load_2d(void* dst_smem, const void* tmap, int x, int y, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
