@@ -493,12 +493,13 @@ def run_sekv(args, rank, world, local_rank):
     sid = comp.cuda_stream
     bud = args.budget
     if cold:
-        d_route = cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud)
+        d_route = cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud, static_ready=True)
         d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_ATTEND, O=O, lse=lse, slot=fetcher.slot_dev,
-                                   arena=fetcher.arena, zmask=zm, budget=bud, zoom_hint=zoom_hint)
+                                   arena=fetcher.arena, zmask=zm, budget=bud, zoom_hint=zoom_hint,
+                                   static_ready=True)
     else:
         d_attn = cache.decode_desc(q_buf, theta, phase=P.SEKV_FUSED, O=O, lse=lse, zmask=zm, budget=bud,
-                                   zoom_hint=zoom_hint)
+                                   zoom_hint=zoom_hint, static_ready=True)
 
     def one_step(q, rec=None):
         if q is not None:
@@ -757,7 +758,7 @@ def latency_form(P, torch, cache, wl, q_buf, q, theta, O, lse, zm, fetcher, cold
     try:
         q_buf.copy_(q)
         if cold:
-            dr_ = cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud)
+            dr_ = cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud, static_ready=True)
             P.check(P.sekv.sekv_decode_attn(dr_, torch.cuda.current_stream().cuda_stream), "route")
             fetcher.fetch(zm)
             torch.cuda.current_stream().wait_event(fetcher.done)
@@ -766,10 +767,10 @@ def latency_form(P, torch, cache, wl, q_buf, q, theta, O, lse, zm, fetcher, cold
             if cold:
                 descs.append(cache.decode_desc(q_buf, theta, phase=P.SEKV_ATTEND, O=O, lse=lse,
                                                slot=fetcher.slot_dev, arena=fetcher.arena, zmask=zm, budget=bud,
-                                               zoom_hint=zoom_hint, l0=l, l1=l + 1))
+                                               zoom_hint=zoom_hint, l0=l, l1=l + 1, static_ready=True))
             else:
                 descs.append(cache.decode_desc(q_buf, theta, phase=P.SEKV_FUSED, O=O, lse=lse, zmask=zm,
-                                               budget=bud, zoom_hint=zoom_hint, l0=l, l1=l + 1))
+                                               budget=bud, zoom_hint=zoom_hint, l0=l, l1=l + 1, static_ready=True))
         torch.cuda.synchronize()
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
@@ -816,11 +817,11 @@ def prefetch_pipeline(P, torch, cache, wl, q_buf, qpool, theta, O, lse, zm, aren
         fetcher = P.ColdFetcher(cache, arena_elems=arena_elems, keep=True)
         comp = torch.cuda.current_stream()
         sid = comp.cuda_stream
-        route = [cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud, l0=l, l1=l + 1)
-                 for l in range(wl.L)]
+        route = [cache.decode_desc(q_buf, theta, phase=P.SEKV_ROUTE, zmask=zm, budget=bud, l0=l, l1=l + 1,
+                                   static_ready=True) for l in range(wl.L)]
         attend = [cache.decode_desc(q_buf, theta, phase=P.SEKV_ATTEND, O=O, lse=lse, slot=fetcher.slot_dev,
-                                    arena=fetcher.arena, zmask=zm, budget=bud, zoom_hint=zoom_hint, l0=l, l1=l + 1)
-                  for l in range(wl.L)]
+                                    arena=fetcher.arena, zmask=zm, budget=bud, zoom_hint=zoom_hint, l0=l, l1=l + 1,
+                                    static_ready=True) for l in range(wl.L)]
         evs = [torch.cuda.Event() for _ in range(wl.L)]
         stats = {"bytes": 0, "copies": 0, "resident": 0, "spans": 0, "evicted": 0}
 

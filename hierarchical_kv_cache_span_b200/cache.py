@@ -166,7 +166,12 @@ class SpanCache:
     # ------------------------------------------------------------------ decode
     def decode_desc(self, q, theta, phase=S.SEKV_FUSED, scale=None, O=None, lse=None, zmask=None,
                     route_logits=None, nsplit=0, slot=None, arena=None, l0=0, l1=None,
-                    workspace=None, rows_hint=None, budget=0, zoom_hint=0) -> S.sekv_decode_desc:
+                    workspace=None, rows_hint=None, budget=0, zoom_hint=0,
+                    static_ready=False) -> S.sekv_decode_desc:
+        """static_ready=True promises that nothing still in flight on the stream writes
+        the cache's build outputs (e.g. the stream was synchronised after build()), so
+        the kernels may read the counts and their first tiles while the previous kernel
+        finishes (sekv_decode_desc.static_ready)."""
         d = S.sekv_decode_desc()
         d.q = _ptr(q)
         d.a_count, d.m_count, d.span_beg, d.span_end = (_ptr(self.a_count), _ptr(self.m_count),
@@ -193,6 +198,7 @@ class SpanCache:
         d.rows_hint = self.rows_hint if rows_hint is None else int(rows_hint)
         d.budget = int(budget)
         d.zoom_hint = int(zoom_hint)
+        d.static_ready = 1 if static_ready else 0
         need = S.sekv_decode_workspace_bytes(d)
         if workspace is None:
             key = (d.l0, d.l1, nsplit, d.rows_hint, d.budget > 0 and phase != S.SEKV_ATTEND)

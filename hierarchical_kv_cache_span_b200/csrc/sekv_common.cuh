@@ -158,6 +158,12 @@ SEKV_DEV void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uin
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(smem_u32(dst_smem)), "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
+// 16 bytes global -> this thread's shared memory, cached in L2 only (both addresses
+// 16-byte aligned); visible to the issuing thread after cp_async_wait_all()
+SEKV_DEV void cp_async16(void* dst_smem, const void* src_gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
+}
+SEKV_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // warp-level tensor-core helpers (ldmatrix + mma.sync m16n8k16 bf16 -> fp32)

@@ -133,6 +133,7 @@ struct DecArgs {
     int zwords;       // zoom-mask words per head in shared memory (the split's span range)
     uint32_t polls;   // poll limit of every bounded barrier wait
     int starve;       // test hook: the producer issues no copy, so every wait runs out
+    int static_ready; // the build outputs are settled: counts and first tiles are read before the dependency wait
     uint32_t* arrive; // [B][L][Hkv] arrival counters (the last CTA of a unit merges), or null
     float* O;         // [B][L][Hq][D] and [B][L][Hq]: written by the merging CTA
     float* lse;
@@ -1251,27 +1252,41 @@ SEKV_DEV void store_state_lanes(const DecSmem& sm, int idx, int lane, const floa
 // log-sum-exp, in split order, with the arithmetic of merge_kernel below (so the
 // two forms give the same bits): M = max_j m_j, L = sum_j l_j 2^(m_j - M),
 // O = sum_j o_j 2^(m_j - M) / L, lse = (M + log2 L) ln 2. The partials of the
-// other CTAs are read past L1 (they were written by other SMs).
-template <int D, int G>
+// other CTAs are read past L1 (they were written by other SMs). All of a thread's
+// loads are issued before the factors are formed: the first PS splits' output
+// quads as asynchronous copies into the free stage memory (RINGB bytes), up to KT
+// more into registers, and the (m, l) pairs; only splits beyond those wait for the
+// factors.
+template <int D, int G, int RINGB>
 SEKV_DEV void merge_unit(const DecArgs& a, const DecSmem& sm, int64_t lunit, int b, int l, int kvh, int tid) {
     constexpr int NT = (kNW + 1) * 32;
-    constexpr int KB = 16;                                      // splits' loads in flight per thread
+    constexpr int NQ = G * D / 4;                               // output quads of the unit
+    constexpr int QPT = (NQ + NT - 1) / NT;                     // quads per thread
+    constexpr int KT = 16 / QPT;                                // split quads per output quad in registers
+    constexpr int KB = 16;                                      // loads per round past those
     const int ns = a.nsplit;
     const int lane = tid & 31, warp = tid >> 5;
     float* fac = reinterpret_cast<float*>(sm.stages);          // [G][ns] m_j, then 2^(m_j - M) (the ring is free)
     float* lsv = fac + G * ns;                                  // [G][ns] l_j
     float* Mh = lsv + G * ns;                                   // [G]
     float* Lh = Mh + G;                                         // [G]
-    // this thread's first output quad: its first KB splits are loaded now, so they
-    // arrive while the factors are formed
-    constexpr int K0 = 8;
-    const int i0 = tid;
-    const float4* po0 = reinterpret_cast<const float4*>(a.part_o + (lunit * G + i0 / (D / 4)) * ns * D) + i0 % (D / 4);
-    float4 v0[K0];
+    const int off = ((2 * G * ns + 2 * G) * 4 + 15) & ~15;
+    const int PS = max(0, min(ns, (RINGB - off) / (NQ * 16))); // splits staged in shared memory
+    unsigned char* stg = sm.stages + off;                       // [PS][NQ] quads
+    const int PT = min(ns - PS, KT);                            // splits in registers
+    float4 vt[QPT][KT];
 #pragma unroll
-    for (int k = 0; k < K0; ++k)
-        v0[k] = (i0 < G * D / 4 && k < ns) ? __ldcg(po0 + (int64_t)k * (D / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    // every (head, split) pair's (m, l) in one round of loads
+    for (int qq = 0; qq < QPT; ++qq) {
+        const int i = tid + qq * NT;
+        if (i < NQ) {
+            const float4* po = reinterpret_cast<const float4*>(a.part_o + (lunit * G + i / (D / 4)) * ns * D) + i % (D / 4);
+            for (int j = 0; j < PS; ++j) cp_async16(stg + ((size_t)j * NQ + i) * 16, po + (int64_t)j * (D / 4));
+#pragma unroll
+            for (int k = 0; k < KT; ++k)
+                vt[qq][k] = k < PT ? __ldcg(po + (int64_t)(PS + k) * (D / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    // every (head, split) pair's (m, l)
     const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + lunit * G * ns;
     for (int i = tid; i < G * ns; i += NT) {
         const float2 v = __ldcg(ml + i);
@@ -1289,36 +1304,47 @@ SEKV_DEV void merge_unit(const DecArgs& a, const DecSmem& sm, int64_t lunit, int
         __syncwarp();
         if (lane == 0) {
             float Ls = 0.f;
-            if (M != -INFINITY)
-                for (int j = 0; j < ns; ++j) Ls = fmaf(lsv[h * ns + j], fh[j], Ls);
+            if (M != -INFINITY) {
+                const float* lh = lsv + h * ns;
+#pragma unroll 8
+                for (int j = 0; j < ns; ++j) Ls = fmaf(lh[j], fh[j], Ls);
+            }
             Mh[h] = M;
             Lh[h] = Ls;
         }
     }
     __syncthreads();
+    cp_async_wait_all();
     // four output dims per thread: O = sum_j o_j f_j / L, summed in split order
-    for (int i = tid; i < G * D / 4; i += NT) {
+#pragma unroll
+    for (int qq = 0; qq < QPT; ++qq) {
+        const int i = tid + qq * NT;
+        if (i >= NQ) continue;
         const int h = i / (D / 4), k4 = i % (D / 4);
         const float M = Mh[h], Ls = Lh[h];
         const float* fj = fac + h * ns;
-        const float4* po = reinterpret_cast<const float4*>(a.part_o + (lunit * G + h) * ns * D) + k4;
         float4 os = make_float4(0.f, 0.f, 0.f, 0.f);
-        int js = 0;
-        if (M != -INFINITY && i == i0) {
+        if (M != -INFINITY) {
+            for (int j = 0; j < PS; ++j) {
+                const float4 v = *reinterpret_cast<const float4*>(stg + ((size_t)j * NQ + i) * 16);
+                const float f = fj[j];
+                os.x = fmaf(v.x, f, os.x);
+                os.y = fmaf(v.y, f, os.y);
+                os.z = fmaf(v.z, f, os.z);
+                os.w = fmaf(v.w, f, os.w);
+            }
 #pragma unroll
-            for (int k = 0; k < K0; ++k) {
-                if (k < ns) {
-                    const float f = fj[k];
-                    os.x = fmaf(v0[k].x, f, os.x);
-                    os.y = fmaf(v0[k].y, f, os.y);
-                    os.z = fmaf(v0[k].z, f, os.z);
-                    os.w = fmaf(v0[k].w, f, os.w);
+            for (int k = 0; k < KT; ++k) {
+                if (k < PT) {
+                    const float f = fj[PS + k];
+                    os.x = fmaf(vt[qq][k].x, f, os.x);
+                    os.y = fmaf(vt[qq][k].y, f, os.y);
+                    os.z = fmaf(vt[qq][k].z, f, os.z);
+                    os.w = fmaf(vt[qq][k].w, f, os.w);
                 }
             }
-            js = K0;
-        }
-        if (M != -INFINITY) {
-            for (int j0 = js; j0 < ns; j0 += KB) {
+            const float4* po = reinterpret_cast<const float4*>(a.part_o + (lunit * G + h) * ns * D) + k4;
+            for (int j0 = PS + PT; j0 < ns; j0 += KB) {
                 float4 v[KB];
 #pragma unroll
                 for (int k = 0; k < KB; ++k)
@@ -1353,11 +1379,16 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     using C = DecCfg<DT, D, G>;
     constexpr int DPL = C::DPL, R = C::R, TR = C::TR, NS = C::NS;
     // Programmatic dependent launch: the grid may be scheduled while the previous
-    // kernel on the stream finishes; nothing is read before that kernel has
-    // completed and its writes are visible. Once every CTA of this grid has started,
+    // kernel on the stream finishes; no input is read before that kernel has
+    // completed and its writes are visible, except (static_ready: the caller
+    // guarantees that nothing in flight writes them) the cache's counts and the
+    // first anchor / summary tiles. Once every CTA of this grid has passed the wait,
     // the next kernel may be scheduled likewise.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const bool pre = a.static_ready != 0;
+    if (!pre) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    }
     extern __shared__ __align__(1024) unsigned char sm_raw[];
     unsigned char* base = sm_raw + ((1024 - (smem_u32(sm_raw) & 1023)) & 1023);
     const int zwords = a.zwords;
@@ -1377,8 +1408,41 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     const int64_t lunit = ((int64_t)b * a.Lr + li) * a.Hkv + kvh;         // within this launch
     const bool route_only = a.phase == SEKV_ROUTE;
 
-    const int ab = min(a.a_count[b], a.a_cap);
-    const int mb = min(a.m_count[b], a.m_cap);
+    // The loads that need no count are issued together with the counts, so their
+    // latencies overlap: the G query rows (held in registers until they are stored to
+    // shared memory below), the consumer lanes' thresholds and, when the unit's whole
+    // mask is dealt from, its mask words.
+    constexpr int NT = (kNW + 1) * 32;
+    constexpr int QV = G * C::ROWB / 16;                  // 16-byte pieces of the G query rows
+    constexpr int QPT = (QV + NT - 1) / NT;
+    const uint4* qg = reinterpret_cast<const uint4*>(a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB);
+    uint4 qv[QPT];
+    float thp[2] = {INFINITY, INFINITY};                  // heads 2c, 2c+1 of a consumer lane
+    const bool zpre = C::MMA && a.zin && a.deal;          // words 0 .. zwords-1 of the unit's mask
+    constexpr int ZPT = C::MMA ? (kDealMaskBytes / 4 + NT - 1) / NT : 1;
+    uint32_t zv[ZPT];
+    auto load_inputs = [&]() {
+#pragma unroll
+        for (int k = 0; k < QPT; ++k)
+            if (tid + k * NT < QV) qv[k] = qg[tid + k * NT];
+        if (C::MMA && warp < kNW) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                if (2 * (lane & 3) + hh < G) thp[hh] = a.theta[(int64_t)l * a.Hq + kvh * G + 2 * (lane & 3) + hh];
+        }
+        if (zpre) {
+#pragma unroll
+            for (int k = 0; k < ZPT; ++k) {
+                const int i = tid + k * NT;
+                zv[k] = i < G * zwords
+                            ? a.zmask[(((int64_t)b * a.L + l) * a.Hq + kvh * G + i / zwords) * a.mw + i % zwords]
+                            : 0u;
+            }
+        }
+    };
+    if (!pre) load_inputs();
+    const int ab = min(__ldcg(a.a_count + b), a.a_cap);     // past L1: may be read before the wait
+    const int mb = min(__ldcg(a.m_count + b), a.m_cap);
     int a0 = 0, a1 = 0;
     if (!route_only) {
         const int ach = (ab + a.nsplit - 1) / a.nsplit;
@@ -1472,27 +1536,44 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         if (!a.starve)
             for (int i = 0; i < early; ++i) issue_tile(i);
     }
+    if (pre) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+        load_inputs();
+    }
     // zoom-mask words: routed in this kernel (zero here, bits or-ed in by the stream),
     // or (tensor-core path, zin) the caller's mask: the split's words, or with deal the
     // unit's, bits of spans outside them cleared
     const int zbase = a.deal ? 0 : s0;          // span of bit 0 of word 0
     const int zend = a.deal ? mb : s1;          // spans >= zend are not in the words
-    for (int i = tid; i < G * zwords; i += blockDim.x) {
-        uint32_t v = 0u;
-        if (C::MMA && a.zin) {
-            const int h = i / zwords, w = i % zwords;
-            const int S = zbase + 32 * w;
-            if (S < zend) {
-                v = a.zmask[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.mw + (S >> 5)];
-                if (zend - S < 32) v &= (1u << (zend - S)) - 1u;
+    if (zpre) {
+#pragma unroll
+        for (int k = 0; k < ZPT; ++k) {
+            const int i = tid + k * NT;
+            if (i < G * zwords) {
+                const int S = 32 * (i % zwords);
+                uint32_t v = S < zend ? zv[k] : 0u;
+                if (S < zend && zend - S < 32) v &= (1u << (zend - S)) - 1u;
+                sm.zw[i] = v;
             }
         }
-        sm.zw[i] = v;
+    } else {
+        for (int i = tid; i < G * zwords; i += blockDim.x) {
+            uint32_t v = 0u;
+            if (C::MMA && a.zin) {
+                const int h = i / zwords, w = i % zwords;
+                const int S = zbase + 32 * w;
+                if (S < zend) {
+                    v = a.zmask[(((int64_t)b * a.L + l) * a.Hq + kvh * G + h) * a.mw + (S >> 5)];
+                    if (zend - S < 32) v &= (1u << (zend - S)) - 1u;
+                }
+            }
+            sm.zw[i] = v;
+        }
     }
-    {
-        const uint4* qg = reinterpret_cast<const uint4*>(a.q + (((int64_t)b * a.L + l) * a.Hq + (int64_t)kvh * G) * C::ROWB);
-        for (int i = tid; i < G * C::ROWB / 16; i += blockDim.x) reinterpret_cast<uint4*>(sm.qs)[i] = qg[i];
-    }
+#pragma unroll
+    for (int k = 0; k < QPT; ++k)
+        if (tid + k * NT < QV) reinterpret_cast<uint4*>(sm.qs)[tid + k * NT] = qv[k];
     if (C::MMA && a.deal)
         for (int w = tid; w < zwords; w += blockDim.x) sm.zu[w] = 0;
     __syncthreads();
@@ -1557,8 +1638,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
         // and its coarse attention logit.
         constexpr uint32_t FULL = 0xffffffffu;
         const int g = lane >> 2, c = lane & 3, lj = lane >> 3, lr = lane & 7;
-        const float th0 = 2 * c < G ? a.theta[(int64_t)l * a.Hq + kvh * G + 2 * c] : INFINITY;
-        const float th1 = 2 * c + 1 < G ? a.theta[(int64_t)l * a.Hq + kvh * G + 2 * c + 1] : INFINITY;
+        const float th0 = thp[0], th1 = thp[1];
         {
             const uint32_t* qp = reinterpret_cast<const uint32_t*>(sm.qs + (g < G ? g : 0) * C::ROWB);
 #pragma unroll
@@ -1881,7 +1961,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
     }
     __syncthreads();
     if (!*sm.last) return;
-    merge_unit<D, G>(a, sm, lunit, b, l, kvh, tid);
+    merge_unit<D, G, C::RING>(a, sm, lunit, b, l, kvh, tid);
 }
 
 // one CTA of D threads per (b, l, query head)
@@ -2176,6 +2256,7 @@ static cudaError_t launch_t(const sekv_decode_desc& d, const DecodePlan& p, void
     a.zin = zin;
     // test hook (sekv_decode_desc.test_flags bit 0): no copies and short waits
     a.starve = (d.test_flags & 1) ? 1 : 0;
+    a.static_ready = d.static_ready ? 1 : 0;
     a.polls = a.starve ? 4096u : kWaitPolls;
     a.arrive = d.phase != SEKV_ROUTE ? d.arrive : nullptr;
     a.O = d.O;

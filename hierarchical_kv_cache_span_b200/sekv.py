@@ -62,7 +62,7 @@ class sekv_decode_desc(C.Structure):
         ("B", _i32), ("L", _i32), ("Hq", _i32), ("Hkv", _i32), ("d", _i32), ("dtype", _i32),
         ("l0", _i32), ("l1", _i32), ("a_cap", _i32), ("m_cap", _i32), ("rank", _i32),
         ("phase", _i32), ("nsplit", _i32), ("rows_hint", _i32), ("budget", _i32), ("zoom_hint", _i32),
-        ("dr", _i32), ("test_flags", _i32),
+        ("dr", _i32), ("test_flags", _i32), ("static_ready", _i32),
     ]
 
 

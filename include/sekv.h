@@ -253,6 +253,18 @@ typedef struct sekv_decode_desc {
                                 kernels issue no copy and give every bounded wait ~4096 polls,
                                 so the waits run out, *dev_status reads SEKV_ERR_TIMEOUT and the
                                 kernels return with nothing in flight (O = 0, lse = -inf).   */
+    int32_t static_ready;    /* 0 (default) or 1. The decode kernels are launched with
+                                programmatic dependent launch: a grid may start while the
+                                previous kernel on the stream finishes, and waits for it
+                                before it reads its inputs. With 1 the caller guarantees
+                                that no work still in flight on the stream writes the cache's
+                                build outputs (a_count, m_count, Ka, Va, kbar, vbar, inv_norm,
+                                logS), e.g. the stream was synchronised after the build; the
+                                kernel then reads the counts and its first anchor / summary
+                                tiles before that wait, so their latency overlaps the previous
+                                kernel's end (a layer-by-layer decode loop). Everything else
+                                (q, theta, zmask, the bases, the workspace) is still read
+                                after the wait. Results are the same bits either way.     */
 } sekv_decode_desc;
 
 size_t sekv_decode_workspace_bytes(const sekv_decode_desc* desc);

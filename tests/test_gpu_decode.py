@@ -264,6 +264,64 @@ def test_layer_range_calls_equal_one_call():
     _compare(wl, c, q, theta, scale, segs, units, O_p, lse_p, zm_p)
 
 
+@pytest.mark.parametrize("name,over", [("c2", dict(n=4096, L=3)), ("c4", dict(B=2, n=2048, L=2))])
+def test_static_ready_calls_give_the_same_bits(name, over):
+    """with static_ready the kernels read the counts and their first anchor / summary
+    tiles before the programmatic-launch wait; once the cache is settled (stream
+    synchronised after the upload) back-to-back calls give the same bits as without:
+    FUSED per layer and over all layers (device bases), ROUTE per layer, then fetch
+    and ATTEND per layer with the routed mask (bases in host memory)"""
+    P = _lib()
+    S = P.sekv
+    wl = WORKLOADS[name].scaled(**over)
+    H, K, V, segs, units, q, theta, scale = _setup(wl)
+    hot = _cache(wl)
+    T.upload_oracle_cache(hot, segs, units)
+    cold = _cache(wl, home="host")
+    T.upload_oracle_cache(cold, segs, units)
+    th = torch.tensor(theta, dtype=torch.float32, device="cuda")
+    qd = q.cuda()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream().cuda_stream
+    runs = {}
+    for ready in (False, True):
+        zm_f = hot.new_zmask()
+        O_f, lse_f = hot.new_outputs()
+        O_f.fill_(float("nan"))
+        # calls enqueued back to back: each one's early reads overlap the previous kernel
+        for l in range(wl.L):
+            d = hot.decode_desc(qd, th, phase=S.SEKV_FUSED, O=O_f, lse=lse_f, zmask=zm_f, l0=l, l1=l + 1,
+                                static_ready=ready)
+            S.check(S.sekv_decode_attn(d, stream), "fused")
+        O_1, lse_1 = hot.new_outputs()
+        zm_1 = hot.new_zmask()
+        d = hot.decode_desc(qd, th, phase=S.SEKV_FUSED, O=O_1, lse=lse_1, zmask=zm_1, static_ready=ready)
+        S.check(S.sekv_decode_attn(d, stream), "fused, all layers")
+        zm_r = cold.new_zmask()
+        for l in range(wl.L):
+            d = cold.decode_desc(qd, th, phase=S.SEKV_ROUTE, zmask=zm_r, l0=l, l1=l + 1, static_ready=ready)
+            S.check(S.sekv_decode_attn(d, stream), "route")
+        fetch = P.ColdFetcher(cold, arena_elems=cold.region * wl.L)
+        fetch.fetch(zm_r)
+        torch.cuda.current_stream().wait_event(fetch.done)
+        O_a, lse_a = cold.new_outputs()
+        O_a.fill_(float("nan"))
+        for l in range(wl.L):
+            d = cold.decode_desc(qd, th, phase=S.SEKV_ATTEND, O=O_a, lse=lse_a, zmask=zm_r, slot=fetch.slot_dev,
+                                 arena=fetch.arena, l0=l, l1=l + 1, static_ready=ready)
+            S.check(S.sekv_decode_attn(d, stream), "attend")
+        torch.cuda.synchronize()
+        assert hot.read_status() == 0 and cold.read_status() == 0
+        runs[ready] = (zm_f, O_f, lse_f, zm_1, O_1, lse_1, zm_r, O_a, lse_a)
+    for a, b in zip(runs[False], runs[True]):
+        assert torch.equal(a, b)
+    zm_f, O_f, lse_f, zm_1, O_1, lse_1, zm_r, O_a, lse_a = runs[True]
+    assert torch.equal(zm_r, zm_f) and torch.equal(zm_1, zm_f)
+    _compare(wl, hot, q, theta, scale, segs, units, O_f, lse_f, zm_f)
+    _compare(wl, hot, q, theta, scale, segs, units, O_1, lse_1, zm_1)
+    _compare(wl, cold, q, theta, scale, segs, units, O_a, lse_a, zm_r)
+
+
 def test_route_fetch_attend_equals_fused():
     """cold bases in pinned host memory: ROUTE, fetch zoomed bases, ATTEND"""
     P = _lib()
