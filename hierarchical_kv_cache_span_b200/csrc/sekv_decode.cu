@@ -774,6 +774,23 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
             }
         }
     };
+    // span S: its length (0 when invalid) and block offset (-1 when cold); the bounds
+    // and the offset are loaded together (one round trip)
+    auto span_look = [&](int S, int& len, long long& off) {
+        const int64_t si = (int64_t)b * a.m_cap + S;
+        const int beg = a.span_beg[si], end = a.span_end[si];
+        const long long o = a.slot ? a.slot[((int64_t)b * a.L + l) * a.m_cap + S]
+                                   : ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S];
+        len = end - beg;
+        off = -1;
+        if (len < 1) {
+            set_status(a.status, SEKV_ERR_INVALID_ARG);
+            len = 0;
+        } else {
+            off = o;
+            if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
+        }
+    };
     // Walk the zoomed spans (any head of the group) in span order, up to 32 at a time:
     // visit(len, hm, off, n) gets this lane's span of the batch (len 0: none or
     // invalid; off < 0: cold) and the batch size n (warp-uniform); it returns false
@@ -811,17 +828,7 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
                     const int S = s0 + (w0 + kw) * 32 + bit;
 #pragma unroll
                     for (int h = 0; h < G; ++h) hm |= ((sm.zw[h * zwords + w0 + kw] >> bit) & 1u) << h;
-                    const int beg = a.span_beg[(int64_t)b * a.m_cap + S];
-                    len = a.span_end[(int64_t)b * a.m_cap + S] - beg;
-                    if (len < 1) {
-                        set_status(a.status, SEKV_ERR_INVALID_ARG);
-                        len = 0;
-                    } else if (a.slot) {
-                        off = a.slot[((int64_t)b * a.L + l) * a.m_cap + S];
-                        if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
-                    } else {
-                        off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S];
-                    }
+                    span_look(S, len, off);
                 }
                 if (!visit(len, hm, off, min(32, total - e0))) return;
             }
@@ -874,16 +881,7 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
                     const int S = s0 + wk * 32 + bit;
 #pragma unroll
                     for (int h = 0; h < G; ++h) hm |= ((sm.zw[h * zwords + wk] >> bit) & 1u) << h;
-                    len = a.span_end[(int64_t)b * a.m_cap + S] - a.span_beg[(int64_t)b * a.m_cap + S];
-                    if (len < 1) {
-                        set_status(a.status, SEKV_ERR_INVALID_ARG);
-                        len = 0;
-                    } else if (a.slot) {
-                        off = a.slot[((int64_t)b * a.L + l) * a.m_cap + S];
-                        if (off < 0) set_status(a.status, SEKV_ERR_COLD_SPAN);
-                    } else {
-                        off = ((int64_t)b * a.L + l) * a.region + a.blk_off[(int64_t)b * (a.m_cap + 1) + S];
-                    }
+                    span_look(S, len, off);
                 }
                 const int nu = len >= 1 ? (len + 31) >> 5 : 0;
                 int ex = nu;
