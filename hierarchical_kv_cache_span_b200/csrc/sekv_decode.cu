@@ -683,7 +683,7 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
                 } else {
                     mbar_arrive_expect_tx(&sm.zfull[slot], tot);
                     for (int k = 0; k < nparts; ++k)
-                        if (bytes[k]) bulk_g2s(dst + off[k], src[k], bytes[k], &sm.zfull[slot]);
+                        if (bytes[k]) bulk_g2s_ef(dst + off[k], src[k], bytes[k], &sm.zfull[slot], l2_evict_first());
                 }
             } else {
                 set_status(a.status, SEKV_ERR_TIMEOUT);
@@ -1469,6 +1469,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                         : sm.stages + (size_t)(s >> 1) * C::STAGE + 2 * C::TILE + (s & 1) * C::META;
     };
     auto issue_tile = [&](int i) {
+        const uint64_t pol = l2_evict_first();     // rows of this unit are read once per call
         const int s = i % NP;
         unsigned char* st = pos_key(s);
         if (i < nta) {
@@ -1478,8 +1479,8 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                 mbar_arrive_expect_tx(&sm.full[s], 2 * C::NBOX * 8192);
 #pragma unroll
                 for (int h = 0; h < C::NBOX; ++h) {
-                    tma_load_2d(st + h * 8192, &maps.Ka, 64 * h, y, &sm.full[s]);
-                    tma_load_2d(st + C::TILE + h * 8192, &maps.Va, 64 * h, y, &sm.full[s]);
+                    tma_load_2d_ef(st + h * 8192, &maps.Ka, 64 * h, y, &sm.full[s], pol);
+                    tma_load_2d_ef(st + C::TILE + h * 8192, &maps.Va, 64 * h, y, &sm.full[s], pol);
                 }
             } else {
                 const uint32_t bytes = (uint32_t)min(TR, a1 - r0) * C::ROWB;
@@ -1497,8 +1498,8 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                 mbar_arrive_expect_tx(&sm.full[s], (route_only ? 1 : 2) * C::NBOX * 8192 + 2 * mbytes);
 #pragma unroll
                 for (int h = 0; h < C::NBOX; ++h) {
-                    tma_load_2d(st + h * 8192, &maps.kbar, 64 * h, y, &sm.full[s]);
-                    if (!route_only) tma_load_2d(st + C::TILE + h * 8192, &maps.vbar, 64 * h, y, &sm.full[s]);
+                    tma_load_2d_ef(st + h * 8192, &maps.kbar, 64 * h, y, &sm.full[s], pol);
+                    if (!route_only) tma_load_2d_ef(st + C::TILE + h * 8192, &maps.vbar, 64 * h, y, &sm.full[s], pol);
                 }
             } else {
                 const uint32_t bytes = (uint32_t)rows * C::ROWB;
@@ -1507,7 +1508,7 @@ decode_kernel(const DecArgs a, const __grid_constant__ DecMaps maps) {
                 bulk_g2s(st, a.kbar + off, bytes, &sm.full[s]);
                 if (!route_only) bulk_g2s(st + C::TILE, a.vbar + off, bytes, &sm.full[s]);
             }
-            bulk_g2s(pos_meta(s), a.inv_norm + unit * a.m_cap + S0, mbytes, &sm.full[s]);
+            bulk_g2s_ef(pos_meta(s), a.inv_norm + unit * a.m_cap + S0, mbytes, &sm.full[s], pol);
             bulk_g2s(pos_meta(s) + TR * 4, a.logS + (int64_t)b * a.m_cap + S0, mbytes, &sm.full[s]);
         }
     };
