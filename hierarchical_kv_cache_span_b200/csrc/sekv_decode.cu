@@ -683,7 +683,12 @@ SEKV_DEV void zoom_produce(const DecArgs& a, const DecSmem& sm, int lane, int b,
                 } else {
                     mbar_arrive_expect_tx(&sm.zfull[slot], tot);
                     for (int k = 0; k < nparts; ++k)
-                        if (bytes[k]) bulk_g2s_ef(dst + off[k], src[k], bytes[k], &sm.zfull[slot], l2_evict_first());
+                        if (bytes[k]) {
+                            // zoom-dense calls (whole-span pieces) measured faster without
+                            // the evict-first policy on their many small block copies
+                            if constexpr (SP) bulk_g2s(dst + off[k], src[k], bytes[k], &sm.zfull[slot]);
+                            else bulk_g2s_ef(dst + off[k], src[k], bytes[k], &sm.zfull[slot], l2_evict_first());
+                        }
                 }
             } else {
                 set_status(a.status, SEKV_ERR_TIMEOUT);
